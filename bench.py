@@ -1,0 +1,382 @@
+#!/usr/bin/env python
+"""Benchmark of the weight-only quantized linear on B200.
+
+Default workload (one step): the 28-layer, Qwen2.5-7B-shaped decode stack at
+M = 1 token, INT4 g128: per layer qkv 4608x3584, o 3584x3584, gate_up
+37888x3584, down 3584x18944 (112 projections, 3.47 GB of packed weights,
+larger than L2, so no flush is needed), run through one zq_linear_stack call.
+Weights are synthetic (N(0, 0.02), seeded per tensor) and quantized on the GPU
+by zq_quantize_pack; activations N(0, 1) rounded to fp16.
+
+Metric: algorithmic HBM bytes per step (packed codes + fp16 scales/zeros + x +
+out) / device time, in GB/s; also % of 8 TB/s and tokens/s-equivalent
+(linear layers only: attention, norms, embeddings and lm_head excluded).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zq|reference]
+                    [--workload decode|prefill] [--m M]
+
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).  With N > 1 (torchrun), each rank
+runs an independent replica on its own GPU (the path has no exchange step);
+value is the total over ranks / the max over ranks of the device time.
+"""
+import argparse
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import zq_inputs as zi  # noqa: E402
+
+METRIC = "quantized-linear HBM GB/s (% of 8 TB/s) at M=1; tokens/s-equiv per layer stack"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+
+
+# --------------------------------------------------------------- plumbing --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(backend):
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def max_over_ranks(value, world, device="cpu"):
+    if world == 1:
+        return value
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while running."""
+
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index, period_s=0.005):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = torch.cuda.get_device_properties(device_index).uuid
+            handle = None
+            for i in range(pynvml.nvmlDeviceGetCount()):
+                h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                u = pynvml.nvmlDeviceGetUUID(h)
+                u = u.decode() if isinstance(u, bytes) else u
+                if u.replace("GPU-", "") == str(uuid).replace("GPU-", ""):
+                    handle = h
+            self._nvml, self._h = pynvml, handle
+            if handle is not None:
+                self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nvml, self._h = None, None
+
+    def _run(self):
+        while not self._stop.is_set():
+            self.sample()
+            time.sleep(self.period)
+
+    def sample(self):
+        if self._h is None:
+            return
+        p = self._nvml
+        try:
+            self.samples.append(p.nvmlDeviceGetClockInfo(self._h, p.NVML_CLOCK_SM))
+            mask = p.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            for name, bit in self.REASONS.items():
+                if mask & bit:
+                    self.reasons.add(name)
+        except Exception:
+            pass
+
+    def __enter__(self):
+        if self._h is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        self.sample()  # one more right at the end of the region
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml"}
+
+
+# --------------------------------------------------------------- workload --
+
+def op_bytes(M, N, K, bits):
+    return N * K * bits // 8 + 4 * N * K // 128 + 2 * M * K + 2 * M * N
+
+
+def decode_stack_shapes(layers=zi.QWEN7B_LAYERS):
+    return [(layer, t, name, N, K, 4) for layer in range(layers)
+            for t, (name, N, K) in enumerate(zi.QWEN7B)]
+
+
+class StackWorkload:
+    """All tensors of the decode stack resident on the GPU: one contiguous x
+    buffer, one contiguous out buffer (views per op), packed weights per op."""
+
+    def __init__(self, zq, M, device, layers=zi.QWEN7B_LAYERS):
+        self.M = M
+        shapes = decode_stack_shapes(layers)
+        ks = sorted({K for (_, _, _, _, K, _) in shapes})
+        x_elems = sum(M * K for K in ks)
+        self.x_all = torch.empty(x_elems, dtype=torch.float16, device=device)
+        xoff, self.x = 0, {}
+        for K in ks:
+            v = self.x_all[xoff:xoff + M * K].view(M, K)
+            v.copy_(zi.activations(M, K, zi.seed_for(0, zi.X_SEED), device=device))
+            self.x[K] = v
+            xoff += M * K
+        out_elems = sum(M * N for (_, _, _, N, _, _) in shapes)
+        self.out_all = torch.empty(out_elems, dtype=torch.float16, device=device)
+        self.ops, self.weights, self.bytes, self.flops = [], [], 0, 0
+        ooff = 0
+        for (layer, t, name, N, K, bits) in shapes:
+            w = zi.weight(N, K, zi.seed_for(layer, t), device=device)
+            q = zq.quantize(w, bits)
+            del w
+            out = self.out_all[ooff:ooff + M * N].view(M, N)
+            ooff += M * N
+            self.weights.append((layer, name, N, K, bits, q))
+            self.ops.append((self.x[K], *q, out, bits, 128, M, N, K))
+            self.bytes += op_bytes(M, N, K, bits)
+            self.flops += 2 * M * N * K
+        self.descs, self.n_ops = zq.make_descs(self.ops)
+        torch.cuda.synchronize()
+
+
+# ------------------------------------------------------------ oracle legs --
+
+def oracle_layer_sample(M, seed_layer=0, frac=1.0, device_weights=None):
+    """Host inputs for the oracle: the 4 projections of one layer (rows sample).
+    device_weights: list of (name, N, K, bits, (packed, scales, zeros)) on GPU
+    to copy; else the layer is drawn on the CPU and quantized by the oracle."""
+    import oracle as orc
+    items = []
+    for t, (name, N, K) in enumerate(zi.QWEN7B):
+        if device_weights is not None:
+            q = device_weights[t][4]
+            p = q[0].view(torch.int32).cpu().numpy().view(np.uint32).reshape(N, -1)
+            s = q[1].cpu().numpy().view(np.uint16)
+            z = q[2].cpu().numpy().view(np.uint16)
+        else:
+            w = zi.weight(N, K, zi.seed_for(seed_layer, t)).numpy()
+            p, s, z = orc.quantize_pack(w, 4)
+        x = zi.activations(M, K, zi.seed_for(0, zi.X_SEED)).numpy().view(np.uint16)
+        rows = np.arange(0, N, max(1, int(round(1 / frac))), dtype=np.int64)
+        items.append((x, p, s, z, N, K, rows))
+    return items
+
+
+def time_oracle(items, M, budget_s=None):
+    """Runs the oracle over the sample (repeating until budget_s if given);
+    returns (GB/s, seconds, bytes, threads)."""
+    import oracle as orc
+    done_bytes, t0 = 0, time.perf_counter()
+    while True:
+        for (x, p, s, z, N, K, rows) in items:
+            orc.linear(x, p, s, z, 4, N, K, rows=rows)
+            done_bytes += op_bytes(M, len(rows), K, 4)
+        el = time.perf_counter() - t0
+        if budget_s is None or el >= budget_s:
+            break
+    return done_bytes / el / 1e9, el, done_bytes, orc.get_threads()
+
+
+# ------------------------------------------------------------------- arms --
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    M = args.m
+    items = oracle_layer_sample(M, frac=args.ref_frac)
+    for _ in range(args.warmup):
+        time_oracle(items, M)
+    vals, secs, nbytes = [], 0.0, 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, el, b, threads = time_oracle(items, M)
+        secs += el
+        nbytes += b
+    total = time.perf_counter() - t0
+    value = nbytes / total / 1e9
+    sample = (f"each step: oracle linear on every {int(round(1 / args.ref_frac))}th row of the 4 "
+              f"projections of one 7B-shaped INT4 layer at M={M} (fp64, OpenMP over rows)")
+    line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"qwen2.5-7b-shaped decode stack, M={M}, INT4 g128 (sampled rows)"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_zq(args):
+    world, rank, local = dist_init("nccl")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    import weight_only_quantized_zq_b200 as zq
+    peaks = load_peaks()
+    M = args.m
+    wl = StackWorkload(zq, M, dev, args.layers)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def step():
+        zq.zq_linear_stack(wl.descs, wl.n_ops, sp)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    launches0 = zq.zq_kernel_launches()
+    with ClockSampler(local) as clk:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+    launches = zq.zq_kernel_launches() - launches0
+    barrier(world)
+    ms = ev0.elapsed_time(ev1)
+    ms_max = max_over_ranks(ms, world, dev)
+    ms_step = ms_max / args.steps
+    value = world * wl.bytes * args.steps / (ms_max / 1e3) / 1e9
+
+    # End to end through the public API with host buffers: pinned H2D of the
+    # step's activations, the stack, D2H of every output, per step.
+    x_host = torch.empty(wl.x_all.numel(), dtype=torch.float16, pin_memory=True)
+    x_host.copy_(wl.x_all)
+    out_host = torch.empty(wl.out_all.numel(), dtype=torch.float16, pin_memory=True)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        wl.x_all.copy_(x_host, non_blocking=True)
+        step()
+        out_host.copy_(wl.out_all, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_value = world * wl.bytes * args.steps / (e2e_ms / 1e3) / 1e9
+
+    # Roofline of the dominant kernel (the grouped decode launch): the step is
+    # one prep launch + one decode launch, timed together by the events above.
+    achieved = wl.bytes / (ms_step / 1e3) / 1e9
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                "peak_source": peaks["source"], "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel"}
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            items = oracle_layer_sample(M, device_weights=[w[1:] for w in wl.weights[:4]], frac=1.0)
+            v, el, b, threads = time_oracle(items, M, budget_s=args.cpu_seconds)
+            cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                   "sample": f"oracle linear (fp64, OpenMP over rows) on all 4 projections of layer 0 "
+                             f"at M={M}, repeated for {el:.1f} s ({b / 1e9:.2f} GB of algorithmic bytes)"}
+        line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "f16 in, f32 accumulate, int4 weights", "data": "synthetic",
+                "config": {"workload": f"qwen2.5-7b-shaped decode stack: {args.layers} layers x (qkv, o, "
+                                       f"gate_up, down), M={M}, INT4 g128, one zq_linear_stack call",
+                           "layers": args.layers, "M": M, "bits": 4, "group": 128,
+                           "bytes_per_step": wl.bytes, "flops_per_step": wl.flops,
+                           "l2": f"inputs larger than L2 ({wl.bytes / 1e9:.2f} GB per step)",
+                           "parallelism": f"replicas x{world}"},
+                "pct_of_8tbs": 100 * achieved / NOMINAL_HBM_GBS,
+                "tokens_per_s_equiv": world * M / (ms_step / 1e3),
+                "roofline": roofline,
+                "cpu_baseline": cpu,
+                "e2e": {"value": e2e_value, "unit": "GB/s",
+                        "h2d_bytes_per_step": wl.x_all.numel() * 2,
+                        "d2h_bytes_per_step": wl.out_all.numel() * 2,
+                        "ms_per_step": e2e_ms / args.steps},
+                "gpu_launches": launches,
+                "clocks": clk.summary()}
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def zq_mt(M):
+    return 1 if M <= 8 else 2 if M <= 16 else 4 if M <= 32 else 8
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("zq", "reference"), default="zq")
+    ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
+    ap.add_argument("--layers", type=int, default=zi.QWEN7B_LAYERS, help="layers in the stack")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-frac", type=float, default=0.25, help="row fraction per reference step")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_zq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,163 @@
+/*
+ * zq.h — C ABI of the weight-only quantized linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes y = x · dequant(W)^T, the projection that dominates every
+ * decode and prefill step of a pre-quantized LLM inference engine.
+ *
+ * Sources (cited by page title and section):
+ *   [wiki]  "ZSE - open-source движок для запуска LLM локально на GPU - 2026"
+ *           (wiki.iphoster.net). Section "Формат модели .zse": asymmetric
+ *           group-wise quantization with groups of 128, scale = (max-min)/15,
+ *           zero = min, q = clamp(round((w-zero)/scale), 0, 15), two INT4 codes
+ *           per byte with the low nibble first, fp16 scales and zeros, and
+ *           quantization done once at conversion time. Section "Оркестратор и
+ *           GPU-ядра": INT4 GEMV with 128-bit weight loads, batched launches and
+ *           graph capture to cut launch latency.
+ *   [lavx]  "ZSE: A Memory-Efficient LLM Inference Engine with Smart Resource
+ *           Orchestration", section "Technical Architecture": per-tensor INT2-8
+ *           mixed precision (zQuantize).
+ *
+ * Tensor format (all buffers row-major and contiguous):
+ *   W       N x K weights (output features x input features; y = x W^T).
+ *   bits    b in {2, 3, 4, 8}, chosen per tensor.  L = 2^b - 1.
+ *   group   128 consecutive weights along K share one fp16 scale and one fp16
+ *           zero.  K must be a multiple of 128.  G = K / 128.
+ *   packed  uint32 N x (K*b/32).  The codes of one row form a little-endian
+ *           bitstream: code k occupies stream bits [k*b, k*b+b), and stream bit
+ *           t is bit (t % 32) of word t / 32.  At b = 4 this is the pages'
+ *           "two codes per byte, low nibble first".  At b = 3 codes straddle
+ *           word boundaries; a group is always exactly 4*b words.
+ *   scales  fp16 (as uint16 bit patterns) N x G.
+ *   zeros   fp16 (as uint16 bit patterns) N x G.  The zero is the group's
+ *           float minimum, not an integer zero point:
+ *           dequant(W)[n][k] = q[n][k] * scale[n][k/128] + zero[n][k/128].
+ *   x       fp16 M x K activations;  out  fp16 M x N.
+ *   Arithmetic: fp16 in, fp32 accumulation, fp16 out (round to nearest even).
+ *
+ * Conventions for every entry point:
+ *   - Pointers are device pointers unless stated otherwise, and must be
+ *     16-byte aligned.  The caller owns every buffer.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *     enqueued on it; zq_linear and zq_linear_stack return without waiting.
+ *   - Errors: a non-OK status is returned and nothing is enqueued when the
+ *     arguments are rejected.  zq_last_error() gives a message for the most
+ *     recent failure on the calling thread.  ZQ_ERR_CUDA means a CUDA call
+ *     failed (launch error, out of memory); the CUDA error is in the message.
+ *   - Stream order: a call's kernels read their inputs only after all work
+ *     enqueued earlier on `stream` has completed (programmatic dependent
+ *     launch is used only to overlap launch latency, never to read early).
+ *   - The library keeps one workspace per (device, stream) for activation
+ *     staging and split-K partial sums.  It is allocated (and zeroed) by the
+ *     first call on that stream that needs it and grown when a larger call
+ *     arrives; run such a call once before capturing the stream into a CUDA
+ *     graph, or call zq_reserve_workspace().  Calls on the same stream are
+ *     ordered; calls on different streams use different workspaces.
+ */
+#ifndef ZQ_H
+#define ZQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ZQ_API __attribute__((visibility("default")))
+#else
+#define ZQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st;
+typedef struct CUstream_st *zq_stream_t; /* identical to cudaStream_t */
+
+typedef enum {
+    ZQ_OK = 0,
+    ZQ_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer          */
+    ZQ_ERR_UNSUPPORTED = 2, /* bits not in {2,3,4,8} or group != 128          */
+    ZQ_ERR_NONFINITE = 3,   /* a weight is NaN/Inf or |w| > 65504 (fp16 max)  */
+    ZQ_ERR_CUDA = 4,        /* a CUDA runtime call failed                     */
+    ZQ_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up             */
+} zq_status;
+
+/* Number of uint32 words of a packed N x K tensor: N * K * bits / 32.
+ * Returns 0 for unsupported bits or sizes (K % 128 != 0, N <= 0, K <= 0). */
+ZQ_API size_t zq_packed_words(int N, int K, int bits);
+
+/* Quantize and pack a weight tensor on the GPU, [wiki] "Формат модели .zse",
+ * generalised to L = 2^bits - 1 ([lavx] "Technical Architecture").
+ *   w       device, fp32 N x K row-major.
+ *   packed  device, uint32 N x (K*bits/32), written.
+ *   scales  device, fp16 bits N x (K/128), written.
+ *   zeros   device, fp16 bits N x (K/128), written.
+ * Per group: zero = fp16(min), scale = fp16((max - min) / L) computed in fp64
+ * and rounded once; q = clamp(round_half_even((w - zero) / scale), 0, L) with
+ * the stored fp16 scale and zero, in fp64; a group whose fp16 scale is 0 gets
+ * all q = 0.  Bit-exact with the reference quantizer.
+ * SYNCHRONOUS: the call waits for `stream` so it can report ZQ_ERR_NONFINITE
+ * (any NaN, Inf or |w| > 65504); then the outputs are unspecified.  Not
+ * capturable into a CUDA graph. */
+ZQ_API zq_status zq_quantize_pack(const float *w, int N, int K, int bits, int group,
+                           uint32_t *packed, uint16_t *scales, uint16_t *zeros,
+                           zq_stream_t stream);
+
+/* y = x · dequant(W)^T.
+ *   x       device, fp16 M x K.      out  device, fp16 M x N (written).
+ *   packed/scales/zeros as produced by zq_quantize_pack.
+ * M <= 64 runs the decode family (tensor-core skinny GEMM streaming the
+ * packed weights once); larger M runs the prefill family.  Asynchronous. */
+ZQ_API zq_status zq_linear(const uint16_t *x, const uint32_t *packed,
+                    const uint16_t *scales, const uint16_t *zeros,
+                    int bits, int group, int M, int N, int K,
+                    uint16_t *out, zq_stream_t stream);
+
+/* One operation of a stack: the arguments of one zq_linear call. */
+typedef struct {
+    const uint16_t *x;
+    const uint32_t *packed;
+    const uint16_t *scales;
+    const uint16_t *zeros;
+    uint16_t *out;
+    int bits, group, M, N, K;
+} zq_linear_desc;
+
+/* Run n_ops linear layers with the result of calling zq_linear on each, in
+ * array order ([wiki] "Оркестратор и GPU-ядра": batched launches, graphs).
+ * `ops` is a HOST array, read before the call returns.  An op's x may alias
+ * an earlier op's out: the library detects overlapping buffers and keeps
+ * such ops ordered; runs of independent ops are fused into one launch per
+ * (bits, batch class).  All ops are validated before anything is enqueued.
+ * Asynchronous. */
+ZQ_API zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream);
+
+/* Test hook: unpack codes with the same device unpack routine zq_linear
+ * uses.  codes: device uint8 N x K (written).  Asynchronous. */
+ZQ_API zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits,
+                    uint8_t *codes, zq_stream_t stream);
+
+/* Pre-size the workspace of (current device, stream) to at least `bytes`.
+ * Useful before graph capture.  Synchronous. */
+ZQ_API zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream);
+
+/* Workspace bytes zq_linear needs for these sizes (0 if none). */
+ZQ_API size_t zq_linear_workspace_bytes(int bits, int M, int N, int K);
+
+/* Human-readable name of a status code (static storage). */
+ZQ_API const char *zq_status_string(zq_status status);
+
+/* Message of the most recent failure on the calling thread ("" if none). */
+ZQ_API const char *zq_last_error(void);
+
+/* Number of kernels this library has launched in this process (all devices).
+ * Lets a caller count device work, e.g. inside a timed region. */
+ZQ_API uint64_t zq_kernel_launches(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+ZQ_API int zq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ZQ_H */

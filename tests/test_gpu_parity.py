@@ -1,0 +1,205 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
+
+Bit-exact: quantize_pack (codes, scales, zeros) and unpack.
+Tolerance (the linear): |y_gpu - y_ref| <= 2e-3 * sum|x||w_hat| + 1e-3 per element.
+"""
+import numpy as np
+import pytest
+import torch
+
+import zq_inputs as zi
+from zq_testutil import assert_linear_close, u16, u32
+
+pytestmark = pytest.mark.gpu
+
+BITS = (2, 3, 4, 8)
+
+
+@pytest.fixture(scope="module")
+def zq():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import weight_only_quantized_zq_b200 as m
+    return m
+
+
+def _quantize_both(zq, orc, w, bits):
+    """Quantize on the GPU and with the oracle; assert bit-exact; return GPU buffers."""
+    N, K = w.shape
+    packed, scales, zeros = zq.quantize(w, bits)
+    torch.cuda.synchronize()
+    p_ref, s_ref, z_ref = orc.quantize_pack(w.cpu().numpy(), bits)
+    assert np.array_equal(u16(scales).reshape(N, -1), s_ref), "scales differ"
+    assert np.array_equal(u16(zeros).reshape(N, -1), z_ref), "zeros differ"
+    assert np.array_equal(u32(packed).reshape(N, -1), p_ref), "packed codes differ"
+    return packed, scales, zeros, (p_ref, s_ref, z_ref)
+
+
+def _check_linear(zq, orc, x, qbufs, ref_bufs, bits, N, what, rows=None):
+    M, K = x.shape
+    packed, scales, zeros = qbufs
+    out = zq.linear(x, packed, scales, zeros, bits, N)
+    torch.cuda.synchronize()
+    p_ref, s_ref, z_ref = ref_bufs
+    y_ref, bound = orc.linear(u16(x), p_ref, s_ref, z_ref, bits, N, K, rows=rows)
+    got = out if rows is None else out[:, torch.as_tensor(rows, device=out.device)]
+    return assert_linear_close(got, y_ref, bound, what)
+
+
+# ------------------------------------------------------------- bit-exact --
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantize_pack_bit_exact(zq, orc, bits):
+    for N, K, seed, outl in ((1, 128, 1, False), (37, 512, 2, True), (64, 3584, 3, False),
+                             (5, 27648, 4, True)):
+        w = zi.weight(N, K, seed + 100 * bits, device="cuda", outliers=outl)
+        _quantize_both(zq, orc, w, bits)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantize_pack_edge_groups(zq, orc, bits):
+    """Constant groups (scale 0), exact ties, fp16-range extremes, subnormal scales."""
+    K = 1024
+    w = torch.zeros(6, K)
+    w[0] = 0.0123                                  # constant group everywhere
+    w[1, :128] = torch.arange(128) % 16 / 16.0     # ties at (j+1/2)/16 below
+    w[1, 2:17] = (torch.arange(15) + 0.5) / 16
+    w[1, 0], w[1, 1] = 0.0, 15.0 / 16
+    w[2] = torch.linspace(-65504, 65504, K)        # largest magnitudes
+    w[3] = torch.linspace(0, 1e-6, K)              # fp16 subnormal scales
+    w[4] = torch.randn(K) * 1e-3 - 3.0
+    w[5, ::2] = 1.0
+    _quantize_both(zq, orc, w.cuda().contiguous(), bits)
+
+
+def test_quantize_pack_rejects_nonfinite(zq):
+    for bad in (float("nan"), float("inf"), 70000.0):
+        w = torch.zeros(4, 256, device="cuda")
+        w[2, 77] = bad
+        with pytest.raises(zq.ZQError) as e:
+            zq.quantize(w, 4)
+        assert e.value.status == zq.ZQ_ERR_NONFINITE
+    zq.quantize(torch.zeros(4, 256, device="cuda"), 4)  # next call is clean
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_unpack_bit_exact(zq, orc, bits):
+    for N, K in ((1, 128), (19, 640), (8, 27648)):
+        codes = zi.codes(N, K, bits, seed=7 + bits).numpy()
+        packed_np = np.stack([orc.pack_row(c, bits) for c in codes])
+        packed = torch.from_numpy(packed_np.view(np.int32)).cuda()
+        out = torch.empty(N, K, dtype=torch.uint8, device="cuda")
+        zq.zq_unpack(packed, N, K, bits, out)
+        torch.cuda.synchronize()
+        assert np.array_equal(out.cpu().numpy(), orc.unpack(packed_np, N, K, bits))
+
+
+# ---------------------------------------------------------------- linear --
+
+@pytest.mark.parametrize("bits", BITS)
+def test_linear_shapes(zq, orc, bits):
+    """Ragged N, every decode token tile, split-K and the multi-piece path."""
+    cases = [(1, 1, 128), (1, 17, 512), (2, 100, 384), (3, 33, 1024), (5, 512, 512),
+             (8, 257, 1280), (9, 64, 512), (16, 130, 256), (17, 48, 640), (32, 96, 512),
+             (33, 40, 384), (64, 200, 768), (65, 31, 256), (130, 70, 512)]
+    for i, (M, N, K) in enumerate(cases):
+        w = zi.weight(N, K, seed=1000 + 10 * bits + i, device="cuda", outliers=(i % 3 == 0))
+        q = _quantize_both(zq, orc, w, bits)
+        x = zi.activations(M, K, seed=2000 + i, device="cuda")
+        _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"bits={bits} M={M} N={N} K={K}")
+
+
+def test_linear_adversarial_all_positive(zq, orc):
+    """All-positive x and weights: errors cannot cancel (worst case of fp32
+    accumulation against the bound)."""
+    for bits in BITS:
+        N, K = 64, 18944
+        w = zi.weight(N, K, seed=31 + bits, device="cuda").abs()
+        q = _quantize_both(zq, orc, w, bits)
+        x = zi.activations(4, K, seed=32, device="cuda").abs()
+        _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"all-positive bits={bits}")
+
+
+def test_config1_single_layer(zq, orc):
+    """M=1, N=K=512 INT4; W ~ N(0,0.02) seed 0 quantized by the oracle, x seed 15."""
+    N = K = 512
+    w = zi.weight(N, K, seed=0)  # CPU draw, as the oracle gets it
+    p_ref, s_ref, z_ref = orc.quantize_pack(w.numpy(), 4)
+    packed = torch.from_numpy(p_ref.view(np.int32).reshape(-1)).cuda()
+    scales = torch.from_numpy(s_ref.view(np.int16)).cuda()
+    zeros = torch.from_numpy(z_ref.view(np.int16)).cuda()
+    x = zi.activations(1, K, seed=zi.X_SEED).cuda()
+    _check_linear(zq, orc, x, (packed, scales, zeros), (p_ref, s_ref, z_ref), 4, N, "config1")
+
+
+def test_config2_7b_decode_projections(zq, orc):
+    for t, (name, N, K) in enumerate(zi.QWEN7B):
+        w = zi.weight(N, K, zi.seed_for(0, t), device="cuda")
+        q = _quantize_both(zq, orc, w, 4)
+        del w
+        x = zi.activations(1, K, zi.seed_for(0, zi.X_SEED), device="cuda")
+        _check_linear(zq, orc, x, q[:3], q[3], 4, N, f"7b {name}")
+
+
+def test_config4_32b_mixed_precision(zq, orc):
+    for t, (name, N, K, bits) in enumerate(zi.QWEN32B_MIXED):
+        w = zi.weight(N, K, zi.seed_for(0, t), device="cuda", outliers=True)
+        q = _quantize_both(zq, orc, w, bits)
+        del w
+        x = zi.activations(1, K, zi.seed_for(0, zi.X_SEED), device="cuda")
+        _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"32b {name} int{bits}")
+
+
+# ----------------------------------------------------------------- stack --
+
+def _layer(zq, orc, N, K, bits, seed):
+    w = zi.weight(N, K, seed, device="cuda")
+    q = zq.quantize(w, bits)
+    torch.cuda.synchronize()
+    ref = orc.quantize_pack(w.cpu().numpy(), bits)
+    return q, ref
+
+
+def test_stack_against_oracle(zq, orc):
+    """Independent ops of mixed bits and batch sizes (fused into shared
+    launches) and a dependent chain (x of an op is the out of the previous
+    one), all through one zq_linear_stack call."""
+    specs = [(4, 512, 512, 4), (4, 256, 512, 3), (4, 512, 256, 8), (4, 1024, 512, 2),
+             (12, 512, 512, 4), (1, 384, 512, 4), (40, 128, 384, 4)]
+    layers = [_layer(zq, orc, N, K, b, 50 + i) for i, (M, N, K, b) in enumerate(specs)]
+    xs = [zi.activations(M, K, 60 + i, device="cuda") for i, (M, N, K, b) in enumerate(specs)]
+    outs = [torch.empty(M, N, dtype=torch.float16, device="cuda") for (M, N, K, b) in specs]
+    ops = [(xs[i], *layers[i][0], outs[i], b, 128, M, N, K) for i, (M, N, K, b) in enumerate(specs)]
+    # chain: A (K=512 -> N=512) feeds B (K=512 -> N=256), which feeds C (K=256)
+    qa, ra = _layer(zq, orc, 512, 512, 4, 70)
+    qb, rb = _layer(zq, orc, 256, 512, 3, 71)
+    qc, rc = _layer(zq, orc, 384, 256, 8, 73)
+    xa = zi.activations(2, 512, 72, device="cuda")
+    ya = torch.empty(2, 512, dtype=torch.float16, device="cuda")
+    yb = torch.empty(2, 256, dtype=torch.float16, device="cuda")
+    yc = torch.empty(2, 384, dtype=torch.float16, device="cuda")
+    ops += [(xa, *qa, ya, 4, 128, 2, 512, 512), (ya, *qb, yb, 3, 128, 2, 256, 512),
+            (yb, *qc, yc, 8, 128, 2, 384, 256)]
+    zq.zq_linear_stack(ops)
+    torch.cuda.synchronize()
+    for i, (M, N, K, b) in enumerate(specs):
+        p, s, z = layers[i][1]
+        y_ref, bound = orc.linear(u16(xs[i]), p, s, z, b, N, K)
+        assert_linear_close(outs[i], y_ref, bound, f"stack op {i}")
+    for x_in, y_out, ref, b, N, K in ((xa, ya, ra, 4, 512, 512), (ya, yb, rb, 3, 256, 512),
+                                       (yb, yc, rc, 8, 384, 256)):
+        y_ref, bound = orc.linear(u16(x_in), *ref, b, N, K)
+        assert_linear_close(y_out, y_ref, bound, "stack chain")
+
+
+def test_stack_validation_enqueues_nothing(zq, orc):
+    q, _ = _layer(zq, orc, 64, 256, 4, 80)
+    x = zi.activations(1, 256, 81, device="cuda")
+    out = torch.full((1, 64), 7.0, dtype=torch.float16, device="cuda")
+    bad = (x, *q, out, 5, 128, 1, 64, 256)
+    good = (x, *q, out, 4, 128, 1, 64, 256)
+    with pytest.raises(zq.ZQError) as e:
+        zq.zq_linear_stack([good, bad])
+    assert e.value.status == zq.ZQ_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert torch.all(out == 7.0)

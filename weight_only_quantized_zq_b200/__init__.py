@@ -1,0 +1,186 @@
+"""Python binding of libzq, the B200 (sm_100a) weight-only quantized linear.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI of ``include/zq.h``.  The functions carry the C names;
+tensor arguments are torch CUDA tensors (their device pointers are passed), and
+``stream`` defaults to torch's current stream on the tensor's device.
+
+There is no CPU fallback: importing this package raises if ``libzq.so`` has
+not been built (``python weight_only_quantized_zq_b200/build.py``).
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libzq.so")
+
+ZQ_OK = 0
+ZQ_ERR_INVALID_ARG = 1
+ZQ_ERR_UNSUPPORTED = 2
+ZQ_ERR_NONFINITE = 3
+ZQ_ERR_CUDA = 4
+ZQ_ERR_TIMEOUT = 5
+GROUP = 128
+
+# Every symbol the header declares (checked by the CPU test suite).
+EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_linear", "zq_linear_stack",
+           "zq_unpack", "zq_reserve_workspace", "zq_linear_workspace_bytes",
+           "zq_status_string", "zq_last_error", "zq_kernel_launches", "zq_version")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing; build it with "
+                      "`python weight_only_quantized_zq_b200/build.py`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_S = ctypes.c_size_t
+
+_lib.zq_packed_words.argtypes = [_I, _I, _I]
+_lib.zq_packed_words.restype = _S
+_lib.zq_quantize_pack.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
+_lib.zq_quantize_pack.restype = _I
+_lib.zq_linear.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
+_lib.zq_linear.restype = _I
+_lib.zq_linear_stack.argtypes = [_P, _I, _P]
+_lib.zq_linear_stack.restype = _I
+_lib.zq_unpack.argtypes = [_P, _I, _I, _I, _P, _P]
+_lib.zq_unpack.restype = _I
+_lib.zq_reserve_workspace.argtypes = [_S, _P]
+_lib.zq_reserve_workspace.restype = _I
+_lib.zq_linear_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.zq_linear_workspace_bytes.restype = _S
+_lib.zq_status_string.argtypes = [_I]
+_lib.zq_status_string.restype = ctypes.c_char_p
+_lib.zq_last_error.argtypes = []
+_lib.zq_last_error.restype = ctypes.c_char_p
+_lib.zq_kernel_launches.argtypes = []
+_lib.zq_kernel_launches.restype = ctypes.c_uint64
+_lib.zq_version.argtypes = []
+_lib.zq_version.restype = _I
+
+
+class ZQError(RuntimeError):
+    def __init__(self, status, message):
+        super().__init__(f"{zq_status_string(status)}: {message}")
+        self.status = status
+
+
+class zq_linear_desc(ctypes.Structure):
+    _fields_ = [("x", _P), ("packed", _P), ("scales", _P), ("zeros", _P), ("out", _P),
+                ("bits", _I), ("group", _I), ("M", _I), ("N", _I), ("K", _I)]
+
+
+def _check(status):
+    if status != ZQ_OK:
+        raise ZQError(status, zq_last_error())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream, like=None):
+    if stream is None:
+        dev = like.device if isinstance(like, torch.Tensor) else None
+        return torch.cuda.current_stream(dev).cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def zq_status_string(status):
+    return _lib.zq_status_string(int(status)).decode()
+
+
+def zq_last_error():
+    return _lib.zq_last_error().decode()
+
+
+def zq_version():
+    return _lib.zq_version()
+
+
+def zq_kernel_launches():
+    return _lib.zq_kernel_launches()
+
+
+def zq_packed_words(N, K, bits):
+    return _lib.zq_packed_words(N, K, bits)
+
+
+def zq_linear_workspace_bytes(bits, M, N, K):
+    return _lib.zq_linear_workspace_bytes(bits, M, N, K)
+
+
+def zq_reserve_workspace(nbytes, stream=None):
+    _check(_lib.zq_reserve_workspace(nbytes, _stream(stream)))
+
+
+def zq_quantize_pack(w, N, K, bits, group, packed, scales, zeros, stream=None):
+    _check(_lib.zq_quantize_pack(_ptr(w), N, K, bits, group, _ptr(packed), _ptr(scales),
+                                 _ptr(zeros), _stream(stream, w)))
+
+
+def zq_linear(x, packed, scales, zeros, bits, group, M, N, K, out, stream=None):
+    _check(_lib.zq_linear(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), bits, group,
+                          M, N, K, _ptr(out), _stream(stream, x)))
+
+
+def make_descs(ops):
+    """ops: iterable of dicts/tuples (x, packed, scales, zeros, out, bits, group, M, N, K)."""
+    ops = list(ops)
+    arr = (zq_linear_desc * max(len(ops), 1))()
+    for i, o in enumerate(ops):
+        if isinstance(o, dict):
+            o = (o["x"], o["packed"], o["scales"], o["zeros"], o["out"], o["bits"],
+                 o.get("group", GROUP), o["M"], o["N"], o["K"])
+        x, packed, scales, zeros, out, bits, group, M, N, K = o
+        arr[i] = zq_linear_desc(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(out),
+                                bits, group, M, N, K)
+    return arr, len(ops)
+
+
+def zq_linear_stack(ops, n_ops=None, stream=None):
+    """ops: a ctypes array from make_descs(), or an iterable accepted by it."""
+    if not isinstance(ops, ctypes.Array):
+        ops, n = make_descs(ops)
+        n_ops = n if n_ops is None else n_ops
+    _check(_lib.zq_linear_stack(ops, n_ops, _stream(stream)))
+
+
+def zq_unpack(packed, N, K, bits, codes, stream=None):
+    _check(_lib.zq_unpack(_ptr(packed), N, K, bits, _ptr(codes), _stream(stream, packed)))
+
+
+# ------------------------------------------------------------ conveniences --
+
+def alloc_quantized(N, K, bits, device="cuda"):
+    """Empty (packed, scales, zeros) buffers for an N x K tensor."""
+    packed = torch.empty(N * K * bits // 32, dtype=torch.int32, device=device)
+    scales = torch.empty(N, K // GROUP, dtype=torch.int16, device=device)
+    zeros = torch.empty(N, K // GROUP, dtype=torch.int16, device=device)
+    return packed, scales, zeros
+
+
+def quantize(w, bits, stream=None):
+    """fp32 CUDA tensor N x K -> (packed, scales, zeros) via zq_quantize_pack."""
+    N, K = w.shape
+    packed, scales, zeros = alloc_quantized(N, K, bits, w.device)
+    zq_quantize_pack(w, N, K, bits, GROUP, packed, scales, zeros, stream)
+    return packed, scales, zeros
+
+
+def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
+    """fp16 CUDA x (M x K) -> fp16 out (M x N) via zq_linear."""
+    M, K = x.shape
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float16, device=x.device)
+    zq_linear(x, packed, scales, zeros, bits, GROUP, M, N, K, out, stream)
+    return out

@@ -1,0 +1,517 @@
+// zq_api.cu — host side of the C ABI declared in include/zq.h: argument
+// validation, the per-(device, stream) workspace, planning of decode launches
+// (cost-balanced units, split-K choice, fusion of independent stack ops) and
+// dispatch to the kernels.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "zq.h"
+#include "zq_internal.h"
+
+using namespace zq;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<unsigned long long> g_quant_call{1};
+std::atomic<uint64_t> g_launches{0};
+
+zq_status fail(zq_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
+zq_status fail(zq_status st, const char *fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return st;
+}
+
+zq_status cuda_fail(cudaError_t e, const char *what) {
+    return fail(ZQ_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
+
+zq_status check_format(int bits, int group, int N, int K) {
+    if (!bits_ok(bits)) return fail(ZQ_ERR_UNSUPPORTED, "bits=%d not in {2,3,4,8}", bits);
+    if (group != kGroup) return fail(ZQ_ERR_UNSUPPORTED, "group=%d, only 128 is supported", group);
+    if (N <= 0 || K <= 0) return fail(ZQ_ERR_INVALID_ARG, "N=%d K=%d must be positive", N, K);
+    if (K % kGroup != 0) return fail(ZQ_ERR_INVALID_ARG, "K=%d is not a multiple of 128", K);
+    if (static_cast<long long>(N) * K > (1LL << 40))
+        return fail(ZQ_ERR_INVALID_ARG, "N*K=%lld too large", static_cast<long long>(N) * K);
+    return ZQ_OK;
+}
+
+zq_status check_ptr(const void *p, const char *name) {
+    if (p == nullptr) return fail(ZQ_ERR_INVALID_ARG, "%s is null", name);
+    if (!aligned16(p)) return fail(ZQ_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+    return ZQ_OK;
+}
+
+zq_status check_linear(const zq_linear_desc &d) {
+    zq_status st = check_format(d.bits, d.group, d.N, d.K);
+    if (st != ZQ_OK) return st;
+    if (d.M <= 0) return fail(ZQ_ERR_INVALID_ARG, "M=%d must be positive", d.M);
+    if ((st = check_ptr(d.x, "x")) != ZQ_OK) return st;
+    if ((st = check_ptr(d.packed, "packed")) != ZQ_OK) return st;
+    if ((st = check_ptr(d.scales, "scales")) != ZQ_OK) return st;
+    if ((st = check_ptr(d.zeros, "zeros")) != ZQ_OK) return st;
+    if ((st = check_ptr(d.out, "out")) != ZQ_OK) return st;
+    return ZQ_OK;
+}
+
+// ---------------------------------------------------------------- device --
+
+struct DeviceInfo {
+    int sms = 0;
+    int occ[9][9] = {};  // [bits][mt] decode CTAs per SM
+};
+std::mutex g_dev_mu;
+std::map<int, DeviceInfo> g_dev;
+
+zq_status device_info(DeviceInfo **out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    auto it = g_dev.find(dev);
+    if (it == g_dev.end()) {
+        DeviceInfo info;
+        e = cudaDeviceGetAttribute(&info.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceGetAttribute");
+        it = g_dev.emplace(dev, info).first;
+    }
+    *out = &it->second;
+    return ZQ_OK;
+}
+
+zq_status decode_occupancy(DeviceInfo *info, int bits, int mt, int *ctas) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    int &o = info->occ[bits][mt];
+    if (o == 0) {
+        cudaError_t e = decode_ctas_per_sm(bits, mt, &o);
+        if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
+        if (o <= 0) return fail(ZQ_ERR_CUDA, "decode kernel does not fit on an SM");
+    }
+    *ctas = o;
+    return ZQ_OK;
+}
+
+// ------------------------------------------------------------- workspace --
+// One buffer per (device, stream).  Layout: [counters | data].  Counters are
+// zeroed at allocation and every kernel that uses one resets it to zero.
+
+constexpr size_t kCounterBytes = 256 * 1024;
+constexpr size_t kMaxCounters = kCounterBytes / sizeof(unsigned int);
+
+struct Workspace {
+    void *ptr = nullptr;
+    size_t bytes = 0;
+};
+std::mutex g_ws_mu;
+std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+
+zq_status workspace(cudaStream_t stream, size_t data_bytes, uint8_t **base) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const size_t need = kCounterBytes + data_bytes;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    Workspace &ws = g_ws[{dev, stream}];
+    if (ws.bytes < need) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        e = cudaStreamIsCapturing(stream, &cap);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
+        if (cap != cudaStreamCaptureStatusNone)
+            return fail(ZQ_ERR_CUDA,
+                        "workspace of %zu bytes needed while the stream is being captured; "
+                        "run the call once before capture or use zq_reserve_workspace",
+                        need);
+        size_t grow = std::max(need, ws.bytes + ws.bytes / 2);
+        grow = std::max(grow, static_cast<size_t>(8) << 20);
+        if (ws.ptr) {
+            e = cudaStreamSynchronize(stream);
+            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+            cudaFree(ws.ptr);
+            ws.ptr = nullptr;
+            ws.bytes = 0;
+        }
+        e = cudaMalloc(&ws.ptr, grow);
+        if (e != cudaSuccess) {
+            ws.ptr = nullptr;
+            return cuda_fail(e, "cudaMalloc(workspace)");
+        }
+        e = cudaMemset(ws.ptr, 0, kCounterBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(workspace)");
+        ws.bytes = grow;
+    }
+    *base = static_cast<uint8_t *>(ws.ptr);
+    return ZQ_OK;
+}
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+// ------------------------------------------------------------ decode plan --
+
+struct PrepKey {
+    const uint16_t *x;
+    int M, K, bits;
+    bool operator==(const PrepKey &o) const { return x == o.x && M == o.M && K == o.K && bits == o.bits; }
+};
+
+// Plans and launches one decode launch over ops that share bits and MT and are
+// mutually independent.  With `dry_bytes` set, only computes the workspace size.
+zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, cudaStream_t stream,
+                     size_t *dry_bytes = nullptr) {
+    DeviceInfo *info = nullptr;
+    zq_status st = device_info(&info);
+    if (st != ZQ_OK) return st;
+    int occ = 0;
+    if ((st = decode_occupancy(info, bits, mt, &occ)) != ZQ_OK) return st;
+    const int rows = decode_rows(mt);
+    const int mpad = 8 * mt;
+    const long long max_warps = static_cast<long long>(occ) * info->sms * kDecodeWarpsPerCta;
+
+    // Prep entries (distinct activation buffers).
+    std::vector<PrepKey> keys;
+    std::vector<int> op_entry(ops.size());
+    for (size_t i = 0; i < ops.size(); ++i) {
+        PrepKey k{ops[i].x, ops[i].M, ops[i].K, bits};
+        auto it = std::find(keys.begin(), keys.end(), k);
+        if (it == keys.end()) {
+            keys.push_back(k);
+            op_entry[i] = static_cast<int>(keys.size()) - 1;
+        } else {
+            op_entry[i] = static_cast<int>(it - keys.begin());
+        }
+    }
+    if (keys.size() > static_cast<size_t>(kMaxPrepEntries) || ops.size() > static_cast<size_t>(kMaxDecodeOps))
+        return fail(ZQ_ERR_INVALID_ARG, "internal: decode launch too large");
+
+    // Split-K: only when the row blocks alone cannot keep every warp busy.
+    long long rb_total = 0;
+    std::vector<int> rbs(ops.size()), S(ops.size(), 1), gps(ops.size());
+    for (size_t i = 0; i < ops.size(); ++i) {
+        rbs[i] = (ops[i].N + rows - 1) / rows;
+        rb_total += rbs[i];
+        gps[i] = ops[i].K / kGroup;
+    }
+    const long long target = 2 * max_warps;
+    size_t counters = 0;
+    if (rb_total < target) {
+        const double f = static_cast<double>(target) / static_cast<double>(rb_total);
+        for (size_t i = 0; i < ops.size(); ++i) {
+            const int G = ops[i].K / kGroup;
+            int s = std::min(G, static_cast<int>(f + 0.999));
+            if (s <= 1 || counters + rbs[i] > kMaxCounters) continue;
+            gps[i] = (G + s - 1) / s;
+            S[i] = (G + gps[i] - 1) / gps[i];
+            if (S[i] > 1) counters += rbs[i];
+        }
+    }
+
+    // Workspace layout.
+    size_t off = 0;
+    std::vector<size_t> prep_off(keys.size()), part_off(ops.size(), 0);
+    for (size_t e = 0; e < keys.size(); ++e) {
+        prep_off[e] = off;
+        const size_t G = keys[e].K / kGroup;
+        off += align256(static_cast<size_t>(mpad) * keys[e].K * 2) + align256(G * mpad * 4);
+    }
+    for (size_t i = 0; i < ops.size(); ++i)
+        if (S[i] > 1) {
+            part_off[i] = off;
+            off += align256(static_cast<size_t>(rbs[i]) * S[i] * rows * mpad * 4);
+        }
+    if (dry_bytes) {
+        *dry_bytes = off + kCounterBytes;
+        return ZQ_OK;
+    }
+    uint8_t *ws = nullptr;
+    if ((st = workspace(stream, off, &ws)) != ZQ_OK) return st;
+    unsigned int *cnt_base = reinterpret_cast<unsigned int *>(ws);
+    uint8_t *data = ws + kCounterBytes;
+
+    PrepParams pp;
+    std::memset(&pp, 0, sizeof(pp));
+    pp.n_entries = static_cast<int>(keys.size());
+    long long wsum = 0;
+    for (size_t e = 0; e < keys.size(); ++e) {
+        PrepEntry &en = pp.e[e];
+        const size_t G = keys[e].K / kGroup;
+        en.x = keys[e].x;
+        en.xperm = reinterpret_cast<uint16_t *>(data + prep_off[e]);
+        en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(static_cast<size_t>(mpad) * keys[e].K * 2));
+        en.M = keys[e].M;
+        en.M_pad = mpad;
+        en.K = keys[e].K;
+        en.bits = bits;
+        pp.warp_prefix[e] = wsum;
+        wsum += static_cast<long long>(mpad) * G;
+    }
+    pp.warp_prefix[keys.size()] = wsum;
+
+    DecodeParams dp;
+    std::memset(&dp, 0, sizeof(dp));
+    dp.n_ops = static_cast<int>(ops.size());
+    long long cost = 0, units = 0;
+    size_t cnt_off = 0;
+    for (size_t i = 0; i < ops.size(); ++i) {
+        DecodeOp &o = dp.ops[i];
+        const PrepEntry &en = pp.e[op_entry[i]];
+        o.packed = ops[i].packed;
+        o.scales = ops[i].scales;
+        o.zeros = ops[i].zeros;
+        o.xperm = en.xperm;
+        o.sx = en.sx;
+        o.out = ops[i].out;
+        o.M = ops[i].M;
+        o.N = ops[i].N;
+        o.K = ops[i].K;
+        o.G = ops[i].K / kGroup;
+        o.S = S[i];
+        o.gps = gps[i];
+        o.row_blocks = rbs[i];
+        if (S[i] > 1) {
+            o.part = reinterpret_cast<float *>(data + part_off[i]);
+            o.cnt = cnt_base + cnt_off;
+            cnt_off += rbs[i];
+        }
+        o.cost0 = cost;
+        o.unit_cost = static_cast<long long>(rows) * gps[i] * (16 * bits + 4);
+        cost += o.unit_cost * rbs[i] * S[i];
+        units += static_cast<long long>(rbs[i]) * S[i];
+    }
+    dp.total_cost = cost;
+
+    const long long want_ctas = (units + kDecodeWarpsPerCta - 1) / kDecodeWarpsPerCta;
+    const int n_ctas = static_cast<int>(std::max(1LL, std::min(want_ctas, static_cast<long long>(occ) * info->sms)));
+
+    cudaError_t e = launch_prep(pp, wsum, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prep launch");
+    e = launch_decode(dp, bits, mt, n_ctas, stream);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    g_launches += 2;
+    return ZQ_OK;
+}
+
+// Byte range of each buffer an op touches.
+struct Range {
+    uintptr_t lo, hi;
+};
+bool overlap(const Range &a, const Range &b) { return a.lo < b.hi && b.lo < a.hi; }
+
+struct OpRanges {
+    Range x, packed, scales, zeros, out;
+};
+
+OpRanges ranges_of(const zq_linear_desc &d) {
+    const size_t G = d.K / kGroup;
+    auto r = [](const void *p, size_t n) {
+        const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+        return Range{a, a + n};
+    };
+    return OpRanges{r(d.x, static_cast<size_t>(d.M) * d.K * 2),
+                    r(d.packed, static_cast<size_t>(d.N) * d.K * d.bits / 8),
+                    r(d.scales, static_cast<size_t>(d.N) * G * 2), r(d.zeros, static_cast<size_t>(d.N) * G * 2),
+                    r(d.out, static_cast<size_t>(d.M) * d.N * 2)};
+}
+
+// b depends on a (a earlier) if they share memory with at least one write.
+bool conflicts(const OpRanges &a, const OpRanges &b) {
+    const Range *reads_a[] = {&a.x, &a.packed, &a.scales, &a.zeros};
+    const Range *reads_b[] = {&b.x, &b.packed, &b.scales, &b.zeros};
+    for (const Range *r : reads_b)
+        if (overlap(a.out, *r)) return true;
+    for (const Range *r : reads_a)
+        if (overlap(b.out, *r)) return true;
+    return overlap(a.out, b.out);
+}
+
+// Expands a linear op into decode-sized pieces (M <= 64 per piece).
+void split_tokens(const zq_linear_desc &d, std::vector<zq_linear_desc> &out) {
+    for (int m0 = 0; m0 < d.M; m0 += 64) {
+        zq_linear_desc p = d;
+        p.M = std::min(64, d.M - m0);
+        p.x = d.x + static_cast<size_t>(m0) * d.K;
+        p.out = d.out + static_cast<size_t>(m0) * d.N;
+        out.push_back(p);
+    }
+}
+
+// Launches a batch of mutually independent ops: one launch per (bits, MT)
+// class, each holding at most kMaxDecodeOps ops and kMaxPrepEntries inputs.
+zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t stream) {
+    std::vector<zq_linear_desc> pieces;
+    for (const auto &d : batch) split_tokens(d, pieces);
+    const int bits_list[4] = {2, 3, 4, 8};
+    const int mt_list[4] = {1, 2, 4, 8};
+    for (int bits : bits_list)
+        for (int mt : mt_list) {
+            std::vector<zq_linear_desc> cls;
+            for (const auto &d : pieces)
+                if (d.bits == bits && mt_for_m(d.M) == mt) cls.push_back(d);
+            size_t i = 0;
+            while (i < cls.size()) {
+                std::vector<zq_linear_desc> launch;
+                std::vector<std::pair<const uint16_t *, int>> inputs;
+                while (i < cls.size() && launch.size() < static_cast<size_t>(kMaxDecodeOps)) {
+                    std::pair<const uint16_t *, int> key{cls[i].x, cls[i].M * 1000003 + cls[i].K};
+                    const bool known = std::find(inputs.begin(), inputs.end(), key) != inputs.end();
+                    if (!known && inputs.size() == static_cast<size_t>(kMaxPrepEntries)) break;
+                    if (!known) inputs.push_back(key);
+                    launch.push_back(cls[i++]);
+                }
+                zq_status st = run_decode(launch, bits, mt, stream);
+                if (st != ZQ_OK) return st;
+            }
+        }
+    return ZQ_OK;
+}
+
+}  // namespace
+
+// =================================================================== C ABI ==
+
+extern "C" {
+
+size_t zq_packed_words(int N, int K, int bits) {
+    if (!bits_ok(bits) || N <= 0 || K <= 0 || K % kGroup != 0) return 0;
+    return static_cast<size_t>(N) * K * bits / 32;
+}
+
+zq_status zq_quantize_pack(const float *w, int N, int K, int bits, int group, uint32_t *packed,
+                           uint16_t *scales, uint16_t *zeros, zq_stream_t stream) {
+    zq_status st = check_format(bits, group, N, K);
+    if (st != ZQ_OK) return st;
+    if ((st = check_ptr(w, "w")) != ZQ_OK) return st;
+    if ((st = check_ptr(packed, "packed")) != ZQ_OK) return st;
+    if ((st = check_ptr(scales, "scales")) != ZQ_OK) return st;
+    if ((st = check_ptr(zeros, "zeros")) != ZQ_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned long long id = g_quant_call.fetch_add(1);
+    const int slot = static_cast<int>(id % kQuantStatusSlots);
+    cudaError_t e = launch_quantize_pack(w, N, K, bits, packed, scales, zeros, slot, id, s);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    ++g_launches;
+    unsigned long long got = 0;
+    e = read_quant_status(slot, &got, s);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize status");
+    if (got == id) return fail(ZQ_ERR_NONFINITE, "weights contain NaN/Inf or |w| > 65504");
+    return ZQ_OK;
+}
+
+zq_status zq_linear(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                    const uint16_t *zeros, int bits, int group, int M, int N, int K, uint16_t *out,
+                    zq_stream_t stream) {
+    zq_linear_desc d{x, packed, scales, zeros, out, bits, group, M, N, K};
+    zq_status st = check_linear(d);
+    if (st != ZQ_OK) return st;
+    std::vector<zq_linear_desc> one{d};
+    return run_batch(one, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream) {
+    if (n_ops < 0 || (n_ops > 0 && ops == nullptr))
+        return fail(ZQ_ERR_INVALID_ARG, "ops is null or n_ops < 0");
+    for (int i = 0; i < n_ops; ++i) {
+        zq_status st = check_linear(ops[i]);
+        if (st != ZQ_OK) {
+            std::string msg = g_last_error;
+            return fail(st, "op %d: %s", i, msg.c_str());
+        }
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::vector<zq_linear_desc> batch;
+    std::vector<OpRanges> br;
+    constexpr size_t kMaxBatch = 1024;
+    for (int i = 0; i < n_ops; ++i) {
+        const OpRanges r = ranges_of(ops[i]);
+        bool dep = batch.size() >= kMaxBatch;
+        for (size_t j = 0; j < br.size() && !dep; ++j) dep = conflicts(br[j], r);
+        if (dep) {
+            zq_status st = run_batch(batch, s);
+            if (st != ZQ_OK) return st;
+            batch.clear();
+            br.clear();
+        }
+        batch.push_back(ops[i]);
+        br.push_back(r);
+    }
+    if (!batch.empty()) return run_batch(batch, s);
+    return ZQ_OK;
+}
+
+zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes, zq_stream_t stream) {
+    zq_status st = check_format(bits, kGroup, N, K);
+    if (st != ZQ_OK) return st;
+    if ((st = check_ptr(packed, "packed")) != ZQ_OK) return st;
+    if ((st = check_ptr(codes, "codes")) != ZQ_OK) return st;
+    cudaError_t e = launch_unpack(packed, N, K, bits, codes, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "unpack launch");
+    ++g_launches;
+    return ZQ_OK;
+}
+
+zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream) {
+    uint8_t *base = nullptr;
+    return workspace(reinterpret_cast<cudaStream_t>(stream), bytes, &base);
+}
+
+size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
+    zq_linear_desc d{nullptr, nullptr, nullptr, nullptr, nullptr, bits, kGroup, M, N, K};
+    if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
+    std::vector<zq_linear_desc> pieces;
+    split_tokens(d, pieces);
+    size_t worst = 0;
+    // pieces of one op share bits; group them as run_batch would
+    for (int mt : {1, 2, 4, 8}) {
+        std::vector<zq_linear_desc> cls;
+        for (const auto &p : pieces)
+            if (mt_for_m(p.M) == mt) cls.push_back(p);
+        for (size_t i = 0; i < cls.size(); i += kMaxPrepEntries) {
+            std::vector<zq_linear_desc> launch(cls.begin() + i,
+                                               cls.begin() + std::min(cls.size(), i + kMaxPrepEntries));
+            // distinct x per piece: give them distinct fake addresses
+            for (size_t k = 0; k < launch.size(); ++k)
+                launch[k].x = reinterpret_cast<const uint16_t *>(static_cast<uintptr_t>(16 * (k + 1)));
+            size_t b = 0;
+            if (run_decode(launch, bits, mt, nullptr, &b) != ZQ_OK) return 0;
+            worst = std::max(worst, b);
+        }
+    }
+    return worst;
+}
+
+const char *zq_status_string(zq_status status) {
+    switch (status) {
+        case ZQ_OK: return "ZQ_OK";
+        case ZQ_ERR_INVALID_ARG: return "ZQ_ERR_INVALID_ARG";
+        case ZQ_ERR_UNSUPPORTED: return "ZQ_ERR_UNSUPPORTED";
+        case ZQ_ERR_NONFINITE: return "ZQ_ERR_NONFINITE";
+        case ZQ_ERR_CUDA: return "ZQ_ERR_CUDA";
+        case ZQ_ERR_TIMEOUT: return "ZQ_ERR_TIMEOUT";
+    }
+    return "ZQ_UNKNOWN_STATUS";
+}
+
+const char *zq_last_error(void) { return g_last_error.c_str(); }
+
+uint64_t zq_kernel_launches(void) { return g_launches.load(); }
+
+int zq_version(void) { return 100; }
+
+}  // extern "C"

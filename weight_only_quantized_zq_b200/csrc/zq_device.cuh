@@ -1,0 +1,165 @@
+// zq_device.cuh — device building blocks shared by the zq kernels (sm_100a).
+//
+// Code unpack ([wiki] = "ZSE - open-source движок для запуска LLM локально на
+// GPU - 2026", section "Формат модели .zse": b-bit codes, asymmetric scale and
+// zero per 128 weights; the pages' DSL names INT4 unpack intrinsics in section
+// "Компилятор").  The codes are turned into exact fp16 integers with the
+// magic-exponent construction: a code q placed in the mantissa bits [s, s+b) of
+// a binary16 whose exponent field encodes 1024 reads as 1024 + q * 2^s, and one
+// fused multiply-add by (2^-s, -1024 * 2^-s) gives q exactly.  One LOP3 builds
+// two such halves at once (one per 16-bit half of a 32-bit register), so the
+// unpack yields half2 PAIRS of codes.  Which two codes share a pair depends on
+// b; it is fixed by pair_lo()/pair_hi() below, and the activation side is
+// permuted to the same order, so no repack of the canonical layout is needed.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace zq {
+
+// ---------------------------------------------------------------- PTX bits --
+
+__device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32_t magic) {
+    uint32_t r;  // (a & mask) | magic
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "r"(mask), "r"(magic));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t hfma2_bits(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t shf_r(uint32_t lo, uint32_t hi, uint32_t s) {
+    uint32_t r;  // low 32 bits of (hi:lo) >> s, s < 32
+    asm("shf.r.clamp.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(lo), "r"(hi), "r"(s));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// D = A * B + C, m16n8k16, A row-major fp16, B col-major fp16, fp32 accumulate.
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1,
+                                          const float (&c)[4]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 "
+        "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%11,%12,%13};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(c[0]), "f"(c[1]),
+          "f"(c[2]), "f"(c[3]));
+}
+
+// Programmatic dependent launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Ampere-style asynchronous global->shared copies, 16 bytes, L2 only.
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(s), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ldg_u16_nc(const uint16_t *p) {
+    unsigned short v;
+    asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ldg_u4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float h2f_bits(uint32_t h) {
+    return __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
+}
+
+// ------------------------------------------------------------ code unpack --
+//
+// A thread owns one 32-code chunk of a group: b consecutive uint32 words that
+// hold codes 0..31 of the chunk (the chunk starts on a word boundary for every
+// b because 32*b bits is a whole number of words).  pair p (0..15) is a half2
+// whose low half is code pair_lo(p) and whose high half is code pair_hi(p).
+
+template <int B>
+__host__ __device__ constexpr int pair_lo(int p) {
+    return B == 2 ? 16 * (p / 8) + p % 8
+         : B == 3 ? p
+         : B == 4 ? 8 * (p / 4) + p % 4
+                  : 4 * (p / 2) + p % 2;
+}
+template <int B>
+__host__ __device__ constexpr int pair_hi(int p) {
+    return pair_lo<B>(p) + (B == 2 ? 8 : B == 3 ? 16 : B == 4 ? 4 : 2);
+}
+
+// fp16x2 constants: magic 1024 in both halves; 2^-s; -1024 * 2^-s.
+constexpr uint32_t kMagic = 0x64006400u;
+__host__ __device__ constexpr uint32_t mul_s(int s) { return ((15u - s) << 10) * 0x10001u; }
+__host__ __device__ constexpr uint32_t add_s(int s) { return (0x8000u | ((25u - s) << 10)) * 0x10001u; }
+
+// code pair -> exact fp16x2 of the two integer codes.
+__device__ __forceinline__ uint32_t fix(uint32_t v, int s) { return hfma2_bits(v, mul_s(s), add_s(s)); }
+
+template <int B>
+__device__ __forceinline__ uint32_t unpack_pair(const uint32_t (&w)[B], int p);
+
+// b = 2: word i holds codes 16i..16i+15 at bits 2j.  Codes j and j+8 sit 16
+// bits apart; j = 0..4 are at mantissa offsets 0..8 of their halves, j = 5..7
+// are read from the word shifted right by 10.
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<2>(const uint32_t (&w)[2], int p) {
+    const uint32_t u = w[p / 8];
+    const int j = p % 8;
+    if (j < 5) return fix(lop_and_or(u, 0x00030003u << (2 * j), kMagic), 2 * j);
+    return fix(lop_and_or(u >> 10, 0x00030003u << (2 * (j - 5)), kMagic), 2 * (j - 5));
+}
+
+// b = 3: the chunk is 96 bits; codes p and p+16 are 48 bits apart.  Window m
+// (m = 0..5) joins stream bits [9m, 9m+16) and [9m+48, 9m+64) into one
+// register, where codes 3m+j and 3m+j+16 (j = 0..2) sit at offset 3j of the
+// two halves.
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<3>(const uint32_t (&w)[3], int p) {
+    const int m = p / 3, j = p % 3;
+    const int a = 9 * m;
+    const uint32_t lo = a < 32 ? shf_r(w[0], w[1], a) : shf_r(w[1], w[2], a - 32);
+    const uint32_t hi = a + 16 < 32 ? shf_r(w[1], w[2], a + 16) : (w[2] >> (a - 16));
+    const uint32_t r = prmt(lo, hi, 0x5410u);
+    return fix(lop_and_or(r, 0x00070007u << (3 * j), kMagic), 3 * j);
+}
+
+// b = 4: word i holds codes 8i..8i+7 (nibbles); pairs (j, j+4) at mantissa
+// offsets 0 and 4, from the word and from the word shifted right by 8.
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<4>(const uint32_t (&w)[4], int p) {
+    const uint32_t u = (p % 4) < 2 ? w[p / 4] : (w[p / 4] >> 8);
+    return (p % 2) == 0 ? fix(lop_and_or(u, 0x000F000Fu, kMagic), 0)
+                        : fix(lop_and_or(u, 0x00F000F0u, kMagic), 4);
+}
+
+// b = 8: word i holds codes 4i..4i+3 (bytes); pairs (0,2) and (1,3).
+template <>
+__device__ __forceinline__ uint32_t unpack_pair<8>(const uint32_t (&w)[8], int p) {
+    const uint32_t u = (p % 2) == 0 ? w[p / 2] : (w[p / 2] >> 8);
+    return fix(lop_and_or(u, 0x00FF00FFu, kMagic), 0);
+}
+
+}  // namespace zq

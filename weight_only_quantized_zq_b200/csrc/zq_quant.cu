@@ -1,0 +1,152 @@
+// zq_quant.cu — quantize-and-pack and the unpack test hook (sm_100a).
+//
+// Quantizer: [wiki] "ZSE - open-source движок для запуска LLM локально на GPU -
+// 2026", section "Формат модели .zse" (scale = (max - min)/15, zero = min,
+// q = clamp(round((w - zero)/scale), 0, 15), fp16 scale/zero, two INT4 codes per
+// byte, low nibble first), generalised to L = 2^b - 1 for the per-tensor INT2-8
+// widths of "ZSE: A Memory-Efficient LLM Inference Engine with Smart Resource
+// Orchestration", section "Technical Architecture".
+//
+// Arithmetic: fp64 with explicit round-to-nearest intrinsics (no contraction),
+// one rounding to fp16 for the stored scale and zero, q from the STORED fp16
+// values, round half to even.  This makes the result bit-identical to any
+// IEEE-754 implementation of the same steps.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "zq_device.cuh"
+#include "zq_internal.h"
+
+namespace zq {
+
+// Per-call status words for the non-finite check.  A call owns one slot, keyed
+// by a unique call id, so no clearing is needed between calls.
+__device__ unsigned long long g_quant_status[kQuantStatusSlots];
+
+__device__ __forceinline__ uint16_t f64_to_f16_bits(double v) {
+    return __half_as_ushort(__double2half(v));
+}
+
+// One warp per (row, group).  Each lane owns 4 consecutive weights.
+__global__ void __launch_bounds__(256) quantize_pack_kernel(
+    const float *__restrict__ w, int N, int K, int bits, uint32_t *__restrict__ packed,
+    uint16_t *__restrict__ scales, uint16_t *__restrict__ zeros, int slot,
+    unsigned long long call_id) {
+    __shared__ uint32_t words[8][32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = K / 128;
+    const long long item = static_cast<long long>(blockIdx.x) * 8 + warp;
+    if (item >= static_cast<long long>(N) * G) return;
+    const int n = static_cast<int>(item / G), g = static_cast<int>(item % G);
+    const int L = (1 << bits) - 1;
+
+    const float4 v4 = *reinterpret_cast<const float4 *>(w + static_cast<size_t>(n) * K +
+                                                        static_cast<size_t>(g) * 128 + lane * 4);
+    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+    bool bad = false;
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        bad |= !(fabsf(v[i]) <= 65504.0f);  // NaN compares false
+        mn = fminf(mn, v[i]);
+        mx = fmaxf(mx, v[i]);
+    }
+    if (__any_sync(0xffffffffu, bad)) {
+        if (lane == 0) atomicExch(&g_quant_status[slot], call_id);
+        return;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const uint16_t z16 = f64_to_f16_bits(static_cast<double>(mn));
+    const uint16_t s16 = f64_to_f16_bits(
+        __ddiv_rn(__dsub_rn(static_cast<double>(mx), static_cast<double>(mn)), static_cast<double>(L)));
+    const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
+    const double z = static_cast<double>(__half2float(__ushort_as_half(z16)));
+
+    uint32_t chunk = 0;  // this lane's 4 codes, 4*bits bits
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t q = 0;
+        if (s != 0.0) {
+            double t = rint(__ddiv_rn(__dsub_rn(static_cast<double>(v[i]), z), s));
+            t = fmin(fmax(t, 0.0), static_cast<double>(L));
+            q = static_cast<uint32_t>(t);
+        }
+        chunk |= q << (bits * i);
+    }
+    // Assemble the group's 4*bits words: lane's chunk starts at stream bit 4*bits*lane.
+    const int nw = 4 * bits;
+    if (lane < nw) words[warp][lane] = 0;
+    __syncwarp();
+    const int bit0 = 4 * bits * lane;
+    const int wi = bit0 >> 5, off = bit0 & 31;
+    atomicOr(&words[warp][wi], chunk << off);
+    if (off + 4 * bits > 32) atomicOr(&words[warp][wi + 1], chunk >> (32 - off));
+    __syncwarp();
+    const size_t wpr = static_cast<size_t>(K) * bits / 32;
+    if (lane < nw) packed[static_cast<size_t>(n) * wpr + static_cast<size_t>(g) * nw + lane] = words[warp][lane];
+    if (lane == 0) {
+        scales[static_cast<size_t>(n) * G + g] = s16;
+        zeros[static_cast<size_t>(n) * G + g] = z16;
+    }
+}
+
+// Unpack test hook: one thread per 32-code chunk, through unpack_pair<B>, the
+// routine the linear kernels use.
+template <int B>
+__global__ void unpack_kernel(const uint32_t *__restrict__ packed, int N, int K,
+                              uint8_t *__restrict__ codes) {
+    const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int chunks_per_row = K / 32;
+    if (t >= static_cast<long long>(N) * chunks_per_row) return;
+    const int n = static_cast<int>(t / chunks_per_row), c = static_cast<int>(t % chunks_per_row);
+    const uint32_t *src = packed + static_cast<size_t>(n) * (static_cast<size_t>(K) * B / 32) +
+                          static_cast<size_t>(c) * B;
+    uint32_t w[B];
+#pragma unroll
+    for (int i = 0; i < B; ++i) w[i] = src[i];
+    uint8_t *dst = codes + static_cast<size_t>(n) * K + static_cast<size_t>(c) * 32;
+#pragma unroll
+    for (int p = 0; p < 16; ++p) {
+        const uint32_t h2 = unpack_pair<B>(w, p);
+        const float lo = h2f_bits(h2 & 0xFFFFu), hi = h2f_bits(h2 >> 16);
+        dst[pair_lo<B>(p)] = static_cast<uint8_t>(lo);
+        dst[pair_hi<B>(p)] = static_cast<uint8_t>(hi);
+    }
+}
+
+cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, uint32_t *packed,
+                                 uint16_t *scales, uint16_t *zeros, int slot,
+                                 unsigned long long call_id, cudaStream_t stream) {
+    const long long items = static_cast<long long>(N) * (K / 128);
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    quantize_pack_kernel<<<blocks, 256, 0, stream>>>(w, N, K, bits, packed, scales, zeros, slot,
+                                                     call_id);
+    return cudaGetLastError();
+}
+
+cudaError_t read_quant_status(int slot, unsigned long long *value, cudaStream_t stream) {
+    cudaError_t e = cudaMemcpyFromSymbolAsync(value, g_quant_status, sizeof(unsigned long long),
+                                              sizeof(unsigned long long) * slot,
+                                              cudaMemcpyDeviceToHost, stream);
+    if (e != cudaSuccess) return e;
+    return cudaStreamSynchronize(stream);
+}
+
+cudaError_t launch_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes,
+                          cudaStream_t stream) {
+    const long long threads = static_cast<long long>(N) * (K / 32);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    switch (bits) {
+        case 2: unpack_kernel<2><<<blocks, 256, 0, stream>>>(packed, N, K, codes); break;
+        case 3: unpack_kernel<3><<<blocks, 256, 0, stream>>>(packed, N, K, codes); break;
+        case 4: unpack_kernel<4><<<blocks, 256, 0, stream>>>(packed, N, K, codes); break;
+        default: unpack_kernel<8><<<blocks, 256, 0, stream>>>(packed, N, K, codes); break;
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace zq
