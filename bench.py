@@ -315,12 +315,22 @@ def run_zq(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = world * wl.bytes * args.steps / (e2e_ms / 1e3) / 1e9
 
-    # Roofline of the dominant kernel (the grouped decode launch): the step is
-    # one prep launch + one decode launch, timed together by the events above.
+    # Roofline of the dominant kernel.  Decode (M <= 64): the grouped decode
+    # launch; the step is one prep launch + one decode launch, timed together
+    # by the events above, so the figure is a lower bound for the kernel.
+    # Prefill (M > 64): the tcgen05 kernels, one launch per projection.
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": achieved / peaks["hbm_gbs"], "traffic": None,
-                "peak_source": peaks["source"], "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel"}
+    if M <= 64:
+        roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                    "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "peak_source": peaks["source"], "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel"}
+    else:
+        tflops = wl.flops / (ms_step / 1e3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
+                    "frac": tflops / peak, "traffic": None,
+                    "peak_source": peaks["source"] + " (dense bf16 sustained; fp16 has the same dense rate)",
+                    "kernel": "prefill_kernel<4>", "tflops_vs_nominal_2250": tflops / 2250.0}
 
     line = None
     if rank == 0:
@@ -335,8 +345,9 @@ def run_zq(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f16 in, f32 accumulate, int4 weights", "data": "synthetic",
-                "config": {"workload": f"qwen2.5-7b-shaped decode stack: {args.layers} layers x (qkv, o, "
-                                       f"gate_up, down), M={M}, INT4 g128, one zq_linear_stack call",
+                "config": {"workload": f"qwen2.5-7b-shaped {'decode' if M <= 64 else 'prefill'} stack: "
+                                       f"{args.layers} layers x (qkv, o, gate_up, down), M={M}, INT4 g128, "
+                                       f"one zq_linear_stack call",
                            "layers": args.layers, "M": M, "bits": 4, "group": 128,
                            "bytes_per_step": wl.bytes, "flops_per_step": wl.flops,
                            "l2": f"inputs larger than L2 ({wl.bytes / 1e9:.2f} GB per step)",

@@ -140,7 +140,8 @@ ZQ_API zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits,
  * Useful before graph capture.  Synchronous. */
 ZQ_API zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream);
 
-/* Workspace bytes zq_linear needs for these sizes (0 if none). */
+/* Workspace bytes zq_linear needs for these sizes (0 if none; M > 64 needs
+ * none). */
 ZQ_API size_t zq_linear_workspace_bytes(int bits, int M, int N, int K);
 
 /* Human-readable name of a status code (static storage). */
@@ -148,6 +149,11 @@ ZQ_API const char *zq_status_string(zq_status status);
 
 /* Message of the most recent failure on the calling thread ("" if none). */
 ZQ_API const char *zq_last_error(void);
+
+/* Waits for the current device to finish all work, then reports whether any
+ * of this library's kernels gave up a bounded wait (ZQ_ERR_TIMEOUT) since the
+ * last call; clears that record.  Synchronous. */
+ZQ_API zq_status zq_check_device(void);
 
 /* Number of kernels this library has launched in this process (all devices).
  * Lets a caller count device work, e.g. inside a timed region. */

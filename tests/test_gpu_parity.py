@@ -109,6 +109,20 @@ def test_linear_shapes(zq, orc, bits):
         _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"bits={bits} M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("bits", BITS)
+def test_prefill_shapes(zq, orc, bits):
+    """M > 64 runs the tcgen05 prefill family: ragged token tiles (TMA zero
+    fill), ragged weight-row tiles, N not a multiple of 8 (scalar stores)."""
+    cases = [(65, 31, 256), (130, 70, 512), (256, 256, 128), (300, 520, 1024), (257, 264, 384),
+             (512, 256, 3584), (1000, 1000, 640)]
+    for i, (M, N, K) in enumerate(cases):
+        w = zi.weight(N, K, seed=3000 + 10 * bits + i, device="cuda", outliers=(i % 2 == 0))
+        q = _quantize_both(zq, orc, w, bits)
+        x = zi.activations(M, K, seed=4000 + i, device="cuda")
+        _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"prefill bits={bits} M={M} N={N} K={K}")
+    zq.zq_check_device()
+
+
 def test_linear_adversarial_all_positive(zq, orc):
     """All-positive x and weights: errors cannot cancel (worst case of fp32
     accumulation against the bound)."""
@@ -116,8 +130,9 @@ def test_linear_adversarial_all_positive(zq, orc):
         N, K = 64, 18944
         w = zi.weight(N, K, seed=31 + bits, device="cuda").abs()
         q = _quantize_both(zq, orc, w, bits)
-        x = zi.activations(4, K, seed=32, device="cuda").abs()
-        _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"all-positive bits={bits}")
+        for M in (4, 300):
+            x = zi.activations(M, K, seed=32, device="cuda").abs()
+            _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"all-positive bits={bits} M={M}")
 
 
 def test_config1_single_layer(zq, orc):

@@ -27,7 +27,8 @@ GROUP = 128
 # Every symbol the header declares (checked by the CPU test suite).
 EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_linear", "zq_linear_stack",
            "zq_unpack", "zq_reserve_workspace", "zq_linear_workspace_bytes",
-           "zq_status_string", "zq_last_error", "zq_kernel_launches", "zq_version")
+           "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
+           "zq_version")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -56,6 +57,8 @@ _lib.zq_status_string.argtypes = [_I]
 _lib.zq_status_string.restype = ctypes.c_char_p
 _lib.zq_last_error.argtypes = []
 _lib.zq_last_error.restype = ctypes.c_char_p
+_lib.zq_check_device.argtypes = []
+_lib.zq_check_device.restype = _I
 _lib.zq_kernel_launches.argtypes = []
 _lib.zq_kernel_launches.restype = ctypes.c_uint64
 _lib.zq_version.argtypes = []
@@ -105,6 +108,10 @@ def zq_last_error():
 
 def zq_version():
     return _lib.zq_version()
+
+
+def zq_check_device():
+    _check(_lib.zq_check_device())
 
 
 def zq_kernel_launches():

@@ -201,26 +201,31 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     if (keys.size() > static_cast<size_t>(kMaxPrepEntries) || ops.size() > static_cast<size_t>(kMaxDecodeOps))
         return fail(ZQ_ERR_INVALID_ARG, "internal: decode launch too large");
 
-    // Split-K: only when the row blocks alone cannot keep every warp busy.
-    long long rb_total = 0;
+    // Split-K.  Work is spread over warps by byte cost, each warp taking the
+    // units that start in its share; a unit may overrun the share, so units
+    // are capped at 1/16 of a share (load balance), and small launches are
+    // split until every warp has work.
+    long long rb_total = 0, cost_total = 0;
     std::vector<int> rbs(ops.size()), S(ops.size(), 1), gps(ops.size());
     for (size_t i = 0; i < ops.size(); ++i) {
         rbs[i] = (ops[i].N + rows - 1) / rows;
         rb_total += rbs[i];
         gps[i] = ops[i].K / kGroup;
+        cost_total += static_cast<long long>(rbs[i]) * rows * gps[i] * (16 * bits + 4);
     }
-    const long long target = 2 * max_warps;
+    const long long share = std::max(1LL, cost_total / max_warps);
+    const long long cap = std::max(1LL, share / 16);
+    const double fill = rb_total < 2 * max_warps ? static_cast<double>(2 * max_warps) / rb_total : 1.0;
     size_t counters = 0;
-    if (rb_total < target) {
-        const double f = static_cast<double>(target) / static_cast<double>(rb_total);
-        for (size_t i = 0; i < ops.size(); ++i) {
-            const int G = ops[i].K / kGroup;
-            int s = std::min(G, static_cast<int>(f + 0.999));
-            if (s <= 1 || counters + rbs[i] > kMaxCounters) continue;
-            gps[i] = (G + s - 1) / s;
-            S[i] = (G + gps[i] - 1) / gps[i];
-            if (S[i] > 1) counters += rbs[i];
-        }
+    for (size_t i = 0; i < ops.size(); ++i) {
+        const int G = ops[i].K / kGroup;
+        const long long unit1 = static_cast<long long>(rows) * G * (16 * bits + 4);
+        long long want = std::max(static_cast<long long>(fill + 0.999), (unit1 + cap - 1) / cap);
+        int s = static_cast<int>(std::min<long long>(G, want));
+        if (s <= 1 || counters + rbs[i] > kMaxCounters) continue;
+        gps[i] = (G + s - 1) / s;
+        S[i] = (G + gps[i] - 1) / gps[i];
+        if (S[i] > 1) counters += rbs[i];
     }
 
     // Workspace layout.
@@ -229,7 +234,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     for (size_t e = 0; e < keys.size(); ++e) {
         prep_off[e] = off;
         const size_t G = keys[e].K / kGroup;
-        off += align256(static_cast<size_t>(mpad) * keys[e].K * 2) + align256(G * mpad * 4);
+        off += align256(static_cast<size_t>(mpad) * keys[e].K * 2) + align256(G * mpad * 8);
     }
     for (size_t i = 0; i < ops.size(); ++i)
         if (S[i] > 1) {
@@ -341,22 +346,41 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
     return overlap(a.out, b.out);
 }
 
-// Expands a linear op into decode-sized pieces (M <= 64 per piece).
+// Expands a linear op into decode-sized pieces (M <= 64 per piece); only used
+// for ops that the prefill family does not take.
 void split_tokens(const zq_linear_desc &d, std::vector<zq_linear_desc> &out) {
-    for (int m0 = 0; m0 < d.M; m0 += 64) {
+    for (int m0 = 0; m0 < d.M; m0 += kDecodeMaxM) {
         zq_linear_desc p = d;
-        p.M = std::min(64, d.M - m0);
+        p.M = std::min(kDecodeMaxM, d.M - m0);
         p.x = d.x + static_cast<size_t>(m0) * d.K;
         p.out = d.out + static_cast<size_t>(m0) * d.N;
         out.push_back(p);
     }
 }
 
+zq_status run_prefill(const zq_linear_desc &d, cudaStream_t stream) {
+    DeviceInfo *info = nullptr;
+    zq_status st = device_info(&info);
+    if (st != ZQ_OK) return st;
+    cudaError_t e = launch_prefill(d.x, d.packed, d.scales, d.zeros, d.bits, d.M, d.N, d.K, d.out, info->sms,
+                                   stream);
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    g_launches += 1;
+    return ZQ_OK;
+}
+
 // Launches a batch of mutually independent ops: one launch per (bits, MT)
 // class, each holding at most kMaxDecodeOps ops and kMaxPrepEntries inputs.
 zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t stream) {
     std::vector<zq_linear_desc> pieces;
-    for (const auto &d : batch) split_tokens(d, pieces);
+    for (const auto &d : batch) {
+        if (d.M > kDecodeMaxM) {
+            zq_status st = run_prefill(d, stream);
+            if (st != ZQ_OK) return st;
+        } else {
+            pieces.push_back(d);
+        }
+    }
     const int bits_list[4] = {2, 3, 4, 8};
     const int mt_list[4] = {1, 2, 4, 8};
     for (int bits : bits_list)
@@ -473,7 +497,7 @@ zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream) {
 
 size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
     zq_linear_desc d{nullptr, nullptr, nullptr, nullptr, nullptr, bits, kGroup, M, N, K};
-    if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
+    if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0 || M > kDecodeMaxM) return 0;
     std::vector<zq_linear_desc> pieces;
     split_tokens(d, pieces);
     size_t worst = 0;
@@ -511,6 +535,16 @@ const char *zq_status_string(zq_status status) {
 const char *zq_last_error(void) { return g_last_error.c_str(); }
 
 uint64_t zq_kernel_launches(void) { return g_launches.load(); }
+
+zq_status zq_check_device(void) {
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    int err = 0;
+    e = read_prefill_error(&err);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (err != 0) return fail(static_cast<zq_status>(err), "a kernel gave up a bounded wait");
+    return ZQ_OK;
+}
 
 int zq_version(void) { return 100; }
 

@@ -14,9 +14,12 @@
 //    applied once per group in fp32.  sum_k x_k per group is precomputed.
 //  * Swap-AB: weight rows fill the 16-row side of the MMA, tokens the 8-column
 //    side, so M = 1..8 costs one MMA column tile.
-//  * Codes become fp16 pairs with one LOP3 + one HFMA2 per two codes
-//    (zq_device.cuh).  The activations are pre-permuted once per call into the
-//    same pair order, so the canonical packed layout is consumed as stored.
+//  * Codes become biased fp16 pairs, 1024 + q * 2^s, with one LOP3 per two codes
+//    (zq_device.cuh) and go to the tensor cores as they are: the activations
+//    are pre-permuted once per call into the same pair order and pre-scaled by
+//    2^-s (exact), so each product is 1024 * x' + q * x, and the per-group bias
+//    1024 * sum(x') is subtracted in fp32 once per group.  The canonical packed
+//    layout is consumed as stored.
 //  * Packed codes stream through a per-warp shared-memory ring with cp.async
 //    (16-byte chunks, several steps in flight, no register cost); the ring is
 //    per warp, so no block-level barrier is needed.
@@ -37,15 +40,19 @@ namespace zq {
 // x and the fp32 group sum.  Tokens >= M are written as zeros.
 
 template <int B>
-__device__ __forceinline__ void prep_group(const uint16_t *xrow, uint16_t *prow, int lane) {
+__device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow, int lane) {
+    float bias = 0.0f;  // sum of the scaled activations written by this lane
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int q = lane + 32 * h;  // 64 pairs per group
         const int c = q / 16, p = q % 16;
-        const uint32_t lo = xrow[32 * c + pair_lo<B>(p)];
-        const uint32_t hi = xrow[32 * c + pair_hi<B>(p)];
-        reinterpret_cast<uint32_t *>(prow)[16 * c + p] = lo | (hi << 16);
+        const float sc = 1.0f / static_cast<float>(1 << pair_shift<B>(p));  // exact power of two
+        const __half lo = __float2half_rn(h2f_bits(xrow[32 * c + pair_lo<B>(p)]) * sc);
+        const __half hi = __float2half_rn(h2f_bits(xrow[32 * c + pair_hi<B>(p)]) * sc);
+        bias += __half2float(lo) + __half2float(hi);
+        reinterpret_cast<uint32_t *>(prow)[16 * c + p] = __half_as_ushort(lo) | (__half_as_ushort(hi) << 16);
     }
+    return bias;
 }
 
 __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepParams p,
@@ -61,23 +68,28 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
         const int G = en.K / kGroup;
         const int t = static_cast<int>(local / G), g = static_cast<int>(local % G);
         uint16_t *prow = en.xperm + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
+        float2 *dst = reinterpret_cast<float2 *>(en.sx) + static_cast<size_t>(g) * en.M_pad + t;
         if (t >= en.M) {
             reinterpret_cast<uint2 *>(prow)[lane] = make_uint2(0u, 0u);
-            if (lane == 0) en.sx[static_cast<size_t>(g) * en.M_pad + t] = 0.0f;
+            if (lane == 0) *dst = make_float2(0.0f, 0.0f);
         } else {
             const uint16_t *xrow = en.x + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             const uint2 v = reinterpret_cast<const uint2 *>(xrow)[lane];
             float s = h2f_bits(v.x & 0xFFFFu) + h2f_bits(v.x >> 16) + h2f_bits(v.y & 0xFFFFu) +
                       h2f_bits(v.y >> 16);
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-            if (lane == 0) en.sx[static_cast<size_t>(g) * en.M_pad + t] = s;
+            float b;
             switch (en.bits) {
-                case 2: prep_group<2>(xrow, prow, lane); break;
-                case 3: prep_group<3>(xrow, prow, lane); break;
-                case 4: prep_group<4>(xrow, prow, lane); break;
-                default: prep_group<8>(xrow, prow, lane); break;
+                case 2: b = prep_group<2>(xrow, prow, lane); break;
+                case 3: b = prep_group<3>(xrow, prow, lane); break;
+                case 4: b = prep_group<4>(xrow, prow, lane); break;
+                default: b = prep_group<8>(xrow, prow, lane); break;
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                s += __shfl_xor_sync(0xffffffffu, s, o);
+                b += __shfl_xor_sync(0xffffffffu, b, o);
+            }
+            if (lane == 0) *dst = make_float2(s, 1024.0f * b);
         }
     }
     // Dependents may be scheduled only now, i.e. after everything enqueued
@@ -118,12 +130,58 @@ __device__ __forceinline__ void cursor_next(Cursor &cu, const DecodeParams &p, l
     }
 }
 
+// Per-step operands other than the codes (activations, group sums, scales,
+// zeros), loaded one step ahead into registers so their L1/L2 latency overlaps
+// the previous step's math.
+template <int MT, int RT>
+struct StepOperands {
+    uint32_t xf[MT][16];  // B fragments: 16 half2 pairs per token tile
+    float4 sb[MT];        // (sum x, bias) for this thread's two C-fragment tokens
+    uint32_t sz[RT][2];   // (scale | zero << 16) of this thread's C-fragment rows
+};
+
+template <int MT, int RT>
+__device__ __forceinline__ void load_operands(StepOperands<MT, RT> &v, const DecodeOp &op, const Cursor &cu,
+                                              int gq, int c) {
+    constexpr int MPAD = 8 * MT;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int tok = 8 * mt + gq;
+        if (tok < op.M) {
+            const uint16_t *xp = op.xperm + static_cast<size_t>(tok) * op.K + static_cast<size_t>(cu.g) * kGroup + 32 * c;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = ldg_u4(xp + 8 * q);
+                v.xf[mt][4 * q + 0] = w.x;
+                v.xf[mt][4 * q + 1] = w.y;
+                v.xf[mt][4 * q + 2] = w.z;
+                v.xf[mt][4 * q + 3] = w.w;
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) v.xf[mt][q] = 0u;
+        }
+        if (8 * mt + 2 * c < op.M)
+            v.sb[mt] = *reinterpret_cast<const float4 *>(op.sx + 2 * (static_cast<size_t>(cu.g) * MPAD + 8 * mt + 2 * c));
+        else
+            v.sb[mt] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int r = min(cu.r0 + rt * 16 + h * 8 + gq, op.N - 1);
+            const size_t idx = static_cast<size_t>(r) * op.G + cu.g;
+            v.sz[rt][h] = ldg_u16_nc(op.scales + idx) | (ldg_u16_nc(op.zeros + idx) << 16);
+        }
+}
+
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32)
+__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 1)
     decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int RT = decode_rt(MT);
     constexpr int ROWS = 16 * RT;
-    constexpr int D = decode_depth(BITS);
+    constexpr int D = decode_depth(BITS, MT);
     constexpr int ROW_BYTES = 16 * BITS;  // one row of one group
     constexpr int STAGE = ROWS * ROW_BYTES;
     constexpr int CHUNKS = ROWS * BITS;   // 16-byte chunks per stage
@@ -141,17 +199,17 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32)
     const long long c_begin = p.total_cost * gw / W;
     const long long c_end = p.total_cost * (gw + 1) / W;
 
-    Cursor cs;
+    Cursor nx;  // next step to compute (operands prefetched for it)
     {
         int o = 0;
         while (o + 1 < p.n_ops && p.ops[o + 1].cost0 <= c_begin) ++o;
         const DecodeOp &op = p.ops[o];
         const long long rel = c_begin - op.cost0;
-        cs.o = o;
-        cs.u = static_cast<int>((rel + op.unit_cost - 1) / op.unit_cost);
-        cursor_unit<ROWS>(cs, p, c_end);
+        nx.o = o;
+        nx.u = static_cast<int>((rel + op.unit_cost - 1) / op.unit_cost);
+        cursor_unit<ROWS>(nx, p, c_end);
     }
-    Cursor ld = cs;
+    Cursor ld = nx;
 
     auto issue = [&](const Cursor &cu, int slot) {
         const DecodeOp &op = p.ops[cu.o];
@@ -185,6 +243,9 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32)
     pdl_wait();  // the prepared activations come from the previous kernel
     pdl_launch_dependents();
 
+    StepOperands<MT, RT> opA, opB;
+    if (nx.valid) load_operands<MT, RT>(opA, p.ops[nx.o], nx, gq, c);
+
     float tot[RT][MT][4];
 #pragma unroll
     for (int a = 0; a < RT; ++a)
@@ -194,8 +255,13 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32)
             for (int i = 0; i < 4; ++i) tot[a][b][i] = 0.0f;
     const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 
-#pragma unroll 1
-    while (cs.valid) {
+    // One step: consume `cv` (operands of the step at `nx`), prefetch the next
+    // step's operands into `nv`.
+    auto step = [&](const StepOperands<MT, RT> &cv, StepOperands<MT, RT> &nv) {
+        const Cursor cs = nx;
+        cursor_next<ROWS>(nx, p, c_end);
+        if (nx.valid) load_operands<MT, RT>(nv, p.ops[nx.o], nx, gq, c);
+
         __syncwarp();
         if (ld.valid) {
             issue(ld, slot_ld);
@@ -204,102 +270,72 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32)
         cp_async_commit();
         slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
 
-        const DecodeOp &op = p.ops[cs.o];
-        // Activations, group sums, scales and zeros of this step (L1/L2 hits).
-        uint32_t xf[MT][16];
-        float sxv[MT][2];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const uint16_t *xp = op.xperm + static_cast<size_t>(8 * mt + gq) * op.K +
-                                 static_cast<size_t>(cs.g) * kGroup + 32 * c;
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const uint4 q = ldg_u4(xp + 8 * v);
-                xf[mt][4 * v + 0] = q.x;
-                xf[mt][4 * v + 1] = q.y;
-                xf[mt][4 * v + 2] = q.z;
-                xf[mt][4 * v + 3] = q.w;
-            }
-            const float2 s2 = *reinterpret_cast<const float2 *>(op.sx + static_cast<size_t>(cs.g) * MPAD + 8 * mt + 2 * c);
-            sxv[mt][0] = s2.x;
-            sxv[mt][1] = s2.y;
-        }
-        float sc[RT][2], zr[RT][2];
-#pragma unroll
-        for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = min(cs.r0 + rt * 16 + h * 8 + gq, op.N - 1);
-                const size_t idx = static_cast<size_t>(r) * op.G + cs.g;
-                sc[rt][h] = h2f_bits(ldg_u16_nc(op.scales + idx));
-                zr[rt][h] = h2f_bits(ldg_u16_nc(op.zeros + idx));
-            }
-
         cp_async_wait<D - 1>();
         __syncwarp();
         const uint8_t *st = ring + slot_cs * STAGE;
         slot_cs = slot_cs + 1 == D ? 0 : slot_cs + 1;
 
-        uint32_t wv[RT][2][BITS];
 #pragma unroll
-        for (int rt = 0; rt < RT; ++rt)
+        for (int rt = 0; rt < RT; ++rt) {
+            uint32_t wv[2][BITS];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int row = rt * 16 + h * 8 + gq;
                 const uint8_t *rp = st + row * ROW_BYTES;
                 if constexpr (BITS == 2) {
                     const uint2 v = *reinterpret_cast<const uint2 *>(rp + 8 * c);
-                    wv[rt][h][0] = v.x;
-                    wv[rt][h][1] = v.y;
+                    wv[h][0] = v.x;
+                    wv[h][1] = v.y;
                 } else if constexpr (BITS == 3) {
                     const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + 12 * c);
-                    wv[rt][h][0] = q[0];
-                    wv[rt][h][1] = q[1];
-                    wv[rt][h][2] = q[2];
+                    wv[h][0] = q[0];
+                    wv[h][1] = q[1];
+                    wv[h][2] = q[2];
                 } else if constexpr (BITS == 4) {
                     const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * c);
-                    wv[rt][h][0] = v.x;
-                    wv[rt][h][1] = v.y;
-                    wv[rt][h][2] = v.z;
-                    wv[rt][h][3] = v.w;
+                    wv[h][0] = v.x;
+                    wv[h][1] = v.y;
+                    wv[h][2] = v.z;
+                    wv[h][3] = v.w;
                 } else {
                     const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + 16 * ((2 * c) ^ (row & 7)));
                     const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + 16 * ((2 * c + 1) ^ (row & 7)));
-                    wv[rt][h][0] = v0.x; wv[rt][h][1] = v0.y; wv[rt][h][2] = v0.z; wv[rt][h][3] = v0.w;
-                    wv[rt][h][4] = v1.x; wv[rt][h][5] = v1.y; wv[rt][h][6] = v1.z; wv[rt][h][7] = v1.w;
+                    wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
+                    wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
                 }
             }
-
-        float acc[RT][MT][4];
+            float acc[MT][4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-#pragma unroll
-            for (int rt = 0; rt < RT; ++rt) {
-                const uint32_t a0 = unpack_pair<BITS>(wv[rt][0], 2 * j);
-                const uint32_t a1 = unpack_pair<BITS>(wv[rt][1], 2 * j);
-                const uint32_t a2 = unpack_pair<BITS>(wv[rt][0], 2 * j + 1);
-                const uint32_t a3 = unpack_pair<BITS>(wv[rt][1], 2 * j + 1);
+            for (int j = 0; j < 8; ++j) {
+                const uint32_t a0 = unpack_biased<BITS>(wv[0], 2 * j);
+                const uint32_t a1 = unpack_biased<BITS>(wv[1], 2 * j);
+                const uint32_t a2 = unpack_biased<BITS>(wv[0], 2 * j + 1);
+                const uint32_t a3 = unpack_biased<BITS>(wv[1], 2 * j + 1);
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
                     if (j == 0)
-                        mma_16816(acc[rt][mt], a0, a1, a2, a3, xf[mt][2 * j], xf[mt][2 * j + 1], zero4);
+                        mma_16816(acc[mt], a0, a1, a2, a3, cv.xf[mt][2 * j], cv.xf[mt][2 * j + 1], zero4);
                     else
-                        mma_16816(acc[rt][mt], a0, a1, a2, a3, xf[mt][2 * j], xf[mt][2 * j + 1], acc[rt][mt]);
+                        mma_16816(acc[mt], a0, a1, a2, a3, cv.xf[mt][2 * j], cv.xf[mt][2 * j + 1], acc[mt]);
+                }
+            }
+            // Per-group epilogue: tot += s * (acc - bias) + z * sum(x).
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const float sc = h2f_bits(cv.sz[rt][h] & 0xFFFFu);
+                const float zr = h2f_bits(cv.sz[rt][h] >> 16);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    float &t0 = tot[rt][mt][2 * h], &t1 = tot[rt][mt][2 * h + 1];
+                    t0 = fmaf(sc, acc[mt][2 * h] - cv.sb[mt].y, fmaf(zr, cv.sb[mt].x, t0));
+                    t1 = fmaf(sc, acc[mt][2 * h + 1] - cv.sb[mt].w, fmaf(zr, cv.sb[mt].z, t1));
                 }
             }
         }
-        // Per-group epilogue: tot += s * sum(q x) + z * sum(x).
-#pragma unroll
-        for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    tot[rt][mt][i] = fmaf(sc[rt][i >> 1], acc[rt][mt][i],
-                                          fmaf(zr[rt][i >> 1], sxv[mt][i & 1], tot[rt][mt][i]));
 
         if (cs.g + 1 == cs.g_end) {
             // End of a unit: emit.
+            const DecodeOp &op = p.ops[cs.o];
             if (op.S == 1) {
 #pragma unroll
                 for (int rt = 0; rt < RT; ++rt)
@@ -352,7 +388,13 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) tot[rt][mt][i] = 0.0f;
         }
-        cursor_next<ROWS>(cs, p, c_end);
+    };
+
+#pragma unroll 1
+    while (nx.valid) {
+        step(opA, opB);
+        if (!nx.valid) break;
+        step(opB, opA);
     }
     cp_async_wait<0>();
 }

@@ -5,10 +5,10 @@
 // zero per 128 weights; the pages' DSL names INT4 unpack intrinsics in section
 // "Компилятор").  The codes are turned into exact fp16 integers with the
 // magic-exponent construction: a code q placed in the mantissa bits [s, s+b) of
-// a binary16 whose exponent field encodes 1024 reads as 1024 + q * 2^s, and one
-// fused multiply-add by (2^-s, -1024 * 2^-s) gives q exactly.  One LOP3 builds
-// two such halves at once (one per 16-bit half of a 32-bit register), so the
-// unpack yields half2 PAIRS of codes.  Which two codes share a pair depends on
+// a binary16 whose exponent field encodes 1024 reads as 1024 + q * 2^s (the
+// "biased" value); one fused multiply-add by (2^-s, -1024 * 2^-s) gives q
+// exactly.  One LOP3 builds two such halves at once (one per 16-bit half of a
+// 32-bit register), so the unpack yields half2 PAIRS of codes.  Which two codes share a pair depends on
 // b; it is fixed by pair_lo()/pair_hi() below, and the activation side is
 // permuted to the same order, so no repack of the canonical layout is needed.
 #pragma once
@@ -115,21 +115,29 @@ constexpr uint32_t kMagic = 0x64006400u;
 __host__ __device__ constexpr uint32_t mul_s(int s) { return ((15u - s) << 10) * 0x10001u; }
 __host__ __device__ constexpr uint32_t add_s(int s) { return (0x8000u | ((25u - s) << 10)) * 0x10001u; }
 
-// code pair -> exact fp16x2 of the two integer codes.
-__device__ __forceinline__ uint32_t fix(uint32_t v, int s) { return hfma2_bits(v, mul_s(s), add_s(s)); }
-
+// Mantissa offset s of the codes of pair p: the biased pair reads
+// (1024 + q_lo * 2^s, 1024 + q_hi * 2^s).
 template <int B>
-__device__ __forceinline__ uint32_t unpack_pair(const uint32_t (&w)[B], int p);
+__host__ __device__ constexpr int pair_shift(int p) {
+    return B == 2 ? ((p % 8) < 5 ? 2 * (p % 8) : 2 * (p % 8 - 5))
+         : B == 3 ? 3 * (p % 3)
+         : B == 4 ? 4 * (p % 2)
+                  : 0;
+}
+
+// Biased pair: one LOP3 (plus a shift shared by several pairs).
+template <int B>
+__device__ __forceinline__ uint32_t unpack_biased(const uint32_t (&w)[B], int p);
 
 // b = 2: word i holds codes 16i..16i+15 at bits 2j.  Codes j and j+8 sit 16
 // bits apart; j = 0..4 are at mantissa offsets 0..8 of their halves, j = 5..7
 // are read from the word shifted right by 10.
 template <>
-__device__ __forceinline__ uint32_t unpack_pair<2>(const uint32_t (&w)[2], int p) {
+__device__ __forceinline__ uint32_t unpack_biased<2>(const uint32_t (&w)[2], int p) {
     const uint32_t u = w[p / 8];
     const int j = p % 8;
-    if (j < 5) return fix(lop_and_or(u, 0x00030003u << (2 * j), kMagic), 2 * j);
-    return fix(lop_and_or(u >> 10, 0x00030003u << (2 * (j - 5)), kMagic), 2 * (j - 5));
+    if (j < 5) return lop_and_or(u, 0x00030003u << (2 * j), kMagic);
+    return lop_and_or(u >> 10, 0x00030003u << (2 * (j - 5)), kMagic);
 }
 
 // b = 3: the chunk is 96 bits; codes p and p+16 are 48 bits apart.  Window m
@@ -137,29 +145,35 @@ __device__ __forceinline__ uint32_t unpack_pair<2>(const uint32_t (&w)[2], int p
 // register, where codes 3m+j and 3m+j+16 (j = 0..2) sit at offset 3j of the
 // two halves.
 template <>
-__device__ __forceinline__ uint32_t unpack_pair<3>(const uint32_t (&w)[3], int p) {
+__device__ __forceinline__ uint32_t unpack_biased<3>(const uint32_t (&w)[3], int p) {
     const int m = p / 3, j = p % 3;
     const int a = 9 * m;
     const uint32_t lo = a < 32 ? shf_r(w[0], w[1], a) : shf_r(w[1], w[2], a - 32);
     const uint32_t hi = a + 16 < 32 ? shf_r(w[1], w[2], a + 16) : (w[2] >> (a - 16));
     const uint32_t r = prmt(lo, hi, 0x5410u);
-    return fix(lop_and_or(r, 0x00070007u << (3 * j), kMagic), 3 * j);
+    return lop_and_or(r, 0x00070007u << (3 * j), kMagic);
 }
 
 // b = 4: word i holds codes 8i..8i+7 (nibbles); pairs (j, j+4) at mantissa
 // offsets 0 and 4, from the word and from the word shifted right by 8.
 template <>
-__device__ __forceinline__ uint32_t unpack_pair<4>(const uint32_t (&w)[4], int p) {
+__device__ __forceinline__ uint32_t unpack_biased<4>(const uint32_t (&w)[4], int p) {
     const uint32_t u = (p % 4) < 2 ? w[p / 4] : (w[p / 4] >> 8);
-    return (p % 2) == 0 ? fix(lop_and_or(u, 0x000F000Fu, kMagic), 0)
-                        : fix(lop_and_or(u, 0x00F000F0u, kMagic), 4);
+    return (p % 2) == 0 ? lop_and_or(u, 0x000F000Fu, kMagic) : lop_and_or(u, 0x00F000F0u, kMagic);
 }
 
 // b = 8: word i holds codes 4i..4i+3 (bytes); pairs (0,2) and (1,3).
 template <>
-__device__ __forceinline__ uint32_t unpack_pair<8>(const uint32_t (&w)[8], int p) {
+__device__ __forceinline__ uint32_t unpack_biased<8>(const uint32_t (&w)[8], int p) {
     const uint32_t u = (p % 2) == 0 ? w[p / 2] : (w[p / 2] >> 8);
-    return fix(lop_and_or(u, 0x00FF00FFu, kMagic), 0);
+    return lop_and_or(u, 0x00FF00FFu, kMagic);
+}
+
+// Exact codes: one HFMA2 by (2^-s, -1024 * 2^-s) removes bias and offset.
+template <int B>
+__device__ __forceinline__ uint32_t unpack_pair(const uint32_t (&w)[B], int p) {
+    const int s = pair_shift<B>(p);
+    return hfma2_bits(unpack_biased<B>(w, p), mul_s(s), add_s(s));
 }
 
 }  // namespace zq

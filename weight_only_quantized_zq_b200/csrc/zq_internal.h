@@ -25,7 +25,7 @@ struct DecodeOp {
     const uint16_t *scales;
     const uint16_t *zeros;
     const uint16_t *xperm;  // workspace: M_pad x K fp16, chunk-permuted activations
-    const float *sx;        // workspace: G x M_pad fp32 per-group activation sums
+    const float *sx;        // workspace: G x M_pad x 2 fp32 (sum x, bias) per group and token
     uint16_t *out;          // M x N fp16
     float *part;            // workspace: split-K partials (S > 1) or null
     unsigned int *cnt;      // workspace: split-K arrival counters (S > 1) or null
@@ -48,7 +48,7 @@ struct DecodeParams {
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
     uint16_t *xperm;    // M_pad x K
-    float *sx;          // G x M_pad
+    float *sx;          // G x M_pad x 2: (sum of x, 1024 * sum of scaled x)
     int M, M_pad, K, bits;
 };
 
@@ -60,13 +60,16 @@ struct PrepParams {
 };
 
 // Decode tiling for a token-tile count MT (tokens padded to 8*MT).
-__host__ __device__ constexpr int decode_rt(int mt) { return mt <= 2 ? 2 : 1; }
+__host__ __device__ constexpr int decode_rt(int mt) { return mt == 1 ? 4 : mt == 2 ? 2 : 1; }
 __host__ __device__ constexpr int decode_rows(int mt) { return 16 * decode_rt(mt); }
-__host__ __device__ constexpr int decode_depth(int bits) {
-    return bits == 2 ? 8 : bits == 3 ? 6 : bits == 4 ? 4 : 3;
+// cp.async ring depth: about 12 KB of codes per warp.
+__host__ __device__ constexpr int decode_depth(int bits, int mt) {
+    return (12288 / (decode_rows(mt) * 16 * bits)) < 2 ? 2
+         : (12288 / (decode_rows(mt) * 16 * bits)) > 8 ? 8
+                                                       : 12288 / (decode_rows(mt) * 16 * bits);
 }
 inline size_t decode_smem_bytes(int bits, int mt) {
-    return static_cast<size_t>(kDecodeWarpsPerCta) * decode_depth(bits) * decode_rows(mt) * 16 * bits;
+    return static_cast<size_t>(kDecodeWarpsPerCta) * decode_depth(bits, mt) * decode_rows(mt) * 16 * bits;
 }
 inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
@@ -76,6 +79,14 @@ cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, uint32_
 cudaError_t read_quant_status(int slot, unsigned long long *value, cudaStream_t stream);
 cudaError_t launch_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes,
                           cudaStream_t stream);
+
+cudaError_t launch_prefill(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                           const uint16_t *zeros, int bits, int M, int N, int K, uint16_t *out, int num_sms,
+                           cudaStream_t stream);
+cudaError_t read_prefill_error(int *err);
+
+// Largest M handled by the decode family; larger M goes to the prefill family.
+constexpr int kDecodeMaxM = 64;
 
 cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, cudaStream_t stream);

@@ -1,0 +1,519 @@
+// zq_prefill.cu — prefill family (M > 64): dequantize-to-shared-memory GEMM on
+// the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA).
+//
+// What it computes: out = x · dequant(W)^T with dequant(W) = q * scale + zero per
+// group of 128 along K ([wiki] "ZSE - open-source движок для запуска LLM
+// локально на GPU - 2026", section "Формат модели .zse").  The pages' tiled
+// shared-memory matmul (section "Оркестратор и GPU-ядра", TILE = 32) is prior
+// art only.
+//
+// CTA tile: 256 tokens x 256 weight rows, K in slabs of 64 (one 128-byte
+// swizzle atom of fp16).  Warp roles:
+//   warps 0-3  epilogue: TMEM -> registers (tcgen05.ld) -> fp16 -> global;
+//   warp 4     TMA producer for x (2-D tensor map, SWIZZLE_128B) and TMEM owner;
+//   warp 5     MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
+//              for the two 128-token halves into 2 x 256 fp32 TMEM columns;
+//   warps 6-9  dequant producers: packed codes -> exact fp16 codes
+//              (zq_device.cuh) -> fp16(q*s + z) with one fused HFMA2 rounding ->
+//              K-order restored with PRMT -> UMMA K-major SWIZZLE_128B layout.
+// A 3-stage ring of (x, W) slabs is handed over with mbarriers; stage release is
+// tcgen05.commit.  Every wait is bounded: after ~2 s it raises an abort flag,
+// records ZQ_ERR_TIMEOUT in a device word and all roles drain and exit (TMEM
+// is always freed).
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "zq_device.cuh"
+#include "zq_internal.h"
+
+namespace zq {
+
+__device__ int g_prefill_error;  // 0 = ok, else a ZQ_ERR_* code from a kernel
+
+namespace pf {
+
+constexpr int kTokTile = 256;   // tokens per CTA tile (two MMA halves of 128)
+constexpr int kRowTile = 256;   // weight rows per CTA tile (MMA N)
+constexpr int kBK = 64;         // K per slab
+constexpr int kStages = 3;
+constexpr int kSlabA = kTokTile * kBK * 2;  // 32 KB
+constexpr int kSlabB = kRowTile * kBK * 2;  // 32 KB
+constexpr int kEpiWarps = 4;
+constexpr int kTmaWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kDqWarp0 = 6;
+constexpr int kDqWarps = 4;
+constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
+constexpr int kTmemCols = 512;
+constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
+
+struct Smem {
+    uint8_t a[kStages][kSlabA];  // x slabs (TMA, SWIZZLE_128B)
+    uint8_t b[kStages][kSlabB];  // dequantized W slabs (SWIZZLE_128B)
+    unsigned long long full[kStages];
+    unsigned long long empty[kStages];
+    unsigned long long acc_full;
+    unsigned long long acc_empty;
+    uint32_t tmem_base;
+    int abort;
+};
+constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long globaltimer() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long *bar) {
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(unsigned long long *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(unsigned long long *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: false if the CTA is aborting or the limit was reached.
+__device__ __noinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *abort) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 15u) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > kWaitNs) {
+                *abort = 1;
+                atomicExch(&g_prefill_error, 5);  // ZQ_ERR_TIMEOUT
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// UMMA shared-memory descriptor: K-major, SWIZZLE_128B, 8-row groups 1024 B
+// apart (rows of 128 bytes), sm_100 descriptor version 1.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
+    d |= static_cast<uint64_t>(1) << 16;                   // leading byte offset (unused here)
+    d |= static_cast<uint64_t>(1024 >> 4) << 32;           // stride byte offset
+    d |= static_cast<uint64_t>(1) << 46;                   // descriptor version
+    d |= static_cast<uint64_t>(2) << 61;                   // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B (K-major), fp32 D.
+constexpr uint32_t kIdesc = (1u << 4)                       // D format f32
+                            | (0u << 7) | (0u << 10)        // A, B format f16
+                            | (static_cast<uint32_t>(kRowTile >> 3) << 17)  // N
+                            | (static_cast<uint32_t>(128 >> 4) << 24);     // M
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(unsigned long long *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y,
+                                            unsigned long long *bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+    const __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Tile t -> (weight-row tile, token tile); token tiles vary fastest so the
+// CTAs working at the same time share one weight tile (L2 reuse).
+__device__ __forceinline__ void tile_coords(int t, int tok_tiles, int &n0, int &t0) {
+    n0 = (t / tok_tiles) * kRowTile;
+    t0 = (t % tok_tiles) * kTokTile;
+}
+
+// Dequantize this thread's 32-code chunk of one W row into 4 x 16 bytes of
+// natural-K-order fp16 (q*s + z, one rounding), via the shared unpack.
+template <int B>
+__device__ __forceinline__ void dequant_chunk(const uint32_t (&w)[B], uint32_t sz, uint32_t (&o)[16]) {
+    const uint32_t s2 = (sz & 0xFFFFu) * 0x10001u;  // (s, s)
+    const uint32_t z2 = (sz >> 16) * 0x10001u;      // (z, z)
+    uint32_t v[16];
+#pragma unroll
+    for (int p = 0; p < 16; ++p) v[p] = hfma2_bits(unpack_pair<B>(w, p), s2, z2);
+    // Pairs p (even) and p+1 hold codes (lo, hi) and (lo+1, hi+1): two PRMTs
+    // give the natural pairs (lo, lo+1) and (hi, hi+1).
+#pragma unroll
+    for (int p = 0; p < 16; p += 2) {
+        const int lo = pair_lo<B>(p), hi = pair_hi<B>(p);
+        o[lo / 2] = prmt(v[p], v[p + 1], 0x5410u);
+        o[hi / 2] = prmt(v[p], v[p + 1], 0x7632u);
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void load_chunk(uint32_t (&w)[B], const uint32_t *src) {
+    if constexpr (B == 2) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(src);
+        w[0] = v.x;
+        w[1] = v.y;
+    } else if constexpr (B == 3) {
+        w[0] = src[0];
+        w[1] = src[1];
+        w[2] = src[2];
+    } else if constexpr (B == 4) {
+        const uint4 v = *reinterpret_cast<const uint4 *>(src);
+        w[0] = v.x; w[1] = v.y; w[2] = v.z; w[3] = v.w;
+    } else {
+        const uint4 v0 = reinterpret_cast<const uint4 *>(src)[0];
+        const uint4 v1 = reinterpret_cast<const uint4 *>(src)[1];
+        w[0] = v0.x; w[1] = v0.y; w[2] = v0.z; w[3] = v0.w;
+        w[4] = v1.x; w[5] = v1.y; w[6] = v1.z; w[7] = v1.w;
+    }
+}
+
+struct PrefillParams {
+    const uint32_t *packed;
+    const uint16_t *scales;
+    const uint16_t *zeros;
+    uint16_t *out;
+    int M, N, K;
+    int tok_tiles, row_tiles;
+};
+
+template <int B>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PrefillParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_tiles = p.tok_tiles * p.row_tiles;
+    const int slabs = p.K / kBK;
+    volatile int *abort = &sm.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&sm.full[s], 1 + kDqWarps);
+            mbar_init(&sm.empty[s], 1);
+        }
+        mbar_init(&sm.acc_full, 1);
+        mbar_init(&sm.acc_empty, kEpiWarps);
+        sm.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kTmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    pdl_wait();  // x may be produced by the previous kernel in the stream
+    pdl_launch_dependents();
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
+            uint32_t it = 0;
+            for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+                int n0, t0;
+                tile_coords(t, p.tok_tiles, n0, t0);
+                for (int s = 0; s < slabs; ++s, ++it) {
+                    const int st = it % kStages;
+                    const uint32_t round = it / kStages;
+                    if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) break;
+                    mbar_arrive_expect_tx(&sm.full[st], kSlabA);
+                    tma_load_2d(sm.a[st], &xmap, s * kBK, t0, &sm.full[st]);
+                }
+            }
+            // Let copies still in flight land before the CTA can exit.
+            for (uint32_t k = 0; k < kStages && k < it; ++k) {
+                const uint32_t j = it - 1 - k;
+                mbar_wait(&sm.full[j % kStages], (j / kStages) & 1u, abort);
+            }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0) {
+            uint32_t it = 0, tile_i = 0;
+            for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
+                if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort)) break;
+                tc_fence_after();
+                bool ok = true;
+                for (int s = 0; s < slabs; ++s, ++it) {
+                    const int st = it % kStages;
+                    if (!mbar_wait(&sm.full[st], (it / kStages) & 1u, abort)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sm.a[st]);
+                    const uint32_t b0 = smem_u32(sm.b[st]);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t bd = sdesc_sw128(b0 + kk * 32);
+                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                        umma_f16(tmem, sdesc_sw128(a0 + kk * 32), bd, acc);
+                        umma_f16(tmem + kRowTile, sdesc_sw128(a0 + kSlabA / 2 + kk * 32), bd, acc);
+                    }
+                    umma_commit(&sm.empty[st]);
+                }
+                if (!ok) break;
+                umma_commit(&sm.acc_full);
+            }
+        }
+    } else if (warp >= kDqWarp0) {
+        // 128 threads: thread d handles rows d/2 + 64*i (i = 0..3), 32-code chunk d%2.
+        const int d = threadIdx.x - 32 * kDqWarp0;
+        const int ch = d & 1;
+        const size_t wpr = static_cast<size_t>(p.K) * B / 32;
+        const int G = p.K / kGroup;
+        uint32_t it = 0;
+        // register prefetch of the next slab's codes and scale/zero
+        uint32_t wn[4][B], szn[4];
+        auto fetch = [&](int t, int s) {
+            int n0, t0;
+            tile_coords(t, p.tok_tiles, n0, t0);
+            const int kc = s * 2 + ch;  // 32-code chunk index along K
+            const int g = (s * kBK) / kGroup;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int r = min(n0 + d / 2 + 64 * i, p.N - 1);
+                load_chunk<B>(wn[i], p.packed + static_cast<size_t>(r) * wpr + static_cast<size_t>(kc) * B);
+                const size_t si = static_cast<size_t>(r) * G + g;
+                szn[i] = ldg_u16_nc(p.scales + si) | (ldg_u16_nc(p.zeros + si) << 16);
+            }
+        };
+        int t = blockIdx.x, s = 0;
+        if (t < n_tiles) fetch(t, 0);
+        while (t < n_tiles && !*abort) {
+            uint32_t wc[4][B], szc[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                szc[i] = szn[i];
+#pragma unroll
+                for (int q = 0; q < B; ++q) wc[i][q] = wn[i][q];
+            }
+            const int st = it % kStages;
+            const uint32_t round = it / kStages;
+            // advance and prefetch the following slab
+            int t_n = t, s_n = s + 1;
+            if (s_n == slabs) {
+                s_n = 0;
+                t_n += gridDim.x;
+            }
+            if (t_n < n_tiles) fetch(t_n, s_n);
+            if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) break;
+            uint8_t *bs = sm.b[st];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int row = d / 2 + 64 * i;
+                uint32_t o[16];
+                dequant_chunk<B>(wc[i], szc[i], o);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int c16 = (4 * ch + j) ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
+                        make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.full[st]);
+            ++it;
+            t = t_n;
+            s = s_n;
+        }
+    } else {
+        // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = tokens of each half.
+        uint32_t tile_i = 0;
+        for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
+            if (!mbar_wait(&sm.acc_full, tile_i & 1u, abort)) break;
+            tc_fence_after();
+            int n0, t0;
+            tile_coords(t, p.tok_tiles, n0, t0);
+            const bool vec = (p.N % 8) == 0;
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+                const int tok = t0 + 128 * half + 32 * warp + lane;
+#pragma unroll 1
+                for (int cc = 0; cc < kRowTile / 32; ++cc) {
+                    uint32_t r[32];
+                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile + cc * 32, r);
+                    const int col0 = n0 + cc * 32;
+                    if (tok < p.M && col0 < p.N) {
+                        uint16_t *dst = p.out + static_cast<size_t>(tok) * p.N + col0;
+                        if (vec && col0 + 32 <= p.N) {
+#pragma unroll
+                            for (int q = 0; q < 4; ++q)
+                                reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
+                                    pack_half2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1])),
+                                    pack_half2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
+                                    pack_half2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
+                                    pack_half2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (col0 + q < p.N) dst[q] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == kTmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+}  // namespace pf
+
+// ------------------------------------------------------------------ host --
+
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+template <int B>
+static cudaError_t launch_prefill_t(const CUtensorMap &map, const pf::PrefillParams &pp, int n_ctas,
+                                    cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(pf::prefill_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(pf::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
+    cfg.blockDim = dim3(pf::kThreads);
+    cfg.dynamicSmemBytes = pf::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B>, map, pp);
+}
+
+cudaError_t launch_prefill(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                           const uint16_t *zeros, int bits, int M, int N, int K, uint16_t *out, int num_sms,
+                           cudaStream_t stream) {
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) return cudaErrorNotSupported;
+    CUtensorMap map;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {pf::kBK, pf::kTokTile};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<uint16_t *>(x), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    pf::PrefillParams pp;
+    pp.packed = packed;
+    pp.scales = scales;
+    pp.zeros = zeros;
+    pp.out = out;
+    pp.M = M;
+    pp.N = N;
+    pp.K = K;
+    pp.tok_tiles = (M + pf::kTokTile - 1) / pf::kTokTile;
+    pp.row_tiles = (N + pf::kRowTile - 1) / pf::kRowTile;
+    const int tiles = pp.tok_tiles * pp.row_tiles;
+    const int n_ctas = tiles < num_sms ? tiles : num_sms;
+    switch (bits) {
+        case 2: return launch_prefill_t<2>(map, pp, n_ctas, stream);
+        case 3: return launch_prefill_t<3>(map, pp, n_ctas, stream);
+        case 4: return launch_prefill_t<4>(map, pp, n_ctas, stream);
+        default: return launch_prefill_t<8>(map, pp, n_ctas, stream);
+    }
+}
+
+cudaError_t read_prefill_error(int *err) {
+    cudaError_t e = cudaMemcpyFromSymbol(err, g_prefill_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_prefill_error, &zero, sizeof(int));
+}
+
+}  // namespace zq
