@@ -183,7 +183,6 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     if ((st = decode_occupancy(info, bits, mt, &occ)) != ZQ_OK) return st;
     const int rows = decode_rows(mt);
     const int mpad = 8 * mt;
-    const long long max_warps = static_cast<long long>(occ) * info->sms * kDecodeWarpsPerCta;
 
     // Prep entries (distinct activation buffers).
     std::vector<PrepKey> keys;
@@ -201,53 +200,41 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     if (keys.size() > static_cast<size_t>(kMaxPrepEntries) || ops.size() > static_cast<size_t>(kMaxDecodeOps))
         return fail(ZQ_ERR_INVALID_ARG, "internal: decode launch too large");
 
-    // Split-K.  Work is spread over warps by byte cost, each warp taking the
-    // units that start in its share; a unit may overrun the share, so units
-    // are capped at 1/16 of a share (load balance), and small launches are
-    // split until every warp has work.
-    long long rb_total = 0, cost_total = 0;
-    std::vector<int> rbs(ops.size()), S(ops.size(), 1), gps(ops.size());
+    // Stream-K partition: every step (op, row block, group) costs the same
+    // within a launch (same bits), so warps get equal step counts.
+    long long total_steps = 0;
+    int max_m = 1;
+    std::vector<int> rbs(ops.size());
+    const int gps = decode_gps(bits);
     for (size_t i = 0; i < ops.size(); ++i) {
         rbs[i] = (ops[i].N + rows - 1) / rows;
-        rb_total += rbs[i];
-        gps[i] = ops[i].K / kGroup;
-        cost_total += static_cast<long long>(rbs[i]) * rows * gps[i] * (16 * bits + 4);
+        const int su = (ops[i].K / kGroup + gps - 1) / gps;
+        total_steps += static_cast<long long>(rbs[i]) * su;
+        max_m = std::max(max_m, ops[i].M);
     }
-    const long long share = std::max(1LL, cost_total / max_warps);
-    const long long cap = std::max(1LL, share / 16);
-    const double fill = rb_total < 2 * max_warps ? static_cast<double>(2 * max_warps) / rb_total : 1.0;
-    size_t counters = 0;
-    for (size_t i = 0; i < ops.size(); ++i) {
-        const int G = ops[i].K / kGroup;
-        const long long unit1 = static_cast<long long>(rows) * G * (16 * bits + 4);
-        long long want = std::max(static_cast<long long>(fill + 0.999), (unit1 + cap - 1) / cap);
-        int s = static_cast<int>(std::min<long long>(G, want));
-        if (s <= 1 || counters + rbs[i] > kMaxCounters) continue;
-        gps[i] = (G + s - 1) / s;
-        S[i] = (G + gps[i] - 1) / gps[i];
-        if (S[i] > 1) counters += rbs[i];
-    }
+    if (total_steps > 0x7FFFFFFFLL) return fail(ZQ_ERR_INVALID_ARG, "decode launch too large (steps)");
+    const long long want_ctas = std::max(1LL, (total_steps + kDecodeWarpsPerCta - 1) / kDecodeWarpsPerCta);
+    const int n_ctas = static_cast<int>(std::min(want_ctas, static_cast<long long>(occ) * info->sms));
+    const long long n_warps = static_cast<long long>(n_ctas) * kDecodeWarpsPerCta;
+    const int slot_floats = rows * max_m;
 
     // Workspace layout.
     size_t off = 0;
-    std::vector<size_t> prep_off(keys.size()), part_off(ops.size(), 0);
+    std::vector<size_t> prep_off(keys.size());
     for (size_t e = 0; e < keys.size(); ++e) {
         prep_off[e] = off;
         const size_t G = keys[e].K / kGroup;
         off += align256(static_cast<size_t>(mpad) * keys[e].K * 2) + align256(G * mpad * 8);
     }
-    for (size_t i = 0; i < ops.size(); ++i)
-        if (S[i] > 1) {
-            part_off[i] = off;
-            off += align256(static_cast<size_t>(rbs[i]) * S[i] * rows * mpad * 4);
-        }
+    const size_t part_off = off;
+    off += align256(static_cast<size_t>(n_warps) * 2 * slot_floats * 4);
+    if (static_cast<size_t>(n_warps) > kMaxCounters) return fail(ZQ_ERR_INVALID_ARG, "internal: too many warps");
     if (dry_bytes) {
         *dry_bytes = off + kCounterBytes;
         return ZQ_OK;
     }
     uint8_t *ws = nullptr;
     if ((st = workspace(stream, off, &ws)) != ZQ_OK) return st;
-    unsigned int *cnt_base = reinterpret_cast<unsigned int *>(ws);
     uint8_t *data = ws + kCounterBytes;
 
     PrepParams pp;
@@ -272,8 +259,11 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     DecodeParams dp;
     std::memset(&dp, 0, sizeof(dp));
     dp.n_ops = static_cast<int>(ops.size());
-    long long cost = 0, units = 0;
-    size_t cnt_off = 0;
+    dp.total_steps = total_steps;
+    dp.part = reinterpret_cast<float *>(data + part_off);
+    dp.cnt = reinterpret_cast<unsigned int *>(ws);
+    dp.slot_floats = slot_floats;
+    long long step0 = 0;
     for (size_t i = 0; i < ops.size(); ++i) {
         DecodeOp &o = dp.ops[i];
         const PrepEntry &en = pp.e[op_entry[i]];
@@ -287,23 +277,11 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         o.N = ops[i].N;
         o.K = ops[i].K;
         o.G = ops[i].K / kGroup;
-        o.S = S[i];
-        o.gps = gps[i];
         o.row_blocks = rbs[i];
-        if (S[i] > 1) {
-            o.part = reinterpret_cast<float *>(data + part_off[i]);
-            o.cnt = cnt_base + cnt_off;
-            cnt_off += rbs[i];
-        }
-        o.cost0 = cost;
-        o.unit_cost = static_cast<long long>(rows) * gps[i] * (16 * bits + 4);
-        cost += o.unit_cost * rbs[i] * S[i];
-        units += static_cast<long long>(rbs[i]) * S[i];
+        o.su = (o.G + gps - 1) / gps;
+        o.step0 = step0;
+        step0 += static_cast<long long>(rbs[i]) * o.su;
     }
-    dp.total_cost = cost;
-
-    const long long want_ctas = (units + kDecodeWarpsPerCta - 1) / kDecodeWarpsPerCta;
-    const int n_ctas = static_cast<int>(std::max(1LL, std::min(want_ctas, static_cast<long long>(occ) * info->sms)));
 
     cudaError_t e = launch_prep(pp, wsum, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prep launch");

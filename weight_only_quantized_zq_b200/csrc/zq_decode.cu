@@ -23,10 +23,11 @@
 //  * Packed codes stream through a per-warp shared-memory ring with cp.async
 //    (16-byte chunks, several steps in flight, no register cost); the ring is
 //    per warp, so no block-level barrier is needed.
-//  * A persistent grid covers every SM; work units (op, row block, K slice) are
-//    spread over warps by byte cost, so a whole stack of layers runs as one
-//    launch and a single small layer is split along K (partials reduced by the
-//    last-arriving warp in a fixed order, so results are deterministic).
+//  * A persistent grid covers every SM.  The steps (op, row block, group) of
+//    all ops of a launch are cut into one contiguous range per warp (stream-K),
+//    so a whole stack of layers runs as one balanced launch and a small layer
+//    is split along K; a row block cut by a warp boundary is reduced by the
+//    last warp to finish it, in warp order, so results are deterministic.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -100,93 +101,92 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
 // ---------------------------------------------------------------- decode --
 
 struct Cursor {
-    int o, u, g, g_end, r0, rb, slice;
+    int s;         // step index
+    int o, rb, j;  // op, row block, step within the row block
+    int SU, RB;    // steps per row block and row blocks of op o
     bool valid;
 };
 
-template <int ROWS>
-__device__ __forceinline__ void cursor_unit(Cursor &cu, const DecodeParams &p, long long c_end) {
-    while (cu.o < p.n_ops && cu.u >= p.ops[cu.o].row_blocks * p.ops[cu.o].S) {
-        ++cu.o;
-        cu.u = 0;
-    }
-    cu.valid = false;
-    if (cu.o >= p.n_ops) return;
-    const DecodeOp &op = p.ops[cu.o];
-    if (op.cost0 + static_cast<long long>(cu.u) * op.unit_cost >= c_end) return;
-    cu.rb = cu.u / op.S;
-    cu.slice = cu.u - cu.rb * op.S;
-    cu.r0 = cu.rb * ROWS;
-    cu.g = cu.slice * op.gps;
-    cu.g_end = min(op.G, cu.g + op.gps);
-    cu.valid = true;
+__device__ __forceinline__ void cursor_init(Cursor &cu, const DecodeParams &p, int s, int s_end) {
+    cu.s = s;
+    cu.valid = s < s_end;
+    int o = 0;
+    while (o + 1 < p.n_ops && p.ops[o + 1].step0 <= s) ++o;
+    const int local = s - static_cast<int>(p.ops[o].step0);
+    cu.o = o;
+    cu.SU = p.ops[o].su;
+    cu.RB = p.ops[o].row_blocks;
+    cu.rb = local / cu.SU;
+    cu.j = local - cu.rb * cu.SU;
 }
 
-template <int ROWS>
-__device__ __forceinline__ void cursor_next(Cursor &cu, const DecodeParams &p, long long c_end) {
-    if (++cu.g == cu.g_end) {
-        ++cu.u;
-        cursor_unit<ROWS>(cu, p, c_end);
+__device__ __forceinline__ void cursor_next(Cursor &cu, const DecodeParams &p, int s_end) {
+    ++cu.s;
+    cu.valid = cu.s < s_end;
+    if (++cu.j == cu.SU) {
+        cu.j = 0;
+        if (++cu.rb == cu.RB) {
+            cu.rb = 0;
+            if (cu.o + 1 < p.n_ops) {
+                ++cu.o;
+                cu.SU = p.ops[cu.o].su;
+                cu.RB = p.ops[cu.o].row_blocks;
+            }
+        }
     }
 }
 
-// Per-step operands other than the codes (activations, group sums, scales,
-// zeros), loaded one step ahead into registers so their L1/L2 latency overlaps
-// the previous step's math.
-template <int MT, int RT>
-struct StepOperands {
-    uint32_t xf[MT][16];  // B fragments: 16 half2 pairs per token tile
-    float4 sb[MT];        // (sum x, bias) for this thread's two C-fragment tokens
-    uint32_t sz[RT][2];   // (scale | zero << 16) of this thread's C-fragment rows
-};
+// Warp whose step range contains step s (ranges are [T*w/W, T*(w+1)/W)).
+__device__ __forceinline__ int warp_of(long long s, long long W, long long T) {
+    return static_cast<int>(((s + 1) * W - 1) / T);
+}
 
-template <int MT, int RT>
-__device__ __forceinline__ void load_operands(StepOperands<MT, RT> &v, const DecodeOp &op, const Cursor &cu,
-                                              int gq, int c) {
-    constexpr int MPAD = 8 * MT;
+// Scales and zeros of rows (gq, gq + 8) for the GPS groups of a step, packed as
+// fp16 pairs: sz[h][i] holds groups (2i, 2i+1) of row half h; [2 + ...] zeros.
+template <int GPS>
+__device__ __forceinline__ void load_scale_zero(uint32_t (&sz)[2][GPS], const DecodeOp &op, int r0, int g0,
+                                                int gq) {
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        const int tok = 8 * mt + gq;
-        if (tok < op.M) {
-            const uint16_t *xp = op.xperm + static_cast<size_t>(tok) * op.K + static_cast<size_t>(cu.g) * kGroup + 32 * c;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 w = ldg_u4(xp + 8 * q);
-                v.xf[mt][4 * q + 0] = w.x;
-                v.xf[mt][4 * q + 1] = w.y;
-                v.xf[mt][4 * q + 2] = w.z;
-                v.xf[mt][4 * q + 3] = w.w;
+    for (int h = 0; h < 2; ++h) {
+        const int r = min(r0 + h * 8 + gq, op.N - 1);
+        const size_t idx = static_cast<size_t>(r) * op.G + g0;
+        if (((r * op.G + g0) % GPS) == 0 && g0 + GPS <= op.G) {
+            if constexpr (GPS == 4) {
+                const uint2 s2 = *reinterpret_cast<const uint2 *>(op.scales + idx);
+                const uint2 z2 = *reinterpret_cast<const uint2 *>(op.zeros + idx);
+                sz[h][0] = s2.x;
+                sz[h][1] = s2.y;
+                sz[h][2] = z2.x;
+                sz[h][3] = z2.y;
+            } else {
+                sz[h][0] = *reinterpret_cast<const uint32_t *>(op.scales + idx);
+                sz[h][1] = *reinterpret_cast<const uint32_t *>(op.zeros + idx);
             }
         } else {
 #pragma unroll
-            for (int q = 0; q < 16; ++q) v.xf[mt][q] = 0u;
+            for (int i = 0; i < GPS / 2; ++i) {
+                const int ga = min(g0 + 2 * i, op.G - 1), gb = min(g0 + 2 * i + 1, op.G - 1);
+                const size_t ia = static_cast<size_t>(r) * op.G + ga, ib = static_cast<size_t>(r) * op.G + gb;
+                sz[h][i] = ldg_u16_nc(op.scales + ia) | (ldg_u16_nc(op.scales + ib) << 16);
+                sz[h][GPS / 2 + i] = ldg_u16_nc(op.zeros + ia) | (ldg_u16_nc(op.zeros + ib) << 16);
+            }
         }
-        if (8 * mt + 2 * c < op.M)
-            v.sb[mt] = *reinterpret_cast<const float4 *>(op.sx + 2 * (static_cast<size_t>(cu.g) * MPAD + 8 * mt + 2 * c));
-        else
-            v.sb[mt] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
-#pragma unroll
-    for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int r = min(cu.r0 + rt * 16 + h * 8 + gq, op.N - 1);
-            const size_t idx = static_cast<size_t>(r) * op.G + cu.g;
-            v.sz[rt][h] = ldg_u16_nc(op.scales + idx) | (ldg_u16_nc(op.zeros + idx) << 16);
-        }
 }
 
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 1)
+__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     decode_kernel(const __grid_constant__ DecodeParams p) {
-    constexpr int RT = decode_rt(MT);
-    constexpr int ROWS = 16 * RT;
-    constexpr int D = decode_depth(BITS, MT);
-    constexpr int ROW_BYTES = 16 * BITS;  // one row of one group
-    constexpr int STAGE = ROWS * ROW_BYTES;
-    constexpr int CHUNKS = ROWS * BITS;   // 16-byte chunks per stage
-    constexpr int CPL = (CHUNKS + 31) / 32;
+    constexpr int ROWS = 16;
+    constexpr int GPS = decode_gps(BITS);
+    constexpr int GB = 16 * BITS;                 // bytes of one row of one group
+    constexpr int RS = decode_row_stride(BITS);   // shared-memory row stride
+    constexpr int STAGE = decode_stage(BITS);
+    constexpr int CPR = GPS * BITS;               // 16-byte chunks per row per step
+    constexpr int CPL = ROWS * CPR / 32;          // chunks per lane
+    constexpr int D = decode_depth(BITS);
     constexpr int MPAD = 8 * MT;
+    static_assert(ROWS * CPR % 32 == 0, "chunks must split evenly over the warp");
 
     extern __shared__ __align__(128) uint8_t smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -194,37 +194,46 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 1)
     const int c = lane & 3;    // quad position: 32-code chunk (A, B) / token pair (C)
     uint8_t *ring = smem + warp * D * STAGE;
 
-    const long long W = static_cast<long long>(gridDim.x) * kDecodeWarpsPerCta;
-    const long long gw = static_cast<long long>(blockIdx.x) * kDecodeWarpsPerCta + warp;
-    const long long c_begin = p.total_cost * gw / W;
-    const long long c_end = p.total_cost * (gw + 1) / W;
+    // At most one warp per step, so every warp range is non-empty: a row block
+    // split over warps w_first..w_last gets a piece from each of them.
+    const long long T = p.total_steps;
+    const long long W = min(static_cast<long long>(gridDim.x) * kDecodeWarpsPerCta, T);
+    const int gw = blockIdx.x * kDecodeWarpsPerCta + warp;
+    const int s_begin = gw < W ? static_cast<int>(T * gw / W) : 0;
+    const int s_end = gw < W ? static_cast<int>(T * (gw + 1) / W) : 0;
 
-    Cursor nx;  // next step to compute (operands prefetched for it)
-    {
-        int o = 0;
-        while (o + 1 < p.n_ops && p.ops[o + 1].cost0 <= c_begin) ++o;
-        const DecodeOp &op = p.ops[o];
-        const long long rel = c_begin - op.cost0;
-        nx.o = o;
-        nx.u = static_cast<int>((rel + op.unit_cost - 1) / op.unit_cost);
-        cursor_unit<ROWS>(nx, p, c_end);
+    Cursor cs;
+    cursor_init(cs, p, s_begin, s_end);
+    Cursor ld = cs, nx = cs;
+
+    // Row blocks cut by this warp's range (see warp_of); computed once, so the
+    // 64-bit division stays out of the loop.
+    int head_first = 0, head_last = 0, tail_last = 0;
+    if (cs.valid) {
+        const long long u0 = s_begin - cs.j;
+        head_first = warp_of(u0, W, T);
+        head_last = warp_of(u0 + cs.SU - 1, W, T);
+        Cursor lc;
+        cursor_init(lc, p, s_end - 1, s_end);
+        tail_last = warp_of(static_cast<long long>(s_end) - 1 - lc.j + lc.SU - 1, W, T);
     }
-    Cursor ld = nx;
 
     auto issue = [&](const Cursor &cu, int slot) {
         const DecodeOp &op = p.ops[cu.o];
         const size_t row_stride = static_cast<size_t>(op.K) * BITS / 8;  // bytes
-        const uint8_t *base = reinterpret_cast<const uint8_t *>(op.packed) +
-                              static_cast<size_t>(cu.g) * ROW_BYTES;
+        const int g0 = cu.j * GPS;
+        const int ng = min(GPS, op.G - g0);
+        const uint8_t *base = reinterpret_cast<const uint8_t *>(op.packed) + static_cast<size_t>(g0) * GB;
         uint8_t *st = ring + slot * STAGE;
+        const int r0 = cu.rb * ROWS;
 #pragma unroll
         for (int i = 0; i < CPL; ++i) {
             const int ch = lane + 32 * i;
-            if (CHUNKS % 32 == 0 || ch < CHUNKS) {
-                const int row = ch / BITS, part = ch % BITS;
-                const int r = min(cu.r0 + row, op.N - 1);
-                const int pp = BITS == 8 ? (part ^ (row & 7)) : part;
-                cp_async16(st + row * ROW_BYTES + pp * 16, base + static_cast<size_t>(r) * row_stride + part * 16);
+            const int row = ch / CPR, part = ch % CPR;
+            if (part / BITS < ng) {
+                const int r = min(r0 + row, op.N - 1);
+                cp_async16(st + row * RS + decode_swizzle(BITS, row, part) * 16,
+                           base + static_cast<size_t>(r) * row_stride + part * 16);
             }
         }
     };
@@ -235,40 +244,42 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 1)
     for (int i = 0; i < D - 1; ++i) {
         if (ld.valid) {
             issue(ld, slot_ld);
-            cursor_next<ROWS>(ld, p, c_end);
+            cursor_next(ld, p, s_end);
         }
         cp_async_commit();
         slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
     }
+    uint32_t szc[2][GPS];  // scales/zeros of the current step (loaded one step ahead)
+    if (cs.valid) load_scale_zero<GPS>(szc, p.ops[cs.o], cs.rb * ROWS, cs.j * GPS, gq);
     pdl_wait();  // the prepared activations come from the previous kernel
     pdl_launch_dependents();
 
-    StepOperands<MT, RT> opA, opB;
-    if (nx.valid) load_operands<MT, RT>(opA, p.ops[nx.o], nx, gq, c);
-
-    float tot[RT][MT][4];
+    float tot[MT][4];
 #pragma unroll
-    for (int a = 0; a < RT; ++a)
+    for (int b = 0; b < MT; ++b)
 #pragma unroll
-        for (int b = 0; b < MT; ++b)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) tot[a][b][i] = 0.0f;
+        for (int i = 0; i < 4; ++i) tot[b][i] = 0.0f;
     const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 
-    // One step: consume `cv` (operands of the step at `nx`), prefetch the next
-    // step's operands into `nv`.
-    auto step = [&](const StepOperands<MT, RT> &cv, StepOperands<MT, RT> &nv) {
-        const Cursor cs = nx;
-        cursor_next<ROWS>(nx, p, c_end);
-        if (nx.valid) load_operands<MT, RT>(nv, p.ops[nx.o], nx, gq, c);
-
+#pragma unroll 1
+    while (cs.valid) {
         __syncwarp();
         if (ld.valid) {
             issue(ld, slot_ld);
-            cursor_next<ROWS>(ld, p, c_end);
+            cursor_next(ld, p, s_end);
         }
         cp_async_commit();
         slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
+
+        // Scales/zeros of the next step.
+        cursor_next(nx, p, s_end);
+        uint32_t szn[2][GPS];
+        if (nx.valid) load_scale_zero<GPS>(szn, p.ops[nx.o], nx.rb * ROWS, nx.j * GPS, gq);
+
+        const DecodeOp &op = p.ops[cs.o];
+        const int r0 = cs.rb * ROWS;
+        const int g0 = cs.j * GPS;
+        const int ng = min(GPS, op.G - g0);
 
         cp_async_wait<D - 1>();
         __syncwarp();
@@ -276,125 +287,149 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 1)
         slot_cs = slot_cs + 1 == D ? 0 : slot_cs + 1;
 
 #pragma unroll
-        for (int rt = 0; rt < RT; ++rt) {
-            uint32_t wv[2][BITS];
+        for (int gi = 0; gi < GPS; ++gi) {
+            if (gi < ng) {
+                const int g = g0 + gi;
+                // this thread's 32-code chunk of rows gq and gq + 8
+                uint32_t wv[2][BITS];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = rt * 16 + h * 8 + gq;
-                const uint8_t *rp = st + row * ROW_BYTES;
-                if constexpr (BITS == 2) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(rp + 8 * c);
-                    wv[h][0] = v.x;
-                    wv[h][1] = v.y;
-                } else if constexpr (BITS == 3) {
-                    const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + 12 * c);
-                    wv[h][0] = q[0];
-                    wv[h][1] = q[1];
-                    wv[h][2] = q[2];
-                } else if constexpr (BITS == 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * c);
-                    wv[h][0] = v.x;
-                    wv[h][1] = v.y;
-                    wv[h][2] = v.z;
-                    wv[h][3] = v.w;
-                } else {
-                    const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + 16 * ((2 * c) ^ (row & 7)));
-                    const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + 16 * ((2 * c + 1) ^ (row & 7)));
-                    wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
-                    wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
+                for (int h = 0; h < 2; ++h) {
+                    const int row = h * 8 + gq;
+                    const uint8_t *rp = st + row * RS;
+                    if constexpr (BITS == 2) {
+                        const int ch = decode_swizzle(2, row, gi * 2 + (c >> 1));
+                        const uint2 v = *reinterpret_cast<const uint2 *>(rp + ch * 16 + (c & 1) * 8);
+                        wv[h][0] = v.x;
+                        wv[h][1] = v.y;
+                    } else if constexpr (BITS == 3) {
+                        const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + gi * GB + 12 * c);
+                        wv[h][0] = q[0];
+                        wv[h][1] = q[1];
+                        wv[h][2] = q[2];
+                    } else if constexpr (BITS == 4) {
+                        const uint4 v = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(4, row, gi * 4 + c) * 16);
+                        wv[h][0] = v.x;
+                        wv[h][1] = v.y;
+                        wv[h][2] = v.z;
+                        wv[h][3] = v.w;
+                    } else {
+                        const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c) * 16);
+                        const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c + 1) * 16);
+                        wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
+                        wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
+                    }
                 }
-            }
-            float acc[MT][4];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const uint32_t a0 = unpack_biased<BITS>(wv[0], 2 * j);
-                const uint32_t a1 = unpack_biased<BITS>(wv[1], 2 * j);
-                const uint32_t a2 = unpack_biased<BITS>(wv[0], 2 * j + 1);
-                const uint32_t a3 = unpack_biased<BITS>(wv[1], 2 * j + 1);
+                // scale and zero of this group for rows gq, gq + 8
+                const uint32_t sp0 = szc[0][gi / 2], sp1 = szc[1][gi / 2];
+                const uint32_t zp0 = szc[0][GPS / 2 + gi / 2], zp1 = szc[1][GPS / 2 + gi / 2];
+                const float sc[2] = {h2f_bits((gi & 1) ? (sp0 >> 16) : (sp0 & 0xFFFFu)),
+                                     h2f_bits((gi & 1) ? (sp1 >> 16) : (sp1 & 0xFFFFu))};
+                const float zr[2] = {h2f_bits((gi & 1) ? (zp0 >> 16) : (zp0 & 0xFFFFu)),
+                                     h2f_bits((gi & 1) ? (zp1 >> 16) : (zp1 & 0xFFFFu))};
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt) {
-                    if (j == 0)
-                        mma_16816(acc[mt], a0, a1, a2, a3, cv.xf[mt][2 * j], cv.xf[mt][2 * j + 1], zero4);
-                    else
-                        mma_16816(acc[mt], a0, a1, a2, a3, cv.xf[mt][2 * j], cv.xf[mt][2 * j + 1], acc[mt]);
-                }
-            }
-            // Per-group epilogue: tot += s * (acc - bias) + z * sum(x).
+                    // B fragments and group sums of this token tile (L1 hits)
+                    uint32_t xf[16];
+                    const int tok = 8 * mt + gq;
+                    if (tok < op.M) {
+                        const uint16_t *xp = op.xperm + static_cast<size_t>(tok) * op.K +
+                                             static_cast<size_t>(g) * kGroup + 32 * c;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const float sc = h2f_bits(cv.sz[rt][h] & 0xFFFFu);
-                const float zr = h2f_bits(cv.sz[rt][h] >> 16);
+                        for (int q = 0; q < 4; ++q) {
+                            const uint4 w = ldg_u4(xp + 8 * q);
+                            xf[4 * q + 0] = w.x;
+                            xf[4 * q + 1] = w.y;
+                            xf[4 * q + 2] = w.z;
+                            xf[4 * q + 3] = w.w;
+                        }
+                    } else {
 #pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    float &t0 = tot[rt][mt][2 * h], &t1 = tot[rt][mt][2 * h + 1];
-                    t0 = fmaf(sc, acc[mt][2 * h] - cv.sb[mt].y, fmaf(zr, cv.sb[mt].x, t0));
-                    t1 = fmaf(sc, acc[mt][2 * h + 1] - cv.sb[mt].w, fmaf(zr, cv.sb[mt].z, t1));
+                        for (int q = 0; q < 16; ++q) xf[q] = 0u;
+                    }
+                    const float4 sb = (8 * mt + 2 * c < op.M)
+                        ? *reinterpret_cast<const float4 *>(op.sx + 2 * (static_cast<size_t>(g) * MPAD + 8 * mt + 2 * c))
+                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                    float acc[4];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t a0 = unpack_biased<BITS>(wv[0], 2 * j);
+                        const uint32_t a1 = unpack_biased<BITS>(wv[1], 2 * j);
+                        const uint32_t a2 = unpack_biased<BITS>(wv[0], 2 * j + 1);
+                        const uint32_t a3 = unpack_biased<BITS>(wv[1], 2 * j + 1);
+                        if (j == 0)
+                            mma_16816(acc, a0, a1, a2, a3, xf[2 * j], xf[2 * j + 1], zero4);
+                        else
+                            mma_16816(acc, a0, a1, a2, a3, xf[2 * j], xf[2 * j + 1], acc);
+                    }
+                    // tot += s * (acc - bias) + z * sum(x)
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tot[mt][2 * h] = fmaf(sc[h], acc[2 * h] - sb.y, fmaf(zr[h], sb.x, tot[mt][2 * h]));
+                        tot[mt][2 * h + 1] = fmaf(sc[h], acc[2 * h + 1] - sb.w, fmaf(zr[h], sb.z, tot[mt][2 * h + 1]));
+                    }
                 }
             }
         }
 
-        if (cs.g + 1 == cs.g_end) {
-            // End of a unit: emit.
-            const DecodeOp &op = p.ops[cs.o];
-            if (op.S == 1) {
-#pragma unroll
-                for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int row = cs.r0 + rt * 16 + (i >> 1) * 8 + gq;
-                            const int tok = 8 * mt + 2 * c + (i & 1);
-                            if (row < op.N && tok < op.M)
-                                op.out[static_cast<size_t>(tok) * op.N + row] =
-                                    __half_as_ushort(__float2half_rn(tot[rt][mt][i]));
-                        }
-            } else {
-                float *pb = op.part + (static_cast<size_t>(cs.rb) * op.S + cs.slice) * ROWS * MPAD;
-#pragma unroll
-                for (int rt = 0; rt < RT; ++rt)
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int hh = 0; hh < 2; ++hh) {
-                            const int row = rt * 16 + hh * 8 + gq;
-                            *reinterpret_cast<float2 *>(pb + row * MPAD + 8 * mt + 2 * c) =
-                                make_float2(tot[rt][mt][2 * hh], tot[rt][mt][2 * hh + 1]);
-                        }
-                __threadfence();
-                __syncwarp();
-                unsigned int prev = 0;
-                if (lane == 0) prev = atomicAdd(op.cnt + cs.rb, 1u);
-                prev = __shfl_sync(0xffffffffu, prev, 0);
-                if (prev == static_cast<unsigned int>(op.S - 1)) {
-                    __threadfence();
-                    const float *p0 = op.part + static_cast<size_t>(cs.rb) * op.S * ROWS * MPAD;
-                    for (int idx = lane; idx < ROWS * op.M; idx += 32) {
-                        const int row = idx / op.M, tok = idx - row * op.M;
-                        float s = 0.0f;
-                        for (int sl = 0; sl < op.S; ++sl)
-                            s += __ldcg(p0 + (static_cast<size_t>(sl) * ROWS + row) * MPAD + tok);
-                        if (cs.r0 + row < op.N)
-                            op.out[static_cast<size_t>(tok) * op.N + cs.r0 + row] =
-                                __half_as_ushort(__float2half_rn(s));
-                    }
-                    if (lane == 0) op.cnt[cs.rb] = 0u;  // ready for the next call
-                }
-            }
-#pragma unroll
-            for (int rt = 0; rt < RT; ++rt)
+        if (cs.j + 1 == cs.SU || cs.s + 1 == s_end) {
+            // End of this warp's piece of a row block: emit.
+            const int unit_start = cs.s - cs.j;
+            const bool head = unit_start < s_begin;        // started in an earlier warp
+            const bool tail = unit_start + cs.SU > s_end;  // continues in a later warp
+            if (!head && !tail) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) tot[rt][mt][i] = 0.0f;
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = r0 + (i >> 1) * 8 + gq;
+                        const int tok = 8 * mt + 2 * c + (i & 1);
+                        if (row < op.N && tok < op.M)
+                            op.out[static_cast<size_t>(tok) * op.N + row] =
+                                __half_as_ushort(__float2half_rn(tot[mt][i]));
+                    }
+            } else {
+                // Partial piece: slot (w, 0) holds a head piece, (w, 1) a tail piece.
+                float *slot = p.part + (static_cast<size_t>(gw) * 2 + (head ? 0 : 1)) * p.slot_floats;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = (i >> 1) * 8 + gq;
+                        const int tok = 8 * mt + 2 * c + (i & 1);
+                        if (tok < op.M) slot[row * op.M + tok] = tot[mt][i];
+                    }
+                const int w_first = head ? head_first : gw;
+                const int w_last = head ? head_last : tail_last;
+                __threadfence();
+                __syncwarp();
+                unsigned int prev = 0;
+                if (lane == 0) prev = atomicAdd(p.cnt + w_first, 1u);
+                prev = __shfl_sync(0xffffffffu, prev, 0);
+                if (prev == static_cast<unsigned int>(w_last - w_first)) {
+                    // Last piece in: sum the pieces in warp order (deterministic).
+                    __threadfence();
+                    for (int idx = lane; idx < ROWS * op.M; idx += 32) {
+                        float sum = __ldcg(p.part + (static_cast<size_t>(w_first) * 2 + 1) * p.slot_floats + idx);
+                        for (int ww = w_first + 1; ww <= w_last; ++ww)
+                            sum += __ldcg(p.part + static_cast<size_t>(ww) * 2 * p.slot_floats + idx);
+                        const int row = idx / op.M, tok = idx - row * op.M;
+                        if (r0 + row < op.N)
+                            op.out[static_cast<size_t>(tok) * op.N + r0 + row] =
+                                __half_as_ushort(__float2half_rn(sum));
+                    }
+                    if (lane == 0) p.cnt[w_first] = 0u;  // ready for the next call
+                }
+            }
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) tot[mt][i] = 0.0f;
         }
-    };
-
-#pragma unroll 1
-    while (nx.valid) {
-        step(opA, opB);
-        if (!nx.valid) break;
-        step(opB, opA);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int i = 0; i < GPS; ++i) szc[h][i] = szn[h][i];
+        cursor_next(cs, p, s_end);
     }
     cp_async_wait<0>();
 }

@@ -13,8 +13,11 @@ constexpr int kQuantStatusSlots = 64;
 
 // ---------------------------------------------------------------- decode --
 // A decode launch processes up to kMaxDecodeOps independent linear layers of
-// one bit width with M <= 64.  Work is split into units (op, row block,
-// K slice) and spread over all warps of a persistent grid by cost (bytes).
+// one bit width with M <= 64.  The work is a sequence of steps, one step =
+// (op, row block, 128-wide group); op o owns steps [step0, step0 + row_blocks*G)
+// in row-block-major order.  Warp w of W takes steps [T*w/W, T*(w+1)/W)
+// (stream-K): a row block cut by a warp boundary is summed from per-warp
+// partial slots by the last warp to finish it.
 
 constexpr int kMaxDecodeOps = 128;
 constexpr int kMaxPrepEntries = 64;
@@ -24,24 +27,21 @@ struct DecodeOp {
     const uint32_t *packed;
     const uint16_t *scales;
     const uint16_t *zeros;
-    const uint16_t *xperm;  // workspace: M_pad x K fp16, chunk-permuted activations
+    const uint16_t *xperm;  // workspace: M_pad x K fp16, pair-permuted, 2^-s-scaled activations
     const float *sx;        // workspace: G x M_pad x 2 fp32 (sum x, bias) per group and token
     uint16_t *out;          // M x N fp16
-    float *part;            // workspace: split-K partials (S > 1) or null
-    unsigned int *cnt;      // workspace: split-K arrival counters (S > 1) or null
-    long long cost0;        // cost of all earlier ops (prefix)
-    long long unit_cost;    // cost of one unit
+    long long step0;        // first step of this op
     int M, N, K, G;
-    int S;                  // K slices
-    int gps;                // groups per slice (last slice may be shorter)
     int row_blocks;
-    int pad_;
+    int su;                 // steps per row block: ceil(G / GPS)
 };
 
 struct DecodeParams {
-    long long total_cost;
+    long long total_steps;
+    float *part;             // workspace: 2 partial slots per warp, slot_floats each
+    unsigned int *cnt;       // workspace: one arrival counter per warp (zero between calls)
+    int slot_floats;         // rows * max M
     int n_ops;
-    int pad_;
     DecodeOp ops[kMaxDecodeOps];
 };
 
@@ -59,17 +59,25 @@ struct PrepParams {
     PrepEntry e[kMaxPrepEntries];
 };
 
-// Decode tiling for a token-tile count MT (tokens padded to 8*MT).
-__host__ __device__ constexpr int decode_rt(int mt) { return mt == 1 ? 4 : mt == 2 ? 2 : 1; }
-__host__ __device__ constexpr int decode_rows(int mt) { return 16 * decode_rt(mt); }
-// cp.async ring depth: about 12 KB of codes per warp.
-__host__ __device__ constexpr int decode_depth(int bits, int mt) {
-    return (12288 / (decode_rows(mt) * 16 * bits)) < 2 ? 2
-         : (12288 / (decode_rows(mt) * 16 * bits)) > 8 ? 8
-                                                       : 12288 / (decode_rows(mt) * 16 * bits);
+// Decode tiling.  A warp step covers 16 weight rows x GPS groups (a 256-byte
+// row segment at 4 and 8 bits: longer DRAM bursts than one group per row).
+__host__ __device__ constexpr int decode_rows(int) { return 16; }
+__host__ __device__ constexpr int decode_gps(int bits) { return bits == 8 ? 2 : 4; }
+__host__ __device__ constexpr int decode_seg(int bits) { return decode_gps(bits) * 16 * bits; }
+// Shared-memory row stride.  2, 4 and 8 bits use an XOR swizzle of the 16-byte
+// chunks (decode_swizzle) to keep fragment reads bank-conflict free; 3 bits
+// pads each row by 16 bytes instead.
+__host__ __device__ constexpr int decode_row_stride(int bits) { return decode_seg(bits) + (bits == 3 ? 16 : 0); }
+__host__ __device__ constexpr int decode_swizzle(int bits, int row, int chunk) {
+    return bits == 2 ? chunk ^ ((row & 3) << 1) : bits == 4 ? chunk ^ ((row & 1) << 2) : bits == 8 ? chunk ^ (row & 1) : chunk;
 }
-inline size_t decode_smem_bytes(int bits, int mt) {
-    return static_cast<size_t>(kDecodeWarpsPerCta) * decode_depth(bits, mt) * decode_rows(mt) * 16 * bits;
+__host__ __device__ constexpr int decode_stage(int bits) { return 16 * decode_row_stride(bits); }
+// cp.async ring depth: about 12 KB of codes per warp.
+__host__ __device__ constexpr int decode_depth(int bits) {
+    return 12288 / decode_stage(bits) < 2 ? 2 : 12288 / decode_stage(bits) > 8 ? 8 : 12288 / decode_stage(bits);
+}
+inline size_t decode_smem_bytes(int bits, int) {
+    return static_cast<size_t>(kDecodeWarpsPerCta) * decode_depth(bits) * decode_stage(bits);
 }
 inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 

@@ -13,7 +13,7 @@
 //   warp 4     TMA producer for x (2-D tensor map, SWIZZLE_128B) and TMEM owner;
 //   warp 5     MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
 //              for the two 128-token halves into 2 x 256 fp32 TMEM columns;
-//   warps 6-9  dequant producers: packed codes -> exact fp16 codes
+//   warps 6-13 dequant producers: packed codes -> exact fp16 codes
 //              (zq_device.cuh) -> fp16(q*s + z) with one fused HFMA2 rounding ->
 //              K-order restored with PRMT -> UMMA K-major SWIZZLE_128B layout.
 // A 3-stage ring of (x, W) slabs is handed over with mbarriers; stage release is
@@ -46,7 +46,7 @@ constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kDqWarp0 = 6;
-constexpr int kDqWarps = 4;
+constexpr int kDqWarps = 8;
 constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
 constexpr int kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
@@ -328,66 +328,77 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp >= kDqWarp0) {
-        // 128 threads: thread d handles rows d/2 + 64*i (i = 0..3), 32-code chunk d%2.
+        // 256 threads: thread d owns rows d/2 and d/2 + 128 of the tile and the
+        // 32-code chunk d%2 of every slab.  Codes, scales and zeros of the next
+        // group (two slabs) are prefetched into registers.
         const int d = threadIdx.x - 32 * kDqWarp0;
         const int ch = d & 1;
         const size_t wpr = static_cast<size_t>(p.K) * B / 32;
         const int G = p.K / kGroup;
+        const int groups = slabs / 2;
         uint32_t it = 0;
-        // register prefetch of the next slab's codes and scale/zero
-        uint32_t wn[4][B], szn[4];
-        auto fetch = [&](int t, int s) {
+        uint32_t wn[2][2][B], szn[2];  // [slab of group][row][word]
+        auto fetch = [&](int t, int g) {
             int n0, t0;
             tile_coords(t, p.tok_tiles, n0, t0);
-            const int kc = s * 2 + ch;  // 32-code chunk index along K
-            const int g = (s * kBK) / kGroup;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int r = min(n0 + d / 2 + 64 * i, p.N - 1);
-                load_chunk<B>(wn[i], p.packed + static_cast<size_t>(r) * wpr + static_cast<size_t>(kc) * B);
+            for (int i = 0; i < 2; ++i) {
+                const int r = min(n0 + d / 2 + 128 * i, p.N - 1);
+                const uint32_t *rowp = p.packed + static_cast<size_t>(r) * wpr;
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    load_chunk<B>(wn[h][i], rowp + static_cast<size_t>(4 * g + 2 * h + ch) * B);
                 const size_t si = static_cast<size_t>(r) * G + g;
                 szn[i] = ldg_u16_nc(p.scales + si) | (ldg_u16_nc(p.zeros + si) << 16);
             }
         };
-        int t = blockIdx.x, s = 0;
+        int t = blockIdx.x, g = 0;
         if (t < n_tiles) fetch(t, 0);
-        while (t < n_tiles && !*abort) {
-            uint32_t wc[4][B], szc[4];
+        bool ok = true;
+        while (t < n_tiles && ok && !*abort) {
+            uint32_t wc[2][2][B], szc[2];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                szc[i] = szn[i];
+            for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int q = 0; q < B; ++q) wc[i][q] = wn[i][q];
-            }
-            const int st = it % kStages;
-            const uint32_t round = it / kStages;
-            // advance and prefetch the following slab
-            int t_n = t, s_n = s + 1;
-            if (s_n == slabs) {
-                s_n = 0;
+                for (int i = 0; i < 2; ++i)
+#pragma unroll
+                    for (int q = 0; q < B; ++q) wc[h][i][q] = wn[h][i][q];
+            szc[0] = szn[0];
+            szc[1] = szn[1];
+            int t_n = t, g_n = g + 1;
+            if (g_n == groups) {
+                g_n = 0;
                 t_n += gridDim.x;
             }
-            if (t_n < n_tiles) fetch(t_n, s_n);
-            if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) break;
-            uint8_t *bs = sm.b[st];
+            if (t_n < n_tiles) fetch(t_n, g_n);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = d / 2 + 64 * i;
-                uint32_t o[16];
-                dequant_chunk<B>(wc[i], szc[i], o);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int c16 = (4 * ch + j) ^ (row & 7);
-                    *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
-                        make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+            for (int h = 0; h < 2; ++h) {  // the two slabs of this group
+                const int st = it % kStages;
+                const uint32_t round = it / kStages;
+                if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) {
+                    ok = false;
+                    break;
                 }
+                uint8_t *bs = sm.b[st];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int row = d / 2 + 128 * i;
+                    uint32_t o[16];
+                    dequant_chunk<B>(wc[h][i], szc[i], o);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const int c16 = (4 * ch + j) ^ (row & 7);
+                        *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
+                            make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                    }
+                }
+                fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.full[st]);
+                ++it;
             }
-            fence_proxy_async();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.full[st]);
-            ++it;
             t = t_n;
-            s = s_n;
+            g = g_n;
         }
     } else {
         // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = tokens of each half.
