@@ -31,10 +31,25 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <type_traits>
+
 #include "zq_device.cuh"
 #include "zq_internal.h"
 
 namespace zq {
+
+template <int I, int N, typename F>
+__device__ __forceinline__ void static_for_impl(F &f) {
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for_impl<I + 1, N>(f);
+    }
+}
+// Calls f(integral_constant<int, i>) for i = 0 .. N-1 (compile-time indices).
+template <int N, typename F>
+__device__ __forceinline__ void static_for(F &&f) {
+    static_for_impl<0, N>(f);
+}
 
 // ------------------------------------------------------------------ prep --
 // One warp per (entry, padded token, group): writes the pair-permuted copy of
@@ -174,6 +189,37 @@ __device__ __forceinline__ void load_scale_zero(uint32_t (&sz)[2][GPS], const De
     }
 }
 
+// One k16 step of a group: biased codes of pairs 2J, 2J+1 (rows gq, gq + 8)
+// times the activation pairs; J is a compile-time index so the unpack masks
+// are instruction immediates.
+template <int BITS, int J>
+__device__ __forceinline__ void mma_j(float (&acc)[4], const uint32_t (&w)[2][BITS], const uint32_t (&xf)[16],
+                                      uint32_t magic) {
+    const uint32_t a0 = unpack_biased_c<BITS, 2 * J>(w[0], magic);
+    const uint32_t a1 = unpack_biased_c<BITS, 2 * J>(w[1], magic);
+    const uint32_t a2 = unpack_biased_c<BITS, 2 * J + 1>(w[0], magic);
+    const uint32_t a3 = unpack_biased_c<BITS, 2 * J + 1>(w[1], magic);
+    if constexpr (J == 0) {
+        const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        mma_16816(acc, a0, a1, a2, a3, xf[2 * J], xf[2 * J + 1], zero4);
+    } else {
+        mma_16816(acc, a0, a1, a2, a3, xf[2 * J], xf[2 * J + 1], acc);
+    }
+}
+
+template <int BITS>
+__device__ __forceinline__ void mma_group(float (&acc)[4], const uint32_t (&w)[2][BITS], const uint32_t (&xf)[16],
+                                          uint32_t magic) {
+    mma_j<BITS, 0>(acc, w, xf, magic);
+    mma_j<BITS, 1>(acc, w, xf, magic);
+    mma_j<BITS, 2>(acc, w, xf, magic);
+    mma_j<BITS, 3>(acc, w, xf, magic);
+    mma_j<BITS, 4>(acc, w, xf, magic);
+    mma_j<BITS, 5>(acc, w, xf, magic);
+    mma_j<BITS, 6>(acc, w, xf, magic);
+    mma_j<BITS, 7>(acc, w, xf, magic);
+}
+
 template <int BITS, int MT>
 __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -223,17 +269,29 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
         const size_t row_stride = static_cast<size_t>(op.K) * BITS / 8;  // bytes
         const int g0 = cu.j * GPS;
         const int ng = min(GPS, op.G - g0);
-        const uint8_t *base = reinterpret_cast<const uint8_t *>(op.packed) + static_cast<size_t>(g0) * GB;
-        uint8_t *st = ring + slot * STAGE;
         const int r0 = cu.rb * ROWS;
+        uint8_t *st = ring + slot * STAGE;
+        // chunk ch = lane + 32 i: row = ch / CPR, part = ch % CPR.
+        if (ng == GPS && r0 + ROWS <= op.N) {
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(op.packed) + static_cast<size_t>(g0) * GB;
 #pragma unroll
-        for (int i = 0; i < CPL; ++i) {
-            const int ch = lane + 32 * i;
-            const int row = ch / CPR, part = ch % CPR;
-            if (part / BITS < ng) {
-                const int r = min(r0 + row, op.N - 1);
+            for (int i = 0; i < CPL; ++i) {
+                const int ch = lane + 32 * i;
+                const int row = ch / CPR, part = ch % CPR;
                 cp_async16(st + row * RS + decode_swizzle(BITS, row, part) * 16,
-                           base + static_cast<size_t>(r) * row_stride + part * 16);
+                           src + static_cast<size_t>(r0 + row) * row_stride + part * 16);
+            }
+        } else {
+            const uint8_t *src = reinterpret_cast<const uint8_t *>(op.packed) + static_cast<size_t>(g0) * GB;
+#pragma unroll
+            for (int i = 0; i < CPL; ++i) {
+                const int ch = lane + 32 * i;
+                const int row = ch / CPR, part = ch % CPR;
+                if (part / BITS < ng) {
+                    const int r = min(r0 + row, op.N - 1);
+                    cp_async16(st + row * RS + decode_swizzle(BITS, row, part) * 16,
+                               src + static_cast<size_t>(r) * row_stride + part * 16);
+                }
             }
         }
     };
@@ -259,7 +317,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     for (int b = 0; b < MT; ++b)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tot[b][i] = 0.0f;
-    const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    const uint32_t magic = kMagic;
 
 #pragma unroll 1
     while (cs.valid) {
@@ -286,89 +344,98 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
         const uint8_t *st = ring + slot_cs * STAGE;
         slot_cs = slot_cs + 1 == D ? 0 : slot_cs + 1;
 
+        // Per-step bases of the activation fragments and group sums; the
+        // groups of the step are at immediate offsets from them.
+        const uint16_t *xb[MT];
+        const float *sbb[MT];
+        bool xon[MT], sbon[MT];
 #pragma unroll
-        for (int gi = 0; gi < GPS; ++gi) {
-            if (gi < ng) {
-                const int g = g0 + gi;
-                // this thread's 32-code chunk of rows gq and gq + 8
-                uint32_t wv[2][BITS];
+        for (int mt = 0; mt < MT; ++mt) {
+            const int tok = 8 * mt + gq;
+            xon[mt] = tok < op.M;
+            sbon[mt] = 8 * mt + 2 * c < op.M;
+            xb[mt] = op.xperm + static_cast<size_t>(xon[mt] ? tok : 0) * op.K + static_cast<size_t>(g0) * kGroup + 32 * c;
+            sbb[mt] = op.sx + 2 * (static_cast<size_t>(g0) * MPAD + 8 * mt + 2 * c);
+        }
+        const bool one_token = op.M == 1;
+
+        auto group = [&](auto gi_c) {
+            constexpr int gi = decltype(gi_c)::value;
+            // this thread's 32-code chunk of rows gq and gq + 8
+            uint32_t wv[2][BITS];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int row = h * 8 + gq;
-                    const uint8_t *rp = st + row * RS;
-                    if constexpr (BITS == 2) {
-                        const int ch = decode_swizzle(2, row, gi * 2 + (c >> 1));
-                        const uint2 v = *reinterpret_cast<const uint2 *>(rp + ch * 16 + (c & 1) * 8);
-                        wv[h][0] = v.x;
-                        wv[h][1] = v.y;
-                    } else if constexpr (BITS == 3) {
-                        const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + gi * GB + 12 * c);
-                        wv[h][0] = q[0];
-                        wv[h][1] = q[1];
-                        wv[h][2] = q[2];
-                    } else if constexpr (BITS == 4) {
-                        const uint4 v = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(4, row, gi * 4 + c) * 16);
-                        wv[h][0] = v.x;
-                        wv[h][1] = v.y;
-                        wv[h][2] = v.z;
-                        wv[h][3] = v.w;
-                    } else {
-                        const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c) * 16);
-                        const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c + 1) * 16);
-                        wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
-                        wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
-                    }
-                }
-                // scale and zero of this group for rows gq, gq + 8
-                const uint32_t sp0 = szc[0][gi / 2], sp1 = szc[1][gi / 2];
-                const uint32_t zp0 = szc[0][GPS / 2 + gi / 2], zp1 = szc[1][GPS / 2 + gi / 2];
-                const float sc[2] = {h2f_bits((gi & 1) ? (sp0 >> 16) : (sp0 & 0xFFFFu)),
-                                     h2f_bits((gi & 1) ? (sp1 >> 16) : (sp1 & 0xFFFFu))};
-                const float zr[2] = {h2f_bits((gi & 1) ? (zp0 >> 16) : (zp0 & 0xFFFFu)),
-                                     h2f_bits((gi & 1) ? (zp1 >> 16) : (zp1 & 0xFFFFu))};
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    // B fragments and group sums of this token tile (L1 hits)
-                    uint32_t xf[16];
-                    const int tok = 8 * mt + gq;
-                    if (tok < op.M) {
-                        const uint16_t *xp = op.xperm + static_cast<size_t>(tok) * op.K +
-                                             static_cast<size_t>(g) * kGroup + 32 * c;
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            const uint4 w = ldg_u4(xp + 8 * q);
-                            xf[4 * q + 0] = w.x;
-                            xf[4 * q + 1] = w.y;
-                            xf[4 * q + 2] = w.z;
-                            xf[4 * q + 3] = w.w;
-                        }
-                    } else {
-#pragma unroll
-                        for (int q = 0; q < 16; ++q) xf[q] = 0u;
-                    }
-                    const float4 sb = (8 * mt + 2 * c < op.M)
-                        ? *reinterpret_cast<const float4 *>(op.sx + 2 * (static_cast<size_t>(g) * MPAD + 8 * mt + 2 * c))
-                        : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-                    float acc[4];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        const uint32_t a0 = unpack_biased<BITS>(wv[0], 2 * j);
-                        const uint32_t a1 = unpack_biased<BITS>(wv[1], 2 * j);
-                        const uint32_t a2 = unpack_biased<BITS>(wv[0], 2 * j + 1);
-                        const uint32_t a3 = unpack_biased<BITS>(wv[1], 2 * j + 1);
-                        if (j == 0)
-                            mma_16816(acc, a0, a1, a2, a3, xf[2 * j], xf[2 * j + 1], zero4);
-                        else
-                            mma_16816(acc, a0, a1, a2, a3, xf[2 * j], xf[2 * j + 1], acc);
-                    }
-                    // tot += s * (acc - bias) + z * sum(x)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tot[mt][2 * h] = fmaf(sc[h], acc[2 * h] - sb.y, fmaf(zr[h], sb.x, tot[mt][2 * h]));
-                        tot[mt][2 * h + 1] = fmaf(sc[h], acc[2 * h + 1] - sb.w, fmaf(zr[h], sb.z, tot[mt][2 * h + 1]));
-                    }
+            for (int h = 0; h < 2; ++h) {
+                const int row = h * 8 + gq;
+                const uint8_t *rp = st + row * RS;
+                if constexpr (BITS == 2) {
+                    const int ch = decode_swizzle(2, row, gi * 2 + (c >> 1));
+                    const uint2 v = *reinterpret_cast<const uint2 *>(rp + ch * 16 + (c & 1) * 8);
+                    wv[h][0] = v.x;
+                    wv[h][1] = v.y;
+                } else if constexpr (BITS == 3) {
+                    const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + gi * GB + 12 * c);
+                    wv[h][0] = q[0];
+                    wv[h][1] = q[1];
+                    wv[h][2] = q[2];
+                } else if constexpr (BITS == 4) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(4, row, gi * 4 + c) * 16);
+                    wv[h][0] = v.x;
+                    wv[h][1] = v.y;
+                    wv[h][2] = v.z;
+                    wv[h][3] = v.w;
+                } else {
+                    const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c) * 16);
+                    const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c + 1) * 16);
+                    wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
+                    wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
                 }
             }
+            // scale and zero of this group for rows gq, gq + 8
+            constexpr int hi = gi & 1;
+            const uint32_t sp0 = szc[0][gi / 2], sp1 = szc[1][gi / 2];
+            const uint32_t zp0 = szc[0][GPS / 2 + gi / 2], zp1 = szc[1][GPS / 2 + gi / 2];
+            const float sc[2] = {h2f_bits(hi ? (sp0 >> 16) : (sp0 & 0xFFFFu)), h2f_bits(hi ? (sp1 >> 16) : (sp1 & 0xFFFFu))};
+            const float zr[2] = {h2f_bits(hi ? (zp0 >> 16) : (zp0 & 0xFFFFu)), h2f_bits(hi ? (zp1 >> 16) : (zp1 & 0xFFFFu))};
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                // B fragments and group sums of this token tile (L1 hits)
+                uint32_t xf[16];
+                if (xon[mt]) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 w = ldg_u4(xb[mt] + gi * kGroup + 8 * q);
+                        xf[4 * q + 0] = w.x;
+                        xf[4 * q + 1] = w.y;
+                        xf[4 * q + 2] = w.z;
+                        xf[4 * q + 3] = w.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) xf[q] = 0u;
+                }
+                const float4 sb = sbon[mt] ? *reinterpret_cast<const float4 *>(sbb[mt] + gi * 2 * MPAD)
+                                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                float acc[4];
+                mma_group<BITS>(acc, wv, xf, magic);
+                // tot += s * (acc - bias) + z * sum(x); with one token the odd
+                // C columns are padding.
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tot[mt][2 * h] = fmaf(sc[h], acc[2 * h] - sb.y, fmaf(zr[h], sb.x, tot[mt][2 * h]));
+                if (MT > 1 || !one_token) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tot[mt][2 * h + 1] = fmaf(sc[h], acc[2 * h + 1] - sb.w, fmaf(zr[h], sb.z, tot[mt][2 * h + 1]));
+                }
+            }
+        };
+        if (ng == GPS) {
+            static_for<GPS>(group);
+        } else {
+            static_for<GPS>([&](auto gi_c) {
+                constexpr int gv = decltype(gi_c)::value;
+                if (gv < ng) group(gi_c);
+            });
         }
 
         if (cs.j + 1 == cs.SU || cs.s + 1 == s_end) {

@@ -26,6 +26,14 @@ __device__ __forceinline__ uint32_t lop_and_or(uint32_t a, uint32_t mask, uint32
     return r;
 }
 
+// Same with the mask as an instruction immediate (no register for it).
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t lop_and_or_imm(uint32_t a, uint32_t magic) {
+    uint32_t r;  // (a & MASK) | magic
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(a), "n"(MASK), "r"(magic));
+    return r;
+}
+
 __device__ __forceinline__ uint32_t hfma2_bits(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t r;
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
@@ -167,6 +175,28 @@ template <>
 __device__ __forceinline__ uint32_t unpack_biased<8>(const uint32_t (&w)[8], int p) {
     const uint32_t u = (p % 2) == 0 ? w[p / 2] : (w[p / 2] >> 8);
     return lop_and_or(u, 0x00FF00FFu, kMagic);
+}
+
+// Biased pair with the pair index known at compile time: the LOP3 mask is an
+// immediate.  Same pairs as unpack_biased<B>(w, P).
+template <int B, int P>
+__device__ __forceinline__ uint32_t unpack_biased_c(const uint32_t (&w)[B], uint32_t magic) {
+    if constexpr (B == 2) {
+        constexpr int j = P % 8;
+        if constexpr (j < 5) return lop_and_or_imm<(0x00030003u << (2 * j))>(w[P / 8], magic);
+        else return lop_and_or_imm<(0x00030003u << (2 * (j - 5)))>(w[P / 8] >> 10, magic);
+    } else if constexpr (B == 3) {
+        constexpr int m = P / 3, j = P % 3, a = 9 * m;
+        const uint32_t lo = a < 32 ? shf_r(w[0], w[1], a) : shf_r(w[1], w[2], a - 32);
+        const uint32_t hi = a + 16 < 32 ? shf_r(w[1], w[2], a + 16) : (w[2] >> (a - 16));
+        return lop_and_or_imm<(0x00070007u << (3 * j))>(prmt(lo, hi, 0x5410u), magic);
+    } else if constexpr (B == 4) {
+        const uint32_t u = (P % 4) < 2 ? w[P / 4] : (w[P / 4] >> 8);
+        return lop_and_or_imm<((P % 2) == 0 ? 0x000F000Fu : 0x00F000F0u)>(u, magic);
+    } else {
+        const uint32_t u = (P % 2) == 0 ? w[P / 2] : (w[P / 2] >> 8);
+        return lop_and_or_imm<0x00FF00FFu>(u, magic);
+    }
 }
 
 // Exact codes: one HFMA2 by (2^-s, -1024 * 2^-s) removes bias and offset.
