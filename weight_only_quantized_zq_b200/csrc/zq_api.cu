@@ -279,6 +279,13 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         o.G = ops[i].K / kGroup;
         o.row_blocks = rbs[i];
         o.su = (o.G + gps - 1) / gps;
+        o.sz_vec = (o.G % gps) == 0 ? 1 : 0;
+        const uint64_t row_bytes = static_cast<uint64_t>(o.K) * bits / 8;
+        cudaError_t te = encode_tensor_map_2d(&o.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, o.packed, row_bytes,
+                                              static_cast<uint64_t>(o.N), row_bytes,
+                                              static_cast<uint32_t>(decode_seg(bits)), static_cast<uint32_t>(rows),
+                                              CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (te != cudaSuccess) return cuda_fail(te, "tensor map for the packed codes");
         o.step0 = step0;
         step0 += static_cast<long long>(rbs[i]) * o.su;
     }
@@ -517,10 +524,13 @@ uint64_t zq_kernel_launches(void) { return g_launches.load(); }
 zq_status zq_check_device(void) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    int err = 0;
+    int err = 0, err2 = 0;
     e = read_prefill_error(&err);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-    if (err != 0) return fail(static_cast<zq_status>(err), "a kernel gave up a bounded wait");
+    e = read_decode_error(&err2);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (err != 0 || err2 != 0)
+        return fail(static_cast<zq_status>(err ? err : err2), "a kernel gave up a bounded wait");
     return ZQ_OK;
 }
 

@@ -220,25 +220,33 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint32_t (&w)[2
     mma_j<BITS, 7>(acc, w, xf, magic);
 }
 
+// Device record of a decode kernel that gave up a bounded wait (ZQ_ERR_TIMEOUT).
+__device__ int g_decode_error;
+
+constexpr unsigned long long kDecodeWaitNs = 2000000000ull;  // 2 s
+
 template <int BITS, int MT>
 __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int ROWS = 16;
     constexpr int GPS = decode_gps(BITS);
     constexpr int GB = 16 * BITS;                 // bytes of one row of one group
-    constexpr int RS = decode_row_stride(BITS);   // shared-memory row stride
+    constexpr int SEG = decode_seg(BITS);         // bytes of one row per step
+    constexpr int CODES = ROWS * SEG;             // TMA box bytes
     constexpr int STAGE = decode_stage(BITS);
-    constexpr int CPR = GPS * BITS;               // 16-byte chunks per row per step
-    constexpr int CPL = ROWS * CPR / 32;          // chunks per lane
     constexpr int D = decode_depth(BITS);
     constexpr int MPAD = 8 * MT;
-    static_assert(ROWS * CPR % 32 == 0, "chunks must split evenly over the warp");
+    constexpr int SZB = 2 * GPS;                  // bytes of scales (or zeros) of one row per step
 
-    extern __shared__ __align__(128) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem_raw[];
+    // TMA destinations: 128-byte aligned (the host adds 128 bytes of slack).
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2;  // MMA group id: row (A, C) / token (B)
     const int c = lane & 3;    // quad position: 32-code chunk (A, B) / token pair (C)
     uint8_t *ring = smem + warp * D * STAGE;
+    unsigned long long *bars =
+        reinterpret_cast<unsigned long long *>(smem + kDecodeWarpsPerCta * D * STAGE) + warp * D;
 
     // At most one warp per step, so every warp range is non-empty: a row block
     // split over warps w_first..w_last gets a piece from each of them.
@@ -248,9 +256,14 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     const int s_begin = gw < W ? static_cast<int>(T * gw / W) : 0;
     const int s_end = gw < W ? static_cast<int>(T * (gw + 1) / W) : 0;
 
+    if (lane == 0)
+        for (int i = 0; i < D; ++i) mbar_init(&bars[i], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncwarp();
+
     Cursor cs;
     cursor_init(cs, p, s_begin, s_end);
-    Cursor ld = cs, nx = cs;
+    Cursor ld = cs;
 
     // Row blocks cut by this warp's range (see warp_of); computed once, so the
     // 64-bit division stays out of the loop.
@@ -264,51 +277,43 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
         tail_last = warp_of(static_cast<long long>(s_end) - 1 - lc.j + lc.SU - 1, W, T);
     }
 
+    // Loader: codes of 16 rows x GPS groups by one TMA (out-of-range rows and
+    // groups read as zeros), then scales and zeros by one cp.async per lane.
     auto issue = [&](const Cursor &cu, int slot) {
         const DecodeOp &op = p.ops[cu.o];
-        const size_t row_stride = static_cast<size_t>(op.K) * BITS / 8;  // bytes
         const int g0 = cu.j * GPS;
-        const int ng = min(GPS, op.G - g0);
         const int r0 = cu.rb * ROWS;
         uint8_t *st = ring + slot * STAGE;
-        // chunk ch = lane + 32 i: row = ch / CPR, part = ch % CPR.
-        if (ng == GPS && r0 + ROWS <= op.N) {
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(op.packed) + static_cast<size_t>(g0) * GB;
-#pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                const int ch = lane + 32 * i;
-                const int row = ch / CPR, part = ch % CPR;
-                cp_async16(st + row * RS + decode_swizzle(BITS, row, part) * 16,
-                           src + static_cast<size_t>(r0 + row) * row_stride + part * 16);
-            }
-        } else {
-            const uint8_t *src = reinterpret_cast<const uint8_t *>(op.packed) + static_cast<size_t>(g0) * GB;
-#pragma unroll
-            for (int i = 0; i < CPL; ++i) {
-                const int ch = lane + 32 * i;
-                const int row = ch / CPR, part = ch % CPR;
-                if (part / BITS < ng) {
-                    const int r = min(r0 + row, op.N - 1);
-                    cp_async16(st + row * RS + decode_swizzle(BITS, row, part) * 16,
-                               src + static_cast<size_t>(r) * row_stride + part * 16);
-                }
-            }
+        if (lane == 0) {
+            fence_proxy_async();  // the warp's reads of this slot precede the overwrite
+            mbar_arrive_expect_tx(&bars[slot], CODES);
+            tma_load_2d(st, &op.tmap, g0 * GB, r0, &bars[slot]);
+        }
+        if (op.sz_vec) {
+            const int row = lane >> 1;
+            const int r = min(r0 + row, op.N - 1);
+            const uint16_t *src = ((lane & 1) ? op.zeros : op.scales) + static_cast<size_t>(r) * op.G + g0;
+            if constexpr (SZB == 8)
+                cp_async8(st + CODES + lane * 8, src);
+            else
+                cp_async4(st + CODES + lane * SZB, src);
         }
     };
 
     // Prologue: weights do not depend on the previous kernel; start them now.
     int slot_ld = 0, slot_cs = 0;
+    uint32_t par_cs = 0;          // parity of the next phase of slot_cs
+    int n_issued = 0, n_consumed = 0;
 #pragma unroll 1
     for (int i = 0; i < D - 1; ++i) {
         if (ld.valid) {
             issue(ld, slot_ld);
             cursor_next(ld, p, s_end);
+            ++n_issued;
         }
         cp_async_commit();
         slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
     }
-    uint32_t szc[2][GPS];  // scales/zeros of the current step (loaded one step ahead)
-    if (cs.valid) load_scale_zero<GPS>(szc, p.ops[cs.o], cs.rb * ROWS, cs.j * GPS, gq);
     pdl_wait();  // the prepared activations come from the previous kernel
     pdl_launch_dependents();
 
@@ -318,31 +323,23 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tot[b][i] = 0.0f;
     const uint32_t magic = kMagic;
+    bool aborted = false;
 
 #pragma unroll 1
-    while (cs.valid) {
+    while (cs.valid && !aborted) {
         __syncwarp();
         if (ld.valid) {
             issue(ld, slot_ld);
             cursor_next(ld, p, s_end);
+            ++n_issued;
         }
         cp_async_commit();
         slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
-
-        // Scales/zeros of the next step.
-        cursor_next(nx, p, s_end);
-        uint32_t szn[2][GPS];
-        if (nx.valid) load_scale_zero<GPS>(szn, p.ops[nx.o], nx.rb * ROWS, nx.j * GPS, gq);
 
         const DecodeOp &op = p.ops[cs.o];
         const int r0 = cs.rb * ROWS;
         const int g0 = cs.j * GPS;
         const int ng = min(GPS, op.G - g0);
-
-        cp_async_wait<D - 1>();
-        __syncwarp();
-        const uint8_t *st = ring + slot_cs * STAGE;
-        slot_cs = slot_cs + 1 == D ? 0 : slot_cs + 1;
 
         // Per-step bases of the activation fragments and group sums; the
         // groups of the step are at immediate offsets from them.
@@ -358,65 +355,126 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
             sbb[mt] = op.sx + 2 * (static_cast<size_t>(g0) * MPAD + 8 * mt + 2 * c);
         }
         const bool one_token = op.M == 1;
+        // Activation fragments, ping-pong by group parity; group 0 is loaded
+        // before the waits, group gi + 1 while group gi computes.
+        uint32_t xf[2][MT][16];
+        auto load_x = [&](uint32_t (&dst)[MT][16], int gi) {
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                if (xon[mt]) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 w = ldg_u4(xb[mt] + gi * kGroup + 8 * q);
+                        dst[mt][4 * q + 0] = w.x;
+                        dst[mt][4 * q + 1] = w.y;
+                        dst[mt][4 * q + 2] = w.z;
+                        dst[mt][4 * q + 3] = w.w;
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 16; ++q) dst[mt][q] = 0u;
+                }
+            }
+        };
+        load_x(xf[0], 0);
 
-        auto group = [&](auto gi_c) {
-            constexpr int gi = decltype(gi_c)::value;
-            // this thread's 32-code chunk of rows gq and gq + 8
-            uint32_t wv[2][BITS];
+        // Wait for this step's codes (TMA, bounded) and scales/zeros (cp.async).
+        {
+            bool ok = mbar_try_wait(&bars[slot_cs], par_cs);
+            if (!ok) {
+                const unsigned long long t0 = globaltimer();
+                while (!(ok = mbar_try_wait(&bars[slot_cs], par_cs)))
+                    if (globaltimer() - t0 > kDecodeWaitNs) break;
+            }
+            if (!ok) {
+                if (lane == 0) atomicExch(&g_decode_error, 5);  // ZQ_ERR_TIMEOUT
+                aborted = true;
+                break;
+            }
+        }
+        cp_async_wait<D - 1>();
+        __syncwarp();
+        const uint8_t *st = ring + slot_cs * STAGE;
+        ++n_consumed;
+        if (++slot_cs == D) {
+            slot_cs = 0;
+            par_cs ^= 1u;
+        }
+
+        // Scales and zeros of rows gq and gq + 8 for the GPS groups.
+        uint32_t szs[2][GPS / 2], szz[2][GPS / 2];
+        if (op.sz_vec) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 const int row = h * 8 + gq;
-                const uint8_t *rp = st + row * RS;
+                if constexpr (GPS == 4) {
+                    const uint4 v = *reinterpret_cast<const uint4 *>(st + CODES + row * 16);
+                    szs[h][0] = v.x;
+                    szs[h][1] = v.y;
+                    szz[h][0] = v.z;
+                    szz[h][1] = v.w;
+                } else {
+                    const uint2 v = *reinterpret_cast<const uint2 *>(st + CODES + row * 8);
+                    szs[h][0] = v.x;
+                    szz[h][0] = v.y;
+                }
+            }
+        } else {
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = min(r0 + h * 8 + gq, op.N - 1);
+#pragma unroll
+                for (int i = 0; i < GPS / 2; ++i) {
+                    const int ga = min(g0 + 2 * i, op.G - 1), gb = min(g0 + 2 * i + 1, op.G - 1);
+                    const size_t ia = static_cast<size_t>(r) * op.G + ga, ib = static_cast<size_t>(r) * op.G + gb;
+                    szs[h][i] = ldg_u16_nc(op.scales + ia) | (ldg_u16_nc(op.scales + ib) << 16);
+                    szz[h][i] = ldg_u16_nc(op.zeros + ia) | (ldg_u16_nc(op.zeros + ib) << 16);
+                }
+            }
+        }
+
+        auto group = [&](auto gi_c) {
+            constexpr int gi = decltype(gi_c)::value;
+            // next group's activation fragments, one group ahead
+            if (gi + 1 < GPS) load_x(xf[(gi + 1) & 1], gi + 1);
+            // this thread's 32-code chunk of rows gq and gq + 8 (dense rows of SEG bytes)
+            uint32_t wv[2][BITS];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint8_t *rp = st + (h * 8 + gq) * SEG + gi * GB;
                 if constexpr (BITS == 2) {
-                    const int ch = decode_swizzle(2, row, gi * 2 + (c >> 1));
-                    const uint2 v = *reinterpret_cast<const uint2 *>(rp + ch * 16 + (c & 1) * 8);
+                    const uint2 v = *reinterpret_cast<const uint2 *>(rp + 8 * c);
                     wv[h][0] = v.x;
                     wv[h][1] = v.y;
                 } else if constexpr (BITS == 3) {
-                    const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + gi * GB + 12 * c);
+                    const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + 12 * c);
                     wv[h][0] = q[0];
                     wv[h][1] = q[1];
                     wv[h][2] = q[2];
                 } else if constexpr (BITS == 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(4, row, gi * 4 + c) * 16);
+                    const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * c);
                     wv[h][0] = v.x;
                     wv[h][1] = v.y;
                     wv[h][2] = v.z;
                     wv[h][3] = v.w;
                 } else {
-                    const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c) * 16);
-                    const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + decode_swizzle(8, row, gi * 8 + 2 * c + 1) * 16);
+                    const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + 32 * c);
+                    const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + 32 * c + 16);
                     wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
                     wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
                 }
             }
-            // scale and zero of this group for rows gq, gq + 8
             constexpr int hi = gi & 1;
-            const uint32_t sp0 = szc[0][gi / 2], sp1 = szc[1][gi / 2];
-            const uint32_t zp0 = szc[0][GPS / 2 + gi / 2], zp1 = szc[1][GPS / 2 + gi / 2];
-            const float sc[2] = {h2f_bits(hi ? (sp0 >> 16) : (sp0 & 0xFFFFu)), h2f_bits(hi ? (sp1 >> 16) : (sp1 & 0xFFFFu))};
-            const float zr[2] = {h2f_bits(hi ? (zp0 >> 16) : (zp0 & 0xFFFFu)), h2f_bits(hi ? (zp1 >> 16) : (zp1 & 0xFFFFu))};
+            const float sc[2] = {h2f_bits(hi ? (szs[0][gi / 2] >> 16) : (szs[0][gi / 2] & 0xFFFFu)),
+                                 h2f_bits(hi ? (szs[1][gi / 2] >> 16) : (szs[1][gi / 2] & 0xFFFFu))};
+            const float zr[2] = {h2f_bits(hi ? (szz[0][gi / 2] >> 16) : (szz[0][gi / 2] & 0xFFFFu)),
+                                 h2f_bits(hi ? (szz[1][gi / 2] >> 16) : (szz[1][gi / 2] & 0xFFFFu))};
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                // B fragments and group sums of this token tile (L1 hits)
-                uint32_t xf[16];
-                if (xon[mt]) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 w = ldg_u4(xb[mt] + gi * kGroup + 8 * q);
-                        xf[4 * q + 0] = w.x;
-                        xf[4 * q + 1] = w.y;
-                        xf[4 * q + 2] = w.z;
-                        xf[4 * q + 3] = w.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) xf[q] = 0u;
-                }
                 const float4 sb = sbon[mt] ? *reinterpret_cast<const float4 *>(sbb[mt] + gi * 2 * MPAD)
                                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 float acc[4];
-                mma_group<BITS>(acc, wv, xf, magic);
+                mma_group<BITS>(acc, wv, xf[gi & 1][mt], magic);
                 // tot += s * (acc - bias) + z * sum(x); with one token the odd
                 // C columns are padding.
 #pragma unroll
@@ -492,16 +550,26 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) tot[mt][i] = 0.0f;
         }
-#pragma unroll
-        for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int i = 0; i < GPS; ++i) szc[h][i] = szn[h][i];
         cursor_next(cs, p, s_end);
     }
+    // Copies still in flight (only after an abort) must land before the CTA
+    // can exit: wait for every issued, unconsumed stage, bounded.
     cp_async_wait<0>();
+    for (int k = n_consumed; k < n_issued; ++k) {
+        const unsigned long long t0 = globaltimer();
+        while (!mbar_try_wait(&bars[k % D], (k / D) & 1u) && globaltimer() - t0 < kDecodeWaitNs) {
+        }
+    }
 }
 
 // ------------------------------------------------------------------ host --
+
+cudaError_t read_decode_error(int *err) {
+    cudaError_t e = cudaMemcpyFromSymbol(err, g_decode_error, sizeof(int));
+    if (e != cudaSuccess) return e;
+    const int zero = 0;
+    return cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(int));
+}
 
 cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};

@@ -2,6 +2,7 @@
 // kernel translation units of libzq.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -19,11 +20,12 @@ constexpr int kQuantStatusSlots = 64;
 // (stream-K): a row block cut by a warp boundary is summed from per-warp
 // partial slots by the last warp to finish it.
 
-constexpr int kMaxDecodeOps = 128;
+constexpr int kMaxDecodeOps = 112;
 constexpr int kMaxPrepEntries = 64;
 constexpr int kDecodeWarpsPerCta = 4;
 
-struct DecodeOp {
+struct alignas(64) DecodeOp {
+    CUtensorMap tmap;       // packed codes as a 2-D uint8 tensor: box = 16 rows x one step's bytes
     const uint32_t *packed;
     const uint16_t *scales;
     const uint16_t *zeros;
@@ -34,6 +36,8 @@ struct DecodeOp {
     int M, N, K, G;
     int row_blocks;
     int su;                 // steps per row block: ceil(G / GPS)
+    int sz_vec;             // G % GPS == 0: scales/zeros of a step are one aligned vector per row
+    int pad_;
 };
 
 struct DecodeParams {
@@ -44,6 +48,7 @@ struct DecodeParams {
     int n_ops;
     DecodeOp ops[kMaxDecodeOps];
 };
+static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
@@ -64,20 +69,17 @@ struct PrepParams {
 __host__ __device__ constexpr int decode_rows(int) { return 16; }
 __host__ __device__ constexpr int decode_gps(int bits) { return bits == 8 ? 2 : 4; }
 __host__ __device__ constexpr int decode_seg(int bits) { return decode_gps(bits) * 16 * bits; }
-// Shared-memory row stride.  2, 4 and 8 bits use an XOR swizzle of the 16-byte
-// chunks (decode_swizzle) to keep fragment reads bank-conflict free; 3 bits
-// pads each row by 16 bytes instead.
-__host__ __device__ constexpr int decode_row_stride(int bits) { return decode_seg(bits) + (bits == 3 ? 16 : 0); }
-__host__ __device__ constexpr int decode_swizzle(int bits, int row, int chunk) {
-    return bits == 2 ? chunk ^ ((row & 3) << 1) : bits == 4 ? chunk ^ ((row & 1) << 2) : bits == 8 ? chunk ^ (row & 1) : chunk;
-}
-__host__ __device__ constexpr int decode_stage(int bits) { return 16 * decode_row_stride(bits); }
-// cp.async ring depth: about 12 KB of codes per warp.
+// Per-warp ring stage: the step's codes (dense, written by TMA) followed by
+// the step's scales and zeros, 16 rows x {scales, zeros} x GPS halves.
+__host__ __device__ constexpr int decode_sz_bytes(int bits) { return 16 * 2 * decode_gps(bits) * 2; }
+__host__ __device__ constexpr int decode_stage(int bits) { return 16 * decode_seg(bits) + decode_sz_bytes(bits); }
+// Ring depth: about 13 KB per warp, at least 3 stages.
 __host__ __device__ constexpr int decode_depth(int bits) {
-    return 12288 / decode_stage(bits) < 2 ? 2 : 12288 / decode_stage(bits) > 8 ? 8 : 12288 / decode_stage(bits);
+    return 13312 / decode_stage(bits) < 3 ? 3 : 13312 / decode_stage(bits) > 6 ? 6 : 13312 / decode_stage(bits);
 }
 inline size_t decode_smem_bytes(int bits, int) {
-    return static_cast<size_t>(kDecodeWarpsPerCta) * decode_depth(bits) * decode_stage(bits);
+    return static_cast<size_t>(kDecodeWarpsPerCta) * (decode_depth(bits) * decode_stage(bits) + 8 * decode_depth(bits)) +
+           128;
 }
 inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
@@ -92,6 +94,10 @@ cudaError_t launch_prefill(const uint16_t *x, const uint32_t *packed, const uint
                            const uint16_t *zeros, int bits, int M, int N, int K, uint16_t *out, int num_sms,
                            cudaStream_t stream);
 cudaError_t read_prefill_error(int *err);
+cudaError_t read_decode_error(int *err);
+cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t dim0,
+                                 uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                                 CUtensorMapSwizzle swizzle);
 
 // Largest M handled by the decode family; larger M goes to the prefill family.
 constexpr int kDecodeMaxM = 64;
