@@ -112,6 +112,30 @@ ZQ_API zq_status zq_linear(const uint16_t *x, const uint32_t *packed,
                     int bits, int group, int M, int N, int K,
                     uint16_t *out, zq_stream_t stream);
 
+/* Allocation-free zq_linear, for callers that cannot allocate device memory:
+ * code running inside a CUDA stream capture (where cudaMalloc is not
+ * allowed), code under a fixed device-memory budget, or latency-critical
+ * paths that must not risk the device-wide synchronisation cudaMalloc and
+ * cudaFree can cause.  zq_linear keeps a workspace per (device, stream) that
+ * it allocates on first use; this entry point instead uses one fixed 4 MiB
+ * device array compiled into the library, which every GPU that loads the
+ * library holds until the process exits.  (The pages describe no
+ * counterpart: this is a service of the library, not part of the method.)
+ *   Arguments and result: as zq_linear, with 1 <= M <= 8.
+ *   Limits: M > 8, or a call whose scratch (staged activations and split-K
+ *   partial sums) would exceed 4 MiB, returns ZQ_ERR_UNSUPPORTED.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   Every call shares the one array and clears its counters with an
+ *   asynchronous memset on `stream`: calls that overlap on the GPU (other
+ *   streams, other host threads) race and must be serialised by the caller.
+ *   Calls no cudaMalloc, cudaFree or allocating library routine.
+ *   Asynchronous. */
+ZQ_API zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed,
+                                   const uint16_t *scales, const uint16_t *zeros,
+                                   int bits, int group, int M, int N, int K,
+                                   uint16_t *out, zq_stream_t stream);
+
 /* One operation of a stack: the arguments of one zq_linear call. */
 typedef struct {
     const uint16_t *x;

@@ -25,7 +25,7 @@ ZQ_ERR_TIMEOUT = 5
 GROUP = 128
 
 # Every symbol the header declares (checked by the CPU test suite).
-EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_linear", "zq_linear_stack",
+EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_linear", "zq_linear_noalloc", "zq_linear_stack",
            "zq_unpack", "zq_reserve_workspace", "zq_linear_workspace_bytes",
            "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
            "zq_version")
@@ -45,6 +45,8 @@ _lib.zq_quantize_pack.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
 _lib.zq_quantize_pack.restype = _I
 _lib.zq_linear.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
 _lib.zq_linear.restype = _I
+_lib.zq_linear_noalloc.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
+_lib.zq_linear_noalloc.restype = _I
 _lib.zq_linear_stack.argtypes = [_P, _I, _P]
 _lib.zq_linear_stack.restype = _I
 _lib.zq_unpack.argtypes = [_P, _I, _I, _I, _P, _P]
@@ -138,6 +140,11 @@ def zq_quantize_pack(w, N, K, bits, group, packed, scales, zeros, stream=None):
 def zq_linear(x, packed, scales, zeros, bits, group, M, N, K, out, stream=None):
     _check(_lib.zq_linear(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), bits, group,
                           M, N, K, _ptr(out), _stream(stream, x)))
+
+
+def zq_linear_noalloc(x, packed, scales, zeros, bits, group, M, N, K, out, stream=None):
+    _check(_lib.zq_linear_noalloc(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), bits, group,
+                                  M, N, K, _ptr(out), _stream(stream, x)))
 
 
 def make_descs(ops):

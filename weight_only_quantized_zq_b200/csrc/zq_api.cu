@@ -175,7 +175,7 @@ struct PrepKey {
 // Plans and launches one decode launch over ops that share bits and MT and are
 // mutually independent.  With `dry_bytes` set, only computes the workspace size.
 zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, cudaStream_t stream,
-                     size_t *dry_bytes = nullptr) {
+                     size_t *dry_bytes = nullptr, uint8_t *fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
@@ -233,8 +233,13 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         *dry_bytes = off + kCounterBytes;
         return ZQ_OK;
     }
-    uint8_t *ws = nullptr;
-    if ((st = workspace(stream, off, &ws)) != ZQ_OK) return st;
+    uint8_t *ws = fixed_ws;
+    if (ws == nullptr) {
+        if ((st = workspace(stream, off, &ws)) != ZQ_OK) return st;
+    } else if (kCounterBytes + off > fixed_ws_bytes) {
+        return fail(ZQ_ERR_UNSUPPORTED, "call needs %zu bytes of scratch, the fixed scratch holds %zu",
+                    kCounterBytes + off, fixed_ws_bytes);
+    }
     uint8_t *data = ws + kCounterBytes;
 
     PrepParams pp;
@@ -391,6 +396,35 @@ zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t strea
     return ZQ_OK;
 }
 
+// ------------------------------------------------------ allocation-free path --
+// Scratch of zq_linear_noalloc: a fixed device array in this file, so that
+// call never allocates.  Every GPU that loads the library holds it until the
+// process exits.  Device code could name the array directly; host code needs
+// its device address, looked up once per device.
+
+constexpr size_t kNoallocScratchBytes = 4u << 20;  // 4 MiB
+constexpr int kNoallocMaxM = 8;
+static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
+
+std::mutex g_noalloc_mu;
+std::map<int, uint8_t *> g_noalloc_addr;
+
+zq_status noalloc_scratch(uint8_t **ptr) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    auto it = g_noalloc_addr.find(dev);
+    if (it == g_noalloc_addr.end()) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
+        it = g_noalloc_addr.emplace(dev, static_cast<uint8_t *>(p)).first;
+    }
+    *ptr = it->second;
+    return ZQ_OK;
+}
+
 }  // namespace
 
 // =================================================================== C ABI ==
@@ -431,6 +465,30 @@ zq_status zq_linear(const uint16_t *x, const uint32_t *packed, const uint16_t *s
     if (st != ZQ_OK) return st;
     std::vector<zq_linear_desc> one{d};
     return run_batch(one, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                            const uint16_t *zeros, int bits, int group, int M, int N, int K, uint16_t *out,
+                            zq_stream_t stream) {
+    zq_linear_desc d{x, packed, scales, zeros, out, bits, group, M, N, K};
+    zq_status st = check_linear(d);
+    if (st != ZQ_OK) return st;
+    if (M > kNoallocMaxM)
+        return fail(ZQ_ERR_UNSUPPORTED, "zq_linear_noalloc supports M <= %d (got M=%d)", kNoallocMaxM, M);
+    uint8_t *ws = nullptr;
+    if ((st = noalloc_scratch(&ws)) != ZQ_OK) return st;
+    std::vector<zq_linear_desc> one{d};
+    size_t need = 0;
+    if ((st = run_decode(one, bits, mt_for_m(M), nullptr, &need)) != ZQ_OK) return st;
+    if (need > kNoallocScratchBytes)
+        return fail(ZQ_ERR_UNSUPPORTED, "zq_linear_noalloc: this call needs %zu bytes of scratch, the limit is %zu",
+                    need, kNoallocScratchBytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // The split-K arrival counters must start at zero; the array keeps what the
+    // previous call left, so clear them (a memset, not an allocation).
+    cudaError_t e = cudaMemsetAsync(ws, 0, kCounterBytes, s);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch counters");
+    return run_decode(one, bits, mt_for_m(M), s, nullptr, ws, kNoallocScratchBytes);
 }
 
 zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream) {
