@@ -212,11 +212,28 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         total_steps += static_cast<long long>(rbs[i]) * su;
         max_m = std::max(max_m, ops[i].M);
     }
-    if (total_steps > 0x7FFFFFFFLL) return fail(ZQ_ERR_INVALID_ARG, "decode launch too large (steps)");
-    const long long want_ctas = std::max(1LL, (total_steps + kDecodeWarpsPerCta - 1) / kDecodeWarpsPerCta);
-    const int n_ctas = static_cast<int>(std::min(want_ctas, static_cast<long long>(occ) * info->sms));
-    const long long n_warps = static_cast<long long>(n_ctas) * kDecodeWarpsPerCta;
+    if (total_steps > 0x3FFFFFFFLL) return fail(ZQ_ERR_INVALID_ARG, "decode launch too large (steps)");
     const int slot_floats = rows * max_m;
+    // Chunking (see the decode kernel): with enough steps, about 12 chunks of
+    // at least 8 steps per warp, taken dynamically; otherwise one chunk per
+    // warp, every warp busy.
+    const long long wmax = static_cast<long long>(occ) * info->sms * kDecodeWarpsPerCta;
+    int log2c = 0, dynamic = 0, n_ctas = 0;
+    long long n_chunks = 0;
+    if (total_steps >= 16 * wmax) {
+        const long long per = total_steps / (12 * wmax);
+        log2c = 3;
+        while (log2c < 8 && (2LL << log2c) <= per) ++log2c;
+        while (((total_steps + (1LL << log2c) - 1) >> log2c) + 1 > static_cast<long long>(kMaxCounters)) ++log2c;
+        dynamic = 1;
+        n_ctas = static_cast<int>(static_cast<long long>(occ) * info->sms);
+    } else {
+        const long long per = (total_steps + wmax - 1) / wmax;
+        while ((1LL << log2c) < per) ++log2c;
+        n_ctas = static_cast<int>(((((total_steps + (1LL << log2c) - 1) >> log2c)) + kDecodeWarpsPerCta - 1) /
+                                  kDecodeWarpsPerCta);
+    }
+    n_chunks = (total_steps + (1LL << log2c) - 1) >> log2c;
 
     // Workspace layout.
     size_t off = 0;
@@ -227,8 +244,8 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         off += align256(static_cast<size_t>(mpad) * keys[e].K * 2) + align256(G * mpad * 8);
     }
     const size_t part_off = off;
-    off += align256(static_cast<size_t>(n_warps) * 2 * slot_floats * 4);
-    if (static_cast<size_t>(n_warps) > kMaxCounters) return fail(ZQ_ERR_INVALID_ARG, "internal: too many warps");
+    off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
+    if (static_cast<size_t>(n_chunks) + 1 > kMaxCounters) return fail(ZQ_ERR_INVALID_ARG, "internal: too many chunks");
     if (dry_bytes) {
         *dry_bytes = off + kCounterBytes;
         return ZQ_OK;
@@ -245,6 +262,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     PrepParams pp;
     std::memset(&pp, 0, sizeof(pp));
     pp.n_entries = static_cast<int>(keys.size());
+    pp.work = reinterpret_cast<unsigned int *>(ws);
     long long wsum = 0;
     for (size_t e = 0; e < keys.size(); ++e) {
         PrepEntry &en = pp.e[e];
@@ -268,6 +286,9 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     dp.part = reinterpret_cast<float *>(data + part_off);
     dp.cnt = reinterpret_cast<unsigned int *>(ws);
     dp.slot_floats = slot_floats;
+    dp.log2c = log2c;
+    dp.n_chunks = static_cast<int>(n_chunks);
+    dp.dynamic = dynamic;
     long long step0 = 0;
     for (size_t i = 0; i < ops.size(); ++i) {
         DecodeOp &o = dp.ops[i];

@@ -74,6 +74,7 @@ __device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow
 __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepParams p,
                                                    long long total_warps) {
     pdl_wait();  // x may be the output of the previous kernel in the stream
+    if (p.work != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.work = 0u;
     const long long gw = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (gw < total_warps) {
@@ -125,8 +126,13 @@ struct Cursor {
 __device__ __forceinline__ void cursor_init(Cursor &cu, const DecodeParams &p, int s, int s_end) {
     cu.s = s;
     cu.valid = s < s_end;
-    int o = 0;
-    while (o + 1 < p.n_ops && p.ops[o + 1].step0 <= s) ++o;
+    int lo = 0, hi = p.n_ops - 1;  // last op with step0 <= s
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.ops[mid].step0 <= s) lo = mid;
+        else hi = mid - 1;
+    }
+    const int o = lo;
     const int local = s - static_cast<int>(p.ops[o].step0);
     cu.o = o;
     cu.SU = p.ops[o].su;
@@ -248,35 +254,31 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     unsigned long long *bars =
         reinterpret_cast<unsigned long long *>(smem + kDecodeWarpsPerCta * D * STAGE) + warp * D;
 
-    // At most one warp per step, so every warp range is non-empty: a row block
-    // split over warps w_first..w_last gets a piece from each of them.
-    const long long T = p.total_steps;
-    const long long W = min(static_cast<long long>(gridDim.x) * kDecodeWarpsPerCta, T);
+    // Work is cut into chunks of C = 2^log2c consecutive steps.  Warp w starts
+    // with chunk w; in dynamic mode it then takes chunks W, W+1, ... from a
+    // counter (reset by the prep kernel), so faster SMs take more of them.  A
+    // row block cut by chunk boundaries is summed from per-chunk partial slots
+    // by the last piece to finish.
+    const int T = static_cast<int>(p.total_steps);
+    const int log2c = p.log2c;
+    const int nch = p.n_chunks;
+    const int W = gridDim.x * kDecodeWarpsPerCta;
     const int gw = blockIdx.x * kDecodeWarpsPerCta + warp;
-    const int s_begin = gw < W ? static_cast<int>(T * gw / W) : 0;
-    const int s_end = gw < W ? static_cast<int>(T * (gw + 1) / W) : 0;
 
     if (lane == 0)
         for (int i = 0; i < D; ++i) mbar_init(&bars[i], 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncwarp();
 
+    int cs_chunk = gw;  // chunk being computed
+    int cs_end = min((cs_chunk + 1) << log2c, T);
     Cursor cs;
-    cursor_init(cs, p, s_begin, s_end);
+    cursor_init(cs, p, gw < nch ? gw << log2c : T, gw < nch ? cs_end : 0);
     Cursor ld = cs;
-
-    // Row blocks cut by this warp's range (see warp_of); computed once, so the
-    // 64-bit division stays out of the loop.
-    int head_first = 0, head_last = 0, tail_last = 0;
-    if (cs.valid) {
-        const long long u0 = s_begin - cs.j;
-        head_first = warp_of(u0, W, T);
-        head_last = warp_of(u0 + cs.SU - 1, W, T);
-        Cursor lc;
-        cursor_init(lc, p, s_end - 1, s_end);
-        tail_last = warp_of(static_cast<long long>(s_end) - 1 - lc.j + lc.SU - 1, W, T);
-    }
-
+    int ld_end = cs_end;
+    int pend = -1;          // chunk taken by the loader, not yet reached by the consumer
+    bool need_take = false; // the loader ran out of its chunk
+    bool may_take = false;  // the counter may be read (after the PDL wait)
     // Loader: codes of 16 rows x GPS groups by one TMA (out-of-range rows and
     // groups read as zeros), then scales and zeros by one cp.async per lane.
     auto issue = [&](const Cursor &cu, int slot) {
@@ -300,6 +302,25 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
         }
     };
 
+    // Loader cursor: advance; at the end of its chunk take the next one
+    // (dynamic mode, once the counter may be read).
+    auto ld_advance = [&]() {
+        cursor_next(ld, p, ld_end);
+        if (!ld.valid && p.dynamic) need_take = true;
+    };
+    auto ld_take = [&]() {
+        if (!need_take || !may_take) return;
+        need_take = false;
+        int k = 0;
+        if (lane == 0) k = W + static_cast<int>(atomicAdd(p.cnt, 1u));
+        k = __shfl_sync(0xffffffffu, k, 0);
+        if (k < nch) {
+            pend = k;
+            ld_end = min((k + 1) << log2c, T);
+            cursor_init(ld, p, k << log2c, ld_end);
+        }
+    };
+
     // Prologue: weights do not depend on the previous kernel; start them now.
     int slot_ld = 0, slot_cs = 0;
     uint32_t par_cs = 0;          // parity of the next phase of slot_cs
@@ -308,7 +329,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     for (int i = 0; i < D - 1; ++i) {
         if (ld.valid) {
             issue(ld, slot_ld);
-            cursor_next(ld, p, s_end);
+            ld_advance();
             ++n_issued;
         }
         cp_async_commit();
@@ -316,6 +337,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
     }
     pdl_wait();  // the prepared activations come from the previous kernel
     pdl_launch_dependents();
+    may_take = true;
 
     float tot[MT][4];
 #pragma unroll
@@ -328,9 +350,10 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
 #pragma unroll 1
     while (cs.valid && !aborted) {
         __syncwarp();
+        ld_take();
         if (ld.valid) {
             issue(ld, slot_ld);
-            cursor_next(ld, p, s_end);
+            ld_advance();
             ++n_issued;
         }
         cp_async_commit();
@@ -496,11 +519,11 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
             });
         }
 
-        if (cs.j + 1 == cs.SU || cs.s + 1 == s_end) {
-            // End of this warp's piece of a row block: emit.
+        if (cs.j + 1 == cs.SU || cs.s + 1 == cs_end) {
+            // End of this chunk's piece of a row block: emit.
             const int unit_start = cs.s - cs.j;
-            const bool head = unit_start < s_begin;        // started in an earlier warp
-            const bool tail = unit_start + cs.SU > s_end;  // continues in a later warp
+            const bool head = unit_start < (cs_chunk << log2c);  // started in an earlier chunk
+            const bool tail = unit_start + cs.SU > cs_end;      // continues in a later chunk
             if (!head && !tail) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
@@ -513,8 +536,8 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
                                 __half_as_ushort(__float2half_rn(tot[mt][i]));
                     }
             } else {
-                // Partial piece: slot (w, 0) holds a head piece, (w, 1) a tail piece.
-                float *slot = p.part + (static_cast<size_t>(gw) * 2 + (head ? 0 : 1)) * p.slot_floats;
+                // Partial piece: slot (k, 0) holds chunk k's head piece, (k, 1) its tail piece.
+                float *slot = p.part + (static_cast<size_t>(cs_chunk) * 2 + (head ? 0 : 1)) * p.slot_floats;
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
@@ -523,12 +546,12 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
                         const int tok = 8 * mt + 2 * c + (i & 1);
                         if (tok < op.M) slot[row * op.M + tok] = tot[mt][i];
                     }
-                const int w_first = head ? head_first : gw;
-                const int w_last = head ? head_last : tail_last;
+                const int w_first = unit_start >> log2c;                 // chunks holding the
+                const int w_last = (unit_start + cs.SU - 1) >> log2c;    // pieces of this row block
                 __threadfence();
                 __syncwarp();
                 unsigned int prev = 0;
-                if (lane == 0) prev = atomicAdd(p.cnt + w_first, 1u);
+                if (lane == 0) prev = atomicAdd(p.cnt + 1 + w_first, 1u);
                 prev = __shfl_sync(0xffffffffu, prev, 0);
                 if (prev == static_cast<unsigned int>(w_last - w_first)) {
                     // Last piece in: sum the pieces in warp order (deterministic).
@@ -542,7 +565,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
                             op.out[static_cast<size_t>(tok) * op.N + r0 + row] =
                                 __half_as_ushort(__float2half_rn(sum));
                     }
-                    if (lane == 0) p.cnt[w_first] = 0u;  // ready for the next call
+                    if (lane == 0) p.cnt[1 + w_first] = 0u;  // ready for the next call
                 }
             }
 #pragma unroll
@@ -550,7 +573,19 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) tot[mt][i] = 0.0f;
         }
-        cursor_next(cs, p, s_end);
+        if (cs.s + 1 == cs_end) {
+            // chunk done: continue with the chunk the loader took, if any
+            if (pend >= 0) {
+                cs_chunk = pend;
+                pend = -1;
+                cs_end = min((cs_chunk + 1) << log2c, T);
+                cursor_init(cs, p, cs_chunk << log2c, cs_end);
+            } else {
+                cs.valid = false;
+            }
+        } else {
+            cursor_next(cs, p, cs_end);
+        }
     }
     // Copies still in flight (only after an abort) must land before the CTA
     // can exit: wait for every issued, unconsumed stage, bounded.

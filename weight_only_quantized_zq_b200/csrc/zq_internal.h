@@ -42,10 +42,14 @@ struct alignas(64) DecodeOp {
 
 struct DecodeParams {
     long long total_steps;
-    float *part;             // workspace: 2 partial slots per warp, slot_floats each
-    unsigned int *cnt;       // workspace: one arrival counter per warp (zero between calls)
+    float *part;             // workspace: 2 partial slots per chunk, slot_floats each
+    unsigned int *cnt;       // workspace: [0] work counter (reset by prep), [1 + k] arrival counter of chunk k
     int slot_floats;         // rows * max M
     int n_ops;
+    int log2c;               // chunk = 2^log2c consecutive steps
+    int n_chunks;
+    int dynamic;             // 1: chunks beyond the first per warp are taken from cnt[0]
+    int pad_;
     DecodeOp ops[kMaxDecodeOps];
 };
 static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
@@ -58,6 +62,7 @@ struct PrepEntry {
 };
 
 struct PrepParams {
+    unsigned int *work;  // decode work counter, reset to 0 (may be null)
     int n_entries;
     int pad_;
     long long warp_prefix[kMaxPrepEntries + 1];  // warps before entry i
