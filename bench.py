@@ -13,7 +13,10 @@ out) / device time, in GB/s; also % of 8 TB/s and tokens/s-equivalent
 (linear layers only: attention, norms, embeddings and lm_head excluded).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zq|reference]
-                    [--workload decode|prefill] [--m M]
+                    [--m M] [--layers L]
+
+M <= 64 runs the decode family (bandwidth-bound, reported against HBM);
+M > 64 the tcgen05 prefill family (reported against the tensor peak).
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on the host cores (rank 0 only).  With N > 1 (torchrun), each rank
@@ -38,6 +41,25 @@ if ROOT not in sys.path:
 import zq_inputs as zi  # noqa: E402
 
 METRIC = "quantized-linear HBM GB/s (% of 8 TB/s) at M=1; tokens/s-equiv per layer stack"
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
+# kernel, per layer of the stack, from one ncu capture of a 4-layer stack
+# (traffic grows in proportion to the layers).  Keyed by the SHA-256 of the
+# kernel's sources at capture time: once they change the figure is stale and
+# the roofline reports null.
+CSRC = os.path.join(ROOT, "weight_only_quantized_zq_b200", "csrc")
+KERNEL_SOURCES = {
+    "decode": ("zq_decode.cu", "zq_device.cuh", "zq_internal.h"),
+    "prefill": ("zq_prefill.cu", "zq_device.cuh", "zq_internal.h"),
+}
+MEASURED_TRAFFIC = {
+    # (family, M, bits): DRAM bytes per layer of the 7B-shaped stack
+    ("decode", 1, 4): {
+        "sha256": "71cdf3a0911cc03a3632afff5b85a72eef5a8d82ad8fba18ca14879fe383e208",
+        "bytes_per_layer": 125210240,
+        "profile": "profiles/decode_kernel_m1_4layers.md",
+    },
+}
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 
@@ -147,6 +169,24 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml"}
 
 
+def kernel_sha256(family):
+    import hashlib
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[family]:
+        with open(os.path.join(CSRC, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def measured_traffic(family, M, bits, layers):
+    """DRAM bytes per launch for this workload, or None when no capture of the
+    current kernel sources exists."""
+    rec = MEASURED_TRAFFIC.get((family, M, bits))
+    if rec is None or rec["sha256"] != kernel_sha256(family):
+        return None
+    return rec["bytes_per_layer"] * layers
+
+
 # --------------------------------------------------------------- workload --
 
 def op_bytes(M, N, K, bits):
@@ -190,6 +230,19 @@ class StackWorkload:
             self.flops += 2 * M * N * K
         self.descs, self.n_ops = zq.make_descs(self.ops)
         torch.cuda.synchronize()
+
+
+def workload_config(M, layers, world):
+    """The `config` object of the JSON line, shared by both arms."""
+    nbytes = sum(op_bytes(M, N, K, 4) for (_, _, _, N, K, _) in decode_stack_shapes(layers))
+    return {"workload": f"qwen2.5-7b-shaped {'decode' if M <= 64 else 'prefill'} stack: "
+                        f"{layers} layers x (qkv, o, gate_up, down), M={M}, INT4 g128, "
+                        f"one zq_linear_stack call",
+            "layers": layers, "M": M, "bits": 4, "group": 128,
+            "bytes_per_step": nbytes,
+            "flops_per_step": sum(2 * M * N * K for (_, _, _, N, K, _) in decode_stack_shapes(layers)),
+            "l2": f"inputs larger than L2 ({nbytes / 1e9:.2f} GB per step)",
+            "parallelism": f"replicas x{world}"}
 
 
 # ------------------------------------------------------------ oracle legs --
@@ -249,12 +302,13 @@ def run_reference(args):
     total = time.perf_counter() - t0
     value = nbytes / total / 1e9
     sample = (f"each step: oracle linear on every {int(round(1 / args.ref_frac))}th row of the 4 "
-              f"projections of one 7B-shaped INT4 layer at M={M} (fp64, OpenMP over rows)")
+              f"projections of one 7B-shaped INT4 layer at M={M} (fp64, OpenMP over rows); "
+              f"throughput in the same algorithmic-byte units as the GPU arm")
     line = {"metric": METRIC, "impl": "reference", "value": value, "unit": "GB/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"qwen2.5-7b-shaped decode stack, M={M}, INT4 g128 (sampled rows)"},
+            "config": workload_config(M, args.layers, args.gpus),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -322,13 +376,19 @@ def run_zq(args):
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
     if M <= 64:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                    "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                    "frac": achieved / peaks["hbm_gbs"],
+                    "traffic": measured_traffic("decode", M, 4, args.layers),
+                    "algorithmic_bytes": wl.bytes,
                     "peak_source": peaks["source"], "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel"}
     else:
         tflops = wl.flops / (ms_step / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
+        traffic = measured_traffic("prefill", M, 4, args.layers)
         roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
-                    "frac": tflops / peak, "traffic": None,
+                    "frac": tflops / peak,
+                    "traffic": None if traffic is None else traffic / (4 * args.layers),
+                    "traffic_note": "per launch, averaged over the 4 projections of a layer",
+                    "algorithmic_flops": wl.flops,
                     "peak_source": peaks["source"] + " (dense bf16 sustained; fp16 has the same dense rate)",
                     "kernel": "prefill_kernel<4>", "tflops_vs_nominal_2250": tflops / 2250.0}
 
@@ -345,13 +405,7 @@ def run_zq(args):
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f16 in, f32 accumulate, int4 weights", "data": "synthetic",
-                "config": {"workload": f"qwen2.5-7b-shaped {'decode' if M <= 64 else 'prefill'} stack: "
-                                       f"{args.layers} layers x (qkv, o, gate_up, down), M={M}, INT4 g128, "
-                                       f"one zq_linear_stack call",
-                           "layers": args.layers, "M": M, "bits": 4, "group": 128,
-                           "bytes_per_step": wl.bytes, "flops_per_step": wl.flops,
-                           "l2": f"inputs larger than L2 ({wl.bytes / 1e9:.2f} GB per step)",
-                           "parallelism": f"replicas x{world}"},
+                "config": workload_config(M, args.layers, world),
                 "pct_of_8tbs": 100 * achieved / NOMINAL_HBM_GBS,
                 "tokens_per_s_equiv": world * M / (ms_step / 1e3),
                 "roofline": roofline,

@@ -1,0 +1,73 @@
+"""Multi-process host logic of the replica bench, on CPU with gloo.
+
+The path has no exchange step ("replicas only"): ranks share nothing but the
+barrier and the max-over-ranks of their device times.  These tests run that
+plumbing with world_size 2 on the CPU.
+"""
+import io
+import contextlib
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _replica(rank, world, port, out_dir):
+    os.environ.update({"MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "WORLD_SIZE": str(world),
+                       "RANK": str(rank), "LOCAL_RANK": str(rank)})
+    sys.path.insert(0, ROOT)
+    import torch
+    import bench
+    w, r, _ = bench.dist_init("gloo")
+    assert (w, r) == (world, rank)
+    bench.barrier(w)
+    # each rank's "device time" differs; every rank must see the maximum
+    got = bench.max_over_ranks(10.0 * rank + 1.5, w)
+    bench.barrier(w)
+    torch.distributed.destroy_process_group()
+    with open(os.path.join(out_dir, f"rank{rank}.txt"), "w") as f:
+        f.write(repr(got))
+
+
+def test_max_over_ranks_gloo_world2(tmp_path):
+    world = 2
+    mp.start_processes(_replica, args=(world, _free_port(), str(tmp_path)), nprocs=world, join=True,
+                       start_method="spawn")
+    vals = [float(open(tmp_path / f"rank{r}.txt").read()) for r in range(world)]
+    assert vals == [11.5, 11.5]
+
+
+def test_single_rank_needs_no_process_group(monkeypatch):
+    for k in ("WORLD_SIZE", "RANK", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.dist_env() == (1, 0, 0)
+    assert bench.max_over_ranks(3.25, 1) == 3.25
+    bench.barrier(1)  # no-op without a process group
+
+
+def test_reference_arm_non_zero_rank_exits_without_work(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    sys.path.insert(0, ROOT)
+    import bench
+    called = []
+    monkeypatch.setattr(bench, "oracle_layer_sample", lambda *a, **k: called.append(1))
+    buf = io.StringIO()
+    with contextlib.redirect_stdout(buf):
+        rc = bench.main(["--impl", "reference", "--gpus", "2", "--steps", "1", "--warmup", "0"])
+    assert rc == 0
+    assert buf.getvalue() == ""
+    assert called == []

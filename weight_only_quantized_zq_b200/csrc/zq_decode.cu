@@ -198,14 +198,14 @@ __device__ __forceinline__ void load_scale_zero(uint32_t (&sz)[2][GPS], const De
 // One k16 step of a group: biased codes of pairs 2J, 2J+1 (rows gq, gq + 8)
 // times the activation pairs; J is a compile-time index so the unpack masks
 // are instruction immediates.
-template <int BITS, int J>
+template <int BITS, int J, bool INIT>
 __device__ __forceinline__ void mma_j(float (&acc)[4], const uint32_t (&w)[2][BITS], const uint32_t (&xf)[16],
                                       uint32_t magic) {
     const uint32_t a0 = unpack_biased_c<BITS, 2 * J>(w[0], magic);
     const uint32_t a1 = unpack_biased_c<BITS, 2 * J>(w[1], magic);
     const uint32_t a2 = unpack_biased_c<BITS, 2 * J + 1>(w[0], magic);
     const uint32_t a3 = unpack_biased_c<BITS, 2 * J + 1>(w[1], magic);
-    if constexpr (J == 0) {
+    if constexpr (INIT) {
         const float zero4[4] = {0.0f, 0.0f, 0.0f, 0.0f};
         mma_16816(acc, a0, a1, a2, a3, xf[2 * J], xf[2 * J + 1], zero4);
     } else {
@@ -213,17 +213,34 @@ __device__ __forceinline__ void mma_j(float (&acc)[4], const uint32_t (&w)[2][BI
     }
 }
 
-template <int BITS>
+// One group (16 rows x 128 k) into acc.  With SPLIT the even and odd k-steps
+// run as two independent accumulator chains, halving the dependent MMA
+// latency; worth its four registers only when few token tiles are live.
+template <int BITS, bool SPLIT>
 __device__ __forceinline__ void mma_group(float (&acc)[4], const uint32_t (&w)[2][BITS], const uint32_t (&xf)[16],
                                           uint32_t magic) {
-    mma_j<BITS, 0>(acc, w, xf, magic);
-    mma_j<BITS, 1>(acc, w, xf, magic);
-    mma_j<BITS, 2>(acc, w, xf, magic);
-    mma_j<BITS, 3>(acc, w, xf, magic);
-    mma_j<BITS, 4>(acc, w, xf, magic);
-    mma_j<BITS, 5>(acc, w, xf, magic);
-    mma_j<BITS, 6>(acc, w, xf, magic);
-    mma_j<BITS, 7>(acc, w, xf, magic);
+    if constexpr (SPLIT) {
+        float acc2[4];
+        mma_j<BITS, 0, true>(acc, w, xf, magic);
+        mma_j<BITS, 1, true>(acc2, w, xf, magic);
+        mma_j<BITS, 2, false>(acc, w, xf, magic);
+        mma_j<BITS, 3, false>(acc2, w, xf, magic);
+        mma_j<BITS, 4, false>(acc, w, xf, magic);
+        mma_j<BITS, 5, false>(acc2, w, xf, magic);
+        mma_j<BITS, 6, false>(acc, w, xf, magic);
+        mma_j<BITS, 7, false>(acc2, w, xf, magic);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[i] += acc2[i];
+    } else {
+        mma_j<BITS, 0, true>(acc, w, xf, magic);
+        mma_j<BITS, 1, false>(acc, w, xf, magic);
+        mma_j<BITS, 2, false>(acc, w, xf, magic);
+        mma_j<BITS, 3, false>(acc, w, xf, magic);
+        mma_j<BITS, 4, false>(acc, w, xf, magic);
+        mma_j<BITS, 5, false>(acc, w, xf, magic);
+        mma_j<BITS, 6, false>(acc, w, xf, magic);
+        mma_j<BITS, 7, false>(acc, w, xf, magic);
+    }
 }
 
 // Device record of a decode kernel that gave up a bounded wait (ZQ_ERR_TIMEOUT).
@@ -497,7 +514,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
                 const float4 sb = sbon[mt] ? *reinterpret_cast<const float4 *>(sbb[mt] + gi * 2 * MPAD)
                                            : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
                 float acc[4];
-                mma_group<BITS>(acc, wv, xf[gi & 1][mt], magic);
+                mma_group<BITS, MT == 1>(acc, wv, xf[gi & 1][mt], magic);
                 // tot += s * (acc - bias) + z * sum(x); with one token the odd
                 // C columns are padding.
 #pragma unroll
