@@ -12,6 +12,7 @@
 #include <map>
 #include <mutex>
 #include <string>
+#include <tuple>
 #include <utility>
 #include <vector>
 
@@ -77,7 +78,7 @@ zq_status check_linear(const zq_linear_desc &d) {
 
 struct DeviceInfo {
     int sms = 0;
-    int occ[9][9] = {};  // [bits][mt] decode CTAs per SM
+    std::map<std::tuple<int, int, size_t>, int> occ;  // (bits, mt, smem) -> decode CTAs per SM
 };
 std::mutex g_dev_mu;
 std::map<int, DeviceInfo> g_dev;
@@ -98,11 +99,11 @@ zq_status device_info(DeviceInfo **out) {
     return ZQ_OK;
 }
 
-zq_status decode_occupancy(DeviceInfo *info, int bits, int mt, int *ctas) {
+zq_status decode_occupancy(DeviceInfo *info, int bits, int mt, size_t smem, int *ctas) {
     std::lock_guard<std::mutex> lk(g_dev_mu);
-    int &o = info->occ[bits][mt];
+    int &o = info->occ[std::make_tuple(bits, mt, smem)];
     if (o == 0) {
-        cudaError_t e = decode_ctas_per_sm(bits, mt, &o);
+        cudaError_t e = decode_ctas_per_sm(bits, mt, smem, &o);
         if (e != cudaSuccess) return cuda_fail(e, "occupancy query");
         if (o <= 0) return fail(ZQ_ERR_CUDA, "decode kernel does not fit on an SM");
     }
@@ -172,6 +173,11 @@ struct PrepKey {
     bool operator==(const PrepKey &o) const { return x == o.x && M == o.M && K == o.K && bits == o.bits; }
 };
 
+// Shared memory of one decode CTA: `depth` stages, two mbarriers per stage,
+// the producer's scheduling state, and slack to align the ring to 1024 bytes.
+size_t decode_smem(int stage_bytes, int depth) { return static_cast<size_t>(depth) * (stage_bytes + 16) + 64 + 1024; }
+size_t align16(size_t b) { return (b + 15) & ~size_t(15); }
+
 // Plans and launches one decode launch over ops that share bits and MT and are
 // mutually independent.  With `dry_bytes` set, only computes the workspace size.
 zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, cudaStream_t stream,
@@ -179,10 +185,9 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
-    int occ = 0;
-    if ((st = decode_occupancy(info, bits, mt, &occ)) != ZQ_OK) return st;
-    const int rows = decode_rows(mt);
+    const int rows = kDecodeCtaRows;
     const int mpad = 8 * mt;
+    const int gps = decode_gps(bits, mt);
 
     // Prep entries (distinct activation buffers).
     std::vector<PrepKey> keys;
@@ -200,40 +205,80 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     if (keys.size() > static_cast<size_t>(kMaxPrepEntries) || ops.size() > static_cast<size_t>(kMaxDecodeOps))
         return fail(ZQ_ERR_INVALID_ARG, "internal: decode launch too large");
 
-    // Stream-K partition: every step (op, row block, group) costs the same
-    // within a launch (same bits), so warps get equal step counts.
-    long long total_steps = 0;
+    // Work: CTA steps (op, 64-row block, GPS groups), all of equal cost within
+    // a launch (same bits).
+    long long total_steps = 0, total_units = 0;
     int max_m = 1;
-    std::vector<int> rbs(ops.size());
-    const int gps = decode_gps(bits);
+    std::vector<int> rbs(ops.size()), sus(ops.size());
     for (size_t i = 0; i < ops.size(); ++i) {
         rbs[i] = (ops[i].N + rows - 1) / rows;
-        const int su = (ops[i].K / kGroup + gps - 1) / gps;
-        total_steps += static_cast<long long>(rbs[i]) * su;
+        sus[i] = (ops[i].K / kGroup + gps - 1) / gps;
+        total_steps += static_cast<long long>(rbs[i]) * sus[i];
+        total_units += rbs[i];
         max_m = std::max(max_m, ops[i].M);
     }
     if (total_steps > 0x3FFFFFFFLL) return fail(ZQ_ERR_INVALID_ARG, "decode launch too large (steps)");
-    const int slot_floats = rows * max_m;
-    // Chunking (see the decode kernel): with enough steps, about 12 chunks of
-    // at least 8 steps per warp, taken dynamically; otherwise one chunk per
-    // warp, every warp busy.
-    const long long wmax = static_cast<long long>(occ) * info->sms * kDecodeWarpsPerCta;
-    int log2c = 0, dynamic = 0, n_ctas = 0;
-    long long n_chunks = 0;
-    if (total_steps >= 16 * wmax) {
-        const long long per = total_steps / (12 * wmax);
-        log2c = 3;
-        while (log2c < 8 && (2LL << log2c) <= per) ++log2c;
-        while (((total_steps + (1LL << log2c) - 1) >> log2c) + 1 > static_cast<long long>(kMaxCounters)) ++log2c;
-        dynamic = 1;
-        n_ctas = static_cast<int>(static_cast<long long>(occ) * info->sms);
-    } else {
-        const long long per = (total_steps + wmax - 1) / wmax;
-        while ((1LL << log2c) < per) ++log2c;
-        n_ctas = static_cast<int>(((((total_steps + (1LL << log2c) - 1) >> log2c)) + kDecodeWarpsPerCta - 1) /
-                                  kDecodeWarpsPerCta);
+
+    // Stage: codes (64 rows x one step's bytes, a multiple of 1024; all
+    // stages' codes first, so each starts 1024-aligned), then a meta part of
+    // scales and zeros, group sums, activations and the step descriptor.
+    const int codes_bytes = rows * decode_seg(bits, mt);
+    const int off_sz = 0;
+    const int off_sx = off_sz + rows * 4 * gps;
+    const int off_x = off_sx + gps * mpad * 8;
+    const int x_rows_max = mt == 1 ? max_m : mpad;  // staged token rows
+    const int off_desc = off_x + gps * x_rows_max * 256;
+    const int meta_bytes = static_cast<int>(align16(off_desc + 32));
+    const int stage = codes_bytes + meta_bytes;
+    // Depth: at least 3 stages with as many CTAs per SM as the registers allow
+    // (228 KB of shared memory per SM, 1 KB of it reserved per CTA).
+    const int reg_ctas = mt == 1 ? 4 : mt == 2 ? 3 : 2;
+    int depth = 0, want_ctas = reg_ctas;
+    for (; want_ctas >= 1; --want_ctas) {
+        const long long budget = 228 * 1024 / want_ctas - 1024;
+        depth = static_cast<int>(std::min<long long>(6, (budget - 1024 - 64) / (stage + 16)));
+        if (depth >= 3) break;
     }
-    n_chunks = (total_steps + (1LL << log2c) - 1) >> log2c;
+    if (want_ctas < 1) {
+        want_ctas = 1;
+        depth = static_cast<int>(std::min<long long>(6, (227 * 1024 - 1024 - 64) / (stage + 16)));
+        if (depth < 2) return fail(ZQ_ERR_UNSUPPORTED, "decode stage of %d bytes does not fit", stage);
+    }
+    const size_t smem = decode_smem(stage, depth);
+    int occ = 0;
+    if ((st = decode_occupancy(info, bits, mt, smem, &occ)) != ZQ_OK) return st;
+    const long long max_ctas = static_cast<long long>(occ) * info->sms;
+
+    // Chunks.  Large launches: whole row blocks, taken dynamically, longest
+    // row blocks first (so the last ones handed out are short).  Otherwise
+    // chunks of 2^log2c steps: dynamic with at least 16 steps per CTA, else
+    // one chunk per CTA.
+    int log2c = 0, dynamic = 0, units = 0, n_ctas = 0;
+    long long n_chunks = 0;
+    std::vector<size_t> order(ops.size());
+    for (size_t i = 0; i < ops.size(); ++i) order[i] = i;
+    if (total_units >= 4 * max_ctas) {
+        units = 1;
+        dynamic = 1;
+        n_chunks = total_units;
+        n_ctas = static_cast<int>(max_ctas);
+        std::stable_sort(order.begin(), order.end(), [&](size_t a, size_t b) { return sus[a] > sus[b]; });
+    } else if (total_steps >= 16 * max_ctas) {
+        const long long per = total_steps / (12 * max_ctas);
+        log2c = 2;
+        while (log2c < 8 && (2LL << log2c) <= per) ++log2c;
+        dynamic = 1;
+        n_chunks = (total_steps + (1LL << log2c) - 1) >> log2c;
+        n_ctas = static_cast<int>(max_ctas);
+    } else {
+        const long long per = (total_steps + max_ctas - 1) / max_ctas;
+        while ((1LL << log2c) < per) ++log2c;
+        n_chunks = (total_steps + (1LL << log2c) - 1) >> log2c;
+        n_ctas = static_cast<int>(n_chunks);
+    }
+    if (!units && static_cast<size_t>(n_chunks) + 1 > kMaxCounters)
+        return fail(ZQ_ERR_INVALID_ARG, "internal: too many chunks");
+    const int slot_floats = rows * mpad;
 
     // Workspace layout.
     size_t off = 0;
@@ -241,11 +286,11 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     for (size_t e = 0; e < keys.size(); ++e) {
         prep_off[e] = off;
         const size_t G = keys[e].K / kGroup;
-        off += align256(static_cast<size_t>(mpad) * keys[e].K * 2) + align256(G * mpad * 8);
+        const size_t xr = mt == 1 ? keys[e].M : mpad;
+        off += align256(G * xr * kGroup * 2) + align256(G * mpad * 8);
     }
     const size_t part_off = off;
-    off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
-    if (static_cast<size_t>(n_chunks) + 1 > kMaxCounters) return fail(ZQ_ERR_INVALID_ARG, "internal: too many chunks");
+    if (!units) off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
     if (dry_bytes) {
         *dry_bytes = off + kCounterBytes;
         return ZQ_OK;
@@ -268,8 +313,9 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         PrepEntry &en = pp.e[e];
         const size_t G = keys[e].K / kGroup;
         en.x = keys[e].x;
-        en.xperm = reinterpret_cast<uint16_t *>(data + prep_off[e]);
-        en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(static_cast<size_t>(mpad) * keys[e].K * 2));
+        en.xg = reinterpret_cast<uint16_t *>(data + prep_off[e]);
+        en.x_rows = mt == 1 ? keys[e].M : mpad;
+        en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(G * en.x_rows * kGroup * 2));
         en.M = keys[e].M;
         en.M_pad = mpad;
         en.K = keys[e].K;
@@ -281,22 +327,31 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
 
     DecodeParams dp;
     std::memset(&dp, 0, sizeof(dp));
-    dp.n_ops = static_cast<int>(ops.size());
-    dp.total_steps = total_steps;
     dp.part = reinterpret_cast<float *>(data + part_off);
     dp.cnt = reinterpret_cast<unsigned int *>(ws);
+    dp.total_steps = static_cast<int>(total_steps);
+    dp.n_ops = static_cast<int>(ops.size());
     dp.slot_floats = slot_floats;
     dp.log2c = log2c;
     dp.n_chunks = static_cast<int>(n_chunks);
+    dp.units = units;
     dp.dynamic = dynamic;
-    long long step0 = 0;
-    for (size_t i = 0; i < ops.size(); ++i) {
-        DecodeOp &o = dp.ops[i];
+    dp.depth = depth;
+    dp.codes_bytes = codes_bytes;
+    dp.meta_bytes = meta_bytes;
+    dp.off_sz = off_sz;
+    dp.off_sx = off_sx;
+    dp.off_x = off_x;
+    dp.off_desc = off_desc;
+    const bool swz = decode_swizzled(bits, mt);
+    int step0 = 0, unit0 = 0;
+    for (size_t oi = 0; oi < ops.size(); ++oi) {
+        const size_t i = order[oi];
+        DecodeOp &o = dp.ops[oi];
         const PrepEntry &en = pp.e[op_entry[i]];
-        o.packed = ops[i].packed;
         o.scales = ops[i].scales;
         o.zeros = ops[i].zeros;
-        o.xperm = en.xperm;
+        o.xg = en.xg;
         o.sx = en.sx;
         o.out = ops[i].out;
         o.M = ops[i].M;
@@ -304,21 +359,24 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         o.K = ops[i].K;
         o.G = ops[i].K / kGroup;
         o.row_blocks = rbs[i];
-        o.su = (o.G + gps - 1) / gps;
+        o.su = sus[i];
         o.sz_vec = (o.G % gps) == 0 ? 1 : 0;
         const uint64_t row_bytes = static_cast<uint64_t>(o.K) * bits / 8;
-        cudaError_t te = encode_tensor_map_2d(&o.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, o.packed, row_bytes,
+        cudaError_t te = encode_tensor_map_2d(&o.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, ops[i].packed, row_bytes,
                                               static_cast<uint64_t>(o.N), row_bytes,
-                                              static_cast<uint32_t>(decode_seg(bits)), static_cast<uint32_t>(rows),
-                                              CU_TENSOR_MAP_SWIZZLE_NONE);
+                                              static_cast<uint32_t>(decode_box_w(bits, mt)),
+                                              static_cast<uint32_t>(rows),
+                                              swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
         if (te != cudaSuccess) return cuda_fail(te, "tensor map for the packed codes");
         o.step0 = step0;
-        step0 += static_cast<long long>(rbs[i]) * o.su;
+        o.unit0 = unit0;
+        step0 += rbs[i] * sus[i];
+        unit0 += rbs[i];
     }
 
     cudaError_t e = launch_prep(pp, wsum, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prep launch");
-    e = launch_decode(dp, bits, mt, n_ctas, stream);
+    e = launch_decode(dp, bits, mt, n_ctas, smem, stream);
     if (e != cudaSuccess) return cuda_fail(e, "decode launch");
     g_launches += 2;
     return ZQ_OK;

@@ -20,14 +20,19 @@
 //    2^-s (exact), so each product is 1024 * x' + q * x, and the per-group bias
 //    1024 * sum(x') is subtracted in fp32 once per group.  The canonical packed
 //    layout is consumed as stored.
-//  * Packed codes stream through a per-warp shared-memory ring with cp.async
-//    (16-byte chunks, several steps in flight, no register cost); the ring is
-//    per warp, so no block-level barrier is needed.
-//  * A persistent grid covers every SM.  The steps (op, row block, group) of
-//    all ops of a launch are cut into one contiguous range per warp (stream-K),
-//    so a whole stack of layers runs as one balanced launch and a small layer
-//    is split along K; a row block cut by a warp boundary is reduced by the
-//    last warp to finish it, in warp order, so results are deterministic.
+//  * A CTA step is 64 weight rows x GPS groups.  One ring of shared-memory
+//    stages per CTA: warp 0 produces (one TMA 2-D copy per 128-byte column of
+//    the codes, with the 128-byte swizzle so the fragment loads are free of
+//    bank conflicts; bulk copies of the step's activations and group sums;
+//    one cp.async per lane for scales and zeros) and all four warps consume,
+//    each 16 of the rows.  A step descriptor travels in the stage, so the
+//    consumers keep no scheduling state.
+//  * A persistent grid covers every SM.  The steps of all ops of a launch are
+//    cut into chunks: whole row blocks (large launches, longest first) or
+//    2^c consecutive steps (small launches, split along K).  A CTA starts with
+//    chunk blockIdx.x and takes further chunks from a counter.  A row block
+//    cut by a chunk boundary is reduced by the last warp to finish a piece of
+//    it, in chunk order, so results are deterministic.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -52,11 +57,17 @@ __device__ __forceinline__ void static_for(F &&f) {
 }
 
 // ------------------------------------------------------------------ prep --
-// One warp per (entry, padded token, group): writes the pair-permuted copy of
-// x and the fp32 group sum.  Tokens >= M are written as zeros.
+// One warp per (entry, padded token, group).  Tokens < M: the group's 128
+// activations, pair-permuted and 2^-s-scaled, into xg (M x K, row-major).
+// Lane c of the MMA reads 16-byte chunks 4c .. 4c+3 of its token's row; they
+// are stored at x_chunk(c, q, token & 7), so that the 8 lanes of a quarter
+// warp (two tokens x four lanes) always hit 8 different bank groups.  Every
+// padded token gets its (sum x, 1024 * sum x') pair (zeros past M).
+
+__host__ __device__ constexpr int x_chunk(int c, int q, int t7) { return (4 * c + (q ^ (2 * (c >> 1)))) ^ t7; }
 
 template <int B>
-__device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow, int lane) {
+__device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow, int lane, int t7) {
     float bias = 0.0f;  // sum of the scaled activations written by this lane
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -66,7 +77,8 @@ __device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow
         const __half lo = __float2half_rn(h2f_bits(xrow[32 * c + pair_lo<B>(p)]) * sc);
         const __half hi = __float2half_rn(h2f_bits(xrow[32 * c + pair_hi<B>(p)]) * sc);
         bias += __half2float(lo) + __half2float(hi);
-        reinterpret_cast<uint32_t *>(prow)[16 * c + p] = __half_as_ushort(lo) | (__half_as_ushort(hi) << 16);
+        const int word = (x_chunk(c, p >> 2, t7) << 2) | (p & 3);
+        reinterpret_cast<uint32_t *>(prow)[word] = __half_as_ushort(lo) | (__half_as_ushort(hi) << 16);
     }
     return bias;
 }
@@ -84,22 +96,24 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
         const long long local = gw - p.warp_prefix[e];
         const int G = en.K / kGroup;
         const int t = static_cast<int>(local / G), g = static_cast<int>(local % G);
-        uint16_t *prow = en.xperm + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
         float2 *dst = reinterpret_cast<float2 *>(en.sx) + static_cast<size_t>(g) * en.M_pad + t;
         if (t >= en.M) {
-            reinterpret_cast<uint2 *>(prow)[lane] = make_uint2(0u, 0u);
             if (lane == 0) *dst = make_float2(0.0f, 0.0f);
+            if (t < en.x_rows)
+                reinterpret_cast<uint2 *>(en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup)[lane] =
+                    make_uint2(0u, 0u);
         } else {
             const uint16_t *xrow = en.x + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
+            uint16_t *prow = en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             const uint2 v = reinterpret_cast<const uint2 *>(xrow)[lane];
             float s = h2f_bits(v.x & 0xFFFFu) + h2f_bits(v.x >> 16) + h2f_bits(v.y & 0xFFFFu) +
                       h2f_bits(v.y >> 16);
             float b;
             switch (en.bits) {
-                case 2: b = prep_group<2>(xrow, prow, lane); break;
-                case 3: b = prep_group<3>(xrow, prow, lane); break;
-                case 4: b = prep_group<4>(xrow, prow, lane); break;
-                default: b = prep_group<8>(xrow, prow, lane); break;
+                case 2: b = prep_group<2>(xrow, prow, lane, t & 7); break;
+                case 3: b = prep_group<3>(xrow, prow, lane, t & 7); break;
+                case 4: b = prep_group<4>(xrow, prow, lane, t & 7); break;
+                default: b = prep_group<8>(xrow, prow, lane, t & 7); break;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -119,7 +133,6 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
 struct Cursor {
     int s;         // step index
     int o, rb, j;  // op, row block, step within the row block
-    int SU, RB;    // steps per row block and row blocks of op o
     bool valid;
 };
 
@@ -133,67 +146,50 @@ __device__ __forceinline__ void cursor_init(Cursor &cu, const DecodeParams &p, i
         else hi = mid - 1;
     }
     const int o = lo;
-    const int local = s - static_cast<int>(p.ops[o].step0);
+    const int local = s - p.ops[o].step0;
     cu.o = o;
-    cu.SU = p.ops[o].su;
-    cu.RB = p.ops[o].row_blocks;
-    cu.rb = local / cu.SU;
-    cu.j = local - cu.rb * cu.SU;
+    cu.rb = local / p.ops[o].su;
+    cu.j = local - cu.rb * p.ops[o].su;
 }
 
 __device__ __forceinline__ void cursor_next(Cursor &cu, const DecodeParams &p, int s_end) {
     ++cu.s;
     cu.valid = cu.s < s_end;
-    if (++cu.j == cu.SU) {
+    if (++cu.j == p.ops[cu.o].su) {
         cu.j = 0;
-        if (++cu.rb == cu.RB) {
+        if (++cu.rb == p.ops[cu.o].row_blocks) {
             cu.rb = 0;
-            if (cu.o + 1 < p.n_ops) {
-                ++cu.o;
-                cu.SU = p.ops[cu.o].su;
-                cu.RB = p.ops[cu.o].row_blocks;
-            }
+            if (cu.o + 1 < p.n_ops) ++cu.o;
         }
     }
 }
 
-// Warp whose step range contains step s (ranges are [T*w/W, T*(w+1)/W)).
-__device__ __forceinline__ int warp_of(long long s, long long W, long long T) {
-    return static_cast<int>(((s + 1) * W - 1) / T);
-}
-
-// Scales and zeros of rows (gq, gq + 8) for the GPS groups of a step, packed as
-// fp16 pairs: sz[h][i] holds groups (2i, 2i+1) of row half h; [2 + ...] zeros.
-template <int GPS>
-__device__ __forceinline__ void load_scale_zero(uint32_t (&sz)[2][GPS], const DecodeOp &op, int r0, int g0,
-                                                int gq) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const int r = min(r0 + h * 8 + gq, op.N - 1);
-        const size_t idx = static_cast<size_t>(r) * op.G + g0;
-        if (((r * op.G + g0) % GPS) == 0 && g0 + GPS <= op.G) {
-            if constexpr (GPS == 4) {
-                const uint2 s2 = *reinterpret_cast<const uint2 *>(op.scales + idx);
-                const uint2 z2 = *reinterpret_cast<const uint2 *>(op.zeros + idx);
-                sz[h][0] = s2.x;
-                sz[h][1] = s2.y;
-                sz[h][2] = z2.x;
-                sz[h][3] = z2.y;
-            } else {
-                sz[h][0] = *reinterpret_cast<const uint32_t *>(op.scales + idx);
-                sz[h][1] = *reinterpret_cast<const uint32_t *>(op.zeros + idx);
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < GPS / 2; ++i) {
-                const int ga = min(g0 + 2 * i, op.G - 1), gb = min(g0 + 2 * i + 1, op.G - 1);
-                const size_t ia = static_cast<size_t>(r) * op.G + ga, ib = static_cast<size_t>(r) * op.G + gb;
-                sz[h][i] = ldg_u16_nc(op.scales + ia) | (ldg_u16_nc(op.scales + ib) << 16);
-                sz[h][GPS / 2 + i] = ldg_u16_nc(op.zeros + ia) | (ldg_u16_nc(op.zeros + ib) << 16);
-            }
+// Steps [begin, end) of chunk k: one whole row block, or 2^log2c steps.
+__device__ __forceinline__ void chunk_range(const DecodeParams &p, int k, int &begin, int &end) {
+    if (p.units) {
+        int lo = 0, hi = p.n_ops - 1;  // last op with unit0 <= k
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.ops[mid].unit0 <= k) lo = mid;
+            else hi = mid - 1;
         }
+        begin = p.ops[lo].step0 + (k - p.ops[lo].unit0) * p.ops[lo].su;
+        end = begin + p.ops[lo].su;
+    } else {
+        begin = k << p.log2c;
+        end = min(begin + (1 << p.log2c), p.total_steps);
     }
 }
+
+// Step descriptor, written by the producer into the stage (32 bytes).
+//   x: op, y: row block, z: step within the row block,
+//   w: number of groups | flags << 8;
+//   second int4: chunk, first step of the row block, M, unused.
+constexpr int kFlagLast = 1;   // last step of this chunk's piece of the row block: emit
+constexpr int kFlagHead = 2;   // the row block started in an earlier chunk
+constexpr int kFlagTail = 4;   // the row block continues in a later chunk
+constexpr int kFlagEnd = 8;    // no more work for this CTA
+constexpr int kFlagSzVec = 16; // scales and zeros are in the stage
 
 // One k16 step of a group: biased codes of pairs 2J, 2J+1 (rows gq, gq + 8)
 // times the activation pairs; J is a compile-time index so the unpack masks
@@ -248,113 +244,272 @@ __device__ int g_decode_error;
 
 constexpr unsigned long long kDecodeWaitNs = 2000000000ull;  // 2 s
 
-template <int BITS, int MT>
-__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
-    decode_kernel(const __grid_constant__ DecodeParams p) {
-    constexpr int ROWS = 16;
-    constexpr int GPS = decode_gps(BITS);
-    constexpr int GB = 16 * BITS;                 // bytes of one row of one group
-    constexpr int SEG = decode_seg(BITS);         // bytes of one row per step
-    constexpr int CODES = ROWS * SEG;             // TMA box bytes
-    constexpr int STAGE = decode_stage(BITS);
-    constexpr int D = decode_depth(BITS);
-    constexpr int MPAD = 8 * MT;
-    constexpr int SZB = 2 * GPS;                  // bytes of scales (or zeros) of one row per step
+// Bounded wait of the whole warp for a phase of `bar`; the answer is the same
+// in every lane (a lane that ran out makes the warp give up).
+__device__ __forceinline__ bool wait_phase(unsigned long long *bar, uint32_t parity) {
+    bool ok = mbar_try_wait(bar, parity);
+    if (!ok) {
+        const unsigned long long t0 = globaltimer();
+        while (!(ok = mbar_try_wait(bar, parity)))
+            if (globaltimer() - t0 > kDecodeWaitNs) break;
+    }
+    return __all_sync(0xffffffffu, ok);
+}
 
-    extern __shared__ __align__(128) uint8_t smem_raw[];
-    // TMA destinations: 128-byte aligned (the host adds 128 bytes of slack).
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+// Scheduling state of a CTA's producer, handed from one producing warp to
+// the next.
+struct ProdState {
+    int s, o, rb, j, valid;   // cursor of the next step to stage
+    int chunk, begin, end;    // its chunk and that chunk's steps
+    unsigned int ticket;      // counter value for the chunk after this one
+    int done;                 // the end marker has been staged
+    int seq;                  // stages filled so far
+};
+
+__device__ __forceinline__ void st_release_shared(int *a, int v) {
+    asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(smem_u32(a)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_shared(const int *a) {
+    int v;
+    asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(smem_u32(a)) : "memory");
+    return v;
+}
+
+// Bounded wait of the whole warp until *seq == target; it sleeps between
+// polls so that a waiting warp leaves the issue slots to the others.
+__device__ __forceinline__ bool wait_seq(const int *seq, int target) {
+    bool ok = ld_acquire_shared(seq) == target;
+    if (!ok) {
+        const unsigned long long t0 = globaltimer();
+        while (!(ok = ld_acquire_shared(seq) == target)) {
+            if (globaltimer() - t0 > kDecodeWaitNs) break;
+            __nanosleep(64);
+        }
+    }
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Box row (within its 8-row half) that MMA row g of a warp reads.  With the
+// 128-byte swizzle a 16-byte chunk of box row r sits at chunk ^ (r & 7); a
+// quarter warp covers MMA rows 2j and 2j+1, and this choice of box rows puts
+// its 8 fragment loads in 8 different bank groups.
+template <int BITS, int MT>
+__device__ __forceinline__ int box_row(int g) {
+    if constexpr (!decode_swizzled(BITS, MT) || BITS == 8) return g;  // b = 8: chunks 2c ^ g already differ
+    else if constexpr (BITS == 4) return (g >> 1) + 4 * (g & 1);       // rows 2j, 2j+1 -> j, j+4
+    else return 2 * (g & 3) + (g >> 2);                                // b = 2 (half-warp phases)
+}
+
+template <int BITS, int MT>
+__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : MT == 2 ? 3 : 2)
+    decode_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int GPS = decode_gps(BITS, MT);
+    constexpr int SEG = decode_seg(BITS, MT);       // bytes of one row per step
+    constexpr bool SWZ = decode_swizzled(BITS, MT);
+    constexpr int BOXW = decode_box_w(BITS, MT);
+    constexpr int NBOX = decode_boxes(BITS, MT);
+    constexpr int BOXB = BOXW * kDecodeCtaRows;     // bytes of one TMA box
+    constexpr int GB = 16 * BITS;                   // bytes of one row of one group
+    constexpr int MPAD = 8 * MT;
+    constexpr int SZB = 2 * GPS;                    // bytes of scales (or zeros) of one row per step
+
+    extern __shared__ uint8_t smem_raw[];
+    // Swizzled TMA destinations need 1024-byte alignment (the host adds slack).
+    uint8_t *ring = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int D = p.depth, CB = p.codes_bytes, MB = p.meta_bytes;
+    uint8_t *meta = ring + D * CB;  // per stage: scales/zeros, group sums, activations, descriptor
+    unsigned long long *full = reinterpret_cast<unsigned long long *>(meta + D * MB);
+    unsigned long long *empty = full + D;
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int gq = lane >> 2;  // MMA group id: row (A, C) / token (B)
     const int c = lane & 3;    // quad position: 32-code chunk (A, B) / token pair (C)
-    uint8_t *ring = smem + warp * D * STAGE;
-    unsigned long long *bars =
-        reinterpret_cast<unsigned long long *>(smem + kDecodeWarpsPerCta * D * STAGE) + warp * D;
-
-    // Work is cut into chunks of C = 2^log2c consecutive steps.  Warp w starts
-    // with chunk w; in dynamic mode it then takes chunks W, W+1, ... from a
-    // counter (reset by the prep kernel), so faster SMs take more of them.  A
-    // row block cut by chunk boundaries is summed from per-chunk partial slots
-    // by the last piece to finish.
-    const int T = static_cast<int>(p.total_steps);
-    const int log2c = p.log2c;
+    const int gr = box_row<BITS, MT>(gq);  // weight row (mod 8) of MMA row gq
     const int nch = p.n_chunks;
-    const int W = gridDim.x * kDecodeWarpsPerCta;
-    const int gw = blockIdx.x * kDecodeWarpsPerCta + warp;
 
-    if (lane == 0)
-        for (int i = 0; i < D; ++i) mbar_init(&bars[i], 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    __syncwarp();
-
-    int cs_chunk = gw;  // chunk being computed
-    int cs_end = min((cs_chunk + 1) << log2c, T);
-    Cursor cs;
-    cursor_init(cs, p, gw < nch ? gw << log2c : T, gw < nch ? cs_end : 0);
-    Cursor ld = cs;
-    int ld_end = cs_end;
-    int pend = -1;          // chunk taken by the loader, not yet reached by the consumer
-    bool need_take = false; // the loader ran out of its chunk
-    bool may_take = false;  // the counter may be read (after the PDL wait)
-    // Loader: codes of 16 rows x GPS groups by one TMA (out-of-range rows and
-    // groups read as zeros), then scales and zeros by one cp.async per lane.
-    auto issue = [&](const Cursor &cu, int slot) {
-        const DecodeOp &op = p.ops[cu.o];
-        const int g0 = cu.j * GPS;
-        const int r0 = cu.rb * ROWS;
-        uint8_t *st = ring + slot * STAGE;
-        if (lane == 0) {
-            fence_proxy_async();  // the warp's reads of this slot precede the overwrite
-            mbar_arrive_expect_tx(&bars[slot], CODES);
-            tma_load_2d(st, &op.tmap, g0 * GB, r0, &bars[slot]);
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < D; ++i) {
+            mbar_init(&full[i], 33);  // 32 cp.async arrivals + the producer's arrive(.expect_tx)
+            mbar_init(&empty[i], kDecodeWarpsPerCta);
         }
-        if (op.sz_vec) {
-            const int row = lane >> 1;
-            const int r = min(r0 + row, op.N - 1);
-            const uint16_t *src = ((lane & 1) ? op.zeros : op.scales) + static_cast<size_t>(r) * op.G + g0;
-            if constexpr (SZB == 8)
-                cp_async8(st + CODES + lane * 8, src);
-            else
-                cp_async4(st + CODES + lane * SZB, src);
-        }
-    };
-
-    // Loader cursor: advance; at the end of its chunk take the next one
-    // (dynamic mode, once the counter may be read).
-    auto ld_advance = [&]() {
-        cursor_next(ld, p, ld_end);
-        if (!ld.valid && p.dynamic) need_take = true;
-    };
-    auto ld_take = [&]() {
-        if (!need_take || !may_take) return;
-        need_take = false;
-        int k = 0;
-        if (lane == 0) k = W + static_cast<int>(atomicAdd(p.cnt, 1u));
-        k = __shfl_sync(0xffffffffu, k, 0);
-        if (k < nch) {
-            pend = k;
-            ld_end = min((k + 1) << log2c, T);
-            cursor_init(ld, p, k << log2c, ld_end);
-        }
-    };
-
-    // Prologue: weights do not depend on the previous kernel; start them now.
-    int slot_ld = 0, slot_cs = 0;
-    uint32_t par_cs = 0;          // parity of the next phase of slot_cs
-    int n_issued = 0, n_consumed = 0;
-#pragma unroll 1
-    for (int i = 0; i < D - 1; ++i) {
-        if (ld.valid) {
-            issue(ld, slot_ld);
-            ld_advance();
-            ++n_issued;
-        }
-        cp_async_commit();
-        slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    pdl_wait();  // the prepared activations come from the previous kernel
+    __syncthreads();
+
+    pdl_wait();  // the prepared activations and the counter come from the prep kernel
     pdl_launch_dependents();
-    may_take = true;
+
+    // ---- producer ----------------------------------------------------------
+    // Stage t is filled by warp t % 4, in order: the scheduling state (cursor
+    // and chunk) lives in shared memory and is handed from one producing warp
+    // to the next through `seq` (the number of stages filled so far).
+    ProdState *ps = reinterpret_cast<ProdState *>(empty + D);
+    if (threadIdx.x == 0) {
+        int b = 0, e = 0;
+        if (static_cast<int>(blockIdx.x) < nch) chunk_range(p, blockIdx.x, b, e);
+        Cursor cu;
+        cursor_init(cu, p, b, e);
+        ps->s = cu.s;
+        ps->o = cu.o;
+        ps->rb = cu.rb;
+        ps->j = cu.j;
+        ps->valid = cu.valid ? 1 : 0;
+        ps->chunk = blockIdx.x;
+        ps->begin = b;
+        ps->end = e;
+        ps->ticket = p.dynamic ? atomicAdd(p.cnt, 1u) : 0u;  // fetched one chunk ahead of its use
+        ps->done = 0;
+        ps->seq = 0;
+    }
+    __syncthreads();
+
+    // Fills stage `target` (after its previous contents were released by all
+    // warps); false if a wait ran out.  Whole warp, uniform control flow.
+    auto produce = [&](int target) -> bool {
+        if (!wait_seq(&ps->seq, target)) return false;
+        Cursor ld;
+        ld.s = ps->s;
+        ld.o = ps->o;
+        ld.rb = ps->rb;
+        ld.j = ps->j;
+        ld.valid = ps->valid != 0;
+        int ld_chunk = ps->chunk, ld_begin = ps->begin, ld_end = ps->end;
+        unsigned int ticket = ps->ticket;
+        if (ps->done) {
+            __syncwarp();
+            if (lane == 0) st_release_shared(&ps->seq, target + 1);
+            return true;
+        }
+        const int slot_ld = target % D, round_ld = target / D;
+        if (round_ld > 0 && !wait_phase(&empty[slot_ld], (round_ld - 1) & 1)) return false;
+        if (!ld.valid && p.dynamic) {
+            // Chunks only grow, so a CTA stops at its first ticket past the end
+            // and never holds an unused valid one.
+            const int k = static_cast<int>(gridDim.x + ticket);
+            if (k < nch) {
+                if (lane == 0) ticket = atomicAdd(p.cnt, 1u);
+                ld_chunk = k;
+                chunk_range(p, k, ld_begin, ld_end);
+                cursor_init(ld, p, ld_begin, ld_end);
+            }
+        }
+        uint8_t *st = ring + slot_ld * CB;
+        uint8_t *sm = meta + slot_ld * MB;
+        int4 *dsc = reinterpret_cast<int4 *>(sm + p.off_desc);
+        int done = 0;
+        if (ld.valid) {
+            const DecodeOp &op = p.ops[ld.o];
+            const int g0 = ld.j * GPS;
+            const int ng = min(GPS, op.G - g0);
+            const int xrows = MT == 1 ? op.M : MPAD;  // staged token rows
+            const int unit_start = ld.s - ld.j;
+            int flags = 0;
+            const int SU = op.su;
+            if (ld.j + 1 == SU || ld.s + 1 == ld_end) flags |= kFlagLast;
+            if (unit_start < ld_begin) flags |= kFlagHead;
+            if (unit_start + SU > ld_end) flags |= kFlagTail;
+            if (op.sz_vec) {
+                flags |= kFlagSzVec;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int r = lane + 32 * h;
+                    const int rg = min(ld.rb * kDecodeCtaRows + r, op.N - 1);
+                    const size_t src = static_cast<size_t>(rg) * op.G + g0;
+                    uint8_t *dst = sm + p.off_sz + r * 2 * SZB;
+                    if constexpr (SZB == 8) {
+                        cp_async8(dst, op.scales + src);
+                        cp_async8(dst + 8, op.zeros + src);
+                    } else {
+                        cp_async4(dst, op.scales + src);
+                        cp_async4(dst + 4, op.zeros + src);
+                    }
+                }
+            }
+            cp_async_arrive_noinc(&full[slot_ld]);
+            fence_proxy_async();  // earlier reads of this slot precede the async-proxy overwrite
+            if (lane == 0) {
+                dsc[0] = make_int4(ld.o, ld.rb, ld.j, ng | (flags << 8));
+                dsc[1] = make_int4(ld_chunk, unit_start, op.M, 0);
+                const uint32_t xbytes = static_cast<uint32_t>(ng * xrows * 256);
+                const uint32_t sbytes = static_cast<uint32_t>(ng * MPAD * 8);
+                mbar_arrive_expect_tx(&full[slot_ld], NBOX * BOXB + xbytes + sbytes);
+#pragma unroll
+                for (int b = 0; b < NBOX; ++b)
+                    tma_load_2d(st + b * BOXB, &op.tmap, g0 * GB + b * BOXW, ld.rb * kDecodeCtaRows, &full[slot_ld]);
+                bulk_load(sm + p.off_sx, op.sx + static_cast<size_t>(g0) * MPAD * 2, sbytes, &full[slot_ld]);
+            }
+            __syncwarp();
+            // Activations: token t's ng groups (ng * 256 contiguous bytes), one
+            // bulk copy per staged token, issued by lane t after the bytes were
+            // announced.
+            for (int t = lane; t < xrows; t += 32)
+                bulk_load(sm + p.off_x + t * (GPS * 256), op.xg + static_cast<size_t>(t) * op.K + g0 * kGroup,
+                          static_cast<uint32_t>(ng * 256), &full[slot_ld]);
+            cursor_next(ld, p, ld_end);
+        } else {
+            cp_async_arrive_noinc(&full[slot_ld]);
+            if (lane == 0) {
+                dsc[0] = make_int4(0, 0, 0, kFlagEnd << 8);
+                mbar_arrive(&full[slot_ld]);
+            }
+            done = 1;
+        }
+        __syncwarp();
+        if (lane == 0) {
+            ps->s = ld.s;
+            ps->o = ld.o;
+            ps->rb = ld.rb;
+            ps->j = ld.j;
+            ps->valid = ld.valid ? 1 : 0;
+            ps->chunk = ld_chunk;
+            ps->begin = ld_begin;
+            ps->end = ld_end;
+            ps->ticket = ticket;
+            ps->done = done;
+            st_release_shared(&ps->seq, target + 1);
+        }
+        return true;
+    };
+
+    bool aborted = false;
+    for (int t = warp; t < D - 1 && !aborted; t += kDecodeWarpsPerCta) aborted = !produce(t);
+
+    // ---- consumers (all warps) ---------------------------------------------
+    // Per-lane byte offsets into a stage, fixed for the whole kernel (shared
+    // memory is addressed with 32-bit offsets from the stage bases).
+    //   codes: the lane's chunk of group gi of row (warp*16 + h*8 + gr) at
+    //          cofs[h][k] + a compile-time part; with the 128-byte swizzle the
+    //          chunk index is ((gi*GB % 128)/16) ^ lanex.
+    //   x':    token gq's staged row is GPS*256 bytes, group gi at +gi*256,
+    //          the lane's chunk q of it at x_chunk(c, q, gq).
+    //   sums:  (sum x, bias) of tokens (8mt + 2c, +1) of group gi at
+    //          off_sx + (gi*MPAD + 8mt + 2c) * 8.
+    int lanex;
+    if constexpr (BITS == 4) lanex = c ^ gr;
+    else if constexpr (BITS == 2) lanex = (c >> 1) ^ gr;
+    else lanex = (2 * c) ^ gr;  // b = 8: chunks lanex and lanex ^ 1
+    uint32_t cofs[2][2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const uint32_t crow = (warp * 16 + h * 8 + gr) * (SWZ ? 128 : SEG);
+        if constexpr (!SWZ) {
+            cofs[h][0] = cofs[h][1] = crow + 4 * BITS * c;
+        } else if constexpr (BITS == 4) {
+            cofs[h][0] = crow + (lanex << 4);
+            cofs[h][1] = crow + ((lanex ^ 4) << 4);
+        } else if constexpr (BITS == 8) {
+            cofs[h][0] = crow + (lanex << 4);
+            cofs[h][1] = crow + ((lanex ^ 1) << 4);
+        } else {  // b = 2: group gi at chunk (2gi ^ lanex), half c & 1
+            cofs[h][0] = cofs[h][1] = crow + 8 * (c & 1);
+        }
+    }
+    uint32_t xq[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) xq[q] = p.off_x + gq * (GPS * 256) + (x_chunk(c, q, gq) << 4);
+    const uint32_t sxo = p.off_sx + 16 * c;
+    const uint32_t szq0 = p.off_sz + (warp * 16 + gr) * 2 * SZB, szq1 = p.off_sz + (warp * 16 + 8 + gr) * 2 * SZB;
+    const uint32_t ring_s = smem_u32(ring), meta_s = smem_u32(meta);
 
     float tot[MT][4];
 #pragma unroll
@@ -362,107 +517,59 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tot[b][i] = 0.0f;
     const uint32_t magic = kMagic;
-    bool aborted = false;
+    // B fragments (activations) of one token tile.  With one tile only the
+    // lanes of tokens < M load them; the rest keep stale values (their C
+    // columns are never stored), so the fragments live across steps.
+    uint32_t xf1[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) xf1[i] = 0u;
+    int slot = 0, n_seen = 0;  // stages this warp has waited for
+    uint32_t par = 0;
 
 #pragma unroll 1
-    while (cs.valid && !aborted) {
-        __syncwarp();
-        ld_take();
-        if (ld.valid) {
-            issue(ld, slot_ld);
-            ld_advance();
-            ++n_issued;
-        }
-        cp_async_commit();
-        slot_ld = slot_ld + 1 == D ? 0 : slot_ld + 1;
-
-        const DecodeOp &op = p.ops[cs.o];
-        const int r0 = cs.rb * ROWS;
-        const int g0 = cs.j * GPS;
-        const int ng = min(GPS, op.G - g0);
-
-        // Per-step bases of the activation fragments and group sums; the
-        // groups of the step are at immediate offsets from them.
-        const uint16_t *xb[MT];
-        const float *sbb[MT];
-        bool xon[MT], sbon[MT];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-            const int tok = 8 * mt + gq;
-            xon[mt] = tok < op.M;
-            sbon[mt] = 8 * mt + 2 * c < op.M;
-            xb[mt] = op.xperm + static_cast<size_t>(xon[mt] ? tok : 0) * op.K + static_cast<size_t>(g0) * kGroup + 32 * c;
-            sbb[mt] = op.sx + 2 * (static_cast<size_t>(g0) * MPAD + 8 * mt + 2 * c);
-        }
-        const bool one_token = op.M == 1;
-        // Activation fragments, ping-pong by group parity; group 0 is loaded
-        // before the waits, group gi + 1 while group gi computes.
-        uint32_t xf[2][MT][16];
-        auto load_x = [&](uint32_t (&dst)[MT][16], int gi) {
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                if (xon[mt]) {
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const uint4 w = ldg_u4(xb[mt] + gi * kGroup + 8 * q);
-                        dst[mt][4 * q + 0] = w.x;
-                        dst[mt][4 * q + 1] = w.y;
-                        dst[mt][4 * q + 2] = w.z;
-                        dst[mt][4 * q + 3] = w.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) dst[mt][q] = 0u;
-                }
-            }
-        };
-        load_x(xf[0], 0);
-
-        // Wait for this step's codes (TMA, bounded) and scales/zeros (cp.async).
+    while (!aborted) {
         {
-            bool ok = mbar_try_wait(&bars[slot_cs], par_cs);
-            if (!ok) {
-                const unsigned long long t0 = globaltimer();
-                while (!(ok = mbar_try_wait(&bars[slot_cs], par_cs)))
-                    if (globaltimer() - t0 > kDecodeWaitNs) break;
-            }
-            if (!ok) {
-                if (lane == 0) atomicExch(&g_decode_error, 5);  // ZQ_ERR_TIMEOUT
+            const int target = n_seen + D - 1;  // stage to fill now, by its warp
+            if (target % kDecodeWarpsPerCta == warp && !produce(target)) {
                 aborted = true;
                 break;
             }
         }
-        cp_async_wait<D - 1>();
-        __syncwarp();
-        const uint8_t *st = ring + slot_cs * STAGE;
-        ++n_consumed;
-        if (++slot_cs == D) {
-            slot_cs = 0;
-            par_cs ^= 1u;
+        if (!wait_phase(&full[slot], par)) {
+            aborted = true;
+            break;
         }
+        const uint32_t z = opaque_zero();  // orders the stage loads after the wait
+        const uint32_t stb = ring_s + slot * CB + z, smb = meta_s + slot * MB + z;
+        const uint4 d0 = lds_v4(smb + p.off_desc);
+        const uint4 d1 = lds_v4(smb + p.off_desc + 16);
+        const int flags = static_cast<int>(d0.w) >> 8;
+        ++n_seen;
+        if (flags & kFlagEnd) break;
+        const int ng = d0.w & 0xFF;
+        const int M = static_cast<int>(d1.z);
+        const int o = static_cast<int>(d0.x), rb = static_cast<int>(d0.y);
 
-        // Scales and zeros of rows gq and gq + 8 for the GPS groups.
+        // Scales and zeros of rows gr and gr + 8 for the GPS groups.
         uint32_t szs[2][GPS / 2], szz[2][GPS / 2];
-        if (op.sz_vec) {
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = h * 8 + gq;
-                if constexpr (GPS == 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(st + CODES + row * 16);
-                    szs[h][0] = v.x;
-                    szs[h][1] = v.y;
-                    szz[h][0] = v.z;
-                    szz[h][1] = v.w;
-                } else {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(st + CODES + row * 8);
-                    szs[h][0] = v.x;
-                    szz[h][0] = v.y;
-                }
+        if (flags & kFlagSzVec) {
+            if constexpr (GPS == 4) {
+                const uint4 v0 = lds_v4(smb + szq0);
+                const uint4 v1 = lds_v4(smb + szq1);
+                szs[0][0] = v0.x; szs[0][1] = v0.y; szz[0][0] = v0.z; szz[0][1] = v0.w;
+                szs[1][0] = v1.x; szs[1][1] = v1.y; szz[1][0] = v1.z; szz[1][1] = v1.w;
+            } else {
+                const uint2 v0 = lds_v2(smb + szq0);
+                const uint2 v1 = lds_v2(smb + szq1);
+                szs[0][0] = v0.x; szz[0][0] = v0.y;
+                szs[1][0] = v1.x; szz[1][0] = v1.y;
             }
         } else {
+            const DecodeOp &op = p.ops[o];
+            const int g0 = static_cast<int>(d0.z) * GPS;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const int r = min(r0 + h * 8 + gq, op.N - 1);
+                const int r = min(rb * kDecodeCtaRows + warp * 16 + h * 8 + gr, op.N - 1);
 #pragma unroll
                 for (int i = 0; i < GPS / 2; ++i) {
                     const int ga = min(g0 + 2 * i, op.G - 1), gb = min(g0 + 2 * i + 1, op.G - 1);
@@ -473,114 +580,140 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
             }
         }
 
-        auto group = [&](auto gi_c) {
+        auto group = [&](auto gi_c, auto one_c) {
             constexpr int gi = decltype(gi_c)::value;
-            // next group's activation fragments, one group ahead
-            if (gi + 1 < GPS) load_x(xf[(gi + 1) & 1], gi + 1);
-            // this thread's 32-code chunk of rows gq and gq + 8 (dense rows of SEG bytes)
+            constexpr bool one_token = decltype(one_c)::value;
+            // this thread's 32-code chunk of rows gr and gr + 8
             uint32_t wv[2][BITS];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                const uint8_t *rp = st + (h * 8 + gq) * SEG + gi * GB;
-                if constexpr (BITS == 2) {
-                    const uint2 v = *reinterpret_cast<const uint2 *>(rp + 8 * c);
-                    wv[h][0] = v.x;
-                    wv[h][1] = v.y;
-                } else if constexpr (BITS == 3) {
-                    const uint32_t *q = reinterpret_cast<const uint32_t *>(rp + 12 * c);
-                    wv[h][0] = q[0];
-                    wv[h][1] = q[1];
-                    wv[h][2] = q[2];
-                } else if constexpr (BITS == 4) {
-                    const uint4 v = *reinterpret_cast<const uint4 *>(rp + 16 * c);
+                if constexpr (SWZ && BITS == 4) {
+                    const uint4 v = lds_v4(stb + cofs[h][gi & 1] + (gi * GB / 128) * BOXB);
                     wv[h][0] = v.x;
                     wv[h][1] = v.y;
                     wv[h][2] = v.z;
                     wv[h][3] = v.w;
-                } else {
-                    const uint4 v0 = *reinterpret_cast<const uint4 *>(rp + 32 * c);
-                    const uint4 v1 = *reinterpret_cast<const uint4 *>(rp + 32 * c + 16);
+                } else if constexpr (SWZ && BITS == 8) {
+                    const uint4 v0 = lds_v4(stb + cofs[h][0] + gi * BOXB);
+                    const uint4 v1 = lds_v4(stb + cofs[h][1] + gi * BOXB);
                     wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
                     wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
+                } else if constexpr (SWZ) {
+                    static_assert(BITS == 2, "swizzled layouts: b = 2, 4, 8");
+                    const uint2 v = lds_v2(stb + cofs[h][0] + (((2 * gi) ^ lanex) << 4));
+                    wv[h][0] = v.x;
+                    wv[h][1] = v.y;
+                } else if constexpr (BITS == 2) {
+                    const uint2 v = lds_v2(stb + cofs[h][0] + gi * GB);
+                    wv[h][0] = v.x;
+                    wv[h][1] = v.y;
+                } else {
+                    static_assert(BITS == 3, "unswizzled layouts: b = 2 (2 groups per step), 3");
+                    wv[h][0] = lds_u32(stb + cofs[h][0] + gi * GB);
+                    wv[h][1] = lds_u32(stb + cofs[h][0] + gi * GB + 4);
+                    wv[h][2] = lds_u32(stb + cofs[h][0] + gi * GB + 8);
                 }
             }
-            constexpr int hi = gi & 1;
-            const float sc[2] = {h2f_bits(hi ? (szs[0][gi / 2] >> 16) : (szs[0][gi / 2] & 0xFFFFu)),
-                                 h2f_bits(hi ? (szs[1][gi / 2] >> 16) : (szs[1][gi / 2] & 0xFFFFu))};
-            const float zr[2] = {h2f_bits(hi ? (szz[0][gi / 2] >> 16) : (szz[0][gi / 2] & 0xFFFFu)),
-                                 h2f_bits(hi ? (szz[1][gi / 2] >> 16) : (szz[1][gi / 2] & 0xFFFFu))};
+            constexpr bool hi = (gi & 1) != 0;
+            const float sc[2] = {half_of<hi>(szs[0][gi / 2]), half_of<hi>(szs[1][gi / 2])};
+            const float zr[2] = {half_of<hi>(szz[0][gi / 2]), half_of<hi>(szz[1][gi / 2])};
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
-                const float4 sb = sbon[mt] ? *reinterpret_cast<const float4 *>(sbb[mt] + gi * 2 * MPAD)
-                                           : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                uint32_t xfm[16];
+                uint32_t (&xf)[16] = MT == 1 ? xf1 : xfm;
+                // Several tiles: all MPAD token rows are staged (zeros past M).
+                if (MT > 1 || gq < M) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const uint4 v = lds_v4(smb + xq[q] + (mt * 8 * GPS + gi) * 256);
+                        xf[4 * q + 0] = v.x;
+                        xf[4 * q + 1] = v.y;
+                        xf[4 * q + 2] = v.z;
+                        xf[4 * q + 3] = v.w;
+                    }
+                }
+                const uint4 sbv = lds_v4(smb + sxo + (gi * MPAD + 8 * mt) * 8);
+                const float4 sb = make_float4(__uint_as_float(sbv.x), __uint_as_float(sbv.y),
+                                              __uint_as_float(sbv.z), __uint_as_float(sbv.w));
                 float acc[4];
-                mma_group<BITS, MT == 1>(acc, wv, xf[gi & 1][mt], magic);
+                mma_group<BITS, MT == 1>(acc, wv, xf, magic);
                 // tot += s * (acc - bias) + z * sum(x); with one token the odd
                 // C columns are padding.
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     tot[mt][2 * h] = fmaf(sc[h], acc[2 * h] - sb.y, fmaf(zr[h], sb.x, tot[mt][2 * h]));
-                if (MT > 1 || !one_token) {
+                if constexpr (!one_token) {
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tot[mt][2 * h + 1] = fmaf(sc[h], acc[2 * h + 1] - sb.w, fmaf(zr[h], sb.z, tot[mt][2 * h + 1]));
                 }
             }
         };
-        if (ng == GPS) {
-            static_for<GPS>(group);
-        } else {
-            static_for<GPS>([&](auto gi_c) {
-                constexpr int gv = decltype(gi_c)::value;
-                if (gv < ng) group(gi_c);
-            });
+        auto groups = [&](auto one_c) {
+            if (ng == GPS) {
+                static_for<GPS>([&](auto gi_c) { group(gi_c, one_c); });
+            } else {
+                static_for<GPS>([&](auto gi_c) {
+                    constexpr int gv = decltype(gi_c)::value;
+                    if (gv < ng) group(gi_c, one_c);
+                });
+            }
+        };
+        if (MT == 1 && M == 1) groups(std::true_type{});
+        else groups(std::false_type{});
+
+        // Release the stage.
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[slot]);
+        if (++slot == D) {
+            slot = 0;
+            par ^= 1u;
         }
 
-        if (cs.j + 1 == cs.SU || cs.s + 1 == cs_end) {
+        if (flags & kFlagLast) {
             // End of this chunk's piece of a row block: emit.
-            const int unit_start = cs.s - cs.j;
-            const bool head = unit_start < (cs_chunk << log2c);  // started in an earlier chunk
-            const bool tail = unit_start + cs.SU > cs_end;      // continues in a later chunk
-            if (!head && !tail) {
+            const DecodeOp &op = p.ops[o];
+            const int r0 = rb * kDecodeCtaRows;
+            if (!(flags & (kFlagHead | kFlagTail))) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int row = r0 + (i >> 1) * 8 + gq;
+                        const int row = r0 + warp * 16 + (i >> 1) * 8 + gr;
                         const int tok = 8 * mt + 2 * c + (i & 1);
-                        if (row < op.N && tok < op.M)
+                        if (row < op.N && tok < M)
                             op.out[static_cast<size_t>(tok) * op.N + row] =
                                 __half_as_ushort(__float2half_rn(tot[mt][i]));
                     }
             } else {
                 // Partial piece: slot (k, 0) holds chunk k's head piece, (k, 1) its tail piece.
-                float *slot = p.part + (static_cast<size_t>(cs_chunk) * 2 + (head ? 0 : 1)) * p.slot_floats;
+                const int chunk = d1.x, unit_start = d1.y;
+                float *slot_p = p.part + (static_cast<size_t>(chunk) * 2 + ((flags & kFlagHead) ? 0 : 1)) * p.slot_floats;
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
-                        const int row = (i >> 1) * 8 + gq;
+                        const int rl = warp * 16 + (i >> 1) * 8 + gr;
                         const int tok = 8 * mt + 2 * c + (i & 1);
-                        if (tok < op.M) slot[row * op.M + tok] = tot[mt][i];
+                        if (tok < M) slot_p[rl * M + tok] = tot[mt][i];
                     }
-                const int w_first = unit_start >> log2c;                 // chunks holding the
-                const int w_last = (unit_start + cs.SU - 1) >> log2c;    // pieces of this row block
+                const int w_first = unit_start >> p.log2c;               // chunks holding the
+                const int w_last = (unit_start + op.su - 1) >> p.log2c;   // pieces of this row block
                 __threadfence();
                 __syncwarp();
                 unsigned int prev = 0;
                 if (lane == 0) prev = atomicAdd(p.cnt + 1 + w_first, 1u);
                 prev = __shfl_sync(0xffffffffu, prev, 0);
-                if (prev == static_cast<unsigned int>(w_last - w_first)) {
-                    // Last piece in: sum the pieces in warp order (deterministic).
+                if (prev == static_cast<unsigned int>(kDecodeWarpsPerCta * (w_last - w_first + 1) - 1)) {
+                    // Last piece in: sum the pieces in chunk order (deterministic).
                     __threadfence();
-                    for (int idx = lane; idx < ROWS * op.M; idx += 32) {
+                    for (int idx = lane; idx < kDecodeCtaRows * M; idx += 32) {
                         float sum = __ldcg(p.part + (static_cast<size_t>(w_first) * 2 + 1) * p.slot_floats + idx);
                         for (int ww = w_first + 1; ww <= w_last; ++ww)
                             sum += __ldcg(p.part + static_cast<size_t>(ww) * 2 * p.slot_floats + idx);
-                        const int row = idx / op.M, tok = idx - row * op.M;
+                        const int row = idx / M, tok = idx - row * M;
                         if (r0 + row < op.N)
-                            op.out[static_cast<size_t>(tok) * op.N + r0 + row] =
-                                __half_as_ushort(__float2half_rn(sum));
+                            op.out[static_cast<size_t>(tok) * op.N + r0 + row] = __half_as_ushort(__float2half_rn(sum));
                     }
                     if (lane == 0) p.cnt[1 + w_first] = 0u;  // ready for the next call
                 }
@@ -590,26 +723,18 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 2)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) tot[mt][i] = 0.0f;
         }
-        if (cs.s + 1 == cs_end) {
-            // chunk done: continue with the chunk the loader took, if any
-            if (pend >= 0) {
-                cs_chunk = pend;
-                pend = -1;
-                cs_end = min((cs_chunk + 1) << log2c, T);
-                cursor_init(cs, p, cs_chunk << log2c, cs_end);
-            } else {
-                cs.valid = false;
-            }
-        } else {
-            cursor_next(cs, p, cs_end);
-        }
     }
+
+    if (aborted && lane == 0) atomicExch(&g_decode_error, 5);  // ZQ_ERR_TIMEOUT
     // Copies still in flight (only after an abort) must land before the CTA
-    // can exit: wait for every issued, unconsumed stage, bounded.
-    cp_async_wait<0>();
-    for (int k = n_consumed; k < n_issued; ++k) {
-        const unsigned long long t0 = globaltimer();
-        while (!mbar_try_wait(&bars[k % D], (k / D) & 1u) && globaltimer() - t0 < kDecodeWaitNs) {
+    // can exit: every warp waits, bounded, for each stage filled so far that
+    // it did not wait for itself.
+    if (aborted) {
+        const int filled = ld_acquire_shared(&ps->seq);
+        for (int k = n_seen; k < filled; ++k) {
+            const unsigned long long t0 = globaltimer();
+            while (!mbar_try_wait(&full[k % D], (k / D) & 1u) && globaltimer() - t0 < kDecodeWaitNs) {
+            }
         }
     }
 }
@@ -636,17 +761,22 @@ cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t
     return cudaLaunchKernelEx(&cfg, prep_kernel, p, total_warps);
 }
 
+constexpr int kDecodeMaxSmem = 227 * 1024;
+
 template <int BITS, int MT>
-static cudaError_t launch_decode_t(const DecodeParams &p, int n_ctas, cudaStream_t stream) {
-    const size_t smem = decode_smem_bytes(BITS, MT);
+static cudaError_t set_smem_t() {
     static bool configured = false;  // benign race: the attribute call is idempotent
-    if (!configured) {
-        cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, MT>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
-        if (e != cudaSuccess) return e;
-        configured = true;
-    }
+    if (configured) return cudaSuccess;
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kDecodeMaxSmem);
+    if (e == cudaSuccess) configured = true;
+    return e;
+}
+
+template <int BITS, int MT>
+static cudaError_t launch_decode_t(const DecodeParams &p, int n_ctas, size_t smem, cudaStream_t stream) {
+    cudaError_t e = set_smem_t<BITS, MT>();
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
     cfg.blockDim = dim3(kDecodeWarpsPerCta * 32);
@@ -661,14 +791,11 @@ static cudaError_t launch_decode_t(const DecodeParams &p, int n_ctas, cudaStream
 }
 
 template <int BITS, int MT>
-static cudaError_t occupancy_t(int *ctas) {
-    const size_t smem = decode_smem_bytes(BITS, MT);
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, MT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+static cudaError_t occupancy_t(size_t smem, int *ctas) {
+    cudaError_t e = set_smem_t<BITS, MT>();
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, decode_kernel<BITS, MT>,
-                                                         kDecodeWarpsPerCta * 32, smem);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, decode_kernel<BITS, MT>, kDecodeWarpsPerCta * 32,
+                                                         smem);
 }
 
 #define ZQ_DISPATCH_BITS_MT(FN, ...)                                   \
@@ -692,10 +819,12 @@ static cudaError_t occupancy_t(int *ctas) {
         default: return cudaErrorInvalidValue;                         \
     }
 
-cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, cudaStream_t stream) {
-    ZQ_DISPATCH_BITS_MT(launch_decode_t, p, n_ctas, stream)
+cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream) {
+    ZQ_DISPATCH_BITS_MT(launch_decode_t, p, n_ctas, smem, stream)
 }
 
-cudaError_t decode_ctas_per_sm(int bits, int mt, int *ctas) { ZQ_DISPATCH_BITS_MT(occupancy_t, ctas) }
+cudaError_t decode_ctas_per_sm(int bits, int mt, size_t smem, int *ctas) {
+    ZQ_DISPATCH_BITS_MT(occupancy_t, smem, ctas)
+}
 
 }  // namespace zq

@@ -139,6 +139,49 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const void *map, int x, i
         : "memory");
 }
 
+// Shared-memory loads by 32-bit shared-window address.  They carry no memory
+// clobber, so the compiler schedules them freely; a caller that must order
+// them after a barrier wait adds opaque_zero() (taken after the wait) to the
+// address.
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+    uint4 v;
+    asm("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+    uint2 v;
+    asm("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t a) {
+    uint32_t v;
+    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+// A zero the compiler cannot see through, produced at this point of the
+// program order (volatile asm statements keep their relative order).
+__device__ __forceinline__ uint32_t opaque_zero() {
+    uint32_t z;
+    asm volatile("mov.u32 %0, 0;" : "=r"(z));
+    return z;
+}
+
+// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`.
+// Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, unsigned long long *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+// Arrive on `bar` once every cp.async this thread issued so far has landed;
+// the arrival counts toward the barrier's expected count.
+__device__ __forceinline__ void cp_async_arrive_noinc(unsigned long long *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Ampere-style asynchronous copy of 8 bytes (L1-allocating form; sizes 4/8).
 __device__ __forceinline__ void cp_async8(void *smem, const void *gmem) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
@@ -149,6 +192,13 @@ __device__ __forceinline__ void cp_async4(void *smem, const void *gmem) {
 
 __device__ __forceinline__ float h2f_bits(uint32_t h) {
     return __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
+}
+
+// fp16 in the low (HI = false) or high half of a 32-bit word, as float.
+template <bool HI>
+__device__ __forceinline__ float half_of(uint32_t w) {
+    const __half2 h = *reinterpret_cast<const __half2 *>(&w);
+    return HI ? __high2float(h) : __low2float(h);
 }
 
 // ------------------------------------------------------------ code unpack --

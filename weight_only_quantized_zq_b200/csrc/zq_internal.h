@@ -14,77 +14,82 @@ constexpr int kQuantStatusSlots = 64;
 
 // ---------------------------------------------------------------- decode --
 // A decode launch processes up to kMaxDecodeOps independent linear layers of
-// one bit width with M <= 64.  The work is a sequence of steps, one step =
-// (op, row block, 128-wide group); op o owns steps [step0, step0 + row_blocks*G)
-// in row-block-major order.  Warp w of W takes steps [T*w/W, T*(w+1)/W)
-// (stream-K): a row block cut by a warp boundary is summed from per-warp
-// partial slots by the last warp to finish it.
+// one bit width with M <= 64.  The work is a sequence of CTA steps, one step =
+// (op, 64-row block, GPS consecutive groups of 128); op o owns steps
+// [step0, step0 + row_blocks * su) in row-block-major order.  The steps are
+// cut into chunks (whole row blocks, or 2^log2c consecutive steps); a CTA
+// starts with chunk blockIdx.x and, in dynamic mode, takes further chunks from
+// a counter.  A row block cut by a chunk boundary is summed from per-chunk
+// partial slots by the last warp to finish a piece of it.
 
 constexpr int kMaxDecodeOps = 112;
 constexpr int kMaxPrepEntries = 64;
 constexpr int kDecodeWarpsPerCta = 4;
+constexpr int kDecodeCtaRows = 16 * kDecodeWarpsPerCta;  // weight rows per CTA step
 
 struct alignas(64) DecodeOp {
-    CUtensorMap tmap;       // packed codes as a 2-D uint8 tensor: box = 16 rows x one step's bytes
-    const uint32_t *packed;
+    CUtensorMap tmap;       // packed codes as a 2-D uint8 tensor: box = 64 rows x box_w bytes
     const uint16_t *scales;
     const uint16_t *zeros;
-    const uint16_t *xperm;  // workspace: M_pad x K fp16, pair-permuted, 2^-s-scaled activations
-    const float *sx;        // workspace: G x M_pad x 2 fp32 (sum x, bias) per group and token
+    const uint16_t *xg;     // workspace: (M, or M_pad with several token tiles) x K fp16, pair-permuted,
+                            // 2^-s-scaled, chunk-swizzled activations
+    const float *sx;        // workspace: G x M_pad x 2 fp32 (sum x, 1024 * sum x') per group and token
     uint16_t *out;          // M x N fp16
-    long long step0;        // first step of this op
+    int step0;              // first CTA step of this op
+    int unit0;              // first row block of this op (counted over the launch)
     int M, N, K, G;
-    int row_blocks;
+    int row_blocks;         // ceil(N / 64)
     int su;                 // steps per row block: ceil(G / GPS)
-    int sz_vec;             // G % GPS == 0: scales/zeros of a step are one aligned vector per row
-    int pad_;
+    int sz_vec;             // G % GPS == 0: a step's scales/zeros of one row are one aligned vector
 };
 
 struct DecodeParams {
-    long long total_steps;
     float *part;             // workspace: 2 partial slots per chunk, slot_floats each
-    unsigned int *cnt;       // workspace: [0] work counter (reset by prep), [1 + k] arrival counter of chunk k
-    int slot_floats;         // rows * max M
+    unsigned int *cnt;       // workspace: [0] chunk counter (reset by prep), [1 + k] pieces of chunk k's row block
+    int total_steps;
     int n_ops;
-    int log2c;               // chunk = 2^log2c consecutive steps
+    int slot_floats;         // 64 rows x M_pad
+    int log2c;               // fixed chunks: 2^log2c consecutive steps
     int n_chunks;
-    int dynamic;             // 1: chunks beyond the first per warp are taken from cnt[0]
-    int pad_;
+    int units;               // 1: a chunk is one whole row block
+    int dynamic;             // 1: chunks beyond the first per CTA are taken from cnt[0]
+    int depth;               // ring stages
+    int codes_bytes;         // codes of one stage (64 rows x one step's bytes), multiple of 1024
+    int meta_bytes;          // rest of one stage, multiple of 16
+    int off_sz, off_sx, off_x, off_desc;  // offsets inside a stage's meta part
     DecodeOp ops[kMaxDecodeOps];
 };
 static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
-    uint16_t *xperm;    // M_pad x K
+    uint16_t *xg;       // x_rows x K, chunk-swizzled per group and token; rows >= M are zeros
     float *sx;          // G x M_pad x 2: (sum of x, 1024 * sum of scaled x)
-    int M, M_pad, K, bits;
+    int M, M_pad, x_rows, K, bits;
 };
 
 struct PrepParams {
-    unsigned int *work;  // decode work counter, reset to 0 (may be null)
+    unsigned int *work;  // decode chunk counter, reset to 0 (may be null)
     int n_entries;
     int pad_;
     long long warp_prefix[kMaxPrepEntries + 1];  // warps before entry i
     PrepEntry e[kMaxPrepEntries];
 };
 
-// Decode tiling.  A warp step covers 16 weight rows x GPS groups (a 256-byte
-// row segment at 4 and 8 bits: longer DRAM bursts than one group per row).
-__host__ __device__ constexpr int decode_rows(int) { return 16; }
-__host__ __device__ constexpr int decode_gps(int bits) { return bits == 8 ? 2 : 4; }
-__host__ __device__ constexpr int decode_seg(int bits) { return decode_gps(bits) * 16 * bits; }
-// Per-warp ring stage: the step's codes (dense, written by TMA) followed by
-// the step's scales and zeros, 16 rows x {scales, zeros} x GPS halves.
-__host__ __device__ constexpr int decode_sz_bytes(int bits) { return 16 * 2 * decode_gps(bits) * 2; }
-__host__ __device__ constexpr int decode_stage(int bits) { return 16 * decode_seg(bits) + decode_sz_bytes(bits); }
-// Ring depth: about 13 KB per warp, at least 3 stages.
-__host__ __device__ constexpr int decode_depth(int bits) {
-    return 13312 / decode_stage(bits) < 3 ? 3 : 13312 / decode_stage(bits) > 6 ? 6 : 13312 / decode_stage(bits);
+// Decode tiling.  A CTA step covers 64 weight rows x GPS groups; each of the
+// 4 warps computes 16 of the rows.  Fewer groups per step with many tokens
+// keep the staged activations small.
+__host__ __device__ constexpr int decode_gps(int bits, int mt) { return (bits == 8 || mt >= 4) ? 2 : 4; }
+__host__ __device__ constexpr int decode_seg(int bits, int mt) { return decode_gps(bits, mt) * 16 * bits; }
+// Codes of a step land as 128-byte-wide TMA boxes with the 128-byte swizzle
+// when a row segment is a whole number of 128-byte spans; else as one
+// unswizzled box of the whole segment.
+__host__ __device__ constexpr bool decode_swizzled(int bits, int mt) { return decode_seg(bits, mt) % 128 == 0; }
+__host__ __device__ constexpr int decode_box_w(int bits, int mt) {
+    return decode_swizzled(bits, mt) ? 128 : decode_seg(bits, mt);
 }
-inline size_t decode_smem_bytes(int bits, int) {
-    return static_cast<size_t>(kDecodeWarpsPerCta) * (decode_depth(bits) * decode_stage(bits) + 8 * decode_depth(bits)) +
-           128;
+__host__ __device__ constexpr int decode_boxes(int bits, int mt) {
+    return decode_seg(bits, mt) / decode_box_w(bits, mt);
 }
 inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
 
@@ -108,7 +113,9 @@ cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, con
 constexpr int kDecodeMaxM = 64;
 
 cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, cudaStream_t stream);
-cudaError_t decode_ctas_per_sm(int bits, int mt, int *ctas);
+cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream);
+// CTAs per SM that the registers of decode_kernel<bits, mt> allow with `smem`
+// bytes of dynamic shared memory each.
+cudaError_t decode_ctas_per_sm(int bits, int mt, size_t smem, int *ctas);
 
 }  // namespace zq
