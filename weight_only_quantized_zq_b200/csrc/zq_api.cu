@@ -427,12 +427,36 @@ void split_tokens(const zq_linear_desc &d, std::vector<zq_linear_desc> &out) {
     }
 }
 
-zq_status run_prefill(const zq_linear_desc &d, cudaStream_t stream) {
+// One persistent launch over all tiles of independent prefill ops of one bit
+// width (at most kMaxPrefillOps), ops with the longest K first so that the
+// last tiles handed out are the cheap ones.
+zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
-    cudaError_t e = launch_prefill(d.x, d.packed, d.scales, d.zeros, d.bits, d.M, d.N, d.K, d.out, info->sms,
-                                   stream);
+    std::stable_sort(ops.begin(), ops.end(),
+                     [](const zq_linear_desc &a, const zq_linear_desc &b) { return a.K > b.K; });
+    PrefillGroup pg;
+    std::memset(&pg, 0, sizeof(pg));
+    pg.n_ops = static_cast<int>(ops.size());
+    int tiles = 0;
+    for (size_t i = 0; i < ops.size(); ++i) {
+        PrefillOp &o = pg.ops[i];
+        cudaError_t e = prefill_x_map(&o.xmap, ops[i].x, ops[i].M, ops[i].K);
+        if (e != cudaSuccess) return cuda_fail(e, "tensor map for x");
+        o.packed = ops[i].packed;
+        o.scales = ops[i].scales;
+        o.zeros = ops[i].zeros;
+        o.out = ops[i].out;
+        o.M = ops[i].M;
+        o.N = ops[i].N;
+        o.K = ops[i].K;
+        o.tok_tiles = (ops[i].M + 255) / 256;
+        o.tile0 = tiles;
+        tiles += prefill_tiles(ops[i].M, ops[i].N);
+    }
+    pg.n_tiles = tiles;
+    cudaError_t e = launch_prefill_group(pg, ops[0].bits, info->sms, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     g_launches += 1;
     return ZQ_OK;
@@ -442,15 +466,20 @@ zq_status run_prefill(const zq_linear_desc &d, cudaStream_t stream) {
 // class, each holding at most kMaxDecodeOps ops and kMaxPrepEntries inputs.
 zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t stream) {
     std::vector<zq_linear_desc> pieces;
-    for (const auto &d : batch) {
-        if (d.M > kDecodeMaxM) {
-            zq_status st = run_prefill(d, stream);
+    const int bits_list[4] = {2, 3, 4, 8};
+    for (int bits : bits_list) {
+        std::vector<zq_linear_desc> pre;
+        for (const auto &d : batch)
+            if (d.M > kDecodeMaxM && d.bits == bits) pre.push_back(d);
+        for (size_t i = 0; i < pre.size(); i += kMaxPrefillOps) {
+            std::vector<zq_linear_desc> launch(pre.begin() + i,
+                                               pre.begin() + std::min(pre.size(), i + kMaxPrefillOps));
+            zq_status st = run_prefill(launch, stream);
             if (st != ZQ_OK) return st;
-        } else {
-            pieces.push_back(d);
         }
     }
-    const int bits_list[4] = {2, 3, 4, 8};
+    for (const auto &d : batch)
+        if (d.M <= kDecodeMaxM) pieces.push_back(d);
     const int mt_list[4] = {1, 2, 4, 8};
     for (int bits : bits_list)
         for (int mt : mt_list) {

@@ -100,9 +100,32 @@ cudaError_t read_quant_status(int slot, unsigned long long *value, cudaStream_t 
 cudaError_t launch_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes,
                           cudaStream_t stream);
 
-cudaError_t launch_prefill(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
-                           const uint16_t *zeros, int bits, int M, int N, int K, uint16_t *out, int num_sms,
-                           cudaStream_t stream);
+// ---------------------------------------------------------------- prefill --
+// A prefill launch runs up to kMaxPrefillOps independent ops of one bit width
+// as one persistent grid over all their 256 x 256 output tiles.
+constexpr int kMaxPrefillOps = 64;
+
+struct alignas(64) PrefillOp {
+    CUtensorMap xmap;  // x (M x K fp16): 64 k x 256 tokens per box, 128-byte swizzle
+    const uint32_t *packed;
+    const uint16_t *scales;
+    const uint16_t *zeros;
+    uint16_t *out;
+    int M, N, K;
+    int tok_tiles;  // ceil(M / 256)
+    int tile0;      // first tile of this op in the launch
+};
+
+struct PrefillGroup {
+    int n_ops;
+    int n_tiles;
+    PrefillOp ops[kMaxPrefillOps];
+};
+static_assert(sizeof(PrefillGroup) <= 32000, "kernel parameter space");
+
+cudaError_t prefill_x_map(CUtensorMap *map, const uint16_t *x, int M, int K);
+int prefill_tiles(int M, int N);
+cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, cudaStream_t stream);
 cudaError_t read_prefill_error(int *err);
 cudaError_t read_decode_error(int *err);
 cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t dim0,

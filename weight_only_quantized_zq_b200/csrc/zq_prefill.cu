@@ -16,6 +16,9 @@
 //   warps 6-13 dequant producers: packed codes -> exact fp16 codes
 //              (zq_device.cuh) -> fp16(q*s + z) with one fused HFMA2 rounding ->
 //              K-order restored with PRMT -> UMMA K-major SWIZZLE_128B layout.
+// A launch is one persistent grid (a CTA per SM) over all tiles of up to 64
+// independent ops of one bit width, handed out round-robin in op order (the
+// host puts the longest K first).
 // A 3-stage ring of (x, W) slabs is handed over with mbarriers; stage release is
 // tcgen05.commit.  Every wait is bounded: after ~2 s it raises an abort flag,
 // records ZQ_ERR_TIMEOUT in a device word and all roles drain and exit (TMEM
@@ -137,11 +140,23 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     return *reinterpret_cast<const uint32_t *>(&h);
 }
 
-// Tile t -> (weight-row tile, token tile); token tiles vary fastest so the
-// CTAs working at the same time share one weight tile (L2 reuse).
-__device__ __forceinline__ void tile_coords(int t, int tok_tiles, int &n0, int &t0) {
-    n0 = (t / tok_tiles) * kRowTile;
-    t0 = (t % tok_tiles) * kTokTile;
+// Tile t of a launch -> (op, weight-row tile, token tile).  The tiles of op o
+// are [tile0, tile0 + tok_tiles * row_tiles); within an op token tiles vary
+// fastest, so the CTAs working at the same time share one weight tile (L2
+// reuse).
+struct TileRef {
+    int o, n0, t0;
+};
+__device__ __forceinline__ TileRef locate(const PrefillGroup &p, int t) {
+    int lo = 0, hi = p.n_ops - 1;  // last op with tile0 <= t
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.ops[mid].tile0 <= t) lo = mid;
+        else hi = mid - 1;
+    }
+    const int local = t - p.ops[lo].tile0;
+    const int tt = p.ops[lo].tok_tiles;
+    return TileRef{lo, (local / tt) * kRowTile, (local % tt) * kTokTile};
 }
 
 // Dequantize this thread's 32-code chunk of one W row into 4 x 16 bytes of
@@ -184,23 +199,14 @@ __device__ __forceinline__ void load_chunk(uint32_t (&w)[B], const uint32_t *src
     }
 }
 
-struct PrefillParams {
-    const uint32_t *packed;
-    const uint16_t *scales;
-    const uint16_t *zeros;
-    uint16_t *out;
-    int M, N, K;
-    int tok_tiles, row_tiles;
-};
 
 template <int B>
 __global__ void __launch_bounds__(kThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap xmap, const __grid_constant__ PrefillParams p) {
+    prefill_kernel(const __grid_constant__ PrefillGroup p) {
     extern __shared__ uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_tiles = p.tok_tiles * p.row_tiles;
-    const int slabs = p.K / kBK;
+    const int n_tiles = p.n_tiles;
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
@@ -229,17 +235,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == kTmaWarp) {
         if (lane == 0) {
-            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&xmap)) : "memory");
             uint32_t it = 0;
             for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
-                int n0, t0;
-                tile_coords(t, p.tok_tiles, n0, t0);
+                const TileRef tr = locate(p, t);
+                const PrefillOp &op = p.ops[tr.o];
+                const int slabs = op.K / kBK;
                 for (int s = 0; s < slabs; ++s, ++it) {
                     const int st = it % kStages;
                     const uint32_t round = it / kStages;
                     if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) break;
                     mbar_arrive_expect_tx(&sm.full[st], kSlabA);
-                    tma_load_2d(sm.a[st], &xmap, s * kBK, t0, &sm.full[st]);
+                    tma_load_2d(sm.a[st], &op.xmap, s * kBK, tr.t0, &sm.full[st]);
                 }
             }
             // Let copies still in flight land before the CTA can exit.
@@ -252,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t it = 0, tile_i = 0;
             for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
+                const int slabs = p.ops[locate(p, t).o].K / kBK;
                 if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 bool ok = true;
@@ -283,27 +290,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         // group (two slabs) are prefetched into registers.
         const int d = threadIdx.x - 32 * kDqWarp0;
         const int ch = d & 1;
-        const size_t wpr = static_cast<size_t>(p.K) * B / 32;
-        const int G = p.K / kGroup;
-        const int groups = slabs / 2;
         uint32_t it = 0;
         uint32_t wn[2][2][B], szn[2];  // [slab of group][row][word]
-        auto fetch = [&](int t, int g) {
-            int n0, t0;
-            tile_coords(t, p.tok_tiles, n0, t0);
+        // Row pointers of the tile being fetched (set when it starts).
+        const uint32_t *rowp[2];
+        const uint16_t *srow[2], *zrow[2];
+        auto start_tile = [&](int t) -> int {  // returns the tile's group count
+            const TileRef tr = locate(p, t);
+            const PrefillOp &op = p.ops[tr.o];
+            const int G = op.K / kGroup;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
-                const int r = min(n0 + d / 2 + 128 * i, p.N - 1);
-                const uint32_t *rowp = p.packed + static_cast<size_t>(r) * wpr;
+                const int r = min(tr.n0 + d / 2 + 128 * i, op.N - 1);
+                rowp[i] = op.packed + static_cast<size_t>(r) * (static_cast<size_t>(op.K) * B / 32);
+                srow[i] = op.scales + static_cast<size_t>(r) * G;
+                zrow[i] = op.zeros + static_cast<size_t>(r) * G;
+            }
+            return G;
+        };
+        auto fetch = [&](int g) {
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    load_chunk<B>(wn[h][i], rowp + static_cast<size_t>(4 * g + 2 * h + ch) * B);
-                const size_t si = static_cast<size_t>(r) * G + g;
-                szn[i] = ldg_u16_nc(p.scales + si) | (ldg_u16_nc(p.zeros + si) << 16);
+                    load_chunk<B>(wn[h][i], rowp[i] + static_cast<size_t>(4 * g + 2 * h + ch) * B);
+                szn[i] = ldg_u16_nc(srow[i] + g) | (ldg_u16_nc(zrow[i] + g) << 16);
             }
         };
-        int t = blockIdx.x, g = 0;
-        if (t < n_tiles) fetch(t, 0);
+        int t = blockIdx.x, g = 0, groups = 0, groups_n = 0;
+        if (t < n_tiles) {
+            groups = start_tile(t);
+            fetch(0);
+        }
         bool ok = true;
         while (t < n_tiles && ok && !*abort) {
             uint32_t wc[2][2][B], szc[2];
@@ -316,11 +334,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             szc[0] = szn[0];
             szc[1] = szn[1];
             int t_n = t, g_n = g + 1;
+            groups_n = groups;
             if (g_n == groups) {
                 g_n = 0;
                 t_n += gridDim.x;
+                if (t_n < n_tiles) groups_n = start_tile(t_n);
             }
-            if (t_n < n_tiles) fetch(t_n, g_n);
+            if (t_n < n_tiles) fetch(g_n);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // the two slabs of this group
                 const int st = it % kStages;
@@ -349,6 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             t = t_n;
             g = g_n;
+            groups = groups_n;
         }
     } else {
         // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = tokens of each half.
@@ -356,9 +377,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
             if (!mbar_wait(&sm.acc_full, tile_i & 1u, abort)) break;
             tc_fence_after();
-            int n0, t0;
-            tile_coords(t, p.tok_tiles, n0, t0);
-            const bool vec = (p.N % 8) == 0;
+            const TileRef tr = locate(p, t);
+            const PrefillOp &op = p.ops[tr.o];
+            const int n0 = tr.n0, t0 = tr.t0;
+            const bool vec = (op.N % 8) == 0;
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
                 const int tok = t0 + 128 * half + 32 * warp + lane;
@@ -367,9 +389,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t r[32];
                     tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile + cc * 32, r);
                     const int col0 = n0 + cc * 32;
-                    if (tok < p.M && col0 < p.N) {
-                        uint16_t *dst = p.out + static_cast<size_t>(tok) * p.N + col0;
-                        if (vec && col0 + 32 <= p.N) {
+                    if (tok < op.M && col0 < op.N) {
+                        uint16_t *dst = op.out + static_cast<size_t>(tok) * op.N + col0;
+                        if (vec && col0 + 32 <= op.N) {
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
                                 reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
@@ -380,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         } else {
 #pragma unroll
                             for (int q = 0; q < 32; ++q)
-                                if (col0 + q < p.N) dst[q] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
+                                if (col0 + q < op.N) dst[q] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
                         }
                     }
                 }
@@ -405,8 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ------------------------------------------------------------------ host --
 
 template <int B>
-static cudaError_t launch_prefill_t(const CUtensorMap &map, const pf::PrefillParams &pp, int n_ctas,
-                                    cudaStream_t stream) {
+static cudaError_t launch_prefill_t(const PrefillGroup &pg, int n_ctas, cudaStream_t stream) {
     cudaError_t e = cudaFuncSetAttribute(pf::prefill_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(pf::kSmemBytes));
     if (e != cudaSuccess) return e;
@@ -420,34 +441,26 @@ static cudaError_t launch_prefill_t(const CUtensorMap &map, const pf::PrefillPar
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B>, map, pp);
+    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B>, pg);
 }
 
-cudaError_t launch_prefill(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
-                           const uint16_t *zeros, int bits, int M, int N, int K, uint16_t *out, int num_sms,
-                           cudaStream_t stream) {
-    CUtensorMap map;
-    cudaError_t me = encode_tensor_map_2d(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
-                                          static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, pf::kBK,
-                                          pf::kTokTile, CU_TENSOR_MAP_SWIZZLE_128B);
-    if (me != cudaSuccess) return me;
-    pf::PrefillParams pp;
-    pp.packed = packed;
-    pp.scales = scales;
-    pp.zeros = zeros;
-    pp.out = out;
-    pp.M = M;
-    pp.N = N;
-    pp.K = K;
-    pp.tok_tiles = (M + pf::kTokTile - 1) / pf::kTokTile;
-    pp.row_tiles = (N + pf::kRowTile - 1) / pf::kRowTile;
-    const int tiles = pp.tok_tiles * pp.row_tiles;
-    const int n_ctas = tiles < num_sms ? tiles : num_sms;
+cudaError_t prefill_x_map(CUtensorMap *map, const uint16_t *x, int M, int K) {
+    return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
+                                static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, pf::kBK, pf::kTokTile,
+                                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+int prefill_tiles(int M, int N) {
+    return ((M + pf::kTokTile - 1) / pf::kTokTile) * ((N + pf::kRowTile - 1) / pf::kRowTile);
+}
+
+cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, cudaStream_t stream) {
+    const int n_ctas = pg.n_tiles < num_sms ? pg.n_tiles : num_sms;
     switch (bits) {
-        case 2: return launch_prefill_t<2>(map, pp, n_ctas, stream);
-        case 3: return launch_prefill_t<3>(map, pp, n_ctas, stream);
-        case 4: return launch_prefill_t<4>(map, pp, n_ctas, stream);
-        default: return launch_prefill_t<8>(map, pp, n_ctas, stream);
+        case 2: return launch_prefill_t<2>(pg, n_ctas, stream);
+        case 3: return launch_prefill_t<3>(pg, n_ctas, stream);
+        case 4: return launch_prefill_t<4>(pg, n_ctas, stream);
+        default: return launch_prefill_t<8>(pg, n_ctas, stream);
     }
 }
 
