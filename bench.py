@@ -55,8 +55,8 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, M, bits): DRAM bytes per layer of the 7B-shaped stack
     ("decode", 1, 4): {
-        "sha256": "048dfb2376b8dd5f5e9b4bda4b42f53b96213d1ba3f74d07d22b2397abc3f9bc",
-        "bytes_per_layer": 126717504,
+        "sha256": "49df590480ad52561438fcf96a49f9caba1e1792dafd0e363377fed3d6fc6f77",
+        "bytes_per_layer": 125690176,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },
 }
