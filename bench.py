@@ -15,8 +15,9 @@ out) / device time, in GB/s; also % of 8 TB/s and tokens/s-equivalent
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zq|reference]
                     [--m M] [--layers L]
 
-M <= 64 runs the decode family (bandwidth-bound, reported against HBM);
-M > 64 the tcgen05 prefill family (reported against the tensor peak).
+M <= 64 is decode (bandwidth-bound, reported against HBM; the library runs
+M <= 16 on its mma.sync decode kernel and larger M on its tcgen05 tile
+kernel); M > 64 is prefill (reported against the tensor peak).
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
 workload on the host cores (rank 0 only).  With N > 1 (torchrun), each rank
@@ -369,17 +370,18 @@ def run_zq(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_value = world * wl.bytes * args.steps / (e2e_ms / 1e3) / 1e9
 
-    # Roofline of the dominant kernel.  Decode (M <= 64): the grouped decode
-    # launch; the step is one prep launch + one decode launch, timed together
-    # by the events above, so the figure is a lower bound for the kernel.
-    # Prefill (M > 64): the tcgen05 kernels, one launch per projection.
+    # Roofline of the dominant kernel.  Decode (M <= 64): the grouped launch;
+    # with M <= 16 the step is one prep launch + one decode launch, timed
+    # together by the events above, so the figure is a lower bound for the
+    # kernel.  Prefill (M > 64): the grouped tcgen05 launches.
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
     if M <= 64:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
                     "traffic": measured_traffic("decode", M, 4, args.layers),
                     "algorithmic_bytes": wl.bytes,
-                    "peak_source": peaks["source"], "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel"}
+                    "peak_source": peaks["source"],
+                    "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel" if M <= 16 else "prefill_kernel<4>"}
     else:
         tflops = wl.flops / (ms_step / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
@@ -423,7 +425,7 @@ def run_zq(args):
 
 
 def zq_mt(M):
-    return 1 if M <= 8 else 2 if M <= 16 else 4 if M <= 32 else 8
+    return 1 if M <= 8 else 2
 
 
 def main(argv=None):

@@ -105,8 +105,10 @@ ZQ_API zq_status zq_quantize_pack(const float *w, int N, int K, int bits, int gr
 /* y = x · dequant(W)^T.
  *   x       device, fp16 M x K.      out  device, fp16 M x N (written).
  *   packed/scales/zeros as produced by zq_quantize_pack.
- * M <= 64 runs the decode family (tensor-core skinny GEMM streaming the
- * packed weights once); larger M runs the prefill family.  Asynchronous. */
+ * M <= 16 runs the decode kernel (mma.sync skinny GEMM streaming the packed
+ * weights once through a shared-memory ring); larger M runs the tcgen05 tile
+ * kernel (256 x 256 output tiles; with M <= 256 one token tile, so the
+ * weights are again streamed once).  Asynchronous. */
 ZQ_API zq_status zq_linear(const uint16_t *x, const uint32_t *packed,
                     const uint16_t *scales, const uint16_t *zeros,
                     int bits, int group, int M, int N, int K,
@@ -164,7 +166,7 @@ ZQ_API zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits,
  * Useful before graph capture.  Synchronous. */
 ZQ_API zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream);
 
-/* Workspace bytes zq_linear needs for these sizes (0 if none; M > 64 needs
+/* Workspace bytes zq_linear needs for these sizes (0 if none; M > 16 needs
  * none). */
 ZQ_API size_t zq_linear_workspace_bytes(int bits, int M, int N, int K);
 

@@ -111,7 +111,7 @@ def test_linear_shapes(zq, orc, bits):
 
 @pytest.mark.parametrize("bits", BITS)
 def test_prefill_shapes(zq, orc, bits):
-    """M > 64 runs the tcgen05 prefill family: ragged token tiles (TMA zero
+    """M > 16 runs the tcgen05 tile kernel: ragged token tiles (TMA zero
     fill), ragged weight-row tiles, N not a multiple of 8 (scalar stores)."""
     cases = [(65, 31, 256), (130, 70, 512), (256, 256, 128), (300, 520, 1024), (257, 264, 384),
              (512, 256, 3584), (1000, 1000, 640)]

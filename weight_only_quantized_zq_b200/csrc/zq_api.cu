@@ -232,7 +232,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     const int stage = codes_bytes + meta_bytes;
     // Depth: at least 3 stages with as many CTAs per SM as the registers allow
     // (228 KB of shared memory per SM, 1 KB of it reserved per CTA).
-    const int reg_ctas = mt == 1 ? 4 : mt == 2 ? 3 : 2;
+    const int reg_ctas = mt == 1 ? 4 : 3;
     int depth = 0, want_ctas = reg_ctas;
     for (; want_ctas >= 1; --want_ctas) {
         const long long budget = 228 * 1024 / want_ctas - 1024;
@@ -415,7 +415,7 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
     return overlap(a.out, b.out);
 }
 
-// Expands a linear op into decode-sized pieces (M <= 64 per piece); only used
+// Expands a linear op into decode-sized pieces (M <= 16 per piece); only used
 // for ops that the prefill family does not take.
 void split_tokens(const zq_linear_desc &d, std::vector<zq_linear_desc> &out) {
     for (int m0 = 0; m0 < d.M; m0 += kDecodeMaxM) {
@@ -480,7 +480,7 @@ zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t strea
     }
     for (const auto &d : batch)
         if (d.M <= kDecodeMaxM) pieces.push_back(d);
-    const int mt_list[4] = {1, 2, 4, 8};
+    const int mt_list[2] = {1, 2};
     for (int bits : bits_list)
         for (int mt : mt_list) {
             std::vector<zq_linear_desc> cls;
@@ -653,7 +653,7 @@ size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
     split_tokens(d, pieces);
     size_t worst = 0;
     // pieces of one op share bits; group them as run_batch would
-    for (int mt : {1, 2, 4, 8}) {
+    for (int mt : {1, 2}) {
         std::vector<zq_linear_desc> cls;
         for (const auto &p : pieces)
             if (mt_for_m(p.M) == mt) cls.push_back(p);

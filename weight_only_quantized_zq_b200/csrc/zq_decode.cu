@@ -1,5 +1,6 @@
-// zq_decode.cu — decode family (M <= 64): skinny tensor-core GEMM that streams
-// the packed weights exactly once.
+// zq_decode.cu — decode kernel (M <= 16): skinny tensor-core GEMM that streams
+// the packed weights exactly once.  (From 17 tokens on the tcgen05 tile kernel
+// of zq_prefill.cu, with a single token tile, streams them faster.)
 //
 // What it computes: y = x · dequant(W)^T with dequant(W) = q * scale + zero per
 // group of 128 along K ([wiki] "ZSE - open-source движок для запуска LLM
@@ -301,7 +302,7 @@ __device__ __forceinline__ int box_row(int g) {
 }
 
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : MT == 2 ? 3 : 2)
+__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
     decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int GPS = decode_gps(BITS, MT);
     constexpr int SEG = decode_seg(BITS, MT);       // bytes of one row per step
@@ -802,20 +803,12 @@ static cudaError_t occupancy_t(size_t smem, int *ctas) {
     switch (bits * 16 + mt) {                                          \
         case 2 * 16 + 1: return FN<2, 1>(__VA_ARGS__);                 \
         case 2 * 16 + 2: return FN<2, 2>(__VA_ARGS__);                 \
-        case 2 * 16 + 4: return FN<2, 4>(__VA_ARGS__);                 \
-        case 2 * 16 + 8: return FN<2, 8>(__VA_ARGS__);                 \
         case 3 * 16 + 1: return FN<3, 1>(__VA_ARGS__);                 \
         case 3 * 16 + 2: return FN<3, 2>(__VA_ARGS__);                 \
-        case 3 * 16 + 4: return FN<3, 4>(__VA_ARGS__);                 \
-        case 3 * 16 + 8: return FN<3, 8>(__VA_ARGS__);                 \
         case 4 * 16 + 1: return FN<4, 1>(__VA_ARGS__);                 \
         case 4 * 16 + 2: return FN<4, 2>(__VA_ARGS__);                 \
-        case 4 * 16 + 4: return FN<4, 4>(__VA_ARGS__);                 \
-        case 4 * 16 + 8: return FN<4, 8>(__VA_ARGS__);                 \
         case 8 * 16 + 1: return FN<8, 1>(__VA_ARGS__);                 \
         case 8 * 16 + 2: return FN<8, 2>(__VA_ARGS__);                 \
-        case 8 * 16 + 4: return FN<8, 4>(__VA_ARGS__);                 \
-        case 8 * 16 + 8: return FN<8, 8>(__VA_ARGS__);                 \
         default: return cudaErrorInvalidValue;                         \
     }
 

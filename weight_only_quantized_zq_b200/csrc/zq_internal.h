@@ -77,9 +77,8 @@ struct PrepParams {
 };
 
 // Decode tiling.  A CTA step covers 64 weight rows x GPS groups; each of the
-// 4 warps computes 16 of the rows.  Fewer groups per step with many tokens
-// keep the staged activations small.
-__host__ __device__ constexpr int decode_gps(int bits, int mt) { return (bits == 8 || mt >= 4) ? 2 : 4; }
+// 4 warps computes 16 of the rows.
+__host__ __device__ constexpr int decode_gps(int bits, int) { return bits == 8 ? 2 : 4; }
 __host__ __device__ constexpr int decode_seg(int bits, int mt) { return decode_gps(bits, mt) * 16 * bits; }
 // Codes of a step land as 128-byte-wide TMA boxes with the 128-byte swizzle
 // when a row segment is a whole number of 128-byte spans; else as one
@@ -91,7 +90,8 @@ __host__ __device__ constexpr int decode_box_w(int bits, int mt) {
 __host__ __device__ constexpr int decode_boxes(int bits, int mt) {
     return decode_seg(bits, mt) / decode_box_w(bits, mt);
 }
-inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : M <= 32 ? 4 : 8; }
+// Token tiles of 8 for the decode kernel (M <= kDecodeMaxM).
+inline int mt_for_m(int M) { return M <= 8 ? 1 : 2; }
 
 cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, uint32_t *packed,
                                  uint16_t *scales, uint16_t *zeros, int slot,
@@ -132,8 +132,10 @@ cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, con
                                  uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
                                  CUtensorMapSwizzle swizzle);
 
-// Largest M handled by the decode family; larger M goes to the prefill family.
-constexpr int kDecodeMaxM = 64;
+// Largest M handled by the mma.sync decode kernel; larger M goes to the
+// tcgen05 tile kernel (which, with one token tile, also streams the weights
+// once, and from 17 tokens on is the faster of the two).
+constexpr int kDecodeMaxM = 16;
 
 cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream);

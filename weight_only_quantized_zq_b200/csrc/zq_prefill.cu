@@ -1,4 +1,4 @@
-// zq_prefill.cu — prefill family (M > 64): dequantize-to-shared-memory GEMM on
+// zq_prefill.cu — tile kernel (M > 16): dequantize-to-shared-memory GEMM on
 // the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA).
 //
 // What it computes: out = x · dequant(W)^T with dequant(W) = q * scale + zero per
@@ -258,7 +258,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             uint32_t it = 0, tile_i = 0;
             for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
-                const int slabs = p.ops[locate(p, t).o].K / kBK;
+                const TileRef tr = locate(p, t);
+                const int slabs = p.ops[tr.o].K / kBK;
+                // the second 128-token half only when it holds tokens
+                const bool half1 = tr.t0 + 128 < p.ops[tr.o].M;
                 if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 bool ok = true;
@@ -271,12 +274,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sm.a[st]);
                     const uint32_t b0 = smem_u32(sm.b[st]);
+                    if (half1) {
 #pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t bd = sdesc_sw128(b0 + kk * 32);
-                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                        umma_f16(tmem, sdesc_sw128(a0 + kk * 32), bd, acc);
-                        umma_f16(tmem + kRowTile, sdesc_sw128(a0 + kSlabA / 2 + kk * 32), bd, acc);
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint64_t bd = sdesc_sw128(b0 + kk * 32);
+                            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                            umma_f16(tmem, sdesc_sw128(a0 + kk * 32), bd, acc);
+                            umma_f16(tmem + kRowTile, sdesc_sw128(a0 + kSlabA / 2 + kk * 32), bd, acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int kk = 0; kk < kBK / 16; ++kk) {
+                            const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                            umma_f16(tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(b0 + kk * 32), acc);
+                        }
                     }
                     umma_commit(&sm.empty[st]);
                 }
@@ -382,7 +393,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int n0 = tr.n0, t0 = tr.t0;
             const bool vec = (op.N % 8) == 0;
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
+            for (int half = 0; half < (t0 + 128 < op.M ? 2 : 1); ++half) {
                 const int tok = t0 + 128 * half + 32 * warp + lane;
 #pragma unroll 1
                 for (int cc = 0; cc < kRowTile / 32; ++cc) {
