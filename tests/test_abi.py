@@ -2,6 +2,7 @@
 header declares, and its host-side validation rejects bad arguments before any
 CUDA call (these calls never touch a GPU)."""
 import ctypes
+import glob
 import os
 import re
 import shutil
@@ -11,7 +12,7 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-HEADER = os.path.join(ROOT, "include", "zq.h")
+HEADERS = sorted(glob.glob(os.path.join(ROOT, "include", "*.h")))
 
 
 def _build_library():
@@ -31,7 +32,7 @@ def zq():
 
 
 def _declared_functions():
-    text = open(HEADER).read()
+    text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"\b(zq_[a-z_]+)\s*\(", text)))
 

@@ -1,7 +1,8 @@
 """Python binding of libzq, the B200 (sm_100a) weight-only quantized linear.
 
 Argument marshalling only: every step of the computation runs in the CUDA
-kernels behind the C ABI of ``include/zq.h``.  The functions carry the C names;
+kernels behind the C ABI of ``include/zq.h``; the .zse container reader and
+loader of ``include/zq_zse.h`` run in the library's native code.  The functions carry the C names;
 tensor arguments are torch CUDA tensors (their device pointers are passed), and
 ``stream`` defaults to torch's current stream on the tensor's device.
 
@@ -24,11 +25,13 @@ ZQ_ERR_CUDA = 4
 ZQ_ERR_TIMEOUT = 5
 GROUP = 128
 
-# Every symbol the header declares (checked by the CPU test suite).
+# Every symbol the headers declare (checked by the CPU test suite).
 EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_linear", "zq_linear_noalloc", "zq_linear_stack",
            "zq_unpack", "zq_reserve_workspace", "zq_linear_workspace_bytes",
            "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
-           "zq_version")
+           "zq_version",
+           "zq_zse_open", "zq_zse_close", "zq_zse_flags", "zq_zse_tensor_count", "zq_zse_tensor_info",
+           "zq_zse_find", "zq_zse_section", "zq_zse_weight_bytes", "zq_zse_verify", "zq_zse_load_weights")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -65,12 +68,41 @@ _lib.zq_kernel_launches.argtypes = []
 _lib.zq_kernel_launches.restype = ctypes.c_uint64
 _lib.zq_version.argtypes = []
 _lib.zq_version.restype = _I
+_U64 = ctypes.c_uint64
+_lib.zq_zse_open.argtypes = [ctypes.c_char_p, ctypes.POINTER(_P)]
+_lib.zq_zse_open.restype = _I
+_lib.zq_zse_close.argtypes = [_P]
+_lib.zq_zse_close.restype = None
+_lib.zq_zse_flags.argtypes = [_P]
+_lib.zq_zse_flags.restype = ctypes.c_uint32
+_lib.zq_zse_tensor_count.argtypes = [_P]
+_lib.zq_zse_tensor_count.restype = _I
+_lib.zq_zse_find.argtypes = [_P, ctypes.c_char_p]
+_lib.zq_zse_find.restype = _I
+_lib.zq_zse_section.argtypes = [_P, _I, ctypes.POINTER(_U64)]
+_lib.zq_zse_section.restype = _P
+_lib.zq_zse_weight_bytes.argtypes = [_P]
+_lib.zq_zse_weight_bytes.restype = _U64
+_lib.zq_zse_verify.argtypes = [_P]
+_lib.zq_zse_verify.restype = _I
+_lib.zq_zse_load_weights.argtypes = [_P, _P, _U64, _P]
+_lib.zq_zse_load_weights.restype = _I
 
 
 class ZQError(RuntimeError):
     def __init__(self, status, message):
         super().__init__(f"{zq_status_string(status)}: {message}")
         self.status = status
+
+
+class zq_zse_tensor(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char * 64), ("kind", _I), ("bits", _I), ("group", _I),
+                ("rows", _U64), ("cols", _U64), ("data_offset", _U64), ("data_bytes", _U64),
+                ("scales_offset", _U64), ("zeros_offset", _U64)]
+
+
+_lib.zq_zse_tensor_info.argtypes = [_P, _I, ctypes.POINTER(zq_zse_tensor)]
+_lib.zq_zse_tensor_info.restype = _I
 
 
 class zq_linear_desc(ctypes.Structure):
@@ -198,3 +230,64 @@ def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
         out = torch.empty(M, N, dtype=torch.float16, device=x.device)
     zq_linear(x, packed, scales, zeros, bits, GROUP, M, N, K, out, stream)
     return out
+
+
+# ------------------------------------------------------------ .zse reader --
+
+ZSE_CONFIG, ZSE_TOKENIZER, ZSE_WEIGHT_INDEX, ZSE_WEIGHT_DATA, ZSE_KERNELS = 1, 2, 3, 4, 5
+
+
+class ZseFile:
+    """An open .zse file (``zq_zse_open``); close() or use as a context manager."""
+
+    def __init__(self, path):
+        h = _P()
+        _check(_lib.zq_zse_open(os.fsencode(path), ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if self._h:
+            _lib.zq_zse_close(self._h)
+            self._h = None
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+
+    @property
+    def flags(self):
+        return _lib.zq_zse_flags(self._h)
+
+    @property
+    def weight_bytes(self):
+        return _lib.zq_zse_weight_bytes(self._h)
+
+    def tensors(self):
+        out = []
+        for i in range(_lib.zq_zse_tensor_count(self._h)):
+            t = zq_zse_tensor()
+            _check(_lib.zq_zse_tensor_info(self._h, i, ctypes.byref(t)))
+            out.append({"name": t.name.decode(), "kind": t.kind, "bits": t.bits, "group": t.group,
+                        "rows": t.rows, "cols": t.cols, "data_offset": t.data_offset,
+                        "data_bytes": t.data_bytes, "scales_offset": t.scales_offset,
+                        "zeros_offset": t.zeros_offset})
+        return out
+
+    def find(self, name):
+        return _lib.zq_zse_find(self._h, name.encode())
+
+    def section(self, kind):
+        """Bytes of a section (a copy), or None."""
+        n = _U64()
+        p = _lib.zq_zse_section(self._h, kind, ctypes.byref(n))
+        return None if not p else ctypes.string_at(p, n.value)
+
+    def verify(self):
+        _check(_lib.zq_zse_verify(self._h))
+
+    def load_weights(self, dst, stream=None):
+        """Copies WEIGHT_DATA into the uint8 CUDA tensor dst (synchronous)."""
+        _check(_lib.zq_zse_load_weights(self._h, _ptr(dst), dst.numel() * dst.element_size(),
+                                        _stream(stream, dst)))

@@ -703,3 +703,5 @@ zq_status zq_check_device(void) {
 int zq_version(void) { return 100; }
 
 }  // extern "C"
+
+void zq::set_last_error(const char *msg) { g_last_error = msg; }

@@ -10,6 +10,9 @@
 namespace zq {
 
 constexpr int kGroup = 128;
+
+// Records the message returned by zq_last_error() for the calling thread.
+void set_last_error(const char *msg);
 constexpr int kQuantStatusSlots = 64;
 
 // ---------------------------------------------------------------- decode --
