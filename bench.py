@@ -54,8 +54,8 @@ KERNEL_SOURCES = {
     "prefill": ("zq_prefill.cu", "zq_device.cuh", "zq_internal.h"),
 }
 MEASURED_TRAFFIC = {
-    # (family, M, bits): DRAM bytes per layer of the 7B-shaped stack
-    ("decode", 1, 4): {
+    # (family, model, M): DRAM bytes per layer of the stack
+    ("decode", "7b", 1): {
         "sha256": "49df590480ad52561438fcf96a49f9caba1e1792dafd0e363377fed3d6fc6f77",
         "bytes_per_layer": 125690176,
         "profile": "profiles/decode_kernel_m1_4layers.md",
@@ -179,10 +179,10 @@ def kernel_sha256(family):
     return h.hexdigest()
 
 
-def measured_traffic(family, M, bits, layers):
+def measured_traffic(family, model, M, layers):
     """DRAM bytes per launch for this workload, or None when no capture of the
     current kernel sources exists."""
-    rec = MEASURED_TRAFFIC.get((family, M, bits))
+    rec = MEASURED_TRAFFIC.get((family, model, M))
     if rec is None or rec["sha256"] != kernel_sha256(family):
         return None
     return rec["bytes_per_layer"] * layers
@@ -194,18 +194,29 @@ def op_bytes(M, N, K, bits):
     return N * K * bits // 8 + 4 * N * K // 128 + 2 * M * K + 2 * M * N
 
 
-def decode_stack_shapes(layers=zi.QWEN7B_LAYERS):
-    return [(layer, t, name, N, K, 4) for layer in range(layers)
-            for t, (name, N, K) in enumerate(zi.QWEN7B)]
+# Layer shapes per model: (name, N, K, bits); and the default layer count.
+MODELS = {
+    "7b": ([(name, N, K, 4) for (name, N, K) in zi.QWEN7B], zi.QWEN7B_LAYERS,
+           "qwen2.5-7b-shaped", "INT4 g128", "int4 weights"),
+    "32b-mixed": (list(zi.QWEN32B_MIXED), zi.QWEN32B_LAYERS, "qwen2.5-32b-shaped",
+                  "INT8 qkv / INT4 o / INT3 gate_up / INT2 down, g128, 0.1% outliers x20",
+                  "int8/int4/int3/int2 weights"),
+}
+
+
+def decode_stack_shapes(layers=zi.QWEN7B_LAYERS, model="7b"):
+    return [(layer, t, name, N, K, bits) for layer in range(layers)
+            for t, (name, N, K, bits) in enumerate(MODELS[model][0])]
 
 
 class StackWorkload:
     """All tensors of the decode stack resident on the GPU: one contiguous x
     buffer, one contiguous out buffer (views per op), packed weights per op."""
 
-    def __init__(self, zq, M, device, layers=zi.QWEN7B_LAYERS):
+    def __init__(self, zq, M, device, layers=zi.QWEN7B_LAYERS, model="7b"):
         self.M = M
-        shapes = decode_stack_shapes(layers)
+        shapes = decode_stack_shapes(layers, model)
+        outliers = model == "32b-mixed"
         ks = sorted({K for (_, _, _, _, K, _) in shapes})
         x_elems = sum(M * K for K in ks)
         self.x_all = torch.empty(x_elems, dtype=torch.float16, device=device)
@@ -220,7 +231,7 @@ class StackWorkload:
         self.ops, self.weights, self.bytes, self.flops = [], [], 0, 0
         ooff = 0
         for (layer, t, name, N, K, bits) in shapes:
-            w = zi.weight(N, K, zi.seed_for(layer, t), device=device)
+            w = zi.weight(N, K, zi.seed_for(layer, t), device=device, outliers=outliers)
             q = zq.quantize(w, bits)
             del w
             out = self.out_all[ooff:ooff + M * N].view(M, N)
@@ -233,39 +244,42 @@ class StackWorkload:
         torch.cuda.synchronize()
 
 
-def workload_config(M, layers, world):
+def workload_config(M, layers, world, model="7b"):
     """The `config` object of the JSON line, shared by both arms."""
-    nbytes = sum(op_bytes(M, N, K, 4) for (_, _, _, N, K, _) in decode_stack_shapes(layers))
-    return {"workload": f"qwen2.5-7b-shaped {'decode' if M <= 64 else 'prefill'} stack: "
-                        f"{layers} layers x (qkv, o, gate_up, down), M={M}, INT4 g128, "
+    shapes = decode_stack_shapes(layers, model)
+    nbytes = sum(op_bytes(M, N, K, b) for (_, _, _, N, K, b) in shapes)
+    _, _, shaped, fmt, _ = MODELS[model]
+    return {"workload": f"{shaped} {'decode' if M <= 64 else 'prefill'} stack: "
+                        f"{layers} layers x (qkv, o, gate_up, down), M={M}, {fmt}, "
                         f"one zq_linear_stack call",
-            "layers": layers, "M": M, "bits": 4, "group": 128,
+            "model": model, "layers": layers, "M": M,
+            "bits": sorted({b for (*_, b) in shapes}), "group": 128,
             "bytes_per_step": nbytes,
-            "flops_per_step": sum(2 * M * N * K for (_, _, _, N, K, _) in decode_stack_shapes(layers)),
+            "flops_per_step": sum(2 * M * N * K for (_, _, _, N, K, _) in shapes),
             "l2": f"inputs larger than L2 ({nbytes / 1e9:.2f} GB per step)",
             "parallelism": f"replicas x{world}"}
 
 
 # ------------------------------------------------------------ oracle legs --
 
-def oracle_layer_sample(M, seed_layer=0, frac=1.0, device_weights=None):
+def oracle_layer_sample(M, seed_layer=0, frac=1.0, device_weights=None, model="7b"):
     """Host inputs for the oracle: the 4 projections of one layer (rows sample).
     device_weights: list of (name, N, K, bits, (packed, scales, zeros)) on GPU
     to copy; else the layer is drawn on the CPU and quantized by the oracle."""
     import oracle as orc
     items = []
-    for t, (name, N, K) in enumerate(zi.QWEN7B):
+    for t, (name, N, K, bits) in enumerate(MODELS[model][0]):
         if device_weights is not None:
             q = device_weights[t][4]
             p = q[0].view(torch.int32).cpu().numpy().view(np.uint32).reshape(N, -1)
             s = q[1].cpu().numpy().view(np.uint16)
             z = q[2].cpu().numpy().view(np.uint16)
         else:
-            w = zi.weight(N, K, zi.seed_for(seed_layer, t)).numpy()
-            p, s, z = orc.quantize_pack(w, 4)
+            w = zi.weight(N, K, zi.seed_for(seed_layer, t), outliers=model == "32b-mixed").numpy()
+            p, s, z = orc.quantize_pack(w, bits)
         x = zi.activations(M, K, zi.seed_for(0, zi.X_SEED)).numpy().view(np.uint16)
         rows = np.arange(0, N, max(1, int(round(1 / frac))), dtype=np.int64)
-        items.append((x, p, s, z, N, K, rows))
+        items.append((x, p, s, z, N, K, bits, rows))
     return items
 
 
@@ -275,9 +289,9 @@ def time_oracle(items, M, budget_s=None):
     import oracle as orc
     done_bytes, t0 = 0, time.perf_counter()
     while True:
-        for (x, p, s, z, N, K, rows) in items:
-            orc.linear(x, p, s, z, 4, N, K, rows=rows)
-            done_bytes += op_bytes(M, len(rows), K, 4)
+        for (x, p, s, z, N, K, bits, rows) in items:
+            orc.linear(x, p, s, z, bits, N, K, rows=rows)
+            done_bytes += op_bytes(M, len(rows), K, bits)
         el = time.perf_counter() - t0
         if budget_s is None or el >= budget_s:
             break
@@ -291,7 +305,7 @@ def run_reference(args):
     if rank != 0:
         return 0
     M = args.m
-    items = oracle_layer_sample(M, frac=args.ref_frac)
+    items = oracle_layer_sample(M, frac=args.ref_frac, model=args.model)
     for _ in range(args.warmup):
         time_oracle(items, M)
     vals, secs, nbytes = [], 0.0, 0
@@ -309,7 +323,7 @@ def run_reference(args):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": total / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(M, args.layers, args.gpus),
+            "config": workload_config(M, args.layers, args.gpus, args.model),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -324,7 +338,7 @@ def run_zq(args):
     import weight_only_quantized_zq_b200 as zq
     peaks = load_peaks()
     M = args.m
-    wl = StackWorkload(zq, M, dev, args.layers)
+    wl = StackWorkload(zq, M, dev, args.layers, args.model)
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
@@ -375,30 +389,35 @@ def run_zq(args):
     # together by the events above, so the figure is a lower bound for the
     # kernel.  Prefill (M > 64): the grouped tcgen05 launches.
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
+    bits_used = sorted({b for (*_, b) in decode_stack_shapes(args.layers, args.model)}, reverse=True)
     if M <= 64:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": measured_traffic("decode", M, 4, args.layers),
+                    "traffic": measured_traffic("decode", args.model, M, args.layers),
                     "algorithmic_bytes": wl.bytes,
                     "peak_source": peaks["source"],
-                    "kernel": f"decode_kernel<4,{zq_mt(M)}> + prep_kernel" if M <= 16 else "prefill_kernel<4>"}
+                    "kernel": (f"decode_kernel<{'|'.join(str(b) for b in bits_used)},{zq_mt(M)}> + prep_kernel"
+                               + (" (one launch pair per bit width)" if len(bits_used) > 1 else "")
+                               if M <= 16 else "prefill_kernel<" + "|".join(str(b) for b in bits_used) + ">")}
     else:
         tflops = wl.flops / (ms_step / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
-        traffic = measured_traffic("prefill", M, 4, args.layers)
+        traffic = measured_traffic("prefill", args.model, M, args.layers)
         roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                     "frac": tflops / peak,
                     "traffic": None if traffic is None else traffic / (4 * args.layers),
                     "traffic_note": "per launch, averaged over the 4 projections of a layer",
                     "algorithmic_flops": wl.flops,
                     "peak_source": peaks["source"] + " (dense bf16 sustained; fp16 has the same dense rate)",
-                    "kernel": "prefill_kernel<4>", "tflops_vs_nominal_2250": tflops / 2250.0}
+                    "kernel": "prefill_kernel<" + "|".join(str(b) for b in bits_used) + ">",
+                    "tflops_vs_nominal_2250": tflops / 2250.0}
 
     line = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            items = oracle_layer_sample(M, device_weights=[w[1:] for w in wl.weights[:4]], frac=1.0)
+            items = oracle_layer_sample(M, device_weights=[w[1:] for w in wl.weights[:4]], frac=1.0,
+                                        model=args.model)
             v, el, b, threads = time_oracle(items, M, budget_s=args.cpu_seconds)
             cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
                    "sample": f"oracle linear (fp64, OpenMP over rows) on all 4 projections of layer 0 "
@@ -406,8 +425,8 @@ def run_zq(args):
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-                "dtype": "f16 in, f32 accumulate, int4 weights", "data": "synthetic",
-                "config": workload_config(M, args.layers, world),
+                "dtype": f"f16 in, f32 accumulate, {MODELS[args.model][4]}", "data": "synthetic",
+                "config": workload_config(M, args.layers, world, args.model),
                 "pct_of_8tbs": 100 * achieved / NOMINAL_HBM_GBS,
                 "tokens_per_s_equiv": world * M / (ms_step / 1e3),
                 "roofline": roofline,
@@ -435,11 +454,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("zq", "reference"), default="zq")
     ap.add_argument("--m", type=int, default=1, help="tokens per step (decode batch)")
-    ap.add_argument("--layers", type=int, default=zi.QWEN7B_LAYERS, help="layers in the stack")
+    ap.add_argument("--model", choices=sorted(MODELS), default="7b",
+                    help="layer shapes: the 7B INT4 stack (default) or the 32B mixed-precision stack")
+    ap.add_argument("--layers", type=int, default=None, help="layers in the stack (default: the model's)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-frac", type=float, default=0.25, help="row fraction per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
+    if args.layers is None:
+        args.layers = MODELS[args.model][1]
     if args.impl == "reference":
         return run_reference(args)
     return run_zq(args)

@@ -122,11 +122,12 @@ ZQ_API zq_status zq_zse_verify(const zq_zse *z);
 /* Copies WEIGHT_DATA into device memory `dst` (at least
  * zq_zse_weight_bytes bytes; a tensor's arrays then sit at dst + their
  * offsets, 256-byte aligned if dst is).  The section is streamed in 64 MB
- * chunks: host threads copy each chunk from the mapping into one of two
- * pinned buffers while the previous chunk is copied to the device on
- * `stream`.  Returns when the data is on the device (synchronous).
- * ZQ_ERR_INVALID_ARG if dst is NULL or too small, ZQ_ERR_CUDA on a CUDA
- * failure. */
+ * chunks: host threads read each chunk from the file into one of two pinned
+ * buffers while the previous chunk is copied to the device on `stream`.  The
+ * pinned buffers are allocated by the first call and kept with the handle.
+ * Returns when the data is on the device (synchronous).
+ * ZQ_ERR_INVALID_ARG if dst is NULL or too small or the file cannot be read,
+ * ZQ_ERR_CUDA on a CUDA failure. */
 ZQ_API zq_status zq_zse_load_weights(zq_zse *z, void *dst, uint64_t dst_bytes, zq_stream_t stream);
 
 #ifdef __cplusplus

@@ -88,8 +88,13 @@ def test_load_weights_in_chunks(tmp_path, zq):
         wb = f.weight_bytes
         dev = torch.empty(wb, dtype=torch.uint8, device="cuda")
         assert wb > 2 * (64 << 20)
-        t0 = time.perf_counter()
-        f.load_weights(dev)
-        dt = time.perf_counter() - t0
-    assert np.array_equal(dev.cpu().numpy(), np.frombuffer(parsed["payload"]["WEIGHT_DATA"], np.uint8))
-    print(f"zse load: {wb / dt / 1e9:.2f} GB/s ({wb / 1e6:.0f} MB)")
+        times = []
+        for _ in range(2):  # the first call also allocates the pinned staging buffers
+            dev.zero_()
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            f.load_weights(dev)
+            times.append(time.perf_counter() - t0)
+            assert np.array_equal(dev.cpu().numpy(), np.frombuffer(parsed["payload"]["WEIGHT_DATA"], np.uint8))
+    print(f"zse load: first {wb / times[0] / 1e9:.2f} GB/s, again {wb / times[1] / 1e9:.2f} GB/s "
+          f"({wb / 1e6:.0f} MB)")

@@ -341,27 +341,49 @@ zq_status zq_zse_load_weights(zq_zse *z, void *dst, uint64_t dst_bytes, zq_strea
         zq::set_last_error((std::string("staging buffers: ") + cudaGetErrorString(e)).c_str());
         return ZQ_ERR_CUDA;
     }
-    const uint8_t *src = z->map + z->sections[z->weights].off;
     uint8_t *d = static_cast<uint8_t *>(dst);
     const unsigned hw = std::max(1u, std::min(8u, std::thread::hardware_concurrency()));
     uint64_t chunk = 0;
+    bool read_failed = false;
     for (uint64_t off = 0; off < total; off += kChunkBytes, ++chunk) {
         const int b = static_cast<int>(chunk & 1);
         const size_t n = static_cast<size_t>(std::min<uint64_t>(kChunkBytes, total - off));
         if (chunk >= 2 && (e = cudaEventSynchronize(z->done[b])) != cudaSuccess) break;
-        // Parallel read of the chunk from the mapping into pinned memory.
+        // Parallel read of the chunk into pinned memory: each thread preads a
+        // slice straight from the file (no page-table work for the mapping).
         uint8_t *pin = static_cast<uint8_t *>(z->pinned[b]);
         const size_t per = (n + hw - 1) / hw;
+        const uint64_t file_off = z->sections[z->weights].off + off;
         std::vector<std::thread> th;
-        for (unsigned t = 1; t < hw && t * per < n; ++t)
-            th.emplace_back([=] { std::memcpy(pin + t * per, src + off + t * per, std::min(per, n - t * per)); });
-        std::memcpy(pin, src + off, std::min(per, n));
+        std::vector<int> ok(hw, 1);
+        auto slice = [&, pin, per, n, file_off](unsigned t) {
+            size_t done = 0, want = std::min(per, n - t * per);
+            while (done < want) {
+                const ssize_t r = pread(z->fd, pin + t * per + done, want - done,
+                                        static_cast<off_t>(file_off + t * per + done));
+                if (r <= 0) {
+                    ok[t] = 0;
+                    return;
+                }
+                done += static_cast<size_t>(r);
+            }
+        };
+        for (unsigned t = 1; t < hw && t * per < n; ++t) th.emplace_back(slice, t);
+        slice(0);
         for (auto &x : th) x.join();
+        if (std::find(ok.begin(), ok.end(), 0) != ok.end()) {
+            read_failed = true;  // copies in flight are waited for below
+            break;
+        }
         if ((e = cudaMemcpyAsync(d + off, pin, n, cudaMemcpyHostToDevice, s)) != cudaSuccess) break;
         if ((e = cudaEventRecord(z->done[b], s)) != cudaSuccess) break;
     }
     for (int i = 0; i < 2 && e == cudaSuccess; ++i)
         if (chunk > static_cast<uint64_t>(i)) e = cudaEventSynchronize(z->done[i]);
+    if (read_failed && e == cudaSuccess) {
+        zq::set_last_error("reading the weight section failed");
+        return ZQ_ERR_INVALID_ARG;
+    }
     if (e != cudaSuccess) {
         zq::set_last_error((std::string("weight copy: ") + cudaGetErrorString(e)).c_str());
         return ZQ_ERR_CUDA;
