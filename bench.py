@@ -56,8 +56,8 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {
-        "sha256": "49df590480ad52561438fcf96a49f9caba1e1792dafd0e363377fed3d6fc6f77",
-        "bytes_per_layer": 125690176,
+        "sha256": "3a888c2138bd719289484f0d84ece872be0508d129bb271eeac0a3f856ff999a",
+        "bytes_per_layer": 125751936,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },
 }
