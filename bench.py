@@ -56,7 +56,7 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {
-        "sha256": "3a888c2138bd719289484f0d84ece872be0508d129bb271eeac0a3f856ff999a",
+        "sha256": "6b3cf8ccd2363193252fd462974d6fc078dff64692fb133ca7175cc7cba460b4",
         "bytes_per_layer": 125751936,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },

@@ -416,7 +416,7 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
 }
 
 // Expands a linear op into decode-sized pieces (M <= 16 per piece); only used
-// for ops that the prefill family does not take.
+// for ops that the tile kernel does not take.
 void split_tokens(const zq_linear_desc &d, std::vector<zq_linear_desc> &out) {
     for (int m0 = 0; m0 < d.M; m0 += kDecodeMaxM) {
         zq_linear_desc p = d;

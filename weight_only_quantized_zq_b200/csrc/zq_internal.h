@@ -17,7 +17,7 @@ constexpr int kQuantStatusSlots = 64;
 
 // ---------------------------------------------------------------- decode --
 // A decode launch processes up to kMaxDecodeOps independent linear layers of
-// one bit width with M <= 64.  The work is a sequence of CTA steps, one step =
+// one bit width with M <= kDecodeMaxM.  The work is a sequence of CTA steps, one step =
 // (op, 64-row block, GPS consecutive groups of 128); op o owns steps
 // [step0, step0 + row_blocks * su) in row-block-major order.  The steps are
 // cut into chunks (whole row blocks, or 2^log2c consecutive steps); a CTA
