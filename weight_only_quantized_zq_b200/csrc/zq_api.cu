@@ -219,10 +219,10 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     }
     if (total_steps > 0x3FFFFFFFLL) return fail(ZQ_ERR_INVALID_ARG, "decode launch too large (steps)");
 
-    // Stage: codes (64 rows x one step's bytes, a multiple of 1024; all
+    // Stage: codes (64 rows x the box bytes, a multiple of 1024; all
     // stages' codes first, so each starts 1024-aligned), then a meta part of
     // scales and zeros, group sums, activations and the step descriptor.
-    const int codes_bytes = rows * decode_seg(bits, mt);
+    const int codes_bytes = decode_codes_bytes(bits, mt);
     const int off_sz = 0;
     const int off_sx = off_sz + rows * 4 * gps;
     const int off_x = off_sx + gps * mpad * 8;

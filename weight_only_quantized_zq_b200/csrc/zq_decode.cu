@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
     uint32_t cofs[2][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-        const uint32_t crow = (warp * 16 + h * 8 + gr) * (SWZ ? 128 : SEG);
+        const uint32_t crow = (warp * 16 + h * 8 + gr) * (SWZ ? 128 : BOXW);
         if constexpr (!SWZ) {
             cofs[h][0] = cofs[h][1] = crow + 4 * BITS * c;
         } else if constexpr (BITS == 4) {

@@ -84,14 +84,21 @@ struct PrepParams {
 __host__ __device__ constexpr int decode_gps(int bits, int) { return bits == 8 ? 2 : 4; }
 __host__ __device__ constexpr int decode_seg(int bits, int mt) { return decode_gps(bits, mt) * 16 * bits; }
 // Codes of a step land as 128-byte-wide TMA boxes with the 128-byte swizzle
-// when a row segment is a whole number of 128-byte spans; else as one
-// unswizzled box of the whole segment.
+// when a row segment is a whole number of 128-byte spans.  Otherwise (b = 3:
+// 192 bytes) as one unswizzled box 16 bytes wider than the segment: a shared
+// memory row pitch of 208 bytes (52 words) puts the 8 rows of a fragment load
+// in 8 different bank quads, where 192 (48 words) would give only two.  The
+// extra 16 bytes are the start of the next step's codes (or zero fill).
 __host__ __device__ constexpr bool decode_swizzled(int bits, int mt) { return decode_seg(bits, mt) % 128 == 0; }
 __host__ __device__ constexpr int decode_box_w(int bits, int mt) {
-    return decode_swizzled(bits, mt) ? 128 : decode_seg(bits, mt);
+    return decode_swizzled(bits, mt) ? 128 : decode_seg(bits, mt) + 16;
 }
 __host__ __device__ constexpr int decode_boxes(int bits, int mt) {
-    return decode_seg(bits, mt) / decode_box_w(bits, mt);
+    return decode_swizzled(bits, mt) ? decode_seg(bits, mt) / 128 : 1;
+}
+// Shared-memory bytes of one 64-row stage of codes.
+__host__ __device__ constexpr int decode_codes_bytes(int bits, int mt) {
+    return 64 * decode_boxes(bits, mt) * decode_box_w(bits, mt);
 }
 // Token tiles of 8 for the decode kernel (M <= kDecodeMaxM).
 inline int mt_for_m(int M) { return M <= 8 ? 1 : 2; }
