@@ -56,8 +56,8 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {
-        "sha256": "6b3cf8ccd2363193252fd462974d6fc078dff64692fb133ca7175cc7cba460b4",
-        "bytes_per_layer": 125751936,
+        "sha256": "09b63fcb7ccf886ae872d21d350c5db9744078cf81a924fcd47aa6d54bcf2455",
+        "bytes_per_layer": 126511168,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },
 }

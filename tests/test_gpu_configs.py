@@ -4,6 +4,9 @@ benchmark uses (one zq_linear_stack call over the whole stack).
 Config 3: 28 Qwen2.5-7B-shaped layers x (qkv, o, gate_up, down), INT4 g128,
 M in {1, 4, 16, 64}; layers 0 and 27 are quantized on the GPU AND by the oracle
 (bit-exact) and every output of their projections is checked.
+Config 4 (stack): 64 Qwen2.5-32B-shaped layers, INT8 qkv / INT4 o / INT3
+gate_up / INT2 down with 0.1% outliers, M = 1 (the benchmark's 32b-mixed
+workload: one decode launch per bit width); layers 0 and 63 checked in full.
 Config 5: M = 2048 prefill, INT4 g128, the four projections of layers 0 and 27;
 all M rows x 256 sampled output columns per projection are checked.
 """
@@ -61,6 +64,32 @@ def test_config3_decode_stack_28_layers(zq, orc):
             if l in check:
                 y_ref, bound = orc.linear(u16(xs[(M, K)]), *ref, 4, N, K)
                 assert_linear_close(out, y_ref, bound, f"config3 M={M} layer {l} {name}")
+
+
+def test_config4_mixed_stack_64_layers(zq, orc):
+    check = (0, zi.QWEN32B_LAYERS - 1)
+    xs = {K: zi.activations(1, K, zi.seed_for(0, zi.X_SEED), device="cuda") for K in (5120, 27648)}
+    ops, outs = [], []
+    for layer in range(zi.QWEN32B_LAYERS):
+        for t, (name, N, K, bits) in enumerate(zi.QWEN32B_MIXED):
+            w = zi.weight(N, K, zi.seed_for(layer, t), device="cuda", outliers=True)
+            q = zq.quantize(w, bits)
+            ref = None
+            if layer in check:
+                torch.cuda.synchronize()
+                ref = orc.quantize_pack(w.cpu().numpy(), bits)
+                assert np.array_equal(u32(q[0]).reshape(N, -1), ref[0]), f"layer {layer} {name} codes"
+            del w
+            out = torch.empty(1, N, dtype=torch.float16, device="cuda")
+            ops.append((xs[K], *q, out, bits, 128, 1, N, K))
+            outs.append((layer, name, N, K, bits, out, ref))
+    zq.zq_linear_stack(ops)
+    torch.cuda.synchronize()
+    zq.zq_check_device()
+    for (layer, name, N, K, bits, out, ref) in outs:
+        if layer in check:
+            y_ref, bound = orc.linear(u16(xs[K]), *ref, bits, N, K)
+            assert_linear_close(out, y_ref, bound, f"config4 stack layer {layer} {name} int{bits}")
 
 
 def test_config5_prefill_m2048(zq, orc):
