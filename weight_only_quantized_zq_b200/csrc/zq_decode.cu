@@ -525,15 +525,24 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
 #pragma unroll
     for (int i = 0; i < 16; ++i) xf1[i] = 0u;
     int slot = 0, n_seen = 0;  // stages this warp has waited for
+    int deferred = -1;         // stage this warp still has to fill
     uint32_t par = 0;
 
 #pragma unroll 1
     while (!aborted) {
         {
-            const int target = n_seen + D - 1;  // stage to fill now, by its warp
-            if (target % kDecodeWarpsPerCta == warp && !produce(target)) {
-                aborted = true;
-                break;
+            // Stage to fill now, by its warp.  If the previous producer has not
+            // handed over yet, consume first and fill it afterwards.
+            const int target = n_seen + D - 1;
+            if (target % kDecodeWarpsPerCta == warp) {
+                if (__all_sync(0xffffffffu, ld_acquire_shared(&ps->seq) == target)) {
+                    if (!produce(target)) {
+                        aborted = true;
+                        break;
+                    }
+                } else {
+                    deferred = target;
+                }
             }
         }
         if (!wait_phase(&full[slot], par)) {
@@ -546,7 +555,10 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
         const uint4 d1 = lds_v4(smb + p.off_desc + 16);
         const int flags = static_cast<int>(d0.w) >> 8;
         ++n_seen;
-        if (flags & kFlagEnd) break;
+        if (flags & kFlagEnd) {
+            if (deferred >= 0 && !produce(deferred)) aborted = true;  // later producers wait for it
+            break;
+        }
         const int ng = d0.w & 0xFF;
         const int M = static_cast<int>(d1.z);
         const int o = static_cast<int>(d0.x), rb = static_cast<int>(d0.y);
@@ -669,6 +681,14 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
         if (++slot == D) {
             slot = 0;
             par ^= 1u;
+        }
+        if (deferred >= 0) {
+            const bool ok = produce(deferred);
+            deferred = -1;
+            if (!ok) {
+                aborted = true;
+                break;
+            }
         }
 
         if (flags & kFlagLast) {
