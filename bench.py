@@ -56,8 +56,8 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {
-        "sha256": "09b63fcb7ccf886ae872d21d350c5db9744078cf81a924fcd47aa6d54bcf2455",
-        "bytes_per_layer": 126511168,
+        "sha256": "5512377e1a34955ab1b352556eaa33c0c5361bdafa91cda6f12565a167d3f631",
+        "bytes_per_layer": 125936384,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },
 }
