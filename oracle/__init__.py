@@ -46,6 +46,10 @@ def _load():
         lib.zo_unpack_row.restype = None
         lib.zo_quantize_pack.argtypes = [P, I, I, I, I, P, P, P]
         lib.zo_quantize_pack.restype = I
+        lib.zo_quantize_group_symmetric.argtypes = [P, I, I, P, P, P]
+        lib.zo_quantize_group_symmetric.restype = I
+        lib.zo_quantize_pack_symmetric.argtypes = [P, I, I, I, I, P, P, P]
+        lib.zo_quantize_pack_symmetric.restype = I
         lib.zo_unpack.argtypes = [P, I, I, I, P]
         lib.zo_unpack.restype = I
         lib.zo_dequant.argtypes = [P, P, P, I, I, I, I, P]
@@ -100,6 +104,20 @@ def quantize_group(w, bits):
     return s.value, z.value, q
 
 
+def quantize_group_symmetric(w, bits):
+    """Symmetric quantizer, one group; returns (s16_bits, z16_bits, stored
+    codes uint8 array, code = q + 2^(bits-1))."""
+    w = _c(w, np.float32)
+    q = np.zeros(w.size, np.uint8)
+    s = ctypes.c_uint16()
+    z = ctypes.c_uint16()
+    st = _load().zo_quantize_group_symmetric(_ptr(w), w.size, bits,
+                                             ctypes.byref(s), ctypes.byref(z), _ptr(q))
+    if st != OK:
+        raise OracleError(st)
+    return s.value, z.value, q
+
+
 def pack_row(codes, bits):
     codes = _c(codes, np.uint8)
     K = codes.size
@@ -125,6 +143,21 @@ def quantize_pack(w, bits, group=GROUP):
     zeros = np.zeros((N, G), np.uint16)
     st = _load().zo_quantize_pack(_ptr(w), N, K, bits, group,
                                   _ptr(packed), _ptr(scales), _ptr(zeros))
+    if st != OK:
+        raise OracleError(st)
+    return packed, scales, zeros
+
+
+def quantize_pack_symmetric(w, bits, group=GROUP):
+    """Symmetric quantizer over W (N x K fp32); same outputs as quantize_pack."""
+    w = _c(w, np.float32)
+    N, K = w.shape
+    G = max(K // group, 1)
+    packed = np.zeros((N, max(K * bits // 32, 1)), np.uint32)
+    scales = np.zeros((N, G), np.uint16)
+    zeros = np.zeros((N, G), np.uint16)
+    st = _load().zo_quantize_pack_symmetric(_ptr(w), N, K, bits, group,
+                                            _ptr(packed), _ptr(scales), _ptr(zeros))
     if st != OK:
         raise OracleError(st)
     return packed, scales, zeros

@@ -30,6 +30,10 @@
  *     zero point), computed exactly in fp64.
  *   - linear: y[m][n] = sum_k x[m][k]*w_hat[n][k] in fp64 (W is N x K, the
  *     PyTorch Linear convention y = x W^T); bound = sum_k |x||w_hat|.
+ *   - symmetric quantization (listed by [wiki] for INT8 without a formula):
+ *     Q = 2^(b-1) - 1, scale = fp16(max|w| / Q), q = clamp(round(w/scale),
+ *     -Q, Q); stored as code = q + 2^(b-1), zero = -2^(b-1)*scale (exact), so
+ *     the same dequant gives q*scale.  A zero below -65504 is rejected.
  *
  * Build: gcc -O2 -std=c11 -fPIC -shared -fopenmp -ffp-contract=off
  *        (no -ffast-math: the fp64 steps must be plain IEEE operations).
@@ -132,6 +136,46 @@ int zo_quantize_group(const float *w, int n, int L,
 }
 
 /* ------------------------------------------------------------------------ */
+/* Symmetric quantizer: one group.  [wiki] "Формат модели .zse" lists       */
+/* symmetric INT8 quantization (reserved) beside the asymmetric INT4 one,   */
+/* without a formula.  Reading: Q = 2^(b-1) - 1 (127 at b = 8),             */
+/* scale = max|w| / Q, q = clamp(round(w / scale), -Q, Q), w_hat = q*scale, */
+/* with the same fp64 steps and fp16 rounding as the asymmetric quantizer.  */
+/* Stored in the asymmetric format: code = q + 2^(b-1), zero = -2^(b-1) *   */
+/* s16 (exact, a power-of-two multiple), so code*s16 + zero = q*s16.        */
+/* ------------------------------------------------------------------------ */
+
+int zo_quantize_group_symmetric(const float *w, int n, int bits,
+                                uint16_t *s16_out, uint16_t *z16_out, uint8_t *codes)
+{
+    for (int i = 0; i < n; ++i)
+        if (!isfinite(w[i]) || fabs((double)w[i]) > 65504.0)
+            return ZO_NONFINITE;
+    double half = (double)(1 << (bits - 1));          /* code offset 2^(b-1) */
+    double Q = half - 1.0;                            /* largest |q|         */
+    double amax = 0.0;
+    for (int i = 0; i < n; ++i)
+        if (fabs((double)w[i]) > amax) amax = fabs((double)w[i]);
+    uint16_t s16 = zo_f64_to_f16(amax / Q);           /* scale               */
+    double s = zo_f16_to_f64(s16);
+    double z = -half * s;                             /* zero, exact in fp64 */
+    if (z < -65504.0)
+        return ZO_NONFINITE;                          /* zero not storable   */
+    for (int i = 0; i < n; ++i) {
+        double t = 0.0;
+        if (s != 0.0) {
+            t = rint((double)w[i] / s);               /* round half even     */
+            if (t < -Q) t = -Q;
+            if (t > Q) t = Q;
+        }
+        codes[i] = (uint8_t)(t + half);
+    }
+    *s16_out = s16;
+    *z16_out = zo_f64_to_f16(z);
+    return ZO_OK;
+}
+
+/* ------------------------------------------------------------------------ */
 /* Bitstream packing of one row: code i -> stream bits [i*b, i*b+b);        */
 /* stream bit t -> bit (t % 32) of word t / 32. Done bit by bit on purpose. */
 /* ------------------------------------------------------------------------ */
@@ -189,6 +233,35 @@ int zo_quantize_pack(const float *w, int N, int K, int bits, int group,
                                       &scales[(size_t)n * G + g],
                                       &zeros[(size_t)n * G + g],
                                       codes + (size_t)g * group);
+            if (r != ZO_OK) {
+#pragma omp atomic write
+                status = r;
+            }
+        }
+        zo_pack_row(codes, K, bits, packed + (size_t)n * wpr);
+        free(codes);
+    }
+    return status;
+}
+
+/* Whole tensor, symmetric quantizer; output layout as zo_quantize_pack. */
+int zo_quantize_pack_symmetric(const float *w, int N, int K, int bits, int group,
+                               uint32_t *packed, uint16_t *scales, uint16_t *zeros)
+{
+    int st = zo_check_format(N, K, bits, group);
+    if (st != ZO_OK)
+        return st;
+    int G = K / group;
+    int wpr = K * bits / 32;
+    int status = ZO_OK;
+#pragma omp parallel for schedule(dynamic, 16)
+    for (int n = 0; n < N; ++n) {
+        uint8_t *codes = (uint8_t *)malloc((size_t)K);
+        for (int g = 0; g < G; ++g) {
+            int r = zo_quantize_group_symmetric(w + (size_t)n * K + (size_t)g * group, group, bits,
+                                                &scales[(size_t)n * G + g],
+                                                &zeros[(size_t)n * G + g],
+                                                codes + (size_t)g * group);
             if (r != ZO_OK) {
 #pragma omp atomic write
                 status = r;

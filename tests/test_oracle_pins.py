@@ -294,6 +294,129 @@ def test_quantize_pack_rejects_bad_format(orc):
     assert e.value.status == orc.INVALID
 
 
+# ------------------------------------------------------- symmetric quantizer --
+# The wiki section "Формат модели .zse" lists symmetric INT8 quantization
+# without a formula; the reading (Q = 2^(b-1) - 1, scale = fp16(max|w|/Q),
+# q = clamp(round(w/scale), -Q, Q), stored code = q + 2^(b-1), zero =
+# -2^(b-1)*scale) is pinned here by hand-derived examples, numpy's fp16, exact
+# rational brute force, odd symmetry and the dequantized values.
+
+def test_symmetric_worked_examples(orc):
+    n_lines = 0
+    with open(os.path.join(GOLDEN, "quant_symmetric_examples.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            head, ws, qs = [p.strip() for p in line.split("|")]
+            bits, s_bits, z_bits = head.split()
+            w = np.array([float(v) for v in ws.split()], np.float32)
+            s, z, q = orc.quantize_group_symmetric(w, int(bits))
+            assert (s, z) == (int(s_bits, 16), int(z_bits, 16))
+            assert list(q) == [int(v) for v in qs.split()]
+            n_lines += 1
+    assert n_lines == 2
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_symmetric_scale_zero_and_range(orc, bits):
+    """s16 = numpy fp16(max|w| / Q), z16 = numpy fp16(-2^(b-1) * s16) (exact),
+    codes in [1, 2^b - 1], |w - q*s16| <= s16/2 unless clamped at +-Q."""
+    rng = np.random.default_rng(70 + bits)
+    half, Q = 1 << (bits - 1), (1 << (bits - 1)) - 1
+    for _ in range(200):
+        w = (rng.normal(0, 0.02, 128) * rng.choice([1, 20], 128, p=[.99, .01])).astype(np.float32)
+        s_b, z_b, codes = orc.quantize_group_symmetric(w, bits)
+        amax = np.abs(w.astype(np.float64)).max()
+        assert s_b == np.float16(amax / Q).view(np.uint16)
+        s = float(np.uint16(s_b).view(np.float16))
+        assert float(np.uint16(z_b).view(np.float16)) == -half * s
+        q = codes.astype(np.int64) - half
+        assert codes.min() >= 1 and codes.max() <= (1 << bits) - 1
+        err = np.abs(w.astype(np.float64) - q * s)
+        inside = np.abs(q) < Q
+        assert np.all(err[inside] <= s / 2)
+        assert np.all(err[~inside] <= max(s / 2, amax - Q * s) + 1e-300)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_symmetric_odd_symmetry(orc, bits):
+    """Negating the group negates every q and keeps the scale (round half to
+    even is symmetric about zero)."""
+    rng = np.random.default_rng(80 + bits)
+    half = 1 << (bits - 1)
+    for _ in range(50):
+        w = rng.normal(0, 0.02, 128).astype(np.float32)
+        s1, z1, c1 = orc.quantize_group_symmetric(w, bits)
+        s2, z2, c2 = orc.quantize_group_symmetric(-w, bits)
+        assert (s1, z1) == (s2, z2)
+        assert np.array_equal(c1.astype(int) - half, -(c2.astype(int) - half))
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_symmetric_brute_force_exact(orc, bits):
+    """Exhaustive search over q in [-Q, Q] with exact rationals: the chosen q
+    minimises |w - q*s16|, ties to the even q."""
+    rng = np.random.default_rng(90 + bits)
+    half, Q = 1 << (bits - 1), (1 << (bits - 1)) - 1
+    for trial in range(40):
+        n = int(rng.integers(2, 24))
+        w = (rng.normal(0, 0.02, n) * (20 if trial % 7 == 0 else 1)).astype(np.float32)
+        s_b, _, codes = orc.quantize_group_symmetric(w, bits)
+        s = Fraction(float(np.uint16(s_b).view(np.float16)))
+        for i in range(n):
+            wi = Fraction(float(w[i]))
+            best = None
+            for cand in range(-Q, Q + 1):
+                d = abs(wi - cand * s)
+                if best is None or d < best[0] or (d == best[0] and cand % 2 == 0):
+                    best = (d, cand)
+            assert int(codes[i]) - half == best[1], (trial, i, codes[i], best)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_symmetric_dequant_is_q_times_scale(orc, bits):
+    """Through the ordinary dequantizer (code*s16 + z16) a symmetric tensor
+    gives exactly q*s16, computed here in numpy from the bit fields."""
+    rng = np.random.default_rng(100 + bits)
+    N, K = 4, 384
+    half = 1 << (bits - 1)
+    w = rng.normal(0, 0.02, (N, K)).astype(np.float32)
+    w[1, 128:256] = 0.0                                   # an all-zero group
+    packed, scales, zeros = orc.quantize_pack_symmetric(w, bits)
+    codes = np.stack([_stream_codes_numpy(packed[n], K, bits) for n in range(N)]).astype(np.int64)
+    s = scales.view(np.float16).astype(np.float64).repeat(128, axis=1)
+    assert np.array_equal(orc.dequant(packed, scales, zeros, bits, N, K), (codes - half) * s)
+    assert scales[1, 1] == 0 and np.all(codes[1, 128:256] == half)
+    for n in range(N):
+        for g in range(K // 128):
+            sg, zg, cg = orc.quantize_group_symmetric(w[n, g * 128:(g + 1) * 128], bits)
+            assert scales[n, g] == sg and zeros[n, g] == zg
+            assert np.array_equal(codes[n, g * 128:(g + 1) * 128], cg)
+
+
+def test_symmetric_rejects(orc):
+    for bad in (np.nan, np.inf, 65505.0):
+        w = np.zeros(128, np.float32)
+        w[5] = bad
+        with pytest.raises(orc.OracleError) as e:
+            orc.quantize_group_symmetric(w, 8)
+        assert e.value.status == orc.NONFINITE
+    # zero = -2^(b-1)*scale must be a finite fp16: 65400/127 -> 515, 128*515 > 65504
+    for bits, big in ((8, 65400.0), (2, 40000.0)):
+        w = np.zeros(128, np.float32)
+        w[0] = big
+        with pytest.raises(orc.OracleError) as e:
+            orc.quantize_group_symmetric(w, bits)
+        assert e.value.status == orc.NONFINITE
+    w = np.zeros(128, np.float32)
+    w[0] = 32000.0                     # 128 * fp16(32000/127) = 32256: storable
+    orc.quantize_group_symmetric(w, 8)
+    with pytest.raises(orc.OracleError) as e:
+        orc.quantize_pack_symmetric(np.zeros((2, 256), np.float32), 5)
+    assert e.value.status == orc.UNSUPPORTED
+
+
 # ------------------------------------------------------------ dequant/linear --
 
 def _numpy_dequant(packed, scales, zeros, bits, N, K):
