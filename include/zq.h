@@ -102,6 +102,22 @@ ZQ_API zq_status zq_quantize_pack(const float *w, int N, int K, int bits, int gr
                            uint32_t *packed, uint16_t *scales, uint16_t *zeros,
                            zq_stream_t stream);
 
+/* Symmetric variant of zq_quantize_pack ([wiki] "Формат модели .zse" lists
+ * symmetric INT8 quantization, reserved, without a formula; the same step is
+ * offered for every supported width).  Arguments, layout, synchronisation and
+ * errors as zq_quantize_pack.  Per group of 128, with Q = 2^(bits-1) - 1:
+ * scale = fp16(max|w| / Q) computed in fp64 and rounded once;
+ * q = clamp(round_half_even(w / scale), -Q, Q) with the stored fp16 scale
+ * (q = 0 when the scale is 0).  The result is stored in the ordinary format:
+ * code = q + 2^(bits-1) and zero = -2^(bits-1) * scale (exact), so zq_linear
+ * and every other consumer compute code*scale + zero = q*scale unchanged.
+ * Bit-exact with the reference quantizer.  ZQ_ERR_NONFINITE also when a
+ * group's zero would fall below -65504 (max|w| above about 65000 at 8 bits,
+ * 32752 at 2 bits). */
+ZQ_API zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bits, int group,
+                                            uint32_t *packed, uint16_t *scales, uint16_t *zeros,
+                                            zq_stream_t stream);
+
 /* y = x · dequant(W)^T.
  *   x       device, fp16 M x K.      out  device, fp16 M x N (written).
  *   packed/scales/zeros as produced by zq_quantize_pack.

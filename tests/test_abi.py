@@ -94,13 +94,15 @@ def test_linear_rejects(zq, kw, status):
     assert zq.zq_last_error() != ""
 
 
-def test_quantize_rejects(zq):
-    q = zq._lib.zq_quantize_pack
+@pytest.mark.parametrize("name", ["zq_quantize_pack", "zq_quantize_pack_symmetric"])
+def test_quantize_rejects(zq, name):
+    q = getattr(zq._lib, name)
     assert q(A, 4, 256, 5, 128, A, A, A, None) == zq.ZQ_ERR_UNSUPPORTED
     assert q(A, 4, 256, 4, 32, A, A, A, None) == zq.ZQ_ERR_UNSUPPORTED
     assert q(A, 4, 200, 4, 128, A, A, A, None) == zq.ZQ_ERR_INVALID_ARG
     assert q(0, 4, 256, 4, 128, A, A, A, None) == zq.ZQ_ERR_INVALID_ARG
     assert q(A, 4, 256, 4, 128, A + 1, A, A, None) == zq.ZQ_ERR_INVALID_ARG
+    assert q(A, 4, 256, 4, 128, A, A, 0, None) == zq.ZQ_ERR_INVALID_ARG
 
 
 def test_unpack_rejects(zq):

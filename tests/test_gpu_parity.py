@@ -1,6 +1,7 @@
 """GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
 
-Bit-exact: quantize_pack (codes, scales, zeros) and unpack.
+Bit-exact: quantize_pack and quantize_pack_symmetric (codes, scales, zeros)
+and unpack.
 Tolerance (the linear): |y_gpu - y_ref| <= 2e-3 * sum|x||w_hat| + 1e-3 per element.
 """
 import numpy as np
@@ -80,6 +81,59 @@ def test_quantize_pack_rejects_nonfinite(zq):
             zq.quantize(w, 4)
         assert e.value.status == zq.ZQ_ERR_NONFINITE
     zq.quantize(torch.zeros(4, 256, device="cuda"), 4)  # next call is clean
+
+
+def _quantize_both_symmetric(zq, orc, w, bits):
+    N, K = w.shape
+    packed, scales, zeros = zq.quantize(w, bits, symmetric=True)
+    torch.cuda.synchronize()
+    p_ref, s_ref, z_ref = orc.quantize_pack_symmetric(w.cpu().numpy(), bits)
+    assert np.array_equal(u16(scales).reshape(N, -1), s_ref), "scales differ"
+    assert np.array_equal(u16(zeros).reshape(N, -1), z_ref), "zeros differ"
+    assert np.array_equal(u32(packed).reshape(N, -1), p_ref), "packed codes differ"
+    return packed, scales, zeros, (p_ref, s_ref, z_ref)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_quantize_pack_symmetric_bit_exact(zq, orc, bits):
+    """The symmetric quantizer (INT8-symmetric of the .zse format section, at
+    every width) against the oracle, bit for bit, including edge groups."""
+    for N, K, seed, outl in ((1, 128, 11, False), (37, 512, 12, True), (5, 27648, 14, True)):
+        w = zi.weight(N, K, seed + 100 * bits, device="cuda", outliers=outl)
+        _quantize_both_symmetric(zq, orc, w, bits)
+    Q = (1 << (bits - 1)) - 1
+    K = 768
+    w = torch.zeros(6, K)                          # row 0: all-zero groups (scale 0)
+    w[1, 0] = Q / 128.0                            # scale exactly 2^-7 ...
+    j = torch.arange(Q, dtype=torch.float32)
+    w[1, 1:1 + Q] = (j + 0.5) / 128                # ... so these are exact ties
+    w[1, 64:64 + Q] = -(j + 0.5) / 128
+    w[2] = torch.linspace(-32000, 32000, K)        # large, still storable zeros
+    w[3] = torch.linspace(0, 1e-6, K)              # fp16 subnormal scales
+    w[4] = torch.randn(K) * 1e-3 - 3.0             # one-signed groups
+    w[5, ::2] = 1.0
+    _quantize_both_symmetric(zq, orc, w.cuda().contiguous(), bits)
+
+
+def test_quantize_pack_symmetric_rejects(zq):
+    for bits, bad in ((8, float("nan")), (8, 70000.0), (8, 65400.0), (2, 40000.0)):
+        w = torch.zeros(4, 256, device="cuda")
+        w[1, 200] = bad
+        with pytest.raises(zq.ZQError) as e:
+            zq.quantize(w, bits, symmetric=True)
+        assert e.value.status == zq.ZQ_ERR_NONFINITE
+    zq.quantize(torch.zeros(4, 256, device="cuda"), 8, symmetric=True)  # next call is clean
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_linear_symmetric_weights(zq, orc, bits):
+    """Symmetric tensors run through the unchanged linear kernels (decode and
+    tile) and meet the oracle tolerance."""
+    for i, (M, N, K) in enumerate(((1, 130, 512), (7, 64, 1280), (16, 33, 384), (40, 264, 640))):
+        w = zi.weight(N, K, seed=5000 + 10 * bits + i, device="cuda", outliers=(i % 2 == 1))
+        q = _quantize_both_symmetric(zq, orc, w, bits)
+        x = zi.activations(M, K, seed=5100 + i, device="cuda")
+        _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"symmetric bits={bits} M={M} N={N} K={K}")
 
 
 @pytest.mark.parametrize("bits", BITS)

@@ -26,7 +26,7 @@ ZQ_ERR_TIMEOUT = 5
 GROUP = 128
 
 # Every symbol the headers declare (checked by the CPU test suite).
-EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_linear", "zq_linear_noalloc", "zq_linear_stack",
+EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_quantize_pack_symmetric", "zq_linear", "zq_linear_noalloc", "zq_linear_stack",
            "zq_unpack", "zq_reserve_workspace", "zq_linear_workspace_bytes",
            "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
            "zq_version",
@@ -46,6 +46,8 @@ _lib.zq_packed_words.argtypes = [_I, _I, _I]
 _lib.zq_packed_words.restype = _S
 _lib.zq_quantize_pack.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
 _lib.zq_quantize_pack.restype = _I
+_lib.zq_quantize_pack_symmetric.argtypes = [_P, _I, _I, _I, _I, _P, _P, _P, _P]
+_lib.zq_quantize_pack_symmetric.restype = _I
 _lib.zq_linear.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
 _lib.zq_linear.restype = _I
 _lib.zq_linear_noalloc.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
@@ -169,6 +171,11 @@ def zq_quantize_pack(w, N, K, bits, group, packed, scales, zeros, stream=None):
                                  _ptr(zeros), _stream(stream, w)))
 
 
+def zq_quantize_pack_symmetric(w, N, K, bits, group, packed, scales, zeros, stream=None):
+    _check(_lib.zq_quantize_pack_symmetric(_ptr(w), N, K, bits, group, _ptr(packed), _ptr(scales),
+                                           _ptr(zeros), _stream(stream, w)))
+
+
 def zq_linear(x, packed, scales, zeros, bits, group, M, N, K, out, stream=None):
     _check(_lib.zq_linear(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), bits, group,
                           M, N, K, _ptr(out), _stream(stream, x)))
@@ -215,11 +222,13 @@ def alloc_quantized(N, K, bits, device="cuda"):
     return packed, scales, zeros
 
 
-def quantize(w, bits, stream=None):
-    """fp32 CUDA tensor N x K -> (packed, scales, zeros) via zq_quantize_pack."""
+def quantize(w, bits, stream=None, symmetric=False):
+    """fp32 CUDA tensor N x K -> (packed, scales, zeros) via zq_quantize_pack
+    (or zq_quantize_pack_symmetric); both give the same storage format."""
     N, K = w.shape
     packed, scales, zeros = alloc_quantized(N, K, bits, w.device)
-    zq_quantize_pack(w, N, K, bits, GROUP, packed, scales, zeros, stream)
+    fn = zq_quantize_pack_symmetric if symmetric else zq_quantize_pack
+    fn(w, N, K, bits, GROUP, packed, scales, zeros, stream)
     return packed, scales, zeros
 
 

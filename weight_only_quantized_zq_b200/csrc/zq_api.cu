@@ -18,6 +18,7 @@
 
 #include "zq.h"
 #include "zq_internal.h"
+#include "zq_quant.h"
 
 using namespace zq;
 
@@ -562,6 +563,30 @@ zq_status zq_quantize_pack(const float *w, int N, int K, int bits, int group, ui
     e = read_quant_status(slot, &got, s);
     if (e != cudaSuccess) return cuda_fail(e, "quantize status");
     if (got == id) return fail(ZQ_ERR_NONFINITE, "weights contain NaN/Inf or |w| > 65504");
+    return ZQ_OK;
+}
+
+zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bits, int group, uint32_t *packed,
+                                     uint16_t *scales, uint16_t *zeros, zq_stream_t stream) {
+    zq_status st = check_format(bits, group, N, K);
+    if (st != ZQ_OK) return st;
+    if ((st = check_ptr(w, "w")) != ZQ_OK) return st;
+    if ((st = check_ptr(packed, "packed")) != ZQ_OK) return st;
+    if ((st = check_ptr(scales, "scales")) != ZQ_OK) return st;
+    if ((st = check_ptr(zeros, "zeros")) != ZQ_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const unsigned long long id = g_quant_call.fetch_add(1);
+    const int slot = static_cast<int>(id % kQuantStatusSlots);
+    cudaError_t e = launch_quantize_pack_symmetric(w, N, K, bits, packed, scales, zeros, slot, id, s);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    ++g_launches;
+    unsigned long long got = 0;
+    e = read_quant_status(slot, &got, s);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize status");
+    if (got == id)
+        return fail(ZQ_ERR_NONFINITE,
+                    "weights contain NaN/Inf or |w| > 65504, or a group's symmetric zero "
+                    "-2^(bits-1)*scale is not a finite fp16");
     return ZQ_OK;
 }
 

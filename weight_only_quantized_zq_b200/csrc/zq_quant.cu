@@ -7,6 +7,12 @@
 // widths of "ZSE: A Memory-Efficient LLM Inference Engine with Smart Resource
 // Orchestration", section "Technical Architecture".
 //
+// Symmetric variant: the same section lists symmetric INT8 quantization
+// (reserved) without a formula.  Q = 2^(b-1) - 1, scale = fp16(max|w| / Q),
+// q = clamp(round(w / scale), -Q, Q), stored in the asymmetric format as
+// code = q + 2^(b-1) with zero = -2^(b-1) * scale (exact: a power-of-two
+// multiple), so every linear kernel computes code*scale + zero = q*scale.
+//
 // Arithmetic: fp64 with explicit round-to-nearest intrinsics (no contraction),
 // one rounding to fp16 for the stored scale and zero, q from the STORED fp16
 // values, round half to even.  This makes the result bit-identical to any
@@ -16,6 +22,7 @@
 
 #include "zq_device.cuh"
 #include "zq_internal.h"
+#include "zq_quant.h"
 
 namespace zq {
 
@@ -28,6 +35,7 @@ __device__ __forceinline__ uint16_t f64_to_f16_bits(double v) {
 }
 
 // One warp per (row, group).  Each lane owns 4 consecutive weights.
+template <bool SYMMETRIC>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(
     const float *__restrict__ w, int N, int K, int bits, uint32_t *__restrict__ packed,
     uint16_t *__restrict__ scales, uint16_t *__restrict__ zeros, int slot,
@@ -60,22 +68,40 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
         mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
         mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     }
-    const uint16_t z16 = f64_to_f16_bits(static_cast<double>(mn));
-    const uint16_t s16 = f64_to_f16_bits(
-        __ddiv_rn(__dsub_rn(static_cast<double>(mx), static_cast<double>(mn)), static_cast<double>(L)));
-    const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
-    const double z = static_cast<double>(__half2float(__ushort_as_half(z16)));
-
+    uint16_t s16, z16;
     uint32_t chunk = 0;  // this lane's 4 codes, 4*bits bits
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        uint32_t q = 0;
-        if (s != 0.0) {
-            double t = rint(__ddiv_rn(__dsub_rn(static_cast<double>(v[i]), z), s));
-            t = fmin(fmax(t, 0.0), static_cast<double>(L));
-            q = static_cast<uint32_t>(t);
+    if constexpr (SYMMETRIC) {
+        const double half = static_cast<double>(1 << (bits - 1)), Q = half - 1.0;
+        s16 = f64_to_f16_bits(__ddiv_rn(static_cast<double>(fmaxf(-mn, mx)), Q));
+        const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
+        const double z = __dmul_rn(-half, s);
+        if (z < -65504.0) {  // the zero would not be a finite fp16 (uniform across the warp)
+            if (lane == 0) atomicExch(&g_quant_status[slot], call_id);
+            return;
         }
-        chunk |= q << (bits * i);
+        z16 = f64_to_f16_bits(z);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            double t = 0.0;
+            if (s != 0.0) t = fmin(fmax(rint(__ddiv_rn(static_cast<double>(v[i]), s)), -Q), Q);
+            chunk |= static_cast<uint32_t>(t + half) << (bits * i);
+        }
+    } else {
+        z16 = f64_to_f16_bits(static_cast<double>(mn));
+        s16 = f64_to_f16_bits(
+            __ddiv_rn(__dsub_rn(static_cast<double>(mx), static_cast<double>(mn)), static_cast<double>(L)));
+        const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
+        const double z = static_cast<double>(__half2float(__ushort_as_half(z16)));
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            uint32_t q = 0;
+            if (s != 0.0) {
+                double t = rint(__ddiv_rn(__dsub_rn(static_cast<double>(v[i]), z), s));
+                t = fmin(fmax(t, 0.0), static_cast<double>(L));
+                q = static_cast<uint32_t>(t);
+            }
+            chunk |= q << (bits * i);
+        }
     }
     // Assemble the group's 4*bits words: lane's chunk starts at stream bit 4*bits*lane.
     const int nw = 4 * bits;
@@ -123,8 +149,18 @@ cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, uint32_
                                  unsigned long long call_id, cudaStream_t stream) {
     const long long items = static_cast<long long>(N) * (K / 128);
     const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
-    quantize_pack_kernel<<<blocks, 256, 0, stream>>>(w, N, K, bits, packed, scales, zeros, slot,
-                                                     call_id);
+    quantize_pack_kernel<false><<<blocks, 256, 0, stream>>>(w, N, K, bits, packed, scales, zeros, slot,
+                                                            call_id);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_quantize_pack_symmetric(const float *w, int N, int K, int bits, uint32_t *packed,
+                                           uint16_t *scales, uint16_t *zeros, int slot,
+                                           unsigned long long call_id, cudaStream_t stream) {
+    const long long items = static_cast<long long>(N) * (K / 128);
+    const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
+    quantize_pack_kernel<true><<<blocks, 256, 0, stream>>>(w, N, K, bits, packed, scales, zeros, slot,
+                                                           call_id);
     return cudaGetLastError();
 }
 
