@@ -261,6 +261,27 @@ def test_stack_against_oracle(zq, orc):
         assert_linear_close(y_out, y_ref, bound, "stack chain")
 
 
+@pytest.mark.parametrize("bits", BITS)
+def test_prefill_grouped_plans(zq, orc, bits):
+    """Grouped tile-kernel launches of independent ops: one whose ops all have
+    17..128 tokens (one-token-half plan: 128-token x boxes, cp.async code ring;
+    several row tiles per op, ops of different K so tiles of different group
+    counts follow each other in a CTA), and one that mixes such ops with a
+    larger M (two-half plan)."""
+    for specs in ([(17, 520, 640), (100, 264, 1280), (128, 256, 384), (64, 300, 3584)],
+                  [(40, 264, 640), (200, 130, 384), (128, 512, 512)]):
+        layers = [_layer(zq, orc, N, K, bits, 90 + 7 * i + bits) for i, (M, N, K) in enumerate(specs)]
+        xs = [zi.activations(M, K, 95 + i, device="cuda") for i, (M, N, K) in enumerate(specs)]
+        outs = [torch.empty(M, N, dtype=torch.float16, device="cuda") for (M, N, K) in specs]
+        zq.zq_linear_stack([(xs[i], *layers[i][0], outs[i], bits, 128, M, N, K)
+                            for i, (M, N, K) in enumerate(specs)])
+        torch.cuda.synchronize()
+        for i, (M, N, K) in enumerate(specs):
+            p, s, z = layers[i][1]
+            y_ref, bound = orc.linear(u16(xs[i]), p, s, z, bits, N, K)
+            assert_linear_close(outs[i], y_ref, bound, f"grouped bits={bits} M={M} N={N} K={K}")
+
+
 def test_stack_validation_enqueues_nothing(zq, orc):
     q, _ = _layer(zq, orc, 64, 256, 4, 80)
     x = zi.activations(1, 256, 81, device="cuda")

@@ -18,6 +18,7 @@
 
 #include "zq.h"
 #include "zq_internal.h"
+#include "zq_prefill.h"
 #include "zq_quant.h"
 
 using namespace zq;
@@ -440,10 +441,12 @@ zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
     PrefillGroup pg;
     std::memset(&pg, 0, sizeof(pg));
     pg.n_ops = static_cast<int>(ops.size());
+    for (size_t i = 0; i < ops.size(); ++i) pg.ops[i].M = ops[i].M;
+    const int box_rows = prefill_box_rows(pg);  // the plan the launch will run
     int tiles = 0;
     for (size_t i = 0; i < ops.size(); ++i) {
         PrefillOp &o = pg.ops[i];
-        cudaError_t e = prefill_x_map(&o.xmap, ops[i].x, ops[i].M, ops[i].K);
+        cudaError_t e = prefill_x_map_rows(&o.xmap, ops[i].x, ops[i].M, ops[i].K, box_rows);
         if (e != cudaSuccess) return cuda_fail(e, "tensor map for x");
         o.packed = ops[i].packed;
         o.scales = ops[i].scales;

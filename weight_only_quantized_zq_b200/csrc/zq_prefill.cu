@@ -19,10 +19,19 @@
 // A launch is one persistent grid (a CTA per SM) over all tiles of up to 64
 // independent ops of one bit width, handed out round-robin in op order (the
 // host puts the longest K first).
-// A 3-stage ring of (x, W) slabs is handed over with mbarriers; stage release is
+// A ring of (x, W) slabs is handed over with mbarriers; stage release is
 // tcgen05.commit.  Every wait is bounded: after ~2 s it raises an abort flag,
 // records ZQ_ERR_TIMEOUT in a device word and all roles drain and exit (TMEM
 // is always freed).
+//
+// Two shared-memory plans:
+//   * two token halves (a launch with some M > 128): 3 stages of
+//     (x 256 x 64, W 256 x 64); the dequant threads keep the codes, scales and
+//     zeros of the next group in registers;
+//   * one token half (every M <= 128, i.e. 17..128 tokens): the x stages hold
+//     128 tokens, and the space this frees becomes a ring of per-thread code
+//     slots that cp.async fills several groups ahead, so that enough weight
+//     bytes are in flight per SM to stream them at HBM speed.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -30,6 +39,7 @@
 
 #include "zq_device.cuh"
 #include "zq_internal.h"
+#include "zq_prefill.h"
 
 namespace zq {
 
@@ -40,8 +50,7 @@ namespace pf {
 constexpr int kTokTile = 256;   // tokens per CTA tile (two MMA halves of 128)
 constexpr int kRowTile = 256;   // weight rows per CTA tile (MMA N)
 constexpr int kBK = 64;         // K per slab
-constexpr int kStages = 3;
-constexpr int kSlabA = kTokTile * kBK * 2;  // 32 KB
+constexpr int kMaxStages = 3;
 constexpr int kSlabB = kRowTile * kBK * 2;  // 32 KB
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
@@ -52,17 +61,38 @@ constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
 constexpr int kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
 
-struct Smem {
-    uint8_t a[kStages][kSlabA];  // x slabs (TMA, SWIZZLE_128B)
-    uint8_t b[kStages][kSlabB];  // dequantized W slabs (SWIZZLE_128B)
-    unsigned long long full[kStages];
-    unsigned long long empty[kStages];
+struct Ctl {
+    unsigned long long full[kMaxStages];
+    unsigned long long empty[kMaxStages];
     unsigned long long acc_full;
     unsigned long long acc_empty;
     uint32_t tmem_base;
     int abort;
 };
-constexpr size_t kSmemBytes = sizeof(Smem) + 1024;  // + alignment slack
+
+// Shared-memory plan (byte offsets from a 1024-byte aligned base):
+//   [0, kOffB)          x slabs, kStages x kSlabA (TMA, SWIZZLE_128B)
+//   [kOffB, kOffCodes)  dequantized W slabs, kStages x kSlabB (SWIZZLE_128B)
+//   [kOffCodes, kOffCtl) code slots (one token half only): slot = one group
+//                       of the tile's 256 rows, laid out per thread (below),
+//                       then the 2 (scale | zero << 16) words of each thread
+//   [kOffCtl, ...)      barriers and flags
+template <int B, bool ONE>
+struct Plan {
+    static constexpr int kStages = (ONE && B == 8) ? 2 : 3;
+    static constexpr int kSlabA = (ONE ? kPrefillHalfTokens : kTokTile) * kBK * 2;
+    static constexpr int kSlots = !ONE ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
+    static constexpr int kSlotCodes = 256 * 4 * (4 * B);  // 256 threads x 4 chunks of 32 codes
+    static constexpr int kSlotBytes = kSlotCodes + 256 * 2 * 4;
+    static constexpr int kOffB = kStages * kSlabA;
+    static constexpr int kOffCodes = kOffB + kStages * kSlabB;
+    static constexpr int kOffCtl = kOffCodes + kSlots * kSlotBytes;
+    static constexpr size_t kBytes = kOffCtl + sizeof(Ctl) + 1024;  // + alignment slack
+    static_assert(kStages <= kMaxStages, "barrier arrays");
+    static_assert(kOffB % 1024 == 0 && kOffCodes % 1024 == 0, "SWIZZLE_128B stages need 1024-byte alignment");
+    static_assert(kBytes <= 232448, "227 KB of shared memory per CTA");
+    static_assert(!ONE || kSlots >= 3, "the scale/zero hand-off needs a prefetch distance of 2 groups");
+};
 
 // Bounded wait: false if the CTA is aborting or the limit was reached.
 __device__ __noinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *abort) {
@@ -200,17 +230,177 @@ __device__ __forceinline__ void load_chunk(uint32_t (&w)[B], const uint32_t *src
 }
 
 
+// cp.async of U bytes (16, 8 or 4) global -> shared.
+template <int U>
+__device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
+    if constexpr (U == 16) cp_async16(dst, src);
+    else if constexpr (U == 8) cp_async8(dst, src);
+    else cp_async4(dst, src);
+}
+
+// Dequant producer of the one-token-half plan.  Thread d (0..255) owns rows
+// d/2 and d/2 + 128 of the tile and the 32-code chunk d%2 of each slab, as in
+// the two-half plan, but its codes travel through a ring of kSlots shared-
+// memory slots filled by cp.async kSlots-1 groups ahead.  Within a slot each
+// thread's data is spread in U-byte units, unit u of thread d at
+// (u * 256 + d) * U, so the copies and the loads of a warp are contiguous.
+// Scales and zeros (2-byte aligned, too small for cp.async) are loaded into a
+// register set when their group's codes are issued and written to the slot
+// two groups later; the two register sets alternate, hence the loop below is
+// unrolled twice.
 template <int B>
+__device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb, uint8_t *scode, Ctl &c,
+                                             int d, int lane) {
+    using P = Plan<B, true>;
+    constexpr int kS = P::kSlots;
+    constexpr int PD = kS - 1;                        // groups in flight
+    constexpr int U = B == 3 ? 4 : B == 2 ? 8 : 16;   // bytes per copy
+    constexpr int UPC = 4 * B / U;                    // copies per 32-code chunk
+    const int n_tiles = p.n_tiles;
+    volatile int *abort = &c.abort;
+    const int ch = d & 1;
+
+    // Issue cursor: the group whose codes are copied next.
+    int tp = blockIdx.x, gp = 0, Gp = 0;
+    const uint32_t *prow[2] = {nullptr, nullptr};
+    const uint16_t *psr[2] = {nullptr, nullptr}, *pzr[2] = {nullptr, nullptr};
+    auto start_issue = [&]() {
+        if (tp < n_tiles) {
+            const TileRef tr = locate(p, tp);
+            const PrefillOp &op = p.ops[tr.o];
+            Gp = op.K / kGroup;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int r = min(tr.n0 + d / 2 + 128 * i, op.N - 1);
+                prow[i] = op.packed + static_cast<size_t>(r) * (static_cast<size_t>(op.K) * B / 32);
+                psr[i] = op.scales + static_cast<size_t>(r) * Gp;
+                pzr[i] = op.zeros + static_cast<size_t>(r) * Gp;
+            }
+        }
+    };
+    start_issue();
+    uint32_t szA[2] = {0u, 0u}, szB[2] = {0u, 0u};
+    // Group j of this CTA's sequence: first store the scale/zero words of
+    // group j - 2 (held in `set`) into its slot, then copy group j's codes into
+    // slot j % kS and load its scales and zeros into `set`.  Past the last
+    // group only the store and an empty commit remain, so that every group
+    // index commits exactly one cp.async group.
+    auto issue = [&](int j, uint32_t (&set)[2]) {
+        if (j >= 2) {
+            uint32_t *zs = reinterpret_cast<uint32_t *>(scode + ((j - 2) % kS) * P::kSlotBytes + P::kSlotCodes);
+            zs[d] = set[0];
+            zs[256 + d] = set[1];
+        }
+        if (tp < n_tiles) {
+            uint8_t *cs = scode + (j % kS) * P::kSlotBytes;
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint8_t *src = reinterpret_cast<const uint8_t *>(prow[i] + (4 * gp + 2 * h + ch) * B);
+#pragma unroll
+                    for (int u = 0; u < UPC; ++u)
+                        cp_async_u<U>(cs + (((2 * h + i) * UPC + u) * 256 + d) * U, src + u * U);
+                }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) set[i] = ldg_u16_nc(psr[i] + gp) | (ldg_u16_nc(pzr[i] + gp) << 16);
+            if (++gp == Gp) {
+                gp = 0;
+                tp += gridDim.x;
+                start_issue();
+            }
+        }
+        cp_async_commit();
+    };
+#pragma unroll
+    for (int j = 0; j + 1 < PD; j += 2) {  // group j uses register set j & 1
+        issue(j, szA);
+        issue(j + 1, szB);
+    }
+    if constexpr (PD & 1) issue(PD - 1, szA);
+
+    // Consume cursor: group i of tile t.
+    int t = blockIdx.x, g = 0, G = t < n_tiles ? p.ops[locate(p, t).o].K / kGroup : 0;
+    uint32_t it = 0;  // W stages filled so far
+    auto consume = [&](int i) -> bool {
+        cp_async_wait<PD>();               // this thread's copies of group i have landed
+        const uint32_t z = opaque_zero();  // orders the slot loads after the wait
+        const uint32_t cs = smem_u32(scode + (i % kS) * P::kSlotBytes) + z;
+        const uint32_t sz[2] = {lds_u32(cs + P::kSlotCodes + 4 * d), lds_u32(cs + P::kSlotCodes + 4 * (256 + d))};
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // the two slabs of this group
+            const int st = it % P::kStages;
+            const uint32_t round = it / P::kStages;
+            if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort)) return false;
+            uint8_t *bs = sb + st * kSlabB;
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                uint32_t w[B];
+#pragma unroll
+                for (int u = 0; u < UPC; ++u) {
+                    const uint32_t a = cs + (((2 * h + i) * UPC + u) * 256 + d) * U;
+                    if constexpr (U == 16) {
+                        const uint4 v = lds_v4(a);
+                        w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
+                    } else if constexpr (U == 8) {
+                        const uint2 v = lds_v2(a);
+                        w[2 * u] = v.x; w[2 * u + 1] = v.y;
+                    } else {
+                        w[u] = lds_u32(a);
+                    }
+                }
+                const int row = d / 2 + 128 * i;
+                uint32_t o[16];
+                dequant_chunk<B>(w, sz[i], o);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int c16 = (4 * ch + j) ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
+                        make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&c.full[st]);
+            ++it;
+        }
+        if (++g == G) {
+            g = 0;
+            t += gridDim.x;
+            if (t < n_tiles) G = p.ops[locate(p, t).o].K / kGroup;
+        }
+        return true;
+    };
+    uint32_t (&set_even)[2] = (PD & 1) ? szB : szA;  // register set of group i + PD, i even
+    uint32_t (&set_odd)[2] = (PD & 1) ? szA : szB;
+#pragma unroll 1
+    for (int i = 0;; i += 2) {
+        if (t >= n_tiles || *abort) break;
+        issue(i + PD, set_even);
+        if (!consume(i)) break;
+        if (t >= n_tiles || *abort) break;
+        issue(i + 1 + PD, set_odd);
+        if (!consume(i + 1)) break;
+    }
+    cp_async_wait<0>();  // no copy may land after the CTA has exited
+}
+
+template <int B, bool ONE>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillGroup p) {
+    using P = Plan<B, ONE>;
     extern __shared__ uint8_t smem_raw[];
-    Smem &sm = *reinterpret_cast<Smem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sa = base;                  // x slabs
+    uint8_t *sb = base + P::kOffB;       // W slabs
+    uint8_t *scode = base + P::kOffCodes;
+    Ctl &sm = *reinterpret_cast<Ctl *>(base + P::kOffCtl);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_tiles = p.n_tiles;
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < P::kStages; ++s) {
             mbar_init(&sm.full[s], 1 + kDqWarps);
             mbar_init(&sm.empty[s], 1);
         }
@@ -241,17 +431,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const PrefillOp &op = p.ops[tr.o];
                 const int slabs = op.K / kBK;
                 for (int s = 0; s < slabs; ++s, ++it) {
-                    const int st = it % kStages;
-                    const uint32_t round = it / kStages;
+                    const int st = it % P::kStages;
+                    const uint32_t round = it / P::kStages;
                     if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) break;
-                    mbar_arrive_expect_tx(&sm.full[st], kSlabA);
-                    tma_load_2d(sm.a[st], &op.xmap, s * kBK, tr.t0, &sm.full[st]);
+                    mbar_arrive_expect_tx(&sm.full[st], P::kSlabA);
+                    tma_load_2d(sa + st * P::kSlabA, &op.xmap, s * kBK, tr.t0, &sm.full[st]);
                 }
             }
             // Let copies still in flight land before the CTA can exit.
-            for (uint32_t k = 0; k < kStages && k < it; ++k) {
+            for (uint32_t k = 0; k < P::kStages && k < it; ++k) {
                 const uint32_t j = it - 1 - k;
-                mbar_wait(&sm.full[j % kStages], (j / kStages) & 1u, abort);
+                mbar_wait(&sm.full[j % P::kStages], (j / P::kStages) & 1u, abort);
             }
         }
     } else if (warp == kMmaWarp) {
@@ -261,26 +451,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const TileRef tr = locate(p, t);
                 const int slabs = p.ops[tr.o].K / kBK;
                 // the second 128-token half only when it holds tokens
-                const bool half1 = tr.t0 + 128 < p.ops[tr.o].M;
+                const bool half1 = !ONE && tr.t0 + 128 < p.ops[tr.o].M;
                 if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort)) break;
                 tc_fence_after();
                 bool ok = true;
                 for (int s = 0; s < slabs; ++s, ++it) {
-                    const int st = it % kStages;
-                    if (!mbar_wait(&sm.full[st], (it / kStages) & 1u, abort)) {
+                    const int st = it % P::kStages;
+                    if (!mbar_wait(&sm.full[st], (it / P::kStages) & 1u, abort)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(sm.a[st]);
-                    const uint32_t b0 = smem_u32(sm.b[st]);
+                    const uint32_t a0 = smem_u32(sa + st * P::kSlabA);
+                    const uint32_t b0 = smem_u32(sb + st * kSlabB);
                     if (half1) {
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk) {
                             const uint64_t bd = sdesc_sw128(b0 + kk * 32);
                             const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
                             umma_f16(tmem, sdesc_sw128(a0 + kk * 32), bd, acc);
-                            umma_f16(tmem + kRowTile, sdesc_sw128(a0 + kSlabA / 2 + kk * 32), bd, acc);
+                            umma_f16(tmem + kRowTile, sdesc_sw128(a0 + P::kSlabA / 2 + kk * 32), bd, acc);
                         }
                     } else {
 #pragma unroll
@@ -296,6 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
     } else if (warp >= kDqWarp0) {
+        if constexpr (ONE) {
+            dequant_ring<B>(p, sb, scode, sm, threadIdx.x - 32 * kDqWarp0, lane);
+        } else {
         // 256 threads: thread d owns rows d/2 and d/2 + 128 of the tile and the
         // 32-code chunk d%2 of every slab.  Codes, scales and zeros of the next
         // group (two slabs) are prefetched into registers.
@@ -354,13 +547,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (t_n < n_tiles) fetch(g_n);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // the two slabs of this group
-                const int st = it % kStages;
-                const uint32_t round = it / kStages;
+                const int st = it % P::kStages;
+                const uint32_t round = it / P::kStages;
                 if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) {
                     ok = false;
                     break;
                 }
-                uint8_t *bs = sm.b[st];
+                uint8_t *bs = sb + st * kSlabB;
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     const int row = d / 2 + 128 * i;
@@ -381,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             t = t_n;
             g = g_n;
             groups = groups_n;
+        }
         }
     } else {
         // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = tokens of each half.
@@ -437,41 +631,60 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 // ------------------------------------------------------------------ host --
 
-template <int B>
+template <int B, bool ONE>
 static cudaError_t launch_prefill_t(const PrefillGroup &pg, int n_ctas, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(pf::prefill_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(pf::kSmemBytes));
+    constexpr size_t smem = pf::Plan<B, ONE>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(pf::prefill_kernel<B, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
     cfg.blockDim = dim3(pf::kThreads);
-    cfg.dynamicSmemBytes = pf::kSmemBytes;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B>, pg);
+    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B, ONE>, pg);
 }
 
 cudaError_t prefill_x_map(CUtensorMap *map, const uint16_t *x, int M, int K) {
+    return prefill_x_map_rows(map, x, M, K, pf::kTokTile);
+}
+
+cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K, int box_rows) {
     return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, x, static_cast<uint64_t>(K),
-                                static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, pf::kBK, pf::kTokTile,
-                                CU_TENSOR_MAP_SWIZZLE_128B);
+                                static_cast<uint64_t>(M), static_cast<uint64_t>(K) * 2, pf::kBK,
+                                static_cast<uint32_t>(box_rows), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 int prefill_tiles(int M, int N) {
     return ((M + pf::kTokTile - 1) / pf::kTokTile) * ((N + pf::kRowTile - 1) / pf::kRowTile);
 }
 
+int prefill_box_rows(const PrefillGroup &pg) {
+    int max_m = 0;
+    for (int i = 0; i < pg.n_ops; ++i) max_m = pg.ops[i].M > max_m ? pg.ops[i].M : max_m;
+    return max_m <= kPrefillHalfTokens ? kPrefillHalfTokens : pf::kTokTile;
+}
+
 cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, cudaStream_t stream) {
     const int n_ctas = pg.n_tiles < num_sms ? pg.n_tiles : num_sms;
+    if (prefill_box_rows(pg) == kPrefillHalfTokens) {
+        switch (bits) {
+            case 2: return launch_prefill_t<2, true>(pg, n_ctas, stream);
+            case 3: return launch_prefill_t<3, true>(pg, n_ctas, stream);
+            case 4: return launch_prefill_t<4, true>(pg, n_ctas, stream);
+            default: return launch_prefill_t<8, true>(pg, n_ctas, stream);
+        }
+    }
     switch (bits) {
-        case 2: return launch_prefill_t<2>(pg, n_ctas, stream);
-        case 3: return launch_prefill_t<3>(pg, n_ctas, stream);
-        case 4: return launch_prefill_t<4>(pg, n_ctas, stream);
-        default: return launch_prefill_t<8>(pg, n_ctas, stream);
+        case 2: return launch_prefill_t<2, false>(pg, n_ctas, stream);
+        case 3: return launch_prefill_t<3, false>(pg, n_ctas, stream);
+        case 4: return launch_prefill_t<4, false>(pg, n_ctas, stream);
+        default: return launch_prefill_t<8, false>(pg, n_ctas, stream);
     }
 }
 
