@@ -13,7 +13,7 @@
 //   warp 4     TMA producer for x (2-D tensor map, SWIZZLE_128B) and TMEM owner;
 //   warp 5     MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
 //              for the two 128-token halves into 2 x 256 fp32 TMEM columns;
-//   warps 6-13 dequant producers: packed codes -> exact fp16 codes
+//   warps 6-13 (6-21 in the one-half plan) dequant producers: packed codes -> exact fp16 codes
 //              (zq_device.cuh) -> fp16(q*s + z) with one fused HFMA2 rounding ->
 //              K-order restored with PRMT -> UMMA K-major SWIZZLE_128B layout.
 // A launch is one persistent grid (a CTA per SM) over all tiles of up to 64
@@ -31,7 +31,8 @@
 //   * one token half (every M <= 128, i.e. 17..128 tokens): the x stages hold
 //     128 tokens, and the space this frees becomes a ring of per-thread code
 //     slots that cp.async fills several groups ahead, so that enough weight
-//     bytes are in flight per SM to stream them at HBM speed.
+//     bytes are in flight per SM; with the codes out of the registers, 16
+//     dequant warps fit, each owning one row chunk per slab.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -56,8 +57,6 @@ constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kDqWarp0 = 6;
-constexpr int kDqWarps = 8;
-constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
 constexpr int kTmemCols = 512;
 constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
 
@@ -79,11 +78,15 @@ struct Ctl {
 //   [kOffCtl, ...)      barriers and flags
 template <int B, bool ONE>
 struct Plan {
+    // Dequant warps: 16 in the one-half plan (its code ring keeps their
+    // registers low), 8 in the two-half plan (register prefetch).
+    static constexpr int kDqWarps = ONE ? 16 : 8;
+    static constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
     static constexpr int kStages = (ONE && B == 8) ? 2 : 3;
     static constexpr int kSlabA = (ONE ? kPrefillHalfTokens : kTokTile) * kBK * 2;
     static constexpr int kSlots = !ONE ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
-    static constexpr int kSlotCodes = 256 * 4 * (4 * B);  // 256 threads x 4 chunks of 32 codes
-    static constexpr int kSlotBytes = kSlotCodes + 256 * 2 * 4;
+    static constexpr int kSlotCodes = 1024 * (4 * B);  // 256 rows x 2 slabs x 2 chunks of 32 codes
+    static constexpr int kSlotBytes = kSlotCodes + 512 * 4;  // + a (scale | zero << 16) word per (row, chunk)
     static constexpr int kOffB = kStages * kSlabA;
     static constexpr int kOffCodes = kOffB + kStages * kSlabB;
     static constexpr int kOffCtl = kOffCodes + kSlots * kSlotBytes;
@@ -238,12 +241,13 @@ __device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
     else cp_async4(dst, src);
 }
 
-// Dequant producer of the one-token-half plan.  Thread d (0..255) owns rows
-// d/2 and d/2 + 128 of the tile and the 32-code chunk d%2 of each slab, as in
-// the two-half plan, but its codes travel through a ring of kSlots shared-
-// memory slots filled by cp.async kSlots-1 groups ahead.  Within a slot each
-// thread's data is spread in U-byte units, unit u of thread d at
-// (u * 256 + d) * U, so the copies and the loads of a warp are contiguous.
+// Dequant producer of the one-token-half plan.  Its NT threads own the 512
+// (row, chunk) pairs of each slab, pair q = d + NT * r (r < 512 / NT) of
+// thread d being row (q % 256) / 2 + 128 * (q / 256), 32-code chunk q % 2 --
+// the two-half plan's assignment when NT = 256.  Codes travel through a ring
+// of kSlots shared-memory slots filled by cp.async kSlots - 1 groups ahead.
+// Within a slot each thread's data is spread in U-byte units, unit u of thread
+// d at (u * NT + d) * U, so the copies and the loads of a warp are contiguous.
 // Scales and zeros (2-byte aligned, too small for cp.async) are loaded into a
 // register set when their group's codes are issued and written to the slot
 // two groups later; the two register sets alternate, hence the loop below is
@@ -252,58 +256,69 @@ template <int B>
 __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb, uint8_t *scode, Ctl &c,
                                              int d, int lane) {
     using P = Plan<B, true>;
+    constexpr int NT = 32 * P::kDqWarps;
+    constexpr int RPT = 512 / NT;                     // rows per thread
     constexpr int kS = P::kSlots;
     constexpr int PD = kS - 1;                        // groups in flight
     constexpr int U = B == 3 ? 4 : B == 2 ? 8 : 16;   // bytes per copy
     constexpr int UPC = 4 * B / U;                    // copies per 32-code chunk
+    static_assert(RPT * NT == 512, "thread count");
     const int n_tiles = p.n_tiles;
     volatile int *abort = &c.abort;
     const int ch = d & 1;
+    int rows[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) {
+        const int q = d + NT * r;
+        rows[r] = (q % 256) / 2 + 128 * (q / 256);
+    }
 
     // Issue cursor: the group whose codes are copied next.
     int tp = blockIdx.x, gp = 0, Gp = 0;
-    const uint32_t *prow[2] = {nullptr, nullptr};
-    const uint16_t *psr[2] = {nullptr, nullptr}, *pzr[2] = {nullptr, nullptr};
+    const uint32_t *prow[RPT];
+    const uint16_t *psr[RPT], *pzr[RPT];
     auto start_issue = [&]() {
         if (tp < n_tiles) {
             const TileRef tr = locate(p, tp);
             const PrefillOp &op = p.ops[tr.o];
             Gp = op.K / kGroup;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int r = min(tr.n0 + d / 2 + 128 * i, op.N - 1);
-                prow[i] = op.packed + static_cast<size_t>(r) * (static_cast<size_t>(op.K) * B / 32);
-                psr[i] = op.scales + static_cast<size_t>(r) * Gp;
-                pzr[i] = op.zeros + static_cast<size_t>(r) * Gp;
+            for (int r = 0; r < RPT; ++r) {
+                const int n = min(tr.n0 + rows[r], op.N - 1);
+                prow[r] = op.packed + static_cast<size_t>(n) * (static_cast<size_t>(op.K) * B / 32);
+                psr[r] = op.scales + static_cast<size_t>(n) * Gp;
+                pzr[r] = op.zeros + static_cast<size_t>(n) * Gp;
             }
         }
     };
     start_issue();
-    uint32_t szA[2] = {0u, 0u}, szB[2] = {0u, 0u};
+    uint32_t szA[RPT], szB[RPT];
+#pragma unroll
+    for (int r = 0; r < RPT; ++r) szA[r] = szB[r] = 0u;
     // Group j of this CTA's sequence: first store the scale/zero words of
     // group j - 2 (held in `set`) into its slot, then copy group j's codes into
     // slot j % kS and load its scales and zeros into `set`.  Past the last
     // group only the store and an empty commit remain, so that every group
     // index commits exactly one cp.async group.
-    auto issue = [&](int j, uint32_t (&set)[2]) {
+    auto issue = [&](int j, uint32_t (&set)[RPT]) {
         if (j >= 2) {
             uint32_t *zs = reinterpret_cast<uint32_t *>(scode + ((j - 2) % kS) * P::kSlotBytes + P::kSlotCodes);
-            zs[d] = set[0];
-            zs[256 + d] = set[1];
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) zs[r * NT + d] = set[r];
         }
         if (tp < n_tiles) {
             uint8_t *cs = scode + (j % kS) * P::kSlotBytes;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const uint8_t *src = reinterpret_cast<const uint8_t *>(prow[i] + (4 * gp + 2 * h + ch) * B);
+                for (int r = 0; r < RPT; ++r) {
+                    const uint8_t *src = reinterpret_cast<const uint8_t *>(prow[r] + (4 * gp + 2 * h + ch) * B);
 #pragma unroll
                     for (int u = 0; u < UPC; ++u)
-                        cp_async_u<U>(cs + (((2 * h + i) * UPC + u) * 256 + d) * U, src + u * U);
+                        cp_async_u<U>(cs + (((h * RPT + r) * UPC + u) * NT + d) * U, src + u * U);
                 }
 #pragma unroll
-            for (int i = 0; i < 2; ++i) set[i] = ldg_u16_nc(psr[i] + gp) | (ldg_u16_nc(pzr[i] + gp) << 16);
+            for (int r = 0; r < RPT; ++r) set[r] = ldg_u16_nc(psr[r] + gp) | (ldg_u16_nc(pzr[r] + gp) << 16);
             if (++gp == Gp) {
                 gp = 0;
                 tp += gridDim.x;
@@ -326,7 +341,9 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         cp_async_wait<PD>();               // this thread's copies of group i have landed
         const uint32_t z = opaque_zero();  // orders the slot loads after the wait
         const uint32_t cs = smem_u32(scode + (i % kS) * P::kSlotBytes) + z;
-        const uint32_t sz[2] = {lds_u32(cs + P::kSlotCodes + 4 * d), lds_u32(cs + P::kSlotCodes + 4 * (256 + d))};
+        uint32_t sz[RPT];
+#pragma unroll
+        for (int r = 0; r < RPT; ++r) sz[r] = lds_u32(cs + P::kSlotCodes + 4 * (r * NT + d));
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // the two slabs of this group
             const int st = it % P::kStages;
@@ -334,11 +351,11 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
             if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort)) return false;
             uint8_t *bs = sb + st * kSlabB;
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int r = 0; r < RPT; ++r) {
                 uint32_t w[B];
 #pragma unroll
                 for (int u = 0; u < UPC; ++u) {
-                    const uint32_t a = cs + (((2 * h + i) * UPC + u) * 256 + d) * U;
+                    const uint32_t a = cs + (((h * RPT + r) * UPC + u) * NT + d) * U;
                     if constexpr (U == 16) {
                         const uint4 v = lds_v4(a);
                         w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
@@ -349,9 +366,9 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                         w[u] = lds_u32(a);
                     }
                 }
-                const int row = d / 2 + 128 * i;
+                const int row = rows[r];
                 uint32_t o[16];
-                dequant_chunk<B>(w, sz[i], o);
+                dequant_chunk<B>(w, sz[r], o);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c16 = (4 * ch + j) ^ (row & 7);
@@ -371,8 +388,8 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         }
         return true;
     };
-    uint32_t (&set_even)[2] = (PD & 1) ? szB : szA;  // register set of group i + PD, i even
-    uint32_t (&set_odd)[2] = (PD & 1) ? szA : szB;
+    uint32_t (&set_even)[RPT] = (PD & 1) ? szB : szA;  // register set of group i + PD, i even
+    uint32_t (&set_odd)[RPT] = (PD & 1) ? szA : szB;
 #pragma unroll 1
     for (int i = 0;; i += 2) {
         if (t >= n_tiles || *abort) break;
@@ -386,7 +403,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
 }
 
 template <int B, bool ONE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillGroup p) {
     using P = Plan<B, ONE>;
     extern __shared__ uint8_t smem_raw[];
@@ -401,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P::kStages; ++s) {
-            mbar_init(&sm.full[s], 1 + kDqWarps);
+            mbar_init(&sm.full[s], 1 + P::kDqWarps);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
@@ -639,7 +656,7 @@ static cudaError_t launch_prefill_t(const PrefillGroup &pg, int n_ctas, cudaStre
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
-    cfg.blockDim = dim3(pf::kThreads);
+    cfg.blockDim = dim3(pf::Plan<B, ONE>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
