@@ -60,6 +60,12 @@ MEASURED_TRAFFIC = {
         "bytes_per_layer": 125936384,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },
+    # tile kernel, one-token-half plan: a one-layer launch at M = 64
+    ("prefill", "7b", 64): {
+        "sha256": "4a2d190753ffe71ee91d1e03900814d66a2c8e425b631bafac7bff6246456468",
+        "bytes_per_layer": 130899200,
+        "profile": "profiles/prefill_kernel_m64_1layer.md",
+    },
 }
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
@@ -390,15 +396,20 @@ def run_zq(args):
     # kernel.  Prefill (M > 64): the grouped tcgen05 launches.
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
     bits_used = sorted({b for (*_, b) in decode_stack_shapes(args.layers, args.model)}, reverse=True)
+    # The tile kernel's shared-memory plan: one token half when every M <= 128.
+    tile_kernel = ("prefill_kernel<" + "|".join(str(b) for b in bits_used)
+                   + (",true> (one-token-half plan)" if M <= 128 else ",false> (two-token-half plan)"))
     if M <= 64:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": measured_traffic("decode", args.model, M, args.layers),
+                    "traffic": measured_traffic("decode" if M <= 16 else "prefill", args.model, M, args.layers),
+                    "traffic_note": ("per step (one decode launch)" if M <= 16 else
+                                     "per step (the stack's grouped tile-kernel launches)"),
                     "algorithmic_bytes": wl.bytes,
                     "peak_source": peaks["source"],
                     "kernel": (f"decode_kernel<{'|'.join(str(b) for b in bits_used)},{zq_mt(M)}> + prep_kernel"
                                + (" (one launch pair per bit width)" if len(bits_used) > 1 else "")
-                               if M <= 16 else "prefill_kernel<" + "|".join(str(b) for b in bits_used) + ">")}
+                               if M <= 16 else tile_kernel)}
     else:
         tflops = wl.flops / (ms_step / 1e3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
@@ -409,7 +420,7 @@ def run_zq(args):
                     "traffic_note": "per launch, averaged over the 4 projections of a layer",
                     "algorithmic_flops": wl.flops,
                     "peak_source": peaks["source"] + " (dense bf16 sustained; fp16 has the same dense rate)",
-                    "kernel": "prefill_kernel<" + "|".join(str(b) for b in bits_used) + ">",
+                    "kernel": tile_kernel,
                     "tflops_vs_nominal_2250": tflops / 2250.0}
 
     line = None
