@@ -105,6 +105,22 @@ def test_quantize_rejects(zq, name):
     assert q(A, 4, 256, 4, 128, A, A, 0, None) == zq.ZQ_ERR_INVALID_ARG
 
 
+def test_kv_plane_bytes_and_rejects(zq):
+    # ring 256 x 4 x 128 fp16 + store 4096 x 4 x (64 code bytes) + 2 x 4096 x 4 x 2 (scales, zeros)
+    assert zq.zq_kv_plane_bytes(256, 4096, 4, 128, 4) == 262144 + 1048576 + 2 * 32768
+    assert zq.zq_kv_plane_bytes(256, 4096, 4, 100, 4) == 0
+    assert zq.zq_kv_plane_bytes(256, 4096, 4, 128, 5) == 0
+    pl = zq.zq_kv_plane(A, A, A, A, 8, 8, 1, 128, 4)
+    assert zq._lib.zq_kv_append(ctypes.byref(pl), 5, A, 4, None) == zq.ZQ_ERR_INVALID_ARG  # past capacity
+    assert zq._lib.zq_kv_append(ctypes.byref(pl), 0, A + 2, 1, None) == zq.ZQ_ERR_INVALID_ARG  # misaligned
+    assert zq._lib.zq_kv_append(ctypes.byref(pl), 0, A, 0, None) == zq.ZQ_OK  # nothing to do
+    assert zq._lib.zq_kv_gather(ctypes.byref(pl), 4, 3, 5, A, None) == zq.ZQ_ERR_INVALID_ARG
+    assert zq._lib.zq_kv_gather(ctypes.byref(pl), 4, 2, 2, A, None) == zq.ZQ_OK
+    bad = zq.zq_kv_plane(A, A, A, A, 8, 8, 1, 128, 6)
+    assert zq._lib.zq_kv_append(ctypes.byref(bad), 0, A, 1, None) == zq.ZQ_ERR_UNSUPPORTED
+    assert zq._lib.zq_kv_append(None, 0, A, 1, None) == zq.ZQ_ERR_INVALID_ARG
+
+
 def test_unpack_rejects(zq):
     u = zq._lib.zq_unpack
     assert u(A, 4, 256, 6, A, None) == zq.ZQ_ERR_UNSUPPORTED

@@ -31,7 +31,8 @@ EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_quantize_pack_symmetric", 
            "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
            "zq_version",
            "zq_zse_open", "zq_zse_close", "zq_zse_flags", "zq_zse_tensor_count", "zq_zse_tensor_info",
-           "zq_zse_find", "zq_zse_section", "zq_zse_weight_bytes", "zq_zse_verify", "zq_zse_load_weights")
+           "zq_zse_find", "zq_zse_section", "zq_zse_weight_bytes", "zq_zse_verify", "zq_zse_load_weights",
+           "zq_kv_plane_bytes", "zq_kv_append", "zq_kv_gather")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -107,6 +108,19 @@ _lib.zq_zse_tensor_info.argtypes = [_P, _I, ctypes.POINTER(zq_zse_tensor)]
 _lib.zq_zse_tensor_info.restype = _I
 
 
+class zq_kv_plane(ctypes.Structure):
+    _fields_ = [("ring", _P), ("packed", _P), ("scales", _P), ("zeros", _P), ("window", _I),
+                ("capacity", _I), ("heads", _I), ("dim", _I), ("bits", _I)]
+
+
+_lib.zq_kv_plane_bytes.argtypes = [_I, _I, _I, _I, _I]
+_lib.zq_kv_plane_bytes.restype = _S
+_lib.zq_kv_append.argtypes = [ctypes.POINTER(zq_kv_plane), _I, _P, _I, _P]
+_lib.zq_kv_append.restype = _I
+_lib.zq_kv_gather.argtypes = [ctypes.POINTER(zq_kv_plane), _I, _I, _I, _P, _P]
+_lib.zq_kv_gather.restype = _I
+
+
 class zq_linear_desc(ctypes.Structure):
     _fields_ = [("x", _P), ("packed", _P), ("scales", _P), ("zeros", _P), ("out", _P),
                 ("bits", _I), ("group", _I), ("M", _I), ("N", _I), ("K", _I)]
@@ -144,6 +158,10 @@ def zq_last_error():
 
 def zq_version():
     return _lib.zq_version()
+
+
+def zq_kv_plane_bytes(window, capacity, heads, dim, bits):
+    return _lib.zq_kv_plane_bytes(window, capacity, heads, dim, bits)
 
 
 def zq_check_device():
@@ -244,6 +262,38 @@ def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
 # ------------------------------------------------------------ .zse reader --
 
 ZSE_CONFIG, ZSE_TOKENIZER, ZSE_WEIGHT_INDEX, ZSE_WEIGHT_DATA, ZSE_KERNELS = 1, 2, 3, 4, 5
+
+
+class KVPlane:
+    """One K or V plane of the quantized KV cache (zq_kv.h): the newest
+    `window` tokens in an fp16 ring, older ones quantized at `bits` in the
+    store.  Owns its device buffers; `tokens` counts what it holds."""
+
+    def __init__(self, window, capacity, heads, dim, bits=4, device="cuda"):
+        if zq_kv_plane_bytes(window, capacity, heads, dim, bits) == 0:
+            raise ZQError(ZQ_ERR_INVALID_ARG, f"bad plane shape {(window, capacity, heads, dim, bits)}")
+        self.ring = torch.empty(window, heads, dim, dtype=torch.float16, device=device)
+        self.packed = torch.empty(capacity, heads, dim * bits // 32, dtype=torch.int32, device=device)
+        self.scales = torch.empty(capacity, heads, dim // GROUP, dtype=torch.int16, device=device)
+        self.zeros = torch.empty(capacity, heads, dim // GROUP, dtype=torch.int16, device=device)
+        self.desc = zq_kv_plane(_ptr(self.ring), _ptr(self.packed), _ptr(self.scales), _ptr(self.zeros),
+                                window, capacity, heads, dim, bits)
+        self.window, self.capacity, self.heads, self.dim, self.bits = window, capacity, heads, dim, bits
+        self.tokens = 0
+
+    def append(self, rows, stream=None):
+        """rows: fp16 CUDA tensor (n, heads, dim)."""
+        n = rows.shape[0]
+        _check(_lib.zq_kv_append(ctypes.byref(self.desc), self.tokens, _ptr(rows), n, _stream(stream, rows)))
+        self.tokens += n
+
+    def gather(self, a=0, b=None, out=None, stream=None):
+        """Tokens [a, b) as an fp16 tensor (b - a, heads, dim)."""
+        b = self.tokens if b is None else b
+        if out is None:
+            out = torch.empty(max(b - a, 0), self.heads, self.dim, dtype=torch.float16, device=self.ring.device)
+        _check(_lib.zq_kv_gather(ctypes.byref(self.desc), self.tokens, a, b, _ptr(out), _stream(stream, out)))
+        return out
 
 
 class ZseFile:

@@ -17,6 +17,7 @@
 #include <vector>
 
 #include "zq.h"
+#include "zq_kv.h"
 #include "zq_internal.h"
 #include "zq_prefill.h"
 #include "zq_quant.h"
@@ -718,13 +719,74 @@ uint64_t zq_kernel_launches(void) { return g_launches.load(); }
 zq_status zq_check_device(void) {
     cudaError_t e = cudaDeviceSynchronize();
     if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
-    int err = 0, err2 = 0;
+    int err = 0, err2 = 0, err3 = 0;
     e = read_prefill_error(&err);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     e = read_decode_error(&err2);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    e = read_kv_error(&err3);
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     if (err != 0 || err2 != 0)
         return fail(static_cast<zq_status>(err ? err : err2), "a kernel gave up a bounded wait");
+    if (err3 != 0) return fail(static_cast<zq_status>(err3), "a KV-cache row held NaN or Inf");
+    return ZQ_OK;
+}
+
+// ------------------------------------------------------------------ zKV --
+
+static size_t round256(size_t v) { return (v + 255) / 256 * 256; }
+
+size_t zq_kv_plane_bytes(int window, int capacity, int heads, int dim, int bits) {
+    if (window < 1 || capacity < 1 || heads < 1 || dim < 128 || dim % 128 != 0) return 0;
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8)) return 0;
+    const size_t hr = static_cast<size_t>(capacity) * heads;  // (token, head) rows of the store
+    return round256(static_cast<size_t>(window) * heads * dim * 2) + round256(hr * dim * bits / 8) +
+           2 * round256(hr * (dim / 128) * 2);
+}
+
+static zq_status check_plane(const zq_kv_plane *pl, KvArgs *a) {
+    if (pl == nullptr) return fail(ZQ_ERR_INVALID_ARG, "plane is NULL");
+    if (!(pl->bits == 2 || pl->bits == 3 || pl->bits == 4 || pl->bits == 8))
+        return fail(ZQ_ERR_UNSUPPORTED, "plane bits must be 2, 3, 4 or 8 (got %d)", pl->bits);
+    if (pl->window < 1 || pl->capacity < 1 || pl->heads < 1 || pl->dim < 128 || pl->dim % 128 != 0)
+        return fail(ZQ_ERR_INVALID_ARG, "plane shape: window=%d capacity=%d heads=%d dim=%d (dim a multiple of 128)",
+                    pl->window, pl->capacity, pl->heads, pl->dim);
+    zq_status st;
+    if ((st = check_ptr(pl->ring, "ring")) != ZQ_OK) return st;
+    if ((st = check_ptr(pl->packed, "packed")) != ZQ_OK) return st;
+    if ((st = check_ptr(pl->scales, "scales")) != ZQ_OK) return st;
+    if ((st = check_ptr(pl->zeros, "zeros")) != ZQ_OK) return st;
+    *a = KvArgs{pl->ring, pl->packed, pl->scales, pl->zeros, pl->window, pl->heads, pl->dim, pl->bits};
+    return ZQ_OK;
+}
+
+zq_status zq_kv_append(const zq_kv_plane *plane, int t0, const uint16_t *rows, int n, zq_stream_t stream) {
+    KvArgs a;
+    zq_status st = check_plane(plane, &a);
+    if (st != ZQ_OK) return st;
+    if (t0 < 0 || n < 0 || static_cast<long long>(t0) + n > plane->capacity)
+        return fail(ZQ_ERR_INVALID_ARG, "append of %d tokens to %d: capacity is %d", n, t0, plane->capacity);
+    if (n == 0) return ZQ_OK;
+    if ((st = check_ptr(rows, "rows")) != ZQ_OK) return st;
+    cudaError_t e = launch_kv_append(a, rows, t0, n, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kv append launch");
+    ++g_launches;
+    return ZQ_OK;
+}
+
+zq_status zq_kv_gather(const zq_kv_plane *plane, int t_total, int a_tok, int b_tok, uint16_t *out,
+                       zq_stream_t stream) {
+    KvArgs a;
+    zq_status st = check_plane(plane, &a);
+    if (st != ZQ_OK) return st;
+    if (!(0 <= a_tok && a_tok <= b_tok && b_tok <= t_total && t_total <= plane->capacity))
+        return fail(ZQ_ERR_INVALID_ARG, "gather [%d, %d) of %d tokens (capacity %d)", a_tok, b_tok, t_total,
+                    plane->capacity);
+    if (a_tok == b_tok) return ZQ_OK;
+    if ((st = check_ptr(out, "out")) != ZQ_OK) return st;
+    cudaError_t e = launch_kv_gather(a, t_total, a_tok, b_tok, out, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "kv gather launch");
+    ++g_launches;
     return ZQ_OK;
 }
 

@@ -23,16 +23,13 @@
 #include "zq_device.cuh"
 #include "zq_internal.h"
 #include "zq_quant.h"
+#include "zq_quant_warp.cuh"
 
 namespace zq {
 
 // Per-call status words for the non-finite check.  A call owns one slot, keyed
 // by a unique call id, so no clearing is needed between calls.
 __device__ unsigned long long g_quant_status[kQuantStatusSlots];
-
-__device__ __forceinline__ uint16_t f64_to_f16_bits(double v) {
-    return __half_as_ushort(__double2half(v));
-}
 
 // One warp per (row, group).  Each lane owns 4 consecutive weights.
 template <bool SYMMETRIC>
@@ -46,72 +43,16 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
     const long long item = static_cast<long long>(blockIdx.x) * 8 + warp;
     if (item >= static_cast<long long>(N) * G) return;
     const int n = static_cast<int>(item / G), g = static_cast<int>(item % G);
-    const int L = (1 << bits) - 1;
 
     const float4 v4 = *reinterpret_cast<const float4 *>(w + static_cast<size_t>(n) * K +
                                                         static_cast<size_t>(g) * 128 + lane * 4);
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
-    bool bad = false;
-    float mn = v[0], mx = v[0];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        bad |= !(fabsf(v[i]) <= 65504.0f);  // NaN compares false
-        mn = fminf(mn, v[i]);
-        mx = fmaxf(mx, v[i]);
-    }
-    if (__any_sync(0xffffffffu, bad)) {
+    uint16_t s16, z16;
+    if (!quantize_group_warp<SYMMETRIC>(v, bits, lane, words[warp], s16, z16)) {
         if (lane == 0) atomicExch(&g_quant_status[slot], call_id);
         return;
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-    }
-    uint16_t s16, z16;
-    uint32_t chunk = 0;  // this lane's 4 codes, 4*bits bits
-    if constexpr (SYMMETRIC) {
-        const double half = static_cast<double>(1 << (bits - 1)), Q = half - 1.0;
-        s16 = f64_to_f16_bits(__ddiv_rn(static_cast<double>(fmaxf(-mn, mx)), Q));
-        const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
-        const double z = __dmul_rn(-half, s);
-        if (z < -65504.0) {  // the zero would not be a finite fp16 (uniform across the warp)
-            if (lane == 0) atomicExch(&g_quant_status[slot], call_id);
-            return;
-        }
-        z16 = f64_to_f16_bits(z);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            double t = 0.0;
-            if (s != 0.0) t = fmin(fmax(rint(__ddiv_rn(static_cast<double>(v[i]), s)), -Q), Q);
-            chunk |= static_cast<uint32_t>(t + half) << (bits * i);
-        }
-    } else {
-        z16 = f64_to_f16_bits(static_cast<double>(mn));
-        s16 = f64_to_f16_bits(
-            __ddiv_rn(__dsub_rn(static_cast<double>(mx), static_cast<double>(mn)), static_cast<double>(L)));
-        const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
-        const double z = static_cast<double>(__half2float(__ushort_as_half(z16)));
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            uint32_t q = 0;
-            if (s != 0.0) {
-                double t = rint(__ddiv_rn(__dsub_rn(static_cast<double>(v[i]), z), s));
-                t = fmin(fmax(t, 0.0), static_cast<double>(L));
-                q = static_cast<uint32_t>(t);
-            }
-            chunk |= q << (bits * i);
-        }
-    }
-    // Assemble the group's 4*bits words: lane's chunk starts at stream bit 4*bits*lane.
     const int nw = 4 * bits;
-    if (lane < nw) words[warp][lane] = 0;
-    __syncwarp();
-    const int bit0 = 4 * bits * lane;
-    const int wi = bit0 >> 5, off = bit0 & 31;
-    atomicOr(&words[warp][wi], chunk << off);
-    if (off + 4 * bits > 32) atomicOr(&words[warp][wi + 1], chunk >> (32 - off));
-    __syncwarp();
     const size_t wpr = static_cast<size_t>(K) * bits / 32;
     if (lane < nw) packed[static_cast<size_t>(n) * wpr + static_cast<size_t>(g) * nw + lane] = words[warp][lane];
     if (lane == 0) {
