@@ -46,8 +46,8 @@ METRIC = "quantized-linear HBM GB/s (% of 8 TB/s) at M=1; tokens/s-equiv per lay
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of the dominant
 # kernel, per layer of the stack, from one ncu capture of a 4-layer stack
 # (traffic grows in proportion to the layers).  Keyed by the SHA-256 of the
-# kernel's sources at capture time: once they change the figure is stale and
-# the roofline reports null.
+# kernel's code (sources without comments) at capture time: once the code
+# changes the figure is stale and the roofline reports null.
 CSRC = os.path.join(ROOT, "weight_only_quantized_zq_b200", "csrc")
 KERNEL_SOURCES = {
     "decode": ("zq_decode.cu", "zq_device.cuh", "zq_internal.h"),
@@ -56,13 +56,13 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {
-        "sha256": "5512377e1a34955ab1b352556eaa33c0c5361bdafa91cda6f12565a167d3f631",
+        "sha256": "de5ba2b057c180a01e9bb424bb070c58dd692ae81c675a7a034337d946fed283",
         "bytes_per_layer": 125936384,
         "profile": "profiles/decode_kernel_m1_4layers.md",
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
-        "sha256": "4a2d190753ffe71ee91d1e03900814d66a2c8e425b631bafac7bff6246456468",
+        "sha256": "260f2fe4c7aa0f6d088d2e6e869092dca1d8734c3b4b93f72061af7d315bb0e1",
         "bytes_per_layer": 130899200,
         "profile": "profiles/prefill_kernel_m64_1layer.md",
     },
@@ -176,12 +176,44 @@ class ClockSampler:
                 "samples": len(self.samples), "source": "nvml"}
 
 
+def strip_comments(src):
+    """C/C++/CUDA source without its comments, each comment replaced by one
+    space, string and character literals kept as they are."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+            out.append(" ")
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return "".join(out)
+
+
 def kernel_sha256(family):
+    """SHA-256 of the kernel family's code: its sources with comments removed
+    and whitespace runs collapsed, so that a comment edit keeps a capture's
+    traffic valid and any change to the code does not."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[family]:
-        with open(os.path.join(CSRC, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(CSRC, name), encoding="utf-8") as f:
+            code = re.sub(r"\s+", " ", strip_comments(f.read())).strip()
+        h.update(code.encode("utf-8"))
+        h.update(b"\0")
     return h.hexdigest()
 
 

@@ -71,3 +71,17 @@ def test_reference_arm_non_zero_rank_exits_without_work(monkeypatch):
     assert rc == 0
     assert buf.getvalue() == ""
     assert called == []
+
+
+def test_traffic_key_ignores_comments_only():
+    """The bench keys a captured DRAM traffic figure by a hash of the kernel's
+    code: comments and whitespace do not change it, code does, and string
+    literals that look like comments are code."""
+    import bench
+    src = 'int a = 1; // note\n/* block\n comment */ const char *s = "x//y /* z */";\nchar q = \'\\\'\';\n'
+    assert bench.strip_comments(src).split() == ["int", "a", "=", "1;", "const", "char", "*s", "=",
+                                                 '"x//y', "/*", 'z', '*/";', "char", "q", "=", "'\\'';"]
+    assert bench.strip_comments("a /* unterminated") == "a  "
+    assert bench.strip_comments("b // to the end") == "b  "
+    h = bench.kernel_sha256("decode")
+    assert len(h) == 64 and h == bench.kernel_sha256("decode")

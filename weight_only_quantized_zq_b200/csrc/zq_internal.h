@@ -112,11 +112,11 @@ cudaError_t launch_unpack(const uint32_t *packed, int N, int K, int bits, uint8_
 
 // ---------------------------------------------------------------- prefill --
 // A prefill launch runs up to kMaxPrefillOps independent ops of one bit width
-// as one persistent grid over all their 256 x 256 output tiles.
+// as one persistent grid over all their 256-token x 256-row output tiles.
 constexpr int kMaxPrefillOps = 64;
 
 struct alignas(64) PrefillOp {
-    CUtensorMap xmap;  // x (M x K fp16): 64 k x 256 tokens per box, 128-byte swizzle
+    CUtensorMap xmap;  // x (M x K fp16): 64 k x 256 (one-half plan: 128) tokens per box, 128-byte swizzle
     const uint32_t *packed;
     const uint16_t *scales;
     const uint16_t *zeros;
