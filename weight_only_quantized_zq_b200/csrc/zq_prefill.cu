@@ -13,9 +13,10 @@
 //   warp 4     TMA producer for x (2-D tensor map, SWIZZLE_128B) and TMEM owner;
 //   warp 5     MMA issuer: one thread issues tcgen05.mma (M=128, N=256, K=16)
 //              for the two 128-token halves into 2 x 256 fp32 TMEM columns;
-//   warps 6-13 (6-21 in the one-half plan) dequant producers: packed codes -> exact fp16 codes
-//              (zq_device.cuh) -> fp16(q*s + z) with one fused HFMA2 rounding ->
-//              K-order restored with PRMT -> UMMA K-major SWIZZLE_128B layout.
+//   warps 6-13 dequant producers (6-21 in the one-half plan): packed codes ->
+//              exact fp16 codes (zq_device.cuh) -> fp16(q*s + z) with one
+//              fused HFMA2 rounding -> K-order restored with PRMT -> UMMA
+//              K-major SWIZZLE_128B layout.
 // A launch is one persistent grid (a CTA per SM) over all tiles of up to 64
 // independent ops of one bit width, handed out round-robin in op order (the
 // host puts the longest K first).
@@ -74,7 +75,7 @@ struct Ctl {
 //   [kOffB, kOffCodes)  dequantized W slabs, kStages x kSlabB (SWIZZLE_128B)
 //   [kOffCodes, kOffCtl) code slots (one token half only): slot = one group
 //                       of the tile's 256 rows, laid out per thread (below),
-//                       then the 2 (scale | zero << 16) words of each thread
+//                       then one (scale | zero << 16) word per (row, chunk)
 //   [kOffCtl, ...)      barriers and flags
 template <int B, bool ONE>
 struct Plan {
