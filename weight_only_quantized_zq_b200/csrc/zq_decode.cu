@@ -22,12 +22,14 @@
 //    1024 * sum(x') is subtracted in fp32 once per group.  The canonical packed
 //    layout is consumed as stored.
 //  * A CTA step is 64 weight rows x GPS groups.  One ring of shared-memory
-//    stages per CTA: warp 0 produces (one TMA 2-D copy per 128-byte column of
-//    the codes, with the 128-byte swizzle so the fragment loads are free of
-//    bank conflicts; bulk copies of the step's activations and group sums;
-//    one cp.async per lane for scales and zeros) and all four warps consume,
-//    each 16 of the rows.  A step descriptor travels in the stage, so the
-//    consumers keep no scheduling state.
+//    stages per CTA, filled in turn by the four warps (stage t by warp t % 4,
+//    the scheduling state handed from one producing warp to the next through
+//    shared memory): one TMA 2-D copy per 128-byte column of the codes, with
+//    the 128-byte swizzle so the fragment loads are free of bank conflicts
+//    (one unswizzled 208-byte box at b = 3); bulk copies of the step's
+//    activations and group sums; cp.async for scales and zeros.  All four
+//    warps consume, each 16 of the rows.  A step descriptor travels in the
+//    stage, so the consumers keep no scheduling state.
 //  * A persistent grid covers every SM.  The steps of all ops of a launch are
 //    cut into chunks: whole row blocks (large launches, longest first) or
 //    2^c consecutive steps (small launches, split along K).  A CTA starts with
