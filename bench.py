@@ -290,7 +290,8 @@ def workload_config(M, layers, world, model="7b"):
     return {"workload": f"{shaped} {'decode' if M <= 64 else 'prefill'} stack: "
                         f"{layers} layers x (qkv, o, gate_up, down), M={M}, {fmt}, "
                         f"one zq_linear_stack call",
-            "model": model, "layers": layers, "M": M,
+            "layer_shapes": ", ".join(f"{name} {N}x{K} INT{b}" for (name, N, K, b) in MODELS[model][0]),
+            "layers": layers, "M": M,
             "bits": sorted({b for (*_, b) in shapes}), "group": 128,
             "bytes_per_step": nbytes,
             "flops_per_step": sum(2 * M * N * K for (_, _, _, N, K, _) in shapes),
