@@ -85,3 +85,19 @@ def test_traffic_key_ignores_comments_only():
     assert bench.strip_comments("b // to the end") == "b  "
     h = bench.kernel_sha256("decode")
     assert len(h) == 64 and h == bench.kernel_sha256("decode")
+
+
+def test_algorithmic_bytes_and_flops_of_the_workloads():
+    """The bench's accounting (codes + fp16 scales/zeros + x + out per op;
+    2*M*N*K flops) against the per-config totals worked out from that formula
+    for the 7B- and 32B-shaped layers."""
+    import bench
+    one = bench.workload_config(1, 1, 1)
+    assert one["bytes_per_step"] == 123_964_416                    # one 7B layer, M = 1
+    for M, gb in ((1, 3.471), (4, 3.484), (16, 3.538), (64, 3.751)):  # 28 layers
+        assert round(bench.workload_config(M, 28, 1)["bytes_per_step"] / 1e9, 3) == gb
+    assert bench.workload_config(1, 1, 1, "32b-mixed")["bytes_per_step"] == 206_833_664
+    pre = bench.workload_config(2048, 28, 1)
+    assert round(pre["bytes_per_step"] / 1e9, 2) == 12.57
+    assert round(pre["flops_per_step"] / 1e12, 2) == 26.73
+    assert round(bench.workload_config(1, 1, 1)["flops_per_step"] / 1e6) == 466  # MFLOP per 7B layer
