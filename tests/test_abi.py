@@ -146,3 +146,18 @@ def test_import_fails_loudly_without_library(tmp_path):
     code = "import weight_only_quantized_zq_b200"
     r = subprocess.run([sys.executable, "-c", code], cwd=tmp_path, capture_output=True, text=True)
     assert r.returncode != 0 and "libzq.so" in r.stderr
+
+
+def test_kv_plane_binding_checks_shapes(zq):
+    """The Python plane rejects mis-shaped or mistyped rows before any call
+    into the library (a wrong shape would make the kernel read out of bounds)."""
+    import torch
+    pl = zq.KVPlane(4, 16, 2, 128, 4, device="cpu")
+    for bad in (torch.zeros(3, 2, 64, dtype=torch.float16), torch.zeros(3, 2, 128, dtype=torch.float32),
+                torch.zeros(2, 3, 128, dtype=torch.float16).transpose(0, 1)):
+        with pytest.raises(zq.ZQError) as e:
+            pl.append(bad)
+        assert e.value.status == zq.ZQ_ERR_INVALID_ARG
+    assert pl.tokens == 0
+    with pytest.raises(zq.ZQError):
+        pl.gather(0, 0, out=torch.zeros(1, 2, 128, dtype=torch.float16))

@@ -281,9 +281,17 @@ class KVPlane:
         self.window, self.capacity, self.heads, self.dim, self.bits = window, capacity, heads, dim, bits
         self.tokens = 0
 
+    def _rows_ok(self, t, n, what):
+        if (t.dtype != torch.float16 or not t.is_contiguous() or tuple(t.shape) != (n, self.heads, self.dim)
+                or t.device != self.ring.device):
+            raise ZQError(ZQ_ERR_INVALID_ARG, f"{what} must be a contiguous fp16 tensor of shape "
+                          f"{(n, self.heads, self.dim)} on {self.ring.device}, got {tuple(t.shape)} "
+                          f"{t.dtype} on {t.device}")
+
     def append(self, rows, stream=None):
         """rows: fp16 CUDA tensor (n, heads, dim)."""
         n = rows.shape[0]
+        self._rows_ok(rows, n, "rows")
         _check(_lib.zq_kv_append(ctypes.byref(self.desc), self.tokens, _ptr(rows), n, _stream(stream, rows)))
         self.tokens += n
 
@@ -292,6 +300,7 @@ class KVPlane:
         b = self.tokens if b is None else b
         if out is None:
             out = torch.empty(max(b - a, 0), self.heads, self.dim, dtype=torch.float16, device=self.ring.device)
+        self._rows_ok(out, max(b - a, 0), "out")
         _check(_lib.zq_kv_gather(ctypes.byref(self.desc), self.tokens, a, b, _ptr(out), _stream(stream, out)))
         return out
 
