@@ -161,3 +161,22 @@ def test_kv_plane_binding_checks_shapes(zq):
     assert pl.tokens == 0
     with pytest.raises(zq.ZQError):
         pl.gather(0, 0, out=torch.zeros(1, 2, 128, dtype=torch.float16))
+
+
+def test_linear_and_quantize_wrappers_check_buffers(zq):
+    """The convenience wrappers size every buffer against (M, N, K, bits)
+    before calling the library, which sees only pointers."""
+    import torch
+    x = torch.zeros(2, 256, dtype=torch.float16)
+    p, s, z = zq.alloc_quantized(64, 256, 4, device="cpu")
+    for args in ((x, p[:-1], s, z), (x, p, s[:-1], z), (x, p, s, z[:, :1]), (x.float(), p, s, z),
+                 (x[:, :128], p, s, z)):
+        with pytest.raises(zq.ZQError) as e:
+            zq.linear(*args, 4, 64)
+        assert e.value.status == zq.ZQ_ERR_INVALID_ARG
+    with pytest.raises(zq.ZQError):
+        zq.linear(x, p, s, z, 4, 64, out=torch.zeros(2, 63, dtype=torch.float16))
+    with pytest.raises(zq.ZQError):
+        zq.quantize(torch.zeros(4, 256, dtype=torch.float16), 4)
+    with pytest.raises(zq.ZQError):
+        zq.quantize(torch.zeros(256, 4).t(), 4)  # not contiguous

@@ -240,10 +240,21 @@ def alloc_quantized(N, K, bits, device="cuda"):
     return packed, scales, zeros
 
 
+def _need(t, nbytes, dtype, what, device):
+    if (not isinstance(t, torch.Tensor) or t.dtype != dtype or not t.is_contiguous()
+            or t.numel() * t.element_size() != nbytes or t.device != device):
+        raise ZQError(ZQ_ERR_INVALID_ARG, f"{what}: need a contiguous {dtype} tensor of {nbytes} bytes on "
+                      f"{device}, got {getattr(t, 'dtype', type(t))} of "
+                      f"{t.numel() * t.element_size() if isinstance(t, torch.Tensor) else '?'} bytes")
+
+
 def quantize(w, bits, stream=None, symmetric=False):
     """fp32 CUDA tensor N x K -> (packed, scales, zeros) via zq_quantize_pack
     (or zq_quantize_pack_symmetric); both give the same storage format."""
+    if w.dim() != 2:
+        raise ZQError(ZQ_ERR_INVALID_ARG, f"w must be 2-D (N x K), got shape {tuple(w.shape)}")
     N, K = w.shape
+    _need(w, N * K * 4, torch.float32, "w", w.device)
     packed, scales, zeros = alloc_quantized(N, K, bits, w.device)
     fn = zq_quantize_pack_symmetric if symmetric else zq_quantize_pack
     fn(w, N, K, bits, GROUP, packed, scales, zeros, stream)
@@ -252,9 +263,17 @@ def quantize(w, bits, stream=None, symmetric=False):
 
 def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
     """fp16 CUDA x (M x K) -> fp16 out (M x N) via zq_linear."""
+    if x.dim() != 2:
+        raise ZQError(ZQ_ERR_INVALID_ARG, f"x must be 2-D (M x K), got shape {tuple(x.shape)}")
     M, K = x.shape
+    _need(x, M * K * 2, torch.float16, "x", x.device)
+    if K % GROUP == 0 and bits in (2, 3, 4, 8):  # other formats: the library reports them
+        _need(packed, N * K * bits // 8, packed.dtype, "packed", x.device)
+        _need(scales, N * (K // GROUP) * 2, scales.dtype, "scales", x.device)
+        _need(zeros, N * (K // GROUP) * 2, zeros.dtype, "zeros", x.device)
     if out is None:
         out = torch.empty(M, N, dtype=torch.float16, device=x.device)
+    _need(out, M * N * 2, torch.float16, "out", x.device)
     zq_linear(x, packed, scales, zeros, bits, GROUP, M, N, K, out, stream)
     return out
 
