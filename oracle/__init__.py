@@ -9,8 +9,10 @@ What it computes follows the ZSE wiki article "ZSE - open-source движок д
 asymmetric min/max quantizer, low-nibble-first packing, fp16 scale/zero),
 generalised to b in {2,3,4,8} per the per-tensor INT2-8 scheme of "ZSE: A
 Memory-Efficient LLM Inference Engine with Smart Resource Orchestration",
-section "Technical Architecture". The C source states every reading taken where
-the pages are silent.
+section "Technical Architecture". The same section's symmetric INT8 variant
+(listed without a formula) is ``quantize_group_symmetric`` /
+``quantize_pack_symmetric``; ``zkv_oracle`` holds the quantized KV cache. The C
+source states every reading taken where the pages are silent.
 
 Arrays are numpy; fp16 values travel as uint16 bit patterns.
 """
