@@ -210,3 +210,20 @@ def test_native_load_rejects_null_destination(tmp_path, zq):
         assert zq._lib.zq_zse_load_weights(f._h, None, 1 << 20, None) == zq.ZQ_ERR_INVALID_ARG
         assert zq._lib.zq_zse_load_weights(f._h, 256, 16, None) == zq.ZQ_ERR_INVALID_ARG  # too small
     assert zq._lib.zq_zse_open(b"/nonexistent/x.zse", __import__("ctypes").byref(zq._P())) == zq.ZQ_ERR_INVALID_ARG
+
+
+def test_no_quantize_patterns():
+    """Embeddings, layer norms and every bias stay fp16; projections are
+    quantized; tensors the format cannot hold (1-D, K not a multiple of 128)
+    stay fp16 too."""
+    from weight_only_quantized_zq_b200.zse import keep_fp16
+    stay = ["model.embed_tokens.weight", "model.layers.0.input_layernorm.weight",
+            "model.layers.3.post_attention_layernorm.weight", "model.norm.weight",
+            "model.layers.0.self_attn.q_proj.bias", "transformer.h.0.ln_1.weight", "transformer.ln_f.weight",
+            "model.decoder.embed_positions.weight"]
+    quantize = ["model.layers.0.self_attn.q_proj.weight", "model.layers.0.mlp.gate_proj.weight",
+                "model.layers.27.mlp.down_proj.weight", "lm_head.weight"]
+    assert all(keep_fp16(n) for n in stay)
+    assert not any(keep_fp16(n, (4096, 4096)) for n in quantize)
+    assert keep_fp16("model.layers.0.mlp.down_proj.weight", (4096, 1000))
+    assert keep_fp16("some.vector", (4096,))

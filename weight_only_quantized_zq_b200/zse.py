@@ -26,6 +26,29 @@ TENSOR_ALIGN = 256
 GROUP = 128
 
 
+# Tensors that stay fp16 ([wiki] "Формат модели .zse": embeddings, layer
+# norms and every bias are kept unquantized, through an exclusion list of name
+# patterns).  Matched against Hugging Face-style tensor names.
+NO_QUANTIZE_PATTERNS = (
+    r"(^|\.)embed",        # token / position embeddings
+    r"norm(\.|_|$)",       # layernorm, rmsnorm, input_layernorm, ...
+    r"(^|\.)ln_?\w*\.",   # GPT-style ln_1., ln_f.
+    r"\.bias$",            # every bias
+)
+
+
+def keep_fp16(name, shape=None):
+    """True if the tensor `name` stays fp16: it matches NO_QUANTIZE_PATTERNS,
+    or it cannot be stored in the quantized format (not 2-D, or the number of
+    columns is not a multiple of the group of 128)."""
+    import re
+    if any(re.search(p, name) for p in NO_QUANTIZE_PATTERNS):
+        return True
+    if shape is not None and (len(shape) != 2 or shape[1] % GROUP != 0):
+        return True
+    return False
+
+
 def _bytes(a):
     """A flat read-only byte view of a numpy array, torch CPU tensor or bytes."""
     if isinstance(a, (bytes, bytearray, memoryview)):
