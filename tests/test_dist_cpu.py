@@ -101,3 +101,36 @@ def test_algorithmic_bytes_and_flops_of_the_workloads():
     assert round(pre["bytes_per_step"] / 1e9, 2) == 12.57
     assert round(pre["flops_per_step"] / 1e12, 2) == 26.73
     assert round(bench.workload_config(1, 1, 1)["flops_per_step"] / 1e6) == 466  # MFLOP per 7B layer
+
+
+def test_clock_sampler_decodes_reasons_with_a_fake_nvml():
+    """The clocks key of the bench line: median SM clock under load and the
+    throttle reasons seen, from NVML's clock-event mask (a fake NVML here;
+    nothing is set on any device)."""
+    import threading
+    import bench
+
+    class FakeNvml:
+        NVML_CLOCK_SM = 1
+
+        def __init__(self):
+            self.clocks = iter([1965, 1950, 1582, 1965, 1300])
+            self.masks = iter([0x0, 0x4, 0x4, 0x0, 0x4 | 0x40])
+
+        def nvmlDeviceGetClockInfo(self, handle, kind):
+            assert handle == "h0" and kind == self.NVML_CLOCK_SM
+            return next(self.clocks)
+
+        def nvmlDeviceGetCurrentClocksEventReasons(self, handle):
+            return next(self.masks)
+
+    s = bench.ClockSampler.__new__(bench.ClockSampler)
+    s.samples, s.reasons, s.max_mhz, s.period = [], set(), 1965, 0.0
+    s._stop, s._thread, s._nvml, s._h = threading.Event(), None, FakeNvml(), "h0"
+    for _ in range(5):
+        s.sample()
+    out = s.summary()
+    assert out["sm_mhz"] == 1950 and out["sm_max_mhz"] == 1965
+    assert out["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
+    s.sample()  # an NVML error (exhausted fake) is ignored, not raised
+    assert len(s.samples) == 5
