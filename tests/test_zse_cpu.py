@@ -227,3 +227,29 @@ def test_no_quantize_patterns():
     assert not any(keep_fp16(n, (4096, 4096)) for n in quantize)
     assert keep_fp16("model.layers.0.mlp.down_proj.weight", (4096, 1000))
     assert keep_fp16("some.vector", (4096,))
+
+
+def test_views_into_the_weight_section(tmp_path, zq):
+    """ZseFile.views slices a buffer holding WEIGHT_DATA into every tensor's
+    arrays (here a host copy of the section; on the GPU the buffer that
+    load_weights filled), equal to what was written."""
+    import torch
+    from weight_only_quantized_zq_b200.zse import write_zse
+    path = tmp_path / "v.zse"
+    tensors = _tensors(5)
+    write_zse(path, tensors)
+    with zq.ZseFile(path) as f:
+        data = f.section(zq.ZSE_WEIGHT_DATA)
+        buf = torch.frombuffer(bytearray(data), dtype=torch.uint8)
+        views = f.views(buf)
+        with pytest.raises(zq.ZQError):
+            f.views(buf[:-1])
+    for t in tensors:
+        v = views[t["name"]]
+        if "data" in t:
+            assert np.array_equal(v["data"].numpy(), t["data"])
+        else:
+            assert v["packed"].shape == (t["rows"], t["cols"] * t["bits"] // 32)
+            assert np.array_equal(v["packed"].numpy().view(np.uint32).reshape(-1), t["packed"])
+            assert np.array_equal(v["scales"].numpy().view(np.uint16), t["scales"])
+            assert np.array_equal(v["zeros"].numpy().view(np.uint16), t["zeros"])

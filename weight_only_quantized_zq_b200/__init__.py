@@ -378,3 +378,31 @@ class ZseFile:
         """Copies WEIGHT_DATA into the uint8 CUDA tensor dst (synchronous)."""
         _check(_lib.zq_zse_load_weights(self._h, _ptr(dst), dst.numel() * dst.element_size(),
                                         _stream(stream, dst)))
+
+    def views(self, weights):
+        """Per-tensor views into `weights`, a uint8 tensor holding WEIGHT_DATA
+        (as filled by load_weights): name -> {"bits", "rows", "cols", and
+        "packed" (int32 rows x cols*bits/32), "scales", "zeros" (int16 rows x
+        cols/128) for a quantized tensor, or "data" (fp16 rows x cols)}.  No
+        copy: the views share the buffer, ready for zq_linear / zq_linear_stack."""
+        if weights.dtype != torch.uint8 or weights.dim() != 1 or weights.numel() < self.weight_bytes:
+            raise ZQError(ZQ_ERR_INVALID_ARG, "weights must be a 1-D uint8 tensor of at least "
+                          f"{self.weight_bytes} bytes")
+        out = {}
+        for t in self.tensors():
+            rows, cols = t["rows"], t["cols"]
+
+            def view(off, nbytes, dtype, shape):
+                return weights[off:off + nbytes].view(dtype).view(*shape)
+
+            if t["kind"] == 1:
+                G = cols // t["group"]
+                out[t["name"]] = {
+                    "bits": t["bits"], "rows": rows, "cols": cols,
+                    "packed": view(t["data_offset"], t["data_bytes"], torch.int32, (rows, cols * t["bits"] // 32)),
+                    "scales": view(t["scales_offset"], rows * G * 2, torch.int16, (rows, G)),
+                    "zeros": view(t["zeros_offset"], rows * G * 2, torch.int16, (rows, G))}
+            else:
+                out[t["name"]] = {"bits": 16, "rows": rows, "cols": cols,
+                                  "data": view(t["data_offset"], t["data_bytes"], torch.float16, (rows, cols))}
+        return out
