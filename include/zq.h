@@ -193,8 +193,9 @@ ZQ_API const char *zq_status_string(zq_status status);
 ZQ_API const char *zq_last_error(void);
 
 /* Waits for the current device to finish all work, then reports whether any
- * of this library's kernels gave up a bounded wait (ZQ_ERR_TIMEOUT) since the
- * last call; clears that record.  Synchronous. */
+ * of this library's kernels gave up a bounded wait (ZQ_ERR_TIMEOUT) or a KV
+ * append met a NaN or Inf row (ZQ_ERR_NONFINITE, zq_kv.h) since the last call;
+ * clears those records.  Synchronous. */
 ZQ_API zq_status zq_check_device(void);
 
 /* Number of kernels this library has launched in this process (all devices).
