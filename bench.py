@@ -337,6 +337,31 @@ def time_oracle(items, M, budget_s=None):
     return done_bytes / el / 1e9, el, done_bytes, orc.get_threads()
 
 
+def oracle_config1_one_core(budget_s=0.5):
+    """The small single-layer workload (M=1, N=K=512, INT4; W seed 0, x seed
+    15) through the oracle on one host core, repeated for budget_s: time per
+    call and GB/s of algorithmic bytes."""
+    import oracle as orc
+    w = zi.weight(512, 512, 0).numpy()
+    p, s, z = orc.quantize_pack(w, 4)
+    x = zi.activations(1, 512, zi.X_SEED).numpy().view(np.uint16)
+    prev = orc.get_threads()
+    orc.set_threads(1)
+    try:
+        calls, t0 = 0, time.perf_counter()
+        while True:
+            orc.linear(x, p, s, z, 4, 512, 512)
+            calls += 1
+            el = time.perf_counter() - t0
+            if el >= budget_s:
+                break
+    finally:
+        orc.set_threads(prev)
+    us = el / calls * 1e6
+    return {"us_per_call": us, "value": op_bytes(1, 512, 512, 4) / (us * 1e-6) / 1e9, "unit": "GB/s",
+            "cores": 1, "sample": f"M=1, N=K=512, INT4 g128: {calls} oracle calls in {el:.2f} s"}
+
+
 # ------------------------------------------------------------------- arms --
 
 def run_reference(args):
@@ -465,7 +490,8 @@ def run_zq(args):
             v, el, b, threads = time_oracle(items, M, budget_s=args.cpu_seconds)
             cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle",
                    "sample": f"oracle linear (fp64, OpenMP over rows) on all 4 projections of layer 0 "
-                             f"at M={M}, repeated for {el:.1f} s ({b / 1e9:.2f} GB of algorithmic bytes)"}
+                             f"at M={M}, repeated for {el:.1f} s ({b / 1e9:.2f} GB of algorithmic bytes)",
+                   "one_core_small_layer": oracle_config1_one_core()}
         line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,

@@ -134,3 +134,14 @@ def test_clock_sampler_decodes_reasons_with_a_fake_nvml():
     assert out["reasons"] == ["hw_thermal_slowdown", "sw_power_cap"]
     s.sample()  # an NVML error (exhausted fake) is ignored, not raised
     assert len(s.samples) == 5
+
+
+def test_oracle_small_layer_on_one_core():
+    """The bench's one-core oracle figure for the M=1, N=K=512 INT4 layer runs
+    on the CPU and leaves the oracle's thread count as it found it."""
+    import bench
+    import oracle as orc
+    before = orc.get_threads()
+    r = bench.oracle_config1_one_core(budget_s=0.05)
+    assert r["cores"] == 1 and r["us_per_call"] > 0 and r["value"] > 0
+    assert orc.get_threads() == before
