@@ -282,6 +282,18 @@ def test_prefill_grouped_plans(zq, orc, bits):
             assert_linear_close(outs[i], y_ref, bound, f"grouped bits={bits} M={M} N={N} K={K}")
 
 
+@pytest.mark.parametrize("bits", (2, 8))
+def test_prefill_one_half_many_short_tiles(zq, orc, bits):
+    """One-half plan with more row tiles than SMs and one group per tile
+    (K = 128): the code-ring issue cursor runs whole tiles ahead of the
+    consumer (INT2: 5 groups in flight, INT8: 2)."""
+    M, N, K = 40, 157 * 256 - 13, 128
+    w = zi.weight(N, K, seed=6100 + bits, device="cuda")
+    q = _quantize_both(zq, orc, w, bits)
+    x = zi.activations(M, K, seed=6200, device="cuda")
+    _check_linear(zq, orc, x, q[:3], q[3], bits, N, f"many short tiles bits={bits}")
+
+
 def test_stack_validation_enqueues_nothing(zq, orc):
     q, _ = _layer(zq, orc, 64, 256, 4, 80)
     x = zi.activations(1, 256, 81, device="cuda")
