@@ -36,11 +36,21 @@ def _quantize_both(zq, orc, w, bits):
     return packed, scales, zeros, (p_ref, s_ref, z_ref)
 
 
+CANARY = 0x5A5A  # fp16 bit pattern of the guard regions around an output
+GUARD = 64       # guard halves on each side (128 bytes keeps the output 16-byte aligned)
+
+
 def _check_linear(zq, orc, x, qbufs, ref_bufs, bits, N, what, rows=None):
     M, K = x.shape
     packed, scales, zeros = qbufs
-    out = zq.linear(x, packed, scales, zeros, bits, N)
+    # the output sits between two guard regions: a kernel writing outside the
+    # M x N result would change them
+    buf = torch.full((GUARD + M * N + GUARD,), CANARY, dtype=torch.int16, device=x.device)
+    out = buf[GUARD:GUARD + M * N].view(torch.float16).view(M, N)
+    zq.linear(x, packed, scales, zeros, bits, N, out=out)
     torch.cuda.synchronize()
+    guards = torch.cat([buf[:GUARD], buf[GUARD + M * N:]])
+    assert bool((guards == CANARY).all()), f"{what}: write outside the output"
     p_ref, s_ref, z_ref = ref_bufs
     y_ref, bound = orc.linear(u16(x), p_ref, s_ref, z_ref, bits, N, K, rows=rows)
     got = out if rows is None else out[:, torch.as_tensor(rows, device=out.device)]
