@@ -406,6 +406,9 @@ def run_zq(args):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
+    # the stack's workspace is reserved once, outside every timed region
+    zq.ensure_workspace(zq.zq_linear_stack_workspace_bytes(wl.descs, wl.n_ops), stream)
+
     def step():
         zq.zq_linear_stack(wl.descs, wl.n_ops, sp)
 

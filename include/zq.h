@@ -46,12 +46,18 @@
  *   - Stream order: a call's kernels read their inputs only after all work
  *     enqueued earlier on `stream` has completed (programmatic dependent
  *     launch is used only to overlap launch latency, never to read early).
- *   - The library keeps one workspace per (device, stream) for activation
- *     staging and split-K partial sums.  It is allocated (and zeroed) by the
- *     first call on that stream that needs it and grown when a larger call
- *     arrives; run such a call once before capturing the stream into a CUDA
- *     graph, or call zq_reserve_workspace().  Calls on the same stream are
- *     ordered; calls on different streams use different workspaces.
+ *   - Workspace: zq_linear and zq_linear_stack use one device buffer per
+ *     (device, stream) for activation staging, split-K partial sums and work
+ *     counters.  The calls themselves never allocate, free or synchronise: the
+ *     buffer is reserved beforehand with zq_reserve_workspace (the library
+ *     allocates it) or attached with zq_attach_workspace (the caller owns it),
+ *     sized by zq_linear_workspace_bytes / zq_linear_stack_workspace_bytes.  A
+ *     call that needs more than its stream holds returns ZQ_ERR_INVALID_ARG
+ *     and enqueues nothing.  Streams are told apart by their unique id
+ *     (cudaStreamGetId), so a handle reused by CUDA after cudaStreamDestroy
+ *     starts without a workspace; release a stream's workspace
+ *     (zq_release_workspace) before destroying the stream.  Calls on the same
+ *     stream are ordered; calls on different streams use different buffers.
  */
 #ifndef ZQ_H
 #define ZQ_H
@@ -81,7 +87,9 @@ typedef enum {
     ZQ_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up             */
 } zq_status;
 
-/* Number of uint32 words of a packed N x K tensor: N * K * bits / 32.
+/* Number of uint32 words of a packed N x K tensor: N * K * bits / 32
+ * ([wiki] "Формат модели .zse": b-bit codes packed densely, two INT4 codes per
+ * byte; [lavx] "Technical Architecture": b from 2 to 8 per tensor).
  * Returns 0 for unsupported bits or sizes (K % 128 != 0, N <= 0, K <= 0). */
 ZQ_API size_t zq_packed_words(int N, int K, int bits);
 
@@ -118,13 +126,17 @@ ZQ_API zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bi
                                             uint32_t *packed, uint16_t *scales, uint16_t *zeros,
                                             zq_stream_t stream);
 
-/* y = x · dequant(W)^T.
+/* y = x · dequant(W)^T, the quantized projection of [wiki] "Оркестратор и
+ * GPU-ядра" (INT4 GEMV for decode, tiled matmul for prefill) over the format
+ * of [wiki] "Формат модели .zse" (dequant(W) = q * scale + zero per group).
  *   x       device, fp16 M x K.      out  device, fp16 M x N (written).
  *   packed/scales/zeros as produced by zq_quantize_pack.
  * M <= 16 runs the decode kernel (mma.sync skinny GEMM streaming the packed
  * weights once through a shared-memory ring); larger M runs the tcgen05 tile
  * kernel (256 x 256 output tiles; with M <= 256 one token tile, so the
- * weights are again streamed once).  Asynchronous. */
+ * weights are again streamed once).  Needs a workspace of
+ * zq_linear_workspace_bytes(bits, M, N, K) on `stream` (see Conventions).
+ * Asynchronous; fp32 accumulation, fp16 output rounded to nearest even. */
 ZQ_API zq_status zq_linear(const uint16_t *x, const uint32_t *packed,
                     const uint16_t *scales, const uint16_t *zeros,
                     int bits, int group, int M, int N, int K,
@@ -169,22 +181,56 @@ typedef struct {
  * `ops` is a HOST array, read before the call returns.  An op's x may alias
  * an earlier op's out: the library detects overlapping buffers and keeps
  * such ops ordered; runs of independent ops are fused into one launch per
- * (bits, batch class).  All ops are validated before anything is enqueued.
- * Asynchronous. */
+ * (bits, batch class).  All ops, and the workspace the stack needs
+ * (zq_linear_stack_workspace_bytes), are checked before anything is
+ * enqueued.  Asynchronous. */
 ZQ_API zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream);
 
 /* Test hook: unpack codes with the same device unpack routine zq_linear
- * uses.  codes: device uint8 N x K (written).  Asynchronous. */
+ * uses; the inverse of the packing of [wiki] "Формат модели .zse" (code k of
+ * a row at stream bits [k*b, k*b+b)).  codes: device uint8 N x K (written).
+ * Asynchronous. */
 ZQ_API zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits,
                     uint8_t *codes, zq_stream_t stream);
 
-/* Pre-size the workspace of (current device, stream) to at least `bytes`.
- * Useful before graph capture.  Synchronous. */
+/* Workspace (see Conventions).  The pages describe no counterpart: these are
+ * services of the library, not part of the method.
+ *
+ * zq_reserve_workspace: gives (current device, stream) a library-allocated
+ *   workspace of at least `bytes` (at least 256 KB), replacing a smaller or
+ *   attached one.  SYNCHRONOUS when it allocates (waits for `stream` first so
+ *   the old buffer is no longer in use); a no-op when the stream already holds
+ *   enough.  Call it before capturing the stream into a CUDA graph.
+ * zq_attach_workspace: makes the caller's device buffer (256-byte aligned, at
+ *   least 256 KB) the workspace of (current device, stream); a library-owned
+ *   one is freed (after waiting for the stream).  Its first 256 KB of counters
+ *   are cleared by an asynchronous memset on `stream`.  The caller keeps the
+ *   buffer alive and unused by anything else until it releases it; no other
+ *   stream may share it.
+ * zq_release_workspace: waits for `stream`, then frees (library-owned) or
+ *   forgets (attached) its workspace.  ZQ_OK if it has none.
+ * zq_release_all_workspaces: waits for the current device, then releases the
+ *   workspaces of all its streams. */
 ZQ_API zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream);
+ZQ_API zq_status zq_attach_workspace(void *buffer, size_t bytes, zq_stream_t stream);
+ZQ_API zq_status zq_release_workspace(zq_stream_t stream);
+ZQ_API zq_status zq_release_all_workspaces(void);
 
-/* Workspace bytes zq_linear needs for these sizes (0 if none; M > 16 needs
- * none). */
+/* Workspace bytes a zq_linear call with these sizes needs (0 for invalid
+ * sizes).  Host only; no device work. */
 ZQ_API size_t zq_linear_workspace_bytes(int bits, int M, int N, int K);
+
+/* Workspace bytes zq_linear_stack(ops, n_ops) needs (0 for an invalid op).
+ * Host only; reads the HOST array `ops`. */
+ZQ_API size_t zq_linear_stack_workspace_bytes(const zq_linear_desc *ops, int n_ops);
+
+/* Test hook: limit, in nanoseconds, of the bounded waits of the linear
+ * kernels launched after this call, on every device (default 2000000000, i.e.
+ * 2 s; the limit travels with each launch).  A wait that runs out makes its
+ * kernel stop and drain and zq_check_device report ZQ_ERR_TIMEOUT; the drain
+ * of copies and MMAs already issued keeps its own 2 s bound.  Lets a test make
+ * waits run out without any fault.  Host only. */
+ZQ_API zq_status zq_set_wait_limit_ns(uint64_t ns);
 
 /* Human-readable name of a status code (static storage). */
 ZQ_API const char *zq_status_string(zq_status status);
@@ -195,7 +241,9 @@ ZQ_API const char *zq_last_error(void);
 /* Waits for the current device to finish all work, then reports whether any
  * of this library's kernels gave up a bounded wait (ZQ_ERR_TIMEOUT) or a KV
  * append met a NaN or Inf row (ZQ_ERR_NONFINITE, zq_kv.h) since the last call;
- * clears those records.  Synchronous. */
+ * clears those records.  After a timeout the outputs of the calls involved
+ * are unspecified; the workspaces of the device are marked so that the next
+ * call on each stream first clears its counters.  Synchronous. */
 ZQ_API zq_status zq_check_device(void);
 
 /* Number of kernels this library has launched in this process (all devices).

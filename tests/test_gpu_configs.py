@@ -58,7 +58,7 @@ def test_config3_decode_stack_28_layers(zq, orc):
                 out = torch.empty(M, N, dtype=torch.float16, device="cuda")
                 ops.append((xs[(M, K)], *q, out, 4, 128, M, N, K))
                 outs.append((l, name, N, K, out, ref))
-        zq.zq_linear_stack(ops)
+        zq.linear_stack(ops)
         torch.cuda.synchronize()
         for (l, name, N, K, out, ref) in outs:
             if l in check:
@@ -83,7 +83,7 @@ def test_config4_mixed_stack_64_layers(zq, orc):
             out = torch.empty(1, N, dtype=torch.float16, device="cuda")
             ops.append((xs[K], *q, out, bits, 128, 1, N, K))
             outs.append((layer, name, N, K, bits, out, ref))
-    zq.zq_linear_stack(ops)
+    zq.linear_stack(ops)
     torch.cuda.synchronize()
     zq.zq_check_device()
     for (layer, name, N, K, bits, out, ref) in outs:
@@ -104,7 +104,7 @@ def test_config5_prefill_m2048(zq, orc):
             out = torch.empty(M, N, dtype=torch.float16, device="cuda")
             ops.append((xs[K], *q, out, 4, 128, M, N, K))
             outs.append((name, N, K, out, ref))
-        zq.zq_linear_stack(ops)
+        zq.linear_stack(ops)
         torch.cuda.synchronize()
         zq.zq_check_device()
         for (name, N, K, out, ref) in outs:

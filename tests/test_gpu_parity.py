@@ -259,7 +259,7 @@ def test_stack_against_oracle(zq, orc):
     yc = torch.empty(2, 384, dtype=torch.float16, device="cuda")
     ops += [(xa, *qa, ya, 4, 128, 2, 512, 512), (ya, *qb, yb, 3, 128, 2, 256, 512),
             (yb, *qc, yc, 8, 128, 2, 384, 256)]
-    zq.zq_linear_stack(ops)
+    zq.linear_stack(ops)
     torch.cuda.synchronize()
     for i, (M, N, K, b) in enumerate(specs):
         p, s, z = layers[i][1]
@@ -283,7 +283,7 @@ def test_prefill_grouped_plans(zq, orc, bits):
         layers = [_layer(zq, orc, N, K, bits, 90 + 7 * i + bits) for i, (M, N, K) in enumerate(specs)]
         xs = [zi.activations(M, K, 95 + i, device="cuda") for i, (M, N, K) in enumerate(specs)]
         outs = [torch.empty(M, N, dtype=torch.float16, device="cuda") for (M, N, K) in specs]
-        zq.zq_linear_stack([(xs[i], *layers[i][0], outs[i], bits, 128, M, N, K)
+        zq.linear_stack([(xs[i], *layers[i][0], outs[i], bits, 128, M, N, K)
                             for i, (M, N, K) in enumerate(specs)])
         torch.cuda.synchronize()
         for i, (M, N, K) in enumerate(specs):

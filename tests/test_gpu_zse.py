@@ -57,7 +57,7 @@ def test_load_weights_bit_exact_then_linear(tmp_path, zq, orc):
         out = torch.empty(3, N, dtype=torch.float16, device="cuda")
         ops.append((x[K], packed, scales, zeros, out, bits, 128, 3, N, K))
         outs.append((name, bits, N, K, out))
-    zq.zq_linear_stack(ops)
+    zq.linear_stack(ops)
     torch.cuda.synchronize()
     for (name, bits, N, K, out) in outs:
         data, s, z = zo.tensor_arrays(parsed, name)

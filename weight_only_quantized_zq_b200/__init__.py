@@ -27,8 +27,9 @@ GROUP = 128
 
 # Every symbol the headers declare (checked by the CPU test suite).
 EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_quantize_pack_symmetric", "zq_linear", "zq_linear_noalloc", "zq_linear_stack",
-           "zq_unpack", "zq_reserve_workspace", "zq_linear_workspace_bytes",
-           "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
+           "zq_unpack", "zq_reserve_workspace", "zq_attach_workspace", "zq_release_workspace",
+           "zq_release_all_workspaces", "zq_linear_workspace_bytes", "zq_linear_stack_workspace_bytes",
+           "zq_set_wait_limit_ns", "zq_status_string", "zq_last_error", "zq_check_device", "zq_kernel_launches",
            "zq_version",
            "zq_zse_open", "zq_zse_close", "zq_zse_flags", "zq_zse_tensor_count", "zq_zse_tensor_info",
            "zq_zse_find", "zq_zse_section", "zq_zse_weight_bytes", "zq_zse_verify", "zq_zse_load_weights",
@@ -59,8 +60,16 @@ _lib.zq_unpack.argtypes = [_P, _I, _I, _I, _P, _P]
 _lib.zq_unpack.restype = _I
 _lib.zq_reserve_workspace.argtypes = [_S, _P]
 _lib.zq_reserve_workspace.restype = _I
+_lib.zq_attach_workspace.argtypes = [_P, _S, _P]
+_lib.zq_attach_workspace.restype = _I
+_lib.zq_release_workspace.argtypes = [_P]
+_lib.zq_release_workspace.restype = _I
+_lib.zq_release_all_workspaces.argtypes = []
+_lib.zq_release_all_workspaces.restype = _I
 _lib.zq_linear_workspace_bytes.argtypes = [_I, _I, _I, _I]
 _lib.zq_linear_workspace_bytes.restype = _S
+_lib.zq_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+_lib.zq_set_wait_limit_ns.restype = _I
 _lib.zq_status_string.argtypes = [_I]
 _lib.zq_status_string.restype = ctypes.c_char_p
 _lib.zq_last_error.argtypes = []
@@ -126,6 +135,10 @@ class zq_linear_desc(ctypes.Structure):
                 ("bits", _I), ("group", _I), ("M", _I), ("N", _I), ("K", _I)]
 
 
+_lib.zq_linear_stack_workspace_bytes.argtypes = [_P, _I]
+_lib.zq_linear_stack_workspace_bytes.restype = _S
+
+
 def _check(status):
     if status != ZQ_OK:
         raise ZQError(status, zq_last_error())
@@ -182,6 +195,30 @@ def zq_linear_workspace_bytes(bits, M, N, K):
 
 def zq_reserve_workspace(nbytes, stream=None):
     _check(_lib.zq_reserve_workspace(nbytes, _stream(stream)))
+
+
+def zq_attach_workspace(buffer, nbytes, stream=None):
+    _check(_lib.zq_attach_workspace(_ptr(buffer), nbytes, _stream(stream, buffer)))
+
+
+def zq_release_workspace(stream=None):
+    _check(_lib.zq_release_workspace(_stream(stream)))
+
+
+def zq_release_all_workspaces():
+    _check(_lib.zq_release_all_workspaces())
+
+
+def zq_linear_stack_workspace_bytes(ops, n_ops=None):
+    """ops: a ctypes array from make_descs(), or an iterable accepted by it."""
+    if not isinstance(ops, ctypes.Array):
+        ops, n = make_descs(ops)
+        n_ops = n if n_ops is None else n_ops
+    return _lib.zq_linear_stack_workspace_bytes(ops, n_ops)
+
+
+def zq_set_wait_limit_ns(ns):
+    _check(_lib.zq_set_wait_limit_ns(int(ns)))
 
 
 def zq_quantize_pack(w, N, K, bits, group, packed, scales, zeros, stream=None):
@@ -261,8 +298,26 @@ def quantize(w, bits, stream=None, symmetric=False):
     return packed, scales, zeros
 
 
+def ensure_workspace(nbytes, stream=None):
+    """Reserves a workspace of at least `nbytes` on `stream` (default: torch's
+    current stream) unless it already holds that much.  A reservation that
+    grows the buffer waits for the stream; this happens here, between calls,
+    never inside zq_linear or zq_linear_stack."""
+    if nbytes > 0:
+        zq_reserve_workspace(nbytes, stream)
+
+
+def linear_stack(ops, stream=None):
+    """zq_linear_stack over `ops` (see make_descs) after making sure the
+    stream's workspace covers it."""
+    arr, n = ops if isinstance(ops, tuple) and isinstance(ops[0], ctypes.Array) else make_descs(ops)
+    ensure_workspace(zq_linear_stack_workspace_bytes(arr, n), stream)
+    zq_linear_stack(arr, n, stream)
+
+
 def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
-    """fp16 CUDA x (M x K) -> fp16 out (M x N) via zq_linear."""
+    """fp16 CUDA x (M x K) -> fp16 out (M x N) via zq_linear (reserving the
+    workspace it needs on the stream first)."""
     if x.dim() != 2:
         raise ZQError(ZQ_ERR_INVALID_ARG, f"x must be 2-D (M x K), got shape {tuple(x.shape)}")
     M, K = x.shape
@@ -274,6 +329,8 @@ def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
     if out is None:
         out = torch.empty(M, N, dtype=torch.float16, device=x.device)
     _need(out, M * N * 2, torch.float16, "out", x.device)
+    ensure_workspace(zq_linear_workspace_bytes(bits, M, N, K), stream if stream is not None else
+                     torch.cuda.current_stream(x.device))
     zq_linear(x, packed, scales, zeros, bits, GROUP, M, N, K, out, stream)
     return out
 

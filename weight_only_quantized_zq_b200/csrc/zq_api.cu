@@ -2,7 +2,9 @@
 // validation, the per-(device, stream) workspace, planning of decode launches
 // (cost-balanced units, split-K choice, fusion of independent stack ops) and
 // dispatch to the kernels.
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <algorithm>
 #include <atomic>
@@ -29,6 +31,7 @@ namespace {
 thread_local std::string g_last_error;
 std::atomic<unsigned long long> g_quant_call{1};
 std::atomic<uint64_t> g_launches{0};
+std::atomic<unsigned long long> g_wait_ns{2000000000ull};  // limit of the kernels' bounded waits
 
 zq_status fail(zq_status st, const char *fmt, ...) __attribute__((format(printf, 2, 3)));
 zq_status fail(zq_status st, const char *fmt, ...) {
@@ -115,8 +118,16 @@ zq_status decode_occupancy(DeviceInfo *info, int bits, int mt, size_t smem, int 
 }
 
 // ------------------------------------------------------------- workspace --
-// One buffer per (device, stream).  Layout: [counters | data].  Counters are
-// zeroed at allocation and every kernel that uses one resets it to zero.
+// One buffer per (device, stream), keyed by the stream's unique id (so a
+// stream handle that CUDA recycles after cudaStreamDestroy never inherits
+// another stream's buffer).  Layout: [counters | data].  The counters are
+// zeroed when the buffer is reserved or attached, every kernel that uses one
+// resets it to zero, and after a kernel gave up a wait (which can leave them
+// set) zq_check_device marks the buffers dirty: the next call on the stream
+// clears them with an asynchronous memset before its launches.
+// Calls never allocate, free or synchronise: a buffer comes from
+// zq_reserve_workspace (the library allocates it) or zq_attach_workspace (the
+// caller owns it), and a call that needs more than the stream holds fails.
 
 constexpr size_t kCounterBytes = 256 * 1024;
 constexpr size_t kMaxCounters = kCounterBytes / sizeof(unsigned int);
@@ -124,46 +135,53 @@ constexpr size_t kMaxCounters = kCounterBytes / sizeof(unsigned int);
 struct Workspace {
     void *ptr = nullptr;
     size_t bytes = 0;
+    bool owned = false;  // allocated by zq_reserve_workspace (else the caller's)
+    bool dirty = false;  // counters must be cleared before the next use
 };
 std::mutex g_ws_mu;
-std::map<std::pair<int, cudaStream_t>, Workspace> g_ws;
+std::map<std::pair<int, unsigned long long>, Workspace> g_ws;
 
-zq_status workspace(cudaStream_t stream, size_t data_bytes, uint8_t **base) {
+zq_status stream_key(cudaStream_t stream, std::pair<int, unsigned long long> *key) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    unsigned long long id = 0;
+    e = cudaStreamGetId(stream, &id);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamGetId");
+    *key = {dev, id};
+    return ZQ_OK;
+}
+
+// Base of the stream's workspace if it holds kCounterBytes + data_bytes;
+// clears dirty counters first (stream-ordered).  Never allocates.
+zq_status workspace(cudaStream_t stream, size_t data_bytes, uint8_t **base) {
+    std::pair<int, unsigned long long> key;
+    zq_status st = stream_key(stream, &key);
+    if (st != ZQ_OK) return st;
     const size_t need = kCounterBytes + data_bytes;
     std::lock_guard<std::mutex> lk(g_ws_mu);
-    Workspace &ws = g_ws[{dev, stream}];
-    if (ws.bytes < need) {
-        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
-        e = cudaStreamIsCapturing(stream, &cap);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamIsCapturing");
-        if (cap != cudaStreamCaptureStatusNone)
-            return fail(ZQ_ERR_CUDA,
-                        "workspace of %zu bytes needed while the stream is being captured; "
-                        "run the call once before capture or use zq_reserve_workspace",
-                        need);
-        size_t grow = std::max(need, ws.bytes + ws.bytes / 2);
-        grow = std::max(grow, static_cast<size_t>(8) << 20);
-        if (ws.ptr) {
-            e = cudaStreamSynchronize(stream);
-            if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
-            cudaFree(ws.ptr);
-            ws.ptr = nullptr;
-            ws.bytes = 0;
-        }
-        e = cudaMalloc(&ws.ptr, grow);
-        if (e != cudaSuccess) {
-            ws.ptr = nullptr;
-            return cuda_fail(e, "cudaMalloc(workspace)");
-        }
-        e = cudaMemset(ws.ptr, 0, kCounterBytes);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaMemset(workspace)");
-        ws.bytes = grow;
+    auto it = g_ws.find(key);
+    const size_t have = it == g_ws.end() ? 0 : it->second.bytes;
+    if (have < need)
+        return fail(ZQ_ERR_INVALID_ARG,
+                    "this call needs a workspace of %zu bytes on its stream, which holds %zu; reserve it "
+                    "beforehand with zq_reserve_workspace (or attach one with zq_attach_workspace)",
+                    need, have);
+    Workspace &ws = it->second;
+    if (ws.dirty) {
+        cudaError_t e = cudaMemsetAsync(ws.ptr, 0, kCounterBytes, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace counters");
+        ws.dirty = false;
     }
     *base = static_cast<uint8_t *>(ws.ptr);
     return ZQ_OK;
+}
+
+// Marks every workspace of `dev` dirty (after a kernel gave up a wait).
+void workspaces_dirty(int dev) {
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    for (auto &kv : g_ws)
+        if (kv.first.first == dev) kv.second.dirty = true;
 }
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -228,7 +246,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     const int codes_bytes = decode_codes_bytes(bits, mt);
     const int off_sz = 0;
     const int off_sx = off_sz + rows * 4 * gps;
-    const int off_x = off_sx + gps * mpad * 8;
+    const int off_x = off_sx + gps * mpad * 16;
     const int x_rows_max = mt == 1 ? max_m : mpad;  // staged token rows
     const int off_desc = off_x + gps * x_rows_max * 256;
     const int meta_bytes = static_cast<int>(align16(off_desc + 32));
@@ -290,7 +308,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         prep_off[e] = off;
         const size_t G = keys[e].K / kGroup;
         const size_t xr = mt == 1 ? keys[e].M : mpad;
-        off += align256(G * xr * kGroup * 2) + align256(G * mpad * 8);
+        off += align256(G * xr * kGroup * 2) + align256(G * mpad * 16);
     }
     const size_t part_off = off;
     if (!units) off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
@@ -346,6 +364,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     dp.off_sx = off_sx;
     dp.off_x = off_x;
     dp.off_desc = off_desc;
+    dp.wait_ns = g_wait_ns.load();
     const bool swz = decode_swizzled(bits, mt);
     int step0 = 0, unit0 = 0;
     for (size_t oi = 0; oi < ops.size(); ++oi) {
@@ -418,18 +437,6 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
     return overlap(a.out, b.out);
 }
 
-// Expands a linear op into decode-sized pieces (M <= 16 per piece); only used
-// for ops that the tile kernel does not take.
-void split_tokens(const zq_linear_desc &d, std::vector<zq_linear_desc> &out) {
-    for (int m0 = 0; m0 < d.M; m0 += kDecodeMaxM) {
-        zq_linear_desc p = d;
-        p.M = std::min(kDecodeMaxM, d.M - m0);
-        p.x = d.x + static_cast<size_t>(m0) * d.K;
-        p.out = d.out + static_cast<size_t>(m0) * d.N;
-        out.push_back(p);
-    }
-}
-
 // One persistent launch over all tiles of independent prefill ops of one bit
 // width (at most kMaxPrefillOps), ops with the longest K first so that the
 // last tiles handed out are the cheap ones.
@@ -461,6 +468,7 @@ zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
         tiles += prefill_tiles(ops[i].M, ops[i].N);
     }
     pg.n_tiles = tiles;
+    pg.wait_ns = g_wait_ns.load();
     cudaError_t e = launch_prefill_group(pg, ops[0].bits, info->sms, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     g_launches += 1;
@@ -469,14 +477,17 @@ zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
 
 // Launches a batch of mutually independent ops: one launch per (bits, MT)
 // class, each holding at most kMaxDecodeOps ops and kMaxPrepEntries inputs.
-zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t stream) {
+// With `dry` set nothing is launched: *dry becomes the largest workspace any
+// of the launches needs (at least the counters).
+zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t stream, size_t *dry = nullptr) {
     std::vector<zq_linear_desc> pieces;
     const int bits_list[4] = {2, 3, 4, 8};
+    if (dry) *dry = std::max(*dry, kCounterBytes);
     for (int bits : bits_list) {
         std::vector<zq_linear_desc> pre;
         for (const auto &d : batch)
             if (d.M > kDecodeMaxM && d.bits == bits) pre.push_back(d);
-        for (size_t i = 0; i < pre.size(); i += kMaxPrefillOps) {
+        for (size_t i = 0; i < pre.size() && !dry; i += kMaxPrefillOps) {
             std::vector<zq_linear_desc> launch(pre.begin() + i,
                                                pre.begin() + std::min(pre.size(), i + kMaxPrefillOps));
             zq_status st = run_prefill(launch, stream);
@@ -502,11 +513,50 @@ zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t strea
                     if (!known) inputs.push_back(key);
                     launch.push_back(cls[i++]);
                 }
-                zq_status st = run_decode(launch, bits, mt, stream);
+                size_t b = 0;
+                zq_status st = run_decode(launch, bits, mt, stream, dry ? &b : nullptr);
                 if (st != ZQ_OK) return st;
+                if (dry) *dry = std::max(*dry, b);
             }
         }
     return ZQ_OK;
+}
+
+// Splits a stack into batches of mutually independent ops (an op that shares
+// written memory with an earlier op of the batch starts the next batch) and
+// runs them in order; with `dry` set, only sizes the workspace.
+zq_status run_stack(const zq_linear_desc *ops, int n_ops, cudaStream_t s, size_t *dry) {
+    std::vector<zq_linear_desc> batch;
+    std::vector<OpRanges> br;
+    constexpr size_t kMaxBatch = 1024;
+    for (int i = 0; i < n_ops; ++i) {
+        const OpRanges r = ranges_of(ops[i]);
+        bool dep = batch.size() >= kMaxBatch;
+        for (size_t j = 0; j < br.size() && !dep; ++j) dep = conflicts(br[j], r);
+        if (dep) {
+            zq_status st = run_batch(batch, s, dry);
+            if (st != ZQ_OK) return st;
+            batch.clear();
+            br.clear();
+        }
+        batch.push_back(ops[i]);
+        br.push_back(r);
+    }
+    if (!batch.empty()) return run_batch(batch, s, dry);
+    return ZQ_OK;
+}
+
+// Checks that the stream's workspace covers the stack (nothing is enqueued
+// when it does not, apart from clearing counters a failed kernel left set),
+// then runs it.
+zq_status checked_stack(const zq_linear_desc *ops, int n_ops, cudaStream_t s) {
+    if (n_ops == 0) return ZQ_OK;
+    size_t need = kCounterBytes;
+    zq_status st = run_stack(ops, n_ops, s, &need);
+    if (st != ZQ_OK) return st;
+    uint8_t *base = nullptr;
+    if ((st = workspace(s, need - kCounterBytes, &base)) != ZQ_OK) return st;
+    return run_stack(ops, n_ops, s, nullptr);
 }
 
 // ------------------------------------------------------ allocation-free path --
@@ -520,19 +570,51 @@ constexpr int kNoallocMaxM = 8;
 static __device__ __align__(256) uint8_t g_noalloc_scratch[kNoallocScratchBytes];
 
 std::mutex g_noalloc_mu;
-std::map<int, uint8_t *> g_noalloc_addr;
+std::map<std::pair<int, unsigned long long>, uint8_t *> g_noalloc_addr;  // (device, context id) -> address
 
+// Unique id of the calling thread's current CUDA context (0 if none or not
+// available).  A context torn down and created again (cudaDeviceReset) gets a
+// new id, so an address cached for the old one is never reused.
+unsigned long long current_context_id() {
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(f);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+    if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current device's context, looked
+// up once per (device, context) with that device current.
 zq_status noalloc_scratch(uint8_t **ptr) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    const unsigned long long ctx = current_context_id();
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    auto it = g_noalloc_addr.find(dev);
-    if (it == g_noalloc_addr.end()) {
+    auto it = g_noalloc_addr.find({dev, ctx});
+    if (it == g_noalloc_addr.end() || ctx == 0) {
         void *p = nullptr;
         e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
         if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(scratch)");
-        it = g_noalloc_addr.emplace(dev, static_cast<uint8_t *>(p)).first;
+        const unsigned long long ctx_now = current_context_id();  // the lookup may have created the context
+        if (ctx_now == 0) {
+            *ptr = static_cast<uint8_t *>(p);
+            return ZQ_OK;
+        }
+        it = g_noalloc_addr.insert_or_assign({dev, ctx_now}, static_cast<uint8_t *>(p)).first;
     }
     *ptr = it->second;
     return ZQ_OK;
@@ -600,8 +682,7 @@ zq_status zq_linear(const uint16_t *x, const uint32_t *packed, const uint16_t *s
     zq_linear_desc d{x, packed, scales, zeros, out, bits, group, M, N, K};
     zq_status st = check_linear(d);
     if (st != ZQ_OK) return st;
-    std::vector<zq_linear_desc> one{d};
-    return run_batch(one, reinterpret_cast<cudaStream_t>(stream));
+    return checked_stack(&d, 1, reinterpret_cast<cudaStream_t>(stream));
 }
 
 zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
@@ -638,25 +719,16 @@ zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stre
             return fail(st, "op %d: %s", i, msg.c_str());
         }
     }
-    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    std::vector<zq_linear_desc> batch;
-    std::vector<OpRanges> br;
-    constexpr size_t kMaxBatch = 1024;
-    for (int i = 0; i < n_ops; ++i) {
-        const OpRanges r = ranges_of(ops[i]);
-        bool dep = batch.size() >= kMaxBatch;
-        for (size_t j = 0; j < br.size() && !dep; ++j) dep = conflicts(br[j], r);
-        if (dep) {
-            zq_status st = run_batch(batch, s);
-            if (st != ZQ_OK) return st;
-            batch.clear();
-            br.clear();
-        }
-        batch.push_back(ops[i]);
-        br.push_back(r);
-    }
-    if (!batch.empty()) return run_batch(batch, s);
-    return ZQ_OK;
+    return checked_stack(ops, n_ops, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t zq_linear_stack_workspace_bytes(const zq_linear_desc *ops, int n_ops) {
+    if (n_ops < 0 || (n_ops > 0 && ops == nullptr)) return 0;
+    for (int i = 0; i < n_ops; ++i)
+        if (check_linear(ops[i]) != ZQ_OK) return 0;
+    size_t need = 0;
+    if (run_stack(ops, n_ops, nullptr, &need) != ZQ_OK) return 0;
+    return need;
 }
 
 zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes, zq_stream_t stream) {
@@ -671,33 +743,116 @@ zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *cod
 }
 
 zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream) {
-    uint8_t *base = nullptr;
-    return workspace(reinterpret_cast<cudaStream_t>(stream), bytes, &base);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::pair<int, unsigned long long> key;
+    zq_status st = stream_key(s, &key);
+    if (st != ZQ_OK) return st;
+    const size_t need = std::max(bytes, kCounterBytes);
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    Workspace &ws = g_ws[key];
+    if (ws.bytes >= need) return ZQ_OK;
+    // The old buffer may still be in use by work queued on the stream.
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    if (ws.owned && ws.ptr) cudaFree(ws.ptr);
+    ws = Workspace{};
+    void *p = nullptr;
+    e = cudaMalloc(&p, need);
+    if (e != cudaSuccess) {
+        g_ws.erase(key);
+        return cuda_fail(e, "cudaMalloc(workspace)");
+    }
+    e = cudaMemset(p, 0, kCounterBytes);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        g_ws.erase(key);
+        return cuda_fail(e, "cudaMemset(workspace)");
+    }
+    ws.ptr = p;
+    ws.bytes = need;
+    ws.owned = true;
+    return ZQ_OK;
+}
+
+zq_status zq_attach_workspace(void *buffer, size_t bytes, zq_stream_t stream) {
+    if (buffer == nullptr) return fail(ZQ_ERR_INVALID_ARG, "buffer is null");
+    if ((reinterpret_cast<uintptr_t>(buffer) & 255u) != 0)
+        return fail(ZQ_ERR_INVALID_ARG, "buffer is not 256-byte aligned");
+    if (bytes < kCounterBytes)
+        return fail(ZQ_ERR_INVALID_ARG, "a workspace needs at least %zu bytes (got %zu)", kCounterBytes, bytes);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::pair<int, unsigned long long> key;
+    zq_status st = stream_key(s, &key);
+    if (st != ZQ_OK) return st;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    Workspace &ws = g_ws[key];
+    if (ws.owned && ws.ptr) {
+        cudaError_t e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+        cudaFree(ws.ptr);
+    }
+    ws = Workspace{};
+    cudaError_t e = cudaMemsetAsync(buffer, 0, kCounterBytes, s);
+    if (e != cudaSuccess) {
+        g_ws.erase(key);
+        return cuda_fail(e, "clearing the workspace counters");
+    }
+    ws.ptr = buffer;
+    ws.bytes = bytes;
+    return ZQ_OK;
+}
+
+zq_status zq_release_workspace(zq_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    std::pair<int, unsigned long long> key;
+    zq_status st = stream_key(s, &key);
+    if (st != ZQ_OK) return st;
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    auto it = g_ws.find(key);
+    if (it == g_ws.end()) return ZQ_OK;
+    cudaError_t e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    if (it->second.owned && it->second.ptr) {
+        e = cudaFree(it->second.ptr);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFree(workspace)");
+    }
+    g_ws.erase(it);
+    return ZQ_OK;
+}
+
+zq_status zq_release_all_workspaces(void) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    std::lock_guard<std::mutex> lk(g_ws_mu);
+    for (auto it = g_ws.begin(); it != g_ws.end();) {
+        if (it->first.first != dev) {
+            ++it;
+            continue;
+        }
+        if (it->second.owned && it->second.ptr) cudaFree(it->second.ptr);
+        it = g_ws.erase(it);
+    }
+    return ZQ_OK;
 }
 
 size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
-    zq_linear_desc d{nullptr, nullptr, nullptr, nullptr, nullptr, bits, kGroup, M, N, K};
-    if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0 || M > kDecodeMaxM) return 0;
-    std::vector<zq_linear_desc> pieces;
-    split_tokens(d, pieces);
-    size_t worst = 0;
-    // pieces of one op share bits; group them as run_batch would
-    for (int mt : {1, 2}) {
-        std::vector<zq_linear_desc> cls;
-        for (const auto &p : pieces)
-            if (mt_for_m(p.M) == mt) cls.push_back(p);
-        for (size_t i = 0; i < cls.size(); i += kMaxPrepEntries) {
-            std::vector<zq_linear_desc> launch(cls.begin() + i,
-                                               cls.begin() + std::min(cls.size(), i + kMaxPrepEntries));
-            // distinct x per piece: give them distinct fake addresses
-            for (size_t k = 0; k < launch.size(); ++k)
-                launch[k].x = reinterpret_cast<const uint16_t *>(static_cast<uintptr_t>(16 * (k + 1)));
-            size_t b = 0;
-            if (run_decode(launch, bits, mt, nullptr, &b) != ZQ_OK) return 0;
-            worst = std::max(worst, b);
-        }
-    }
-    return worst;
+    if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
+    // the plan needs only the sizes: any aligned, distinct fake pointers do
+    const auto fake = [](uintptr_t i) { return reinterpret_cast<void *>(i << 20); };
+    zq_linear_desc d{static_cast<const uint16_t *>(fake(1)), static_cast<const uint32_t *>(fake(2)),
+                     static_cast<const uint16_t *>(fake(3)), static_cast<const uint16_t *>(fake(4)),
+                     static_cast<uint16_t *>(fake(1 << 20)), bits, kGroup, M, N, K};
+    size_t need = 0;
+    if (run_stack(&d, 1, nullptr, &need) != ZQ_OK) return 0;
+    return need;
+}
+
+zq_status zq_set_wait_limit_ns(uint64_t ns) {
+    g_wait_ns.store(ns);
+    return ZQ_OK;
 }
 
 const char *zq_status_string(zq_status status) {
@@ -726,6 +881,11 @@ zq_status zq_check_device(void) {
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     e = read_kv_error(&err3);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
+    if (err2 != 0) {
+        // A decode kernel that gave up may have left split-K counters set.
+        int dev = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess) workspaces_dirty(dev);
+    }
     if (err != 0 || err2 != 0)
         return fail(static_cast<zq_status>(err ? err : err2), "a kernel gave up a bounded wait");
     if (err3 != 0) return fail(static_cast<zq_status>(err3), "a KV-cache row held NaN or Inf");
@@ -795,3 +955,5 @@ int zq_version(void) { return 100; }
 }  // extern "C"
 
 void zq::set_last_error(const char *msg) { g_last_error = msg; }
+
+unsigned long long zq::wait_limit_ns() { return g_wait_ns.load(); }

@@ -18,9 +18,10 @@
 //  * Codes become biased fp16 pairs, 1024 + q * 2^s, with one LOP3 per two codes
 //    (zq_device.cuh) and go to the tensor cores as they are: the activations
 //    are pre-permuted once per call into the same pair order and pre-scaled by
-//    2^-s (exact), so each product is 1024 * x' + q * x, and the per-group bias
-//    1024 * sum(x') is subtracted in fp32 once per group.  The canonical packed
-//    layout is consumed as stored.
+//    2^(E - s) (exact; E per token and group keeps x' in fp16's normal range),
+//    so each product is 1024 * x' + 2^E * q * x, and the per-group bias
+//    1024 * sum(x') is subtracted, and 2^E divided out, in fp32 once per group.
+//    The canonical packed layout is consumed as stored.
 //  * A CTA step is 64 weight rows x GPS groups.  One ring of shared-memory
 //    stages per CTA, filled in turn by the four warps (stage t by warp t % 4,
 //    the scheduling state handed from one producing warp to the next through
@@ -61,22 +62,39 @@ __device__ __forceinline__ void static_for(F &&f) {
 
 // ------------------------------------------------------------------ prep --
 // One warp per (entry, padded token, group).  Tokens < M: the group's 128
-// activations, pair-permuted and 2^-s-scaled, into xg (M x K, row-major).
+// activations, pair-permuted and scaled by 2^(E - s), into xg (M x K,
+// row-major).  E is chosen per (token, group) from the group's largest |x| so
+// that the scaled values sit near 2^14: whatever the magnitude of the
+// activations (fp16 subnormals included), x' keeps fp16's full precision
+// instead of sliding into the subnormal range, where x * 2^-s would lose bits
+// or flush to zero.  Every scaling is by a power of two, so it is exact and the
+// kernel undoes it with the factor f = 2^-E in fp32.
 // Lane c of the MMA reads 16-byte chunks 4c .. 4c+3 of its token's row; they
 // are stored at x_chunk(c, q, token & 7), so that the 8 lanes of a quarter
 // warp (two tokens x four lanes) always hit 8 different bank groups.  Every
-// padded token gets its (sum x, 1024 * sum x') pair (zeros past M).
+// padded token gets its group record (sum x, -f * 1024 * sum x', f, 0):
+// zeros past M.
 
 __host__ __device__ constexpr int x_chunk(int c, int q, int t7) { return (4 * c + (q ^ (2 * (c >> 1)))) ^ t7; }
 
+// Exponent E of the (token, group) scaling: 2^E * max|x| lies in [2^14, 2^15);
+// E = 0 for an all-zero group.
+__device__ __forceinline__ int prep_exponent(float amax) {
+    if (!(amax > 0.0f)) return 0;
+    const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127;  // floor(log2 amax), amax normal
+    return 14 - ex;
+}
+
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
+
 template <int B>
-__device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow, int lane, int t7) {
+__device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow, int lane, int t7, int E) {
     float bias = 0.0f;  // sum of the scaled activations written by this lane
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const int q = lane + 32 * h;  // 64 pairs per group
         const int c = q / 16, p = q % 16;
-        const float sc = 1.0f / static_cast<float>(1 << pair_shift<B>(p));  // exact power of two
+        const float sc = pow2f(E - pair_shift<B>(p));  // exact power of two
         const __half lo = __float2half_rn(h2f_bits(xrow[32 * c + pair_lo<B>(p)]) * sc);
         const __half hi = __float2half_rn(h2f_bits(xrow[32 * c + pair_hi<B>(p)]) * sc);
         bias += __half2float(lo) + __half2float(hi);
@@ -99,9 +117,9 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
         const long long local = gw - p.warp_prefix[e];
         const int G = en.K / kGroup;
         const int t = static_cast<int>(local / G), g = static_cast<int>(local % G);
-        float2 *dst = reinterpret_cast<float2 *>(en.sx) + static_cast<size_t>(g) * en.M_pad + t;
+        float4 *dst = reinterpret_cast<float4 *>(en.sx) + static_cast<size_t>(g) * en.M_pad + t;
         if (t >= en.M) {
-            if (lane == 0) *dst = make_float2(0.0f, 0.0f);
+            if (lane == 0) *dst = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             if (t < en.x_rows)
                 reinterpret_cast<uint2 *>(en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup)[lane] =
                     make_uint2(0u, 0u);
@@ -109,21 +127,29 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
             const uint16_t *xrow = en.x + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             uint16_t *prow = en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             const uint2 v = reinterpret_cast<const uint2 *>(xrow)[lane];
-            float s = h2f_bits(v.x & 0xFFFFu) + h2f_bits(v.x >> 16) + h2f_bits(v.y & 0xFFFFu) +
-                      h2f_bits(v.y >> 16);
+            const float x0 = h2f_bits(v.x & 0xFFFFu), x1 = h2f_bits(v.x >> 16);
+            const float x2 = h2f_bits(v.y & 0xFFFFu), x3 = h2f_bits(v.y >> 16);
+            float s = x0 + x1 + x2 + x3;
+            float amax = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            const int E = prep_exponent(amax);
             float b;
             switch (en.bits) {
-                case 2: b = prep_group<2>(xrow, prow, lane, t & 7); break;
-                case 3: b = prep_group<3>(xrow, prow, lane, t & 7); break;
-                case 4: b = prep_group<4>(xrow, prow, lane, t & 7); break;
-                default: b = prep_group<8>(xrow, prow, lane, t & 7); break;
+                case 2: b = prep_group<2>(xrow, prow, lane, t & 7, E); break;
+                case 3: b = prep_group<3>(xrow, prow, lane, t & 7, E); break;
+                case 4: b = prep_group<4>(xrow, prow, lane, t & 7, E); break;
+                default: b = prep_group<8>(xrow, prow, lane, t & 7, E); break;
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
                 s += __shfl_xor_sync(0xffffffffu, s, o);
                 b += __shfl_xor_sync(0xffffffffu, b, o);
             }
-            if (lane == 0) *dst = make_float2(s, 1024.0f * b);
+            // f * (acc - 1024 * b) = fma(acc, f, -f * 1024 * b): the products
+            // by the power of two f are exact.
+            const float f = pow2f(-E);
+            if (lane == 0) *dst = make_float4(s, -(f * (1024.0f * b)), f, 0.0f);
         }
     }
     // Dependents may be scheduled only now, i.e. after everything enqueued
@@ -245,16 +271,18 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint32_t (&w)[2
 // Device record of a decode kernel that gave up a bounded wait (ZQ_ERR_TIMEOUT).
 __device__ int g_decode_error;
 
-constexpr unsigned long long kDecodeWaitNs = 2000000000ull;  // 2 s
+// Bound of the drain after an abort, which waits for copies already issued
+// and does not follow the adjustable limit of the other waits (p.wait_ns).
+constexpr unsigned long long kDecodeDrainNs = 2000000000ull;  // 2 s
 
 // Bounded wait of the whole warp for a phase of `bar`; the answer is the same
 // in every lane (a lane that ran out makes the warp give up).
-__device__ __forceinline__ bool wait_phase(unsigned long long *bar, uint32_t parity) {
+__device__ __forceinline__ bool wait_phase(unsigned long long *bar, uint32_t parity, unsigned long long limit) {
     bool ok = mbar_try_wait(bar, parity);
     if (!ok) {
         const unsigned long long t0 = globaltimer();
         while (!(ok = mbar_try_wait(bar, parity)))
-            if (globaltimer() - t0 > kDecodeWaitNs) break;
+            if (globaltimer() - t0 > limit) break;
     }
     return __all_sync(0xffffffffu, ok);
 }
@@ -280,12 +308,12 @@ __device__ __forceinline__ int ld_acquire_shared(const int *a) {
 
 // Bounded wait of the whole warp until *seq == target; it sleeps between
 // polls so that a waiting warp leaves the issue slots to the others.
-__device__ __forceinline__ bool wait_seq(const int *seq, int target) {
+__device__ __forceinline__ bool wait_seq(const int *seq, int target, unsigned long long limit) {
     bool ok = ld_acquire_shared(seq) == target;
     if (!ok) {
         const unsigned long long t0 = globaltimer();
         while (!(ok = ld_acquire_shared(seq) == target)) {
-            if (globaltimer() - t0 > kDecodeWaitNs) break;
+            if (globaltimer() - t0 > limit) break;
             __nanosleep(64);
         }
     }
@@ -369,7 +397,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
     // Fills stage `target` (after its previous contents were released by all
     // warps); false if a wait ran out.  Whole warp, uniform control flow.
     auto produce = [&](int target) -> bool {
-        if (!wait_seq(&ps->seq, target)) return false;
+        if (!wait_seq(&ps->seq, target, p.wait_ns)) return false;
         Cursor ld;
         ld.s = ps->s;
         ld.o = ps->o;
@@ -384,7 +412,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
             return true;
         }
         const int slot_ld = target % D, round_ld = target / D;
-        if (round_ld > 0 && !wait_phase(&empty[slot_ld], (round_ld - 1) & 1)) return false;
+        if (round_ld > 0 && !wait_phase(&empty[slot_ld], (round_ld - 1) & 1, p.wait_ns)) return false;
         if (!ld.valid && p.dynamic) {
             // Chunks only grow, so a CTA stops at its first ticket past the end
             // and never holds an unused valid one.
@@ -434,12 +462,12 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                 dsc[0] = make_int4(ld.o, ld.rb, ld.j, ng | (flags << 8));
                 dsc[1] = make_int4(ld_chunk, unit_start, op.M, 0);
                 const uint32_t xbytes = static_cast<uint32_t>(ng * xrows * 256);
-                const uint32_t sbytes = static_cast<uint32_t>(ng * MPAD * 8);
+                const uint32_t sbytes = static_cast<uint32_t>(ng * MPAD * 16);
                 mbar_arrive_expect_tx(&full[slot_ld], NBOX * BOXB + xbytes + sbytes);
 #pragma unroll
                 for (int b = 0; b < NBOX; ++b)
                     tma_load_2d(st + b * BOXB, &op.tmap, g0 * GB + b * BOXW, ld.rb * kDecodeCtaRows, &full[slot_ld]);
-                bulk_load(sm + p.off_sx, op.sx + static_cast<size_t>(g0) * MPAD * 2, sbytes, &full[slot_ld]);
+                bulk_load(sm + p.off_sx, op.sx + static_cast<size_t>(g0) * MPAD * 4, sbytes, &full[slot_ld]);
             }
             __syncwarp();
             // Activations: token t's ng groups (ng * 256 contiguous bytes), one
@@ -485,8 +513,8 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
     //          chunk index is ((gi*GB % 128)/16) ^ lanex.
     //   x':    token gq's staged row is GPS*256 bytes, group gi at +gi*256,
     //          the lane's chunk q of it at x_chunk(c, q, gq).
-    //   sums:  (sum x, bias) of tokens (8mt + 2c, +1) of group gi at
-    //          off_sx + (gi*MPAD + 8mt + 2c) * 8.
+    //   sums:  (sum x, -f * bias, f, 0) of token 8mt + 2c of group gi at
+    //          off_sx + (gi*MPAD + 8mt + 2c) * 16, token 8mt + 2c + 1 16 bytes on.
     int lanex;
     if constexpr (BITS == 4) lanex = c ^ gr;
     else if constexpr (BITS == 2) lanex = (c >> 1) ^ gr;
@@ -510,7 +538,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
     uint32_t xq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) xq[q] = p.off_x + gq * (GPS * 256) + (x_chunk(c, q, gq) << 4);
-    const uint32_t sxo = p.off_sx + 16 * c;
+    const uint32_t sxo = p.off_sx + 32 * c;
     const uint32_t szq0 = p.off_sz + (warp * 16 + gr) * 2 * SZB, szq1 = p.off_sz + (warp * 16 + 8 + gr) * 2 * SZB;
     const uint32_t ring_s = smem_u32(ring), meta_s = smem_u32(meta);
 
@@ -547,7 +575,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                 }
             }
         }
-        if (!wait_phase(&full[slot], par)) {
+        if (!wait_phase(&full[slot], par, p.wait_ns)) {
             aborted = true;
             break;
         }
@@ -647,20 +675,25 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                         xf[4 * q + 3] = v.w;
                     }
                 }
-                const uint4 sbv = lds_v4(smb + sxo + (gi * MPAD + 8 * mt) * 8);
-                const float4 sb = make_float4(__uint_as_float(sbv.x), __uint_as_float(sbv.y),
-                                              __uint_as_float(sbv.z), __uint_as_float(sbv.w));
+                const uint32_t sa_a = smb + sxo + (gi * MPAD + 8 * mt) * 16;
+                const uint2 sa = lds_v2(sa_a);
                 float acc[4];
                 mma_group<BITS, MT == 1>(acc, wv, xf, magic);
-                // tot += s * (acc - bias) + z * sum(x); with one token the odd
-                // C columns are padding.
+                const float fa = __uint_as_float(lds_u32(sa_a + 8));
+                // tot += s * f * (acc - bias) + z * sum(x), with f * (acc - bias)
+                // as one FMA (f is the token's power-of-two x' scale); with one
+                // token the odd C columns are padding.
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
-                    tot[mt][2 * h] = fmaf(sc[h], acc[2 * h] - sb.y, fmaf(zr[h], sb.x, tot[mt][2 * h]));
+                    tot[mt][2 * h] = fmaf(sc[h], fmaf(acc[2 * h], fa, __uint_as_float(sa.y)),
+                                          fmaf(zr[h], __uint_as_float(sa.x), tot[mt][2 * h]));
                 if constexpr (!one_token) {
+                    const uint4 sb = lds_v4(smb + sxo + (gi * MPAD + 8 * mt) * 16 + 16);
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
-                        tot[mt][2 * h + 1] = fmaf(sc[h], acc[2 * h + 1] - sb.w, fmaf(zr[h], sb.z, tot[mt][2 * h + 1]));
+                        tot[mt][2 * h + 1] =
+                            fmaf(sc[h], fmaf(acc[2 * h + 1], __uint_as_float(sb.z), __uint_as_float(sb.y)),
+                                 fmaf(zr[h], __uint_as_float(sb.x), tot[mt][2 * h + 1]));
                 }
             }
         };
@@ -756,7 +789,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
         const int filled = ld_acquire_shared(&ps->seq);
         for (int k = n_seen; k < filled; ++k) {
             const unsigned long long t0 = globaltimer();
-            while (!mbar_try_wait(&full[k % D], (k / D) & 1u) && globaltimer() - t0 < kDecodeWaitNs) {
+            while (!mbar_try_wait(&full[k % D], (k / D) & 1u) && globaltimer() - t0 < kDecodeDrainNs) {
             }
         }
     }

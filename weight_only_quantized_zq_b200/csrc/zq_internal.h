@@ -35,8 +35,9 @@ struct alignas(64) DecodeOp {
     const uint16_t *scales;
     const uint16_t *zeros;
     const uint16_t *xg;     // workspace: (M, or M_pad with several token tiles) x K fp16, pair-permuted,
-                            // 2^-s-scaled, chunk-swizzled activations
-    const float *sx;        // workspace: G x M_pad x 2 fp32 (sum x, 1024 * sum x') per group and token
+                            // 2^(E-s)-scaled, chunk-swizzled activations
+    const float *sx;        // workspace: G x M_pad x 4 fp32 (sum x, -f * 1024 * sum x', f, 0) per group and
+                            // token; f = 2^-E undoes the token's power-of-two x' scale
     uint16_t *out;          // M x N fp16
     int step0;              // first CTA step of this op
     int unit0;              // first row block of this op (counted over the launch)
@@ -60,6 +61,7 @@ struct DecodeParams {
     int codes_bytes;         // codes of one stage (64 rows x one step's bytes), multiple of 1024
     int meta_bytes;          // rest of one stage, multiple of 16
     int off_sz, off_sx, off_x, off_desc;  // offsets inside a stage's meta part
+    unsigned long long wait_ns;           // limit of a bounded wait (see wait_limit_ns)
     DecodeOp ops[kMaxDecodeOps];
 };
 static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
@@ -67,7 +69,7 @@ static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
     uint16_t *xg;       // x_rows x K, chunk-swizzled per group and token; rows >= M are zeros
-    float *sx;          // G x M_pad x 2: (sum of x, 1024 * sum of scaled x)
+    float *sx;          // G x M_pad x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0)
     int M, M_pad, x_rows, K, bits;
 };
 
@@ -129,6 +131,7 @@ struct alignas(64) PrefillOp {
 struct PrefillGroup {
     int n_ops;
     int n_tiles;
+    unsigned long long wait_ns;  // limit of a bounded wait (see wait_limit_ns)
     PrefillOp ops[kMaxPrefillOps];
 };
 static_assert(sizeof(PrefillGroup) <= 32000, "kernel parameter space");
@@ -138,6 +141,9 @@ int prefill_tiles(int M, int N);
 cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, cudaStream_t stream);
 cudaError_t read_prefill_error(int *err);
 cudaError_t read_decode_error(int *err);
+// Limit of the kernels' bounded waits, passed to every launch as a kernel
+// parameter (2 s unless the test hook zq_set_wait_limit_ns changed it).
+unsigned long long wait_limit_ns();
 cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t dim0,
                                  uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
                                  CUtensorMapSwizzle swizzle);

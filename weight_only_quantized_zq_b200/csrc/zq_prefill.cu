@@ -59,13 +59,17 @@ constexpr int kTmaWarp = 4;
 constexpr int kMmaWarp = 5;
 constexpr int kDqWarp0 = 6;
 constexpr int kTmemCols = 512;
-constexpr unsigned long long kWaitNs = 2000000000ull;  // 2 s
+// Drains after an abort wait for copies and MMAs already issued; they ignore
+// the abort flag and the adjustable limit and give up only after this bound.
+constexpr unsigned long long kDrainNs = 2000000000ull;  // 2 s
 
 struct Ctl {
-    unsigned long long full[kMaxStages];
+    unsigned long long full[kMaxStages];   // W slab dequantized (one arrival per dequant warp)
+    unsigned long long xfull[kMaxStages];  // x slab landed (the TMA warp's expect_tx + the copy's bytes)
     unsigned long long empty[kMaxStages];
     unsigned long long acc_full;
     unsigned long long acc_empty;
+    unsigned long long mma_done;           // every tcgen05.mma this CTA issued has completed
     uint32_t tmem_base;
     int abort;
 };
@@ -99,20 +103,29 @@ struct Plan {
 };
 
 // Bounded wait: false if the CTA is aborting or the limit was reached.
-__device__ __noinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *abort) {
+__device__ __noinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *abort,
+                                       unsigned long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((it & 15u) == 0) {
             if (*abort) return false;
-            if (globaltimer() - t0 > kWaitNs) {
+            if (globaltimer() - t0 > limit) {
                 *abort = 1;
                 atomicExch(&g_prefill_error, 5);  // ZQ_ERR_TIMEOUT
                 return false;
             }
         }
     }
+}
+
+// Wait of a drain: for a phase that work already issued will complete; no
+// abort check, bounded by kDrainNs.
+__device__ __noinline__ void mbar_drain(unsigned long long *bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kDrainNs) break;
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -193,15 +206,37 @@ __device__ __forceinline__ TileRef locate(const PrefillGroup &p, int t) {
     return TileRef{lo, (local / tt) * kRowTile, (local % tt) * kTokTile};
 }
 
-// Dequantize this thread's 32-code chunk of one W row into 4 x 16 bytes of
-// natural-K-order fp16 (q*s + z, one rounding), via the shared unpack.
+// True when some code of the group dequantizes past the fp16 range: the top
+// of the group, L*s + z (s >= 0, so every q*s + z is at most that), rounds to
+// +inf.  Only groups whose range reaches the fp16 limit (|w| near 65504) do.
 template <int B>
-__device__ __forceinline__ void dequant_chunk(const uint32_t (&w)[B], uint32_t sz, uint32_t (&o)[16]) {
+__device__ __forceinline__ bool dequant_overflows(uint32_t sz) {
+    constexpr uint32_t kL2 = (B == 2 ? 0x4200u : B == 3 ? 0x4700u : B == 4 ? 0x4B80u : 0x5BF8u) * 0x10001u;  // (L, L)
+    const uint32_t top = hfma2_bits(kL2, (sz & 0xFFFFu) * 0x10001u, (sz >> 16) * 0x10001u);
+    return (top & 0x7FFFu) == 0x7C00u;
+}
+
+__device__ __forceinline__ uint32_t hmin2_bits(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("min.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Dequantize this thread's 32-code chunk of one W row into 4 x 16 bytes of
+// natural-K-order fp16 (q*s + z, one rounding), via the shared unpack.  In a
+// group that reaches past the fp16 range (`ovf`), values that round to +inf
+// are held at 65504, the largest finite fp16 (a relative change below 2^-11).
+template <int B>
+__device__ __forceinline__ void dequant_chunk(const uint32_t (&w)[B], uint32_t sz, uint32_t (&o)[16], bool ovf) {
     const uint32_t s2 = (sz & 0xFFFFu) * 0x10001u;  // (s, s)
     const uint32_t z2 = (sz >> 16) * 0x10001u;      // (z, z)
     uint32_t v[16];
 #pragma unroll
     for (int p = 0; p < 16; ++p) v[p] = hfma2_bits(unpack_pair<B>(w, p), s2, z2);
+    if (ovf) {
+#pragma unroll
+        for (int p = 0; p < 16; ++p) v[p] = hmin2_bits(v[p], 0x7BFF7BFFu);
+    }
     // Pairs p (even) and p+1 hold codes (lo, hi) and (lo+1, hi+1): two PRMTs
     // give the natural pairs (lo, lo+1) and (hi, hi+1).
 #pragma unroll
@@ -343,13 +378,17 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         const uint32_t z = opaque_zero();  // orders the slot loads after the wait
         const uint32_t cs = smem_u32(scode + (i % kS) * P::kSlotBytes) + z;
         uint32_t sz[RPT];
+        bool ovf[RPT];
 #pragma unroll
-        for (int r = 0; r < RPT; ++r) sz[r] = lds_u32(cs + P::kSlotCodes + 4 * (r * NT + d));
+        for (int r = 0; r < RPT; ++r) {
+            sz[r] = lds_u32(cs + P::kSlotCodes + 4 * (r * NT + d));
+            ovf[r] = dequant_overflows<B>(sz[r]);
+        }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // the two slabs of this group
             const int st = it % P::kStages;
             const uint32_t round = it / P::kStages;
-            if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort)) return false;
+            if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) return false;
             uint8_t *bs = sb + st * kSlabB;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
@@ -369,7 +408,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                 }
                 const int row = rows[r];
                 uint32_t o[16];
-                dequant_chunk<B>(w, sz[r], o);
+                dequant_chunk<B>(w, sz[r], o, ovf[r]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c16 = (4 * ch + j) ^ (row & 7);
@@ -419,11 +458,13 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P::kStages; ++s) {
-            mbar_init(&sm.full[s], 1 + P::kDqWarps);
+            mbar_init(&sm.full[s], P::kDqWarps);
+            mbar_init(&sm.xfull[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         mbar_init(&sm.acc_full, 1);
         mbar_init(&sm.acc_empty, kEpiWarps);
+        mbar_init(&sm.mma_done, 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -451,35 +492,42 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                 for (int s = 0; s < slabs; ++s, ++it) {
                     const int st = it % P::kStages;
                     const uint32_t round = it / P::kStages;
-                    if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) break;
-                    mbar_arrive_expect_tx(&sm.full[st], P::kSlabA);
-                    tma_load_2d(sa + st * P::kSlabA, &op.xmap, s * kBK, tr.t0, &sm.full[st]);
+                    if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) break;
+                    mbar_arrive_expect_tx(&sm.xfull[st], P::kSlabA);
+                    tma_load_2d(sa + st * P::kSlabA, &op.xmap, s * kBK, tr.t0, &sm.xfull[st]);
                 }
             }
-            // Let copies still in flight land before the CTA can exit.
+            // Copies still in flight (only after an abort) must land before
+            // the CTA can exit.  `it` copies were issued; a slot is refilled only
+            // after the MMA consumed its previous copy, so only the last
+            // kStages can be pending, one per slot.  The x-only barriers
+            // complete on the copies' bytes alone, whatever the other roles did.
             for (uint32_t k = 0; k < P::kStages && k < it; ++k) {
                 const uint32_t j = it - 1 - k;
-                mbar_wait(&sm.full[j % P::kStages], (j / P::kStages) & 1u, abort);
+                mbar_drain(&sm.xfull[j % P::kStages], (j / P::kStages) & 1u);
             }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0) {
             uint32_t it = 0, tile_i = 0;
+            bool issued = false;
             for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
                 const TileRef tr = locate(p, t);
                 const int slabs = p.ops[tr.o].K / kBK;
                 // the second 128-token half only when it holds tokens
                 const bool half1 = !ONE && tr.t0 + 128 < p.ops[tr.o].M;
-                if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort)) break;
+                if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort, p.wait_ns)) break;
                 tc_fence_after();
                 bool ok = true;
                 for (int s = 0; s < slabs; ++s, ++it) {
                     const int st = it % P::kStages;
-                    if (!mbar_wait(&sm.full[st], (it / P::kStages) & 1u, abort)) {
+                    if (!mbar_wait(&sm.xfull[st], (it / P::kStages) & 1u, abort, p.wait_ns) ||
+                        !mbar_wait(&sm.full[st], (it / P::kStages) & 1u, abort, p.wait_ns)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
+                    issued = true;
                     const uint32_t a0 = smem_u32(sa + st * P::kSlabA);
                     const uint32_t b0 = smem_u32(sb + st * kSlabB);
                     if (half1) {
@@ -501,6 +549,12 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                 }
                 if (!ok) break;
                 umma_commit(&sm.acc_full);
+            }
+            // Every MMA issued must have completed before TMEM is freed and the
+            // CTA exits (after an abort no epilogue waited for them).
+            if (issued) {
+                umma_commit(&sm.mma_done);
+                mbar_drain(&sm.mma_done, 0u);
             }
         }
     } else if (warp >= kDqWarp0) {
@@ -555,6 +609,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                     for (int q = 0; q < B; ++q) wc[h][i][q] = wn[h][i][q];
             szc[0] = szn[0];
             szc[1] = szn[1];
+            const bool ovf[2] = {dequant_overflows<B>(szc[0]), dequant_overflows<B>(szc[1])};
             int t_n = t, g_n = g + 1;
             groups_n = groups;
             if (g_n == groups) {
@@ -567,7 +622,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
             for (int h = 0; h < 2; ++h) {  // the two slabs of this group
                 const int st = it % P::kStages;
                 const uint32_t round = it / P::kStages;
-                if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort)) {
+                if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) {
                     ok = false;
                     break;
                 }
@@ -576,7 +631,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                 for (int i = 0; i < 2; ++i) {
                     const int row = d / 2 + 128 * i;
                     uint32_t o[16];
-                    dequant_chunk<B>(wc[h][i], szc[i], o);
+                    dequant_chunk<B>(wc[h][i], szc[i], o, ovf[i]);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int c16 = (4 * ch + j) ^ (row & 7);
@@ -598,7 +653,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = tokens of each half.
         uint32_t tile_i = 0;
         for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
-            if (!mbar_wait(&sm.acc_full, tile_i & 1u, abort)) break;
+            if (!mbar_wait(&sm.acc_full, tile_i & 1u, abort, p.wait_ns)) break;
             tc_fence_after();
             const TileRef tr = locate(p, t);
             const PrefillOp &op = p.ops[tr.o];
