@@ -58,13 +58,11 @@ MEASURED_TRAFFIC = {
     ("decode", "7b", 1): {
         "sha256": "de5ba2b057c180a01e9bb424bb070c58dd692ae81c675a7a034337d946fed283",
         "bytes_per_layer": 125936384,
-        "profile": "profiles/decode_kernel_m1_4layers.md",
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
         "sha256": "260f2fe4c7aa0f6d088d2e6e869092dca1d8734c3b4b93f72061af7d315bb0e1",
         "bytes_per_layer": 130899200,
-        "profile": "profiles/prefill_kernel_m64_1layer.md",
     },
 }
 NOMINAL_HBM_GBS = 8000.0
@@ -249,9 +247,11 @@ def decode_stack_shapes(layers=zi.QWEN7B_LAYERS, model="7b"):
 
 class StackWorkload:
     """All tensors of the decode stack resident on the GPU: one contiguous x
-    buffer, one contiguous out buffer (views per op), packed weights per op."""
+    buffer, one contiguous out buffer (views per op), packed weights per op.
+    `weights` (another workload's .weights of the same model and layers) are
+    reused instead of drawing and quantizing new ones."""
 
-    def __init__(self, zq, M, device, layers=zi.QWEN7B_LAYERS, model="7b"):
+    def __init__(self, zq, M, device, layers=zi.QWEN7B_LAYERS, model="7b", weights=None):
         self.M = M
         shapes = decode_stack_shapes(layers, model)
         outliers = model == "32b-mixed"
@@ -268,10 +268,13 @@ class StackWorkload:
         self.out_all = torch.empty(out_elems, dtype=torch.float16, device=device)
         self.ops, self.weights, self.bytes, self.flops = [], [], 0, 0
         ooff = 0
-        for (layer, t, name, N, K, bits) in shapes:
-            w = zi.weight(N, K, zi.seed_for(layer, t), device=device, outliers=outliers)
-            q = zq.quantize(w, bits)
-            del w
+        for i, (layer, t, name, N, K, bits) in enumerate(shapes):
+            if weights is None:
+                w = zi.weight(N, K, zi.seed_for(layer, t), device=device, outliers=outliers)
+                q = zq.quantize(w, bits)
+                del w
+            else:
+                q = weights[i][5]
             out = self.out_all[ooff:ooff + M * N].view(M, N)
             ooff += M * N
             self.weights.append((layer, name, N, K, bits, q))
@@ -337,14 +340,17 @@ def time_oracle(items, M, budget_s=None):
     return done_bytes / el / 1e9, el, done_bytes, orc.get_threads()
 
 
+CONFIG1_SEED = 0  # the single-layer workload draws W and x from seed 0
+
+
 def oracle_config1_one_core(budget_s=0.5):
-    """The small single-layer workload (M=1, N=K=512, INT4; W seed 0, x seed
-    15) through the oracle on one host core, repeated for budget_s: time per
-    call and GB/s of algorithmic bytes."""
+    """The small single-layer workload (M=1, N=K=512, INT4; W and x seed 0)
+    through the oracle on one host core, repeated for budget_s: time per call
+    and GB/s of algorithmic bytes."""
     import oracle as orc
-    w = zi.weight(512, 512, 0).numpy()
+    w = zi.weight(512, 512, CONFIG1_SEED).numpy()
     p, s, z = orc.quantize_pack(w, 4)
-    x = zi.activations(1, 512, zi.X_SEED).numpy().view(np.uint16)
+    x = zi.activations(1, 512, CONFIG1_SEED).numpy().view(np.uint16)
     prev = orc.get_threads()
     orc.set_threads(1)
     try:
@@ -359,7 +365,122 @@ def oracle_config1_one_core(budget_s=0.5):
         orc.set_threads(prev)
     us = el / calls * 1e6
     return {"us_per_call": us, "value": op_bytes(1, 512, 512, 4) / (us * 1e-6) / 1e9, "unit": "GB/s",
-            "cores": 1, "sample": f"M=1, N=K=512, INT4 g128: {calls} oracle calls in {el:.2f} s"}
+            "cores": 1, "sample": f"M=1, N=K=512, INT4 g128, W and x seed 0: {calls} oracle calls in {el:.2f} s"}
+
+
+# ------------------------------------------------------- all five configs --
+
+def _timed(fn, stream, steps, warmup, device_index):
+    """Mean device time per call of fn (CUDA events on `stream`, after
+    warm-up, synchronised on both sides) and the clocks seen meanwhile."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device_index) as clk:
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / steps, clk.summary()
+
+
+def _hbm_entry(workload, nbytes, ms, peaks, clocks, **extra):
+    gbs = nbytes / (ms / 1e3) / 1e9
+    d = {"workload": workload, "value": gbs, "unit": "GB/s", "ms": ms,
+         "bound": "hbm", "frac": gbs / peaks["hbm_gbs"], "peak": peaks["hbm_gbs"],
+         "pct_of_8tbs": 100 * gbs / NOMINAL_HBM_GBS, "algorithmic_bytes": nbytes, "clocks": clocks}
+    d.update(extra)
+    return d
+
+
+def run_all_configs(zq, wl, dev, stream, peaks, args, device_index):
+    """Every workload the method is specified on, each timed on its own after
+    the headline (which they do not touch): the single 512 x 512 layer, the
+    four 7B-shaped projections one call at a time, the 7B stack at M = 4, 16
+    and 64 and at M = 2048 (prefill), and the 32B-shaped mixed-precision stack.
+    The 7B workloads reuse the headline's 28 layers of weights."""
+    import oracle as orc
+    sp = stream.cuda_stream
+    out = {}
+
+    # Config 1: M = 1, N = K = 512, INT4; W quantized by the oracle; 8 copies
+    # in rotation (all of them fit in L2: the call is latency-bound).
+    N = K = 512
+    p, sc, z = orc.quantize_pack(zi.weight(N, K, CONFIG1_SEED).numpy(), 4)
+    copies = [tuple(torch.from_numpy(a.view(np.int32 if a.dtype == np.uint32 else np.int16).copy()).to(dev)
+                    for a in (p, sc, z)) for _ in range(8)]
+    x1 = zi.activations(1, K, CONFIG1_SEED, device=dev)
+    y1 = torch.empty(1, N, dtype=torch.float16, device=dev)
+    zq.ensure_workspace(zq.zq_linear_workspace_bytes(4, 1, N, K), stream)
+    state = {"i": 0}
+
+    def call1():
+        q = copies[state["i"] % 8]
+        state["i"] += 1
+        zq.zq_linear(x1, q[0], q[1], q[2], 4, 128, 1, N, K, y1, sp)
+
+    ms, clk = _timed(call1, stream, 400, 20, device_index)
+    out["config1_single_layer"] = _hbm_entry(
+        "M=1, N=K=512, INT4 g128, one zq_linear call (W and x seed 0; 8 weight copies in rotation, "
+        "141 KB each, L2-resident: latency-bound, not gated on the roofline)",
+        op_bytes(1, N, K, 4), ms, peaks, clk, us_per_call=ms * 1e3)
+
+    # Config 2: the four 7B-shaped projections at M = 1, one zq_linear call each,
+    # rotating over the 28 layers' distinct weights (3.47 GB, no L2 reuse).
+    per = {}
+    x_by_k = {K: wl.x[K][:1] for K in wl.x}
+    for t, (name, N, K, bits) in enumerate(MODELS["7b"][0]):
+        layers = [w for w in wl.weights if w[1] == name]
+        yb = torch.empty(1, N, dtype=torch.float16, device=dev)
+        zq.ensure_workspace(zq.zq_linear_workspace_bytes(bits, 1, N, K), stream)
+
+        def calls(layers=layers, N=N, K=K, bits=bits, yb=yb):
+            for (_, _, _, _, _, q) in layers:
+                zq.zq_linear(x_by_k[K], q[0], q[1], q[2], bits, 128, 1, N, K, yb, sp)
+
+        ms, clk = _timed(calls, stream, 10, 3, device_index)
+        ms_call = ms / len(layers)
+        per[name] = _hbm_entry(f"{name} {N}x{K} INT4, M=1, one zq_linear call", op_bytes(1, N, K, bits),
+                               ms_call, peaks, clk, us_per_call=ms_call * 1e3)
+    out["config2_7b_projections_m1"] = per
+
+    # Config 3 at M = 4, 16, 64 and config 5 (M = 2048): the 28-layer 7B stack.
+    for M, steps, key in ((4, 20, "config3_7b_stack_m4"), (16, 20, "config3_7b_stack_m16"),
+                          (64, 20, "config3_7b_stack_m64"), (2048, 5, "config5_7b_prefill_m2048")):
+        w2 = StackWorkload(zq, M, dev, zi.QWEN7B_LAYERS, "7b", weights=wl.weights)
+        zq.ensure_workspace(zq.zq_linear_stack_workspace_bytes(w2.descs, w2.n_ops), stream)
+        ms, clk = _timed(lambda w2=w2: zq.zq_linear_stack(w2.descs, w2.n_ops, sp), stream, steps, 3,
+                         device_index)
+        name = f"28-layer 7B-shaped INT4 stack, M={M}, one zq_linear_stack call"
+        if M <= 64:
+            out[key] = _hbm_entry(name, w2.bytes, ms, peaks, clk, tokens_per_s_equiv=M / (ms / 1e3))
+        else:
+            tf = w2.flops / (ms / 1e3) / 1e12
+            out[key] = {"workload": name, "value": tf, "unit": "TFLOP/s", "ms": ms, "bound": "tensor",
+                        "frac": tf / peaks["bf16_tflops"], "peak": peaks["bf16_tflops"],
+                        "peak_note": "measured dense bf16 burst rate (a step of tens of ms timed alone); "
+                                     "fp16 has the same dense rate",
+                        "frac_of_nominal_2250": tf / 2250.0, "algorithmic_flops": w2.flops,
+                        "tokens_per_s_equiv": M / (ms / 1e3), "clocks": clk}
+        del w2
+        torch.cuda.empty_cache()
+
+    # Config 4: the 32B-shaped mixed-precision stack (INT8 qkv, INT4 o, INT3
+    # gate_up, INT2 down, 0.1% outliers x20) at M = 1.
+    L32 = args.extra_32b_layers
+    w4 = StackWorkload(zq, 1, dev, L32, "32b-mixed")
+    zq.ensure_workspace(zq.zq_linear_stack_workspace_bytes(w4.descs, w4.n_ops), stream)
+    ms, clk = _timed(lambda: zq.zq_linear_stack(w4.descs, w4.n_ops, sp), stream, 20, 3, device_index)
+    out["config4_32b_mixed_m1"] = _hbm_entry(
+        f"{L32}-layer 32B-shaped mixed-precision stack (qkv 7168x5120 INT8, o 5120x5120 INT4, "
+        f"gate_up 55296x5120 INT3, down 5120x27648 INT2), M=1, one zq_linear_stack call "
+        f"({w4.bytes / 1e9:.2f} GB of weights, larger than L2)", w4.bytes, ms, peaks, clk,
+        tokens_per_s_equiv=1 / (ms / 1e3), layers=L32)
+    del w4
+    torch.cuda.empty_cache()
+    return out
 
 
 # ------------------------------------------------------------------- arms --
@@ -473,16 +594,20 @@ def run_zq(args):
                                if M <= 16 else tile_kernel)}
     else:
         tflops = wl.flops / (ms_step / 1e3) / 1e12
-        peak = peaks["bf16_tflops_sustained"]
+        peak = peaks["bf16_tflops"]  # burst: a step of tens of ms, timed alone
         traffic = measured_traffic("prefill", args.model, M, args.layers)
         roofline = {"bound": "tensor", "achieved": tflops, "peak": peak, "unit": "TFLOP/s",
                     "frac": tflops / peak,
                     "traffic": None if traffic is None else traffic / (4 * args.layers),
                     "traffic_note": "per launch, averaged over the 4 projections of a layer",
                     "algorithmic_flops": wl.flops,
-                    "peak_source": peaks["source"] + " (dense bf16 sustained; fp16 has the same dense rate)",
+                    "peak_source": peaks["source"] + " (dense bf16 burst; fp16 has the same dense rate)",
                     "kernel": tile_kernel,
                     "tflops_vs_nominal_2250": tflops / 2250.0}
+
+    configs = None
+    if world == 1 and not args.no_extra:
+        configs = run_all_configs(zq, wl, dev, stream, peaks, args, local)
 
     line = None
     if rank == 0:
@@ -509,7 +634,8 @@ def run_zq(args):
                         "d2h_bytes_per_step": wl.out_all.numel() * 2,
                         "ms_per_step": e2e_ms / args.steps},
                 "gpu_launches": launches,
-                "clocks": clk.summary()}
+                "clocks": clk.summary(),
+                "configs": configs}
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.destroy_process_group()
@@ -533,6 +659,10 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--ref-frac", type=float, default=0.25, help="row fraction per reference step")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads (single layer, projections, M = 4/16/64/2048, 32B mixed)")
+    ap.add_argument("--extra-32b-layers", type=int, default=16,
+                    help="layers of the 32B mixed-precision stack among the other workloads")
     args = ap.parse_args(argv)
     if args.layers is None:
         args.layers = MODELS[args.model][1]

@@ -33,7 +33,9 @@ EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_quantize_pack_symmetric", 
            "zq_version",
            "zq_zse_open", "zq_zse_close", "zq_zse_flags", "zq_zse_tensor_count", "zq_zse_tensor_info",
            "zq_zse_find", "zq_zse_section", "zq_zse_weight_bytes", "zq_zse_verify", "zq_zse_load_weights",
-           "zq_kv_plane_bytes", "zq_kv_append", "zq_kv_gather")
+           "zq_kv_plane_bytes", "zq_kv_append", "zq_kv_gather",
+           "zq_linear_partial", "zq_linear_partial_stack", "zq_linear_partial_stack_workspace_bytes",
+           "zq_reduce_partials")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -137,6 +139,21 @@ class zq_linear_desc(ctypes.Structure):
 
 _lib.zq_linear_stack_workspace_bytes.argtypes = [_P, _I]
 _lib.zq_linear_stack_workspace_bytes.restype = _S
+
+
+class zq_partial_desc(ctypes.Structure):
+    _fields_ = [("x", _P), ("packed", _P), ("scales", _P), ("zeros", _P), ("out", _P),
+                ("bits", _I), ("group", _I), ("M", _I), ("N", _I), ("K", _I)]
+
+
+_lib.zq_linear_partial.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
+_lib.zq_linear_partial.restype = _I
+_lib.zq_linear_partial_stack.argtypes = [_P, _I, _P]
+_lib.zq_linear_partial_stack.restype = _I
+_lib.zq_linear_partial_stack_workspace_bytes.argtypes = [_P, _I]
+_lib.zq_linear_partial_stack_workspace_bytes.restype = _S
+_lib.zq_reduce_partials.argtypes = [ctypes.POINTER(_P), _I, _S, _P, _P]
+_lib.zq_reduce_partials.restype = _I
 
 
 def _check(status):
@@ -263,6 +280,43 @@ def zq_linear_stack(ops, n_ops=None, stream=None):
     _check(_lib.zq_linear_stack(ops, n_ops, _stream(stream)))
 
 
+def zq_linear_partial(x, packed, scales, zeros, bits, group, M, N, K, out, stream=None):
+    _check(_lib.zq_linear_partial(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), bits, group,
+                                  M, N, K, _ptr(out), _stream(stream, x)))
+
+
+def make_partial_descs(ops):
+    """ops: iterable of tuples (x, packed, scales, zeros, out_fp32, bits, group, M, N, K)."""
+    ops = list(ops)
+    arr = (zq_partial_desc * max(len(ops), 1))()
+    for i, (x, packed, scales, zeros, out, bits, group, M, N, K) in enumerate(ops):
+        arr[i] = zq_partial_desc(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), _ptr(out),
+                                 bits, group, M, N, K)
+    return arr, len(ops)
+
+
+def zq_linear_partial_stack(ops, n_ops=None, stream=None):
+    """ops: a ctypes array from make_partial_descs(), or an iterable accepted by it."""
+    if not isinstance(ops, ctypes.Array):
+        ops, n = make_partial_descs(ops)
+        n_ops = n if n_ops is None else n_ops
+    _check(_lib.zq_linear_partial_stack(ops, n_ops, _stream(stream)))
+
+
+def zq_linear_partial_stack_workspace_bytes(ops, n_ops=None):
+    if not isinstance(ops, ctypes.Array):
+        ops, n = make_partial_descs(ops)
+        n_ops = n if n_ops is None else n_ops
+    return _lib.zq_linear_partial_stack_workspace_bytes(ops, n_ops)
+
+
+def zq_reduce_partials(parts, count, out, stream=None):
+    """parts: sequence of fp32 device buffers (tensors or addresses), summed in order."""
+    arr = (_P * len(parts))(*[_ptr(p) for p in parts])
+    _check(_lib.zq_reduce_partials(arr, len(parts), count, _ptr(out),
+                                   _stream(stream, out if isinstance(out, torch.Tensor) else None)))
+
+
 def zq_unpack(packed, N, K, bits, codes, stream=None):
     _check(_lib.zq_unpack(_ptr(packed), N, K, bits, _ptr(codes), _stream(stream, packed)))
 
@@ -313,6 +367,19 @@ def linear_stack(ops, stream=None):
     arr, n = ops if isinstance(ops, tuple) and isinstance(ops[0], ctypes.Array) else make_descs(ops)
     ensure_workspace(zq_linear_stack_workspace_bytes(arr, n), stream)
     zq_linear_stack(arr, n, stream)
+
+
+def linear_partial(x, packed, scales, zeros, bits, N, out=None, stream=None):
+    """fp16 CUDA x (M x K) -> fp32 partial sums (M x N) via zq_linear_partial."""
+    M, K = x.shape
+    _need(x, M * K * 2, torch.float16, "x", x.device)
+    if out is None:
+        out = torch.empty(M, N, dtype=torch.float32, device=x.device)
+    _need(out, M * N * 4, torch.float32, "out", x.device)
+    ensure_workspace(zq_linear_workspace_bytes(bits, M, N, K), stream if stream is not None else
+                     torch.cuda.current_stream(x.device))
+    zq_linear_partial(x, packed, scales, zeros, bits, GROUP, M, N, K, out, stream)
+    return out
 
 
 def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):

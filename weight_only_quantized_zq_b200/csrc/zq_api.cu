@@ -20,6 +20,7 @@
 
 #include "zq.h"
 #include "zq_kv.h"
+#include "zq_tp.h"
 #include "zq_internal.h"
 #include "zq_prefill.h"
 #include "zq_quant.h"
@@ -78,6 +79,26 @@ zq_status check_linear(const zq_linear_desc &d) {
     if ((st = check_ptr(d.zeros, "zeros")) != ZQ_OK) return st;
     if ((st = check_ptr(d.out, "out")) != ZQ_OK) return st;
     return ZQ_OK;
+}
+
+// One linear operation inside the library: the arguments of a zq_linear call,
+// with the output either fp16 (out) or, for partial sums, fp32 (out32; then
+// out is null).
+struct Op : zq_linear_desc {
+    float *out32 = nullptr;
+};
+
+Op make_op(const zq_linear_desc &d) {
+    Op o;
+    static_cast<zq_linear_desc &>(o) = d;
+    return o;
+}
+
+// Validation of an op with an fp32 output.
+zq_status check_partial(const zq_linear_desc &d, const float *out32) {
+    zq_linear_desc t = d;
+    t.out = reinterpret_cast<uint16_t *>(const_cast<float *>(out32));
+    return check_linear(t);
 }
 
 // ---------------------------------------------------------------- device --
@@ -201,7 +222,7 @@ size_t align16(size_t b) { return (b + 15) & ~size_t(15); }
 
 // Plans and launches one decode launch over ops that share bits and MT and are
 // mutually independent.  With `dry_bytes` set, only computes the workspace size.
-zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, cudaStream_t stream,
+zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t stream,
                      size_t *dry_bytes = nullptr, uint8_t *fixed_ws = nullptr, size_t fixed_ws_bytes = 0) {
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
@@ -246,8 +267,8 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
     const int codes_bytes = decode_codes_bytes(bits, mt);
     const int off_sz = 0;
     const int off_sx = off_sz + rows * 4 * gps;
-    const int off_x = off_sx + gps * mpad * 16;
-    const int x_rows_max = mt == 1 ? max_m : mpad;  // staged token rows
+    const int x_rows_max = mt == 1 ? max_m : mpad;  // staged token rows (and group records)
+    const int off_x = off_sx + gps * x_rows_max * 16;
     const int off_desc = off_x + gps * x_rows_max * 256;
     const int meta_bytes = static_cast<int>(align16(off_desc + 32));
     const int stage = codes_bytes + meta_bytes;
@@ -308,7 +329,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         prep_off[e] = off;
         const size_t G = keys[e].K / kGroup;
         const size_t xr = mt == 1 ? keys[e].M : mpad;
-        off += align256(G * xr * kGroup * 2) + align256(G * mpad * 16);
+        off += align256(G * xr * kGroup * 2) + align256(G * xr * 16);
     }
     const size_t part_off = off;
     if (!units) off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
@@ -338,11 +359,10 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         en.x_rows = mt == 1 ? keys[e].M : mpad;
         en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(G * en.x_rows * kGroup * 2));
         en.M = keys[e].M;
-        en.M_pad = mpad;
         en.K = keys[e].K;
         en.bits = bits;
         pp.warp_prefix[e] = wsum;
-        wsum += static_cast<long long>(mpad) * G;
+        wsum += static_cast<long long>(en.x_rows) * G;
     }
     pp.warp_prefix[keys.size()] = wsum;
 
@@ -376,6 +396,7 @@ zq_status run_decode(const std::vector<zq_linear_desc> &ops, int bits, int mt, c
         o.xg = en.xg;
         o.sx = en.sx;
         o.out = ops[i].out;
+        o.out32 = ops[i].out32;
         o.M = ops[i].M;
         o.N = ops[i].N;
         o.K = ops[i].K;
@@ -414,7 +435,7 @@ struct OpRanges {
     Range x, packed, scales, zeros, out;
 };
 
-OpRanges ranges_of(const zq_linear_desc &d) {
+OpRanges ranges_of(const Op &d) {
     const size_t G = d.K / kGroup;
     auto r = [](const void *p, size_t n) {
         const uintptr_t a = reinterpret_cast<uintptr_t>(p);
@@ -423,7 +444,8 @@ OpRanges ranges_of(const zq_linear_desc &d) {
     return OpRanges{r(d.x, static_cast<size_t>(d.M) * d.K * 2),
                     r(d.packed, static_cast<size_t>(d.N) * d.K * d.bits / 8),
                     r(d.scales, static_cast<size_t>(d.N) * G * 2), r(d.zeros, static_cast<size_t>(d.N) * G * 2),
-                    r(d.out, static_cast<size_t>(d.M) * d.N * 2)};
+                    d.out32 ? r(d.out32, static_cast<size_t>(d.M) * d.N * 4)
+                            : r(d.out, static_cast<size_t>(d.M) * d.N * 2)};
 }
 
 // b depends on a (a earlier) if they share memory with at least one write.
@@ -440,12 +462,11 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
 // One persistent launch over all tiles of independent prefill ops of one bit
 // width (at most kMaxPrefillOps), ops with the longest K first so that the
 // last tiles handed out are the cheap ones.
-zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
+zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
-    std::stable_sort(ops.begin(), ops.end(),
-                     [](const zq_linear_desc &a, const zq_linear_desc &b) { return a.K > b.K; });
+    std::stable_sort(ops.begin(), ops.end(), [](const Op &a, const Op &b) { return a.K > b.K; });
     PrefillGroup pg;
     std::memset(&pg, 0, sizeof(pg));
     pg.n_ops = static_cast<int>(ops.size());
@@ -460,6 +481,7 @@ zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
         o.scales = ops[i].scales;
         o.zeros = ops[i].zeros;
         o.out = ops[i].out;
+        o.out32 = ops[i].out32;
         o.M = ops[i].M;
         o.N = ops[i].N;
         o.K = ops[i].K;
@@ -479,16 +501,16 @@ zq_status run_prefill(std::vector<zq_linear_desc> ops, cudaStream_t stream) {
 // class, each holding at most kMaxDecodeOps ops and kMaxPrepEntries inputs.
 // With `dry` set nothing is launched: *dry becomes the largest workspace any
 // of the launches needs (at least the counters).
-zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t stream, size_t *dry = nullptr) {
-    std::vector<zq_linear_desc> pieces;
+zq_status run_batch(const std::vector<Op> &batch, cudaStream_t stream, size_t *dry = nullptr) {
+    std::vector<Op> pieces;
     const int bits_list[4] = {2, 3, 4, 8};
     if (dry) *dry = std::max(*dry, kCounterBytes);
     for (int bits : bits_list) {
-        std::vector<zq_linear_desc> pre;
+        std::vector<Op> pre;
         for (const auto &d : batch)
             if (d.M > kDecodeMaxM && d.bits == bits) pre.push_back(d);
         for (size_t i = 0; i < pre.size() && !dry; i += kMaxPrefillOps) {
-            std::vector<zq_linear_desc> launch(pre.begin() + i,
+            std::vector<Op> launch(pre.begin() + i,
                                                pre.begin() + std::min(pre.size(), i + kMaxPrefillOps));
             zq_status st = run_prefill(launch, stream);
             if (st != ZQ_OK) return st;
@@ -499,12 +521,12 @@ zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t strea
     const int mt_list[2] = {1, 2};
     for (int bits : bits_list)
         for (int mt : mt_list) {
-            std::vector<zq_linear_desc> cls;
+            std::vector<Op> cls;
             for (const auto &d : pieces)
                 if (d.bits == bits && mt_for_m(d.M) == mt) cls.push_back(d);
             size_t i = 0;
             while (i < cls.size()) {
-                std::vector<zq_linear_desc> launch;
+                std::vector<Op> launch;
                 std::vector<std::pair<const uint16_t *, int>> inputs;
                 while (i < cls.size() && launch.size() < static_cast<size_t>(kMaxDecodeOps)) {
                     std::pair<const uint16_t *, int> key{cls[i].x, cls[i].M * 1000003 + cls[i].K};
@@ -525,8 +547,8 @@ zq_status run_batch(const std::vector<zq_linear_desc> &batch, cudaStream_t strea
 // Splits a stack into batches of mutually independent ops (an op that shares
 // written memory with an earlier op of the batch starts the next batch) and
 // runs them in order; with `dry` set, only sizes the workspace.
-zq_status run_stack(const zq_linear_desc *ops, int n_ops, cudaStream_t s, size_t *dry) {
-    std::vector<zq_linear_desc> batch;
+zq_status run_stack(const Op *ops, int n_ops, cudaStream_t s, size_t *dry) {
+    std::vector<Op> batch;
     std::vector<OpRanges> br;
     constexpr size_t kMaxBatch = 1024;
     for (int i = 0; i < n_ops; ++i) {
@@ -549,7 +571,7 @@ zq_status run_stack(const zq_linear_desc *ops, int n_ops, cudaStream_t s, size_t
 // Checks that the stream's workspace covers the stack (nothing is enqueued
 // when it does not, apart from clearing counters a failed kernel left set),
 // then runs it.
-zq_status checked_stack(const zq_linear_desc *ops, int n_ops, cudaStream_t s) {
+zq_status checked_stack(const Op *ops, int n_ops, cudaStream_t s) {
     if (n_ops == 0) return ZQ_OK;
     size_t need = kCounterBytes;
     zq_status st = run_stack(ops, n_ops, s, &need);
@@ -682,7 +704,19 @@ zq_status zq_linear(const uint16_t *x, const uint32_t *packed, const uint16_t *s
     zq_linear_desc d{x, packed, scales, zeros, out, bits, group, M, N, K};
     zq_status st = check_linear(d);
     if (st != ZQ_OK) return st;
-    return checked_stack(&d, 1, reinterpret_cast<cudaStream_t>(stream));
+    const Op op = make_op(d);
+    return checked_stack(&op, 1, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zq_status zq_linear_partial(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                            const uint16_t *zeros, int bits, int group, int M, int N, int K, float *out,
+                            zq_stream_t stream) {
+    zq_linear_desc d{x, packed, scales, zeros, nullptr, bits, group, M, N, K};
+    zq_status st = check_partial(d, out);
+    if (st != ZQ_OK) return st;
+    Op op = make_op(d);
+    op.out32 = out;
+    return checked_stack(&op, 1, reinterpret_cast<cudaStream_t>(stream));
 }
 
 zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
@@ -695,7 +729,7 @@ zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uin
         return fail(ZQ_ERR_UNSUPPORTED, "zq_linear_noalloc supports M <= %d (got M=%d)", kNoallocMaxM, M);
     uint8_t *ws = nullptr;
     if ((st = noalloc_scratch(&ws)) != ZQ_OK) return st;
-    std::vector<zq_linear_desc> one{d};
+    std::vector<Op> one{make_op(d)};
     size_t need = 0;
     if ((st = run_decode(one, bits, mt_for_m(M), nullptr, &need)) != ZQ_OK) return st;
     if (need > kNoallocScratchBytes)
@@ -709,26 +743,78 @@ zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uin
     return run_decode(one, bits, mt_for_m(M), s, nullptr, ws, kNoallocScratchBytes);
 }
 
-zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream) {
-    if (n_ops < 0 || (n_ops > 0 && ops == nullptr))
+// Validates the public descriptors of a stack (fp16 outputs, or fp32 partial
+// sums when `partial`) into internal ops; reports the first bad op.
+zq_status stack_ops(const zq_linear_desc *ops, const zq_partial_desc *pops, int n_ops, std::vector<Op> *out) {
+    if (n_ops < 0 || (n_ops > 0 && ops == nullptr && pops == nullptr))
         return fail(ZQ_ERR_INVALID_ARG, "ops is null or n_ops < 0");
+    out->clear();
+    out->reserve(n_ops);
     for (int i = 0; i < n_ops; ++i) {
-        zq_status st = check_linear(ops[i]);
+        Op op;
+        zq_status st;
+        if (ops) {
+            op = make_op(ops[i]);
+            st = check_linear(ops[i]);
+        } else {
+            const zq_partial_desc &p = pops[i];
+            op = make_op(zq_linear_desc{p.x, p.packed, p.scales, p.zeros, nullptr, p.bits, p.group, p.M, p.N, p.K});
+            op.out32 = p.out;
+            st = check_partial(op, p.out);
+        }
         if (st != ZQ_OK) {
             std::string msg = g_last_error;
             return fail(st, "op %d: %s", i, msg.c_str());
         }
+        out->push_back(op);
     }
-    return checked_stack(ops, n_ops, reinterpret_cast<cudaStream_t>(stream));
+    return ZQ_OK;
+}
+
+zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream) {
+    std::vector<Op> v;
+    zq_status st = stack_ops(ops, nullptr, n_ops, &v);
+    if (st != ZQ_OK) return st;
+    return checked_stack(v.data(), n_ops, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zq_status zq_linear_partial_stack(const zq_partial_desc *ops, int n_ops, zq_stream_t stream) {
+    std::vector<Op> v;
+    zq_status st = stack_ops(nullptr, ops, n_ops, &v);
+    if (st != ZQ_OK) return st;
+    return checked_stack(v.data(), n_ops, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t zq_linear_stack_workspace_bytes(const zq_linear_desc *ops, int n_ops) {
-    if (n_ops < 0 || (n_ops > 0 && ops == nullptr)) return 0;
-    for (int i = 0; i < n_ops; ++i)
-        if (check_linear(ops[i]) != ZQ_OK) return 0;
+    std::vector<Op> v;
+    if (stack_ops(ops, nullptr, n_ops, &v) != ZQ_OK) return 0;
     size_t need = 0;
-    if (run_stack(ops, n_ops, nullptr, &need) != ZQ_OK) return 0;
+    if (run_stack(v.data(), n_ops, nullptr, &need) != ZQ_OK) return 0;
     return need;
+}
+
+size_t zq_linear_partial_stack_workspace_bytes(const zq_partial_desc *ops, int n_ops) {
+    std::vector<Op> v;
+    if (stack_ops(nullptr, ops, n_ops, &v) != ZQ_OK) return 0;
+    size_t need = 0;
+    if (run_stack(v.data(), n_ops, nullptr, &need) != ZQ_OK) return 0;
+    return need;
+}
+
+zq_status zq_reduce_partials(const float *const *parts, int n_parts, size_t count, uint16_t *out,
+                             zq_stream_t stream) {
+    if (n_parts < 1 || n_parts > kMaxReduceParts)
+        return fail(ZQ_ERR_INVALID_ARG, "n_parts=%d must be in [1, %d]", n_parts, kMaxReduceParts);
+    if (parts == nullptr) return fail(ZQ_ERR_INVALID_ARG, "parts is null");
+    if (count == 0) return ZQ_OK;
+    zq_status st;
+    for (int i = 0; i < n_parts; ++i)
+        if ((st = check_ptr(parts[i], "parts[i]")) != ZQ_OK) return st;
+    if ((st = check_ptr(out, "out")) != ZQ_OK) return st;
+    cudaError_t e = launch_reduce_partials(parts, n_parts, count, out, reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
+    ++g_launches;
+    return ZQ_OK;
 }
 
 zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes, zq_stream_t stream) {
@@ -842,9 +928,11 @@ size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
     if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
     // the plan needs only the sizes: any aligned, distinct fake pointers do
     const auto fake = [](uintptr_t i) { return reinterpret_cast<void *>(i << 20); };
-    zq_linear_desc d{static_cast<const uint16_t *>(fake(1)), static_cast<const uint32_t *>(fake(2)),
-                     static_cast<const uint16_t *>(fake(3)), static_cast<const uint16_t *>(fake(4)),
-                     static_cast<uint16_t *>(fake(1 << 20)), bits, kGroup, M, N, K};
+    const Op d = make_op(zq_linear_desc{static_cast<const uint16_t *>(fake(1)),
+                                        static_cast<const uint32_t *>(fake(2)),
+                                        static_cast<const uint16_t *>(fake(3)),
+                                        static_cast<const uint16_t *>(fake(4)),
+                                        static_cast<uint16_t *>(fake(1 << 20)), bits, kGroup, M, N, K});
     size_t need = 0;
     if (run_stack(&d, 1, nullptr, &need) != ZQ_OK) return 0;
     return need;

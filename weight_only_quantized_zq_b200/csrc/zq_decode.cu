@@ -117,11 +117,10 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
         const long long local = gw - p.warp_prefix[e];
         const int G = en.K / kGroup;
         const int t = static_cast<int>(local / G), g = static_cast<int>(local % G);
-        float4 *dst = reinterpret_cast<float4 *>(en.sx) + static_cast<size_t>(g) * en.M_pad + t;
+        float4 *dst = reinterpret_cast<float4 *>(en.sx) + static_cast<size_t>(g) * en.x_rows + t;
         if (t >= en.M) {
             if (lane == 0) *dst = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (t < en.x_rows)
-                reinterpret_cast<uint2 *>(en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup)[lane] =
+            reinterpret_cast<uint2 *>(en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup)[lane] =
                     make_uint2(0u, 0u);
         } else {
             const uint16_t *xrow = en.x + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
@@ -294,6 +293,7 @@ struct ProdState {
     int chunk, begin, end;    // its chunk and that chunk's steps
     unsigned int ticket;      // counter value for the chunk after this one
     int done;                 // the end marker has been staged
+    int slot, round;          // ring slot and round of the next stage: seq = round * depth + slot
     int seq;                  // stages filled so far
 };
 
@@ -331,8 +331,16 @@ __device__ __forceinline__ int box_row(int g) {
     else return 2 * (g & 3) + (g >> 2);                                // b = 2 (half-warp phases)
 }
 
+// CTAs per SM the register budget is sized for: the shared memory of the
+// host's ring (at least 3 stages) leaves room for 4 CTAs of one token tile,
+// except at b = 4, whose 18.5 KB stages fit 3.
 template <int BITS, int MT>
-__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
+__host__ __device__ constexpr int decode_min_ctas() {
+    return MT == 1 && BITS != 4 ? 4 : 3;
+}
+
+template <int BITS, int MT>
+__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS, MT>())
     decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int GPS = decode_gps(BITS, MT);
     constexpr int SEG = decode_seg(BITS, MT);       // bytes of one row per step
@@ -390,6 +398,8 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
         ps->end = e;
         ps->ticket = p.dynamic ? atomicAdd(p.cnt, 1u) : 0u;  // fetched one chunk ahead of its use
         ps->done = 0;
+        ps->slot = 0;
+        ps->round = 0;
         ps->seq = 0;
     }
     __syncthreads();
@@ -406,12 +416,18 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
         ld.valid = ps->valid != 0;
         int ld_chunk = ps->chunk, ld_begin = ps->begin, ld_end = ps->end;
         unsigned int ticket = ps->ticket;
+        // slot and round of stage `target` (no division by the runtime depth)
+        const int slot_ld = ps->slot, round_ld = ps->round;
+        const bool wrap = slot_ld + 1 == D;
         if (ps->done) {
             __syncwarp();
-            if (lane == 0) st_release_shared(&ps->seq, target + 1);
+            if (lane == 0) {
+                ps->slot = wrap ? 0 : slot_ld + 1;
+                ps->round = round_ld + (wrap ? 1 : 0);
+                st_release_shared(&ps->seq, target + 1);
+            }
             return true;
         }
-        const int slot_ld = target % D, round_ld = target / D;
         if (round_ld > 0 && !wait_phase(&empty[slot_ld], (round_ld - 1) & 1, p.wait_ns)) return false;
         if (!ld.valid && p.dynamic) {
             // Chunks only grow, so a CTA stops at its first ticket past the end
@@ -462,12 +478,12 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                 dsc[0] = make_int4(ld.o, ld.rb, ld.j, ng | (flags << 8));
                 dsc[1] = make_int4(ld_chunk, unit_start, op.M, 0);
                 const uint32_t xbytes = static_cast<uint32_t>(ng * xrows * 256);
-                const uint32_t sbytes = static_cast<uint32_t>(ng * MPAD * 16);
+                const uint32_t sbytes = static_cast<uint32_t>(ng * xrows * 16);
                 mbar_arrive_expect_tx(&full[slot_ld], NBOX * BOXB + xbytes + sbytes);
 #pragma unroll
                 for (int b = 0; b < NBOX; ++b)
                     tma_load_2d(st + b * BOXB, &op.tmap, g0 * GB + b * BOXW, ld.rb * kDecodeCtaRows, &full[slot_ld]);
-                bulk_load(sm + p.off_sx, op.sx + static_cast<size_t>(g0) * MPAD * 4, sbytes, &full[slot_ld]);
+                bulk_load(sm + p.off_sx, op.sx + static_cast<size_t>(g0) * xrows * 4, sbytes, &full[slot_ld]);
             }
             __syncwarp();
             // Activations: token t's ng groups (ng * 256 contiguous bytes), one
@@ -497,6 +513,8 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
             ps->end = ld_end;
             ps->ticket = ticket;
             ps->done = done;
+            ps->slot = wrap ? 0 : slot_ld + 1;
+            ps->round = round_ld + (wrap ? 1 : 0);
             st_release_shared(&ps->seq, target + 1);
         }
         return true;
@@ -514,7 +532,10 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
     //   x':    token gq's staged row is GPS*256 bytes, group gi at +gi*256,
     //          the lane's chunk q of it at x_chunk(c, q, gq).
     //   sums:  (sum x, -f * bias, f, 0) of token 8mt + 2c of group gi at
-    //          off_sx + (gi*MPAD + 8mt + 2c) * 16, token 8mt + 2c + 1 16 bytes on.
+    //          off_sx + (gi*R + 8mt + 2c) * 16, token 8mt + 2c + 1 16 bytes on,
+    //          R = the staged token rows (M with one token tile, else MPAD);
+    //          lanes of tokens >= M read other bytes of the stage (their
+    //          columns are padding).
     int lanex;
     if constexpr (BITS == 4) lanex = c ^ gr;
     else if constexpr (BITS == 2) lanex = (c >> 1) ^ gr;
@@ -591,6 +612,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
         }
         const int ng = d0.w & 0xFF;
         const int M = static_cast<int>(d1.z);
+        const int R = MT == 1 ? M : MPAD;  // staged group records per group (one per staged token)
         const int o = static_cast<int>(d0.x), rb = static_cast<int>(d0.y);
 
         // Scales and zeros of rows gr and gr + 8 for the GPS groups.
@@ -675,11 +697,10 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                         xf[4 * q + 3] = v.w;
                     }
                 }
-                const uint32_t sa_a = smb + sxo + (gi * MPAD + 8 * mt) * 16;
-                const uint2 sa = lds_v2(sa_a);
+                const uint4 sa = lds_v4(smb + sxo + (gi * R + 8 * mt) * 16);
                 float acc[4];
                 mma_group<BITS, MT == 1>(acc, wv, xf, magic);
-                const float fa = __uint_as_float(lds_u32(sa_a + 8));
+                const float fa = __uint_as_float(sa.z);
                 // tot += s * f * (acc - bias) + z * sum(x), with f * (acc - bias)
                 // as one FMA (f is the token's power-of-two x' scale); with one
                 // token the odd C columns are padding.
@@ -688,7 +709,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                     tot[mt][2 * h] = fmaf(sc[h], fmaf(acc[2 * h], fa, __uint_as_float(sa.y)),
                                           fmaf(zr[h], __uint_as_float(sa.x), tot[mt][2 * h]));
                 if constexpr (!one_token) {
-                    const uint4 sb = lds_v4(smb + sxo + (gi * MPAD + 8 * mt) * 16 + 16);
+                    const uint4 sb = lds_v4(smb + sxo + (gi * R + 8 * mt) * 16 + 16);
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tot[mt][2 * h + 1] =
@@ -737,9 +758,11 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                     for (int i = 0; i < 4; ++i) {
                         const int row = r0 + warp * 16 + (i >> 1) * 8 + gr;
                         const int tok = 8 * mt + 2 * c + (i & 1);
-                        if (row < op.N && tok < M)
-                            op.out[static_cast<size_t>(tok) * op.N + row] =
-                                __half_as_ushort(__float2half_rn(tot[mt][i]));
+                        if (row < op.N && tok < M) {
+                            const size_t at = static_cast<size_t>(tok) * op.N + row;
+                            if (op.out32) op.out32[at] = tot[mt][i];
+                            else op.out[at] = __half_as_ushort(__float2half_rn(tot[mt][i]));
+                        }
                     }
             } else {
                 // Partial piece: slot (k, 0) holds chunk k's head piece, (k, 1) its tail piece.
@@ -768,8 +791,11 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, MT == 1 ? 4 : 3)
                         for (int ww = w_first + 1; ww <= w_last; ++ww)
                             sum += __ldcg(p.part + static_cast<size_t>(ww) * 2 * p.slot_floats + idx);
                         const int row = idx / M, tok = idx - row * M;
-                        if (r0 + row < op.N)
-                            op.out[static_cast<size_t>(tok) * op.N + r0 + row] = __half_as_ushort(__float2half_rn(sum));
+                        if (r0 + row < op.N) {
+                            const size_t at = static_cast<size_t>(tok) * op.N + r0 + row;
+                            if (op.out32) op.out32[at] = sum;
+                            else op.out[at] = __half_as_ushort(__float2half_rn(sum));
+                        }
                     }
                     if (lane == 0) p.cnt[1 + w_first] = 0u;  // ready for the next call
                 }

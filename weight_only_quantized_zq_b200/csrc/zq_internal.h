@@ -36,9 +36,11 @@ struct alignas(64) DecodeOp {
     const uint16_t *zeros;
     const uint16_t *xg;     // workspace: (M, or M_pad with several token tiles) x K fp16, pair-permuted,
                             // 2^(E-s)-scaled, chunk-swizzled activations
-    const float *sx;        // workspace: G x M_pad x 4 fp32 (sum x, -f * 1024 * sum x', f, 0) per group and
-                            // token; f = 2^-E undoes the token's power-of-two x' scale
-    uint16_t *out;          // M x N fp16
+    const float *sx;        // workspace: G x R x 4 fp32 (sum x, -f * 1024 * sum x', f, 0) per group and
+                            // token, R = M (one token tile) or M_pad; f = 2^-E undoes the power-of-two
+                            // x' scale
+    uint16_t *out;          // M x N fp16, or null when out32 is set
+    float *out32;           // M x N fp32 (partial sums, not rounded), or null
     int step0;              // first CTA step of this op
     int unit0;              // first row block of this op (counted over the launch)
     int M, N, K, G;
@@ -69,8 +71,8 @@ static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
     uint16_t *xg;       // x_rows x K, chunk-swizzled per group and token; rows >= M are zeros
-    float *sx;          // G x M_pad x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0)
-    int M, M_pad, x_rows, K, bits;
+    float *sx;          // G x x_rows x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
+    int M, x_rows, K, bits;  // x_rows: M with one token tile, else the padded M_pad
 };
 
 struct PrepParams {
@@ -122,7 +124,8 @@ struct alignas(64) PrefillOp {
     const uint32_t *packed;
     const uint16_t *scales;
     const uint16_t *zeros;
-    uint16_t *out;
+    uint16_t *out;   // M x N fp16, or null when out32 is set
+    float *out32;    // M x N fp32 (partial sums, not rounded), or null
     int M, N, K;
     int tok_tiles;  // ceil(M / 256)
     int tile0;      // first tile of this op in the launch
@@ -152,6 +155,11 @@ cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, con
 // tcgen05 tile kernel (which, with one token tile, also streams the weights
 // once, and from 17 tokens on is the faster of the two).
 constexpr int kDecodeMaxM = 16;
+
+// Partial-sum reduction: out[i] = fp16(sum of parts[p][i], p in order).
+constexpr int kMaxReduceParts = 16;
+cudaError_t launch_reduce_partials(const float *const *parts, int n_parts, size_t count, uint16_t *out,
+                                   cudaStream_t stream);
 
 cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream);

@@ -667,7 +667,20 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                     uint32_t r[32];
                     tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile + cc * 32, r);
                     const int col0 = n0 + cc * 32;
-                    if (tok < op.M && col0 < op.N) {
+                    if (tok < op.M && col0 < op.N && op.out32) {
+                        // fp32 partial sums (a K-split shard), not rounded
+                        float *dst = op.out32 + static_cast<size_t>(tok) * op.N + col0;
+                        if ((op.N % 4) == 0 && col0 + 32 <= op.N) {
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                reinterpret_cast<uint4 *>(dst)[q] =
+                                    make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < 32; ++q)
+                                if (col0 + q < op.N) dst[q] = __uint_as_float(r[q]);
+                        }
+                    } else if (tok < op.M && col0 < op.N) {
                         uint16_t *dst = op.out + static_cast<size_t>(tok) * op.N + col0;
                         if (vec && col0 + 32 <= op.N) {
 #pragma unroll
