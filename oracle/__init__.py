@@ -58,6 +58,12 @@ def _load():
         lib.zo_dequant.restype = I
         lib.zo_linear_rows.argtypes = [P, I, I, P, P, P, I, I, I, P, I, P, P]
         lib.zo_linear_rows.restype = I
+        lib.zo_linear_rows_ex.argtypes = [P, I, I, I, P, P, P, I, I, I, P, I, P, P]
+        lib.zo_linear_rows_ex.restype = I
+        lib.zo_bf16_to_f64.argtypes = [ctypes.c_uint16]
+        lib.zo_bf16_to_f64.restype = ctypes.c_double
+        lib.zo_f64_to_bf16.argtypes = [ctypes.c_double]
+        lib.zo_f64_to_bf16.restype = ctypes.c_uint16
         lib.zo_set_threads.argtypes = [I]
         lib.zo_set_threads.restype = None
         lib.zo_get_threads.argtypes = []
@@ -91,6 +97,14 @@ def f16_to_f64(h):
 
 def f64_to_f16(v):
     return _load().zo_f64_to_f16(float(v))
+
+
+def bf16_to_f64(b):
+    return _load().zo_bf16_to_f64(int(b))
+
+
+def f64_to_bf16(v):
+    return _load().zo_f64_to_bf16(float(v))
 
 
 def quantize_group(w, bits):
@@ -186,14 +200,21 @@ def dequant(packed, scales, zeros, bits, N, K, group=GROUP):
     return w_hat
 
 
-def linear(x16, packed, scales, zeros, bits, N, K, rows=None, group=GROUP):
-    """x16: M x K uint16 (fp16 bits). Returns (y, bound), each M x len(rows)
-    (or M x N when rows is None), fp64."""
+def linear(x16, packed, scales, zeros, bits, N, K, rows=None, group=GROUP, xfmt="f16"):
+    """x16: M x K uint16 (fp16 bits, or bf16 bits with xfmt="bf16"). Returns
+    (y, bound), each M x len(rows) (or M x N when rows is None), fp64.
+    bits=16: `packed` is the N x K fp16 weights (uint16 bits) and scales/zeros
+    are not used (pass None)."""
     x16 = _c(x16, np.uint16)
     M = x16.shape[0]
-    packed = _c(packed, np.uint32)
-    scales = _c(scales, np.uint16)
-    zeros = _c(zeros, np.uint16)
+    if bits == 16:
+        packed = _c(packed, np.uint16)
+        scales = np.zeros(1, np.uint16) if scales is None else _c(scales, np.uint16)
+        zeros = np.zeros(1, np.uint16) if zeros is None else _c(zeros, np.uint16)
+    else:
+        packed = _c(packed, np.uint32)
+        scales = _c(scales, np.uint16)
+        zeros = _c(zeros, np.uint16)
     if rows is None:
         nrows = N
         rows_p = None
@@ -203,9 +224,9 @@ def linear(x16, packed, scales, zeros, bits, N, K, rows=None, group=GROUP):
         rows_p = _ptr(rows)
     y = np.zeros((M, nrows), np.float64)
     bound = np.zeros((M, nrows), np.float64)
-    st = _load().zo_linear_rows(_ptr(x16), M, K, _ptr(packed), _ptr(scales),
-                                _ptr(zeros), bits, group, N, rows_p, nrows,
-                                _ptr(y), _ptr(bound))
+    st = _load().zo_linear_rows_ex(_ptr(x16), {"f16": 0, "bf16": 1}[xfmt], M, K, _ptr(packed),
+                                   _ptr(scales), _ptr(zeros), bits, group, N, rows_p, nrows,
+                                   _ptr(y), _ptr(bound))
     if st != OK:
         raise OracleError(st)
     return y, bound

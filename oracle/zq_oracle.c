@@ -30,6 +30,12 @@
  *     zero point), computed exactly in fp64.
  *   - linear: y[m][n] = sum_k x[m][k]*w_hat[n][k] in fp64 (W is N x K, the
  *     PyTorch Linear convention y = x W^T); bound = sum_k |x||w_hat|.
+ *   - group sizes: 128 (the pages' figure) and also 32 and 64 (the encoding
+ *     variants: the same quantizer on shorter groups, scale/zero per group).
+ *   - fp16 passthrough (the .zse format keeps some tensors unquantized):
+ *     bits = 16 means the weights are fp16 values used as they are.
+ *   - bf16 activations: x given as bfloat16 (the top 16 bits of a binary32),
+ *     decoded exactly.
  *   - symmetric quantization (listed by [wiki] for INT8 without a formula):
  *     Q = 2^(b-1) - 1, scale = fp16(max|w| / Q), q = clamp(round(w/scale),
  *     -Q, Q); stored as code = q + 2^(b-1), zero = -2^(b-1)*scale (exact), so
@@ -50,6 +56,53 @@
 #define ZO_INVALID 1
 #define ZO_UNSUPPORTED 2
 #define ZO_NONFINITE 3
+
+/* bfloat16, written from its definition: the upper half of an IEEE binary32 */
+/*   1 sign bit, 8 exponent bits (bias 127), 7 fraction bits;               */
+/*   e in 1..254: 2^(e-127) * (1 + f/128); e == 0: 2^-126 * f/128;          */
+/*   e == 255: infinity (f == 0) or NaN.                                    */
+double zo_bf16_to_f64(uint16_t b)
+{
+    int sign = (b >> 15) & 1;
+    int e = (b >> 7) & 0xFF;
+    int f = b & 0x7F;
+    double v;
+    if (e == 0)
+        v = ldexp((double)f, -133);              /* f * 2^-126 / 128 */
+    else if (e == 255)
+        v = f ? NAN : INFINITY;
+    else
+        v = ldexp((double)(128 + f), e - 134);   /* (128+f) * 2^(e-127-7) */
+    return sign ? -v : v;
+}
+
+/* Round-to-nearest, ties-to-even conversion of an fp64 value to bfloat16
+ * (the largest finite value is (2 - 2^-7) * 2^127; the midpoint above it
+ * overflows to infinity). */
+uint16_t zo_f64_to_bf16(double v)
+{
+    if (isnan(v))
+        return 0x7FC0;
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs(v);
+    if (a >= ldexp(255.5, 120))                  /* (2 - 2^-8) * 2^127 */
+        return sign | 0x7F80;
+    if (a < ldexp(1.0, -126)) {
+        double m = rint(ldexp(a, 133));          /* multiples of 2^-133: 0 .. 128 */
+        return sign | (uint16_t)m;               /* m == 128 encodes 2^-126 */
+    }
+    int ex;
+    (void)frexp(a, &ex);
+    int E = ex - 1;                              /* 2^E <= a < 2^(E+1) */
+    double m = rint(ldexp(a, 7 - E));            /* 128 .. 256 */
+    if (m == 256.0) {
+        m = 128.0;
+        E += 1;
+    }
+    if (E > 127)
+        return sign | 0x7F80;
+    return sign | (uint16_t)((E + 127) << 7) | (uint16_t)(m - 128.0);
+}
 
 /* ------------------------------------------------------------------------ */
 /* IEEE-754 binary16, written from the format's definition:                 */
@@ -206,7 +259,8 @@ void zo_unpack_row(const uint32_t *words, int K, int bits, uint8_t *codes)
 
 static int zo_check_format(int N, int K, int bits, int group)
 {
-    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8) || group != 128)
+    if (!(bits == 2 || bits == 3 || bits == 4 || bits == 8) ||
+        !(group == 32 || group == 64 || group == 128))
         return ZO_UNSUPPORTED;
     if (N <= 0 || K <= 0 || K % group != 0)
         return ZO_INVALID;
@@ -275,7 +329,7 @@ int zo_quantize_pack_symmetric(const float *w, int N, int K, int bits, int group
 
 int zo_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes)
 {
-    int st = zo_check_format(N, K, bits, 128);
+    int st = zo_check_format(N, K, bits, 32);  /* rows of whole words: K a multiple of 32 */
     if (st != ZO_OK)
         return st;
     int wpr = K * bits / 32;
@@ -312,15 +366,20 @@ int zo_dequant(const uint32_t *packed, const uint16_t *scales, const uint16_t *z
 /* Linear on a subset of output columns: for each listed row r of W (output
  * feature), y[m][i] = sum_k x[m][k] * w_hat[r][k] and
  * bound[m][i] = sum_k |x[m][k]| * |w_hat[r][k]|, both fp64. x is M x K fp16
- * bit patterns; y and bound are M x nrows. Pass rows == NULL for all N rows. */
-int zo_linear_rows(const uint16_t *x, int M, int K,
-                   const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros,
-                   int bits, int group, int N, const int64_t *rows, int nrows,
-                   double *y, double *bound)
+ * (xfmt 0) or bf16 (xfmt 1) bit patterns; y and bound are M x nrows. Pass
+ * rows == NULL for all N rows.  bits == 16: `packed` holds the weights as
+ * fp16 bit patterns, N x K (read as uint16), w_hat is their value, and
+ * scales/zeros are not read. */
+int zo_linear_rows_ex(const uint16_t *x, int xfmt, int M, int K,
+                      const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros,
+                      int bits, int group, int N, const int64_t *rows, int nrows,
+                      double *y, double *bound)
 {
-    int st = zo_check_format(N, K, bits, group);
+    int st = bits == 16 ? ((N <= 0 || K <= 0) ? ZO_INVALID : ZO_OK) : zo_check_format(N, K, bits, group);
     if (st != ZO_OK)
         return st;
+    if (xfmt != 0 && xfmt != 1)
+        return ZO_UNSUPPORTED;
     if (M <= 0)
         return ZO_INVALID;
     if (rows == NULL)
@@ -330,22 +389,28 @@ int zo_linear_rows(const uint16_t *x, int M, int K,
         if (r < 0 || r >= N)
             return ZO_INVALID;
     }
-    int G = K / group;
-    int wpr = K * bits / 32;
+    int G = bits == 16 ? 0 : K / group;
+    int wpr = bits == 16 ? 0 : K * bits / 32;
     double *xd = (double *)malloc((size_t)M * K * sizeof(double));
     for (size_t i = 0; i < (size_t)M * K; ++i)
-        xd[i] = zo_f16_to_f64(x[i]);
+        xd[i] = xfmt == 1 ? zo_bf16_to_f64(x[i]) : zo_f16_to_f64(x[i]);
 #pragma omp parallel for schedule(dynamic, 4)
     for (int i = 0; i < nrows; ++i) {
         long r = rows ? (long)rows[i] : i;
         uint8_t *codes = (uint8_t *)malloc((size_t)K);
         double *wh = (double *)malloc((size_t)K * sizeof(double));
-        zo_unpack_row(packed + (size_t)r * wpr, K, bits, codes);
-        for (int k = 0; k < K; ++k) {
-            int g = k / group;
-            double s = zo_f16_to_f64(scales[(size_t)r * G + g]);
-            double z = zo_f16_to_f64(zeros[(size_t)r * G + g]);
-            wh[k] = (double)codes[k] * s + z;
+        if (bits == 16) {
+            const uint16_t *w16 = (const uint16_t *)packed + (size_t)r * K;
+            for (int k = 0; k < K; ++k)
+                wh[k] = zo_f16_to_f64(w16[k]);
+        } else {
+            zo_unpack_row(packed + (size_t)r * wpr, K, bits, codes);
+            for (int k = 0; k < K; ++k) {
+                int g = k / group;
+                double s = zo_f16_to_f64(scales[(size_t)r * G + g]);
+                double z = zo_f16_to_f64(zeros[(size_t)r * G + g]);
+                wh[k] = (double)codes[k] * s + z;
+            }
         }
         for (int m = 0; m < M; ++m) {
             double acc = 0.0, bnd = 0.0;
@@ -362,6 +427,15 @@ int zo_linear_rows(const uint16_t *x, int M, int K,
     }
     free(xd);
     return ZO_OK;
+}
+
+/* fp16 activations; see zo_linear_rows_ex. */
+int zo_linear_rows(const uint16_t *x, int M, int K,
+                   const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros,
+                   int bits, int group, int N, const int64_t *rows, int nrows,
+                   double *y, double *bound)
+{
+    return zo_linear_rows_ex(x, 0, M, K, packed, scales, zeros, bits, group, N, rows, nrows, y, bound);
 }
 
 /* Thread control for timing the oracle on the host cores. */
