@@ -19,9 +19,11 @@
  *
  * Tensor format (all buffers row-major and contiguous):
  *   W       N x K weights (output features x input features; y = x W^T).
- *   bits    b in {2, 3, 4, 8}, chosen per tensor.  L = 2^b - 1.
- *   group   128 consecutive weights along K share one fp16 scale and one fp16
- *           zero.  K must be a multiple of 128.  G = K / 128.
+ *   bits    b in {2, 3, 4, 8}, chosen per tensor.  L = 2^b - 1.  (bits = 16:
+ *           fp16 weights kept unquantized, see zq_linear.)
+ *   group   g consecutive weights along K share one fp16 scale and one fp16
+ *           zero: g = 128 (the pages' figure), or 64 or 32 (the encoding
+ *           variants).  K must be a multiple of 128.  G = K / g.
  *   packed  uint32 N x (K*b/32).  The codes of one row form a little-endian
  *           bitstream: code k occupies stream bits [k*b, k*b+b), and stream bit
  *           t is bit (t % 32) of word t / 32.  At b = 4 this is the pages'
@@ -81,7 +83,7 @@ typedef struct CUstream_st *zq_stream_t; /* identical to cudaStream_t */
 typedef enum {
     ZQ_OK = 0,
     ZQ_ERR_INVALID_ARG = 1, /* bad size, null or misaligned pointer          */
-    ZQ_ERR_UNSUPPORTED = 2, /* bits not in {2,3,4,8} or group != 128          */
+    ZQ_ERR_UNSUPPORTED = 2, /* bits not in {2,3,4,8} or group not in {32,64,128} */
     ZQ_ERR_NONFINITE = 3,   /* a weight is NaN/Inf or |w| > 65504 (fp16 max)  */
     ZQ_ERR_CUDA = 4,        /* a CUDA runtime call failed                     */
     ZQ_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up             */
@@ -132,15 +134,37 @@ ZQ_API zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bi
  *   x       device, fp16 M x K.      out  device, fp16 M x N (written).
  *   packed/scales/zeros as produced by zq_quantize_pack.
  * M <= 16 runs the decode kernel (mma.sync skinny GEMM streaming the packed
- * weights once through a shared-memory ring); larger M runs the tcgen05 tile
- * kernel (256 x 256 output tiles; with M <= 256 one token tile, so the
- * weights are again streamed once).  Needs a workspace of
- * zq_linear_workspace_bytes(bits, M, N, K) on `stream` (see Conventions).
+ * weights once through a shared-memory ring); larger M, and groups of 32 or
+ * 64 at any M, run the tcgen05 tile kernel (256 x 256 output tiles; with
+ * M <= 256 one token tile, so the weights are again streamed once).
+ * bits = 16 is the fp16 passthrough of the .zse format ([wiki] "Формат
+ * модели .zse": tensors kept unquantized): `packed` then holds the weights as
+ * fp16 N x K, `scales`, `zeros` and `group` are not read (may be NULL / any).
+ * Needs a workspace of zq_linear_workspace_bytes(bits, M, N, K) on `stream`
+ * (see Conventions; the size for group 128 covers every group size).
  * Asynchronous; fp32 accumulation, fp16 output rounded to nearest even. */
 ZQ_API zq_status zq_linear(const uint16_t *x, const uint32_t *packed,
                     const uint16_t *scales, const uint16_t *zeros,
                     int bits, int group, int M, int N, int K,
                     uint16_t *out, zq_stream_t stream);
+
+/* zq_linear with bfloat16 activations and output (the encoding variants next
+ * to [wiki] "Формат модели .zse"; the pages fix no activation type).
+ *   x    device, bfloat16 bit patterns M x K.   out  device, bfloat16 M x N.
+ * Weights, formats, kernels and errors as zq_linear.  The products still run
+ * in fp16 on the tensor cores: each activation group (decode kernel) or token
+ * row (tile kernel) is scaled by a power of two into fp16's range, exactly
+ * for every value within 2^24 of the largest, and the factor is divided out
+ * in fp32; activations of magnitude 2^55 or more are out of range.  The tile
+ * kernel keeps that fp16 copy in the workspace: size it with
+ * zq_linear_bf16_workspace_bytes.  Output rounded once to bfloat16 (nearest
+ * even).  Asynchronous. */
+ZQ_API zq_status zq_linear_bf16(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                                const uint16_t *zeros, int bits, int group, int M, int N, int K,
+                                uint16_t *out, zq_stream_t stream);
+
+/* Workspace bytes of zq_linear_bf16 with these sizes (0 for invalid sizes). */
+ZQ_API size_t zq_linear_bf16_workspace_bytes(int bits, int M, int N, int K);
 
 /* Allocation-free zq_linear, for callers that cannot allocate device memory:
  * code running inside a CUDA stream capture (where cudaMalloc is not
@@ -185,6 +209,13 @@ typedef struct {
  * (zq_linear_stack_workspace_bytes), are checked before anything is
  * enqueued.  Asynchronous. */
 ZQ_API zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stream);
+
+/* zq_linear_stack with bfloat16 activations and outputs: every op's x and out
+ * hold bfloat16 (see zq_linear_bf16); `ops` as zq_linear_stack.  The
+ * workspace it needs is zq_linear_stack_bf16_workspace_bytes(ops, n_ops).
+ * Asynchronous. */
+ZQ_API zq_status zq_linear_stack_bf16(const zq_linear_desc *ops, int n_ops, zq_stream_t stream);
+ZQ_API size_t zq_linear_stack_bf16_workspace_bytes(const zq_linear_desc *ops, int n_ops);
 
 /* Test hook: unpack codes with the same device unpack routine zq_linear
  * uses; the inverse of the packing of [wiki] "Формат модели .zse" (code k of

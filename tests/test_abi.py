@@ -34,7 +34,7 @@ def zq():
 def _declared_functions():
     text = "".join(open(h).read() for h in HEADERS)
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(zq_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(zq_[a-z0-9_]+)\s*\(", text)))
 
 
 def test_header_declares_expected_entry_points(zq):
@@ -84,7 +84,8 @@ def _lin(zq, **kw):
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(bits=5), 2), (dict(bits=1), 2), (dict(bits=16), 2), (dict(group=64), 2),
+    (dict(bits=5), 2), (dict(bits=1), 2), (dict(bits=12), 2), (dict(group=48), 2), (dict(group=256), 2),
+    (dict(group=16), 2), (dict(bits=16, K=100), 1), (dict(bits=16, x=0), 1),
     (dict(K=100), 1), (dict(K=0), 1), (dict(N=0), 1), (dict(M=0), 1), (dict(M=-3), 1),
     (dict(x=0), 1), (dict(packed=0), 1), (dict(scales=0), 1), (dict(zeros=0), 1),
     (dict(out=0), 1), (dict(x=A + 8), 1), (dict(out=A + 2), 1), (dict(packed=A + 4), 1),
@@ -98,7 +99,8 @@ def test_linear_rejects(zq, kw, status):
 def test_quantize_rejects(zq, name):
     q = getattr(zq._lib, name)
     assert q(A, 4, 256, 5, 128, A, A, A, None) == zq.ZQ_ERR_UNSUPPORTED
-    assert q(A, 4, 256, 4, 32, A, A, A, None) == zq.ZQ_ERR_UNSUPPORTED
+    assert q(A, 4, 256, 4, 16, A, A, A, None) == zq.ZQ_ERR_UNSUPPORTED
+    assert q(A, 4, 256, 16, 128, A, A, A, None) == zq.ZQ_ERR_UNSUPPORTED  # fp16 weights are not quantized
     assert q(A, 4, 200, 4, 128, A, A, A, None) == zq.ZQ_ERR_INVALID_ARG
     assert q(0, 4, 256, 4, 128, A, A, A, None) == zq.ZQ_ERR_INVALID_ARG
     assert q(A, 4, 256, 4, 128, A + 1, A, A, None) == zq.ZQ_ERR_INVALID_ARG

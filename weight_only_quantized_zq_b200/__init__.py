@@ -35,7 +35,8 @@ EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_quantize_pack_symmetric", 
            "zq_zse_find", "zq_zse_section", "zq_zse_weight_bytes", "zq_zse_verify", "zq_zse_load_weights",
            "zq_kv_plane_bytes", "zq_kv_append", "zq_kv_gather",
            "zq_linear_partial", "zq_linear_partial_stack", "zq_linear_partial_stack_workspace_bytes",
-           "zq_reduce_partials")
+           "zq_reduce_partials", "zq_linear_bf16", "zq_linear_bf16_workspace_bytes", "zq_linear_stack_bf16",
+           "zq_linear_stack_bf16_workspace_bytes")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -154,6 +155,14 @@ _lib.zq_linear_partial_stack_workspace_bytes.argtypes = [_P, _I]
 _lib.zq_linear_partial_stack_workspace_bytes.restype = _S
 _lib.zq_reduce_partials.argtypes = [ctypes.POINTER(_P), _I, _S, _P, _P]
 _lib.zq_reduce_partials.restype = _I
+_lib.zq_linear_bf16.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P]
+_lib.zq_linear_bf16.restype = _I
+_lib.zq_linear_bf16_workspace_bytes.argtypes = [_I, _I, _I, _I]
+_lib.zq_linear_bf16_workspace_bytes.restype = _S
+_lib.zq_linear_stack_bf16.argtypes = [_P, _I, _P]
+_lib.zq_linear_stack_bf16.restype = _I
+_lib.zq_linear_stack_bf16_workspace_bytes.argtypes = [_P, _I]
+_lib.zq_linear_stack_bf16_workspace_bytes.restype = _S
 
 
 def _check(status):
@@ -317,17 +326,40 @@ def zq_reduce_partials(parts, count, out, stream=None):
                                    _stream(stream, out if isinstance(out, torch.Tensor) else None)))
 
 
+def zq_linear_bf16(x, packed, scales, zeros, bits, group, M, N, K, out, stream=None):
+    _check(_lib.zq_linear_bf16(_ptr(x), _ptr(packed), _ptr(scales), _ptr(zeros), bits, group,
+                               M, N, K, _ptr(out), _stream(stream, x)))
+
+
+def zq_linear_bf16_workspace_bytes(bits, M, N, K):
+    return _lib.zq_linear_bf16_workspace_bytes(bits, M, N, K)
+
+
+def zq_linear_stack_bf16(ops, n_ops=None, stream=None):
+    if not isinstance(ops, ctypes.Array):
+        ops, n = make_descs(ops)
+        n_ops = n if n_ops is None else n_ops
+    _check(_lib.zq_linear_stack_bf16(ops, n_ops, _stream(stream)))
+
+
+def zq_linear_stack_bf16_workspace_bytes(ops, n_ops=None):
+    if not isinstance(ops, ctypes.Array):
+        ops, n = make_descs(ops)
+        n_ops = n if n_ops is None else n_ops
+    return _lib.zq_linear_stack_bf16_workspace_bytes(ops, n_ops)
+
+
 def zq_unpack(packed, N, K, bits, codes, stream=None):
     _check(_lib.zq_unpack(_ptr(packed), N, K, bits, _ptr(codes), _stream(stream, packed)))
 
 
 # ------------------------------------------------------------ conveniences --
 
-def alloc_quantized(N, K, bits, device="cuda"):
+def alloc_quantized(N, K, bits, device="cuda", group=GROUP):
     """Empty (packed, scales, zeros) buffers for an N x K tensor."""
     packed = torch.empty(N * K * bits // 32, dtype=torch.int32, device=device)
-    scales = torch.empty(N, K // GROUP, dtype=torch.int16, device=device)
-    zeros = torch.empty(N, K // GROUP, dtype=torch.int16, device=device)
+    scales = torch.empty(N, K // group, dtype=torch.int16, device=device)
+    zeros = torch.empty(N, K // group, dtype=torch.int16, device=device)
     return packed, scales, zeros
 
 
@@ -339,16 +371,20 @@ def _need(t, nbytes, dtype, what, device):
                       f"{t.numel() * t.element_size() if isinstance(t, torch.Tensor) else '?'} bytes")
 
 
-def quantize(w, bits, stream=None, symmetric=False):
+def quantize(w, bits, stream=None, symmetric=False, group=GROUP):
     """fp32 CUDA tensor N x K -> (packed, scales, zeros) via zq_quantize_pack
-    (or zq_quantize_pack_symmetric); both give the same storage format."""
+    (or zq_quantize_pack_symmetric); both give the same storage format.
+    group: 128 (default), 64 or 32 weights per scale and zero."""
     if w.dim() != 2:
         raise ZQError(ZQ_ERR_INVALID_ARG, f"w must be 2-D (N x K), got shape {tuple(w.shape)}")
     N, K = w.shape
     _need(w, N * K * 4, torch.float32, "w", w.device)
-    packed, scales, zeros = alloc_quantized(N, K, bits, w.device)
+    if group not in (32, 64, 128) or K % 128:
+        raise ZQError(ZQ_ERR_UNSUPPORTED if group not in (32, 64, 128) else ZQ_ERR_INVALID_ARG,
+                      f"group={group} (32, 64 or 128) and K={K} (a multiple of 128)")
+    packed, scales, zeros = alloc_quantized(N, K, bits, w.device, group)
     fn = zq_quantize_pack_symmetric if symmetric else zq_quantize_pack
-    fn(w, N, K, bits, GROUP, packed, scales, zeros, stream)
+    fn(w, N, K, bits, group, packed, scales, zeros, stream)
     return packed, scales, zeros
 
 
@@ -382,23 +418,28 @@ def linear_partial(x, packed, scales, zeros, bits, N, out=None, stream=None):
     return out
 
 
-def linear(x, packed, scales, zeros, bits, N, out=None, stream=None):
-    """fp16 CUDA x (M x K) -> fp16 out (M x N) via zq_linear (reserving the
-    workspace it needs on the stream first)."""
+def linear(x, packed, scales, zeros, bits, N, out=None, stream=None, group=GROUP):
+    """fp16 (or bfloat16) CUDA x (M x K) -> out (M x N) of the same type via
+    zq_linear (zq_linear_bf16), reserving the workspace it needs on the stream
+    first.  bits=16: `packed` is the fp16 weights (N x K) and scales/zeros may
+    be None."""
     if x.dim() != 2:
         raise ZQError(ZQ_ERR_INVALID_ARG, f"x must be 2-D (M x K), got shape {tuple(x.shape)}")
     M, K = x.shape
-    _need(x, M * K * 2, torch.float16, "x", x.device)
-    if K % GROUP == 0 and bits in (2, 3, 4, 8):  # other formats: the library reports them
+    bf16 = x.dtype == torch.bfloat16
+    xt = torch.bfloat16 if bf16 else torch.float16
+    _need(x, M * K * 2, xt, "x", x.device)
+    if K % 128 == 0 and bits in (2, 3, 4, 8, 16) and group in (32, 64, 128):  # else the library reports it
         _need(packed, N * K * bits // 8, packed.dtype, "packed", x.device)
-        _need(scales, N * (K // GROUP) * 2, scales.dtype, "scales", x.device)
-        _need(zeros, N * (K // GROUP) * 2, zeros.dtype, "zeros", x.device)
+        if bits != 16:
+            _need(scales, N * (K // group) * 2, scales.dtype, "scales", x.device)
+            _need(zeros, N * (K // group) * 2, zeros.dtype, "zeros", x.device)
     if out is None:
-        out = torch.empty(M, N, dtype=torch.float16, device=x.device)
-    _need(out, M * N * 2, torch.float16, "out", x.device)
-    ensure_workspace(zq_linear_workspace_bytes(bits, M, N, K), stream if stream is not None else
-                     torch.cuda.current_stream(x.device))
-    zq_linear(x, packed, scales, zeros, bits, GROUP, M, N, K, out, stream)
+        out = torch.empty(M, N, dtype=xt, device=x.device)
+    _need(out, M * N * 2, xt, "out", x.device)
+    ws = zq_linear_bf16_workspace_bytes if bf16 else zq_linear_workspace_bytes
+    ensure_workspace(ws(bits, M, N, K), stream if stream is not None else torch.cuda.current_stream(x.device))
+    (zq_linear_bf16 if bf16 else zq_linear)(x, packed, scales, zeros, bits, group, M, N, K, out, stream)
     return out
 
 

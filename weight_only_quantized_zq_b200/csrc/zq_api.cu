@@ -53,9 +53,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool bits_ok(int bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
 
+bool group_ok(int group) { return group == 32 || group == 64 || group == 128; }
+
 zq_status check_format(int bits, int group, int N, int K) {
     if (!bits_ok(bits)) return fail(ZQ_ERR_UNSUPPORTED, "bits=%d not in {2,3,4,8}", bits);
-    if (group != kGroup) return fail(ZQ_ERR_UNSUPPORTED, "group=%d, only 128 is supported", group);
+    if (!group_ok(group)) return fail(ZQ_ERR_UNSUPPORTED, "group=%d not in {32, 64, 128}", group);
     if (N <= 0 || K <= 0) return fail(ZQ_ERR_INVALID_ARG, "N=%d K=%d must be positive", N, K);
     if (K % kGroup != 0) return fail(ZQ_ERR_INVALID_ARG, "K=%d is not a multiple of 128", K);
     if (static_cast<long long>(N) * K > (1LL << 40))
@@ -69,14 +71,17 @@ zq_status check_ptr(const void *p, const char *name) {
     return ZQ_OK;
 }
 
+// bits == 16: fp16 weights (N x K in `packed`), no scales or zeros, group not read.
 zq_status check_linear(const zq_linear_desc &d) {
-    zq_status st = check_format(d.bits, d.group, d.N, d.K);
+    zq_status st = d.bits == 16 ? check_format(4, kGroup, d.N, d.K) : check_format(d.bits, d.group, d.N, d.K);
     if (st != ZQ_OK) return st;
     if (d.M <= 0) return fail(ZQ_ERR_INVALID_ARG, "M=%d must be positive", d.M);
     if ((st = check_ptr(d.x, "x")) != ZQ_OK) return st;
     if ((st = check_ptr(d.packed, "packed")) != ZQ_OK) return st;
-    if ((st = check_ptr(d.scales, "scales")) != ZQ_OK) return st;
-    if ((st = check_ptr(d.zeros, "zeros")) != ZQ_OK) return st;
+    if (d.bits != 16) {
+        if ((st = check_ptr(d.scales, "scales")) != ZQ_OK) return st;
+        if ((st = check_ptr(d.zeros, "zeros")) != ZQ_OK) return st;
+    }
     if ((st = check_ptr(d.out, "out")) != ZQ_OK) return st;
     return ZQ_OK;
 }
@@ -86,6 +91,7 @@ zq_status check_linear(const zq_linear_desc &d) {
 // out is null).
 struct Op : zq_linear_desc {
     float *out32 = nullptr;
+    int xbf16 = 0;  // x and out hold bfloat16 (out32 must then be null)
 };
 
 Op make_op(const zq_linear_desc &d) {
@@ -211,8 +217,10 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct PrepKey {
     const uint16_t *x;
-    int M, K, bits;
-    bool operator==(const PrepKey &o) const { return x == o.x && M == o.M && K == o.K && bits == o.bits; }
+    int M, K, bits, xbf16;
+    bool operator==(const PrepKey &o) const {
+        return x == o.x && M == o.M && K == o.K && bits == o.bits && xbf16 == o.xbf16;
+    }
 };
 
 // Shared memory of one decode CTA: `depth` stages, two mbarriers per stage,
@@ -235,7 +243,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     std::vector<PrepKey> keys;
     std::vector<int> op_entry(ops.size());
     for (size_t i = 0; i < ops.size(); ++i) {
-        PrepKey k{ops[i].x, ops[i].M, ops[i].K, bits};
+        PrepKey k{ops[i].x, ops[i].M, ops[i].K, bits, ops[i].xbf16};
         auto it = std::find(keys.begin(), keys.end(), k);
         if (it == keys.end()) {
             keys.push_back(k);
@@ -359,6 +367,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         en.x_rows = mt == 1 ? keys[e].M : mpad;
         en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(G * en.x_rows * kGroup * 2));
         en.M = keys[e].M;
+        en.x_bf16 = keys[e].xbf16;
         en.K = keys[e].K;
         en.bits = bits;
         pp.warp_prefix[e] = wsum;
@@ -403,7 +412,8 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         o.G = ops[i].K / kGroup;
         o.row_blocks = rbs[i];
         o.su = sus[i];
-        o.sz_vec = (o.G % gps) == 0 ? 1 : 0;
+        o.sz_vec = (bits != 16 && (o.G % gps) == 0) ? 1 : 0;  // fp16 weights have no scales or zeros
+        o.out_bf16 = ops[i].xbf16;
         const uint64_t row_bytes = static_cast<uint64_t>(o.K) * bits / 8;
         cudaError_t te = encode_tensor_map_2d(&o.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, ops[i].packed, row_bytes,
                                               static_cast<uint64_t>(o.N), row_bytes,
@@ -436,7 +446,7 @@ struct OpRanges {
 };
 
 OpRanges ranges_of(const Op &d) {
-    const size_t G = d.K / kGroup;
+    const size_t G = d.bits == 16 ? 0 : d.K / d.group;  // fp16 weights have no scales or zeros
     auto r = [](const void *p, size_t n) {
         const uintptr_t a = reinterpret_cast<uintptr_t>(p);
         return Range{a, a + n};
@@ -462,11 +472,46 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
 // One persistent launch over all tiles of independent prefill ops of one bit
 // width (at most kMaxPrefillOps), ops with the longest K first so that the
 // last tiles handed out are the cheap ones.
+// Workspace bytes of a tile-kernel launch: the fp16 copies (and per-token
+// factors) of its distinct bf16 activations.
+size_t prefill_data_bytes(const std::vector<Op> &ops) {
+    std::vector<const uint16_t *> seen;
+    size_t b = 0;
+    for (const auto &d : ops)
+        if (d.xbf16 && std::find(seen.begin(), seen.end(), d.x) == seen.end()) {
+            seen.push_back(d.x);
+            b += align256(static_cast<size_t>(d.M) * d.K * 2) + align256(static_cast<size_t>(d.M) * 4);
+        }
+    return b;
+}
+
 zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
     std::stable_sort(ops.begin(), ops.end(), [](const Op &a, const Op &b) { return a.K > b.K; });
+    // bf16 activations: an fp16 copy per distinct x, scaled per token, in the
+    // workspace (see zq_act.cu); the launch reads the copy.
+    std::vector<std::pair<const uint16_t *, std::pair<uint16_t *, float *>>> conv;
+    if (const size_t need = prefill_data_bytes(ops)) {
+        uint8_t *ws = nullptr;
+        if ((st = workspace(stream, need, &ws)) != ZQ_OK) return st;
+        uint8_t *at = ws + kCounterBytes;
+        for (const auto &d : ops) {
+            if (!d.xbf16) continue;
+            bool known = false;
+            for (const auto &c : conv) known = known || c.first == d.x;
+            if (known) continue;
+            uint16_t *x16 = reinterpret_cast<uint16_t *>(at);
+            at += align256(static_cast<size_t>(d.M) * d.K * 2);
+            float *f = reinterpret_cast<float *>(at);
+            at += align256(static_cast<size_t>(d.M) * 4);
+            cudaError_t e = launch_bf16_rows_to_f16(d.x, d.M, d.K, x16, f, stream);
+            if (e != cudaSuccess) return cuda_fail(e, "bf16 activation launch");
+            g_launches += 1;
+            conv.push_back({d.x, {x16, f}});
+        }
+    }
     PrefillGroup pg;
     std::memset(&pg, 0, sizeof(pg));
     pg.n_ops = static_cast<int>(ops.size());
@@ -475,8 +520,20 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     int tiles = 0;
     for (size_t i = 0; i < ops.size(); ++i) {
         PrefillOp &o = pg.ops[i];
-        cudaError_t e = prefill_x_map_rows(&o.xmap, ops[i].x, ops[i].M, ops[i].K, box_rows);
+        const uint16_t *xa = ops[i].x;
+        if (ops[i].xbf16)
+            for (const auto &c : conv)
+                if (c.first == ops[i].x) {
+                    xa = c.second.first;
+                    o.xscale = c.second.second;
+                }
+        o.out_bf16 = ops[i].xbf16;
+        cudaError_t e = prefill_x_map_rows(&o.xmap, xa, ops[i].M, ops[i].K, box_rows);
         if (e != cudaSuccess) return cuda_fail(e, "tensor map for x");
+        if (ops[i].bits == 16) {
+            e = prefill_w_map(&o.wmap, reinterpret_cast<const uint16_t *>(ops[i].packed), ops[i].N, ops[i].K);
+            if (e != cudaSuccess) return cuda_fail(e, "tensor map for the fp16 weights");
+        }
         o.packed = ops[i].packed;
         o.scales = ops[i].scales;
         o.zeros = ops[i].zeros;
@@ -485,6 +542,7 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
         o.M = ops[i].M;
         o.N = ops[i].N;
         o.K = ops[i].K;
+        o.gshift = ops[i].bits == 16 ? 2 : (ops[i].group == 32 ? 0 : ops[i].group == 64 ? 1 : 2);
         o.tok_tiles = (ops[i].M + 255) / 256;
         o.tile0 = tiles;
         tiles += prefill_tiles(ops[i].M, ops[i].N);
@@ -503,21 +561,28 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
 // of the launches needs (at least the counters).
 zq_status run_batch(const std::vector<Op> &batch, cudaStream_t stream, size_t *dry = nullptr) {
     std::vector<Op> pieces;
-    const int bits_list[4] = {2, 3, 4, 8};
+    const int bits_list[5] = {2, 3, 4, 8, 16};
     if (dry) *dry = std::max(*dry, kCounterBytes);
+    // The decode kernel applies one scale and zero per 128-code block, so
+    // groups of 32 or 64 run on the tile kernel at any M.
+    const auto on_tile = [](const Op &d) { return d.M > kDecodeMaxM || (d.bits != 16 && d.group != kGroup); };
     for (int bits : bits_list) {
         std::vector<Op> pre;
         for (const auto &d : batch)
-            if (d.M > kDecodeMaxM && d.bits == bits) pre.push_back(d);
-        for (size_t i = 0; i < pre.size() && !dry; i += kMaxPrefillOps) {
+            if (on_tile(d) && d.bits == bits) pre.push_back(d);
+        for (size_t i = 0; i < pre.size(); i += kMaxPrefillOps) {
             std::vector<Op> launch(pre.begin() + i,
                                                pre.begin() + std::min(pre.size(), i + kMaxPrefillOps));
+            if (dry) {
+                *dry = std::max(*dry, kCounterBytes + prefill_data_bytes(launch));
+                continue;
+            }
             zq_status st = run_prefill(launch, stream);
             if (st != ZQ_OK) return st;
         }
     }
     for (const auto &d : batch)
-        if (d.M <= kDecodeMaxM) pieces.push_back(d);
+        if (!on_tile(d)) pieces.push_back(d);
     const int mt_list[2] = {1, 2};
     for (int bits : bits_list)
         for (int mt : mt_list) {
@@ -664,7 +729,7 @@ zq_status zq_quantize_pack(const float *w, int N, int K, int bits, int group, ui
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long id = g_quant_call.fetch_add(1);
     const int slot = static_cast<int>(id % kQuantStatusSlots);
-    cudaError_t e = launch_quantize_pack(w, N, K, bits, packed, scales, zeros, slot, id, s);
+    cudaError_t e = launch_quantize_pack(w, N, K, bits, group, packed, scales, zeros, slot, id, s);
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     ++g_launches;
     unsigned long long got = 0;
@@ -685,7 +750,7 @@ zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bits, int
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const unsigned long long id = g_quant_call.fetch_add(1);
     const int slot = static_cast<int>(id % kQuantStatusSlots);
-    cudaError_t e = launch_quantize_pack_symmetric(w, N, K, bits, packed, scales, zeros, slot, id, s);
+    cudaError_t e = launch_quantize_pack_symmetric(w, N, K, bits, group, packed, scales, zeros, slot, id, s);
     if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
     ++g_launches;
     unsigned long long got = 0;
@@ -727,6 +792,8 @@ zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uin
     if (st != ZQ_OK) return st;
     if (M > kNoallocMaxM)
         return fail(ZQ_ERR_UNSUPPORTED, "zq_linear_noalloc supports M <= %d (got M=%d)", kNoallocMaxM, M);
+    if (bits != 16 && group != kGroup)
+        return fail(ZQ_ERR_UNSUPPORTED, "zq_linear_noalloc supports groups of 128 (got %d)", group);
     uint8_t *ws = nullptr;
     if ((st = noalloc_scratch(&ws)) != ZQ_OK) return st;
     std::vector<Op> one{make_op(d)};
@@ -741,6 +808,17 @@ zq_status zq_linear_noalloc(const uint16_t *x, const uint32_t *packed, const uin
     cudaError_t e = cudaMemsetAsync(ws, 0, kCounterBytes, s);
     if (e != cudaSuccess) return cuda_fail(e, "clearing the scratch counters");
     return run_decode(one, bits, mt_for_m(M), s, nullptr, ws, kNoallocScratchBytes);
+}
+
+zq_status zq_linear_bf16(const uint16_t *x, const uint32_t *packed, const uint16_t *scales,
+                         const uint16_t *zeros, int bits, int group, int M, int N, int K, uint16_t *out,
+                         zq_stream_t stream) {
+    zq_linear_desc d{x, packed, scales, zeros, out, bits, group, M, N, K};
+    zq_status st = check_linear(d);
+    if (st != ZQ_OK) return st;
+    Op op = make_op(d);
+    op.xbf16 = 1;
+    return checked_stack(&op, 1, reinterpret_cast<cudaStream_t>(stream));
 }
 
 // Validates the public descriptors of a stack (fp16 outputs, or fp32 partial
@@ -776,6 +854,23 @@ zq_status zq_linear_stack(const zq_linear_desc *ops, int n_ops, zq_stream_t stre
     zq_status st = stack_ops(ops, nullptr, n_ops, &v);
     if (st != ZQ_OK) return st;
     return checked_stack(v.data(), n_ops, reinterpret_cast<cudaStream_t>(stream));
+}
+
+zq_status zq_linear_stack_bf16(const zq_linear_desc *ops, int n_ops, zq_stream_t stream) {
+    std::vector<Op> v;
+    zq_status st = stack_ops(ops, nullptr, n_ops, &v);
+    if (st != ZQ_OK) return st;
+    for (auto &op : v) op.xbf16 = 1;
+    return checked_stack(v.data(), n_ops, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t zq_linear_stack_bf16_workspace_bytes(const zq_linear_desc *ops, int n_ops) {
+    std::vector<Op> v;
+    if (stack_ops(ops, nullptr, n_ops, &v) != ZQ_OK) return 0;
+    for (auto &op : v) op.xbf16 = 1;
+    size_t need = 0;
+    if (run_stack(v.data(), n_ops, nullptr, &need) != ZQ_OK) return 0;
+    return need;
 }
 
 zq_status zq_linear_partial_stack(const zq_partial_desc *ops, int n_ops, zq_stream_t stream) {
@@ -925,7 +1020,7 @@ zq_status zq_release_all_workspaces(void) {
 }
 
 size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
-    if (check_format(bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
+    if (check_format(bits == 16 ? 4 : bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
     // the plan needs only the sizes: any aligned, distinct fake pointers do
     const auto fake = [](uintptr_t i) { return reinterpret_cast<void *>(i << 20); };
     const Op d = make_op(zq_linear_desc{static_cast<const uint16_t *>(fake(1)),
@@ -933,6 +1028,18 @@ size_t zq_linear_workspace_bytes(int bits, int M, int N, int K) {
                                         static_cast<const uint16_t *>(fake(3)),
                                         static_cast<const uint16_t *>(fake(4)),
                                         static_cast<uint16_t *>(fake(1 << 20)), bits, kGroup, M, N, K});
+    size_t need = 0;
+    if (run_stack(&d, 1, nullptr, &need) != ZQ_OK) return 0;
+    return need;
+}
+
+size_t zq_linear_bf16_workspace_bytes(int bits, int M, int N, int K) {
+    if (check_format(bits == 16 ? 4 : bits, kGroup, N, K) != ZQ_OK || M <= 0) return 0;
+    const auto fake = [](uintptr_t i) { return reinterpret_cast<void *>(i << 20); };
+    Op d = make_op(zq_linear_desc{static_cast<const uint16_t *>(fake(1)), static_cast<const uint32_t *>(fake(2)),
+                                  static_cast<const uint16_t *>(fake(3)), static_cast<const uint16_t *>(fake(4)),
+                                  static_cast<uint16_t *>(fake(1 << 20)), bits, kGroup, M, N, K});
+    d.xbf16 = 1;
     size_t need = 0;
     if (run_stack(&d, 1, nullptr, &need) != ZQ_OK) return 0;
     return need;

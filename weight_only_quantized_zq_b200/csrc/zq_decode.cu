@@ -37,6 +37,7 @@
 //    chunk blockIdx.x and takes further chunks from a counter.  A row block
 //    cut by a chunk boundary is reduced by the last warp to finish a piece of
 //    it, in chunk order, so results are deterministic.
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -78,16 +79,25 @@ __device__ __forceinline__ void static_for(F &&f) {
 __host__ __device__ constexpr int x_chunk(int c, int q, int t7) { return (4 * c + (q ^ (2 * (c >> 1)))) ^ t7; }
 
 // Exponent E of the (token, group) scaling: 2^E * max|x| lies in [2^14, 2^15);
-// E = 0 for an all-zero group.
+// E = 0 for an all-zero group.  fp16 activations give E in [-1, 38]; bf16
+// ones (fp32's exponent range) are held to [-40, 100], i.e. groups whose
+// largest |x| is in [2^-86, 2^55).
 __device__ __forceinline__ int prep_exponent(float amax) {
     if (!(amax > 0.0f)) return 0;
-    const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127;  // floor(log2 amax), amax normal
-    return 14 - ex;
+    const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu) - 127;  // floor(log2 amax)
+    return max(-40, min(14 - ex, 100));
+}
+
+// One activation as float: fp16 bits, or bfloat16 bits (the top half of a binary32).
+template <bool BF16>
+__device__ __forceinline__ float act_bits(uint32_t h) {
+    if constexpr (BF16) return __uint_as_float(h << 16);
+    else return h2f_bits(h);
 }
 
 __device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(127 + e) << 23); }
 
-template <int B>
+template <int B, bool BF16>
 __device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow, int lane, int t7, int E) {
     float bias = 0.0f;  // sum of the scaled activations written by this lane
 #pragma unroll
@@ -95,8 +105,8 @@ __device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow
         const int q = lane + 32 * h;  // 64 pairs per group
         const int c = q / 16, p = q % 16;
         const float sc = pow2f(E - pair_shift<B>(p));  // exact power of two
-        const __half lo = __float2half_rn(h2f_bits(xrow[32 * c + pair_lo<B>(p)]) * sc);
-        const __half hi = __float2half_rn(h2f_bits(xrow[32 * c + pair_hi<B>(p)]) * sc);
+        const __half lo = __float2half_rn(act_bits<BF16>(xrow[32 * c + pair_lo<B>(p)]) * sc);
+        const __half hi = __float2half_rn(act_bits<BF16>(xrow[32 * c + pair_hi<B>(p)]) * sc);
         bias += __half2float(lo) + __half2float(hi);
         const int word = (x_chunk(c, p >> 2, t7) << 2) | (p & 3);
         reinterpret_cast<uint32_t *>(prow)[word] = __half_as_ushort(lo) | (__half_as_ushort(hi) << 16);
@@ -126,19 +136,33 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
             const uint16_t *xrow = en.x + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             uint16_t *prow = en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             const uint2 v = reinterpret_cast<const uint2 *>(xrow)[lane];
-            const float x0 = h2f_bits(v.x & 0xFFFFu), x1 = h2f_bits(v.x >> 16);
-            const float x2 = h2f_bits(v.y & 0xFFFFu), x3 = h2f_bits(v.y >> 16);
+            const bool bf = en.x_bf16 != 0;
+            const float x0 = bf ? act_bits<true>(v.x & 0xFFFFu) : act_bits<false>(v.x & 0xFFFFu);
+            const float x1 = bf ? act_bits<true>(v.x >> 16) : act_bits<false>(v.x >> 16);
+            const float x2 = bf ? act_bits<true>(v.y & 0xFFFFu) : act_bits<false>(v.y & 0xFFFFu);
+            const float x3 = bf ? act_bits<true>(v.y >> 16) : act_bits<false>(v.y >> 16);
             float s = x0 + x1 + x2 + x3;
             float amax = fmaxf(fmaxf(fabsf(x0), fabsf(x1)), fmaxf(fabsf(x2), fabsf(x3)));
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
             const int E = prep_exponent(amax);
             float b;
-            switch (en.bits) {
-                case 2: b = prep_group<2>(xrow, prow, lane, t & 7, E); break;
-                case 3: b = prep_group<3>(xrow, prow, lane, t & 7, E); break;
-                case 4: b = prep_group<4>(xrow, prow, lane, t & 7, E); break;
-                default: b = prep_group<8>(xrow, prow, lane, t & 7, E); break;
+            if (bf) {
+                switch (en.bits) {
+                    case 2: b = prep_group<2, true>(xrow, prow, lane, t & 7, E); break;
+                    case 3: b = prep_group<3, true>(xrow, prow, lane, t & 7, E); break;
+                    case 4: b = prep_group<4, true>(xrow, prow, lane, t & 7, E); break;
+                    case 8: b = prep_group<8, true>(xrow, prow, lane, t & 7, E); break;
+                    default: b = prep_group<16, true>(xrow, prow, lane, t & 7, E); break;
+                }
+            } else {
+                switch (en.bits) {
+                    case 2: b = prep_group<2, false>(xrow, prow, lane, t & 7, E); break;
+                    case 3: b = prep_group<3, false>(xrow, prow, lane, t & 7, E); break;
+                    case 4: b = prep_group<4, false>(xrow, prow, lane, t & 7, E); break;
+                    case 8: b = prep_group<8, false>(xrow, prow, lane, t & 7, E); break;
+                    default: b = prep_group<16, false>(xrow, prow, lane, t & 7, E); break;
+                }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
@@ -148,7 +172,9 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
             // f * (acc - 1024 * b) = fma(acc, f, -f * 1024 * b): the products
             // by the power of two f are exact.
             const float f = pow2f(-E);
-            if (lane == 0) *dst = make_float4(s, -(f * (1024.0f * b)), f, 0.0f);
+            // fp16 weights (bits 16) carry no 1024 bias
+            const float bias = en.bits == 16 ? 0.0f : 1024.0f * b;
+            if (lane == 0) *dst = make_float4(s, -(f * bias), f, 0.0f);
         }
     }
     // Dependents may be scheduled only now, i.e. after everything enqueued
@@ -267,6 +293,12 @@ __device__ __forceinline__ void mma_group(float (&acc)[4], const uint32_t (&w)[2
     }
 }
 
+// The output value rounded to fp16, or to bfloat16 for bf16 activations
+// (nearest even, either way).
+__device__ __forceinline__ uint16_t round_out(float v, int bf16) {
+    return bf16 ? __bfloat16_as_ushort(__float2bfloat16_rn(v)) : __half_as_ushort(__float2half_rn(v));
+}
+
 // Device record of a decode kernel that gave up a bounded wait (ZQ_ERR_TIMEOUT).
 __device__ int g_decode_error;
 
@@ -326,17 +358,17 @@ __device__ __forceinline__ bool wait_seq(const int *seq, int target, unsigned lo
 // its 8 fragment loads in 8 different bank groups.
 template <int BITS, int MT>
 __device__ __forceinline__ int box_row(int g) {
-    if constexpr (!decode_swizzled(BITS, MT) || BITS == 8) return g;  // b = 8: chunks 2c ^ g already differ
+    if constexpr (!decode_swizzled(BITS, MT) || BITS == 8 || BITS == 16) return g;  // b = 8: chunks 2c ^ g differ
     else if constexpr (BITS == 4) return (g >> 1) + 4 * (g & 1);       // rows 2j, 2j+1 -> j, j+4
     else return 2 * (g & 3) + (g >> 2);                                // b = 2 (half-warp phases)
 }
 
-// CTAs per SM the register budget is sized for: the shared memory of the
-// host's ring (at least 3 stages) leaves room for 4 CTAs of one token tile,
-// except at b = 4, whose 18.5 KB stages fit 3.
+// CTAs per SM the register budget is sized for: with one token tile the
+// host's ring (3 stages) leaves shared memory for 4 CTAs (16 warps per SM,
+// 128 registers each), with two token tiles for 3.
 template <int BITS, int MT>
 __host__ __device__ constexpr int decode_min_ctas() {
-    return MT == 1 && BITS != 4 ? 4 : 3;
+    return MT == 1 ? 4 : 3;
 }
 
 template <int BITS, int MT>
@@ -539,12 +571,15 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     int lanex;
     if constexpr (BITS == 4) lanex = c ^ gr;
     else if constexpr (BITS == 2) lanex = (c >> 1) ^ gr;
+    else if constexpr (BITS == 16) lanex = 4 * (c & 1);  // fp16: box c >> 1, chunks (lanex + j) ^ gr
     else lanex = (2 * c) ^ gr;  // b = 8: chunks lanex and lanex ^ 1
     uint32_t cofs[2][2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
         const uint32_t crow = (warp * 16 + h * 8 + gr) * (SWZ ? 128 : BOXW);
-        if constexpr (!SWZ) {
+        if constexpr (BITS == 16) {
+            cofs[h][0] = cofs[h][1] = crow + (c >> 1) * BOXB;
+        } else if constexpr (!SWZ) {
             cofs[h][0] = cofs[h][1] = crow + 4 * BITS * c;
         } else if constexpr (BITS == 4) {
             cofs[h][0] = crow + (lanex << 4);
@@ -616,8 +651,10 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
         const int o = static_cast<int>(d0.x), rb = static_cast<int>(d0.y);
 
         // Scales and zeros of rows gr and gr + 8 for the GPS groups.
-        uint32_t szs[2][GPS / 2], szz[2][GPS / 2];
-        if (flags & kFlagSzVec) {
+        uint32_t szs[2][(GPS + 1) / 2], szz[2][(GPS + 1) / 2];
+        if constexpr (BITS == 16) {
+            // fp16 weights: no scales or zeros
+        } else if (flags & kFlagSzVec) {
             if constexpr (GPS == 4) {
                 const uint4 v0 = lds_v4(smb + szq0);
                 const uint4 v1 = lds_v4(smb + szq1);
@@ -652,7 +689,19 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
             uint32_t wv[2][BITS];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-                if constexpr (SWZ && BITS == 4) {
+                if constexpr (BITS == 16) {
+                    // fp16 weights: the lane's 32 codes are 64 bytes, 4 chunks
+                    // of box c >> 1 (2-way bank conflicts: lanes c and c + 2
+                    // read the same chunks of the two boxes)
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        const uint4 v = lds_v4(stb + cofs[h][0] + (((lanex + j) ^ gr) << 4));
+                        wv[h][4 * j] = v.x;
+                        wv[h][4 * j + 1] = v.y;
+                        wv[h][4 * j + 2] = v.z;
+                        wv[h][4 * j + 3] = v.w;
+                    }
+                } else if constexpr (SWZ && BITS == 4) {
                     const uint4 v = lds_v4(stb + cofs[h][gi & 1] + (gi * GB / 128) * BOXB);
                     wv[h][0] = v.x;
                     wv[h][1] = v.y;
@@ -679,9 +728,14 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                     wv[h][2] = lds_u32(stb + cofs[h][0] + gi * GB + 8);
                 }
             }
-            constexpr bool hi = (gi & 1) != 0;
-            const float sc[2] = {half_of<hi>(szs[0][gi / 2]), half_of<hi>(szs[1][gi / 2])};
-            const float zr[2] = {half_of<hi>(szz[0][gi / 2]), half_of<hi>(szz[1][gi / 2])};
+            float sc[2] = {1.0f, 1.0f}, zr[2] = {0.0f, 0.0f};  // fp16 weights: no scale, no zero
+            if constexpr (BITS != 16) {
+                constexpr bool hi = (gi & 1) != 0;
+                sc[0] = half_of<hi>(szs[0][gi / 2]);
+                sc[1] = half_of<hi>(szs[1][gi / 2]);
+                zr[0] = half_of<hi>(szz[0][gi / 2]);
+                zr[1] = half_of<hi>(szz[1][gi / 2]);
+            }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 uint32_t xfm[16];
@@ -698,23 +752,32 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                     }
                 }
                 const uint4 sa = lds_v4(smb + sxo + (gi * R + 8 * mt) * 16);
-                float acc[4];
-                mma_group<BITS, MT == 1>(acc, wv, xf, magic);
-                const float fa = __uint_as_float(sa.z);
-                // tot += s * f * (acc - bias) + z * sum(x), with f * (acc - bias)
-                // as one FMA (f is the token's power-of-two x' scale); with one
-                // token the odd C columns are padding.
+                // tot += s * f * (acc - bias) + z * sum(x): the z * sum(x) term
+                // first (it needs no MMA result, and its operands die early),
+                // then s * f * (acc - bias) with f * (acc - bias) as one FMA (f
+                // is the token's power-of-two x' scale); with one token the odd
+                // C columns are padding.
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    tot[mt][2 * h] = fmaf(sc[h], fmaf(acc[2 * h], fa, __uint_as_float(sa.y)),
-                                          fmaf(zr[h], __uint_as_float(sa.x), tot[mt][2 * h]));
+                for (int h = 0; h < 2; ++h) tot[mt][2 * h] = fmaf(zr[h], __uint_as_float(sa.x), tot[mt][2 * h]);
+                uint4 sb = make_uint4(0u, 0u, 0u, 0u);
                 if constexpr (!one_token) {
-                    const uint4 sb = lds_v4(smb + sxo + (gi * R + 8 * mt) * 16 + 16);
+                    sb = lds_v4(smb + sxo + (gi * R + 8 * mt) * 16 + 16);
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
-                        tot[mt][2 * h + 1] =
-                            fmaf(sc[h], fmaf(acc[2 * h + 1], __uint_as_float(sb.z), __uint_as_float(sb.y)),
-                                 fmaf(zr[h], __uint_as_float(sb.x), tot[mt][2 * h + 1]));
+                        tot[mt][2 * h + 1] = fmaf(zr[h], __uint_as_float(sb.x), tot[mt][2 * h + 1]);
+                }
+                float acc[4];
+                mma_group<BITS, MT == 1>(acc, wv, xf, magic);
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+                    tot[mt][2 * h] =
+                        fmaf(sc[h], fmaf(acc[2 * h], __uint_as_float(sa.z), __uint_as_float(sa.y)), tot[mt][2 * h]);
+                if constexpr (!one_token) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        tot[mt][2 * h + 1] = fmaf(
+                            sc[h], fmaf(acc[2 * h + 1], __uint_as_float(sb.z), __uint_as_float(sb.y)),
+                            tot[mt][2 * h + 1]);
                 }
             }
         };
@@ -761,7 +824,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                         if (row < op.N && tok < M) {
                             const size_t at = static_cast<size_t>(tok) * op.N + row;
                             if (op.out32) op.out32[at] = tot[mt][i];
-                            else op.out[at] = __half_as_ushort(__float2half_rn(tot[mt][i]));
+                            else op.out[at] = round_out(tot[mt][i], op.out_bf16);
                         }
                     }
             } else {
@@ -794,7 +857,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                         if (r0 + row < op.N) {
                             const size_t at = static_cast<size_t>(tok) * op.N + r0 + row;
                             if (op.out32) op.out32[at] = sum;
-                            else op.out[at] = __half_as_ushort(__float2half_rn(sum));
+                            else op.out[at] = round_out(sum, op.out_bf16);
                         }
                     }
                     if (lane == 0) p.cnt[1 + w_first] = 0u;  // ready for the next call
@@ -890,6 +953,8 @@ static cudaError_t occupancy_t(size_t smem, int *ctas) {
         case 4 * 16 + 2: return FN<4, 2>(__VA_ARGS__);                 \
         case 8 * 16 + 1: return FN<8, 1>(__VA_ARGS__);                 \
         case 8 * 16 + 2: return FN<8, 2>(__VA_ARGS__);                 \
+        case 16 * 16 + 1: return FN<16, 1>(__VA_ARGS__);               \
+        case 16 * 16 + 2: return FN<16, 2>(__VA_ARGS__);               \
         default: return cudaErrorInvalidValue;                         \
     }
 

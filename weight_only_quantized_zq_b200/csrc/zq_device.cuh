@@ -213,11 +213,12 @@ __host__ __device__ constexpr int pair_lo(int p) {
     return B == 2 ? 16 * (p / 8) + p % 8
          : B == 3 ? p
          : B == 4 ? 8 * (p / 4) + p % 4
-                  : 4 * (p / 2) + p % 2;
+         : B == 8 ? 4 * (p / 2) + p % 2
+                  : 2 * p;  // B = 16 (fp16 weights): word p holds codes 2p, 2p + 1
 }
 template <int B>
 __host__ __device__ constexpr int pair_hi(int p) {
-    return pair_lo<B>(p) + (B == 2 ? 8 : B == 3 ? 16 : B == 4 ? 4 : 2);
+    return pair_lo<B>(p) + (B == 2 ? 8 : B == 3 ? 16 : B == 4 ? 4 : B == 8 ? 2 : 1);
 }
 
 // fp16x2 constants: magic 1024 in both halves; 2^-s; -1024 * 2^-s.
@@ -232,7 +233,7 @@ __host__ __device__ constexpr int pair_shift(int p) {
     return B == 2 ? ((p % 8) < 5 ? 2 * (p % 8) : 2 * (p % 8 - 5))
          : B == 3 ? 3 * (p % 3)
          : B == 4 ? 4 * (p % 2)
-                  : 0;
+                  : 0;  // b = 8, and fp16 weights (no offset, no bias)
 }
 
 // Biased pair: one LOP3 (plus a shift shared by several pairs).
@@ -295,9 +296,12 @@ __device__ __forceinline__ uint32_t unpack_biased_c(const uint32_t (&w)[B], uint
     } else if constexpr (B == 4) {
         const uint32_t u = (P % 4) < 2 ? w[P / 4] : (w[P / 4] >> 8);
         return lop_and_or_imm<((P % 2) == 0 ? 0x000F000Fu : 0x00F000F0u)>(u, magic);
-    } else {
+    } else if constexpr (B == 8) {
         const uint32_t u = (P % 2) == 0 ? w[P / 2] : (w[P / 2] >> 8);
         return lop_and_or_imm<0x00FF00FFu>(u, magic);
+    } else {
+        static_assert(B == 16, "b = 2, 3, 4, 8 or fp16 weights");
+        return w[P];  // fp16 weights: the pair as stored, no bias
     }
 }
 

@@ -47,6 +47,7 @@ struct alignas(64) DecodeOp {
     int row_blocks;         // ceil(N / 64)
     int su;                 // steps per row block: ceil(G / GPS)
     int sz_vec;             // G % GPS == 0: a step's scales/zeros of one row are one aligned vector
+    int out_bf16;           // 1: out holds bfloat16 (bf16 activations), else fp16
 };
 
 struct DecodeParams {
@@ -73,6 +74,7 @@ struct PrepEntry {
     uint16_t *xg;       // x_rows x K, chunk-swizzled per group and token; rows >= M are zeros
     float *sx;          // G x x_rows x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
     int M, x_rows, K, bits;  // x_rows: M with one token tile, else the padded M_pad
+    int x_bf16;              // 1: x holds bfloat16, else fp16
 };
 
 struct PrepParams {
@@ -85,7 +87,7 @@ struct PrepParams {
 
 // Decode tiling.  A CTA step covers 64 weight rows x GPS groups; each of the
 // 4 warps computes 16 of the rows.
-__host__ __device__ constexpr int decode_gps(int bits, int) { return bits == 8 ? 2 : 4; }
+__host__ __device__ constexpr int decode_gps(int bits, int) { return bits == 16 ? 1 : bits == 8 ? 2 : 4; }
 __host__ __device__ constexpr int decode_seg(int bits, int mt) { return decode_gps(bits, mt) * 16 * bits; }
 // Codes of a step land as 128-byte-wide TMA boxes with the 128-byte swizzle
 // when a row segment is a whole number of 128-byte spans.  Otherwise (b = 3:
@@ -107,7 +109,7 @@ __host__ __device__ constexpr int decode_codes_bytes(int bits, int mt) {
 // Token tiles of 8 for the decode kernel (M <= kDecodeMaxM).
 inline int mt_for_m(int M) { return M <= 8 ? 1 : 2; }
 
-cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, uint32_t *packed,
+cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, int group, uint32_t *packed,
                                  uint16_t *scales, uint16_t *zeros, int slot,
                                  unsigned long long call_id, cudaStream_t stream);
 cudaError_t read_quant_status(int slot, unsigned long long *value, cudaStream_t stream);
@@ -121,12 +123,16 @@ constexpr int kMaxPrefillOps = 64;
 
 struct alignas(64) PrefillOp {
     CUtensorMap xmap;  // x (M x K fp16): 64 k x 256 (one-half plan: 128) tokens per box, 128-byte swizzle
+    CUtensorMap wmap;  // fp16 weights only (bits 16): W (N x K fp16), 64 k x 256 rows per box, 128-byte swizzle
     const uint32_t *packed;
     const uint16_t *scales;
     const uint16_t *zeros;
-    uint16_t *out;   // M x N fp16, or null when out32 is set
+    uint16_t *out;   // M x N fp16 (bf16 with out_bf16), or null when out32 is set
     float *out32;    // M x N fp32 (partial sums, not rounded), or null
+    const float *xscale;  // bf16 activations: per-token factor 2^-E of the fp16 copy xmap reads, else null
     int M, N, K;
+    int gshift;     // log2(group) - 5: groups of 32, 64 or 128 codes
+    int out_bf16;   // 1: round the output to bfloat16
     int tok_tiles;  // ceil(M / 256)
     int tile0;      // first tile of this op in the launch
 };
@@ -155,6 +161,11 @@ cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, con
 // tcgen05 tile kernel (which, with one token tile, also streams the weights
 // once, and from 17 tokens on is the faster of the two).
 constexpr int kDecodeMaxM = 16;
+
+// bf16 activations for the tile kernel: each token row of x (M x K bfloat16)
+// scaled by a power of two 2^E (E per row, from the row's largest |x|) and
+// rounded to fp16 into x16; f[m] = 2^-E undoes it in the epilogue.
+cudaError_t launch_bf16_rows_to_f16(const uint16_t *x, int M, int K, uint16_t *x16, float *f, cudaStream_t stream);
 
 // Partial-sum reduction: out[i] = fp16(sum of parts[p][i], p in order).
 constexpr int kMaxReduceParts = 16;

@@ -35,6 +35,7 @@
 //     bytes are in flight per SM; with the codes out of the registers, 16
 //     dequant warps fit, each owning one row chunk per slab.
 #include <cuda.h>
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
@@ -84,14 +85,17 @@ struct Ctl {
 template <int B, bool ONE>
 struct Plan {
     // Dequant warps: 16 in the one-half plan (its code ring keeps their
-    // registers low), 8 in the two-half plan (register prefetch).
-    static constexpr int kDqWarps = ONE ? 16 : 8;
+    // registers low), 8 in the two-half plan (register prefetch); none for
+    // fp16 weights (B = 16), which TMA copies into the W stages as they are.
+    static constexpr int kDqWarps = B == 16 ? 0 : ONE ? 16 : 8;
     static constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
-    static constexpr int kStages = (ONE && B == 8) ? 2 : 3;
+    static constexpr int kStages = B == 16 ? 3 : (ONE && B == 8) ? 2 : 3;
     static constexpr int kSlabA = (ONE ? kPrefillHalfTokens : kTokTile) * kBK * 2;
-    static constexpr int kSlots = !ONE ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
+    static constexpr int kSlots = (!ONE || B == 16) ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
     static constexpr int kSlotCodes = 1024 * (4 * B);  // 256 rows x 2 slabs x 2 chunks of 32 codes
-    static constexpr int kSlotBytes = kSlotCodes + 512 * 4;  // + a (scale | zero << 16) word per (row, chunk)
+    // + a (scale | zero << 16) word per (row, chunk, slab): the two slabs of a
+    // block of 128 codes fall in different groups when groups are 32 or 64
+    static constexpr int kSlotBytes = kSlotCodes + 1024 * 4;
     static constexpr int kOffB = kStages * kSlabA;
     static constexpr int kOffCodes = kOffB + kStages * kSlabB;
     static constexpr int kOffCtl = kOffCodes + kSlots * kSlotBytes;
@@ -99,7 +103,7 @@ struct Plan {
     static_assert(kStages <= kMaxStages, "barrier arrays");
     static_assert(kOffB % 1024 == 0 && kOffCodes % 1024 == 0, "SWIZZLE_128B stages need 1024-byte alignment");
     static_assert(kBytes <= 232448, "227 KB of shared memory per CTA");
-    static_assert(!ONE || kSlots >= 3, "the scale/zero hand-off needs a prefetch distance of 2 groups");
+    static_assert(!ONE || B == 16 || kSlots >= 3, "the scale/zero hand-off needs a prefetch distance of 2 groups");
 };
 
 // Bounded wait: false if the CTA is aborting or the limit was reached.
@@ -185,6 +189,15 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
+}
+
+// Two outputs rounded (nearest even) to fp16, or to bfloat16 for bf16 activations.
+__device__ __forceinline__ uint32_t pack_out2(float lo, float hi, int bf16) {
+    if (bf16) {
+        const __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+        return *reinterpret_cast<const uint32_t *>(&b);
+    }
+    return pack_half2(lo, hi);
 }
 
 // Tile t of a launch -> (op, weight-row tile, token tile).  The tiles of op o
@@ -309,8 +322,8 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         rows[r] = (q % 256) / 2 + 128 * (q / 256);
     }
 
-    // Issue cursor: the group whose codes are copied next.
-    int tp = blockIdx.x, gp = 0, Gp = 0;
+    // Issue cursor: the block of 128 codes whose codes are copied next.
+    int tp = blockIdx.x, gp = 0, Gp = 0, gsh = 2;
     const uint32_t *prow[RPT];
     const uint16_t *psr[RPT], *pzr[RPT];
     auto start_issue = [&]() {
@@ -318,29 +331,35 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
             const TileRef tr = locate(p, tp);
             const PrefillOp &op = p.ops[tr.o];
             Gp = op.K / kGroup;
+            gsh = op.gshift;
+            const size_t gs = static_cast<size_t>(op.K) >> (op.gshift + 5);  // scales per row
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const int n = min(tr.n0 + rows[r], op.N - 1);
                 prow[r] = op.packed + static_cast<size_t>(n) * (static_cast<size_t>(op.K) * B / 32);
-                psr[r] = op.scales + static_cast<size_t>(n) * Gp;
-                pzr[r] = op.zeros + static_cast<size_t>(n) * Gp;
+                psr[r] = op.scales + static_cast<size_t>(n) * gs;
+                pzr[r] = op.zeros + static_cast<size_t>(n) * gs;
             }
         }
     };
     start_issue();
-    uint32_t szA[RPT], szB[RPT];
+    uint32_t szA[RPT][2], szB[RPT][2];
 #pragma unroll
-    for (int r = 0; r < RPT; ++r) szA[r] = szB[r] = 0u;
-    // Group j of this CTA's sequence: first store the scale/zero words of
-    // group j - 2 (held in `set`) into its slot, then copy group j's codes into
-    // slot j % kS and load its scales and zeros into `set`.  Past the last
-    // group only the store and an empty commit remain, so that every group
-    // index commits exactly one cp.async group.
-    auto issue = [&](int j, uint32_t (&set)[RPT]) {
+    for (int r = 0; r < RPT; ++r) szA[r][0] = szA[r][1] = szB[r][0] = szB[r][1] = 0u;
+    // Block j of this CTA's sequence: first store the scale/zero words of
+    // block j - 2 (held in `set`) into its slot, then copy block j's codes into
+    // slot j % kS and load its scales and zeros into `set`: slab h of the
+    // block uses group (4 * gp + 2h + ch) >> gshift.  Past the last block only
+    // the store and an empty commit remain, so that every block index commits
+    // exactly one cp.async group.
+    auto issue = [&](int j, uint32_t (&set)[RPT][2]) {
         if (j >= 2) {
             uint32_t *zs = reinterpret_cast<uint32_t *>(scode + ((j - 2) % kS) * P::kSlotBytes + P::kSlotCodes);
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) zs[r * NT + d] = set[r];
+            for (int r = 0; r < RPT; ++r) {
+                zs[(2 * r) * NT + d] = set[r][0];
+                zs[(2 * r + 1) * NT + d] = set[r][1];
+            }
         }
         if (tp < n_tiles) {
             uint8_t *cs = scode + (j % kS) * P::kSlotBytes;
@@ -353,8 +372,12 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                     for (int u = 0; u < UPC; ++u)
                         cp_async_u<U>(cs + (((h * RPT + r) * UPC + u) * NT + d) * U, src + u * U);
                 }
+            const int g0 = (4 * gp + ch) >> gsh, g1 = (4 * gp + 2 + ch) >> gsh;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) set[r] = ldg_u16_nc(psr[r] + gp) | (ldg_u16_nc(pzr[r] + gp) << 16);
+            for (int r = 0; r < RPT; ++r) {
+                set[r][0] = ldg_u16_nc(psr[r] + g0) | (ldg_u16_nc(pzr[r] + g0) << 16);
+                set[r][1] = g1 == g0 ? set[r][0] : ldg_u16_nc(psr[r] + g1) | (ldg_u16_nc(pzr[r] + g1) << 16);
+            }
             if (++gp == Gp) {
                 gp = 0;
                 tp += gridDim.x;
@@ -377,13 +400,15 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         cp_async_wait<PD>();               // this thread's copies of group i have landed
         const uint32_t z = opaque_zero();  // orders the slot loads after the wait
         const uint32_t cs = smem_u32(scode + (i % kS) * P::kSlotBytes) + z;
-        uint32_t sz[RPT];
-        bool ovf[RPT];
+        uint32_t sz[RPT][2];
+        bool ovf[RPT][2];
 #pragma unroll
-        for (int r = 0; r < RPT; ++r) {
-            sz[r] = lds_u32(cs + P::kSlotCodes + 4 * (r * NT + d));
-            ovf[r] = dequant_overflows<B>(sz[r]);
-        }
+        for (int r = 0; r < RPT; ++r)
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                sz[r][h] = lds_u32(cs + P::kSlotCodes + 4 * ((2 * r + h) * NT + d));
+                ovf[r][h] = dequant_overflows<B>(sz[r][h]);
+            }
 #pragma unroll
         for (int h = 0; h < 2; ++h) {  // the two slabs of this group
             const int st = it % P::kStages;
@@ -408,7 +433,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                 }
                 const int row = rows[r];
                 uint32_t o[16];
-                dequant_chunk<B>(w, sz[r], o, ovf[r]);
+                dequant_chunk<B>(w, sz[r][h], o, ovf[r][h]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c16 = (4 * ch + j) ^ (row & 7);
@@ -428,8 +453,8 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         }
         return true;
     };
-    uint32_t (&set_even)[RPT] = (PD & 1) ? szB : szA;  // register set of group i + PD, i even
-    uint32_t (&set_odd)[RPT] = (PD & 1) ? szA : szB;
+    uint32_t (&set_even)[RPT][2] = (PD & 1) ? szB : szA;  // register set of block i + PD, i even
+    uint32_t (&set_odd)[RPT][2] = (PD & 1) ? szA : szB;
 #pragma unroll 1
     for (int i = 0;; i += 2) {
         if (t >= n_tiles || *abort) break;
@@ -458,7 +483,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < P::kStages; ++s) {
-            mbar_init(&sm.full[s], P::kDqWarps);
+            if constexpr (B != 16) mbar_init(&sm.full[s], P::kDqWarps);
             mbar_init(&sm.xfull[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
@@ -493,7 +518,14 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                     const int st = it % P::kStages;
                     const uint32_t round = it / P::kStages;
                     if (!mbar_wait(&sm.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) break;
-                    mbar_arrive_expect_tx(&sm.xfull[st], P::kSlabA);
+                    if constexpr (B == 16) {
+                        // fp16 weights: the W slab is copied as it is, in the same
+                        // 128-byte swizzled K-major layout the dequant warps write
+                        mbar_arrive_expect_tx(&sm.xfull[st], P::kSlabA + kSlabB);
+                        tma_load_2d(sb + st * kSlabB, &op.wmap, s * kBK, tr.n0, &sm.xfull[st]);
+                    } else {
+                        mbar_arrive_expect_tx(&sm.xfull[st], P::kSlabA);
+                    }
                     tma_load_2d(sa + st * P::kSlabA, &op.xmap, s * kBK, tr.t0, &sm.xfull[st]);
                 }
             }
@@ -522,7 +554,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                 for (int s = 0; s < slabs; ++s, ++it) {
                     const int st = it % P::kStages;
                     if (!mbar_wait(&sm.xfull[st], (it / P::kStages) & 1u, abort, p.wait_ns) ||
-                        !mbar_wait(&sm.full[st], (it / P::kStages) & 1u, abort, p.wait_ns)) {
+                        (B != 16 && !mbar_wait(&sm.full[st], (it / P::kStages) & 1u, abort, p.wait_ns))) {
                         ok = false;
                         break;
                     }
@@ -558,7 +590,9 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
             }
         }
     } else if (warp >= kDqWarp0) {
-        if constexpr (ONE) {
+        if constexpr (B == 16) {
+            // no dequant warps for fp16 weights
+        } else if constexpr (ONE) {
             dequant_ring<B>(p, sb, scode, sm, threadIdx.x - 32 * kDqWarp0, lane);
         } else {
         // 256 threads: thread d owns rows d/2 and d/2 + 128 of the tile and the
@@ -567,30 +601,36 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         const int d = threadIdx.x - 32 * kDqWarp0;
         const int ch = d & 1;
         uint32_t it = 0;
-        uint32_t wn[2][2][B], szn[2];  // [slab of group][row][word]
+        uint32_t wn[2][2][B], szn[2][2];  // [slab of block][row][word], [slab][row]
         // Row pointers of the tile being fetched (set when it starts).
         const uint32_t *rowp[2];
         const uint16_t *srow[2], *zrow[2];
-        auto start_tile = [&](int t) -> int {  // returns the tile's group count
+        int gsh = 2;                      // log2(group) - 5 of the tile being fetched
+        auto start_tile = [&](int t) -> int {  // returns the tile's count of 128-code blocks
             const TileRef tr = locate(p, t);
             const PrefillOp &op = p.ops[tr.o];
             const int G = op.K / kGroup;
+            gsh = op.gshift;
+            const size_t gs = static_cast<size_t>(op.K) >> (op.gshift + 5);  // scales per row
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
                 const int r = min(tr.n0 + d / 2 + 128 * i, op.N - 1);
                 rowp[i] = op.packed + static_cast<size_t>(r) * (static_cast<size_t>(op.K) * B / 32);
-                srow[i] = op.scales + static_cast<size_t>(r) * G;
-                zrow[i] = op.zeros + static_cast<size_t>(r) * G;
+                srow[i] = op.scales + static_cast<size_t>(r) * gs;
+                zrow[i] = op.zeros + static_cast<size_t>(r) * gs;
             }
             return G;
         };
         auto fetch = [&](int g) {
+            // slab h of block g: codes 128g + 64h + 32ch .. +31, group (4g + 2h + ch) >> gsh
+            const int g0 = (4 * g + ch) >> gsh, g1 = (4 * g + 2 + ch) >> gsh;
 #pragma unroll
             for (int i = 0; i < 2; ++i) {
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     load_chunk<B>(wn[h][i], rowp[i] + static_cast<size_t>(4 * g + 2 * h + ch) * B);
-                szn[i] = ldg_u16_nc(srow[i] + g) | (ldg_u16_nc(zrow[i] + g) << 16);
+                szn[0][i] = ldg_u16_nc(srow[i] + g0) | (ldg_u16_nc(zrow[i] + g0) << 16);
+                szn[1][i] = g1 == g0 ? szn[0][i] : ldg_u16_nc(srow[i] + g1) | (ldg_u16_nc(zrow[i] + g1) << 16);
             }
         };
         int t = blockIdx.x, g = 0, groups = 0, groups_n = 0;
@@ -600,16 +640,21 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         }
         bool ok = true;
         while (t < n_tiles && ok && !*abort) {
-            uint32_t wc[2][2][B], szc[2];
+            uint32_t wc[2][2][B], szc[2][2];
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
                 for (int i = 0; i < 2; ++i)
 #pragma unroll
                     for (int q = 0; q < B; ++q) wc[h][i][q] = wn[h][i][q];
-            szc[0] = szn[0];
-            szc[1] = szn[1];
-            const bool ovf[2] = {dequant_overflows<B>(szc[0]), dequant_overflows<B>(szc[1])};
+            bool ovf[2][2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    szc[h][i] = szn[h][i];
+                    ovf[h][i] = dequant_overflows<B>(szc[h][i]);
+                }
             int t_n = t, g_n = g + 1;
             groups_n = groups;
             if (g_n == groups) {
@@ -631,7 +676,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                 for (int i = 0; i < 2; ++i) {
                     const int row = d / 2 + 128 * i;
                     uint32_t o[16];
-                    dequant_chunk<B>(wc[h][i], szc[i], o, ovf[i]);
+                    dequant_chunk<B>(wc[h][i], szc[h][i], o, ovf[h][i]);
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
                         const int c16 = (4 * ch + j) ^ (row & 7);
@@ -662,10 +707,17 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
 #pragma unroll 1
             for (int half = 0; half < (t0 + 128 < op.M ? 2 : 1); ++half) {
                 const int tok = t0 + 128 * half + 32 * warp + lane;
+                // bf16 activations: the token's power-of-two factor undoes the
+                // scaling of the fp16 copy the MMAs read
+                const float fs = (op.xscale != nullptr && tok < op.M) ? op.xscale[tok] : 1.0f;
 #pragma unroll 1
                 for (int cc = 0; cc < kRowTile / 32; ++cc) {
                     uint32_t r[32];
                     tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile + cc * 32, r);
+                    if (op.xscale != nullptr) {
+#pragma unroll
+                        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * fs);
+                    }
                     const int col0 = n0 + cc * 32;
                     if (tok < op.M && col0 < op.N && op.out32) {
                         // fp32 partial sums (a K-split shard), not rounded
@@ -686,14 +738,15 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
 #pragma unroll
                             for (int q = 0; q < 4; ++q)
                                 reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                                    pack_half2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1])),
-                                    pack_half2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3])),
-                                    pack_half2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5])),
-                                    pack_half2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7])));
+                                    pack_out2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]), op.out_bf16),
+                                    pack_out2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]), op.out_bf16),
+                                    pack_out2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]), op.out_bf16),
+                                    pack_out2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]), op.out_bf16));
                         } else {
 #pragma unroll
                             for (int q = 0; q < 32; ++q)
-                                if (col0 + q < op.N) dst[q] = __half_as_ushort(__float2half_rn(__uint_as_float(r[q])));
+                                if (col0 + q < op.N)
+                                    dst[q] = static_cast<uint16_t>(pack_out2(__uint_as_float(r[q]), 0.0f, op.out_bf16));
                         }
                     }
                 }
@@ -763,15 +816,23 @@ cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, 
             case 2: return launch_prefill_t<2, true>(pg, n_ctas, stream);
             case 3: return launch_prefill_t<3, true>(pg, n_ctas, stream);
             case 4: return launch_prefill_t<4, true>(pg, n_ctas, stream);
-            default: return launch_prefill_t<8, true>(pg, n_ctas, stream);
+            case 8: return launch_prefill_t<8, true>(pg, n_ctas, stream);
+            default: return launch_prefill_t<16, true>(pg, n_ctas, stream);
         }
     }
     switch (bits) {
         case 2: return launch_prefill_t<2, false>(pg, n_ctas, stream);
         case 3: return launch_prefill_t<3, false>(pg, n_ctas, stream);
         case 4: return launch_prefill_t<4, false>(pg, n_ctas, stream);
-        default: return launch_prefill_t<8, false>(pg, n_ctas, stream);
+        case 8: return launch_prefill_t<8, false>(pg, n_ctas, stream);
+        default: return launch_prefill_t<16, false>(pg, n_ctas, stream);
     }
+}
+
+cudaError_t prefill_w_map(CUtensorMap *map, const uint16_t *w, int N, int K) {
+    return encode_tensor_map_2d(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w, static_cast<uint64_t>(K),
+                                static_cast<uint64_t>(N), static_cast<uint64_t>(K) * 2, pf::kBK,
+                                static_cast<uint32_t>(pf::kRowTile), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 cudaError_t read_prefill_error(int *err) {

@@ -17,6 +17,10 @@ constexpr int kPrefillHalfTokens = 128;
 // Tensor map of x (M x K fp16) with boxes of 64 k x box_rows tokens, 128-byte swizzle.
 cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K, int box_rows);
 
+// Tensor map of fp16 weights W (N x K) with boxes of 64 k x 256 rows, 128-byte
+// swizzle: the W slab of the tile kernel for bits = 16.
+cudaError_t prefill_w_map(CUtensorMap *map, const uint16_t *w, int N, int K);
+
 // Token rows per x box of a launch: 128 if every op has M <= 128, else 256.
 // Reads only the ops' M, so it may be called before their maps are built.
 int prefill_box_rows(const PrefillGroup &pg);

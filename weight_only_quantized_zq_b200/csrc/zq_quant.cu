@@ -31,15 +31,16 @@ namespace zq {
 // by a unique call id, so no clearing is needed between calls.
 __device__ unsigned long long g_quant_status[kQuantStatusSlots];
 
-// One warp per (row, group).  Each lane owns 4 consecutive weights.
+// One warp per (row, block of 128 weights: 1, 2 or 4 groups).  Each lane owns
+// 4 consecutive weights.
 template <bool SYMMETRIC>
 __global__ void __launch_bounds__(256) quantize_pack_kernel(
-    const float *__restrict__ w, int N, int K, int bits, uint32_t *__restrict__ packed,
+    const float *__restrict__ w, int N, int K, int bits, int group, uint32_t *__restrict__ packed,
     uint16_t *__restrict__ scales, uint16_t *__restrict__ zeros, int slot,
     unsigned long long call_id) {
     __shared__ uint32_t words[8][32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = K / 128;
+    const int G = K / 128;  // blocks per row
     const long long item = static_cast<long long>(blockIdx.x) * 8 + warp;
     if (item >= static_cast<long long>(N) * G) return;
     const int n = static_cast<int>(item / G), g = static_cast<int>(item % G);
@@ -48,16 +49,19 @@ __global__ void __launch_bounds__(256) quantize_pack_kernel(
                                                         static_cast<size_t>(g) * 128 + lane * 4);
     const float v[4] = {v4.x, v4.y, v4.z, v4.w};
     uint16_t s16, z16;
-    if (!quantize_group_warp<SYMMETRIC>(v, bits, lane, words[warp], s16, z16)) {
+    if (!quantize_group_warp<SYMMETRIC>(v, bits, lane, words[warp], s16, z16, group)) {
         if (lane == 0) atomicExch(&g_quant_status[slot], call_id);
         return;
     }
     const int nw = 4 * bits;
     const size_t wpr = static_cast<size_t>(K) * bits / 32;
     if (lane < nw) packed[static_cast<size_t>(n) * wpr + static_cast<size_t>(g) * nw + lane] = words[warp][lane];
-    if (lane == 0) {
-        scales[static_cast<size_t>(n) * G + g] = s16;
-        zeros[static_cast<size_t>(n) * G + g] = z16;
+    const int lpg = group >> 2;  // lanes per group; the first lane of each writes its scale and zero
+    if ((lane & (lpg - 1)) == 0) {
+        const int per = 128 / group;
+        const size_t at = static_cast<size_t>(n) * (K / group) + static_cast<size_t>(g) * per + lane / lpg;
+        scales[at] = s16;
+        zeros[at] = z16;
     }
 }
 
@@ -85,22 +89,22 @@ __global__ void unpack_kernel(const uint32_t *__restrict__ packed, int N, int K,
     }
 }
 
-cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, uint32_t *packed,
+cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, int group, uint32_t *packed,
                                  uint16_t *scales, uint16_t *zeros, int slot,
                                  unsigned long long call_id, cudaStream_t stream) {
     const long long items = static_cast<long long>(N) * (K / 128);
     const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
-    quantize_pack_kernel<false><<<blocks, 256, 0, stream>>>(w, N, K, bits, packed, scales, zeros, slot,
+    quantize_pack_kernel<false><<<blocks, 256, 0, stream>>>(w, N, K, bits, group, packed, scales, zeros, slot,
                                                             call_id);
     return cudaGetLastError();
 }
 
-cudaError_t launch_quantize_pack_symmetric(const float *w, int N, int K, int bits, uint32_t *packed,
+cudaError_t launch_quantize_pack_symmetric(const float *w, int N, int K, int bits, int group, uint32_t *packed,
                                            uint16_t *scales, uint16_t *zeros, int slot,
                                            unsigned long long call_id, cudaStream_t stream) {
     const long long items = static_cast<long long>(N) * (K / 128);
     const unsigned blocks = static_cast<unsigned>((items + 7) / 8);
-    quantize_pack_kernel<true><<<blocks, 256, 0, stream>>>(w, N, K, bits, packed, scales, zeros, slot,
+    quantize_pack_kernel<true><<<blocks, 256, 0, stream>>>(w, N, K, bits, group, packed, scales, zeros, slot,
                                                            call_id);
     return cudaGetLastError();
 }

@@ -12,7 +12,7 @@ namespace zq {
 // with zero = -2^(bits-1) * scale.  Same launch shape and status slot protocol
 // as launch_quantize_pack; a group whose zero is not a finite fp16 also sets
 // the status slot.
-cudaError_t launch_quantize_pack_symmetric(const float *w, int N, int K, int bits, uint32_t *packed,
+cudaError_t launch_quantize_pack_symmetric(const float *w, int N, int K, int bits, int group, uint32_t *packed,
                                            uint16_t *scales, uint16_t *zeros, int slot,
                                            unsigned long long call_id, cudaStream_t stream);
 

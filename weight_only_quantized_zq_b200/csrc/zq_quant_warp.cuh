@@ -1,5 +1,6 @@
-// zq_quant_warp.cuh — one warp quantizes one group of 128 weights (shared by
-// quantize-and-pack and the KV-cache store).
+// zq_quant_warp.cuh — one warp quantizes one block of 128 weights: one group
+// of 128, or 2 groups of 64, or 4 of 32 (shared by quantize-and-pack and the
+// KV-cache store).
 //
 // Asymmetric ([wiki] "ZSE - open-source движок для запуска LLM локально на GPU -
 // 2026", section "Формат модели .zse", with L = 2^b - 1): zero = fp16(min),
@@ -20,15 +21,17 @@ __device__ __forceinline__ uint16_t f64_to_f16_bits(double v) {
     return __half_as_ushort(__double2half(v));
 }
 
-// Lane l holds weights 4l .. 4l+3 of the group in v.  On success the group's
-// 4*bits packed words (little-endian bitstream, code k at bits [k*b, k*b+b))
-// are in words[0 .. 4*bits) (this warp's shared-memory scratch) and every
-// lane holds the fp16 bits of the scale and zero.  Returns false, in every
-// lane, if a weight is NaN, infinite or above 65504 in magnitude, or (symmetric)
-// the zero would not be a finite fp16; then nothing is written.
+// Lane l holds weights 4l .. 4l+3 of the block in v; a group is `group`
+// consecutive weights (32, 64 or 128), i.e. the group/4 lanes starting at a
+// multiple of group/4.  On success the block's 4*bits packed words
+// (little-endian bitstream, code k at bits [k*b, k*b+b); groups never straddle
+// words) are in words[0 .. 4*bits) (this warp's shared-memory scratch) and every
+// lane holds the fp16 bits of its group's scale and zero.  Returns false, in
+// every lane, if a weight is NaN, infinite or above 65504 in magnitude, or
+// (symmetric) a zero would not be a finite fp16; then nothing is written.
 template <bool SYMMETRIC>
 __device__ __forceinline__ bool quantize_group_warp(const float (&v)[4], int bits, int lane, uint32_t *words,
-                                                    uint16_t &s16, uint16_t &z16) {
+                                                    uint16_t &s16, uint16_t &z16, int group = 128) {
     const int L = (1 << bits) - 1;
     bool bad = false;
     float mn = v[0], mx = v[0];
@@ -39,10 +42,14 @@ __device__ __forceinline__ bool quantize_group_warp(const float (&v)[4], int bit
         mx = fmaxf(mx, v[i]);
     }
     if (__any_sync(0xffffffffu, bad)) return false;
+    const int lanes_per_group = group >> 2;  // 8, 16 or 32: the xor steps below stay inside a group
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        const float omn = __shfl_xor_sync(0xffffffffu, mn, o), omx = __shfl_xor_sync(0xffffffffu, mx, o);
+        if (o < lanes_per_group) {
+            mn = fminf(mn, omn);
+            mx = fmaxf(mx, omx);
+        }
     }
     uint32_t chunk = 0;  // this lane's 4 codes, 4*bits bits
     if constexpr (SYMMETRIC) {
@@ -50,7 +57,7 @@ __device__ __forceinline__ bool quantize_group_warp(const float (&v)[4], int bit
         s16 = f64_to_f16_bits(__ddiv_rn(static_cast<double>(fmaxf(-mn, mx)), Q));
         const double s = static_cast<double>(__half2float(__ushort_as_half(s16)));
         const double z = __dmul_rn(-half, s);
-        if (z < -65504.0) return false;  // the zero would not be a finite fp16 (uniform across the warp)
+        if (__any_sync(0xffffffffu, z < -65504.0)) return false;  // a zero would not be a finite fp16
         z16 = f64_to_f16_bits(z);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
