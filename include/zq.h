@@ -224,6 +224,15 @@ ZQ_API size_t zq_linear_stack_bf16_workspace_bytes(const zq_linear_desc *ops, in
 ZQ_API zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits,
                     uint8_t *codes, zq_stream_t stream);
 
+/* Test hook: the tile kernel's dequantization ([wiki] "Формат модели .zse":
+ * w_hat = q * scale + zero) over a whole tensor, with the same device routine
+ * the tcgen05 kernel uses before its MMAs: w_hat (device, fp16 N x K, written)
+ * = fp16(q * s + z) rounded once to nearest even, or 65504 where that rounds
+ * to +infinity (groups reaching the top of the fp16 range).  Formats and
+ * errors as zq_linear.  Asynchronous. */
+ZQ_API zq_status zq_dequant(const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros, int bits,
+                            int group, int N, int K, uint16_t *w_hat, zq_stream_t stream);
+
 /* Workspace (see Conventions).  The pages describe no counterpart: these are
  * services of the library, not part of the method.
  *

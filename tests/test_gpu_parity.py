@@ -158,6 +158,35 @@ def test_unpack_bit_exact(zq, orc, bits):
         assert np.array_equal(out.cpu().numpy(), orc.unpack(packed_np, N, K, bits))
 
 
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("group", (32, 64, 128))
+def test_dequant_bit_exact(zq, orc, bits, group):
+    """The tile kernel's dequantization (zq_dequant runs its routine) gives
+    fp16_rne(q * s16 + z16) of the oracle's exact w_hat, bit for bit; where that
+    rounds past the fp16 range the kernel holds 65504."""
+    N, K = 40, 1024
+    w = zi.weight(N, K, seed=9990 + bits + group, outliers=True)
+    w[3] = torch.linspace(-65504.0, 65504.0, group).repeat(K // group)  # top codes round past 65504
+    w[4] = 0.0123                                  # scale 0
+    w[5] = torch.linspace(0, 1e-6, K)              # subnormal scales
+    w[6] = w[6] * 1e3 - 3e3                        # large zero, small scale
+    wd = w.contiguous().cuda()
+    packed, scales, zeros = zq.quantize(wd, bits, group=group)
+    out = torch.empty(N, K, dtype=torch.float16, device="cuda")
+    zq.zq_dequant(packed, scales, zeros, bits, group, N, K, out)
+    torch.cuda.synchronize()
+    p_ref, s_ref, z_ref = orc.quantize_pack(w.numpy(), bits, group=group)
+    exact = orc.dequant(p_ref, s_ref, z_ref, bits, N, K, group=group)
+    with np.errstate(over="ignore"):
+        h = exact.astype(np.float16)  # numpy's round-to-nearest-even, pinned against the oracle's encoder
+    want = h.view(np.uint16).copy()
+    want[np.isinf(h)] = 0x7BFF  # held at the largest finite fp16
+    got = u16(out)
+    bad = got != want
+    assert not bad.any(), (int(bad.sum()), np.argwhere(bad)[:5], got[bad][:5], want[bad][:5])
+    assert (want == 0x7BFF).any()  # the overflow case occurs
+
+
 # ---------------------------------------------------------------- linear --
 
 @pytest.mark.parametrize("bits", BITS)

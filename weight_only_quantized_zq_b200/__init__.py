@@ -36,7 +36,7 @@ EXPORTS = ("zq_packed_words", "zq_quantize_pack", "zq_quantize_pack_symmetric", 
            "zq_kv_plane_bytes", "zq_kv_append", "zq_kv_gather",
            "zq_linear_partial", "zq_linear_partial_stack", "zq_linear_partial_stack_workspace_bytes",
            "zq_reduce_partials", "zq_linear_bf16", "zq_linear_bf16_workspace_bytes", "zq_linear_stack_bf16",
-           "zq_linear_stack_bf16_workspace_bytes")
+           "zq_linear_stack_bf16_workspace_bytes", "zq_dequant")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing; build it with "
@@ -61,6 +61,8 @@ _lib.zq_linear_stack.argtypes = [_P, _I, _P]
 _lib.zq_linear_stack.restype = _I
 _lib.zq_unpack.argtypes = [_P, _I, _I, _I, _P, _P]
 _lib.zq_unpack.restype = _I
+_lib.zq_dequant.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _P]
+_lib.zq_dequant.restype = _I
 _lib.zq_reserve_workspace.argtypes = [_S, _P]
 _lib.zq_reserve_workspace.restype = _I
 _lib.zq_attach_workspace.argtypes = [_P, _S, _P]
@@ -347,6 +349,11 @@ def zq_linear_stack_bf16_workspace_bytes(ops, n_ops=None):
         ops, n = make_descs(ops)
         n_ops = n if n_ops is None else n_ops
     return _lib.zq_linear_stack_bf16_workspace_bytes(ops, n_ops)
+
+
+def zq_dequant(packed, scales, zeros, bits, group, N, K, w_hat, stream=None):
+    _check(_lib.zq_dequant(_ptr(packed), _ptr(scales), _ptr(zeros), bits, group, N, K, _ptr(w_hat),
+                           _stream(stream, packed)))
 
 
 def zq_unpack(packed, N, K, bits, codes, stream=None):

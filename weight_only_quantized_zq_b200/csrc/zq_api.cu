@@ -326,7 +326,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         n_chunks = (total_steps + (1LL << log2c) - 1) >> log2c;
         n_ctas = static_cast<int>(n_chunks);
     }
-    if (!units && static_cast<size_t>(n_chunks) + 1 > kMaxCounters)
+    if (!units && static_cast<size_t>(n_chunks) + 1 > kMaxCounters - 2)  // the last 2 are the tile kernel's
         return fail(ZQ_ERR_INVALID_ARG, "internal: too many chunks");
     const int slot_floats = rows * mpad;
 
@@ -490,12 +490,12 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
     std::stable_sort(ops.begin(), ops.end(), [](const Op &a, const Op &b) { return a.K > b.K; });
+    uint8_t *ws = nullptr;
+    if ((st = workspace(stream, prefill_data_bytes(ops), &ws)) != ZQ_OK) return st;
     // bf16 activations: an fp16 copy per distinct x, scaled per token, in the
     // workspace (see zq_act.cu); the launch reads the copy.
     std::vector<std::pair<const uint16_t *, std::pair<uint16_t *, float *>>> conv;
-    if (const size_t need = prefill_data_bytes(ops)) {
-        uint8_t *ws = nullptr;
-        if ((st = workspace(stream, need, &ws)) != ZQ_OK) return st;
+    if (prefill_data_bytes(ops) > 0) {
         uint8_t *at = ws + kCounterBytes;
         for (const auto &d : ops) {
             if (!d.xbf16) continue;
@@ -549,6 +549,7 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     }
     pg.n_tiles = tiles;
     pg.wait_ns = g_wait_ns.load();
+    pg.tile_ctr = reinterpret_cast<unsigned int *>(ws) + (kMaxCounters - 2);
     cudaError_t e = launch_prefill_group(pg, ops[0].bits, info->sms, stream);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     g_launches += 1;
@@ -923,6 +924,21 @@ zq_status zq_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *cod
     return ZQ_OK;
 }
 
+zq_status zq_dequant(const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros, int bits, int group,
+                     int N, int K, uint16_t *w_hat, zq_stream_t stream) {
+    zq_status st = check_format(bits, group, N, K);
+    if (st != ZQ_OK) return st;
+    if ((st = check_ptr(packed, "packed")) != ZQ_OK) return st;
+    if ((st = check_ptr(scales, "scales")) != ZQ_OK) return st;
+    if ((st = check_ptr(zeros, "zeros")) != ZQ_OK) return st;
+    if ((st = check_ptr(w_hat, "w_hat")) != ZQ_OK) return st;
+    cudaError_t e = launch_dequant_test(packed, scales, zeros, bits, group, N, K, w_hat,
+                                        reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "dequant launch");
+    ++g_launches;
+    return ZQ_OK;
+}
+
 zq_status zq_reserve_workspace(size_t bytes, zq_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     std::pair<int, unsigned long long> key;
@@ -1076,8 +1092,8 @@ zq_status zq_check_device(void) {
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
     e = read_kv_error(&err3);
     if (e != cudaSuccess) return cuda_fail(e, "reading the device status word");
-    if (err2 != 0) {
-        // A decode kernel that gave up may have left split-K counters set.
+    if (err != 0 || err2 != 0) {
+        // A kernel that gave up may have left split-K or tile counters set.
         int dev = 0;
         if (cudaGetDevice(&dev) == cudaSuccess) workspaces_dirty(dev);
     }

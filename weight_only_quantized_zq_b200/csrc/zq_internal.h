@@ -115,10 +115,15 @@ cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, int gro
 cudaError_t read_quant_status(int slot, unsigned long long *value, cudaStream_t stream);
 cudaError_t launch_unpack(const uint32_t *packed, int N, int K, int bits, uint8_t *codes,
                           cudaStream_t stream);
+// The tile kernel's dequant routine over a whole tensor (test hook): w_hat fp16 N x K.
+cudaError_t launch_dequant_test(const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros, int bits,
+                                int group, int N, int K, uint16_t *w_hat, cudaStream_t stream);
 
 // ---------------------------------------------------------------- prefill --
 // A prefill launch runs up to kMaxPrefillOps independent ops of one bit width
-// as one persistent grid over all their 256-token x 256-row output tiles.
+// as one persistent grid over all their 256-token x 256-row output tiles,
+// handed out dynamically from a counter (the last two words of the
+// workspace's counter region).
 constexpr int kMaxPrefillOps = 64;
 
 struct alignas(64) PrefillOp {
@@ -141,6 +146,7 @@ struct PrefillGroup {
     int n_ops;
     int n_tiles;
     unsigned long long wait_ns;  // limit of a bounded wait (see wait_limit_ns)
+    unsigned int *tile_ctr;      // workspace: [0] next tile ticket, [1] CTAs finished; both 0 between launches
     PrefillOp ops[kMaxPrefillOps];
 };
 static_assert(sizeof(PrefillGroup) <= 32000, "kernel parameter space");

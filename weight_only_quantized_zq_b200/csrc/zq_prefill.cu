@@ -64,7 +64,19 @@ constexpr int kTmemCols = 512;
 // the abort flag and the adjustable limit and give up only after this bound.
 constexpr unsigned long long kDrainNs = 2000000000ull;  // 2 s
 
+// Tiles are handed out dynamically: the scheduler warp takes tickets from a
+// counter in the workspace and writes the tile numbers, in order, into a ring
+// of kTileRing entries; every role reads the ring in the same order and
+// releases an entry as soon as it has read it.  The ring is deeper than the
+// furthest any reader runs ahead of another (the dequant issue cursor, a few
+// blocks ahead of its consume cursor, which leads the epilogue by a few
+// slabs), so no reader waits on the scheduler for long.
+constexpr int kTileRing = 16;
+
 struct Ctl {
+    int tq[kTileRing];                     // tile numbers, -1 = no more tiles
+    unsigned long long tq_full[kTileRing];
+    unsigned long long tq_empty[kTileRing];
     unsigned long long full[kMaxStages];   // W slab dequantized (one arrival per dequant warp)
     unsigned long long xfull[kMaxStages];  // x slab landed (the TMA warp's expect_tx + the copy's bytes)
     unsigned long long empty[kMaxStages];
@@ -88,7 +100,10 @@ struct Plan {
     // registers low), 8 in the two-half plan (register prefetch); none for
     // fp16 weights (B = 16), which TMA copies into the W stages as they are.
     static constexpr int kDqWarps = B == 16 ? 0 : ONE ? 16 : 8;
-    static constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
+    static constexpr int kSchedWarp = kDqWarp0 + kDqWarps;  // the tile scheduler (lane 0)
+    static constexpr int kThreads = 32 * (kSchedWarp + 1);
+    // readers of every tile-ring entry: TMA and MMA lanes, epilogue and dequant warps
+    static constexpr int kTileReaders = 2 + kEpiWarps + kDqWarps;
     static constexpr int kStages = B == 16 ? 3 : (ONE && B == 8) ? 2 : 3;
     static constexpr int kSlabA = (ONE ? kPrefillHalfTokens : kTokTile) * kBK * 2;
     static constexpr int kSlots = (!ONE || B == 16) ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
@@ -131,6 +146,15 @@ __device__ __noinline__ void mbar_drain(unsigned long long *bar, uint32_t parity
     while (!mbar_try_wait(bar, parity))
         if (globaltimer() - t0 > kDrainNs) break;
 }
+
+// Tile number of ring entry j (whole warp or one lane): -1 when the tiles are
+// exhausted, -2 when the wait gave up (the CTA is aborting).
+__device__ __forceinline__ int tile_at(Ctl &c, uint32_t j, volatile int *abort, unsigned long long limit) {
+    if (!mbar_wait(&c.tq_full[j % kTileRing], (j / kTileRing) & 1u, abort, limit)) return -2;
+    return *reinterpret_cast<volatile int *>(&c.tq[j % kTileRing]);
+}
+
+__device__ __forceinline__ void tile_release(Ctl &c, uint32_t j) { mbar_arrive(&c.tq_empty[j % kTileRing]); }
 
 __device__ __forceinline__ void tc_fence_before() {
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -312,7 +336,6 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
     constexpr int U = B == 3 ? 4 : B == 2 ? 8 : 16;   // bytes per copy
     constexpr int UPC = 4 * B / U;                    // copies per 32-code chunk
     static_assert(RPT * NT == 512, "thread count");
-    const int n_tiles = p.n_tiles;
     volatile int *abort = &c.abort;
     const int ch = d & 1;
     int rows[RPT];
@@ -322,12 +345,15 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         rows[r] = (q % 256) / 2 + 128 * (q / 256);
     }
 
-    // Issue cursor: the block of 128 codes whose codes are copied next.
-    int tp = blockIdx.x, gp = 0, Gp = 0, gsh = 2;
+    // Issue cursor: the block of 128 codes whose codes are copied next, in the
+    // tile of ring entry jp (the issue cursor reads each entry first; the
+    // consume cursor, later, releases it).
+    uint32_t jp = 0;
+    int tp = tile_at(c, jp, abort, p.wait_ns), gp = 0, Gp = 0, gsh = 2;
     const uint32_t *prow[RPT];
     const uint16_t *psr[RPT], *pzr[RPT];
     auto start_issue = [&]() {
-        if (tp < n_tiles) {
+        if (tp >= 0) {
             const TileRef tr = locate(p, tp);
             const PrefillOp &op = p.ops[tr.o];
             Gp = op.K / kGroup;
@@ -361,7 +387,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                 zs[(2 * r + 1) * NT + d] = set[r][1];
             }
         }
-        if (tp < n_tiles) {
+        if (tp >= 0) {
             uint8_t *cs = scode + (j % kS) * P::kSlotBytes;
 #pragma unroll
             for (int h = 0; h < 2; ++h)
@@ -380,7 +406,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
             }
             if (++gp == Gp) {
                 gp = 0;
-                tp += gridDim.x;
+                tp = tile_at(c, ++jp, abort, p.wait_ns);
                 start_issue();
             }
         }
@@ -393,8 +419,12 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
     }
     if constexpr (PD & 1) issue(PD - 1, szA);
 
-    // Consume cursor: group i of tile t.
-    int t = blockIdx.x, g = 0, G = t < n_tiles ? p.ops[locate(p, t).o].K / kGroup : 0;
+    // Consume cursor: group i of tile t, ring entry jc (released by the warp
+    // once read: the issue cursor has read it already).
+    uint32_t jc = 0;
+    int t = tile_at(c, jc, abort, p.wait_ns), g = 0, G = t >= 0 ? p.ops[locate(p, t).o].K / kGroup : 0;
+    __syncwarp();
+    if (lane == 0) tile_release(c, jc);
     uint32_t it = 0;  // W stages filled so far
     auto consume = [&](int i) -> bool {
         cp_async_wait<PD>();               // this thread's copies of group i have landed
@@ -448,8 +478,10 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         }
         if (++g == G) {
             g = 0;
-            t += gridDim.x;
-            if (t < n_tiles) G = p.ops[locate(p, t).o].K / kGroup;
+            t = tile_at(c, ++jc, abort, p.wait_ns);
+            __syncwarp();
+            if (lane == 0 && t != -2) tile_release(c, jc);
+            if (t >= 0) G = p.ops[locate(p, t).o].K / kGroup;
         }
         return true;
     };
@@ -457,10 +489,10 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
     uint32_t (&set_odd)[RPT][2] = (PD & 1) ? szA : szB;
 #pragma unroll 1
     for (int i = 0;; i += 2) {
-        if (t >= n_tiles || *abort) break;
+        if (t < 0 || *abort) break;
         issue(i + PD, set_even);
         if (!consume(i)) break;
-        if (t >= n_tiles || *abort) break;
+        if (t < 0 || *abort) break;
         issue(i + 1 + PD, set_odd);
         if (!consume(i + 1)) break;
     }
@@ -482,6 +514,10 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
     volatile int *abort = &sm.abort;
 
     if (threadIdx.x == 0) {
+        for (int i = 0; i < kTileRing; ++i) {
+            mbar_init(&sm.tq_full[i], 1);
+            mbar_init(&sm.tq_empty[i], P::kTileReaders);
+        }
         for (int s = 0; s < P::kStages; ++s) {
             if constexpr (B != 16) mbar_init(&sm.full[s], P::kDqWarps);
             mbar_init(&sm.xfull[s], 1);
@@ -507,10 +543,28 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
     pdl_wait();  // x may be produced by the previous kernel in the stream
     pdl_launch_dependents();
 
-    if (warp == kTmaWarp) {
+    if (warp == P::kSchedWarp) {
+        // Tile scheduler: tickets from the launch's counter, in order, into the
+        // ring; an entry is refilled once every reader has released it.
+        if (lane == 0) {
+            for (uint32_t i = 0;; ++i) {
+                if (i >= kTileRing &&
+                    !mbar_wait(&sm.tq_empty[i % kTileRing], ((i / kTileRing) - 1u) & 1u, abort, p.wait_ns))
+                    break;
+                const unsigned int v = atomicAdd(p.tile_ctr, 1u);
+                const int t = v < static_cast<unsigned int>(n_tiles) ? static_cast<int>(v) : -1;
+                *reinterpret_cast<volatile int *>(&sm.tq[i % kTileRing]) = t;
+                mbar_arrive(&sm.tq_full[i % kTileRing]);  // release: publishes the entry
+                if (t < 0) break;
+            }
+        }
+    } else if (warp == kTmaWarp) {
         if (lane == 0) {
             uint32_t it = 0;
-            for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x) {
+            for (uint32_t j = 0;; ++j) {
+                const int t = tile_at(sm, j, abort, p.wait_ns);
+                if (t != -2) tile_release(sm, j);
+                if (t < 0 || *abort) break;
                 const TileRef tr = locate(p, t);
                 const PrefillOp &op = p.ops[tr.o];
                 const int slabs = op.K / kBK;
@@ -543,7 +597,10 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         if (lane == 0) {
             uint32_t it = 0, tile_i = 0;
             bool issued = false;
-            for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
+            for (uint32_t j = 0;; ++j, ++tile_i) {
+                const int t = tile_at(sm, j, abort, p.wait_ns);
+                if (t != -2) tile_release(sm, j);
+                if (t < 0 || *abort) break;
                 const TileRef tr = locate(p, t);
                 const int slabs = p.ops[tr.o].K / kBK;
                 // the second 128-token half only when it holds tokens
@@ -633,13 +690,18 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                 szn[1][i] = g1 == g0 ? szn[0][i] : ldg_u16_nc(srow[i] + g1) | (ldg_u16_nc(zrow[i] + g1) << 16);
             }
         };
-        int t = blockIdx.x, g = 0, groups = 0, groups_n = 0;
-        if (t < n_tiles) {
+        // Tiles from the ring: entry jn is read (and released) by the fetch
+        // cursor, one block ahead of the dequant.
+        uint32_t jn = 0;
+        int t = tile_at(sm, jn, abort, p.wait_ns), g = 0, groups = 0, groups_n = 0;
+        __syncwarp();
+        if (lane == 0 && t != -2) tile_release(sm, jn);
+        if (t >= 0) {
             groups = start_tile(t);
             fetch(0);
         }
         bool ok = true;
-        while (t < n_tiles && ok && !*abort) {
+        while (t >= 0 && ok && !*abort) {
             uint32_t wc[2][2][B], szc[2][2];
 #pragma unroll
             for (int h = 0; h < 2; ++h)
@@ -659,10 +721,12 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
             groups_n = groups;
             if (g_n == groups) {
                 g_n = 0;
-                t_n += gridDim.x;
-                if (t_n < n_tiles) groups_n = start_tile(t_n);
+                t_n = tile_at(sm, ++jn, abort, p.wait_ns);
+                __syncwarp();
+                if (lane == 0 && t_n != -2) tile_release(sm, jn);
+                if (t_n >= 0) groups_n = start_tile(t_n);
             }
-            if (t_n < n_tiles) fetch(g_n);
+            if (t_n >= 0) fetch(g_n);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {  // the two slabs of this group
                 const int st = it % P::kStages;
@@ -697,7 +761,11 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
     } else {
         // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = tokens of each half.
         uint32_t tile_i = 0;
-        for (int t = blockIdx.x; t < n_tiles && !*abort; t += gridDim.x, ++tile_i) {
+        for (uint32_t j = 0;; ++j, ++tile_i) {
+            const int t = tile_at(sm, j, abort, p.wait_ns);
+            __syncwarp();
+            if (lane == 0 && t != -2) tile_release(sm, j);
+            if (t < 0 || *abort) break;
             if (!mbar_wait(&sm.acc_full, tile_i & 1u, abort, p.wait_ns)) break;
             tc_fence_after();
             const TileRef tr = locate(p, t);
@@ -764,9 +832,55 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
     }
+    // The last CTA to finish sets the launch's tile counter back to zero for
+    // the next launch on the stream (which reads it only after this grid has
+    // completed: its schedulers start after griddepcontrol.wait).
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(p.tile_ctr + 1, 1u) == gridDim.x - 1) {
+            atomicExch(p.tile_ctr, 0u);
+            atomicExch(p.tile_ctr + 1, 0u);
+        }
+    }
+}
+
+// Dequant test hook: one thread per (row, 32-code chunk) runs dequant_chunk,
+// the tile kernel's own routine (unpack, one-HFMA2 rounding, K-order restore,
+// overflow hold), and writes the 32 fp16 values to w_hat (N x K, natural order).
+template <int B>
+__global__ void dequant_test_kernel(const uint32_t *__restrict__ packed, const uint16_t *__restrict__ scales,
+                                    const uint16_t *__restrict__ zeros, int N, int K, int gshift,
+                                    uint16_t *__restrict__ w_hat) {
+    const long long t = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const int chunks = K / 32;
+    if (t >= static_cast<long long>(N) * chunks) return;
+    const int n = static_cast<int>(t / chunks), c = static_cast<int>(t % chunks);
+    uint32_t w[B];
+    load_chunk<B>(w, packed + static_cast<size_t>(n) * (static_cast<size_t>(K) * B / 32) + static_cast<size_t>(c) * B);
+    const size_t gi = static_cast<size_t>(n) * (static_cast<size_t>(K) >> (gshift + 5)) + (c >> gshift);
+    const uint32_t sz = scales[gi] | (static_cast<uint32_t>(zeros[gi]) << 16);
+    uint32_t o[16];
+    dequant_chunk<B>(w, sz, o, dequant_overflows<B>(sz));
+    uint4 *dst = reinterpret_cast<uint4 *>(w_hat + static_cast<size_t>(n) * K + static_cast<size_t>(c) * 32);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
 }
 
 }  // namespace pf
+
+cudaError_t launch_dequant_test(const uint32_t *packed, const uint16_t *scales, const uint16_t *zeros, int bits,
+                                int group, int N, int K, uint16_t *w_hat, cudaStream_t stream) {
+    const long long threads = static_cast<long long>(N) * (K / 32);
+    const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+    const int gshift = group == 32 ? 0 : group == 64 ? 1 : 2;
+    switch (bits) {
+        case 2: pf::dequant_test_kernel<2><<<blocks, 256, 0, stream>>>(packed, scales, zeros, N, K, gshift, w_hat); break;
+        case 3: pf::dequant_test_kernel<3><<<blocks, 256, 0, stream>>>(packed, scales, zeros, N, K, gshift, w_hat); break;
+        case 4: pf::dequant_test_kernel<4><<<blocks, 256, 0, stream>>>(packed, scales, zeros, N, K, gshift, w_hat); break;
+        default: pf::dequant_test_kernel<8><<<blocks, 256, 0, stream>>>(packed, scales, zeros, N, K, gshift, w_hat); break;
+    }
+    return cudaGetLastError();
+}
 
 // ------------------------------------------------------------------ host --
 
