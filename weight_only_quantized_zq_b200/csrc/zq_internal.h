@@ -36,9 +36,9 @@ struct alignas(64) DecodeOp {
     const uint16_t *zeros;
     const uint16_t *xg;     // workspace: (M, or M_pad with several token tiles) x K fp16, pair-permuted,
                             // 2^(E-s)-scaled, chunk-swizzled activations
-    const float *sx;        // workspace: G x R x 4 fp32 (sum x, -f * 1024 * sum x', f, 0) per group and
-                            // token, R = M (one token tile) or M_pad; f = 2^-E undoes the power-of-two
-                            // x' scale
+    const float *sx;        // workspace: x_rows x G x 4 fp32 (sum x, -f * 1024 * sum x', f, 0) per token
+                            // and group (x_rows = M with one token tile, else M_pad); f = 2^-E undoes the
+                            // power-of-two x' scale
     uint16_t *out;          // M x N fp16, or null when out32 is set
     float *out32;           // M x N fp32 (partial sums, not rounded), or null
     int step0;              // first CTA step of this op
@@ -72,7 +72,7 @@ static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
     uint16_t *xg;       // x_rows x K, chunk-swizzled per group and token; rows >= M are zeros
-    float *sx;          // G x x_rows x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
+    float *sx;          // x_rows x G x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
     int M, x_rows, K, bits;  // x_rows: M with one token tile, else the padded M_pad
     int x_bf16;              // 1: x holds bfloat16, else fp16
 };
