@@ -276,7 +276,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     const int off_sz = 0;
     const int off_sx = off_sz + rows * 4 * gps;
     const int x_rows_max = mt == 1 ? max_m : mpad;  // staged token rows (and group records)
-    const int off_x = off_sx + gps * x_rows_max * 16;
+    const int off_x = off_sx + decode_rec_stride(bits) * x_rows_max * 16;
     const int off_desc = off_x + gps * x_rows_max * 256;
     const int meta_bytes = static_cast<int>(align16(off_desc + 32));
     const int stage = codes_bytes + meta_bytes;
@@ -337,7 +337,8 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         prep_off[e] = off;
         const size_t G = keys[e].K / kGroup;
         const size_t xr = mt == 1 ? keys[e].M : mpad;
-        off += align256(G * xr * kGroup * 2) + align256(G * xr * 16);
+        const size_t steps = (G + gps - 1) / gps;  // x' and records are stored by step (whole GPS blocks)
+        off += align256(steps * gps * xr * kGroup * 2) + align256(steps * decode_rec_stride(bits) * xr * 16);
     }
     const size_t part_off = off;
     if (!units) off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
@@ -365,7 +366,8 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         en.x = keys[e].x;
         en.xg = reinterpret_cast<uint16_t *>(data + prep_off[e]);
         en.x_rows = mt == 1 ? keys[e].M : mpad;
-        en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(G * en.x_rows * kGroup * 2));
+        const size_t steps = (G + gps - 1) / gps;
+        en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(steps * gps * en.x_rows * kGroup * 2));
         en.M = keys[e].M;
         en.x_bf16 = keys[e].xbf16;
         en.K = keys[e].K;

@@ -127,14 +127,18 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
         const long long local = gw - p.warp_prefix[e];
         const int G = en.K / kGroup;
         const int t = static_cast<int>(local / G), g = static_cast<int>(local % G);
-        float4 *dst = reinterpret_cast<float4 *>(en.sx) + static_cast<size_t>(t) * G + g;  // [token][group]
+        // Both outputs by decode step (GPS groups): [step][token][GPS groups]
+        // of x' and [step][token][RS records], so a step's x' and records for
+        // all staged tokens are two contiguous blocks (two bulk copies).
+        const int gps = decode_gps(en.bits, 1);
+        const size_t blk = static_cast<size_t>(g / gps) * en.x_rows + t;  // (step, token)
+        float4 *dst = reinterpret_cast<float4 *>(en.sx) + blk * decode_rec_stride(en.bits) + g % gps;
+        uint16_t *prow = en.xg + (blk * gps + g % gps) * kGroup;
         if (t >= en.M) {
             if (lane == 0) *dst = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            reinterpret_cast<uint2 *>(en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup)[lane] =
-                    make_uint2(0u, 0u);
+            reinterpret_cast<uint2 *>(prow)[lane] = make_uint2(0u, 0u);
         } else {
             const uint16_t *xrow = en.x + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
-            uint16_t *prow = en.xg + static_cast<size_t>(t) * en.K + static_cast<size_t>(g) * kGroup;
             const uint2 v = reinterpret_cast<const uint2 *>(xrow)[lane];
             const bool bf = en.x_bf16 != 0;
             const float x0 = bf ? act_bits<true>(v.x & 0xFFFFu) : act_bits<false>(v.x & 0xFFFFu);
@@ -383,6 +387,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     constexpr int GB = 16 * BITS;                   // bytes of one row of one group
     constexpr int MPAD = 8 * MT;
     constexpr int SZB = 2 * GPS;                    // bytes of scales (or zeros) of one row per step
+    constexpr int RS = decode_rec_stride(BITS);     // shared-memory record slots per staged token
 
     extern __shared__ uint8_t smem_raw[];
     // Swizzled TMA destinations need 1024-byte alignment (the host adds slack).
@@ -509,23 +514,20 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
             if (lane == 0) {
                 dsc[0] = make_int4(ld.o, ld.rb, ld.j, ng | (flags << 8));
                 dsc[1] = make_int4(ld_chunk, unit_start, op.M, 0);
-                const uint32_t xbytes = static_cast<uint32_t>(ng * xrows * 256);
-                const uint32_t sbytes = static_cast<uint32_t>(ng * xrows * 16);  // ng records per staged token
+                // the step's x' and records for all staged tokens: two
+                // contiguous blocks (a last step with ng < GPS groups copies
+                // its unused group slots too)
+                const uint32_t xbytes = static_cast<uint32_t>(xrows * GPS * 256);
+                const uint32_t sbytes = static_cast<uint32_t>(xrows * RS * 16);
                 mbar_arrive_expect_tx(&full[slot_ld], NBOX * BOXB + xbytes + sbytes);
 #pragma unroll
                 for (int b = 0; b < NBOX; ++b)
                     tma_load_2d(st + b * BOXB, &op.tmap, g0 * GB + b * BOXW, ld.rb * kDecodeCtaRows, &full[slot_ld]);
+                const size_t blk = static_cast<size_t>(ld.j) * xrows;  // first (step, token) block
+                bulk_load(sm + p.off_x, op.xg + blk * (GPS * kGroup), xbytes, &full[slot_ld]);
+                bulk_load(sm + p.off_sx, op.sx + blk * (RS * 4), sbytes, &full[slot_ld]);
             }
             __syncwarp();
-            // Activations and group records: token t's ng groups (ng * 256 and
-            // ng * 16 contiguous bytes), one bulk copy each per staged token,
-            // issued by lane t after the bytes were announced.
-            for (int t = lane; t < xrows; t += 32) {
-                bulk_load(sm + p.off_x + t * (GPS * 256), op.xg + static_cast<size_t>(t) * op.K + g0 * kGroup,
-                          static_cast<uint32_t>(ng * 256), &full[slot_ld]);
-                bulk_load(sm + p.off_sx + t * (GPS * 16), op.sx + (static_cast<size_t>(t) * op.G + g0) * 4,
-                          static_cast<uint32_t>(ng * 16), &full[slot_ld]);
-            }
             cursor_next(ld, p, ld_end);
         } else {
             cp_async_arrive_noinc(&full[slot_ld]);
@@ -566,8 +568,8 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     //   x':    token gq's staged row is GPS*256 bytes, group gi at +gi*256,
     //          the lane's chunk q of it at x_chunk(c, q, gq).
     //   sums:  (sum x, -f * bias, f, 0) of token 8mt + 2c of group gi at
-    //          off_sx + ((8mt + 2c) * GPS + gi) * 16, token 8mt + 2c + 1
-    //          GPS * 16 bytes on; lanes of tokens >= M read other bytes of the
+    //          off_sx + ((8mt + 2c) * RS + gi) * 16, token 8mt + 2c + 1
+    //          RS * 16 bytes on; lanes of tokens >= M read other bytes of the
     //          stage (their columns are padding).
     int lanex;
     if constexpr (BITS == 4) lanex = c ^ gr;
@@ -595,7 +597,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     uint32_t xq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) xq[q] = p.off_x + gq * (GPS * 256) + (x_chunk(c, q, gq) << 4);
-    const uint32_t sxo = p.off_sx + 2 * c * GPS * 16;
+    const uint32_t sxo = p.off_sx + 2 * c * RS * 16;
     const uint32_t szq0 = p.off_sz + (warp * 16 + gr) * 2 * SZB, szq1 = p.off_sz + (warp * 16 + 8 + gr) * 2 * SZB;
     const uint32_t ring_s = smem_u32(ring), meta_s = smem_u32(meta);
 
@@ -751,7 +753,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                         xf[4 * q + 3] = v.w;
                     }
                 }
-                const uint4 sa = lds_v4(smb + sxo + (8 * mt * GPS + gi) * 16);
+                const uint4 sa = lds_v4(smb + sxo + (8 * mt * RS + gi) * 16);
                 // tot += s * f * (acc - bias) + z * sum(x): the z * sum(x) term
                 // first (it needs no MMA result, and its operands die early),
                 // then s * f * (acc - bias) with f * (acc - bias) as one FMA (f
@@ -761,7 +763,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                 for (int h = 0; h < 2; ++h) tot[mt][2 * h] = fmaf(zr[h], __uint_as_float(sa.x), tot[mt][2 * h]);
                 uint4 sb = make_uint4(0u, 0u, 0u, 0u);
                 if constexpr (!one_token) {
-                    sb = lds_v4(smb + sxo + ((8 * mt + 1) * GPS + gi) * 16);
+                    sb = lds_v4(smb + sxo + ((8 * mt + 1) * RS + gi) * 16);
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
                         tot[mt][2 * h + 1] = fmaf(zr[h], __uint_as_float(sb.x), tot[mt][2 * h + 1]);

@@ -34,11 +34,12 @@ struct alignas(64) DecodeOp {
     CUtensorMap tmap;       // packed codes as a 2-D uint8 tensor: box = 64 rows x box_w bytes
     const uint16_t *scales;
     const uint16_t *zeros;
-    const uint16_t *xg;     // workspace: (M, or M_pad with several token tiles) x K fp16, pair-permuted,
-                            // 2^(E-s)-scaled, chunk-swizzled activations
-    const float *sx;        // workspace: x_rows x G x 4 fp32 (sum x, -f * 1024 * sum x', f, 0) per token
-                            // and group (x_rows = M with one token tile, else M_pad); f = 2^-E undoes the
-                            // power-of-two x' scale
+    const uint16_t *xg;     // workspace: pair-permuted, 2^(E-s)-scaled, chunk-swizzled fp16 activations
+                            // by decode step, [K / (128 GPS)][x_rows][GPS x 128] (x_rows = M with one
+                            // token tile, else M_pad)
+    const float *sx;        // workspace: records (sum x, -f * 1024 * sum x', f, 0) fp32 per token and
+                            // group by step, [K / (128 GPS)][x_rows][RS] (RS = decode_rec_stride >= GPS
+                            // slots, group g at slot g % GPS); f = 2^-E undoes the power-of-two x' scale
     uint16_t *out;          // M x N fp16, or null when out32 is set
     float *out32;           // M x N fp32 (partial sums, not rounded), or null
     int step0;              // first CTA step of this op
@@ -71,8 +72,8 @@ static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 
 struct PrepEntry {
     const uint16_t *x;  // M x K fp16
-    uint16_t *xg;       // x_rows x K, chunk-swizzled per group and token; rows >= M are zeros
-    float *sx;          // x_rows x G x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
+    uint16_t *xg;       // [step][x_rows][GPS x 128], chunk-swizzled per group and token; rows >= M are zeros
+    float *sx;          // [step][x_rows][RS] x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
     int M, x_rows, K, bits;  // x_rows: M with one token tile, else the padded M_pad
     int x_bf16;              // 1: x holds bfloat16, else fp16
 };
@@ -89,6 +90,13 @@ struct PrepParams {
 // 4 warps computes 16 of the rows.
 __host__ __device__ constexpr int decode_gps(int bits, int) { return bits == 16 ? 1 : bits == 8 ? 2 : 4; }
 __host__ __device__ constexpr int decode_seg(int bits, int mt) { return decode_gps(bits, mt) * 16 * bits; }
+// Record slots (16 bytes) per token in a decode step's block of records: one
+// spare slot when GPS > 1, so that the records of tokens 2c (c = 0..3),
+// which a quad of lanes reads at once, start in four different bank quads (a
+// token stride of 4 * 16 = 64 bytes would put all four in the same banks).
+__host__ __device__ constexpr int decode_rec_stride(int bits) {
+    return decode_gps(bits, 1) + (decode_gps(bits, 1) > 1 ? 1 : 0);
+}
 // Codes of a step land as 128-byte-wide TMA boxes with the 128-byte swizzle
 // when a row segment is a whole number of 128-byte spans.  Otherwise (b = 3:
 // 192 bytes) as one unswizzled box 16 bytes wider than the segment: a shared

@@ -53,16 +53,7 @@ namespace pf {
 constexpr int kTokTile = 256;   // tokens per CTA tile (two MMA halves of 128)
 constexpr int kRowTile = 256;   // weight rows per CTA tile (MMA N)
 constexpr int kBK = 64;         // K per slab
-constexpr int kMaxStages = 4;
-// One-token-half plan with the dequantized weights in tensor memory: the
-// dequant warps write them with tcgen05.st as the MMA's A operand (weight
-// rows = M, 128 per row block), the x slab is the B operand (tokens = N), and
-// W never passes through shared memory.  TMEM columns: the accumulators of the
-// two row blocks, 128 tokens each, then kTmStages A stages of 2 row blocks x
-// 32 columns (64 k of fp16).
-constexpr bool kTmemW = true;
-constexpr int kTmStages = 4;
-constexpr uint32_t kTmA = 256;  // first A column
+constexpr int kMaxStages = 3;
 constexpr int kSlabB = kRowTile * kBK * 2;  // 32 KB
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
@@ -108,31 +99,26 @@ struct Plan {
     // Dequant warps: 16 in the one-half plan (its code ring keeps their
     // registers low), 8 in the two-half plan (register prefetch); none for
     // fp16 weights (B = 16), which TMA copies into the W stages as they are.
-    static constexpr bool TM = kTmemW && ONE && B != 16;  // weights in tensor memory
     static constexpr int kDqWarps = B == 16 ? 0 : ONE ? 16 : 8;
     static constexpr int kSchedWarp = kDqWarp0 + kDqWarps;  // the tile scheduler (lane 0)
     static constexpr int kThreads = 32 * (kSchedWarp + 1);
     // readers of every tile-ring entry: TMA and MMA lanes, epilogue and dequant warps
     static constexpr int kTileReaders = 2 + kEpiWarps + kDqWarps;
-    static constexpr int kStages = TM ? kTmStages : B == 16 ? 3 : (ONE && B == 8) ? 2 : 3;
+    static constexpr int kStages = B == 16 ? 3 : (ONE && B == 8) ? 2 : 3;
     static constexpr int kSlabA = (ONE ? kPrefillHalfTokens : kTokTile) * kBK * 2;
-    // code slots: with W out of shared memory there is room for more blocks in flight
-    static constexpr int kSlots = (!ONE || B == 16) ? 0
-                                  : TM ? (B == 2 ? 8 : B == 3 ? 7 : B == 4 ? 6 : 4)
-                                       : (B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3);
+    static constexpr int kSlots = (!ONE || B == 16) ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
     static constexpr int kSlotCodes = 1024 * (4 * B);  // 256 rows x 2 slabs x 2 chunks of 32 codes
     // + a (scale | zero << 16) word per (row, chunk, slab): the two slabs of a
     // block of 128 codes fall in different groups when groups are 32 or 64
     static constexpr int kSlotBytes = kSlotCodes + 1024 * 4;
     static constexpr int kOffB = kStages * kSlabA;
-    static constexpr int kOffCodes = kOffB + (TM ? 0 : kStages * kSlabB);
+    static constexpr int kOffCodes = kOffB + kStages * kSlabB;
     static constexpr int kOffCtl = kOffCodes + kSlots * kSlotBytes;
     static constexpr size_t kBytes = kOffCtl + sizeof(Ctl) + 1024;  // + alignment slack
     static_assert(kStages <= kMaxStages, "barrier arrays");
     static_assert(kOffB % 1024 == 0 && kOffCodes % 1024 == 0, "SWIZZLE_128B stages need 1024-byte alignment");
     static_assert(kBytes <= 232448, "227 KB of shared memory per CTA");
     static_assert(!ONE || B == 16 || kSlots >= 3, "the scale/zero hand-off needs a prefetch distance of 2 groups");
-    static_assert(!TM || kTmA + kStages * 64 <= 512, "TMEM columns");
 };
 
 // Bounded wait: false if the CTA is aborting or the limit was reached.
@@ -201,32 +187,6 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
         "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
-        : "memory");
-}
-
-// Instruction descriptor, kind::f16, for the tensor-memory-A plan: fp16 A
-// (weights, from TMEM) and B (tokens, K-major in shared memory), fp32 D,
-// M = 128 weight rows, N = 128 tokens.
-constexpr uint32_t kIdescTm = (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(128 >> 3) << 17) |
-                              (static_cast<uint32_t>(128 >> 4) << 24);
-
-// D (TMEM) += A (TMEM) * B (shared memory descriptor).
-__device__ __forceinline__ void umma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(bdesc), "r"(kIdescTm), "r"(accumulate)
-        : "memory");
-}
-
-// 16 consecutive 32-bit columns of this thread's TMEM lane (the warp's quarter).
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
-        "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
         : "memory");
 }
 
@@ -367,7 +327,7 @@ __device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
 // unrolled twice.
 template <int B>
 __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb, uint8_t *scode, Ctl &c,
-                                             int d, int lane, uint32_t tmem) {
+                                             int d, int lane) {
     using P = Plan<B, true>;
     constexpr int NT = 32 * P::kDqWarps;
     constexpr int RPT = 512 / NT;                     // rows per thread
@@ -377,19 +337,12 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
     constexpr int UPC = 4 * B / U;                    // copies per 32-code chunk
     static_assert(RPT * NT == 512, "thread count");
     volatile int *abort = &c.abort;
-    // (row, chunk) of this thread.  Weights in tensor memory: a warp may only
-    // write its own quarter of the 128 TMEM lanes (lanes 32 * (warp % 4) ..),
-    // so warp wq takes 32 consecutive rows of that quarter, with the row block
-    // and chunk chosen by wq / 4.  Otherwise 16 consecutive rows x 2 chunks.
-    const int wq = d >> 5;
-    const int tq_lane = (kDqWarp0 + wq) & 3;  // TMEM lane quarter
-    const int ch = P::TM ? ((wq >> 2) & 1) : (d & 1);
-    const int tm_blk = (wq >> 3) & 1;         // row block (TM)
+    const int ch = d & 1;
     int rows[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r) {
         const int q = d + NT * r;
-        rows[r] = P::TM ? 128 * tm_blk + 32 * tq_lane + lane : (q % 256) / 2 + 128 * (q / 256);
+        rows[r] = (q % 256) / 2 + 128 * (q / 256);
     }
 
     // Issue cursor: the block of 128 codes whose codes are copied next, in the
@@ -491,8 +444,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
             const int st = it % P::kStages;
             const uint32_t round = it / P::kStages;
             if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) return false;
-            if constexpr (P::TM) tc_fence_after();  // the MMAs that read this A stage have completed
-            uint8_t *bs = sb + (P::TM ? 0 : st * kSlabB);
+            uint8_t *bs = sb + st * kSlabB;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 uint32_t w[B];
@@ -512,26 +464,14 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                 const int row = rows[r];
                 uint32_t o[16];
                 dequant_chunk<B>(w, sz[r][h], o, ovf[r][h]);
-                if constexpr (P::TM) {
-                    // the row's 32 weights of this slab: 16 columns of its lane
-                    tmem_st16(tmem + (static_cast<uint32_t>(32 * tq_lane) << 16) + kTmA + st * 64 + tm_blk * 32 +
-                                  ch * 16,
-                              o);
-                } else {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        const int c16 = (4 * ch + j) ^ (row & 7);
-                        *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
-                            make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-                    }
+                for (int j = 0; j < 4; ++j) {
+                    const int c16 = (4 * ch + j) ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
+                        make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
                 }
             }
-            if constexpr (P::TM) {
-                asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                tc_fence_before();
-            } else {
-                fence_proxy_async();
-            }
+            fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&c.full[st]);
             ++it;
@@ -697,17 +637,8 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
                     tc_fence_after();
                     issued = true;
                     const uint32_t a0 = smem_u32(sa + st * P::kSlabA);
-                    const uint32_t b0 = smem_u32(sb + (P::TM ? 0 : st * kSlabB));
-                    if constexpr (P::TM) {
-                        // D (row block b: TMEM columns b * 128, lanes = weight
-                        // rows) += W (TMEM, A) x x-slab (shared memory, B)
-#pragma unroll
-                        for (int b = 0; b < 2; ++b)
-#pragma unroll
-                            for (int kk = 0; kk < kBK / 16; ++kk)
-                                umma_f16_ta(tmem + b * 128, tmem + kTmA + st * 64 + b * 32 + kk * 8,
-                                            sdesc_sw128(a0 + kk * 32), (s > 0 || kk > 0) ? 1u : 0u);
-                    } else if (half1) {
+                    const uint32_t b0 = smem_u32(sb + st * kSlabB);
+                    if (half1) {
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk) {
                             const uint64_t bd = sdesc_sw128(b0 + kk * 32);
@@ -738,7 +669,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         if constexpr (B == 16) {
             // no dequant warps for fp16 weights
         } else if constexpr (ONE) {
-            dequant_ring<B>(p, sb, scode, sm, threadIdx.x - 32 * kDqWarp0, lane, tmem);
+            dequant_ring<B>(p, sb, scode, sm, threadIdx.x - 32 * kDqWarp0, lane);
         } else {
         // 256 threads: thread d owns rows d/2 and d/2 + 128 of the tile and the
         // 32-code chunk d%2 of every slab.  Codes, scales and zeros of the next
@@ -860,31 +791,6 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
             const PrefillOp &op = p.ops[tr.o];
             const int n0 = tr.n0, t0 = tr.t0;
             const bool vec = (op.N % 8) == 0;
-            if constexpr (P::TM) {
-                // lanes = weight rows (row block b: columns b * 128), columns =
-                // tokens: each thread owns one output column n; for a token the
-                // warp writes 32 consecutive outputs
-#pragma unroll 1
-                for (int b = 0; b < 2; ++b) {
-                    const int n = n0 + 128 * b + 32 * warp + lane;
-#pragma unroll 1
-                    for (int cc = 0; cc < kPrefillHalfTokens / 32 && t0 + 32 * cc < op.M; ++cc) {
-                        uint32_t r[32];
-                        tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + b * 128 + cc * 32, r);
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) {
-                            const int tok = t0 + 32 * cc + q;
-                            if (tok < op.M && n < op.N) {
-                                float v = __uint_as_float(r[q]);
-                                if (op.xscale != nullptr) v *= op.xscale[tok];
-                                const size_t at = static_cast<size_t>(tok) * op.N + n;
-                                if (op.out32) op.out32[at] = v;
-                                else op.out[at] = static_cast<uint16_t>(pack_out2(v, 0.0f, op.out_bf16));
-                            }
-                        }
-                    }
-                }
-            } else
 #pragma unroll 1
             for (int half = 0; half < (t0 + 128 < op.M ? 2 : 1); ++half) {
                 const int tok = t0 + 128 * half + 32 * warp + lane;
