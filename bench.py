@@ -16,7 +16,7 @@ out) / device time, in GB/s; also % of 8 TB/s and tokens/s-equivalent
                     [--m M] [--layers L]
 
 M <= 64 is decode (bandwidth-bound, reported against HBM; the library runs
-M <= 16 on its mma.sync decode kernel and larger M on its tcgen05 tile
+M <= 32 on its mma.sync decode kernel and larger M on its tcgen05 tile
 kernel); M > 64 is prefill (reported against the tensor peak).
 
 --impl reference times the fp64 CPU oracle on a bounded sample of the same
@@ -573,7 +573,7 @@ def run_zq(args):
     e2e_value = world * wl.bytes * args.steps / (e2e_ms / 1e3) / 1e9
 
     # Roofline of the dominant kernel.  Decode (M <= 64): the grouped launch;
-    # with M <= 16 the step is one prep launch + one decode launch, timed
+    # with M <= 32 the step is one prep launch + one decode launch, timed
     # together by the events above, so the figure is a lower bound for the
     # kernel.  Prefill (M > 64): the grouped tcgen05 launches.
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
@@ -584,14 +584,14 @@ def run_zq(args):
     if M <= 64:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
-                    "traffic": measured_traffic("decode" if M <= 16 else "prefill", args.model, M, args.layers),
-                    "traffic_note": ("per step (one decode launch)" if M <= 16 else
+                    "traffic": measured_traffic("decode" if M <= DECODE_MAX_M else "prefill", args.model, M, args.layers),
+                    "traffic_note": ("per step (one decode launch)" if M <= DECODE_MAX_M else
                                      "per step (the stack's grouped tile-kernel launches)"),
                     "algorithmic_bytes": wl.bytes,
                     "peak_source": peaks["source"],
                     "kernel": (f"decode_kernel<{'|'.join(str(b) for b in bits_used)},{zq_mt(M)}> + prep_kernel"
                                + (" (one launch pair per bit width)" if len(bits_used) > 1 else "")
-                               if M <= 16 else tile_kernel)}
+                               if M <= DECODE_MAX_M else tile_kernel)}
     else:
         tflops = wl.flops / (ms_step / 1e3) / 1e12
         peak = peaks["bf16_tflops"]  # burst: a step of tens of ms, timed alone
@@ -642,8 +642,11 @@ def run_zq(args):
     return 0
 
 
+DECODE_MAX_M = 32  # the library runs M <= 32 on the decode kernel
+
+
 def zq_mt(M):
-    return 1 if M <= 8 else 2
+    return 1 if M <= 8 else 2 if M <= 16 else 4
 
 
 def main(argv=None):

@@ -133,7 +133,7 @@ ZQ_API zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bi
  * of [wiki] "Формат модели .zse" (dequant(W) = q * scale + zero per group).
  *   x       device, fp16 M x K.      out  device, fp16 M x N (written).
  *   packed/scales/zeros as produced by zq_quantize_pack.
- * M <= 16 runs the decode kernel (mma.sync skinny GEMM streaming the packed
+ * M <= 32 runs the decode kernel (mma.sync skinny GEMM streaming the packed
  * weights once through a shared-memory ring); larger M, and groups of 32 or
  * 64 at any M, run the tcgen05 tile kernel (256 x 256 output tiles; with
  * M <= 256 one token tile, so the weights are again streamed once).

@@ -194,6 +194,7 @@ def test_linear_shapes(zq, orc, bits):
     """Ragged N, every decode token tile, split-K and the multi-piece path."""
     cases = [(1, 1, 128), (1, 17, 512), (2, 100, 384), (3, 33, 1024), (5, 512, 512),
              (8, 257, 1280), (9, 64, 512), (16, 130, 256), (17, 48, 640), (32, 96, 512),
+             (24, 257, 1152), (31, 64, 384), (20, 300, 3584),
              (33, 40, 384), (64, 200, 768), (65, 31, 256), (130, 70, 512)]
     for i, (M, N, K) in enumerate(cases):
         w = zi.weight(N, K, seed=1000 + 10 * bits + i, device="cuda", outliers=(i % 3 == 0))
@@ -204,7 +205,7 @@ def test_linear_shapes(zq, orc, bits):
 
 @pytest.mark.parametrize("bits", BITS)
 def test_prefill_shapes(zq, orc, bits):
-    """M > 16 runs the tcgen05 tile kernel: ragged token tiles (TMA zero
+    """M > 32 runs the tcgen05 tile kernel: ragged token tiles (TMA zero
     fill), ragged weight-row tiles, N not a multiple of 8 (scalar stores)."""
     cases = [(65, 31, 256), (130, 70, 512), (256, 256, 128), (300, 520, 1024), (257, 264, 384),
              (512, 256, 3584), (1000, 1000, 640)]

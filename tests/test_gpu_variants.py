@@ -76,9 +76,9 @@ def _fp16_weights(N, K, seed):
     return (zi.weight(N, K, seed=seed, device="cuda", outliers=True) * 4).to(torch.float16).contiguous()
 
 
-@pytest.mark.parametrize("M", (1, 3, 8, 9, 16, 17, 64, 130, 300))
+@pytest.mark.parametrize("M", (1, 3, 8, 9, 16, 17, 32, 33, 64, 130, 300))
 def test_fp16_weights_linear(zq, orc, M):
-    """bits = 16: decode kernel for M <= 16, tile kernel above (TMA-fed W)."""
+    """bits = 16: decode kernel for M <= 32, tile kernel above (TMA-fed W)."""
     for i, (N, K) in enumerate(((1, 128), (130, 512), (520, 1280), (64, 3584))):
         w = _fp16_weights(N, K, 8300 + i)
         x = zi.activations(M, K, seed=8400 + i, device="cuda")
@@ -134,7 +134,7 @@ def _bf16_x(M, K, seed, scale=1.0):
 
 
 @pytest.mark.parametrize("bits", BITS + (16,))
-@pytest.mark.parametrize("M", (1, 8, 16, 40, 300))
+@pytest.mark.parametrize("M", (1, 8, 16, 24, 40, 300))
 def test_bf16_activations(zq, orc, bits, M):
     """Both families; activation scales from 1e-6 to 1e4 per token block (bf16's
     range is fp32's, wider than fp16's)."""

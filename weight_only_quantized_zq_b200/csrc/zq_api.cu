@@ -276,13 +276,13 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     const int off_sz = 0;
     const int off_sx = off_sz + rows * 4 * gps;
     const int x_rows_max = mt == 1 ? max_m : mpad;  // staged token rows (and group records)
-    const int off_x = off_sx + decode_rec_stride(bits) * x_rows_max * 16;
+    const int off_x = off_sx + decode_rec_stride(bits, mt) * x_rows_max * 16;
     const int off_desc = off_x + gps * x_rows_max * 256;
     const int meta_bytes = static_cast<int>(align16(off_desc + 32));
     const int stage = codes_bytes + meta_bytes;
     // Depth: at least 3 stages with as many CTAs per SM as the registers allow
     // (228 KB of shared memory per SM, 1 KB of it reserved per CTA).
-    const int reg_ctas = mt == 1 ? 4 : 3;
+    const int reg_ctas = mt == 1 ? 4 : mt == 2 ? 3 : 2;
     int depth = 0, want_ctas = reg_ctas;
     for (; want_ctas >= 1; --want_ctas) {
         const long long budget = 228 * 1024 / want_ctas - 1024;
@@ -338,7 +338,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         const size_t G = keys[e].K / kGroup;
         const size_t xr = mt == 1 ? keys[e].M : mpad;
         const size_t steps = (G + gps - 1) / gps;  // x' and records are stored by step (whole GPS blocks)
-        off += align256(steps * gps * xr * kGroup * 2) + align256(steps * decode_rec_stride(bits) * xr * 16);
+        off += align256(steps * gps * xr * kGroup * 2) + align256(steps * decode_rec_stride(bits, mt) * xr * 16);
     }
     const size_t part_off = off;
     if (!units) off += align256(static_cast<size_t>(n_chunks) * 2 * slot_floats * 4);
@@ -372,6 +372,8 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
         en.x_bf16 = keys[e].xbf16;
         en.K = keys[e].K;
         en.bits = bits;
+        en.gps = gps;
+        en.rs = decode_rec_stride(bits, mt);
         pp.warp_prefix[e] = wsum;
         wsum += static_cast<long long>(en.x_rows) * G;
     }
@@ -586,7 +588,7 @@ zq_status run_batch(const std::vector<Op> &batch, cudaStream_t stream, size_t *d
     }
     for (const auto &d : batch)
         if (!on_tile(d)) pieces.push_back(d);
-    const int mt_list[2] = {1, 2};
+    const int mt_list[3] = {1, 2, 4};
     for (int bits : bits_list)
         for (int mt : mt_list) {
             std::vector<Op> cls;

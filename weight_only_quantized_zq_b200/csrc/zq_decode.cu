@@ -1,4 +1,4 @@
-// zq_decode.cu — decode kernel (M <= 16): skinny tensor-core GEMM that streams
+// zq_decode.cu — decode kernel (M <= 32): skinny tensor-core GEMM that streams
 // the packed weights exactly once.  (From 17 tokens on the tcgen05 tile kernel
 // of zq_prefill.cu, with a single token tile, streams them faster.)
 //
@@ -130,9 +130,9 @@ __global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepP
         // Both outputs by decode step (GPS groups): [step][token][GPS groups]
         // of x' and [step][token][RS records], so a step's x' and records for
         // all staged tokens are two contiguous blocks (two bulk copies).
-        const int gps = decode_gps(en.bits, 1);
+        const int gps = en.gps;
         const size_t blk = static_cast<size_t>(g / gps) * en.x_rows + t;  // (step, token)
-        float4 *dst = reinterpret_cast<float4 *>(en.sx) + blk * decode_rec_stride(en.bits) + g % gps;
+        float4 *dst = reinterpret_cast<float4 *>(en.sx) + blk * en.rs + g % gps;
         uint16_t *prow = en.xg + (blk * gps + g % gps) * kGroup;
         if (t >= en.M) {
             if (lane == 0) *dst = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -369,10 +369,10 @@ __device__ __forceinline__ int box_row(int g) {
 
 // CTAs per SM the register budget is sized for: with one token tile the
 // host's ring (3 stages) leaves shared memory for 4 CTAs (16 warps per SM,
-// 128 registers each), with two token tiles for 3.
+// 128 registers each), with two token tiles for 3, with four for 2.
 template <int BITS, int MT>
 __host__ __device__ constexpr int decode_min_ctas() {
-    return MT == 1 ? 4 : 3;
+    return MT == 1 ? 4 : MT == 2 ? 3 : 2;
 }
 
 template <int BITS, int MT>
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     constexpr int GB = 16 * BITS;                   // bytes of one row of one group
     constexpr int MPAD = 8 * MT;
     constexpr int SZB = 2 * GPS;                    // bytes of scales (or zeros) of one row per step
-    constexpr int RS = decode_rec_stride(BITS);     // shared-memory record slots per staged token
+    constexpr int RS = decode_rec_stride(BITS, MT); // record slots per staged token
 
     extern __shared__ uint8_t smem_raw[];
     // Swizzled TMA destinations need 1024-byte alignment (the host adds slack).
@@ -949,14 +949,19 @@ static cudaError_t occupancy_t(size_t smem, int *ctas) {
     switch (bits * 16 + mt) {                                          \
         case 2 * 16 + 1: return FN<2, 1>(__VA_ARGS__);                 \
         case 2 * 16 + 2: return FN<2, 2>(__VA_ARGS__);                 \
+        case 2 * 16 + 4: return FN<2, 4>(__VA_ARGS__);                 \
         case 3 * 16 + 1: return FN<3, 1>(__VA_ARGS__);                 \
         case 3 * 16 + 2: return FN<3, 2>(__VA_ARGS__);                 \
+        case 3 * 16 + 4: return FN<3, 4>(__VA_ARGS__);                 \
         case 4 * 16 + 1: return FN<4, 1>(__VA_ARGS__);                 \
         case 4 * 16 + 2: return FN<4, 2>(__VA_ARGS__);                 \
+        case 4 * 16 + 4: return FN<4, 4>(__VA_ARGS__);                 \
         case 8 * 16 + 1: return FN<8, 1>(__VA_ARGS__);                 \
         case 8 * 16 + 2: return FN<8, 2>(__VA_ARGS__);                 \
+        case 8 * 16 + 4: return FN<8, 4>(__VA_ARGS__);                 \
         case 16 * 16 + 1: return FN<16, 1>(__VA_ARGS__);               \
         case 16 * 16 + 2: return FN<16, 2>(__VA_ARGS__);               \
+        case 16 * 16 + 4: return FN<16, 4>(__VA_ARGS__);               \
         default: return cudaErrorInvalidValue;                         \
     }
 

@@ -75,6 +75,7 @@ struct PrepEntry {
     uint16_t *xg;       // [step][x_rows][GPS x 128], chunk-swizzled per group and token; rows >= M are zeros
     float *sx;          // [step][x_rows][RS] x 4: (sum of x, -f * 1024 * sum of scaled x, f, 0); zeros for rows >= M
     int M, x_rows, K, bits;  // x_rows: M with one token tile, else the padded M_pad
+    int gps, rs;             // groups per decode step, record slots per token (decode_gps, decode_rec_stride)
     int x_bf16;              // 1: x holds bfloat16, else fp16
 };
 
@@ -87,15 +88,19 @@ struct PrepParams {
 };
 
 // Decode tiling.  A CTA step covers 64 weight rows x GPS groups; each of the
-// 4 warps computes 16 of the rows.
-__host__ __device__ constexpr int decode_gps(int bits, int) { return bits == 16 ? 1 : bits == 8 ? 2 : 4; }
+// 4 warps computes 16 of the rows.  With four token tiles (up to 32 tokens) a
+// step takes at most 2 groups, so that a stage's activations (GPS x 32 x 256
+// bytes) leave room for a 4-stage ring at 2 CTAs per SM.
+__host__ __device__ constexpr int decode_gps(int bits, int mt) {
+    return bits == 16 ? 1 : (bits == 8 || mt >= 4) ? 2 : 4;
+}
 __host__ __device__ constexpr int decode_seg(int bits, int mt) { return decode_gps(bits, mt) * 16 * bits; }
 // Record slots (16 bytes) per token in a decode step's block of records: one
 // spare slot when GPS > 1, so that the records of tokens 2c (c = 0..3),
 // which a quad of lanes reads at once, start in four different bank quads (a
 // token stride of 4 * 16 = 64 bytes would put all four in the same banks).
-__host__ __device__ constexpr int decode_rec_stride(int bits) {
-    return decode_gps(bits, 1) + (decode_gps(bits, 1) > 1 ? 1 : 0);
+__host__ __device__ constexpr int decode_rec_stride(int bits, int mt) {
+    return decode_gps(bits, mt) + (decode_gps(bits, mt) > 1 ? 1 : 0);
 }
 // Codes of a step land as 128-byte-wide TMA boxes with the 128-byte swizzle
 // when a row segment is a whole number of 128-byte spans.  Otherwise (b = 3:
@@ -114,8 +119,8 @@ __host__ __device__ constexpr int decode_boxes(int bits, int mt) {
 __host__ __device__ constexpr int decode_codes_bytes(int bits, int mt) {
     return 64 * decode_boxes(bits, mt) * decode_box_w(bits, mt);
 }
-// Token tiles of 8 for the decode kernel (M <= kDecodeMaxM).
-inline int mt_for_m(int M) { return M <= 8 ? 1 : 2; }
+// Token tiles of 8 for the decode kernel (M <= kDecodeMaxM): 1, 2 or 4.
+inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : 4; }
 
 cudaError_t launch_quantize_pack(const float *w, int N, int K, int bits, int group, uint32_t *packed,
                                  uint16_t *scales, uint16_t *zeros, int slot,
@@ -174,7 +179,7 @@ cudaError_t encode_tensor_map_2d(CUtensorMap *map, CUtensorMapDataType type, con
 // Largest M handled by the mma.sync decode kernel; larger M goes to the
 // tcgen05 tile kernel (which, with one token tile, also streams the weights
 // once, and from 17 tokens on is the faster of the two).
-constexpr int kDecodeMaxM = 16;
+constexpr int kDecodeMaxM = 32;
 
 // bf16 activations for the tile kernel: each token row of x (M x K bfloat16)
 // scaled by a power of two 2^E (E per row, from the row's largest |x|) and

@@ -1,4 +1,4 @@
-// zq_prefill.cu — tile kernel (M > 16): dequantize-to-shared-memory GEMM on
+// zq_prefill.cu — tile kernel (M > 32): dequantize-to-shared-memory GEMM on
 // the 5th-generation tensor cores (tcgen05, TMEM accumulators, TMA).
 //
 // What it computes: out = x · dequant(W)^T with dequant(W) = q * scale + zero per
