@@ -55,9 +55,13 @@ KERNEL_SOURCES = {
 }
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
-    ("decode", "7b", 1): {
-        "sha256": "de5ba2b057c180a01e9bb424bb070c58dd692ae81c675a7a034337d946fed283",
-        "bytes_per_layer": 125936384,
+    ("decode", "7b", 1): {  # an 8-layer launch
+        "sha256": "42194f35a2c56465b0dfe260d08cae476739ef09e42e3b762faebfe0eff62db2",
+        "bytes_per_layer": 125236736,
+    },
+    ("decode", "7b", 32): {  # a 4-layer launch, four token tiles
+        "sha256": "42194f35a2c56465b0dfe260d08cae476739ef09e42e3b762faebfe0eff62db2",
+        "bytes_per_layer": 128282496,
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
