@@ -520,7 +520,8 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     std::memset(&pg, 0, sizeof(pg));
     pg.n_ops = static_cast<int>(ops.size());
     for (size_t i = 0; i < ops.size(); ++i) pg.ops[i].M = ops[i].M;
-    const int box_rows = prefill_box_rows(pg);  // the plan the launch will run
+    const int plan = prefill_plan(pg, ops[0].bits);  // the plan the launch will run
+    const int box_rows = prefill_box_rows(plan), tok_tile = prefill_tok_tile(plan);
     int tiles = 0;
     for (size_t i = 0; i < ops.size(); ++i) {
         PrefillOp &o = pg.ops[i];
@@ -547,9 +548,9 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
         o.N = ops[i].N;
         o.K = ops[i].K;
         o.gshift = ops[i].bits == 16 ? 2 : (ops[i].group == 32 ? 0 : ops[i].group == 64 ? 1 : 2);
-        o.tok_tiles = (ops[i].M + 255) / 256;
+        o.tok_tiles = (ops[i].M + tok_tile - 1) / tok_tile;
         o.tile0 = tiles;
-        tiles += prefill_tiles(ops[i].M, ops[i].N);
+        tiles += prefill_tiles(ops[i].M, ops[i].N, plan);
     }
     pg.n_tiles = tiles;
     pg.wait_ns = g_wait_ns.load();

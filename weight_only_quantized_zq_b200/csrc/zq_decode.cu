@@ -267,34 +267,20 @@ __device__ __forceinline__ void mma_j(float (&acc)[4], const uint32_t (&w)[2][BI
     }
 }
 
-// One group (16 rows x 128 k) into acc.  With SPLIT the even and odd k-steps
-// run as two independent accumulator chains, halving the dependent MMA
-// latency; worth its four registers only when few token tiles are live.
-template <int BITS, bool SPLIT>
+// One group (16 rows x 128 k) into acc: eight dependent k16 steps.  (Two
+// interleaved accumulator chains measured no faster at one token and 5 %
+// slower at four: their four registers cost more than the shorter chain.)
+template <int BITS>
 __device__ __forceinline__ void mma_group(float (&acc)[4], const uint32_t (&w)[2][BITS], const uint32_t (&xf)[16],
                                           uint32_t magic) {
-    if constexpr (SPLIT) {
-        float acc2[4];
-        mma_j<BITS, 0, true>(acc, w, xf, magic);
-        mma_j<BITS, 1, true>(acc2, w, xf, magic);
-        mma_j<BITS, 2, false>(acc, w, xf, magic);
-        mma_j<BITS, 3, false>(acc2, w, xf, magic);
-        mma_j<BITS, 4, false>(acc, w, xf, magic);
-        mma_j<BITS, 5, false>(acc2, w, xf, magic);
-        mma_j<BITS, 6, false>(acc, w, xf, magic);
-        mma_j<BITS, 7, false>(acc2, w, xf, magic);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) acc[i] += acc2[i];
-    } else {
-        mma_j<BITS, 0, true>(acc, w, xf, magic);
-        mma_j<BITS, 1, false>(acc, w, xf, magic);
-        mma_j<BITS, 2, false>(acc, w, xf, magic);
-        mma_j<BITS, 3, false>(acc, w, xf, magic);
-        mma_j<BITS, 4, false>(acc, w, xf, magic);
-        mma_j<BITS, 5, false>(acc, w, xf, magic);
-        mma_j<BITS, 6, false>(acc, w, xf, magic);
-        mma_j<BITS, 7, false>(acc, w, xf, magic);
-    }
+    mma_j<BITS, 0, true>(acc, w, xf, magic);
+    mma_j<BITS, 1, false>(acc, w, xf, magic);
+    mma_j<BITS, 2, false>(acc, w, xf, magic);
+    mma_j<BITS, 3, false>(acc, w, xf, magic);
+    mma_j<BITS, 4, false>(acc, w, xf, magic);
+    mma_j<BITS, 5, false>(acc, w, xf, magic);
+    mma_j<BITS, 6, false>(acc, w, xf, magic);
+    mma_j<BITS, 7, false>(acc, w, xf, magic);
 }
 
 // The output value rounded to fp16, or to bfloat16 for bf16 activations
@@ -769,7 +755,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                         tot[mt][2 * h + 1] = fmaf(zr[h], __uint_as_float(sb.x), tot[mt][2 * h + 1]);
                 }
                 float acc[4];
-                mma_group<BITS, MT == 1>(acc, wv, xf, magic);
+                mma_group<BITS>(acc, wv, xf, magic);
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     tot[mt][2 * h] =

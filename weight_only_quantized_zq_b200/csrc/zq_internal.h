@@ -151,7 +151,7 @@ struct alignas(64) PrefillOp {
     int M, N, K;
     int gshift;     // log2(group) - 5: groups of 32, 64 or 128 codes
     int out_bf16;   // 1: round the output to bfloat16
-    int tok_tiles;  // ceil(M / 256)
+    int tok_tiles;  // ceil(M / tokens per tile): 256, or 512 in the CTA-pair plan
     int tile0;      // first tile of this op in the launch
 };
 
@@ -165,7 +165,6 @@ struct PrefillGroup {
 static_assert(sizeof(PrefillGroup) <= 32000, "kernel parameter space");
 
 cudaError_t prefill_x_map(CUtensorMap *map, const uint16_t *x, int M, int K);
-int prefill_tiles(int M, int N);
 cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, cudaStream_t stream);
 cudaError_t read_prefill_error(int *err);
 cudaError_t read_decode_error(int *err);

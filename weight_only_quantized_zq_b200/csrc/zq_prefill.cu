@@ -40,6 +40,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <atomic>
+
 #include "zq_device.cuh"
 #include "zq_internal.h"
 #include "zq_prefill.h"
@@ -210,6 +212,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// Split form of tmem_ld32: the load is issued, and its registers are valid
+// only after tmem_wait32 on the same array (which waits for every earlier
+// tcgen05.ld of the thread and ties the registers to the wait, so no use of
+// them moves above it).
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait32(uint32_t (&r)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+                   "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]),
+                   "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]),
+                   "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
     const __half2 h = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<const uint32_t *>(&h);
@@ -224,6 +253,46 @@ __device__ __forceinline__ uint32_t pack_out2(float lo, float hi, int bf16) {
     return pack_half2(lo, hi);
 }
 
+// Epilogue store of 32 accumulator columns (weight rows col0 .. col0 + 31) of
+// token row `tok`: scaled by the token's factor fs (bf16 activations), then
+// fp32 partials (out32), or fp16 / bf16 rounded to nearest even; rows and
+// tokens past the op's N and M are not stored.
+__device__ __forceinline__ void store_cols32(const PrefillOp &op, int tok, int col0, uint32_t (&r)[32], float fs) {
+    if (op.xscale != nullptr) {
+#pragma unroll
+        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * fs);
+    }
+    if (tok >= op.M || col0 >= op.N) return;
+    if (op.out32) {
+        // fp32 partial sums (a K-split shard), not rounded
+        float *dst = op.out32 + static_cast<size_t>(tok) * op.N + col0;
+        if ((op.N % 4) == 0 && col0 + 32 <= op.N) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+                reinterpret_cast<uint4 *>(dst)[q] = make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+        } else {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+                if (col0 + q < op.N) dst[q] = __uint_as_float(r[q]);
+        }
+        return;
+    }
+    uint16_t *dst = op.out + static_cast<size_t>(tok) * op.N + col0;
+    if ((op.N % 8) == 0 && col0 + 32 <= op.N) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
+                pack_out2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]), op.out_bf16),
+                pack_out2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]), op.out_bf16),
+                pack_out2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]), op.out_bf16),
+                pack_out2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]), op.out_bf16));
+    } else {
+#pragma unroll
+        for (int q = 0; q < 32; ++q)
+            if (col0 + q < op.N) dst[q] = static_cast<uint16_t>(pack_out2(__uint_as_float(r[q]), 0.0f, op.out_bf16));
+    }
+}
+
 // Tile t of a launch -> (op, weight-row tile, token tile).  The tiles of op o
 // are [tile0, tile0 + tok_tiles * row_tiles); within an op token tiles vary
 // fastest, so the CTAs working at the same time share one weight tile (L2
@@ -231,7 +300,7 @@ __device__ __forceinline__ uint32_t pack_out2(float lo, float hi, int bf16) {
 struct TileRef {
     int o, n0, t0;
 };
-__device__ __forceinline__ TileRef locate(const PrefillGroup &p, int t) {
+__device__ __forceinline__ TileRef locate(const PrefillGroup &p, int t, int tok_tile = kTokTile) {
     int lo = 0, hi = p.n_ops - 1;  // last op with tile0 <= t
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -240,7 +309,7 @@ __device__ __forceinline__ TileRef locate(const PrefillGroup &p, int t) {
     }
     const int local = t - p.ops[lo].tile0;
     const int tt = p.ops[lo].tok_tiles;
-    return TileRef{lo, (local / tt) * kRowTile, (local % tt) * kTokTile};
+    return TileRef{lo, (local / tt) * kRowTile, (local % tt) * tok_tile};
 }
 
 // True when some code of the group dequantizes past the fp16 range: the top
@@ -790,51 +859,34 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
             const TileRef tr = locate(p, t);
             const PrefillOp &op = p.ops[tr.o];
             const int n0 = tr.n0, t0 = tr.t0;
-            const bool vec = (op.N % 8) == 0;
 #pragma unroll 1
             for (int half = 0; half < (t0 + 128 < op.M ? 2 : 1); ++half) {
                 const int tok = t0 + 128 * half + 32 * warp + lane;
                 // bf16 activations: the token's power-of-two factor undoes the
                 // scaling of the fp16 copy the MMAs read
                 const float fs = (op.xscale != nullptr && tok < op.M) ? op.xscale[tok] : 1.0f;
+                const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile;
+                if constexpr (ONE) {
+                    // 22 warps: no registers for a second buffer
 #pragma unroll 1
-                for (int cc = 0; cc < kRowTile / 32; ++cc) {
-                    uint32_t r[32];
-                    tmem_ld32(tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile + cc * 32, r);
-                    if (op.xscale != nullptr) {
-#pragma unroll
-                        for (int q = 0; q < 32; ++q) r[q] = __float_as_uint(__uint_as_float(r[q]) * fs);
+                    for (int cc = 0; cc < kRowTile / 32; ++cc) {
+                        uint32_t r[32];
+                        tmem_ld32(ta + cc * 32, r);
+                        store_cols32(op, tok, n0 + cc * 32, r, fs);
                     }
-                    const int col0 = n0 + cc * 32;
-                    if (tok < op.M && col0 < op.N && op.out32) {
-                        // fp32 partial sums (a K-split shard), not rounded
-                        float *dst = op.out32 + static_cast<size_t>(tok) * op.N + col0;
-                        if ((op.N % 4) == 0 && col0 + 32 <= op.N) {
-#pragma unroll
-                            for (int q = 0; q < 8; ++q)
-                                reinterpret_cast<uint4 *>(dst)[q] =
-                                    make_uint4(r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 32; ++q)
-                                if (col0 + q < op.N) dst[q] = __uint_as_float(r[q]);
-                        }
-                    } else if (tok < op.M && col0 < op.N) {
-                        uint16_t *dst = op.out + static_cast<size_t>(tok) * op.N + col0;
-                        if (vec && col0 + 32 <= op.N) {
-#pragma unroll
-                            for (int q = 0; q < 4; ++q)
-                                reinterpret_cast<uint4 *>(dst)[q] = make_uint4(
-                                    pack_out2(__uint_as_float(r[8 * q + 0]), __uint_as_float(r[8 * q + 1]), op.out_bf16),
-                                    pack_out2(__uint_as_float(r[8 * q + 2]), __uint_as_float(r[8 * q + 3]), op.out_bf16),
-                                    pack_out2(__uint_as_float(r[8 * q + 4]), __uint_as_float(r[8 * q + 5]), op.out_bf16),
-                                    pack_out2(__uint_as_float(r[8 * q + 6]), __uint_as_float(r[8 * q + 7]), op.out_bf16));
-                        } else {
-#pragma unroll
-                            for (int q = 0; q < 32; ++q)
-                                if (col0 + q < op.N)
-                                    dst[q] = static_cast<uint16_t>(pack_out2(__uint_as_float(r[q]), 0.0f, op.out_bf16));
-                        }
+                } else {
+                    // 32 columns at a time, the next load in flight while the
+                    // previous columns are converted and stored
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32_issue(ta, ra);
+#pragma unroll 1
+                    for (int cc = 0; cc < kRowTile / 32; cc += 2) {
+                        tmem_wait32(ra);
+                        tmem_ld32_issue(ta + (cc + 1) * 32, rb);
+                        store_cols32(op, tok, n0 + cc * 32, ra, fs);
+                        tmem_wait32(rb);
+                        if (cc + 2 < kRowTile / 32) tmem_ld32_issue(ta + (cc + 2) * 32, ra);
+                        store_cols32(op, tok, n0 + (cc + 1) * 32, rb, fs);
                     }
                 }
             }
@@ -860,6 +912,448 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
             atomicExch(p.tile_ctr, 0u);
             atomicExch(p.tile_ctr + 1, 0u);
         }
+    }
+}
+
+// ------------------------------------------------------------ CTA pairs --
+// Pair plan (every launch with some M > 128 and b-bit codes): a cluster of
+// two CTAs on two SMs computes a 512-token x 256-row tile with
+// tcgen05.mma.cta_group::2 (M = 256 tokens, N = 256 weight rows, K = 16).  The
+// pair's MMA takes its A operand (x) 128 token rows from each CTA and its B
+// operand (the dequantized W) 128 weight rows from each CTA, and keeps each
+// CTA's 128 token rows of the accumulator in that CTA's tensor memory.  So each
+// SM dequantizes only its own 128 weight rows of a slab for 512 tokens (two
+// MMA halves of 256): half the dequant work per multiply-add of a 256 x 256
+// one-SM tile, and half its shared-memory operand traffic.
+//
+// Per CTA (rank r of the pair): x slab = tokens t0 + 256h + 128r + [0, 128)
+// for halves h = 0, 1 (two TMA boxes of 128 rows, 32 KB), W slab = rows
+// n0 + 128r + [0, 128) (16 KB).  The even CTA (the leader) issues every MMA.
+// Hand-offs between the two CTAs:
+//   * x: both CTAs' TMA copies complete on the leader's xfull barrier (the
+//     pair form of the tensor copy); the leader announces both CTAs' bytes;
+//   * W: the dequant warps arrive on their own CTA's full barrier; in the
+//     peer one relay thread waits for it and arrives on the leader's pfull
+//     barrier (one cluster-scope release per slab, by a thread with no loads
+//     in flight: a cluster-scope release by the dequant threads themselves
+//     would wait for their prefetch loads of the next block);
+//   * stage free, accumulator full, all MMAs done: the leader's
+//     tcgen05.commit arrives on the barrier of both CTAs (multicast commit);
+//   * accumulator drained: the epilogue warps of both CTAs arrive on the
+//     leader's acc_empty barrier (after tcgen05.wait::ld and the tcgen05
+//     fence, so the leader's next MMAs cannot overwrite unread columns).
+// No TMA copy here multicasts: each CTA loads its own operands.  Tiles are
+// assigned statically (pair c takes tiles c, c + pairs, ...), ops with the
+// longest K first.
+constexpr int kPairTok = 512;      // tokens per pair tile
+constexpr int kPairStages = 4;
+
+struct PairCtl {
+    unsigned long long full[kPairStages];   // both: this CTA's W slab written (kDqWarps arrivals)
+    unsigned long long pfull[kPairStages];  // leader: the peer's W slab written (the peer's relay)
+    unsigned long long xfull[kPairStages];  // leader: x slabs of both CTAs landed (expect_tx + both copies)
+    unsigned long long empty[kPairStages];  // both: the pair's MMAs on the stage completed
+    unsigned long long acc_full;            // both: a tile's last MMA completed
+    unsigned long long acc_empty;           // leader: both CTAs' epilogues drained TMEM (2 x kEpiWarps)
+    unsigned long long mma_done;            // both: every MMA the leader issued has completed
+    uint32_t tmem_base;
+    int abort;
+};
+
+struct PairPlan {
+    static constexpr int kDqWarps = 8;  // thread d: row d / 2 of this CTA's 128, 32-code chunk d % 2
+    static constexpr int kThreads = 32 * (kDqWarp0 + kDqWarps);
+    static constexpr int kSlabX = 2 * kPrefillHalfTokens * kBK * 2;  // 32 KB
+    static constexpr int kSlabW = 128 * kBK * 2;                     // 16 KB
+    static constexpr int kOffW = kPairStages * kSlabX;
+    static constexpr int kOffCtl = kOffW + kPairStages * kSlabW;
+    static constexpr size_t kBytes = kOffCtl + sizeof(PairCtl) + 1024;
+    static_assert(kOffW % 1024 == 0 && kOffCtl % 1024 == 0, "SWIZZLE_128B stages need 1024-byte alignment");
+    static_assert(kBytes <= 232448, "227 KB of shared memory per CTA");
+};
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// Shared::cluster address of the same shared-memory location in CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+// Arrival on a barrier of either CTA of the pair: release at cluster scope
+// (orders this thread's earlier memory operations, and what it acquired,
+// before the arrival for a waiter in the other CTA), or at CTA scope (the
+// ordering the tcgen05 fences already give: tensor-memory reads before the
+// leader's next MMAs).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait_cl(unsigned long long *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Bounded wait, with cluster-scope acquire (CL: the barrier's arrivals
+// release data written by the other CTA's threads) or CTA-scope acquire (TMA
+// bytes, tcgen05 commits, tensor-memory hand-offs).  On a timeout both CTAs
+// of the pair are told to abort (their own flag and the peer's) and
+// ZQ_ERR_TIMEOUT is recorded.
+template <bool CL = false>
+__device__ __noinline__ bool pair_wait(unsigned long long *bar, uint32_t parity, volatile int *abort,
+                                       uint32_t peer_abort, unsigned long long limit) {
+    auto ready = [&]() { return CL ? mbar_try_wait_cl(bar, parity) : mbar_try_wait(bar, parity); };
+    if (ready()) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t it = 1;; ++it) {
+        if (ready()) return true;
+        if ((it & 15u) == 0) {
+            if (*abort) return false;
+            if (globaltimer() - t0 > limit) {
+                *abort = 1;
+                asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(peer_abort), "r"(1) : "memory");
+                atomicExch(&g_prefill_error, 5);  // ZQ_ERR_TIMEOUT
+                return false;
+            }
+        }
+    }
+}
+__device__ __noinline__ void pair_drain(unsigned long long *bar, uint32_t parity) {
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait_cl(bar, parity))
+        if (globaltimer() - t0 > kDrainNs) break;
+}
+
+// Pair form of the 2-D tensor copy: lands in this CTA's shared memory and
+// completes its bytes on `bar`, a barrier of either CTA of the pair (here the
+// leader's).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(void *dst, const void *map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
+        "[%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+        : "memory");
+}
+
+// Instruction descriptor, kind::f16 for the pair: fp16 A and B (K-major), fp32
+// D, M = 256 (tokens, 128 per CTA), N = 256 (weight rows, 128 per CTA).
+constexpr uint32_t kIdescPair = (1u << 4) | (static_cast<uint32_t>(256 >> 3) << 17) |
+                                (static_cast<uint32_t>(256 >> 4) << 24);
+
+__device__ __forceinline__ void umma_pair(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(adesc), "l"(bdesc), "r"(kIdescPair), "r"(accumulate)
+        : "memory");
+}
+// Completion of the leader's MMAs issued so far, arriving on `bar` in both CTAs.
+__device__ __forceinline__ void umma_commit_pair(unsigned long long *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(static_cast<uint16_t>(3))
+        : "memory");
+}
+
+template <int B>
+// 14 warps, one CTA per SM: 128 registers per thread (four warps share a
+// sub-partition's 16K registers).
+__global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(const __grid_constant__ PrefillGroup p) {
+    using P = PairPlan;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sx = base;            // x slabs
+    uint8_t *sw = base + P::kOffW;  // W slabs (this CTA's 128 rows)
+    PairCtl &c = *reinterpret_cast<PairCtl *>(base + P::kOffCtl);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const int pair = static_cast<int>(blockIdx.x >> 1), pairs = static_cast<int>(gridDim.x >> 1);
+    const int n_tiles = p.n_tiles;
+    volatile int *abort = &c.abort;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kPairStages; ++s) {
+            mbar_init(&c.full[s], P::kDqWarps);
+            mbar_init(&c.pfull[s], 1);
+            mbar_init(&c.xfull[s], 1);
+            mbar_init(&c.empty[s], 1);
+        }
+        mbar_init(&c.acc_full, 1);
+        mbar_init(&c.acc_empty, 2 * kEpiWarps);
+        mbar_init(&c.mma_done, 1);
+        c.abort = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == kTmaWarp) {
+        // both CTAs' warp kTmaWarp allocate together: the same 512 columns in each
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&c.tmem_base)),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();  // both CTAs' barriers exist before any arrival from the peer
+    tc_fence_after();
+    const uint32_t tmem = c.tmem_base;
+    const uint32_t peer_abort = peer_addr(&c.abort, rank ^ 1u);
+
+    pdl_wait();  // x may be produced by the previous kernel in the stream
+    pdl_launch_dependents();
+
+    if (warp == kTmaWarp) {
+        if (lane == 0) {
+            uint32_t it = 0;
+            for (int t = pair; t < n_tiles && !*abort; t += pairs) {
+                const TileRef tr = locate(p, t, kPairTok);
+                const PrefillOp &op = p.ops[tr.o];
+                const int slabs = op.K / kBK;
+                const int nh = tr.t0 + 256 < op.M ? 2 : 1;  // token halves that hold tokens
+                bool ok = true;
+                for (int s = 0; s < slabs; ++s, ++it) {
+                    const int st = it % kPairStages;
+                    if (!pair_wait(&c.empty[st], ((it / kPairStages) & 1u) ^ 1u, abort, peer_abort, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    if (rank == 0) mbar_arrive_expect_tx(&c.xfull[st], 2u * nh * (P::kSlabX / 2));
+                    const uint32_t bar = peer_addr(&c.xfull[st], 0);
+                    for (int h = 0; h < nh; ++h)
+                        tma_load_2d_pair(sx + st * P::kSlabX + h * (P::kSlabX / 2), &op.xmap, s * kBK,
+                                         tr.t0 + 256 * h + 128 * static_cast<int>(rank), bar);
+                }
+                if (!ok) break;
+            }
+            // After an abort: the copies still in flight complete on the
+            // leader's barriers; the leader waits for the last stages (the
+            // peer stays until the final cluster barrier).
+            if (rank == 0)
+                for (uint32_t k = 0; k < kPairStages && k < it; ++k) {
+                    const uint32_t j = it - 1 - k;
+                    pair_drain(&c.xfull[j % kPairStages], (j / kPairStages) & 1u);
+                }
+        }
+    } else if (warp == kMmaWarp) {
+        if (lane == 0 && rank == 1) {
+            // Relay: each W slab of this CTA, once written, to the leader's pfull.
+            const uint32_t pfull_leader0 = peer_addr(&c.pfull[0], 0);
+            uint32_t it = 0;
+            bool ok = true;
+            for (int t = pair; t < n_tiles && ok && !*abort; t += pairs) {
+                const int slabs = p.ops[locate(p, t, kPairTok).o].K / kBK;
+                for (int s = 0; s < slabs; ++s, ++it) {
+                    const int st = it % kPairStages;
+                    if (!pair_wait(&c.full[st], (it / kPairStages) & 1u, abort, peer_abort, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(pfull_leader0 + st * static_cast<uint32_t>(sizeof(unsigned long long)));
+                }
+            }
+        }
+        if (lane == 0 && rank == 0) {
+            uint32_t it = 0, tile_i = 0;
+            for (int t = pair; t < n_tiles; t += pairs, ++tile_i) {
+                if (*abort) break;
+                const TileRef tr = locate(p, t, kPairTok);
+                const PrefillOp &op = p.ops[tr.o];
+                const int slabs = op.K / kBK;
+                const bool half1 = tr.t0 + 256 < op.M;
+                if (!pair_wait(&c.acc_empty, (tile_i & 1u) ^ 1u, abort, peer_abort, p.wait_ns)) break;
+                tc_fence_after();
+                bool ok = true;
+                for (int s = 0; s < slabs; ++s, ++it) {
+                    const int st = it % kPairStages;
+                    const uint32_t par = (it / kPairStages) & 1u;
+                    if (!pair_wait(&c.xfull[st], par, abort, peer_abort, p.wait_ns) ||
+                        !pair_wait(&c.full[st], par, abort, peer_abort, p.wait_ns) ||
+                        !pair_wait<true>(&c.pfull[st], par, abort, peer_abort, p.wait_ns)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(sx + st * P::kSlabX);
+                    const uint32_t b0 = smem_u32(sw + st * P::kSlabW);
+#pragma unroll
+                    for (int kk = 0; kk < kBK / 16; ++kk) {
+                        const uint64_t bd = sdesc_sw128(b0 + kk * 32);
+                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
+                        umma_pair(tmem, sdesc_sw128(a0 + kk * 32), bd, acc);
+                        if (half1) umma_pair(tmem + 256, sdesc_sw128(a0 + P::kSlabX / 2 + kk * 32), bd, acc);
+                    }
+                    umma_commit_pair(&c.empty[st]);
+                }
+                if (!ok) break;
+                umma_commit_pair(&c.acc_full);
+            }
+            // Always signalled (even with no MMA issued): both CTAs wait for it
+            // before TMEM is freed and before either CTA exits.
+            umma_commit_pair(&c.mma_done);
+        }
+    } else if (warp >= kDqWarp0) {
+        // Thread d: row d / 2 of this CTA's 128 weight rows, 32-code chunk
+        // d % 2 of every slab.  The codes and (scale | zero << 16) words of a
+        // block (128 codes: two slabs) are loaded into registers three blocks
+        // ahead of their use (register sets A, B and C rotate; two at b = 8),
+        // so that about six slabs of dequant time cover the loads' latency.
+        const int d = threadIdx.x - 32 * kDqWarp0;
+        const int row = d >> 1, ch = d & 1;
+        const uint32_t *rowp = nullptr;
+        const uint16_t *srow = nullptr, *zrow = nullptr;
+        int gsh = 2;
+        // fetch cursor: tile tf, block gf of blocks_f
+        int tf = pair, gf = 0, blocks_f = 0;
+        auto start_tile = [&](int t) {
+            const TileRef tr = locate(p, t, kPairTok);
+            const PrefillOp &op = p.ops[tr.o];
+            gsh = op.gshift;
+            const size_t gs = static_cast<size_t>(op.K) >> (op.gshift + 5);  // scales per row
+            const int r = min(tr.n0 + 128 * static_cast<int>(rank) + row, op.N - 1);
+            rowp = op.packed + static_cast<size_t>(r) * (static_cast<size_t>(op.K) * B / 32);
+            srow = op.scales + static_cast<size_t>(r) * gs;
+            zrow = op.zeros + static_cast<size_t>(r) * gs;
+            blocks_f = op.K / kGroup;
+        };
+        if (tf < n_tiles) start_tile(tf);
+        auto fetch_next = [&](uint32_t (&w)[2][B], uint32_t (&sz)[2]) {
+            if (tf >= n_tiles) return;
+            // slab h of block gf: codes 128gf + 64h + 32ch .. +31, group (4gf + 2h + ch) >> gsh
+#pragma unroll
+            for (int h = 0; h < 2; ++h) load_chunk<B>(w[h], rowp + static_cast<size_t>(4 * gf + 2 * h + ch) * B);
+            const int g0 = (4 * gf + ch) >> gsh, g1 = (4 * gf + 2 + ch) >> gsh;  // one group with groups of 128
+            sz[0] = ldg_u16_nc(srow + g0) | (ldg_u16_nc(zrow + g0) << 16);
+            sz[1] = g1 == g0 ? sz[0] : ldg_u16_nc(srow + g1) | (ldg_u16_nc(zrow + g1) << 16);
+            if (++gf == blocks_f) {
+                gf = 0;
+                tf += pairs;
+                if (tf < n_tiles) start_tile(tf);
+            }
+        };
+        // consume cursor: tile tc, block gc of blocks_c; slab counter it
+        int tc = pair, gc = 0;
+        int blocks_c = tc < n_tiles ? p.ops[locate(p, tc, kPairTok).o].K / kGroup : 0;
+        uint32_t it = 0;
+        auto consume = [&](uint32_t (&w)[2][B], uint32_t (&sz)[2]) -> bool {
+            if (tc >= n_tiles || *abort) return false;
+            uint32_t wc[2][B], szc[2];
+            bool ovf[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+#pragma unroll
+                for (int q = 0; q < B; ++q) wc[h][q] = w[h][q];
+                szc[h] = sz[h];
+                ovf[h] = dequant_overflows<B>(szc[h]);
+            }
+            fetch_next(w, sz);  // the set is free again: load the block two ahead
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {  // the two slabs of this block
+                const int st = it % kPairStages;
+                if (!pair_wait(&c.empty[st], ((it / kPairStages) & 1u) ^ 1u, abort, peer_abort, p.wait_ns))
+                    return false;
+                uint8_t *bs = sw + st * P::kSlabW;
+                uint32_t o[16];
+                dequant_chunk<B>(wc[h], szc[h], o, ovf[h]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int c16 = (4 * ch + j) ^ (row & 7);
+                    *reinterpret_cast<uint4 *>(bs + row * 128 + c16 * 16) =
+                        make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+                }
+                fence_proxy_async();  // the generic writes, visible to the MMA's (async-proxy) reads
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&c.full[st]);
+                ++it;
+            }
+            if (++gc == blocks_c) {
+                gc = 0;
+                tc += pairs;
+                if (tc < n_tiles) blocks_c = p.ops[locate(p, tc, kPairTok).o].K / kGroup;
+            }
+            return true;
+        };
+        uint32_t wA[2][B], szA[2], wB[2][B], szB[2], wC[2][B], szC[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            szA[h] = szB[h] = szC[h] = 0u;
+#pragma unroll
+            for (int q = 0; q < B; ++q) wA[h][q] = wB[h][q] = wC[h][q] = 0u;
+        }
+        fetch_next(wA, szA);
+        fetch_next(wB, szB);
+        if constexpr (B == 8) {
+            // b = 8: twice the code words per block; two sets fit the registers
+#pragma unroll 1
+            while (consume(wA, szA) && consume(wB, szB)) {
+            }
+        } else {
+            fetch_next(wC, szC);
+#pragma unroll 1
+            while (consume(wA, szA) && consume(wB, szB) && consume(wC, szC)) {
+            }
+        }
+    } else if (warp < kEpiWarps) {
+        // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = this CTA's token
+        // rows of each half; columns = the tile's 256 weight rows.
+        const uint32_t acc_empty_leader = peer_addr(&c.acc_empty, 0);
+        uint32_t tile_i = 0;
+        for (int t = pair; t < n_tiles; t += pairs, ++tile_i) {
+            if (*abort) break;
+            if (!pair_wait(&c.acc_full, tile_i & 1u, abort, peer_abort, p.wait_ns)) break;
+            tc_fence_after();
+            const TileRef tr = locate(p, t, kPairTok);
+            const PrefillOp &op = p.ops[tr.o];
+#pragma unroll 1
+            for (int half = 0; half < (tr.t0 + 256 < op.M ? 2 : 1); ++half) {
+                const int tok = tr.t0 + 256 * half + 128 * static_cast<int>(rank) + 32 * warp + lane;
+                const float fs = (op.xscale != nullptr && tok < op.M) ? op.xscale[tok] : 1.0f;
+                // 32 columns at a time, the next load in flight while the
+                // previous columns are converted and stored
+                const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile;
+                uint32_t ra[32], rb[32];
+                tmem_ld32_issue(ta, ra);
+#pragma unroll 1
+                for (int cc = 0; cc < kRowTile / 32; cc += 2) {
+                    tmem_wait32(ra);
+                    tmem_ld32_issue(ta + (cc + 1) * 32, rb);
+                    store_cols32(op, tok, tr.n0 + cc * 32, ra, fs);
+                    tmem_wait32(rb);
+                    if (cc + 2 < kRowTile / 32) tmem_ld32_issue(ta + (cc + 2) * 32, ra);
+                    store_cols32(op, tok, tr.n0 + (cc + 1) * 32, rb, fs);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+        }
+    }
+
+    // Every MMA of the pair has completed before either CTA frees TMEM or
+    // exits (the leader's MMAs read both CTAs' shared memory and write both
+    // CTAs' TMEM).
+    if (warp == kMmaWarp && lane == 0) pair_drain(&c.mma_done, 0u);
+    tc_fence_before();
+    __syncthreads();
+    cluster_sync();
+    if (warp == kTmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -932,19 +1426,72 @@ cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K
                                 static_cast<uint32_t>(box_rows), CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int prefill_tiles(int M, int N) {
-    return ((M + pf::kTokTile - 1) / pf::kTokTile) * ((N + pf::kRowTile - 1) / pf::kRowTile);
-}
-
-int prefill_box_rows(const PrefillGroup &pg) {
+int prefill_plan(const PrefillGroup &pg, int bits) {
     int max_m = 0;
     for (int i = 0; i < pg.n_ops; ++i) max_m = pg.ops[i].M > max_m ? pg.ops[i].M : max_m;
-    return max_m <= kPrefillHalfTokens ? kPrefillHalfTokens : pf::kTokTile;
+    if (max_m <= kPrefillHalfTokens) return kPlanOneHalf;
+    // CTA pairs from 512 tokens: below, a pair tile's second token half is
+    // empty and the one-CTA two-half plan was faster (M = 256: 3.4 against
+    // 5.5 ms on the 28-layer stack)
+    return (bits == 16 || max_m < kPairMinM) ? kPlanTwoHalves : kPlanPair;
+}
+
+int prefill_box_rows(int plan) { return plan == kPlanTwoHalves ? pf::kTokTile : kPrefillHalfTokens; }
+
+int prefill_tok_tile(int plan) { return plan == kPlanPair ? pf::kPairTok : pf::kTokTile; }
+
+int prefill_tiles(int M, int N, int plan) {
+    const int tt = prefill_tok_tile(plan);
+    return ((M + tt - 1) / tt) * ((N + pf::kRowTile - 1) / pf::kRowTile);
+}
+
+// Pair plan: clusters of two CTAs, as many pairs as fit at once (at most one
+// per tile); the count that fits is queried once per bit width.
+template <int B>
+static cudaError_t launch_pair_t(const PrefillGroup &pg, int num_sms, cudaStream_t stream) {
+    constexpr size_t smem = pf::PairPlan::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(pf::prefill_pair_kernel<B>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * (num_sms / 2)));
+    cfg.blockDim = dim3(pf::PairPlan::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    static std::atomic<int> fit{0};
+    int pairs_fit = fit.load();
+    if (pairs_fit == 0) {
+        e = cudaOccupancyMaxActiveClusters(&pairs_fit, pf::prefill_pair_kernel<B>, &cfg);
+        if (e != cudaSuccess) return e;
+        if (pairs_fit < 1) return cudaErrorInvalidConfiguration;
+        fit.store(pairs_fit);
+    }
+    const int pairs = pg.n_tiles < pairs_fit ? pg.n_tiles : pairs_fit;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    return cudaLaunchKernelEx(&cfg, pf::prefill_pair_kernel<B>, pg);
 }
 
 cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, cudaStream_t stream) {
     const int n_ctas = pg.n_tiles < num_sms ? pg.n_tiles : num_sms;
-    if (prefill_box_rows(pg) == kPrefillHalfTokens) {
+    const int plan = prefill_plan(pg, bits);
+    if (plan == kPlanPair) {
+        switch (bits) {
+            case 2: return launch_pair_t<2>(pg, num_sms, stream);
+            case 3: return launch_pair_t<3>(pg, num_sms, stream);
+            case 4: return launch_pair_t<4>(pg, num_sms, stream);
+            default: return launch_pair_t<8>(pg, num_sms, stream);
+        }
+    }
+    if (plan == kPlanOneHalf) {
         switch (bits) {
             case 2: return launch_prefill_t<2, true>(pg, n_ctas, stream);
             case 3: return launch_prefill_t<3, true>(pg, n_ctas, stream);

@@ -1,9 +1,11 @@
-// zq_prefill.h — internal declarations of the tile kernel's two shared-memory
-// plans (zq_prefill.cu).  A launch whose ops all have M <= kPrefillHalfTokens
-// runs the one-token-half plan, whose x tensor maps have boxes of
-// kPrefillHalfTokens rows; any other launch runs the two-half plan with boxes
-// of 256 rows.  The host builds every op's map with prefill_box_rows() of the
-// launch, so maps and plan always agree.
+// zq_prefill.h — internal declarations of the tile kernel's three plans
+// (zq_prefill.cu).  A launch whose ops all have M <= kPrefillHalfTokens runs
+// the one-token-half plan (256-token tiles, x boxes of kPrefillHalfTokens
+// rows); a launch of b-bit codes with some M >= kPairMinM runs the CTA-pair
+// plan (512-token tiles, x boxes of kPrefillHalfTokens rows); any other runs
+// the two-half plan (256-token tiles, x boxes of 256 rows).  The host builds every
+// op's map and tile count from prefill_plan() of the launch, so maps, tiles
+// and plan always agree.
 #pragma once
 #include <cuda.h>
 #include <stdint.h>
@@ -21,8 +23,15 @@ cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K
 // swizzle: the W slab of the tile kernel for bits = 16.
 cudaError_t prefill_w_map(CUtensorMap *map, const uint16_t *w, int N, int K);
 
-// Token rows per x box of a launch: 128 if every op has M <= 128, else 256.
-// Reads only the ops' M, so it may be called before their maps are built.
-int prefill_box_rows(const PrefillGroup &pg);
+constexpr int kPlanOneHalf = 0, kPlanTwoHalves = 1, kPlanPair = 2;
+constexpr int kPairMinM = 512;  // the CTA-pair plan runs launches with some M >= 512
+
+// Plan of a launch from its ops' M (read only; may be called before the maps
+// are built) and bit width.
+int prefill_plan(const PrefillGroup &pg, int bits);
+// Token rows per x box, tokens per tile, and tiles of an M x N op, per plan.
+int prefill_box_rows(int plan);
+int prefill_tok_tile(int plan);
+int prefill_tiles(int M, int N, int plan);
 
 }  // namespace zq
