@@ -939,9 +939,11 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
 //     would wait for their prefetch loads of the next block);
 //   * stage free, accumulator full, all MMAs done: the leader's
 //     tcgen05.commit arrives on the barrier of both CTAs (multicast commit);
-//   * accumulator drained: the epilogue warps of both CTAs arrive on the
-//     leader's acc_empty barrier (after tcgen05.wait::ld and the tcgen05
-//     fence, so the leader's next MMAs cannot overwrite unread columns).
+//   * accumulator half drained: the epilogue warps of both CTAs arrive on
+//     the leader's acc_empty barrier of that token half (after
+//     tcgen05.wait::ld and the tcgen05 fence, so the leader's next MMAs
+//     cannot overwrite unread columns); the halves complete and drain one
+//     after the other, so the epilogue overlaps the MMAs (see the issuer).
 // No TMA copy here multicasts: each CTA loads its own operands.  Tiles are
 // assigned statically (pair c takes tiles c, c + pairs, ...), ops with the
 // longest K first.
@@ -953,8 +955,8 @@ struct PairCtl {
     unsigned long long pfull[kPairStages];  // leader: the peer's W slab written (the peer's relay)
     unsigned long long xfull[kPairStages];  // leader: x slabs of both CTAs landed (expect_tx + both copies)
     unsigned long long empty[kPairStages];  // both: the pair's MMAs on the stage completed
-    unsigned long long acc_full;            // both: a tile's last MMA completed
-    unsigned long long acc_empty;           // leader: both CTAs' epilogues drained TMEM (2 x kEpiWarps)
+    unsigned long long acc_full[2];         // both: token half h of a tile's accumulator complete
+    unsigned long long acc_empty[2];        // leader: half h drained by both CTAs' epilogues (2 x kEpiWarps)
     unsigned long long mma_done;            // both: every MMA the leader issued has completed
     uint32_t tmem_base;
     int abort;
@@ -1095,8 +1097,10 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
             mbar_init(&c.xfull[s], 1);
             mbar_init(&c.empty[s], 1);
         }
-        mbar_init(&c.acc_full, 1);
-        mbar_init(&c.acc_empty, 2 * kEpiWarps);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&c.acc_full[h], 1);
+            mbar_init(&c.acc_empty[h], 2 * kEpiWarps);
+        }
         mbar_init(&c.mma_done, 1);
         c.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -1169,39 +1173,83 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
             }
         }
         if (lane == 0 && rank == 0) {
+            // Order of a tile's MMAs: the first H slabs (H = min(stages,
+            // slabs)) for token half 0, then the same slabs for half 1; the
+            // middle slabs both halves each; the last T slabs again half 0
+            // first (then acc_full[0]), then half 1 (then acc_full[1]).  So
+            // half 0 of the accumulator completes, and is drained, while half
+            // 1's last MMAs run, and the next tile's half-0 MMAs run while
+            // half 1 is drained: the tensor pipe waits for the epilogue only
+            // where a drain outlasts H (or T) slabs of one half's MMAs.
             uint32_t it = 0, tile_i = 0;
-            for (int t = pair; t < n_tiles; t += pairs, ++tile_i) {
+            auto operands = [&](uint32_t j) -> bool {  // stage of slab j filled in both CTAs
+                const int st = j % kPairStages;
+                const uint32_t par = (j / kPairStages) & 1u;
+                if (!pair_wait(&c.xfull[st], par, abort, peer_abort, p.wait_ns) ||
+                    !pair_wait(&c.full[st], par, abort, peer_abort, p.wait_ns) ||
+                    !pair_wait<true>(&c.pfull[st], par, abort, peer_abort, p.wait_ns))
+                    return false;
+                tc_fence_after();
+                return true;
+            };
+            auto mma_half = [&](uint32_t j, int s, int h) {  // slab j (s-th of its tile), token half h
+                const int st = j % kPairStages;
+                const uint32_t a0 = smem_u32(sx + st * P::kSlabX + h * (P::kSlabX / 2));
+                const uint32_t b0 = smem_u32(sw + st * P::kSlabW);
+#pragma unroll
+                for (int kk = 0; kk < kBK / 16; ++kk)
+                    umma_pair(tmem + h * kRowTile, sdesc_sw128(a0 + kk * 32), sdesc_sw128(b0 + kk * 32),
+                              (s > 0 || kk > 0) ? 1u : 0u);
+            };
+            bool ok = true;
+            for (int t = pair; t < n_tiles && ok; t += pairs, ++tile_i) {
                 if (*abort) break;
                 const TileRef tr = locate(p, t, kPairTok);
                 const PrefillOp &op = p.ops[tr.o];
-                const int slabs = op.K / kBK;
+                const int S = op.K / kBK;
                 const bool half1 = tr.t0 + 256 < op.M;
-                if (!pair_wait(&c.acc_empty, (tile_i & 1u) ^ 1u, abort, peer_abort, p.wait_ns)) break;
+                const int H = min(kPairStages, S), T = min(kPairStages, S - H);
+                const uint32_t pe = (tile_i & 1u) ^ 1u;  // parity of the previous tile's drains
+                // head: half 0, then half 1 of slabs [0, H)
+                if (!pair_wait(&c.acc_empty[0], pe, abort, peer_abort, p.wait_ns)) break;
                 tc_fence_after();
-                bool ok = true;
-                for (int s = 0; s < slabs; ++s, ++it) {
-                    const int st = it % kPairStages;
-                    const uint32_t par = (it / kPairStages) & 1u;
-                    if (!pair_wait(&c.xfull[st], par, abort, peer_abort, p.wait_ns) ||
-                        !pair_wait(&c.full[st], par, abort, peer_abort, p.wait_ns) ||
-                        !pair_wait<true>(&c.pfull[st], par, abort, peer_abort, p.wait_ns)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t a0 = smem_u32(sx + st * P::kSlabX);
-                    const uint32_t b0 = smem_u32(sw + st * P::kSlabW);
-#pragma unroll
-                    for (int kk = 0; kk < kBK / 16; ++kk) {
-                        const uint64_t bd = sdesc_sw128(b0 + kk * 32);
-                        const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                        umma_pair(tmem, sdesc_sw128(a0 + kk * 32), bd, acc);
-                        if (half1) umma_pair(tmem + 256, sdesc_sw128(a0 + P::kSlabX / 2 + kk * 32), bd, acc);
-                    }
-                    umma_commit_pair(&c.empty[st]);
+                for (int s = 0; s < H && ok; ++s) {
+                    ok = operands(it + s);
+                    if (ok) mma_half(it + s, s, 0);
                 }
                 if (!ok) break;
-                umma_commit_pair(&c.acc_full);
+                if (H == S) umma_commit_pair(&c.acc_full[0]);
+                if (!pair_wait(&c.acc_empty[1], pe, abort, peer_abort, p.wait_ns)) break;
+                tc_fence_after();
+                for (int s = 0; s < H; ++s) {
+                    if (half1) mma_half(it + s, s, 1);
+                    umma_commit_pair(&c.empty[(it + s) % kPairStages]);
+                }
+                if (H == S) umma_commit_pair(&c.acc_full[1]);
+                // middle: both halves per slab
+                for (int s = H; s < S - T && ok; ++s) {
+                    ok = operands(it + s);
+                    if (!ok) break;
+                    mma_half(it + s, s, 0);
+                    if (half1) mma_half(it + s, s, 1);
+                    umma_commit_pair(&c.empty[(it + s) % kPairStages]);
+                }
+                if (!ok) break;
+                // tail: half 0, then half 1 of slabs [S - T, S)
+                if (T > 0) {
+                    for (int s = S - T; s < S && ok; ++s) {
+                        ok = operands(it + s);
+                        if (ok) mma_half(it + s, s, 0);
+                    }
+                    if (!ok) break;
+                    umma_commit_pair(&c.acc_full[0]);
+                    for (int s = S - T; s < S; ++s) {
+                        if (half1) mma_half(it + s, s, 1);
+                        umma_commit_pair(&c.empty[(it + s) % kPairStages]);
+                    }
+                    umma_commit_pair(&c.acc_full[1]);
+                }
+                it += S;
             }
             // Always signalled (even with no MMA issued): both CTAs wait for it
             // before TMEM is freed and before either CTA exits.
@@ -1311,36 +1359,42 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
     } else if (warp < kEpiWarps) {
         // Epilogue warps 0..3: TMEM lanes 32*warp .. +31 = this CTA's token
         // rows of each half; columns = the tile's 256 weight rows.
-        const uint32_t acc_empty_leader = peer_addr(&c.acc_empty, 0);
         uint32_t tile_i = 0;
         for (int t = pair; t < n_tiles; t += pairs, ++tile_i) {
             if (*abort) break;
-            if (!pair_wait(&c.acc_full, tile_i & 1u, abort, peer_abort, p.wait_ns)) break;
-            tc_fence_after();
             const TileRef tr = locate(p, t, kPairTok);
             const PrefillOp &op = p.ops[tr.o];
-#pragma unroll 1
-            for (int half = 0; half < (tr.t0 + 256 < op.M ? 2 : 1); ++half) {
-                const int tok = tr.t0 + 256 * half + 128 * static_cast<int>(rank) + 32 * warp + lane;
-                const float fs = (op.xscale != nullptr && tok < op.M) ? op.xscale[tok] : 1.0f;
-                // 32 columns at a time, the next load in flight while the
-                // previous columns are converted and stored
-                const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile;
-                uint32_t ra[32], rb[32];
-                tmem_ld32_issue(ta, ra);
-#pragma unroll 1
-                for (int cc = 0; cc < kRowTile / 32; cc += 2) {
-                    tmem_wait32(ra);
-                    tmem_ld32_issue(ta + (cc + 1) * 32, rb);
-                    store_cols32(op, tok, tr.n0 + cc * 32, ra, fs);
-                    tmem_wait32(rb);
-                    if (cc + 2 < kRowTile / 32) tmem_ld32_issue(ta + (cc + 2) * 32, ra);
-                    store_cols32(op, tok, tr.n0 + (cc + 1) * 32, rb, fs);
+            const int nh = tr.t0 + 256 < op.M ? 2 : 1;
+            bool ok = true;
+            for (int half = 0; half < 2; ++half) {  // drained in the order the MMAs complete them
+                if (!pair_wait(&c.acc_full[half], tile_i & 1u, abort, peer_abort, p.wait_ns)) {
+                    ok = false;
+                    break;
                 }
+                tc_fence_after();
+                if (half < nh) {
+                    const int tok = tr.t0 + 256 * half + 128 * static_cast<int>(rank) + 32 * warp + lane;
+                    const float fs = (op.xscale != nullptr && tok < op.M) ? op.xscale[tok] : 1.0f;
+                    // 32 columns at a time, the next load in flight while the
+                    // previous columns are converted and stored
+                    const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile;
+                    uint32_t ra[32], rb[32];
+                    tmem_ld32_issue(ta, ra);
+#pragma unroll 1
+                    for (int cc = 0; cc < kRowTile / 32; cc += 2) {
+                        tmem_wait32(ra);
+                        tmem_ld32_issue(ta + (cc + 1) * 32, rb);
+                        store_cols32(op, tok, tr.n0 + cc * 32, ra, fs);
+                        tmem_wait32(rb);
+                        if (cc + 2 < kRowTile / 32) tmem_ld32_issue(ta + (cc + 2) * 32, ra);
+                        store_cols32(op, tok, tr.n0 + (cc + 1) * 32, rb, fs);
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_remote(peer_addr(&c.acc_empty[half], 0));
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_remote(acc_empty_leader);
+            if (!ok) break;
         }
     }
 
