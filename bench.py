@@ -56,17 +56,22 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {  # an 8-layer launch
-        "sha256": "42194f35a2c56465b0dfe260d08cae476739ef09e42e3b762faebfe0eff62db2",
-        "bytes_per_layer": 125236736,
+        "sha256": "403e4d63108402eeb89e2265b6e8f3acf59063a964e6e62c8dca02ff0d42365c",
+        "bytes_per_layer": 125275296,
     },
     ("decode", "7b", 32): {  # a 4-layer launch, four token tiles
-        "sha256": "42194f35a2c56465b0dfe260d08cae476739ef09e42e3b762faebfe0eff62db2",
-        "bytes_per_layer": 128282496,
+        "sha256": "403e4d63108402eeb89e2265b6e8f3acf59063a964e6e62c8dca02ff0d42365c",
+        "bytes_per_layer": 128300544,
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
-        "sha256": "260f2fe4c7aa0f6d088d2e6e869092dca1d8734c3b4b93f72061af7d315bb0e1",
-        "bytes_per_layer": 130899200,
+        "sha256": "00060dca7b6dd6f28142367337b71a4773558ea7245bb245b15d9bbd3f791cdc",
+        "bytes_per_layer": 130827008,
+    },
+    # tile kernel, CTA-pair plan: a one-layer launch at M = 2048
+    ("prefill", "7b", 2048): {
+        "sha256": "00060dca7b6dd6f28142367337b71a4773558ea7245bb245b15d9bbd3f791cdc",
+        "bytes_per_layer": 380465408,
     },
 }
 NOMINAL_HBM_GBS = 8000.0
@@ -583,8 +588,13 @@ def run_zq(args):
     achieved = wl.bytes / (ms_step / 1e3) / 1e9
     bits_used = sorted({b for (*_, b) in decode_stack_shapes(args.layers, args.model)}, reverse=True)
     # The tile kernel's shared-memory plan: one token half when every M <= 128.
-    tile_kernel = ("prefill_kernel<" + "|".join(str(b) for b in bits_used)
-                   + (",true> (one-token-half plan)" if M <= 128 else ",false> (two-token-half plan)"))
+    bits_s = "|".join(str(b) for b in bits_used)
+    if M <= 128:
+        tile_kernel = f"prefill_kernel<{bits_s},true> (one-token-half plan)"
+    elif M >= PAIR_MIN_M and 16 not in bits_used:
+        tile_kernel = f"prefill_pair_kernel<{bits_s}> (CTA pairs, tcgen05.mma.cta_group::2)"
+    else:
+        tile_kernel = f"prefill_kernel<{bits_s},false> (two-token-half plan)"
     if M <= 64:
         roofline = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                     "frac": achieved / peaks["hbm_gbs"],
@@ -647,6 +657,7 @@ def run_zq(args):
 
 
 DECODE_MAX_M = 32  # the library runs M <= 32 on the decode kernel
+PAIR_MIN_M = 512   # and launches of b-bit codes with some M >= 512 on the CTA-pair tile kernel
 
 
 def zq_mt(M):
