@@ -29,7 +29,8 @@ def zq():
 
 
 def test_wait_timeout_is_reported_and_recovered(zq, orc):
-    cases = [(1, 3584, 3584), (4, 1024, 2560), (64, 768, 1280), (300, 512, 1024)]  # decode x2, tile x2
+    # decode x2, tile kernel one-half and two-half plans, CTA-pair plan
+    cases = [(1, 3584, 3584), (4, 1024, 2560), (64, 768, 1280), (300, 512, 1024), (600, 520, 1024)]
     data = []
     for i, (M, N, K) in enumerate(cases):
         w = zi.weight(N, K, seed=9600 + i, device="cuda")

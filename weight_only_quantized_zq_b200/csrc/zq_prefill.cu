@@ -930,13 +930,14 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
 // for halves h = 0, 1 (two TMA boxes of 128 rows, 32 KB), W slab = rows
 // n0 + 128r + [0, 128) (16 KB).  The even CTA (the leader) issues every MMA.
 // Hand-offs between the two CTAs:
-//   * x: both CTAs' TMA copies complete on the leader's xfull barrier (the
-//     pair form of the tensor copy); the leader announces both CTAs' bytes;
-//   * W: the dequant warps arrive on their own CTA's full barrier; in the
-//     peer one relay thread waits for it and arrives on the leader's pfull
-//     barrier (one cluster-scope release per slab, by a thread with no loads
-//     in flight: a cluster-scope release by the dequant threads themselves
-//     would wait for their prefetch loads of the next block);
+//   * x and W: each CTA's TMA copies complete on its own xfull barrier and
+//     its dequant warps arrive on its own full barrier; in the peer one
+//     relay thread waits for both and arrives on the leader's pfull barrier
+//     (one cluster-scope release per slab, by a thread with no loads in
+//     flight: a cluster-scope release by the dequant threads themselves
+//     would wait for their prefetch loads of the next block).  With every
+//     copy completing in its own CTA, each CTA can drain its own copies
+//     after an abort before it leaves;
 //   * stage free, accumulator full, all MMAs done: the leader's
 //     tcgen05.commit arrives on the barrier of both CTAs (multicast commit);
 //   * accumulator half drained: the epilogue warps of both CTAs arrive on
@@ -952,8 +953,8 @@ constexpr int kPairStages = 4;
 
 struct PairCtl {
     unsigned long long full[kPairStages];   // both: this CTA's W slab written (kDqWarps arrivals)
-    unsigned long long pfull[kPairStages];  // leader: the peer's W slab written (the peer's relay)
-    unsigned long long xfull[kPairStages];  // leader: x slabs of both CTAs landed (expect_tx + both copies)
+    unsigned long long pfull[kPairStages];  // leader: the peer's x and W slabs ready (the peer's relay)
+    unsigned long long xfull[kPairStages];  // both: this CTA's x slab landed (expect_tx + the copies)
     unsigned long long empty[kPairStages];  // both: the pair's MMAs on the stage completed
     unsigned long long acc_full[2];         // both: token half h of a tile's accumulator complete
     unsigned long long acc_empty[2];        // leader: half h drained by both CTAs' epilogues (2 x kEpiWarps)
@@ -1041,17 +1042,6 @@ __device__ __noinline__ void pair_drain(unsigned long long *bar, uint32_t parity
         if (globaltimer() - t0 > kDrainNs) break;
 }
 
-// Pair form of the 2-D tensor copy: lands in this CTA's shared memory and
-// completes its bytes on `bar`, a barrier of either CTA of the pair (here the
-// leader's).  No multicast.
-__device__ __forceinline__ void tma_load_2d_pair(void *dst, const void *map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], "
-        "[%4];" ::"r"(smem_u32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-        : "memory");
-}
-
 // Instruction descriptor, kind::f16 for the pair: fp16 A and B (K-major), fp32
 // D, M = 256 (tokens, 128 per CTA), N = 256 (weight rows, 128 per CTA).
 constexpr uint32_t kIdescPair = (1u << 4) | (static_cast<uint32_t>(256 >> 3) << 17) |
@@ -1137,26 +1127,27 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
                         ok = false;
                         break;
                     }
-                    if (rank == 0) mbar_arrive_expect_tx(&c.xfull[st], 2u * nh * (P::kSlabX / 2));
-                    const uint32_t bar = peer_addr(&c.xfull[st], 0);
+                    mbar_arrive_expect_tx(&c.xfull[st], static_cast<uint32_t>(nh * (P::kSlabX / 2)));
                     for (int h = 0; h < nh; ++h)
-                        tma_load_2d_pair(sx + st * P::kSlabX + h * (P::kSlabX / 2), &op.xmap, s * kBK,
-                                         tr.t0 + 256 * h + 128 * static_cast<int>(rank), bar);
+                        tma_load_2d(sx + st * P::kSlabX + h * (P::kSlabX / 2), &op.xmap, s * kBK,
+                                    tr.t0 + 256 * h + 128 * static_cast<int>(rank), &c.xfull[st]);
                 }
                 if (!ok) break;
             }
-            // After an abort: the copies still in flight complete on the
-            // leader's barriers; the leader waits for the last stages (the
-            // peer stays until the final cluster barrier).
-            if (rank == 0)
-                for (uint32_t k = 0; k < kPairStages && k < it; ++k) {
-                    const uint32_t j = it - 1 - k;
-                    pair_drain(&c.xfull[j % kPairStages], (j / kPairStages) & 1u);
-                }
+            // Copies still in flight (only after an abort) must land before
+            // the CTA can exit: a stage is refilled only after the pair's MMAs
+            // consumed its previous copy, so only the last kPairStages copies
+            // can be pending, one per slot; their barriers complete on the
+            // copies' bytes alone.
+            for (uint32_t k = 0; k < kPairStages && k < it; ++k) {
+                const uint32_t j = it - 1 - k;
+                pair_drain(&c.xfull[j % kPairStages], (j / kPairStages) & 1u);
+            }
         }
     } else if (warp == kMmaWarp) {
         if (lane == 0 && rank == 1) {
-            // Relay: each W slab of this CTA, once written, to the leader's pfull.
+            // Relay: each stage of this CTA, once its x slab has landed and
+            // its W slab is written, to the leader's pfull.
             const uint32_t pfull_leader0 = peer_addr(&c.pfull[0], 0);
             uint32_t it = 0;
             bool ok = true;
@@ -1164,7 +1155,9 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
                 const int slabs = p.ops[locate(p, t, kPairTok).o].K / kBK;
                 for (int s = 0; s < slabs; ++s, ++it) {
                     const int st = it % kPairStages;
-                    if (!pair_wait(&c.full[st], (it / kPairStages) & 1u, abort, peer_abort, p.wait_ns)) {
+                    const uint32_t par = (it / kPairStages) & 1u;
+                    if (!pair_wait(&c.xfull[st], par, abort, peer_abort, p.wait_ns) ||
+                        !pair_wait(&c.full[st], par, abort, peer_abort, p.wait_ns)) {
                         ok = false;
                         break;
                     }
