@@ -1,4 +1,6 @@
-// zq_act.cu — activations given as bfloat16, for the tile kernel.
+// zq_act.cu — activation copies for the tile kernel: bfloat16 activations
+// brought into fp16, and the pair-permuted K order of its one-token-half
+// plan.
 //
 // The tensor cores multiply fp16 by fp16 here (the dequantized weights are
 // fp16: bf16 weights would lose three bits), so bf16 activations are brought
@@ -11,14 +13,41 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "zq_device.cuh"
 #include "zq_internal.h"
 
 namespace zq {
 
 __device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
 
-// One block per token row.
-__global__ void __launch_bounds__(256) bf16_rows_to_f16_kernel(const uint16_t *__restrict__ x, int K,
+// Pair-permuted order of a 32-value chunk (the tile kernel's one-token-half
+// plan): position 2w holds value pair_lo<B>(w), position 2w + 1 value
+// pair_hi<B>(w), the order in which the dequant routine yields its fp16
+// weight pairs, so that it stores them without restoring K order.
+template <int B>
+__device__ __forceinline__ void pair_permute(const uint16_t (&h)[32], uint32_t (&o)[16]) {
+#pragma unroll
+    for (int w = 0; w < 16; ++w)
+        o[w] = static_cast<uint32_t>(h[pair_lo<B>(w)]) | (static_cast<uint32_t>(h[pair_hi<B>(w)]) << 16);
+}
+__device__ __forceinline__ void chunk_out(const uint16_t (&h)[32], int perm_bits, uint4 *dst) {
+    uint32_t o[16];
+    switch (perm_bits) {
+        case 2: pair_permute<2>(h, o); break;
+        case 3: pair_permute<3>(h, o); break;
+        case 4: pair_permute<4>(h, o); break;
+        case 8: pair_permute<8>(h, o); break;
+        default:
+#pragma unroll
+            for (int w = 0; w < 16; ++w) o[w] = static_cast<uint32_t>(h[2 * w]) | (static_cast<uint32_t>(h[2 * w + 1]) << 16);
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) dst[j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+}
+
+// One block per token row: the row scaled to fp16 by 2^E, each 32-value
+// chunk in natural order (perm_bits 0) or pair-permuted for b = perm_bits.
+__global__ void __launch_bounds__(256) bf16_rows_to_f16_kernel(const uint16_t *__restrict__ x, int K, int perm_bits,
                                                               uint16_t *__restrict__ x16, float *__restrict__ f) {
     __shared__ float red[8];
     const size_t row = static_cast<size_t>(blockIdx.x) * K;
@@ -47,23 +76,53 @@ __global__ void __launch_bounds__(256) bf16_rows_to_f16_kernel(const uint16_t *_
     E = max(-40, min(E, 100));
     const float up = __uint_as_float(static_cast<uint32_t>(127 + E) << 23);
     uint4 *dst = reinterpret_cast<uint4 *>(x16 + row);
-    for (int i = threadIdx.x; i < n8; i += blockDim.x) {
-        const uint4 v = src[i];
-        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-        uint32_t o[4];
+    for (int c = threadIdx.x; c < K / 32; c += blockDim.x) {  // one 32-value chunk per thread
+        uint16_t h[32];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const __half2 h = __floats2half2_rn(bf16_bits_to_float(w[j] & 0xFFFFu) * up,
-                                                bf16_bits_to_float(w[j] >> 16) * up);
-            o[j] = *reinterpret_cast<const uint32_t *>(&h);
+        for (int q = 0; q < 4; ++q) {
+            const uint4 v = src[4 * c + q];
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                h[8 * q + 2 * j] = __half_as_ushort(__float2half_rn(bf16_bits_to_float(w[j] & 0xFFFFu) * up));
+                h[8 * q + 2 * j + 1] = __half_as_ushort(__float2half_rn(bf16_bits_to_float(w[j] >> 16) * up));
+            }
         }
-        dst[i] = make_uint4(o[0], o[1], o[2], o[3]);
+        chunk_out(h, perm_bits, dst + 4 * c);
     }
     if (threadIdx.x == 0) f[blockIdx.x] = __uint_as_float(static_cast<uint32_t>(127 - E) << 23);
 }
 
-cudaError_t launch_bf16_rows_to_f16(const uint16_t *x, int M, int K, uint16_t *x16, float *f, cudaStream_t stream) {
-    bf16_rows_to_f16_kernel<<<static_cast<unsigned>(M), 256, 0, stream>>>(x, K, x16, f);
+// fp16 rows, each 32-value chunk pair-permuted for b = bits: one chunk (64
+// bytes) per thread.
+__global__ void __launch_bounds__(256) x_pairperm_kernel(const uint16_t *__restrict__ x, long long chunks, int bits,
+                                                        uint16_t *__restrict__ out) {
+    const long long c = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+    if (c >= chunks) return;
+    const uint4 *src = reinterpret_cast<const uint4 *>(x) + 4 * c;
+    uint16_t h[32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 v = src[q];
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            h[8 * q + 2 * j] = static_cast<uint16_t>(w[j] & 0xFFFFu);
+            h[8 * q + 2 * j + 1] = static_cast<uint16_t>(w[j] >> 16);
+        }
+    }
+    chunk_out(h, bits, reinterpret_cast<uint4 *>(out) + 4 * c);
+}
+
+cudaError_t launch_bf16_rows_to_f16(const uint16_t *x, int M, int K, int perm_bits, uint16_t *x16, float *f,
+                                    cudaStream_t stream) {
+    bf16_rows_to_f16_kernel<<<static_cast<unsigned>(M), 256, 0, stream>>>(x, K, perm_bits, x16, f);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_x_pairperm(const uint16_t *x, int M, int K, int bits, uint16_t *out, cudaStream_t stream) {
+    const long long chunks = static_cast<long long>(M) * (K / 32);
+    x_pairperm_kernel<<<static_cast<unsigned>((chunks + 255) / 256), 256, 0, stream>>>(x, chunks, bits, out);
     return cudaGetLastError();
 }
 

@@ -476,16 +476,30 @@ bool conflicts(const OpRanges &a, const OpRanges &b) {
 // One persistent launch over all tiles of independent prefill ops of one bit
 // width (at most kMaxPrefillOps), ops with the longest K first so that the
 // last tiles handed out are the cheap ones.
-// Workspace bytes of a tile-kernel launch: the fp16 copies (and per-token
-// factors) of its distinct bf16 activations.
+// The one-token-half plan (every M <= 128) with b-bit codes reads each x as a
+// copy whose 32-value chunks are pair-permuted (the order of its dequant
+// routine's fp16 pairs); bf16 activations are copied to fp16 whatever the plan.
+bool prefill_perm(const std::vector<Op> &ops) {
+    int max_m = 0;
+    for (const auto &d : ops) max_m = std::max(max_m, d.M);
+    return !ops.empty() && max_m <= kPrefillHalfTokens && ops[0].bits != 16;
+}
+bool prefill_copies(const Op &d, bool perm) { return d.xbf16 || perm; }
+bool same_x(const Op &a, const Op &b) { return a.x == b.x && a.M == b.M && a.K == b.K && a.xbf16 == b.xbf16; }
+
+// Workspace bytes of a tile-kernel launch: the fp16 copies (and, for bf16
+// activations, per-token factors) of its distinct activations.
 size_t prefill_data_bytes(const std::vector<Op> &ops) {
-    std::vector<const uint16_t *> seen;
+    const bool perm = prefill_perm(ops);
     size_t b = 0;
-    for (const auto &d : ops)
-        if (d.xbf16 && std::find(seen.begin(), seen.end(), d.x) == seen.end()) {
-            seen.push_back(d.x);
-            b += align256(static_cast<size_t>(d.M) * d.K * 2) + align256(static_cast<size_t>(d.M) * 4);
-        }
+    for (size_t i = 0; i < ops.size(); ++i) {
+        const Op &d = ops[i];
+        if (!prefill_copies(d, perm)) continue;
+        bool seen = false;
+        for (size_t j = 0; j < i; ++j) seen = seen || same_x(ops[j], d);
+        if (seen) continue;
+        b += align256(static_cast<size_t>(d.M) * d.K * 2) + (d.xbf16 ? align256(static_cast<size_t>(d.M) * 4) : 0);
+    }
     return b;
 }
 
@@ -496,25 +510,36 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     std::stable_sort(ops.begin(), ops.end(), [](const Op &a, const Op &b) { return a.K > b.K; });
     uint8_t *ws = nullptr;
     if ((st = workspace(stream, prefill_data_bytes(ops), &ws)) != ZQ_OK) return st;
-    // bf16 activations: an fp16 copy per distinct x, scaled per token, in the
-    // workspace (see zq_act.cu); the launch reads the copy.
-    std::vector<std::pair<const uint16_t *, std::pair<uint16_t *, float *>>> conv;
-    if (prefill_data_bytes(ops) > 0) {
-        uint8_t *at = ws + kCounterBytes;
-        for (const auto &d : ops) {
-            if (!d.xbf16) continue;
-            bool known = false;
-            for (const auto &c : conv) known = known || c.first == d.x;
-            if (known) continue;
-            uint16_t *x16 = reinterpret_cast<uint16_t *>(at);
-            at += align256(static_cast<size_t>(d.M) * d.K * 2);
-            float *f = reinterpret_cast<float *>(at);
+    // Activation copies in the workspace (see zq_act.cu), one per distinct x;
+    // the launch reads the copy: bf16 x scaled per token into fp16, and with
+    // the one-token-half plan every 32-value chunk pair-permuted.
+    const bool perm = prefill_perm(ops);
+    struct Copy {
+        const Op *src;
+        uint16_t *x16;
+        float *f;
+    };
+    std::vector<Copy> conv;
+    uint8_t *at = ws + kCounterBytes;
+    for (const auto &d : ops) {
+        if (!prefill_copies(d, perm)) continue;
+        bool known = false;
+        for (const auto &c : conv) known = known || same_x(*c.src, d);
+        if (known) continue;
+        uint16_t *x16 = reinterpret_cast<uint16_t *>(at);
+        at += align256(static_cast<size_t>(d.M) * d.K * 2);
+        float *f = nullptr;
+        cudaError_t e;
+        if (d.xbf16) {
+            f = reinterpret_cast<float *>(at);
             at += align256(static_cast<size_t>(d.M) * 4);
-            cudaError_t e = launch_bf16_rows_to_f16(d.x, d.M, d.K, x16, f, stream);
-            if (e != cudaSuccess) return cuda_fail(e, "bf16 activation launch");
-            g_launches += 1;
-            conv.push_back({d.x, {x16, f}});
+            e = launch_bf16_rows_to_f16(d.x, d.M, d.K, perm ? d.bits : 0, x16, f, stream);
+        } else {
+            e = launch_x_pairperm(d.x, d.M, d.K, d.bits, x16, stream);
         }
+        if (e != cudaSuccess) return cuda_fail(e, "activation copy launch");
+        g_launches += 1;
+        conv.push_back({&d, x16, f});
     }
     PrefillGroup pg;
     std::memset(&pg, 0, sizeof(pg));
@@ -526,12 +551,11 @@ zq_status run_prefill(std::vector<Op> ops, cudaStream_t stream) {
     for (size_t i = 0; i < ops.size(); ++i) {
         PrefillOp &o = pg.ops[i];
         const uint16_t *xa = ops[i].x;
-        if (ops[i].xbf16)
-            for (const auto &c : conv)
-                if (c.first == ops[i].x) {
-                    xa = c.second.first;
-                    o.xscale = c.second.second;
-                }
+        for (const auto &c : conv)
+            if (same_x(*c.src, ops[i])) {
+                xa = c.x16;
+                o.xscale = c.f;  // null for fp16 x
+            }
         o.out_bf16 = ops[i].xbf16;
         cudaError_t e = prefill_x_map_rows(&o.xmap, xa, ops[i].M, ops[i].K, box_rows);
         if (e != cudaSuccess) return cuda_fail(e, "tensor map for x");

@@ -182,8 +182,14 @@ constexpr int kDecodeMaxM = 32;
 
 // bf16 activations for the tile kernel: each token row of x (M x K bfloat16)
 // scaled by a power of two 2^E (E per row, from the row's largest |x|) and
-// rounded to fp16 into x16; f[m] = 2^-E undoes it in the epilogue.
-cudaError_t launch_bf16_rows_to_f16(const uint16_t *x, int M, int K, uint16_t *x16, float *f, cudaStream_t stream);
+// rounded to fp16 into x16, each 32-value chunk in natural order (perm_bits 0)
+// or pair-permuted for b = perm_bits (2, 3, 4, 8); f[m] = 2^-E undoes the
+// scaling in the epilogue.
+cudaError_t launch_bf16_rows_to_f16(const uint16_t *x, int M, int K, int perm_bits, uint16_t *x16, float *f,
+                                    cudaStream_t stream);
+// fp16 x (M x K) -> out with every 32-value chunk pair-permuted for b = bits
+// (the x the tile kernel's one-token-half plan reads).
+cudaError_t launch_x_pairperm(const uint16_t *x, int M, int K, int bits, uint16_t *out, cudaStream_t stream);
 
 // Partial-sum reduction: out[i] = fp16(sum of parts[p][i], p in order).
 constexpr int kMaxReduceParts = 16;

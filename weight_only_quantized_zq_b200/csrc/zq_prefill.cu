@@ -329,10 +329,12 @@ __device__ __forceinline__ uint32_t hmin2_bits(uint32_t a, uint32_t b) {
 }
 
 // Dequantize this thread's 32-code chunk of one W row into 4 x 16 bytes of
-// natural-K-order fp16 (q*s + z, one rounding), via the shared unpack.  In a
-// group that reaches past the fp16 range (`ovf`), values that round to +inf
-// are held at 65504, the largest finite fp16 (a relative change below 2^-11).
-template <int B>
+// fp16 (q*s + z, one rounding), via the shared unpack: in natural K order, or
+// (NATURAL = false) in the pair order of the unpack, word p holding codes
+// pair_lo(p) and pair_hi(p), for an x copy permuted the same way.  In a group
+// that reaches past the fp16 range (`ovf`), values that round to +inf are held
+// at 65504, the largest finite fp16 (a relative change below 2^-11).
+template <int B, bool NATURAL = true>
 __device__ __forceinline__ void dequant_chunk(const uint32_t (&w)[B], uint32_t sz, uint32_t (&o)[16], bool ovf) {
     const uint32_t s2 = (sz & 0xFFFFu) * 0x10001u;  // (s, s)
     const uint32_t z2 = (sz >> 16) * 0x10001u;      // (z, z)
@@ -343,13 +345,18 @@ __device__ __forceinline__ void dequant_chunk(const uint32_t (&w)[B], uint32_t s
 #pragma unroll
         for (int p = 0; p < 16; ++p) v[p] = hmin2_bits(v[p], 0x7BFF7BFFu);
     }
-    // Pairs p (even) and p+1 hold codes (lo, hi) and (lo+1, hi+1): two PRMTs
-    // give the natural pairs (lo, lo+1) and (hi, hi+1).
+    if constexpr (!NATURAL) {
 #pragma unroll
-    for (int p = 0; p < 16; p += 2) {
-        const int lo = pair_lo<B>(p), hi = pair_hi<B>(p);
-        o[lo / 2] = prmt(v[p], v[p + 1], 0x5410u);
-        o[hi / 2] = prmt(v[p], v[p + 1], 0x7632u);
+        for (int p = 0; p < 16; ++p) o[p] = v[p];
+    } else {
+        // Pairs p (even) and p+1 hold codes (lo, hi) and (lo+1, hi+1): two
+        // PRMTs give the natural pairs (lo, lo+1) and (hi, hi+1).
+#pragma unroll
+        for (int p = 0; p < 16; p += 2) {
+            const int lo = pair_lo<B>(p), hi = pair_hi<B>(p);
+            o[lo / 2] = prmt(v[p], v[p + 1], 0x5410u);
+            o[hi / 2] = prmt(v[p], v[p + 1], 0x7632u);
+        }
     }
 }
 
@@ -532,7 +539,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                 }
                 const int row = rows[r];
                 uint32_t o[16];
-                dequant_chunk<B>(w, sz[r][h], o, ovf[r][h]);
+                dequant_chunk<B, false>(w, sz[r][h], o, ovf[r][h]);  // x is pair-permuted
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c16 = (4 * ch + j) ^ (row & 7);
