@@ -235,7 +235,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     DeviceInfo *info = nullptr;
     zq_status st = device_info(&info);
     if (st != ZQ_OK) return st;
-    const int rows = kDecodeCtaRows;
+    const int rows = decode_cta_rows(bits, mt);
     const int mpad = 8 * mt;
     const int gps = decode_gps(bits, mt);
 
@@ -255,7 +255,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     if (keys.size() > static_cast<size_t>(kMaxPrepEntries) || ops.size() > static_cast<size_t>(kMaxDecodeOps))
         return fail(ZQ_ERR_INVALID_ARG, "internal: decode launch too large");
 
-    // Work: CTA steps (op, 64-row block, GPS groups), all of equal cost within
+    // Work: CTA steps (op, row block, GPS groups), all of equal cost within
     // a launch (same bits).
     long long total_steps = 0, total_units = 0;
     int max_m = 1;
@@ -269,7 +269,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     }
     if (total_steps > 0x3FFFFFFFLL) return fail(ZQ_ERR_INVALID_ARG, "decode launch too large (steps)");
 
-    // Stage: codes (64 rows x the box bytes, a multiple of 1024; all
+    // Stage: codes (the step's rows x the box bytes, a multiple of 1024; all
     // stages' codes first, so each starts 1024-aligned), then a meta part of
     // scales and zeros, group sums, activations and the step descriptor.
     const int codes_bytes = decode_codes_bytes(bits, mt);
@@ -282,7 +282,7 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     const int stage = codes_bytes + meta_bytes;
     // Depth: at least 3 stages with as many CTAs per SM as the registers allow
     // (228 KB of shared memory per SM, 1 KB of it reserved per CTA).
-    const int reg_ctas = mt == 1 ? 4 : mt == 2 ? 3 : 2;
+    const int reg_ctas = decode_reg_ctas(bits, mt);
     int depth = 0, want_ctas = reg_ctas;
     for (; want_ctas >= 1; --want_ctas) {
         const long long budget = 228 * 1024 / want_ctas - 1024;

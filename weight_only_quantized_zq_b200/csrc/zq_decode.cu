@@ -22,14 +22,16 @@
 //    so each product is 1024 * x' + 2^E * q * x, and the per-group bias
 //    1024 * sum(x') is subtracted, and 2^E divided out, in fp32 once per group.
 //    The canonical packed layout is consumed as stored.
-//  * A CTA step is 64 weight rows x GPS groups.  One ring of shared-memory
+//  * A CTA step is 64 weight rows (128 with four token tiles and b <= 4) x
+//    GPS groups.  One ring of shared-memory
 //    stages per CTA, filled in turn by the four warps (stage t by warp t % 4,
 //    the scheduling state handed from one producing warp to the next through
 //    shared memory): one TMA 2-D copy per 128-byte column of the codes, with
 //    the 128-byte swizzle so the fragment loads are free of bank conflicts
 //    (one unswizzled 208-byte box at b = 3); bulk copies of the step's
 //    activations and group sums; cp.async for scales and zeros.  All four
-//    warps consume, each 16 of the rows.  A step descriptor travels in the
+//    warps consume, each 16 of the rows (32 with 128-row steps: two row tiles
+//    share every activation fragment).  A step descriptor travels in the
 //    stage, so the consumers keep no scheduling state.
 //  * A persistent grid covers every SM.  The steps of all ops of a launch are
 //    cut into chunks: whole row blocks (large launches, longest first) or
@@ -353,23 +355,17 @@ __device__ __forceinline__ int box_row(int g) {
     else return 2 * (g & 3) + (g >> 2);                                // b = 2 (half-warp phases)
 }
 
-// CTAs per SM the register budget is sized for: with one token tile the
-// host's ring (3 stages) leaves shared memory for 4 CTAs (16 warps per SM,
-// 128 registers each), with two token tiles for 3, with four for 2.
 template <int BITS, int MT>
-__host__ __device__ constexpr int decode_min_ctas() {
-    return MT == 1 ? 4 : MT == 2 ? 3 : 2;
-}
-
-template <int BITS, int MT>
-__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS, MT>())
+__global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_reg_ctas(BITS, MT))
     decode_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int GPS = decode_gps(BITS, MT);
     constexpr int SEG = decode_seg(BITS, MT);       // bytes of one row per step
     constexpr bool SWZ = decode_swizzled(BITS, MT);
     constexpr int BOXW = decode_box_w(BITS, MT);
     constexpr int NBOX = decode_boxes(BITS, MT);
-    constexpr int BOXB = BOXW * kDecodeCtaRows;     // bytes of one TMA box
+    constexpr int RT = decode_row_tiles(BITS, MT);  // row tiles of 16 per warp
+    constexpr int ROWS = decode_cta_rows(BITS, MT); // weight rows per CTA step
+    constexpr int BOXB = BOXW * ROWS;               // bytes of one TMA box
     constexpr int GB = 16 * BITS;                   // bytes of one row of one group
     constexpr int MPAD = 8 * MT;
     constexpr int SZB = 2 * GPS;                    // bytes of scales (or zeros) of one row per step
@@ -481,9 +477,9 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
             if (op.sz_vec) {
                 flags |= kFlagSzVec;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < ROWS / 32; ++h) {
                     const int r = lane + 32 * h;
-                    const int rg = min(ld.rb * kDecodeCtaRows + r, op.N - 1);
+                    const int rg = min(ld.rb * ROWS + r, op.N - 1);
                     const size_t src = static_cast<size_t>(rg) * op.G + g0;
                     uint8_t *dst = sm + p.off_sz + r * 2 * SZB;
                     if constexpr (SZB == 8) {
@@ -508,7 +504,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                 mbar_arrive_expect_tx(&full[slot_ld], NBOX * BOXB + xbytes + sbytes);
 #pragma unroll
                 for (int b = 0; b < NBOX; ++b)
-                    tma_load_2d(st + b * BOXB, &op.tmap, g0 * GB + b * BOXW, ld.rb * kDecodeCtaRows, &full[slot_ld]);
+                    tma_load_2d(st + b * BOXB, &op.tmap, g0 * GB + b * BOXW, ld.rb * ROWS, &full[slot_ld]);
                 const size_t blk = static_cast<size_t>(ld.j) * xrows;  // first (step, token) block
                 bulk_load(sm + p.off_x, op.xg + blk * (GPS * kGroup), xbytes, &full[slot_ld]);
                 bulk_load(sm + p.off_sx, op.sx + blk * (RS * 4), sbytes, &full[slot_ld]);
@@ -548,8 +544,9 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     // ---- consumers (all warps) ---------------------------------------------
     // Per-lane byte offsets into a stage, fixed for the whole kernel (shared
     // memory is addressed with 32-bit offsets from the stage bases).
-    //   codes: the lane's chunk of group gi of row (warp*16 + h*8 + gr) at
-    //          cofs[h][k] + a compile-time part; with the 128-byte swizzle the
+    //   codes: the lane's chunk of group gi of row (warp*16*RT + rt*16 +
+    //          h*8 + gr) at cofs[rt][h][k] + a compile-time part (RT row tiles
+    //          of 16 per warp); with the 128-byte swizzle the
     //          chunk index is ((gi*GB % 128)/16) ^ lanex.
     //   x':    token gq's staged row is GPS*256 bytes, group gi at +gi*256,
     //          the lane's chunk q of it at x_chunk(c, q, gq).
@@ -562,36 +559,45 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
     else if constexpr (BITS == 2) lanex = (c >> 1) ^ gr;
     else if constexpr (BITS == 16) lanex = 4 * (c & 1);  // fp16: box c >> 1, chunks (lanex + j) ^ gr
     else lanex = (2 * c) ^ gr;  // b = 8: chunks lanex and lanex ^ 1
-    uint32_t cofs[2][2];
+    uint32_t cofs[RT][2][2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-        const uint32_t crow = (warp * 16 + h * 8 + gr) * (SWZ ? 128 : BOXW);
-        if constexpr (BITS == 16) {
-            cofs[h][0] = cofs[h][1] = crow + (c >> 1) * BOXB;
-        } else if constexpr (!SWZ) {
-            cofs[h][0] = cofs[h][1] = crow + 4 * BITS * c;
-        } else if constexpr (BITS == 4) {
-            cofs[h][0] = crow + (lanex << 4);
-            cofs[h][1] = crow + ((lanex ^ 4) << 4);
-        } else if constexpr (BITS == 8) {
-            cofs[h][0] = crow + (lanex << 4);
-            cofs[h][1] = crow + ((lanex ^ 1) << 4);
-        } else {  // b = 2: group gi at chunk (2gi ^ lanex), half c & 1
-            cofs[h][0] = cofs[h][1] = crow + 8 * (c & 1);
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t crow = (warp * 16 * RT + rt * 16 + h * 8 + gr) * (SWZ ? 128 : BOXW);
+            uint32_t(&cf)[2] = cofs[rt][h];
+            if constexpr (BITS == 16) {
+                cf[0] = cf[1] = crow + (c >> 1) * BOXB;
+            } else if constexpr (!SWZ) {
+                cf[0] = cf[1] = crow + 4 * BITS * c;
+            } else if constexpr (BITS == 4) {
+                cf[0] = crow + (lanex << 4);
+                cf[1] = crow + ((lanex ^ 4) << 4);
+            } else if constexpr (BITS == 8) {
+                cf[0] = crow + (lanex << 4);
+                cf[1] = crow + ((lanex ^ 1) << 4);
+            } else {  // b = 2: group gi at chunk (2gi ^ lanex), half c & 1
+                cf[0] = cf[1] = crow + 8 * (c & 1);
+            }
         }
-    }
     uint32_t xq[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) xq[q] = p.off_x + gq * (GPS * 256) + (x_chunk(c, q, gq) << 4);
     const uint32_t sxo = p.off_sx + 2 * c * RS * 16;
-    const uint32_t szq0 = p.off_sz + (warp * 16 + gr) * 2 * SZB, szq1 = p.off_sz + (warp * 16 + 8 + gr) * 2 * SZB;
+    uint32_t szq[RT][2];  // scale/zero words of rows warp*16*RT + rt*16 + h*8 + gr
+#pragma unroll
+    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) szq[rt][h] = p.off_sz + (warp * 16 * RT + rt * 16 + h * 8 + gr) * 2 * SZB;
     const uint32_t ring_s = smem_u32(ring), meta_s = smem_u32(meta);
 
-    float tot[MT][4];
+    float tot[MT][RT][4];
 #pragma unroll
     for (int b = 0; b < MT; ++b)
 #pragma unroll
-        for (int i = 0; i < 4; ++i) tot[b][i] = 0.0f;
+        for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) tot[b][rt][i] = 0.0f;
     const uint32_t magic = kMagic;
     // B fragments (activations) of one token tile.  With one tile only the
     // lanes of tokens < M load them; the rest keep stale values (their C
@@ -638,43 +644,48 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
         const int M = static_cast<int>(d1.z);
         const int o = static_cast<int>(d0.x), rb = static_cast<int>(d0.y);
 
-        // Scales and zeros of rows gr and gr + 8 for the GPS groups.
-        uint32_t szs[2][(GPS + 1) / 2], szz[2][(GPS + 1) / 2];
+        // Scales and zeros of rows rt*16 + gr and rt*16 + gr + 8 for the GPS groups.
+        uint32_t szs[RT][2][(GPS + 1) / 2], szz[RT][2][(GPS + 1) / 2];
         if constexpr (BITS == 16) {
             // fp16 weights: no scales or zeros
         } else if (flags & kFlagSzVec) {
-            if constexpr (GPS == 4) {
-                const uint4 v0 = lds_v4(smb + szq0);
-                const uint4 v1 = lds_v4(smb + szq1);
-                szs[0][0] = v0.x; szs[0][1] = v0.y; szz[0][0] = v0.z; szz[0][1] = v0.w;
-                szs[1][0] = v1.x; szs[1][1] = v1.y; szz[1][0] = v1.z; szz[1][1] = v1.w;
-            } else {
-                const uint2 v0 = lds_v2(smb + szq0);
-                const uint2 v1 = lds_v2(smb + szq1);
-                szs[0][0] = v0.x; szz[0][0] = v0.y;
-                szs[1][0] = v1.x; szz[1][0] = v1.y;
-            }
+#pragma unroll
+            for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if constexpr (GPS == 4) {
+                        const uint4 v = lds_v4(smb + szq[rt][h]);
+                        szs[rt][h][0] = v.x; szs[rt][h][1] = v.y; szz[rt][h][0] = v.z; szz[rt][h][1] = v.w;
+                    } else {
+                        const uint2 v = lds_v2(smb + szq[rt][h]);
+                        szs[rt][h][0] = v.x; szz[rt][h][0] = v.y;
+                    }
+                }
         } else {
             const DecodeOp &op = p.ops[o];
             const int g0 = static_cast<int>(d0.z) * GPS;
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int r = min(rb * kDecodeCtaRows + warp * 16 + h * 8 + gr, op.N - 1);
+            for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
-                for (int i = 0; i < GPS / 2; ++i) {
-                    const int ga = min(g0 + 2 * i, op.G - 1), gb = min(g0 + 2 * i + 1, op.G - 1);
-                    const size_t ia = static_cast<size_t>(r) * op.G + ga, ib = static_cast<size_t>(r) * op.G + gb;
-                    szs[h][i] = ldg_u16_nc(op.scales + ia) | (ldg_u16_nc(op.scales + ib) << 16);
-                    szz[h][i] = ldg_u16_nc(op.zeros + ia) | (ldg_u16_nc(op.zeros + ib) << 16);
+                for (int h = 0; h < 2; ++h) {
+                    const int r = min(rb * ROWS + warp * 16 * RT + rt * 16 + h * 8 + gr, op.N - 1);
+#pragma unroll
+                    for (int i = 0; i < GPS / 2; ++i) {
+                        const int ga = min(g0 + 2 * i, op.G - 1), gb = min(g0 + 2 * i + 1, op.G - 1);
+                        const size_t ia = static_cast<size_t>(r) * op.G + ga, ib = static_cast<size_t>(r) * op.G + gb;
+                        szs[rt][h][i] = ldg_u16_nc(op.scales + ia) | (ldg_u16_nc(op.scales + ib) << 16);
+                        szz[rt][h][i] = ldg_u16_nc(op.zeros + ia) | (ldg_u16_nc(op.zeros + ib) << 16);
+                    }
                 }
-            }
         }
 
         auto group = [&](auto gi_c, auto one_c) {
             constexpr int gi = decltype(gi_c)::value;
             constexpr bool one_token = decltype(one_c)::value;
-            // this thread's 32-code chunk of rows gr and gr + 8
-            uint32_t wv[2][BITS];
+            // this thread's 32-code chunk of rows rt*16 + gr and rt*16 + gr + 8
+            uint32_t wv[RT][2][BITS];
+#pragma unroll
+            for (int rt = 0; rt < RT; ++rt)
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
                 if constexpr (BITS == 16) {
@@ -683,47 +694,53 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                     // read the same chunks of the two boxes)
 #pragma unroll
                     for (int j = 0; j < 4; ++j) {
-                        const uint4 v = lds_v4(stb + cofs[h][0] + (((lanex + j) ^ gr) << 4));
-                        wv[h][4 * j] = v.x;
-                        wv[h][4 * j + 1] = v.y;
-                        wv[h][4 * j + 2] = v.z;
-                        wv[h][4 * j + 3] = v.w;
+                        const uint4 v = lds_v4(stb + cofs[rt][h][0] + (((lanex + j) ^ gr) << 4));
+                        wv[rt][h][4 * j] = v.x;
+                        wv[rt][h][4 * j + 1] = v.y;
+                        wv[rt][h][4 * j + 2] = v.z;
+                        wv[rt][h][4 * j + 3] = v.w;
                     }
                 } else if constexpr (SWZ && BITS == 4) {
-                    const uint4 v = lds_v4(stb + cofs[h][gi & 1] + (gi * GB / 128) * BOXB);
-                    wv[h][0] = v.x;
-                    wv[h][1] = v.y;
-                    wv[h][2] = v.z;
-                    wv[h][3] = v.w;
+                    const uint4 v = lds_v4(stb + cofs[rt][h][gi & 1] + (gi * GB / 128) * BOXB);
+                    wv[rt][h][0] = v.x;
+                    wv[rt][h][1] = v.y;
+                    wv[rt][h][2] = v.z;
+                    wv[rt][h][3] = v.w;
                 } else if constexpr (SWZ && BITS == 8) {
-                    const uint4 v0 = lds_v4(stb + cofs[h][0] + gi * BOXB);
-                    const uint4 v1 = lds_v4(stb + cofs[h][1] + gi * BOXB);
-                    wv[h][0] = v0.x; wv[h][1] = v0.y; wv[h][2] = v0.z; wv[h][3] = v0.w;
-                    wv[h][4] = v1.x; wv[h][5] = v1.y; wv[h][6] = v1.z; wv[h][7] = v1.w;
+                    const uint4 v0 = lds_v4(stb + cofs[rt][h][0] + gi * BOXB);
+                    const uint4 v1 = lds_v4(stb + cofs[rt][h][1] + gi * BOXB);
+                    wv[rt][h][0] = v0.x; wv[rt][h][1] = v0.y; wv[rt][h][2] = v0.z; wv[rt][h][3] = v0.w;
+                    wv[rt][h][4] = v1.x; wv[rt][h][5] = v1.y; wv[rt][h][6] = v1.z; wv[rt][h][7] = v1.w;
                 } else if constexpr (SWZ) {
                     static_assert(BITS == 2, "swizzled layouts: b = 2, 4, 8");
-                    const uint2 v = lds_v2(stb + cofs[h][0] + (((2 * gi) ^ lanex) << 4));
-                    wv[h][0] = v.x;
-                    wv[h][1] = v.y;
+                    const uint2 v = lds_v2(stb + cofs[rt][h][0] + (((2 * gi) ^ lanex) << 4));
+                    wv[rt][h][0] = v.x;
+                    wv[rt][h][1] = v.y;
                 } else if constexpr (BITS == 2) {
-                    const uint2 v = lds_v2(stb + cofs[h][0] + gi * GB);
-                    wv[h][0] = v.x;
-                    wv[h][1] = v.y;
+                    const uint2 v = lds_v2(stb + cofs[rt][h][0] + gi * GB);
+                    wv[rt][h][0] = v.x;
+                    wv[rt][h][1] = v.y;
                 } else {
                     static_assert(BITS == 3, "unswizzled layouts: b = 2 (2 groups per step), 3");
-                    wv[h][0] = lds_u32(stb + cofs[h][0] + gi * GB);
-                    wv[h][1] = lds_u32(stb + cofs[h][0] + gi * GB + 4);
-                    wv[h][2] = lds_u32(stb + cofs[h][0] + gi * GB + 8);
+                    wv[rt][h][0] = lds_u32(stb + cofs[rt][h][0] + gi * GB);
+                    wv[rt][h][1] = lds_u32(stb + cofs[rt][h][0] + gi * GB + 4);
+                    wv[rt][h][2] = lds_u32(stb + cofs[rt][h][0] + gi * GB + 8);
                 }
             }
-            float sc[2] = {1.0f, 1.0f}, zr[2] = {0.0f, 0.0f};  // fp16 weights: no scale, no zero
-            if constexpr (BITS != 16) {
-                constexpr bool hi = (gi & 1) != 0;
-                sc[0] = half_of<hi>(szs[0][gi / 2]);
-                sc[1] = half_of<hi>(szs[1][gi / 2]);
-                zr[0] = half_of<hi>(szz[0][gi / 2]);
-                zr[1] = half_of<hi>(szz[1][gi / 2]);
-            }
+            float sc[RT][2], zr[RT][2];
+#pragma unroll
+            for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if constexpr (BITS != 16) {
+                        constexpr bool hi = (gi & 1) != 0;
+                        sc[rt][h] = half_of<hi>(szs[rt][h][gi / 2]);
+                        zr[rt][h] = half_of<hi>(szz[rt][h][gi / 2]);
+                    } else {  // fp16 weights: no scale, no zero
+                        sc[rt][h] = 1.0f;
+                        zr[rt][h] = 0.0f;
+                    }
+                }
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt) {
                 uint32_t xfm[16];
@@ -740,32 +757,35 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                     }
                 }
                 const uint4 sa = lds_v4(smb + sxo + (8 * mt * RS + gi) * 16);
+                uint4 sb = make_uint4(0u, 0u, 0u, 0u);
+                if constexpr (!one_token) sb = lds_v4(smb + sxo + ((8 * mt + 1) * RS + gi) * 16);
                 // tot += s * f * (acc - bias) + z * sum(x): the z * sum(x) term
                 // first (it needs no MMA result, and its operands die early),
                 // then s * f * (acc - bias) with f * (acc - bias) as one FMA (f
                 // is the token's power-of-two x' scale); with one token the odd
-                // C columns are padding.
+                // C columns are padding.  The B fragments serve every row tile.
 #pragma unroll
-                for (int h = 0; h < 2; ++h) tot[mt][2 * h] = fmaf(zr[h], __uint_as_float(sa.x), tot[mt][2 * h]);
-                uint4 sb = make_uint4(0u, 0u, 0u, 0u);
-                if constexpr (!one_token) {
-                    sb = lds_v4(smb + sxo + ((8 * mt + 1) * RS + gi) * 16);
+                for (int rt = 0; rt < RT; ++rt) {
+                    float(&tt)[4] = tot[mt][rt];
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-                        tot[mt][2 * h + 1] = fmaf(zr[h], __uint_as_float(sb.x), tot[mt][2 * h + 1]);
-                }
-                float acc[4];
-                mma_group<BITS>(acc, wv, xf, magic);
+                    for (int h = 0; h < 2; ++h) tt[2 * h] = fmaf(zr[rt][h], __uint_as_float(sa.x), tt[2 * h]);
+                    if constexpr (!one_token) {
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-                    tot[mt][2 * h] =
-                        fmaf(sc[h], fmaf(acc[2 * h], __uint_as_float(sa.z), __uint_as_float(sa.y)), tot[mt][2 * h]);
-                if constexpr (!one_token) {
+                        for (int h = 0; h < 2; ++h) tt[2 * h + 1] = fmaf(zr[rt][h], __uint_as_float(sb.x), tt[2 * h + 1]);
+                    }
+                    float acc[4];
+                    mma_group<BITS>(acc, wv[rt], xf, magic);
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
-                        tot[mt][2 * h + 1] = fmaf(
-                            sc[h], fmaf(acc[2 * h + 1], __uint_as_float(sb.z), __uint_as_float(sb.y)),
-                            tot[mt][2 * h + 1]);
+                        tt[2 * h] = fmaf(sc[rt][h], fmaf(acc[2 * h], __uint_as_float(sa.z), __uint_as_float(sa.y)),
+                                         tt[2 * h]);
+                    if constexpr (!one_token) {
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+                            tt[2 * h + 1] = fmaf(
+                                sc[rt][h], fmaf(acc[2 * h + 1], __uint_as_float(sb.z), __uint_as_float(sb.y)),
+                                tt[2 * h + 1]);
+                    }
                 }
             }
         };
@@ -801,20 +821,22 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
         if (flags & kFlagLast) {
             // End of this chunk's piece of a row block: emit.
             const DecodeOp &op = p.ops[o];
-            const int r0 = rb * kDecodeCtaRows;
+            const int r0 = rb * ROWS;
             if (!(flags & (kFlagHead | kFlagTail))) {
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int row = r0 + warp * 16 + (i >> 1) * 8 + gr;
-                        const int tok = 8 * mt + 2 * c + (i & 1);
-                        if (row < op.N && tok < M) {
-                            const size_t at = static_cast<size_t>(tok) * op.N + row;
-                            if (op.out32) op.out32[at] = tot[mt][i];
-                            else op.out[at] = round_out(tot[mt][i], op.out_bf16);
+                    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int row = r0 + warp * 16 * RT + rt * 16 + (i >> 1) * 8 + gr;
+                            const int tok = 8 * mt + 2 * c + (i & 1);
+                            if (row < op.N && tok < M) {
+                                const size_t at = static_cast<size_t>(tok) * op.N + row;
+                                if (op.out32) op.out32[at] = tot[mt][rt][i];
+                                else op.out[at] = round_out(tot[mt][rt][i], op.out_bf16);
+                            }
                         }
-                    }
             } else {
                 // Partial piece: slot (k, 0) holds chunk k's head piece, (k, 1) its tail piece.
                 const int chunk = d1.x, unit_start = d1.y;
@@ -822,11 +844,13 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
 #pragma unroll
                 for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int rl = warp * 16 + (i >> 1) * 8 + gr;
-                        const int tok = 8 * mt + 2 * c + (i & 1);
-                        if (tok < M) slot_p[rl * M + tok] = tot[mt][i];
-                    }
+                    for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            const int rl = warp * 16 * RT + rt * 16 + (i >> 1) * 8 + gr;
+                            const int tok = 8 * mt + 2 * c + (i & 1);
+                            if (tok < M) slot_p[rl * M + tok] = tot[mt][rt][i];
+                        }
                 const int w_first = unit_start >> p.log2c;               // chunks holding the
                 const int w_last = (unit_start + op.su - 1) >> p.log2c;   // pieces of this row block
                 __threadfence();
@@ -837,7 +861,7 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
                 if (prev == static_cast<unsigned int>(kDecodeWarpsPerCta * (w_last - w_first + 1) - 1)) {
                     // Last piece in: sum the pieces in chunk order (deterministic).
                     __threadfence();
-                    for (int idx = lane; idx < kDecodeCtaRows * M; idx += 32) {
+                    for (int idx = lane; idx < ROWS * M; idx += 32) {
                         float sum = __ldcg(p.part + (static_cast<size_t>(w_first) * 2 + 1) * p.slot_floats + idx);
                         for (int ww = w_first + 1; ww <= w_last; ++ww)
                             sum += __ldcg(p.part + static_cast<size_t>(ww) * 2 * p.slot_floats + idx);
@@ -854,7 +878,9 @@ __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_min_ctas<BITS,
 #pragma unroll
             for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) tot[mt][i] = 0.0f;
+                for (int rt = 0; rt < RT; ++rt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) tot[mt][rt][i] = 0.0f;
         }
     }
 

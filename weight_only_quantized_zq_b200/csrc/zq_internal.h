@@ -18,7 +18,7 @@ constexpr int kQuantStatusSlots = 64;
 // ---------------------------------------------------------------- decode --
 // A decode launch processes up to kMaxDecodeOps independent linear layers of
 // one bit width with M <= kDecodeMaxM.  The work is a sequence of CTA steps, one step =
-// (op, 64-row block, GPS consecutive groups of 128); op o owns steps
+// (op, row block of decode_cta_rows rows, GPS consecutive groups of 128); op o owns steps
 // [step0, step0 + row_blocks * su) in row-block-major order.  The steps are
 // cut into chunks (whole row blocks, or 2^log2c consecutive steps); a CTA
 // starts with chunk blockIdx.x and, in dynamic mode, takes further chunks from
@@ -28,10 +28,9 @@ constexpr int kQuantStatusSlots = 64;
 constexpr int kMaxDecodeOps = 112;
 constexpr int kMaxPrepEntries = 64;
 constexpr int kDecodeWarpsPerCta = 4;
-constexpr int kDecodeCtaRows = 16 * kDecodeWarpsPerCta;  // weight rows per CTA step
 
 struct alignas(64) DecodeOp {
-    CUtensorMap tmap;       // packed codes as a 2-D uint8 tensor: box = 64 rows x box_w bytes
+    CUtensorMap tmap;       // packed codes as a 2-D uint8 tensor: box = decode_cta_rows rows x box_w bytes
     const uint16_t *scales;
     const uint16_t *zeros;
     const uint16_t *xg;     // workspace: pair-permuted, 2^(E-s)-scaled, chunk-swizzled fp16 activations
@@ -56,13 +55,13 @@ struct DecodeParams {
     unsigned int *cnt;       // workspace: [0] chunk counter (reset by prep), [1 + k] pieces of chunk k's row block
     int total_steps;
     int n_ops;
-    int slot_floats;         // 64 rows x M_pad
+    int slot_floats;         // decode_cta_rows x M_pad
     int log2c;               // fixed chunks: 2^log2c consecutive steps
     int n_chunks;
     int units;               // 1: a chunk is one whole row block
     int dynamic;             // 1: chunks beyond the first per CTA are taken from cnt[0]
     int depth;               // ring stages
-    int codes_bytes;         // codes of one stage (64 rows x one step's bytes), multiple of 1024
+    int codes_bytes;         // codes of one stage (decode_cta_rows x one step's bytes), multiple of 1024
     int meta_bytes;          // rest of one stage, multiple of 16
     int off_sz, off_sx, off_x, off_desc;  // offsets inside a stage's meta part
     unsigned long long wait_ns;           // limit of a bounded wait (see wait_limit_ns)
@@ -87,10 +86,22 @@ struct PrepParams {
     PrepEntry e[kMaxPrepEntries];
 };
 
-// Decode tiling.  A CTA step covers 64 weight rows x GPS groups; each of the
-// 4 warps computes 16 of the rows.  With four token tiles (up to 32 tokens) a
-// step takes at most 2 groups, so that a stage's activations (GPS x 32 x 256
-// bytes) leave room for a 4-stage ring at 2 CTAs per SM.
+// Decode tiling.  A CTA step covers 64 x RT weight rows x GPS groups; each of
+// the 4 warps computes RT row tiles of 16.  With one or two token tiles RT = 1
+// and GPS = 4 (2 at b = 8); with four token tiles GPS = 2 and, for b <= 4,
+// RT = 2, so that each activation fragment a warp loads serves 32 weight rows
+// while a stage (128 rows of codes, 2 x 32 x 256 bytes of activations) leaves
+// room for a 3-stage ring at 2 CTAs per SM (b = 8 and fp16 weights, twice the
+// code bytes per row, keep 64-row steps).  M = 17-32 ran 27 % faster with
+// RT = 2; M = 9-16 about 1 % slower, so two token tiles keep RT = 1.
+__host__ __device__ constexpr int decode_row_tiles(int bits, int mt) { return (mt >= 4 && bits <= 4) ? 2 : 1; }
+__host__ __device__ constexpr int decode_cta_rows(int bits, int mt) {
+    return 16 * kDecodeWarpsPerCta * decode_row_tiles(bits, mt);
+}
+// CTAs per SM the decode kernel's registers are budgeted for (its launch
+// bounds) and the host's ring sizing aims at: 4 with one token tile (128
+// registers), 3 with two, 2 with four.
+__host__ __device__ constexpr int decode_reg_ctas(int, int mt) { return mt == 1 ? 4 : mt == 2 ? 3 : 2; }
 __host__ __device__ constexpr int decode_gps(int bits, int mt) {
     return bits == 16 ? 1 : (bits == 8 || mt >= 4) ? 2 : 4;
 }
@@ -115,9 +126,9 @@ __host__ __device__ constexpr int decode_box_w(int bits, int mt) {
 __host__ __device__ constexpr int decode_boxes(int bits, int mt) {
     return decode_swizzled(bits, mt) ? decode_seg(bits, mt) / 128 : 1;
 }
-// Shared-memory bytes of one 64-row stage of codes.
+// Shared-memory bytes of one stage of codes.
 __host__ __device__ constexpr int decode_codes_bytes(int bits, int mt) {
-    return 64 * decode_boxes(bits, mt) * decode_box_w(bits, mt);
+    return decode_cta_rows(bits, mt) * decode_boxes(bits, mt) * decode_box_w(bits, mt);
 }
 // Token tiles of 8 for the decode kernel (M <= kDecodeMaxM): 1, 2 or 4.
 inline int mt_for_m(int M) { return M <= 8 ? 1 : M <= 16 ? 2 : 4; }
