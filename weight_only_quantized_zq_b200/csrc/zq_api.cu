@@ -355,86 +355,100 @@ zq_status run_decode(const std::vector<Op> &ops, int bits, int mt, cudaStream_t 
     }
     uint8_t *data = ws + kCounterBytes;
 
-    PrepParams pp;
-    std::memset(&pp, 0, sizeof(pp));
-    pp.n_entries = static_cast<int>(keys.size());
-    pp.work = reinterpret_cast<unsigned int *>(ws);
-    long long wsum = 0;
-    for (size_t e = 0; e < keys.size(); ++e) {
-        PrepEntry &en = pp.e[e];
-        const size_t G = keys[e].K / kGroup;
-        en.x = keys[e].x;
-        en.xg = reinterpret_cast<uint16_t *>(data + prep_off[e]);
-        en.x_rows = mt == 1 ? keys[e].M : mpad;
-        const size_t steps = (G + gps - 1) / gps;
-        en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(steps * gps * en.x_rows * kGroup * 2));
-        en.M = keys[e].M;
-        en.x_bf16 = keys[e].xbf16;
-        en.K = keys[e].K;
-        en.bits = bits;
-        en.gps = gps;
-        en.rs = decode_rec_stride(bits, mt);
-        pp.warp_prefix[e] = wsum;
-        wsum += static_cast<long long>(en.x_rows) * G;
-    }
-    pp.warp_prefix[keys.size()] = wsum;
+    // The kernels' parameter blocks travel with every launch: launches of few
+    // ops and activations use the small blocks.
+    auto fill_and_launch = [&](auto &pp, auto &dp) -> zq_status {
+        std::memset(&pp, 0, sizeof(pp));
+        pp.n_entries = static_cast<int>(keys.size());
+        pp.work = reinterpret_cast<unsigned int *>(ws);
+        long long wsum = 0;
+        for (size_t e = 0; e < keys.size(); ++e) {
+            PrepEntry &en = pp.e[e];
+            const size_t G = keys[e].K / kGroup;
+            en.x = keys[e].x;
+            en.xg = reinterpret_cast<uint16_t *>(data + prep_off[e]);
+            en.x_rows = mt == 1 ? keys[e].M : mpad;
+            const size_t steps = (G + gps - 1) / gps;
+            en.sx = reinterpret_cast<float *>(data + prep_off[e] + align256(steps * gps * en.x_rows * kGroup * 2));
+            en.M = keys[e].M;
+            en.x_bf16 = keys[e].xbf16;
+            en.K = keys[e].K;
+            en.bits = bits;
+            en.gps = gps;
+            en.rs = decode_rec_stride(bits, mt);
+            pp.warp_prefix[e] = wsum;
+            wsum += static_cast<long long>(en.x_rows) * G;
+        }
+        pp.warp_prefix[keys.size()] = wsum;
 
-    DecodeParams dp;
-    std::memset(&dp, 0, sizeof(dp));
-    dp.part = reinterpret_cast<float *>(data + part_off);
-    dp.cnt = reinterpret_cast<unsigned int *>(ws);
-    dp.total_steps = static_cast<int>(total_steps);
-    dp.n_ops = static_cast<int>(ops.size());
-    dp.slot_floats = slot_floats;
-    dp.log2c = log2c;
-    dp.n_chunks = static_cast<int>(n_chunks);
-    dp.units = units;
-    dp.dynamic = dynamic;
-    dp.depth = depth;
-    dp.codes_bytes = codes_bytes;
-    dp.meta_bytes = meta_bytes;
-    dp.off_sz = off_sz;
-    dp.off_sx = off_sx;
-    dp.off_x = off_x;
-    dp.off_desc = off_desc;
-    dp.wait_ns = g_wait_ns.load();
-    const bool swz = decode_swizzled(bits, mt);
-    int step0 = 0, unit0 = 0;
-    for (size_t oi = 0; oi < ops.size(); ++oi) {
-        const size_t i = order[oi];
-        DecodeOp &o = dp.ops[oi];
-        const PrepEntry &en = pp.e[op_entry[i]];
-        o.scales = ops[i].scales;
-        o.zeros = ops[i].zeros;
-        o.xg = en.xg;
-        o.sx = en.sx;
-        o.out = ops[i].out;
-        o.out32 = ops[i].out32;
-        o.M = ops[i].M;
-        o.N = ops[i].N;
-        o.K = ops[i].K;
-        o.G = ops[i].K / kGroup;
-        o.row_blocks = rbs[i];
-        o.su = sus[i];
-        o.sz_vec = (bits != 16 && (o.G % gps) == 0) ? 1 : 0;  // fp16 weights have no scales or zeros
-        o.out_bf16 = ops[i].xbf16;
-        const uint64_t row_bytes = static_cast<uint64_t>(o.K) * bits / 8;
-        cudaError_t te = encode_tensor_map_2d(&o.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, ops[i].packed, row_bytes,
-                                              static_cast<uint64_t>(o.N), row_bytes,
-                                              static_cast<uint32_t>(decode_box_w(bits, mt)),
-                                              static_cast<uint32_t>(rows),
-                                              swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
-        if (te != cudaSuccess) return cuda_fail(te, "tensor map for the packed codes");
-        o.step0 = step0;
-        o.unit0 = unit0;
-        step0 += rbs[i] * sus[i];
-        unit0 += rbs[i];
-    }
+        std::memset(&dp, 0, sizeof(dp));
+        dp.part = reinterpret_cast<float *>(data + part_off);
+        dp.cnt = reinterpret_cast<unsigned int *>(ws);
+        dp.total_steps = static_cast<int>(total_steps);
+        dp.n_ops = static_cast<int>(ops.size());
+        dp.slot_floats = slot_floats;
+        dp.log2c = log2c;
+        dp.n_chunks = static_cast<int>(n_chunks);
+        dp.units = units;
+        dp.dynamic = dynamic;
+        dp.depth = depth;
+        dp.codes_bytes = codes_bytes;
+        dp.meta_bytes = meta_bytes;
+        dp.off_sz = off_sz;
+        dp.off_sx = off_sx;
+        dp.off_x = off_x;
+        dp.off_desc = off_desc;
+        dp.wait_ns = g_wait_ns.load();
+        const bool swz = decode_swizzled(bits, mt);
+        int step0 = 0, unit0 = 0;
+        for (size_t oi = 0; oi < ops.size(); ++oi) {
+            const size_t i = order[oi];
+            DecodeOp &o = dp.ops[oi];
+            const PrepEntry &en = pp.e[op_entry[i]];
+            o.scales = ops[i].scales;
+            o.zeros = ops[i].zeros;
+            o.xg = en.xg;
+            o.sx = en.sx;
+            o.out = ops[i].out;
+            o.out32 = ops[i].out32;
+            o.M = ops[i].M;
+            o.N = ops[i].N;
+            o.K = ops[i].K;
+            o.G = ops[i].K / kGroup;
+            o.row_blocks = rbs[i];
+            o.su = sus[i];
+            o.sz_vec = (bits != 16 && (o.G % gps) == 0) ? 1 : 0;  // fp16 weights have no scales or zeros
+            o.out_bf16 = ops[i].xbf16;
+            const uint64_t row_bytes = static_cast<uint64_t>(o.K) * bits / 8;
+            cudaError_t te = encode_tensor_map_2d(&o.tmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, ops[i].packed, row_bytes,
+                                                  static_cast<uint64_t>(o.N), row_bytes,
+                                                  static_cast<uint32_t>(decode_box_w(bits, mt)),
+                                                  static_cast<uint32_t>(rows),
+                                                  swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE);
+            if (te != cudaSuccess) return cuda_fail(te, "tensor map for the packed codes");
+            o.step0 = step0;
+            o.unit0 = unit0;
+            step0 += rbs[i] * sus[i];
+            unit0 += rbs[i];
+        }
 
-    cudaError_t e = launch_prep(pp, wsum, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "prep launch");
-    e = launch_decode(dp, bits, mt, n_ctas, smem, stream);
-    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+        cudaError_t e = launch_prep(pp, wsum, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "prep launch");
+        e = launch_decode(dp, bits, mt, n_ctas, smem, stream);
+        if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+        return ZQ_OK;
+    };
+    zq_status fs;
+    if (keys.size() <= static_cast<size_t>(kSmallLaunchOps) && ops.size() <= static_cast<size_t>(kSmallLaunchOps)) {
+        PrepParamsSmall pp;
+        DecodeParamsSmall dp;
+        fs = fill_and_launch(pp, dp);
+    } else {
+        PrepParams pp;
+        DecodeParams dp;
+        fs = fill_and_launch(pp, dp);
+    }
+    if (fs != ZQ_OK) return fs;
     g_launches += 2;
     return ZQ_OK;
 }

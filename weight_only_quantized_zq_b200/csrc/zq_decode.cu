@@ -116,7 +116,8 @@ __device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow
     return bias;
 }
 
-__global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PrepParams p,
+template <class PP>
+__global__ void __launch_bounds__(256) prep_kernel(const __grid_constant__ PP p,
                                                    long long total_warps) {
     pdl_wait();  // x may be the output of the previous kernel in the stream
     if (p.work != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *p.work = 0u;
@@ -196,7 +197,8 @@ struct Cursor {
     bool valid;
 };
 
-__device__ __forceinline__ void cursor_init(Cursor &cu, const DecodeParams &p, int s, int s_end) {
+template <class DP>
+__device__ __forceinline__ void cursor_init(Cursor &cu, const DP &p, int s, int s_end) {
     cu.s = s;
     cu.valid = s < s_end;
     int lo = 0, hi = p.n_ops - 1;  // last op with step0 <= s
@@ -212,7 +214,8 @@ __device__ __forceinline__ void cursor_init(Cursor &cu, const DecodeParams &p, i
     cu.j = local - cu.rb * p.ops[o].su;
 }
 
-__device__ __forceinline__ void cursor_next(Cursor &cu, const DecodeParams &p, int s_end) {
+template <class DP>
+__device__ __forceinline__ void cursor_next(Cursor &cu, const DP &p, int s_end) {
     ++cu.s;
     cu.valid = cu.s < s_end;
     if (++cu.j == p.ops[cu.o].su) {
@@ -225,7 +228,8 @@ __device__ __forceinline__ void cursor_next(Cursor &cu, const DecodeParams &p, i
 }
 
 // Steps [begin, end) of chunk k: one whole row block, or 2^log2c steps.
-__device__ __forceinline__ void chunk_range(const DecodeParams &p, int k, int &begin, int &end) {
+template <class DP>
+__device__ __forceinline__ void chunk_range(const DP &p, int k, int &begin, int &end) {
     if (p.units) {
         int lo = 0, hi = p.n_ops - 1;  // last op with unit0 <= k
         while (lo < hi) {
@@ -355,9 +359,9 @@ __device__ __forceinline__ int box_row(int g) {
     else return 2 * (g & 3) + (g >> 2);                                // b = 2 (half-warp phases)
 }
 
-template <int BITS, int MT>
+template <int BITS, int MT, class DP>
 __global__ void __launch_bounds__(kDecodeWarpsPerCta * 32, decode_reg_ctas(BITS, MT))
-    decode_kernel(const __grid_constant__ DecodeParams p) {
+    decode_kernel(const __grid_constant__ DP p) {
     constexpr int GPS = decode_gps(BITS, MT);
     constexpr int SEG = decode_seg(BITS, MT);       // bytes of one row per step
     constexpr bool SWZ = decode_swizzled(BITS, MT);
@@ -907,7 +911,8 @@ cudaError_t read_decode_error(int *err) {
     return cudaMemcpyToSymbol(g_decode_error, &zero, sizeof(int));
 }
 
-cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream) {
+template <class PP>
+static cudaError_t launch_prep_t(const PP &p, long long total_warps, cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>((total_warps + 7) / 8));
     cfg.blockDim = dim3(256);
@@ -917,24 +922,30 @@ cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prep_kernel, p, total_warps);
+    return cudaLaunchKernelEx(&cfg, prep_kernel<PP>, p, total_warps);
+}
+cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream) {
+    return launch_prep_t(p, total_warps, stream);
+}
+cudaError_t launch_prep(const PrepParamsSmall &p, long long total_warps, cudaStream_t stream) {
+    return launch_prep_t(p, total_warps, stream);
 }
 
 constexpr int kDecodeMaxSmem = 227 * 1024;
 
-template <int BITS, int MT>
+template <int BITS, int MT, class DP>
 static cudaError_t set_smem_t() {
     static bool configured = false;  // benign race: the attribute call is idempotent
     if (configured) return cudaSuccess;
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, MT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<BITS, MT, DP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kDecodeMaxSmem);
     if (e == cudaSuccess) configured = true;
     return e;
 }
 
-template <int BITS, int MT>
-static cudaError_t launch_decode_t(const DecodeParams &p, int n_ctas, size_t smem, cudaStream_t stream) {
-    cudaError_t e = set_smem_t<BITS, MT>();
+template <int BITS, int MT, class DP>
+static cudaError_t launch_decode_t(const DP &p, int n_ctas, size_t smem, cudaStream_t stream) {
+    cudaError_t e = set_smem_t<BITS, MT, DP>();
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
@@ -946,15 +957,15 @@ static cudaError_t launch_decode_t(const DecodeParams &p, int n_ctas, size_t sme
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, MT>, p);
+    return cudaLaunchKernelEx(&cfg, decode_kernel<BITS, MT, DP>, p);
 }
 
 template <int BITS, int MT>
 static cudaError_t occupancy_t(size_t smem, int *ctas) {
-    cudaError_t e = set_smem_t<BITS, MT>();
+    cudaError_t e = set_smem_t<BITS, MT, DecodeParams>();
     if (e != cudaSuccess) return e;
-    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, decode_kernel<BITS, MT>, kDecodeWarpsPerCta * 32,
-                                                         smem);
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas, decode_kernel<BITS, MT, DecodeParams>,
+                                                         kDecodeWarpsPerCta * 32, smem);
 }
 
 #define ZQ_DISPATCH_BITS_MT(FN, ...)                                   \
@@ -978,6 +989,10 @@ static cudaError_t occupancy_t(size_t smem, int *ctas) {
     }
 
 cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream) {
+    ZQ_DISPATCH_BITS_MT(launch_decode_t, p, n_ctas, smem, stream)
+}
+cudaError_t launch_decode(const DecodeParamsSmall &p, int bits, int mt, int n_ctas, size_t smem,
+                          cudaStream_t stream) {
     ZQ_DISPATCH_BITS_MT(launch_decode_t, p, n_ctas, smem, stream)
 }
 

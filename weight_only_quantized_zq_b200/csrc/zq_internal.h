@@ -44,13 +44,17 @@ struct alignas(64) DecodeOp {
     int step0;              // first CTA step of this op
     int unit0;              // first row block of this op (counted over the launch)
     int M, N, K, G;
-    int row_blocks;         // ceil(N / 64)
+    int row_blocks;         // ceil(N / decode_cta_rows)
     int su;                 // steps per row block: ceil(G / GPS)
     int sz_vec;             // G % GPS == 0: a step's scales/zeros of one row are one aligned vector
     int out_bf16;           // 1: out holds bfloat16 (bf16 activations), else fp16
 };
 
-struct DecodeParams {
+// Kernel parameters of a decode launch of at most CAP ops.  They travel with
+// every launch, so launches of few ops use a small block (a 28 KB block cost
+// 2-3 us of latency per single-op call).
+template <int CAP>
+struct DecodeParamsT {
     float *part;             // workspace: 2 partial slots per chunk, slot_floats each
     unsigned int *cnt;       // workspace: [0] chunk counter (reset by prep), [1 + k] pieces of chunk k's row block
     int total_steps;
@@ -65,8 +69,11 @@ struct DecodeParams {
     int meta_bytes;          // rest of one stage, multiple of 16
     int off_sz, off_sx, off_x, off_desc;  // offsets inside a stage's meta part
     unsigned long long wait_ns;           // limit of a bounded wait (see wait_limit_ns)
-    DecodeOp ops[kMaxDecodeOps];
+    DecodeOp ops[CAP];
 };
+constexpr int kSmallLaunchOps = 8;  // ops (and distinct activations) of a small decode launch
+using DecodeParams = DecodeParamsT<kMaxDecodeOps>;
+using DecodeParamsSmall = DecodeParamsT<kSmallLaunchOps>;
 static_assert(sizeof(DecodeParams) <= 32000, "kernel parameter space");
 
 struct PrepEntry {
@@ -78,13 +85,16 @@ struct PrepEntry {
     int x_bf16;              // 1: x holds bfloat16, else fp16
 };
 
-struct PrepParams {
+template <int CAP>
+struct PrepParamsT {
     unsigned int *work;  // decode chunk counter, reset to 0 (may be null)
     int n_entries;
     int pad_;
-    long long warp_prefix[kMaxPrepEntries + 1];  // warps before entry i
-    PrepEntry e[kMaxPrepEntries];
+    long long warp_prefix[CAP + 1];  // warps before entry i
+    PrepEntry e[CAP];
 };
+using PrepParams = PrepParamsT<kMaxPrepEntries>;
+using PrepParamsSmall = PrepParamsT<kSmallLaunchOps>;
 
 // Decode tiling.  A CTA step covers 64 x RT weight rows x GPS groups; each of
 // the 4 warps computes RT row tiles of 16.  With one or two token tiles RT = 1
@@ -208,7 +218,9 @@ cudaError_t launch_reduce_partials(const float *const *parts, int n_parts, size_
                                    cudaStream_t stream);
 
 cudaError_t launch_prep(const PrepParams &p, long long total_warps, cudaStream_t stream);
+cudaError_t launch_prep(const PrepParamsSmall &p, long long total_warps, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeParams &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParamsSmall &p, int bits, int mt, int n_ctas, size_t smem, cudaStream_t stream);
 // CTAs per SM that the registers of decode_kernel<bits, mt> allow with `smem`
 // bytes of dynamic shared memory each.
 cudaError_t decode_ctas_per_sm(int bits, int mt, size_t smem, int *ctas);
