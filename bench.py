@@ -56,22 +56,22 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {  # an 8-layer launch
-        "sha256": "403e4d63108402eeb89e2265b6e8f3acf59063a964e6e62c8dca02ff0d42365c",
-        "bytes_per_layer": 125275296,
+        "sha256": "985d2b20a6c71abc9c5155cadcffdf9ba7dd894c5bb01ed078038aaf69abd10b",
+        "bytes_per_layer": 125688064,
     },
     ("decode", "7b", 32): {  # a 4-layer launch, four token tiles
-        "sha256": "403e4d63108402eeb89e2265b6e8f3acf59063a964e6e62c8dca02ff0d42365c",
-        "bytes_per_layer": 128300544,
+        "sha256": "985d2b20a6c71abc9c5155cadcffdf9ba7dd894c5bb01ed078038aaf69abd10b",
+        "bytes_per_layer": 128164416,
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
-        "sha256": "00060dca7b6dd6f28142367337b71a4773558ea7245bb245b15d9bbd3f791cdc",
-        "bytes_per_layer": 130827008,
+        "sha256": "36e5f33ce31dda93dd4f74bb5c3de7180b760277935e0fc7bb10bafd2006b483",
+        "bytes_per_layer": 133761792,
     },
     # tile kernel, CTA-pair plan: a one-layer launch at M = 2048
     ("prefill", "7b", 2048): {
-        "sha256": "00060dca7b6dd6f28142367337b71a4773558ea7245bb245b15d9bbd3f791cdc",
-        "bytes_per_layer": 380465408,
+        "sha256": "36e5f33ce31dda93dd4f74bb5c3de7180b760277935e0fc7bb10bafd2006b483",
+        "bytes_per_layer": 381255936,
     },
 }
 NOMINAL_HBM_GBS = 8000.0

@@ -34,8 +34,8 @@ def _layer(zq, orc, N, K, bits, seed):
 @pytest.mark.parametrize("P", (2, 4))
 def test_column_parallel(zq, orc, P):
     from weight_only_quantized_zq_b200 import tp
-    for i, (M, N, K, bits) in enumerate(((1, 4608, 3584, 4), (16, 1000, 512, 3), (40, 777, 640, 8),
-                                         (300, 520, 384, 2))):
+    for i, (M, N, K, bits) in enumerate(((1, 4608, 3584, 4), (16, 1000, 512, 3), (24, 600, 1024, 4),
+                                         (40, 777, 640, 8), (300, 520, 384, 2))):
         q, ref = _layer(zq, orc, N, K, bits, 9800 + i)
         x = zi.activations(M, K, 9900 + i, device="cuda")
         slices = [tp.ColumnParallelLinear(*q, N, K, bits, r, P).forward(x) for r in range(P)]
@@ -51,7 +51,7 @@ def test_row_parallel_partial_sums(zq, orc, P):
     zq_reduce_partials; K = 640 gives 5 groups, an uneven split over 4."""
     from weight_only_quantized_zq_b200 import tp
     for i, (M, N, K, bits) in enumerate(((1, 3584, 18944, 4), (4, 512, 3584, 2), (9, 300, 640, 8),
-                                         (40, 300, 1280, 3), (300, 256, 640, 4))):
+                                         (24, 600, 1152, 2), (40, 300, 1280, 3), (300, 256, 640, 4))):
         q, ref = _layer(zq, orc, N, K, bits, 9810 + i)
         x = zi.activations(M, K, 9910 + i, device="cuda")
         shards = [tp.RowParallelLinear(*q, N, K, bits, r, P) for r in range(P)]
