@@ -106,9 +106,10 @@ __device__ __forceinline__ float prep_group(const uint16_t *xrow, uint16_t *prow
     for (int h = 0; h < 2; ++h) {
         const int q = lane + 32 * h;  // 64 pairs per group
         const int c = q / 16, p = q % 16;
-        const float sc = pow2f(E - pair_shift<B>(p));  // exact power of two
-        const __half lo = __float2half_rn(act_bits<BF16>(xrow[32 * c + pair_lo<B>(p)]) * sc);
-        const __half hi = __float2half_rn(act_bits<BF16>(xrow[32 * c + pair_hi<B>(p)]) * sc);
+        // exact powers of two: the codes of the two halves may sit at different offsets
+        const float sl = pow2f(E - pair_shift_lo<B>(p)), sh = pow2f(E - pair_shift_hi<B>(p));
+        const __half lo = __float2half_rn(act_bits<BF16>(xrow[32 * c + pair_lo<B>(p)]) * sl);
+        const __half hi = __float2half_rn(act_bits<BF16>(xrow[32 * c + pair_hi<B>(p)]) * sh);
         bias += __half2float(lo) + __half2float(hi);
         const int word = (x_chunk(c, p >> 2, t7) << 2) | (p & 3);
         reinterpret_cast<uint32_t *>(prow)[word] = __half_as_ushort(lo) | (__half_as_ushort(hi) << 16);

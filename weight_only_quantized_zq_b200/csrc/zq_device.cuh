@@ -208,33 +208,77 @@ __device__ __forceinline__ float half_of(uint32_t w) {
 // b because 32*b bits is a whole number of words).  pair p (0..15) is a half2
 // whose low half is code pair_lo(p) and whose high half is code pair_hi(p).
 
+// b = 3: the 96-bit chunk (code j at stream bits 3j..3j+2) is read through
+// eight 32-bit windows (stream bits n..n+31); pairs 2q and 2q+1 come from
+// window q, their low codes at offsets 4..9 or so of the low half and their
+// high codes in the high half.  The windows at n = 0, 32, 64 are the words
+// themselves, the other five cost one shift each: 21 instructions per 32
+// codes.  Codes (a, b) and (a+1, b+1) of each window keep a and b even, so
+// two PRMTs still restore natural K order from pairs 2q and 2q+1.
+__host__ __device__ constexpr int i3_win(int q) {
+    return q == 0 ? 0 : q == 1 ? 4 : q == 2 ? 10 : q == 3 ? 32 : q == 4 ? 38 : q == 5 ? 56 : q == 6 ? 64 : 74;
+}
+__host__ __device__ constexpr int i3_lo(int q) {
+    return q == 0 ? 0 : q == 1 ? 2 : q == 2 ? 4 : q == 3 ? 12 : q == 4 ? 14 : q == 5 ? 20 : q == 6 ? 22 : 26;
+}
+__host__ __device__ constexpr int i3_hi(int q) {
+    return q == 0 ? 6 : q == 1 ? 8 : q == 2 ? 10 : q == 3 ? 16 : q == 4 ? 18 : q == 5 ? 24 : q == 6 ? 28 : 30;
+}
+
 template <int B>
 __host__ __device__ constexpr int pair_lo(int p) {
     return B == 2 ? 16 * (p / 8) + p % 8
-         : B == 3 ? p
+         : B == 3 ? i3_lo(p / 2) + p % 2
          : B == 4 ? 8 * (p / 4) + p % 4
          : B == 8 ? 4 * (p / 2) + p % 2
                   : 2 * p;  // B = 16 (fp16 weights): word p holds codes 2p, 2p + 1
 }
 template <int B>
 __host__ __device__ constexpr int pair_hi(int p) {
-    return pair_lo<B>(p) + (B == 2 ? 8 : B == 3 ? 16 : B == 4 ? 4 : B == 8 ? 2 : 1);
+    return B == 3 ? i3_hi(p / 2) + p % 2 : pair_lo<B>(p) + (B == 2 ? 8 : B == 4 ? 4 : B == 8 ? 2 : 1);
 }
 
-// fp16x2 constants: magic 1024 in both halves; 2^-s; -1024 * 2^-s.
+// fp16x2 constants: magic 1024 in both halves; (2^-s_lo, 2^-s_hi);
+// (-1024 * 2^-s_lo, -1024 * 2^-s_hi).
 constexpr uint32_t kMagic = 0x64006400u;
-__host__ __device__ constexpr uint32_t mul_s(int s) { return ((15u - s) << 10) * 0x10001u; }
-__host__ __device__ constexpr uint32_t add_s(int s) { return (0x8000u | ((25u - s) << 10)) * 0x10001u; }
+__host__ __device__ constexpr uint32_t mul_s2(int slo, int shi) {
+    return ((15u - slo) << 10) | (((15u - shi) << 10) << 16);
+}
+__host__ __device__ constexpr uint32_t add_s2(int slo, int shi) {
+    return (0x8000u | ((25u - slo) << 10)) | ((0x8000u | ((25u - shi) << 10)) << 16);
+}
 
-// Mantissa offset s of the codes of pair p: the biased pair reads
-// (1024 + q_lo * 2^s, 1024 + q_hi * 2^s).
+// Mantissa offsets of the codes of pair p (low and high half): the biased
+// pair reads (1024 + q_lo * 2^s_lo, 1024 + q_hi * 2^s_hi).  Equal in both
+// halves except at b = 3.
 template <int B>
-__host__ __device__ constexpr int pair_shift(int p) {
+__host__ __device__ constexpr int pair_shift_lo(int p) {
     return B == 2 ? ((p % 8) < 5 ? 2 * (p % 8) : 2 * (p % 8 - 5))
-         : B == 3 ? 3 * (p % 3)
+         : B == 3 ? 3 * pair_lo<3>(p) - i3_win(p / 2)
          : B == 4 ? 4 * (p % 2)
                   : 0;  // b = 8, and fp16 weights (no offset, no bias)
 }
+template <int B>
+__host__ __device__ constexpr int pair_shift_hi(int p) {
+    return B == 3 ? 3 * pair_hi<3>(p) - i3_win(p / 2) - 16 : pair_shift_lo<B>(p);
+}
+
+// Every b = 3 pair: codes inside their window half, offsets 0..7 (so that
+// 1024 + q * 2^s, q <= 7, is exact), and the quads the PRMT restore needs.
+__host__ __device__ constexpr bool i3_table_ok() {
+    unsigned seen = 0;
+    for (int p = 0; p < 16; ++p) {
+        const int lo = pair_lo<3>(p), hi = pair_hi<3>(p);
+        const int slo = pair_shift_lo<3>(p), shi = pair_shift_hi<3>(p);
+        if (slo < 0 || slo > 7 || shi < 0 || shi > 7) return false;
+        if ((seen >> lo) & 1u || (seen >> hi) & 1u) return false;
+        seen |= (1u << lo) | (1u << hi);
+        if (p % 2 == 0 && (lo % 2 != 0 || hi % 2 != 0 || pair_lo<3>(p + 1) != lo + 1 || pair_hi<3>(p + 1) != hi + 1))
+            return false;
+    }
+    return seen == 0xFFFFFFFFu;
+}
+static_assert(i3_table_ok(), "b = 3 pair table");
 
 // Biased pair: one LOP3 (plus a shift shared by several pairs).
 template <int B>
@@ -251,18 +295,16 @@ __device__ __forceinline__ uint32_t unpack_biased<2>(const uint32_t (&w)[2], int
     return lop_and_or(u >> 10, 0x00030003u << (2 * (j - 5)), kMagic);
 }
 
-// b = 3: the chunk is 96 bits; codes p and p+16 are 48 bits apart.  Window m
-// (m = 0..5) joins stream bits [9m, 9m+16) and [9m+48, 9m+64) into one
-// register, where codes 3m+j and 3m+j+16 (j = 0..2) sit at offset 3j of the
-// two halves.
+// b = 3: window q = p / 2 of the 96-bit chunk (stream bits n..n+31, n =
+// i3_win(q)), then one LOP3 keeps the pair's two codes.
+__device__ __forceinline__ uint32_t i3_window(const uint32_t (&w)[3], int n) {
+    return n == 0 ? w[0] : n < 32 ? shf_r(w[0], w[1], n) : n == 32 ? w[1] : n < 64 ? shf_r(w[1], w[2], n - 32)
+                         : n == 64 ? w[2] : (w[2] >> (n - 64));
+}
 template <>
 __device__ __forceinline__ uint32_t unpack_biased<3>(const uint32_t (&w)[3], int p) {
-    const int m = p / 3, j = p % 3;
-    const int a = 9 * m;
-    const uint32_t lo = a < 32 ? shf_r(w[0], w[1], a) : shf_r(w[1], w[2], a - 32);
-    const uint32_t hi = a + 16 < 32 ? shf_r(w[1], w[2], a + 16) : (w[2] >> (a - 16));
-    const uint32_t r = prmt(lo, hi, 0x5410u);
-    return lop_and_or(r, 0x00070007u << (3 * j), kMagic);
+    return lop_and_or(i3_window(w, i3_win(p / 2)),
+                      (0x7u << pair_shift_lo<3>(p)) | (0x7u << (16 + pair_shift_hi<3>(p))), kMagic);
 }
 
 // b = 4: word i holds codes 8i..8i+7 (nibbles); pairs (j, j+4) at mantissa
@@ -289,10 +331,8 @@ __device__ __forceinline__ uint32_t unpack_biased_c(const uint32_t (&w)[B], uint
         if constexpr (j < 5) return lop_and_or_imm<(0x00030003u << (2 * j))>(w[P / 8], magic);
         else return lop_and_or_imm<(0x00030003u << (2 * (j - 5)))>(w[P / 8] >> 10, magic);
     } else if constexpr (B == 3) {
-        constexpr int m = P / 3, j = P % 3, a = 9 * m;
-        const uint32_t lo = a < 32 ? shf_r(w[0], w[1], a) : shf_r(w[1], w[2], a - 32);
-        const uint32_t hi = a + 16 < 32 ? shf_r(w[1], w[2], a + 16) : (w[2] >> (a - 16));
-        return lop_and_or_imm<(0x00070007u << (3 * j))>(prmt(lo, hi, 0x5410u), magic);
+        constexpr uint32_t mask = (0x7u << pair_shift_lo<3>(P)) | (0x7u << (16 + pair_shift_hi<3>(P)));
+        return lop_and_or_imm<mask>(i3_window(w, i3_win(P / 2)), magic);
     } else if constexpr (B == 4) {
         const uint32_t u = (P % 4) < 2 ? w[P / 4] : (w[P / 4] >> 8);
         return lop_and_or_imm<((P % 2) == 0 ? 0x000F000Fu : 0x00F000F0u)>(u, magic);
@@ -305,11 +345,12 @@ __device__ __forceinline__ uint32_t unpack_biased_c(const uint32_t (&w)[B], uint
     }
 }
 
-// Exact codes: one HFMA2 by (2^-s, -1024 * 2^-s) removes bias and offset.
+// Exact codes: one HFMA2 by (2^-s, -1024 * 2^-s), per half, removes bias and
+// offset.
 template <int B>
 __device__ __forceinline__ uint32_t unpack_pair(const uint32_t (&w)[B], int p) {
-    const int s = pair_shift<B>(p);
-    return hfma2_bits(unpack_biased<B>(w, p), mul_s(s), add_s(s));
+    const int slo = pair_shift_lo<B>(p), shi = pair_shift_hi<B>(p);
+    return hfma2_bits(unpack_biased<B>(w, p), mul_s2(slo, shi), add_s2(slo, shi));
 }
 
 }  // namespace zq
