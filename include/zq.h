@@ -135,8 +135,10 @@ ZQ_API zq_status zq_quantize_pack_symmetric(const float *w, int N, int K, int bi
  *   packed/scales/zeros as produced by zq_quantize_pack.
  * M <= 32 runs the decode kernel (mma.sync skinny GEMM streaming the packed
  * weights once through a shared-memory ring); larger M, and groups of 32 or
- * 64 at any M, run the tcgen05 tile kernel (256 x 256 output tiles; with
- * M <= 256 one token tile, so the weights are again streamed once).
+ * 64 at any M, run the tcgen05 tile kernel (256-token x 256-row output tiles,
+ * so at M <= 256 the weights are again streamed once; with b-bit codes and
+ * some M >= 512 in the call, 512 x 256 tiles computed by pairs of CTAs on two
+ * SMs with tcgen05.mma.cta_group::2).
  * bits = 16 is the fp16 passthrough of the .zse format ([wiki] "Формат
  * модели .zse": tensors kept unquantized): `packed` then holds the weights as
  * fp16 N x K, `scales`, `zeros` and `group` are not read (may be NULL / any).
