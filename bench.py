@@ -125,7 +125,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index, period_s=0.005):
+    def __init__(self, device_index, period_s=0.001):
         self.samples, self.reasons, self.max_mhz = [], set(), None
         self.period = period_s
         self._stop = threading.Event()
