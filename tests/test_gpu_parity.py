@@ -303,6 +303,44 @@ def test_stack_against_oracle(zq, orc):
         assert_linear_close(y_out, y_ref, bound, "stack chain")
 
 
+def test_stack_every_route_with_a_chain(zq, orc):
+    """One zq_linear_stack call over every route of the library: the decode
+    kernel with one, two and four token tiles (M = 1, 12, 24), the tile
+    kernel's one-half plan (M = 40), two-half plan (M = 200) and CTA-pair plan
+    (M = 600); plus a chain of three ops at M = 24, each reading the previous
+    op's output: INT4 and INT3 on the decode kernel, then INT2 with groups of
+    64 on the tile kernel."""
+    specs = [(1, 520, 640, 4), (12, 264, 1152, 3), (24, 600, 1024, 2), (40, 300, 640, 8),
+             (200, 264, 384, 4), (600, 520, 512, 3)]
+    layers = [_layer(zq, orc, N, K, b, 110 + i) for i, (M, N, K, b) in enumerate(specs)]
+    xs = [zi.activations(M, K, 120 + i, device="cuda") for i, (M, N, K, b) in enumerate(specs)]
+    outs = [torch.empty(M, N, dtype=torch.float16, device="cuda") for (M, N, K, b) in specs]
+    ops = [(xs[i], *layers[i][0], outs[i], b, 128, M, N, K) for i, (M, N, K, b) in enumerate(specs)]
+    # chain at M = 24: INT4 (K=512 -> 384), then INT3 (384 -> 640), then INT2 with groups of 64 (640 -> 256)
+    qa, ra = _layer(zq, orc, 384, 512, 4, 130)
+    qb, rb = _layer(zq, orc, 640, 384, 3, 131)
+    wc = zi.weight(256, 640, seed=132, device="cuda")
+    qc = zq.quantize(wc, 2, group=64)
+    torch.cuda.synchronize()
+    rc = orc.quantize_pack(wc.cpu().numpy(), 2, group=64)
+    xa = zi.activations(24, 512, 133, device="cuda")
+    ya = torch.empty(24, 384, dtype=torch.float16, device="cuda")
+    yb = torch.empty(24, 640, dtype=torch.float16, device="cuda")
+    yc = torch.empty(24, 256, dtype=torch.float16, device="cuda")
+    ops += [(xa, *qa, ya, 4, 128, 24, 384, 512), (ya, *qb, yb, 3, 128, 24, 640, 384),
+            (yb, *qc, yc, 2, 64, 24, 256, 640)]
+    zq.linear_stack(ops)
+    torch.cuda.synchronize()
+    for i, (M, N, K, b) in enumerate(specs):
+        y_ref, bound = orc.linear(u16(xs[i]), *layers[i][1], b, N, K)
+        assert_linear_close(outs[i], y_ref, bound, f"every-route stack op {i} M={M} b={b}")
+    for x_in, y_out, ref, b, N, K, g in ((xa, ya, ra, 4, 384, 512, 128), (ya, yb, rb, 3, 640, 384, 128),
+                                          (yb, yc, rc, 2, 256, 640, 64)):
+        y_ref, bound = orc.linear(u16(x_in), *ref, b, N, K, group=g)
+        assert_linear_close(y_out, y_ref, bound, f"every-route chain b={b} group={g}")
+    zq.zq_check_device()
+
+
 @pytest.mark.parametrize("bits", BITS)
 def test_prefill_grouped_plans(zq, orc, bits):
     """Grouped tile-kernel launches of independent ops: one whose ops all have
