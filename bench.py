@@ -56,22 +56,22 @@ KERNEL_SOURCES = {
 MEASURED_TRAFFIC = {
     # (family, model, M): DRAM bytes per layer of the stack
     ("decode", "7b", 1): {  # an 8-layer launch
-        "sha256": "985d2b20a6c71abc9c5155cadcffdf9ba7dd894c5bb01ed078038aaf69abd10b",
-        "bytes_per_layer": 125688064,
+        "sha256": "f9572bb584c305814c8dd153e79fca8d3eed0579afc9566ea8ef798bd67b14d9",
+        "bytes_per_layer": 125239776,
     },
     ("decode", "7b", 32): {  # a 4-layer launch, four token tiles
-        "sha256": "985d2b20a6c71abc9c5155cadcffdf9ba7dd894c5bb01ed078038aaf69abd10b",
-        "bytes_per_layer": 128164416,
+        "sha256": "f9572bb584c305814c8dd153e79fca8d3eed0579afc9566ea8ef798bd67b14d9",
+        "bytes_per_layer": 128267904,
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
-        "sha256": "36e5f33ce31dda93dd4f74bb5c3de7180b760277935e0fc7bb10bafd2006b483",
-        "bytes_per_layer": 133761792,
+        "sha256": "e6bf1fa048a59c130392cc9d8ea9f0342927ac8fcb08fa6fdd971f7851e0ea37",
+        "bytes_per_layer": 131767808,
     },
     # tile kernel, CTA-pair plan: a one-layer launch at M = 2048
     ("prefill", "7b", 2048): {
-        "sha256": "36e5f33ce31dda93dd4f74bb5c3de7180b760277935e0fc7bb10bafd2006b483",
-        "bytes_per_layer": 381255936,
+        "sha256": "e6bf1fa048a59c130392cc9d8ea9f0342927ac8fcb08fa6fdd971f7851e0ea37",
+        "bytes_per_layer": 381045504,
     },
 }
 NOMINAL_HBM_GBS = 8000.0
