@@ -55,7 +55,7 @@ namespace pf {
 constexpr int kTokTile = 256;   // tokens per CTA tile (two MMA halves of 128)
 constexpr int kRowTile = 256;   // weight rows per CTA tile (MMA N)
 constexpr int kBK = 64;         // K per slab
-constexpr int kMaxStages = 3;
+constexpr int kMaxStages = 4;
 constexpr int kSlabB = kRowTile * kBK * 2;  // 32 KB
 constexpr int kEpiWarps = 4;
 constexpr int kTmaWarp = 4;
@@ -96,7 +96,7 @@ struct Ctl {
 //                       of the tile's 256 rows, laid out per thread (below),
 //                       then one (scale | zero << 16) word per (row, chunk)
 //   [kOffCtl, ...)      barriers and flags
-template <int B, bool ONE>
+template <int B, bool ONE, int XR = ONE ? 128 : 256>
 struct Plan {
     // Dequant warps: 16 in the one-half plan (its code ring keeps their
     // registers low), 8 in the two-half plan (register prefetch); none for
@@ -106,9 +106,15 @@ struct Plan {
     static constexpr int kThreads = 32 * (kSchedWarp + 1);
     // readers of every tile-ring entry: TMA and MMA lanes, epilogue and dequant warps
     static constexpr int kTileReaders = 2 + kEpiWarps + kDqWarps;
-    static constexpr int kStages = B == 16 ? 3 : (ONE && B == 8) ? 2 : 3;
-    static constexpr int kSlabA = (ONE ? kPrefillHalfTokens : kTokTile) * kBK * 2;
-    static constexpr int kSlots = (!ONE || B == 16) ? 0 : B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3;
+    // XR: token rows of an x stage.  With every M <= 64 (XR = 64, b <= 4) the
+    // x stage is half as large and the space becomes a fourth W stage (one
+    // code slot fewer); the MMA still reads 128 A rows, rows 64..127 from the
+    // bytes after the slab, whose accumulator rows are never stored.
+    static constexpr int kStages = B == 16 ? 3 : (ONE && B == 8) ? 2 : XR == 64 ? 4 : 3;
+    static constexpr int kSlabA = XR * kBK * 2;
+    static constexpr int kSlots = (!ONE || B == 16) ? 0
+                                  : XR == 64 ? (B == 2 ? 5 : B == 3 ? 4 : 3)
+                                             : (B == 2 ? 6 : B == 3 ? 5 : B == 4 ? 4 : 3);
     static constexpr int kSlotCodes = 1024 * (4 * B);  // 256 rows x 2 slabs x 2 chunks of 32 codes
     // + a (scale | zero << 16) word per (row, chunk, slab): the two slabs of a
     // block of 128 codes fall in different groups when groups are 32 or 64
@@ -121,6 +127,7 @@ struct Plan {
     static_assert(kOffB % 1024 == 0 && kOffCodes % 1024 == 0, "SWIZZLE_128B stages need 1024-byte alignment");
     static_assert(kBytes <= 232448, "227 KB of shared memory per CTA");
     static_assert(!ONE || B == 16 || kSlots >= 3, "the scale/zero hand-off needs a prefetch distance of 2 groups");
+    static_assert(XR == (ONE ? XR : 256) && (XR != 64 || (ONE && B <= 4)), "x rows per plan");
 };
 
 // Bounded wait: false if the CTA is aborting or the limit was reached.
@@ -401,10 +408,10 @@ __device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
 // register set when their group's codes are issued and written to the slot
 // two groups later; the two register sets alternate, hence the loop below is
 // unrolled twice.
-template <int B>
+template <int B, int XR>
 __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb, uint8_t *scode, Ctl &c,
                                              int d, int lane) {
-    using P = Plan<B, true>;
+    using P = Plan<B, true, XR>;
     constexpr int NT = 32 * P::kDqWarps;
     constexpr int RPT = 512 / NT;                     // rows per thread
     constexpr int kS = P::kSlots;
@@ -575,10 +582,10 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
     cp_async_wait<0>();  // no copy may land after the CTA has exited
 }
 
-template <int B, bool ONE>
-__global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
+template <int B, bool ONE, int XR>
+__global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
     prefill_kernel(const __grid_constant__ PrefillGroup p) {
-    using P = Plan<B, ONE>;
+    using P = Plan<B, ONE, XR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sa = base;                  // x slabs
@@ -745,7 +752,7 @@ __global__ void __launch_bounds__(Plan<B, ONE>::kThreads, 1)
         if constexpr (B == 16) {
             // no dequant warps for fp16 weights
         } else if constexpr (ONE) {
-            dequant_ring<B>(p, sb, scode, sm, threadIdx.x - 32 * kDqWarp0, lane);
+            dequant_ring<B, XR>(p, sb, scode, sm, threadIdx.x - 32 * kDqWarp0, lane);
         } else {
         // 256 threads: thread d owns rows d/2 and d/2 + 128 of the tile and the
         // 32-code chunk d%2 of every slab.  Codes, scales and zeros of the next
@@ -1451,15 +1458,15 @@ cudaError_t launch_dequant_test(const uint32_t *packed, const uint16_t *scales, 
 
 // ------------------------------------------------------------------ host --
 
-template <int B, bool ONE>
+template <int B, bool ONE, int XR = ONE ? 128 : 256>
 static cudaError_t launch_prefill_t(const PrefillGroup &pg, int n_ctas, cudaStream_t stream) {
-    constexpr size_t smem = pf::Plan<B, ONE>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(pf::prefill_kernel<B, ONE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    constexpr size_t smem = pf::Plan<B, ONE, XR>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(pf::prefill_kernel<B, ONE, XR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(n_ctas));
-    cfg.blockDim = dim3(pf::Plan<B, ONE>::kThreads);
+    cfg.blockDim = dim3(pf::Plan<B, ONE, XR>::kThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -1467,7 +1474,7 @@ static cudaError_t launch_prefill_t(const PrefillGroup &pg, int n_ctas, cudaStre
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B, ONE>, pg);
+    return cudaLaunchKernelEx(&cfg, pf::prefill_kernel<B, ONE, XR>, pg);
 }
 
 cudaError_t prefill_x_map(CUtensorMap *map, const uint16_t *x, int M, int K) {
@@ -1483,6 +1490,7 @@ cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K
 int prefill_plan(const PrefillGroup &pg, int bits) {
     int max_m = 0;
     for (int i = 0; i < pg.n_ops; ++i) max_m = pg.ops[i].M > max_m ? pg.ops[i].M : max_m;
+    if (max_m <= kPrefillQuarterTokens && bits <= 4) return kPlanOneHalf64;
     if (max_m <= kPrefillHalfTokens) return kPlanOneHalf;
     // CTA pairs from 512 tokens: below, a pair tile's second token half is
     // empty and the one-CTA two-half plan was faster (M = 256: 3.4 against
@@ -1490,7 +1498,9 @@ int prefill_plan(const PrefillGroup &pg, int bits) {
     return (bits == 16 || max_m < kPairMinM) ? kPlanTwoHalves : kPlanPair;
 }
 
-int prefill_box_rows(int plan) { return plan == kPlanTwoHalves ? pf::kTokTile : kPrefillHalfTokens; }
+int prefill_box_rows(int plan) {
+    return plan == kPlanTwoHalves ? pf::kTokTile : plan == kPlanOneHalf64 ? kPrefillQuarterTokens : kPrefillHalfTokens;
+}
 
 int prefill_tok_tile(int plan) { return plan == kPlanPair ? pf::kPairTok : pf::kTokTile; }
 
@@ -1543,6 +1553,13 @@ cudaError_t launch_prefill_group(const PrefillGroup &pg, int bits, int num_sms, 
             case 3: return launch_pair_t<3>(pg, num_sms, stream);
             case 4: return launch_pair_t<4>(pg, num_sms, stream);
             default: return launch_pair_t<8>(pg, num_sms, stream);
+        }
+    }
+    if (plan == kPlanOneHalf64) {
+        switch (bits) {
+            case 2: return launch_prefill_t<2, true, kPrefillQuarterTokens>(pg, n_ctas, stream);
+            case 3: return launch_prefill_t<3, true, kPrefillQuarterTokens>(pg, n_ctas, stream);
+            default: return launch_prefill_t<4, true, kPrefillQuarterTokens>(pg, n_ctas, stream);
         }
     }
     if (plan == kPlanOneHalf) {

@@ -15,6 +15,7 @@
 namespace zq {
 
 constexpr int kPrefillHalfTokens = 128;
+constexpr int kPrefillQuarterTokens = 64;  // x stage rows of the one-half plan when every M <= 64 (b <= 4)
 
 // Tensor map of x (M x K fp16) with boxes of 64 k x box_rows tokens, 128-byte swizzle.
 cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K, int box_rows);
@@ -23,7 +24,7 @@ cudaError_t prefill_x_map_rows(CUtensorMap *map, const uint16_t *x, int M, int K
 // swizzle: the W slab of the tile kernel for bits = 16.
 cudaError_t prefill_w_map(CUtensorMap *map, const uint16_t *w, int N, int K);
 
-constexpr int kPlanOneHalf = 0, kPlanTwoHalves = 1, kPlanPair = 2;
+constexpr int kPlanOneHalf = 0, kPlanTwoHalves = 1, kPlanPair = 2, kPlanOneHalf64 = 3;
 constexpr int kPairMinM = 512;  // the CTA-pair plan runs launches with some M >= 512
 
 // Plan of a launch from its ops' M (read only; may be called before the maps
