@@ -65,13 +65,13 @@ MEASURED_TRAFFIC = {
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
-        "sha256": "e6bf1fa048a59c130392cc9d8ea9f0342927ac8fcb08fa6fdd971f7851e0ea37",
-        "bytes_per_layer": 131767808,
+        "sha256": "f546777dbd1bb214227aa5485c05a6c6964573c22762de2988661b6f5d954f44",
+        "bytes_per_layer": 131557888,
     },
     # tile kernel, CTA-pair plan: a one-layer launch at M = 2048
     ("prefill", "7b", 2048): {
-        "sha256": "e6bf1fa048a59c130392cc9d8ea9f0342927ac8fcb08fa6fdd971f7851e0ea37",
-        "bytes_per_layer": 381045504,
+        "sha256": "f546777dbd1bb214227aa5485c05a6c6964573c22762de2988661b6f5d954f44",
+        "bytes_per_layer": 380724992,
     },
 }
 NOMINAL_HBM_GBS = 8000.0
