@@ -65,13 +65,13 @@ MEASURED_TRAFFIC = {
     },
     # tile kernel, one-token-half plan: a one-layer launch at M = 64
     ("prefill", "7b", 64): {
-        "sha256": "f546777dbd1bb214227aa5485c05a6c6964573c22762de2988661b6f5d954f44",
-        "bytes_per_layer": 131557888,
+        "sha256": "731fe9bb6c01b2a07244b2d29eaddf0d9e5d87b9272e0f4f7365a2578ca25d5b",
+        "bytes_per_layer": 130703104,
     },
     # tile kernel, CTA-pair plan: a one-layer launch at M = 2048
     ("prefill", "7b", 2048): {
-        "sha256": "f546777dbd1bb214227aa5485c05a6c6964573c22762de2988661b6f5d954f44",
-        "bytes_per_layer": 380724992,
+        "sha256": "731fe9bb6c01b2a07244b2d29eaddf0d9e5d87b9272e0f4f7365a2578ca25d5b",
+        "bytes_per_layer": 381221120,
     },
 }
 NOMINAL_HBM_GBS = 8000.0

@@ -82,8 +82,12 @@ struct Ctl {
     unsigned long long full[kMaxStages];   // W slab dequantized (one arrival per dequant warp)
     unsigned long long xfull[kMaxStages];  // x slab landed (the TMA warp's expect_tx + the copy's bytes)
     unsigned long long empty[kMaxStages];
-    unsigned long long acc_full;
-    unsigned long long acc_empty;
+    // accumulator buffer b complete / drained: the one-token-half plan uses
+    // TMEM columns [256b, 256b + 256) for tile i with b = i % 2, so a tile's
+    // MMAs run while the previous tile is drained; the two-half plan holds
+    // both token halves in its 512 columns and uses buffer 0 alone
+    unsigned long long acc_full[2];
+    unsigned long long acc_empty[2];
     unsigned long long mma_done;           // every tcgen05.mma this CTA issued has completed
     uint32_t tmem_base;
     int abort;
@@ -130,9 +134,12 @@ struct Plan {
     static_assert(XR == (ONE ? XR : 256) && (XR != 64 || (ONE && B <= 4)), "x rows per plan");
 };
 
-// Bounded wait: false if the CTA is aborting or the limit was reached.
-__device__ __noinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *abort,
-                                       unsigned long long limit) {
+// Bounded wait: false if the CTA is aborting or the limit was reached.  The
+// first test of the phase is inline and the polling loop a call, so a wait
+// whose phase has completed costs one try_wait (the call alone cost 6-7 % of
+// the tile kernel's time at 40-256 tokens).
+__device__ __noinline__ bool mbar_wait_poll(unsigned long long *bar, uint32_t parity, volatile int *abort,
+                                            unsigned long long limit) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t it = 1;; ++it) {
@@ -146,6 +153,11 @@ __device__ __noinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity,
             }
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, uint32_t parity, volatile int *abort,
+                                          unsigned long long limit) {
+    return mbar_try_wait(bar, parity) || mbar_wait_poll(bar, parity, abort, limit);
 }
 
 // Wait of a drain: for a phase that work already issued will complete; no
@@ -389,6 +401,13 @@ __device__ __forceinline__ void load_chunk(uint32_t (&w)[B], const uint32_t *src
 }
 
 
+// Two consecutive 16-bit values from a 4-byte aligned address (read-only path).
+__device__ __forceinline__ uint32_t ldg_u32_nc(const uint16_t *p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 // cp.async of U bytes (16, 8 or 4) global -> shared.
 template <int U>
 __device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
@@ -396,6 +415,19 @@ __device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
     else if constexpr (U == 8) cp_async8(dst, src);
     else cp_async4(dst, src);
 }
+
+// Scales and zeros of one block of 128 codes as loaded (not yet packed into
+// the slot's (scale | zero << 16) words), and how they were loaded.
+constexpr int kSzNone = 0;        // nothing loaded (past the last block)
+constexpr int kSzOne = 1;         // one group: s[r][0], z[r][0]
+constexpr int kSzSplit = 2;       // groups of 32 or 64: [r][0] for slab 0, [r][1] for slab 1
+constexpr int kSzPair = 3;        // this group and the next: the low and high halves of s[r][0], z[r][0]
+constexpr int kSzPairSecond = 4;  // the second group of a pair: nothing of its own
+template <int RPT>
+struct ScaleSet {
+    uint32_t s[RPT][2], z[RPT][2];
+    int mode;
+};
 
 // Dequant producer of the one-token-half plan.  Its NT threads own the 512
 // (row, chunk) pairs of each slab, pair q = d + NT * r (r < 512 / NT) of
@@ -406,8 +438,11 @@ __device__ __forceinline__ void cp_async_u(void *dst, const void *src) {
 // d at (u * NT + d) * U, so the copies and the loads of a warp are contiguous.
 // Scales and zeros (2-byte aligned, too small for cp.async) are loaded into a
 // register set when their group's codes are issued and written to the slot
-// two groups later; the two register sets alternate, hence the loop below is
-// unrolled twice.
+// two groups later, packed only then; the two register sets alternate, hence
+// the loop below is unrolled twice.  With groups of 128 and an even number of
+// groups per row, the scales (and zeros) of two consecutive groups are one
+// 4-byte load, made with the first group's codes, and both groups' words are
+// written two groups later.
 template <int B, int XR>
 __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb, uint8_t *scode, Ctl &c,
                                              int d, int lane) {
@@ -433,6 +468,9 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
     // consume cursor, later, releases it).
     uint32_t jp = 0;
     int tp = tile_at(c, jp, abort, p.wait_ns), gp = 0, Gp = 0, gsh = 2;
+    // groups of 128 and an even count per row: with the arrays 16-byte aligned
+    // (checked by the host), the scales of groups 2i and 2i + 1 are 4-byte aligned
+    bool pair2 = false;
     const uint32_t *prow[RPT];
     const uint16_t *psr[RPT], *pzr[RPT];
     auto start_issue = [&]() {
@@ -442,6 +480,7 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
             Gp = op.K / kGroup;
             gsh = op.gshift;
             const size_t gs = static_cast<size_t>(op.K) >> (op.gshift + 5);  // scales per row
+            pair2 = gsh == 2 && (gs & 1) == 0;
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
                 const int n = min(tr.n0 + rows[r], op.N - 1);
@@ -452,24 +491,35 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         }
     };
     start_issue();
-    uint32_t szA[RPT][2], szB[RPT][2];
-#pragma unroll
-    for (int r = 0; r < RPT; ++r) szA[r][0] = szA[r][1] = szB[r][0] = szB[r][1] = 0u;
+    ScaleSet<RPT> szA, szB;
+    szA.mode = szB.mode = kSzNone;
     // Block j of this CTA's sequence: first store the scale/zero words of
-    // block j - 2 (held in `set`) into its slot, then copy block j's codes into
-    // slot j % kS and load its scales and zeros into `set`: slab h of the
-    // block uses group (4 * gp + 2h + ch) >> gshift.  Past the last block only
-    // the store and an empty commit remain, so that every block index commits
-    // exactly one cp.async group.
-    auto issue = [&](int j, uint32_t (&set)[RPT][2]) {
-        if (j >= 2) {
+    // block j - 2 (held in `set`) into its slot (and those of block j - 1
+    // into its slot, after a pair load), then copy block j's codes into slot
+    // j % kS and load its scales and zeros into `set`: slab h of the block
+    // uses group (4 * gp + 2h + ch) >> gshift.  Block j - 1's slot is free for
+    // its words by then: the slot's previous block was consumed before block
+    // j - 1 was issued.  Past the last block only the store and an empty
+    // commit remain, so that every block index commits exactly one cp.async
+    // group.
+    auto issue = [&](int j, ScaleSet<RPT> &set) {
+        if (j >= 2 && set.mode != kSzNone && set.mode != kSzPairSecond) {
+            // the words of block j - 2 (and, after a pair load, of block j - 1)
             uint32_t *zs = reinterpret_cast<uint32_t *>(scode + ((j - 2) % kS) * P::kSlotBytes + P::kSlotCodes);
+            uint32_t *zn = reinterpret_cast<uint32_t *>(scode + ((j - 1) % kS) * P::kSlotBytes + P::kSlotCodes);
 #pragma unroll
             for (int r = 0; r < RPT; ++r) {
-                zs[(2 * r) * NT + d] = set[r][0];
-                zs[(2 * r + 1) * NT + d] = set[r][1];
+                const uint32_t w0 = prmt(set.s[r][0], set.z[r][0], 0x5410u);
+                zs[(2 * r) * NT + d] = w0;
+                zs[(2 * r + 1) * NT + d] = set.mode == kSzSplit ? prmt(set.s[r][1], set.z[r][1], 0x5410u) : w0;
+                if (set.mode == kSzPair) {
+                    const uint32_t w1 = prmt(set.s[r][0], set.z[r][0], 0x7632u);
+                    zn[(2 * r) * NT + d] = w1;
+                    zn[(2 * r + 1) * NT + d] = w1;
+                }
             }
         }
+        set.mode = kSzNone;
         if (tp >= 0) {
             uint8_t *cs = scode + (j % kS) * P::kSlotBytes;
 #pragma unroll
@@ -481,11 +531,37 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                     for (int u = 0; u < UPC; ++u)
                         cp_async_u<U>(cs + (((h * RPT + r) * UPC + u) * NT + d) * U, src + u * U);
                 }
-            const int g0 = (4 * gp + ch) >> gsh, g1 = (4 * gp + 2 + ch) >> gsh;
+            // The loaded values stay as they are until their words are stored
+            // two blocks later: packing them here would wait for the loads.
+            if (gsh != 2) {
+                // groups of 32 or 64: the block's two slabs of this chunk lie in
+                // groups g0 and g1 > g0
+                const int g0 = (4 * gp + ch) >> gsh, g1 = (4 * gp + 2 + ch) >> gsh;
+                set.mode = kSzSplit;
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                set[r][0] = ldg_u16_nc(psr[r] + g0) | (ldg_u16_nc(pzr[r] + g0) << 16);
-                set[r][1] = g1 == g0 ? set[r][0] : ldg_u16_nc(psr[r] + g1) | (ldg_u16_nc(pzr[r] + g1) << 16);
+                for (int r = 0; r < RPT; ++r) {
+                    set.s[r][0] = ldg_u16_nc(psr[r] + g0);
+                    set.z[r][0] = ldg_u16_nc(pzr[r] + g0);
+                    set.s[r][1] = ldg_u16_nc(psr[r] + g1);
+                    set.z[r][1] = ldg_u16_nc(pzr[r] + g1);
+                }
+            } else if (pair2 && (gp & 1) == 0) {
+                // groups gp and gp + 1 with one 4-byte load each of scales and zeros
+                set.mode = kSzPair;
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    set.s[r][0] = ldg_u32_nc(psr[r] + gp);
+                    set.z[r][0] = ldg_u32_nc(pzr[r] + gp);
+                }
+            } else if (pair2) {
+                set.mode = kSzPairSecond;  // loaded, and stored, with block gp - 1
+            } else {
+                set.mode = kSzOne;
+#pragma unroll
+                for (int r = 0; r < RPT; ++r) {
+                    set.s[r][0] = ldg_u16_nc(psr[r] + gp);
+                    set.z[r][0] = ldg_u16_nc(pzr[r] + gp);
+                }
             }
             if (++gp == Gp) {
                 gp = 0;
@@ -522,18 +598,16 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                 sz[r][h] = lds_u32(cs + P::kSlotCodes + 4 * ((2 * r + h) * NT + d));
                 ovf[r][h] = dequant_overflows<B>(sz[r][h]);
             }
+        // both slabs' codes, loaded before the waits for their W stages
+        uint32_t wall[2][RPT][B];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {  // the two slabs of this group
-            const int st = it % P::kStages;
-            const uint32_t round = it / P::kStages;
-            if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) return false;
-            uint8_t *bs = sb + st * kSlabB;
+        for (int h = 0; h < 2; ++h)
 #pragma unroll
-            for (int r = 0; r < RPT; ++r) {
-                uint32_t w[B];
+            for (int r = 0; r < RPT; ++r)
 #pragma unroll
                 for (int u = 0; u < UPC; ++u) {
                     const uint32_t a = cs + (((h * RPT + r) * UPC + u) * NT + d) * U;
+                    uint32_t(&w)[B] = wall[h][r];
                     if constexpr (U == 16) {
                         const uint4 v = lds_v4(a);
                         w[4 * u] = v.x; w[4 * u + 1] = v.y; w[4 * u + 2] = v.z; w[4 * u + 3] = v.w;
@@ -544,9 +618,17 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
                         w[u] = lds_u32(a);
                     }
                 }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {  // the two slabs of this group
+            const int st = it % P::kStages;
+            const uint32_t round = it / P::kStages;
+            if (!mbar_wait(&c.empty[st], (round & 1u) ^ 1u, abort, p.wait_ns)) return false;
+            uint8_t *bs = sb + st * kSlabB;
+#pragma unroll
+            for (int r = 0; r < RPT; ++r) {
                 const int row = rows[r];
                 uint32_t o[16];
-                dequant_chunk<B, false>(w, sz[r][h], o, ovf[r][h]);  // x is pair-permuted
+                dequant_chunk<B, false>(wall[h][r], sz[r][h], o, ovf[r][h]);  // x is pair-permuted
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const int c16 = (4 * ch + j) ^ (row & 7);
@@ -568,8 +650,8 @@ __device__ __forceinline__ void dequant_ring(const PrefillGroup &p, uint8_t *sb,
         }
         return true;
     };
-    uint32_t (&set_even)[RPT][2] = (PD & 1) ? szB : szA;  // register set of block i + PD, i even
-    uint32_t (&set_odd)[RPT][2] = (PD & 1) ? szA : szB;
+    ScaleSet<RPT> &set_even = (PD & 1) ? szB : szA;  // register set of block i + PD, i even
+    ScaleSet<RPT> &set_odd = (PD & 1) ? szA : szB;
 #pragma unroll 1
     for (int i = 0;; i += 2) {
         if (t < 0 || *abort) break;
@@ -606,8 +688,10 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
             mbar_init(&sm.xfull[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
-        mbar_init(&sm.acc_full, 1);
-        mbar_init(&sm.acc_empty, kEpiWarps);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], kEpiWarps);
+        }
         mbar_init(&sm.mma_done, 1);
         sm.abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -707,8 +791,11 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
                 const int slabs = p.ops[tr.o].K / kBK;
                 // the second 128-token half only when it holds tokens
                 const bool half1 = !ONE && tr.t0 + 128 < p.ops[tr.o].M;
-                if (!mbar_wait(&sm.acc_empty, (tile_i & 1u) ^ 1u, abort, p.wait_ns)) break;
+                // accumulator buffer of this tile and the number of earlier uses of it
+                const uint32_t ab = ONE ? (tile_i & 1u) : 0u, au = ONE ? (tile_i >> 1) : tile_i;
+                if (!mbar_wait(&sm.acc_empty[ab], (au & 1u) ^ 1u, abort, p.wait_ns)) break;
                 tc_fence_after();
+                const uint32_t tacc = tmem + ab * kRowTile;
                 bool ok = true;
                 for (int s = 0; s < slabs; ++s, ++it) {
                     const int st = it % P::kStages;
@@ -733,13 +820,13 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
 #pragma unroll
                         for (int kk = 0; kk < kBK / 16; ++kk) {
                             const uint32_t acc = (s > 0 || kk > 0) ? 1u : 0u;
-                            umma_f16(tmem, sdesc_sw128(a0 + kk * 32), sdesc_sw128(b0 + kk * 32), acc);
+                            umma_f16(tacc, sdesc_sw128(a0 + kk * 32), sdesc_sw128(b0 + kk * 32), acc);
                         }
                     }
                     umma_commit(&sm.empty[st]);
                 }
                 if (!ok) break;
-                umma_commit(&sm.acc_full);
+                umma_commit(&sm.acc_full[ab]);
             }
             // Every MMA issued must have completed before TMEM is freed and the
             // CTA exits (after an abort no epilogue waited for them).
@@ -788,8 +875,15 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
                     load_chunk<B>(wn[h][i], rowp[i] + static_cast<size_t>(4 * g + 2 * h + ch) * B);
-                szn[0][i] = ldg_u16_nc(srow[i] + g0) | (ldg_u16_nc(zrow[i] + g0) << 16);
-                szn[1][i] = g1 == g0 ? szn[0][i] : ldg_u16_nc(srow[i] + g1) | (ldg_u16_nc(zrow[i] + g1) << 16);
+                if (gsh == 2) {
+                    // groups of 128: the scale and the zero as loaded, packed
+                    // when the block is used (packing here would wait for them)
+                    szn[0][i] = ldg_u16_nc(srow[i] + g0);
+                    szn[1][i] = ldg_u16_nc(zrow[i] + g0);
+                } else {
+                    szn[0][i] = ldg_u16_nc(srow[i] + g0) | (ldg_u16_nc(zrow[i] + g0) << 16);
+                    szn[1][i] = ldg_u16_nc(srow[i] + g1) | (ldg_u16_nc(zrow[i] + g1) << 16);
+                }
             }
         };
         // Tiles from the ring: entry jn is read (and released) by the fetch
@@ -812,13 +906,19 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
 #pragma unroll
                     for (int q = 0; q < B; ++q) wc[h][i][q] = wn[h][i][q];
             bool ovf[2][2];
+            if (gsh == 2) {  // gsh is still the current tile's
+#pragma unroll
+                for (int i = 0; i < 2; ++i) szc[0][i] = szc[1][i] = prmt(szn[0][i], szn[1][i], 0x5410u);
+            } else {
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) szc[h][i] = szn[h][i];
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h)
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    szc[h][i] = szn[h][i];
-                    ovf[h][i] = dequant_overflows<B>(szc[h][i]);
-                }
+                for (int i = 0; i < 2; ++i) ovf[h][i] = dequant_overflows<B>(szc[h][i]);
             int t_n = t, g_n = g + 1;
             groups_n = groups;
             if (g_n == groups) {
@@ -868,18 +968,19 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
             __syncwarp();
             if (lane == 0 && t != -2) tile_release(sm, j);
             if (t < 0 || *abort) break;
-            if (!mbar_wait(&sm.acc_full, tile_i & 1u, abort, p.wait_ns)) break;
+            const uint32_t ab = ONE ? (tile_i & 1u) : 0u, au = ONE ? (tile_i >> 1) : tile_i;
+            if (!mbar_wait(&sm.acc_full[ab], au & 1u, abort, p.wait_ns)) break;
             tc_fence_after();
             const TileRef tr = locate(p, t);
             const PrefillOp &op = p.ops[tr.o];
             const int n0 = tr.n0, t0 = tr.t0;
 #pragma unroll 1
-            for (int half = 0; half < (t0 + 128 < op.M ? 2 : 1); ++half) {
+            for (int half = 0; half < (!ONE && t0 + 128 < op.M ? 2 : 1); ++half) {
                 const int tok = t0 + 128 * half + 32 * warp + lane;
                 // bf16 activations: the token's power-of-two factor undoes the
                 // scaling of the fp16 copy the MMAs read
                 const float fs = (op.xscale != nullptr && tok < op.M) ? op.xscale[tok] : 1.0f;
-                const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + half * kRowTile;
+                const uint32_t ta = tmem + (static_cast<uint32_t>(32 * warp) << 16) + (half + ab) * kRowTile;
                 if constexpr (ONE) {
                     // 22 warps: no registers for a second buffer
 #pragma unroll 1
@@ -906,7 +1007,7 @@ __global__ void __launch_bounds__(Plan<B, ONE, XR>::kThreads, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty);
+            if (lane == 0) mbar_arrive(&sm.acc_empty[ab]);
         }
     }
 
@@ -1030,10 +1131,10 @@ __device__ __forceinline__ void cluster_sync() {
 // release data written by the other CTA's threads) or CTA-scope acquire (TMA
 // bytes, tcgen05 commits, tensor-memory hand-offs).  On a timeout both CTAs
 // of the pair are told to abort (their own flag and the peer's) and
-// ZQ_ERR_TIMEOUT is recorded.
+// ZQ_ERR_TIMEOUT is recorded.  As in mbar_wait, the first test is inline.
 template <bool CL = false>
-__device__ __noinline__ bool pair_wait(unsigned long long *bar, uint32_t parity, volatile int *abort,
-                                       uint32_t peer_abort, unsigned long long limit) {
+__device__ __noinline__ bool pair_wait_poll(unsigned long long *bar, uint32_t parity, volatile int *abort,
+                                            uint32_t peer_abort, unsigned long long limit) {
     auto ready = [&]() { return CL ? mbar_try_wait_cl(bar, parity) : mbar_try_wait(bar, parity); };
     if (ready()) return true;
     const unsigned long long t0 = globaltimer();
@@ -1049,6 +1150,12 @@ __device__ __noinline__ bool pair_wait(unsigned long long *bar, uint32_t parity,
             }
         }
     }
+}
+template <bool CL = false>
+__device__ __forceinline__ bool pair_wait(unsigned long long *bar, uint32_t parity, volatile int *abort,
+                                          uint32_t peer_abort, unsigned long long limit) {
+    const bool ok = CL ? mbar_try_wait_cl(bar, parity) : mbar_try_wait(bar, parity);
+    return ok || pair_wait_poll<CL>(bar, parity, abort, peer_abort, limit);
 }
 __device__ __noinline__ void pair_drain(unsigned long long *bar, uint32_t parity) {
     const unsigned long long t0 = globaltimer();
@@ -1293,8 +1400,15 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
 #pragma unroll
             for (int h = 0; h < 2; ++h) load_chunk<B>(w[h], rowp + static_cast<size_t>(4 * gf + 2 * h + ch) * B);
             const int g0 = (4 * gf + ch) >> gsh, g1 = (4 * gf + 2 + ch) >> gsh;  // one group with groups of 128
-            sz[0] = ldg_u16_nc(srow + g0) | (ldg_u16_nc(zrow + g0) << 16);
-            sz[1] = g1 == g0 ? sz[0] : ldg_u16_nc(srow + g1) | (ldg_u16_nc(zrow + g1) << 16);
+            if (gsh == 2) {
+                // the scale and the zero as loaded: the consumer packs them
+                // (packing here would wait for the loads)
+                sz[0] = ldg_u16_nc(srow + g0);
+                sz[1] = ldg_u16_nc(zrow + g0);
+            } else {
+                sz[0] = ldg_u16_nc(srow + g0) | (ldg_u16_nc(zrow + g0) << 16);
+                sz[1] = ldg_u16_nc(srow + g1) | (ldg_u16_nc(zrow + g1) << 16);
+            }
             if (++gf == blocks_f) {
                 gf = 0;
                 tf += pairs;
@@ -1302,18 +1416,27 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
             }
         };
         // consume cursor: tile tc, block gc of blocks_c; slab counter it
-        int tc = pair, gc = 0;
-        int blocks_c = tc < n_tiles ? p.ops[locate(p, tc, kPairTok).o].K / kGroup : 0;
+        int tc = pair, gc = 0, blocks_c = 0, gsh_c = 2;
+        if (tc < n_tiles) {
+            const PrefillOp &op = p.ops[locate(p, tc, kPairTok).o];
+            blocks_c = op.K / kGroup;
+            gsh_c = op.gshift;
+        }
         uint32_t it = 0;
         auto consume = [&](uint32_t (&w)[2][B], uint32_t (&sz)[2]) -> bool {
             if (tc >= n_tiles || *abort) return false;
             uint32_t wc[2][B], szc[2];
             bool ovf[2];
+            if (gsh_c == 2) {
+                szc[0] = szc[1] = prmt(sz[0], sz[1], 0x5410u);
+            } else {
+                szc[0] = sz[0];
+                szc[1] = sz[1];
+            }
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
 #pragma unroll
                 for (int q = 0; q < B; ++q) wc[h][q] = w[h][q];
-                szc[h] = sz[h];
                 ovf[h] = dequant_overflows<B>(szc[h]);
             }
             fetch_next(w, sz);  // the set is free again: load the block two ahead
@@ -1339,7 +1462,11 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
             if (++gc == blocks_c) {
                 gc = 0;
                 tc += pairs;
-                if (tc < n_tiles) blocks_c = p.ops[locate(p, tc, kPairTok).o].K / kGroup;
+                if (tc < n_tiles) {
+                    const PrefillOp &op = p.ops[locate(p, tc, kPairTok).o];
+                    blocks_c = op.K / kGroup;
+                    gsh_c = op.gshift;
+                }
             }
             return true;
         };
