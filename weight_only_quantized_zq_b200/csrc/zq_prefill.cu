@@ -1371,10 +1371,12 @@ __global__ void __launch_bounds__(PairPlan::kThreads, 1) prefill_pair_kernel(con
         }
     } else if (warp >= kDqWarp0) {
         // Thread d: row d / 2 of this CTA's 128 weight rows, 32-code chunk
-        // d % 2 of every slab.  The codes and (scale | zero << 16) words of a
-        // block (128 codes: two slabs) are loaded into registers three blocks
-        // ahead of their use (register sets A, B and C rotate; two at b = 8),
-        // so that about six slabs of dequant time cover the loads' latency.
+        // d % 2 of every slab.  The codes, scales and zeros of a block (128
+        // codes: two slabs) are loaded into registers three blocks ahead of
+        // their use (register sets A, B and C rotate; two at b = 8), so that
+        // about six slabs of dequant time cover the loads' latency; with groups
+        // of 128 the scale and the zero stay as loaded until the block is used,
+        // where they become its (scale | zero << 16) word.
         const int d = threadIdx.x - 32 * kDqWarp0;
         const int row = d >> 1, ch = d & 1;
         const uint32_t *rowp = nullptr;
